@@ -1,0 +1,195 @@
+"""QSA layer oracle (Python face of ``oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py``; never by the product path. It is a plain,
+slow, single-threaded statement of the layer (pool -> RMSNorm -> partial RoPE ->
+ReLU-sum indexer score -> top-k_B blocks -> expand + tail -> attention), written
+from the "QSA (Qwen Sparse Attention)" concept page, section "Key math / How it
+works", and the "Qwen Sparse Attention" gallery page, section "How block
+selection works". Every function is pinned by ``tests/test_oracle_pins.py``;
+none is "parity unpinned".
+
+Arrays are numpy: bf16 values travel as their uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_SO = os.path.join(_HERE, "liboracle.so")
+
+GCC_FLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC"]
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _SO) -> str:
+    """Compile oracle.c (plain C, single-threaded, strict IEEE fp64)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        subprocess.check_call(["gcc", *GCC_FLAGS, "-o", out, src, "-lm"])
+    return out
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("r", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("idx_heads", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+                ("rope_dims", ctypes.c_int32), ("rope_base", ctypes.c_double),
+                ("rms_eps", ctypes.c_double),
+                ("q_heads", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("sm_scale", ctypes.c_double)]
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+class Oracle:
+    """The oracle for one layer configuration (shapes of a ``synth.Workload``)."""
+
+    def __init__(self, r=4, K=2048, idx_heads=4, idx_dim=128, rope_dims=64, rope_base=10000.0,
+                 rms_eps=1e-6, q_heads=32, kv_heads=4, head_dim=128, sm_scale=0.0,
+                 lib_path: Optional[str] = None):
+        path = lib_path or build()
+        self.lib = ctypes.CDLL(path)
+        self.cfg = Cfg(r, K, idx_heads, idx_dim, rope_dims, rope_base, rms_eps, q_heads, kv_heads,
+                       head_dim, sm_scale)
+        self._c = ctypes.byref(self.cfg)
+        L = self.lib
+        vp = ctypes.c_void_p
+        L.qsa_oracle_k_blocks.restype = ctypes.c_int64
+        L.qsa_oracle_k_blocks.argtypes = [vp]
+        L.qsa_oracle_rope.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int64, vp]
+        L.qsa_oracle_pool_block.argtypes = [vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp]
+        L.qsa_oracle_compress.argtypes = [vp, vp, ctypes.c_int64, vp, vp]
+        L.qsa_oracle_rotate_query.argtypes = [vp, vp, ctypes.c_int64, vp]
+        L.qsa_oracle_scores.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
+        L.qsa_oracle_select.restype = ctypes.c_int64
+        L.qsa_oracle_select.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp]
+        L.qsa_oracle_token_set.restype = ctypes.c_int64
+        L.qsa_oracle_token_set.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int64, vp]
+        L.qsa_oracle_attention.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp]
+        L.qsa_oracle_row.restype = ctypes.c_int64
+        L.qsa_oracle_row.argtypes = [vp, ctypes.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.qsa_oracle_decode_step.restype = ctypes.c_int64
+        L.qsa_oracle_decode_step.argtypes = [vp, ctypes.c_int64] + [vp] * 13
+
+    @classmethod
+    def for_workload(cls, w, **kw) -> "Oracle":
+        return cls(r=w.r, K=w.K, idx_heads=w.idx_heads, idx_dim=w.idx_dim, rope_dims=w.rope_dims,
+                   rope_base=w.rope_base, rms_eps=w.rms_eps, q_heads=w.q_heads,
+                   kv_heads=w.kv_heads, head_dim=w.head_dim, **kw)
+
+    # ------------------------------------------------------------------ steps
+    @property
+    def k_blocks(self) -> int:
+        return int(self.lib.qsa_oracle_k_blocks(self._c))
+
+    def rope(self, x: np.ndarray, pos: int) -> np.ndarray:
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty_like(x)
+        c = self.cfg
+        self.lib.qsa_oracle_rope(_p(x), x.size, c.rope_dims, c.rope_base, pos, _p(out))
+        return out
+
+    def pool_block(self, keys: np.ndarray, pos: int, w: Optional[np.ndarray] = None) -> dict:
+        keys = _u16(keys)
+        d = self.cfg.idx_dim
+        kbar, knorm, krot = (np.empty(d) for _ in range(3))
+        out = np.empty(d, dtype=np.uint16)
+        w = None if w is None else np.ascontiguousarray(w, dtype=np.float32)
+        self.lib.qsa_oracle_pool_block(self._c, _p(keys), _p(w), pos, _p(kbar), _p(knorm),
+                                       _p(krot), _p(out))
+        return {"kbar": kbar, "knorm": knorm, "krot": krot, "out": out}
+
+    def compress(self, idx_k: np.ndarray, n_blocks: int, w: Optional[np.ndarray] = None) -> np.ndarray:
+        idx_k = _u16(idx_k)
+        assert idx_k.size >= n_blocks * self.cfg.r * self.cfg.idx_dim
+        out = np.empty((n_blocks, self.cfg.idx_dim), dtype=np.uint16)
+        w = None if w is None else np.ascontiguousarray(w, dtype=np.float32)
+        self.lib.qsa_oracle_compress(self._c, _p(idx_k), n_blocks, _p(w), _p(out))
+        return out
+
+    def rotate_query(self, q: np.ndarray, pos: int) -> np.ndarray:
+        q = _u16(q)
+        out = np.empty((self.cfg.idx_heads, self.cfg.idx_dim), dtype=np.uint16)
+        self.lib.qsa_oracle_rotate_query(self._c, _p(q), pos, _p(out))
+        return out
+
+    def scores(self, qrot: np.ndarray, pooled: np.ndarray, n_vis: int) -> np.ndarray:
+        qrot, pooled = _u16(qrot), _u16(pooled)
+        assert pooled.size >= n_vis * self.cfg.idx_dim
+        out = np.empty(n_vis, dtype=np.float32)
+        self.lib.qsa_oracle_scores(self._c, _p(qrot), _p(pooled), n_vis, _p(out))
+        return out
+
+    def select(self, scores: np.ndarray, k_b: Optional[int] = None) -> np.ndarray:
+        scores = np.ascontiguousarray(scores, dtype=np.float32)
+        k_b = self.k_blocks if k_b is None else k_b
+        sel = np.empty(max(min(k_b, scores.size), 1), dtype=np.int32)
+        m = self.lib.qsa_oracle_select(_p(scores), scores.size, k_b, _p(sel))
+        return sel[:m].copy()
+
+    def token_set(self, sel: np.ndarray, i: int) -> np.ndarray:
+        sel = np.ascontiguousarray(sel, dtype=np.int32)
+        out = np.empty(sel.size * self.cfg.r + self.cfg.r, dtype=np.int64)
+        n = self.lib.qsa_oracle_token_set(self._c, _p(sel), sel.size, i, _p(out))
+        return out[:n].copy()
+
+    def attention(self, q: np.ndarray, kc: np.ndarray, vc: np.ndarray, tokens: np.ndarray):
+        q, kc, vc = _u16(q), _u16(kc), _u16(vc)
+        tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+        c = self.cfg
+        out = np.empty((c.q_heads, c.head_dim))
+        lse = np.empty(c.q_heads)
+        self.lib.qsa_oracle_attention(self._c, _p(q), _p(kc), _p(vc), _p(tokens), tokens.size,
+                                      _p(out), _p(lse))
+        return out, lse
+
+    def row(self, i: int, idx_q_row: np.ndarray, pooled: np.ndarray, q_row=None, kc=None, vc=None,
+            want_scores: bool = True) -> dict:
+        """a3'..a7 for query position i. Attention is skipped when q_row is None."""
+        c = self.cfg
+        n_vis = i // c.r
+        assert pooled.size >= n_vis * c.idx_dim
+        # Padded with a sentinel: a row that scores more blocks than are visible is
+        # reported, not a buffer overrun.
+        scores = np.full(n_vis + c.r + 1, -7.0, dtype=np.float32) if want_scores else None
+        sel = np.empty(max(self.k_blocks, 1), dtype=np.int32)
+        out = lse = None
+        if q_row is not None:
+            out = np.empty((c.q_heads, c.head_dim))
+            lse = np.empty(c.q_heads)
+            q_row, kc, vc = _u16(q_row), _u16(kc), _u16(vc)
+        m = self.lib.qsa_oracle_row(self._c, i, _p(_u16(idx_q_row)), _p(_u16(pooled)), _p(q_row),
+                                    _p(kc), _p(vc), _p(scores), _p(sel), _p(out), _p(lse))
+        res = {"sel": sel[:m].copy(), "nsel": int(m), "out": out, "lse": lse}
+        if want_scores:
+            assert (scores[n_vis:] == -7.0).all(), "scored blocks beyond floor(i/r)"
+            res["scores"] = scores[:n_vis].copy()
+        return res
+
+    def decode_step(self, p: int, q_new, k_new, v_new, idx_q_new, idx_k_new, kc, vc, idx_k_cache,
+                    pooled, w: Optional[np.ndarray] = None) -> dict:
+        """a8 + a3'..a7 for the token at position p; updates the caches in place."""
+        c = self.cfg
+        for a in (kc, vc, idx_k_cache, pooled):
+            assert a.flags.c_contiguous and a.dtype == np.uint16
+        sel = np.empty(max(self.k_blocks, 1), dtype=np.int32)
+        out = np.empty((c.q_heads, c.head_dim))
+        lse = np.empty(c.q_heads)
+        w = None if w is None else np.ascontiguousarray(w, dtype=np.float32)
+        m = self.lib.qsa_oracle_decode_step(
+            self._c, p, _p(_u16(q_new)), _p(_u16(k_new)), _p(_u16(v_new)), _p(_u16(idx_q_new)),
+            _p(_u16(idx_k_new)), _p(kc), _p(vc), _p(idx_k_cache), _p(pooled), _p(w), _p(sel),
+            _p(out), _p(lse))
+        return {"sel": sel[:m].copy(), "nsel": int(m), "out": out, "lse": lse}

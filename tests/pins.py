@@ -1,0 +1,330 @@
+"""Pins for the oracle: checks against what the pages and mathematics fix.
+
+Each ``pin_*`` takes a factory ``make(**cfg) -> oracle.Oracle`` and raises
+AssertionError when the oracle it builds is wrong. ``test_oracle_pins.py`` runs
+them on the oracle; ``test_oracle_mutants.py`` runs them on copies of the oracle
+with planted mistakes and requires every mistake to be caught by some pin.
+
+Sources: "QSA (Qwen Sparse Attention)" concept page, "Key math / How it works"
+(A) indexer and (B) sparse core attention, "Config"; "Qwen Sparse Attention"
+gallery page, "How block selection works" and its budget table.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+
+import bruteforce as bfm
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+TINY = synth.Workload(name="pin_tiny", n=256, K=32, q_heads=4, kv_heads=1, base_seed=0x70696E01)
+GQA = synth.Workload(name="pin_gqa", n=96, K=16, q_heads=8, kv_heads=2, base_seed=0x70696E02)
+NEEDLE = synth.Workload(name="pin_needle", n=8192, K=64, q_heads=4, kv_heads=1,
+                        base_seed=0x70696E03, n_needles_prefill=12)
+
+
+def _inputs(w, seq=0):
+    n = w.total
+    return (w.host_full("idx_q", seq).reshape(n, w.idx_heads, w.idx_dim),
+            w.host_full("idx_k", seq),
+            w.host_full("q", seq).reshape(n, w.q_heads, w.head_dim),
+            w.host_full("k", seq).reshape(n, w.kv_heads, w.head_dim),
+            w.host_full("v", seq).reshape(n, w.kv_heads, w.head_dim))
+
+
+def _bits(x):
+    return bfm.f64_to_bf16(np.asarray(x, dtype=np.float64))
+
+
+# ----------------------------------------------------------------------------- golden
+def pin_budget_golden(make):
+    """The gallery page's budget table: a 2,048-token budget with 4-token blocks
+    selects up to 512 blocks (k_B = ceil(K/r)); and the selection never holds
+    more than k_B blocks."""
+    rows = [ln.split("#")[0].split() for ln in open(os.path.join(GOLDEN, "budget.txt"))]
+    for row in rows:
+        if not row:
+            continue
+        kv = dict(x.split("=") for x in row)
+        o = make(r=int(kv["r"]), K=int(kv["K"]))
+        assert o.k_blocks == int(kv["k_B"]), (kv, o.k_blocks)
+    o = make(r=4, K=2048)
+    rng = np.random.default_rng(1)
+    s = rng.standard_normal(5000).astype(np.float32)
+    assert o.select(s).size == 512
+
+
+# ----------------------------------------------------------------------------- RoPE
+def pin_rope_textbook(make):
+    """RoPE = complex rotation z_j * e^{i pos theta_j}, theta_j = base^(-2j/64),
+    on dims 0..63 only; position 0 is the identity; each (j, j+32) pair keeps
+    its norm; rotations compose (R_a R_b = R_{a+b})."""
+    o = make()
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal(128)
+    for pos in (0, 1, 3, 4, 4095, 131068, 1048572):
+        got = o.rope(x, pos)
+        want = bfm.rope_complex(x, pos, 64, 10000.0)
+        assert np.allclose(got, want, rtol=0, atol=1e-9), pos
+        assert np.array_equal(got[64:], x[64:])
+        assert np.allclose(np.hypot(got[:32], got[32:64]), np.hypot(x[:32], x[32:64]), atol=1e-12)
+    assert np.array_equal(o.rope(x, 0), x)
+    assert np.allclose(o.rope(o.rope(x, 17), 1000), o.rope(x, 1017), atol=1e-9)
+
+
+def _basis_angle(vec, j=0):
+    return np.arctan2(vec[j + 32], vec[j])
+
+
+def pin_rope_first_position_of_block(make):
+    """The pooled key of block b is rotated at the block's FIRST position r*b
+    (gallery page); the indexer query at its own position i. With a key/query
+    along dim 0 the rotated pair (0, 32) is (cos(pos), sin(pos)) * norm."""
+    o = make()
+    e = np.zeros((4, 128))
+    e[:, 0] = 1.0
+    e[:, 64] = 1.0
+    keys = _bits(e)
+    for b in (0, 1, 5, 1000):
+        res = o.pool_block(keys, pos=4 * b)
+        ang = _basis_angle(res["krot"])
+        assert abs(np.angle(np.exp(1j * (ang - 4 * b)))) < 1e-9, b
+    idx_k = _bits(np.tile(e[0], (4 * 6, 1)))
+    pooled = o.compress(idx_k, 6)
+    for b in range(6):
+        v = bfm.bf16_to_f64(pooled[b])
+        ang = _basis_angle(v)
+        assert abs(np.angle(np.exp(1j * (ang - 4 * b)))) < 1e-2, (b, ang)
+    q = np.zeros((4, 128))
+    q[:, 0] = 1.0
+    for i in (0, 2, 7, 999):
+        qr = bfm.bf16_to_f64(o.rotate_query(_bits(q), i))
+        for h in range(4):
+            assert abs(np.angle(np.exp(1j * (_basis_angle(qr[h]) - i)))) < 1e-2, (i, h)
+
+
+# ----------------------------------------------------------------------------- pooling + norm
+def pin_pool_mean(make):
+    """The pooled key before RMSNorm is the exact mean of the block's r keys:
+    keys c + d_t with sum_t d_t = 0 pool to c; order of the keys is irrelevant."""
+    o = make()
+    rng = np.random.default_rng(3)
+    c = np.round(rng.standard_normal(128) * 64) / 64
+    d = np.round(rng.standard_normal((2, 128)) * 16) / 64
+    keys = np.stack([c + d[0], c - d[0], c + d[1], c - d[1]])
+    res = o.pool_block(_bits(keys), pos=0)
+    assert np.array_equal(res["kbar"], c)
+    perm = o.pool_block(_bits(keys[[2, 0, 3, 1]]), pos=0)
+    assert np.array_equal(perm["kbar"], res["kbar"])
+    # Needle-style block: 4 identical keys pool to that key.
+    same = o.pool_block(_bits(np.tile(c, (4, 1))), pos=0)
+    assert np.array_equal(same["kbar"], c)
+
+
+def pin_rmsnorm_closed_form(make):
+    """RMSNorm (w = 1): knorm = kbar / sqrt(ms + eps), so mean(knorm^2) =
+    ms / (ms + eps) and knorm is parallel to kbar; the weight scales per dim."""
+    o = make()
+    rng = np.random.default_rng(4)
+    for scale in (1.0, 1e-3):  # at 1e-3 the eps term is half the denominator
+        keys = _bits(rng.standard_normal((4, 128)) * scale)
+        res = o.pool_block(keys, pos=0)
+        ms = np.mean(res["kbar"] ** 2)
+        assert np.isclose(np.mean(res["knorm"] ** 2), ms / (ms + 1e-6), rtol=1e-12)
+        cos = res["knorm"] @ res["kbar"] / np.linalg.norm(res["knorm"]) / np.linalg.norm(res["kbar"])
+        assert np.isclose(cos, 1.0, atol=1e-12)
+        wts = rng.uniform(0.5, 2.0, 128).astype(np.float32)
+        rw = o.pool_block(keys, pos=0, w=wts)
+        assert np.allclose(rw["knorm"], res["knorm"] * wts.astype(np.float64), rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- scores
+def pin_scores_relu_sum(make):
+    """I_ib = sum_h ReLU(<q_i^h, k_b>): with per-head dots (+1, -2, +3, -4) * s
+    the score is 4s; scores are >= 0; doubling q doubles I exactly."""
+    o = make()
+    q = np.zeros((4, 128))
+    q[:, 64] = [1.0, -2.0, 3.0, -4.0]
+    k = np.zeros((3, 128))
+    k[:, 64] = [0.5, 2.0, -1.0]
+    s = o.scores(_bits(q), _bits(k), 3)
+    assert np.array_equal(s, np.array([0.5 * 4, 2.0 * 4, 1.0 * 6], dtype=np.float32)), s
+    rng = np.random.default_rng(5)
+    qr = _bits(rng.standard_normal((4, 128)))
+    kp = _bits(rng.standard_normal((50, 128)))
+    s1 = o.scores(qr, kp, 50)
+    assert (s1 >= 0).all()
+    s2 = o.scores(_bits(bfm.bf16_to_f64(qr) * 2), kp, 50)
+    assert np.array_equal(s2, s1 * 2)
+    assert np.array_equal(o.select(s2, 7), o.select(s1, 7))
+
+
+def pin_block_causal(make):
+    """Query i scores only complete blocks b < floor(i/r); blocks at or after
+    its own block are never read (poisoned here with NaN)."""
+    w = TINY
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    idx_q, idx_k, *_ = _inputs(w)
+    pooled = o.compress(idx_k, w.n // w.r)
+    for i in (0, 3, 4, 7, 8, 101, 255):
+        c = i // w.r
+        poisoned = pooled.copy()
+        poisoned[c:] = 0x7FC0  # bf16 NaN
+        res = o.row(i, idx_q[i], poisoned)
+        assert res["scores"].size == c
+        assert np.isfinite(res["scores"]).all()
+
+
+# ----------------------------------------------------------------------------- select
+def pin_select_order(make):
+    """Top-k_B by (score desc, block asc), returned ascending: equals numpy's
+    lexsort; all-equal scores pick the lowest indices; k_B >= visible selects
+    all; the set grows monotonically with the budget."""
+    o = make()
+    rng = np.random.default_rng(6)
+    for n, k in ((1, 512), (300, 512), (5000, 512), (2000, 7)):
+        s = np.round(rng.standard_normal(n) * 4).astype(np.float32)  # many ties
+        s[rng.random(n) < 0.2] = 0.0
+        want = np.sort(np.lexsort((np.arange(n), -s.astype(np.float64)))[: min(k, n)])
+        assert np.array_equal(o.select(s, k), want), (n, k)
+    z = np.zeros(1000, dtype=np.float32)
+    assert np.array_equal(o.select(z, 10), np.arange(10))
+    s = rng.standard_normal(700).astype(np.float32)
+    prev = set()
+    for k in range(1, 60):
+        cur = set(o.select(s, k).tolist())
+        assert prev <= cur and len(cur) == k
+        prev = cur
+
+
+# ----------------------------------------------------------------------------- expand
+def pin_token_count(make):
+    """|T_i| = r * min(k_B, floor(i/r)) + (i mod r) + 1; every t <= i; no
+    duplicates; the tail r*floor(i/r) .. i is always in."""
+    w = TINY
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    idx_q, idx_k, *_ = _inputs(w)
+    pooled = o.compress(idx_k, w.n // w.r)
+    kB = o.k_blocks
+    for i in range(w.n):
+        res = o.row(i, idx_q[i], pooled, want_scores=False)
+        assert res["nsel"] == min(kB, i // w.r), i
+        toks = o.token_set(res["sel"], i)
+        assert toks.size == w.r * min(kB, i // w.r) + i % w.r + 1, i
+        assert toks.max() <= i and np.unique(toks).size == toks.size
+        assert set(range(w.r * (i // w.r), i + 1)) <= set(toks.tolist())
+
+
+# ----------------------------------------------------------------------------- attention
+def pin_attention_sdpa(make):
+    """Sparse attention on a token set equals torch's scaled_dot_product_attention
+    (fp64, CPU) on the gathered keys/values, with GQA heads h -> floor(h/g)."""
+    import torch
+
+    w = GQA
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    _, _, q, k, v = _inputs(w)
+    rng = np.random.default_rng(7)
+    for i in (5, 40, 95):
+        toks = np.sort(rng.choice(i + 1, size=min(i + 1, 30), replace=False))
+        out, lse = o.attention(q[i], k, v, toks)
+        qt = torch.from_numpy(bfm.bf16_to_f64(q[i]))[:, None, :]           # [Hq][1][d]
+        kt = torch.from_numpy(bfm.bf16_to_f64(k[toks])).permute(1, 0, 2)   # [Hkv][T][d]
+        vt = torch.from_numpy(bfm.bf16_to_f64(v[toks])).permute(1, 0, 2)
+        g = w.q_heads // w.kv_heads
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qt, kt.repeat_interleave(g, 0), vt.repeat_interleave(g, 0))[:, 0, :].numpy()
+        assert np.allclose(out, ref, rtol=0, atol=1e-10), i
+        logits = torch.einsum("hd,htd->ht", qt[:, 0], kt.repeat_interleave(g, 0)) / np.sqrt(128)
+        assert np.allclose(lse, torch.logsumexp(logits, -1).numpy(), atol=1e-10)
+
+
+def pin_dense_when_budget_covers(make):
+    """When k_B >= the visible complete blocks, QSA is dense causal attention:
+    compare with torch's causal SDPA over the whole tiny sequence (K = 1024),
+    and rows i < r*(k_B+1) at the tiny config's K = 32."""
+    import torch
+
+    w = TINY
+    _, idx_k, q, k, v = _inputs(w)
+    idx_q = _inputs(w)[0]
+    qt = torch.from_numpy(bfm.bf16_to_f64(q)).permute(1, 0, 2)  # [H][n][d]
+    kt = torch.from_numpy(bfm.bf16_to_f64(k)).permute(1, 0, 2)
+    vt = torch.from_numpy(bfm.bf16_to_f64(v)).permute(1, 0, 2)
+    g = w.q_heads // w.kv_heads
+    dense = torch.nn.functional.scaled_dot_product_attention(
+        qt, kt.repeat_interleave(g, 0), vt.repeat_interleave(g, 0), is_causal=True)
+    dense = dense.permute(1, 0, 2).numpy()
+    for K, rows in ((1024, range(0, w.n, 7)), (w.K, range(0, 4 * (8 + 1)))):
+        o = make(r=w.r, K=K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+        pooled = o.compress(idx_k, w.n // w.r)
+        for i in rows:
+            res = o.row(i, idx_q[i], pooled, q[i], k, v, want_scores=False)
+            assert np.allclose(res["out"], dense[i], rtol=0, atol=1e-9), (K, i)
+
+
+def pin_bruteforce_dense_mask(make):
+    """Every step on the tiny workload equals the dense brute force of
+    tests/bruteforce.py: pooled keys (bit-exact), scores, the selected block
+    sets (exact) and the attention output through a [n x n] mask."""
+    w = TINY
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    idx_q, idx_k, q, k, v = _inputs(w)
+    ref = bfm.layer(w, idx_q, idx_k, q, k, v)
+    pooled = o.compress(idx_k, w.n // w.r)
+    assert np.array_equal(pooled, ref["pooled"])
+    for i in range(w.n):
+        res = o.row(i, idx_q[i], pooled, q[i], k, v)
+        c = i // w.r
+        assert np.array_equal(o.rotate_query(idx_q[i], i), ref["qrot"][i])
+        assert np.allclose(res["scores"], ref["scores"][i, :c], rtol=1e-6, atol=0), i
+        assert np.array_equal(res["sel"], np.nonzero(ref["block_sel"][i])[0]), i
+        assert np.allclose(res["out"], ref["out"][i], rtol=0, atol=1e-9), i
+        assert np.allclose(res["lse"], ref["lse"][i], rtol=0, atol=1e-9), i
+
+
+def pin_needle_recall(make):
+    """Each planted needle block (keys along its probe query's direction, x4) is
+    selected by its probe query, with budget to spare for the other blocks."""
+    w = NEEDLE
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    idx_k = w.host_full("idx_k", 0)
+    pooled = o.compress(idx_k, w.n // w.r)
+    needles = w.needles(0)
+    probes = sorted({p for _, p in needles})
+    iq = w.host_rows("idx_q", 0, probes).reshape(len(probes), w.idx_heads, w.idx_dim)
+    for p, qrow in zip(probes, iq):
+        res = o.row(p, qrow, pooled)
+        want = {b for b, pp in needles if pp == p}
+        assert want <= set(res["sel"].tolist()), p
+        top = np.argsort(-res["scores"], kind="stable")[: len(want)]
+        assert set(top.tolist()) == want, p
+
+
+def pin_decode_matches_prefill_row(make):
+    """A decode step at position p (append, then query p, then pool the block it
+    closes) gives the prefill row p's selection and output, and leaves the
+    pooled cache equal to pooling the sequence."""
+    w = GQA
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    idx_q, idx_k, q, k, v = _inputs(w)
+    n0 = 80
+    kc = np.zeros_like(k)
+    vc = np.zeros_like(v)
+    ikc = np.zeros_like(idx_k)
+    kc[:n0], vc[:n0], ikc[:n0] = k[:n0], v[:n0], idx_k[:n0]
+    pooled = np.zeros((w.n // w.r, w.idx_dim), dtype=np.uint16)
+    pooled[: n0 // w.r] = o.compress(idx_k, n0 // w.r)
+    full_pooled = o.compress(idx_k, w.n // w.r)
+    for p in range(n0, w.n):
+        res = o.decode_step(p, q[p], k[p], v[p], idx_q[p], idx_k[p], kc, vc, ikc, pooled)
+        ref = o.row(p, idx_q[p], full_pooled, q[p], k, v, want_scores=False)
+        assert np.array_equal(res["sel"], ref["sel"]), p
+        assert np.allclose(res["out"], ref["out"], rtol=0, atol=1e-12), p
+    assert np.array_equal(pooled, full_pooled)
+
+
+ALL_PINS = [v for kname, v in sorted(globals().items()) if kname.startswith("pin_")]
