@@ -1,0 +1,178 @@
+"""Python binding of libqsa.so, the B200 (sm_100a) hot path of the QSA layer.
+
+Thin argument marshalling over the C-ABI of ``include/qsa.h``: every function
+below has the C entry point's name, takes torch tensors (device memory) and
+passes their pointers plus the current CUDA stream. All computation happens in
+the library's CUDA kernels; there is no fallback. Importing this module loads
+the library and raises if it has not been built (``python -m
+block_sparse_long_02_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_long_02_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+QSA_OK = 0
+STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "QSA_ERR_WORKSPACE",
+                4: "QSA_ERR_CAPACITY", 5: "QSA_ERR_CUDA", 6: "QSA_ERR_TIMEOUT", 7: "QSA_ERR_DEVICE_CHECK"}
+OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 3
+
+EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
+           "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error"]
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class qsa_config(ctypes.Structure):
+    _fields_ = [("r", ctypes.c_int32), ("K", ctypes.c_int32), ("idx_heads", ctypes.c_int32),
+                ("idx_dim", ctypes.c_int32), ("rope_dims", ctypes.c_int32), ("rope_base", ctypes.c_double),
+                ("rms_eps", ctypes.c_double), ("q_heads", ctypes.c_int32), ("kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("sm_scale", ctypes.c_double)]
+
+
+@dataclasses.dataclass
+class Config:
+    """The layer as the pages state it (r = 4, K = 2048, 4 x 128 indexer, ...)."""
+
+    r: int = 4
+    K: int = 2048
+    idx_heads: int = 4
+    idx_dim: int = 128
+    rope_dims: int = 64
+    rope_base: float = 10000.0
+    rms_eps: float = 1e-6
+    q_heads: int = 32
+    kv_heads: int = 4
+    head_dim: int = 128
+    sm_scale: float = 0.0
+
+    @property
+    def k_blocks(self) -> int:
+        return -(-self.K // self.r)
+
+    def c(self) -> qsa_config:
+        return qsa_config(self.r, self.K, self.idx_heads, self.idx_dim, self.rope_dims, self.rope_base,
+                          self.rms_eps, self.q_heads, self.kv_heads, self.head_dim, self.sm_scale)
+
+    @classmethod
+    def of(cls, w) -> "Config":
+        """From any object with the same attribute names (e.g. a synth.Workload)."""
+        return cls(**{f.name: getattr(w, f.name) for f in dataclasses.fields(cls) if hasattr(w, f.name)})
+
+
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_CFG = ctypes.POINTER(qsa_config)
+_SIGS = {
+    "qsa_workspace_size": [_CFG, _i32, _i32, _i64, _i64, ctypes.POINTER(_sz)],
+    "qsa_compress_keys": [_CFG, _i32, _vp, _i64, _vp, _i64, _i64, _vp, _vp],
+    "qsa_index_scores": [_CFG, _i32, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _sz, _vp],
+    "qsa_topk_blocks": [_CFG, _i32, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _sz, _vp],
+    "qsa_sparse_attention": [_CFG, _i32, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "qsa_decode_step": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
+                        _vp, _vp, _sz, _vp],
+    "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = ctypes.c_int
+_lib.qsa_last_error.restype = ctypes.c_char_p
+_lib.qsa_last_error.argtypes = []
+
+
+def _check(status: int) -> None:
+    if status != QSA_OK:
+        raise QSAError(status, _lib.qsa_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to libqsa must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libqsa must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def qsa_workspace_size(cfg: Config, op: int, batch: int, cap: int, nq: int = 0) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.qsa_workspace_size(ctypes.byref(cfg.c()), op, batch, cap, nq, ctypes.byref(out)))
+    return out.value
+
+
+def workspace(cfg: Config, op: int, batch: int, cap: int, nq: int = 0, device=None) -> torch.Tensor:
+    """A zero-initialised workspace of the size qsa_workspace_size reports."""
+    n = qsa_workspace_size(cfg, op, batch, cap, nq)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def qsa_compress_keys(cfg: Config, batch: int, idx_k: torch.Tensor, cap: int, rms_w, blk_begin: int,
+                      blk_end: int, pooled: torch.Tensor, stream=None) -> None:
+    _check(_lib.qsa_compress_keys(ctypes.byref(cfg.c()), batch, _ptr(idx_k), cap, _ptr(rms_w), blk_begin,
+                                  blk_end, _ptr(pooled), _stream(stream)))
+
+
+def qsa_index_scores(cfg: Config, batch: int, idx_q: torch.Tensor, q_begin: int, nq: int,
+                     pooled: torch.Tensor, cap: int, scores: torch.Tensor, ld: int, ws: torch.Tensor,
+                     stream=None) -> None:
+    _check(_lib.qsa_index_scores(ctypes.byref(cfg.c()), batch, _ptr(idx_q), q_begin, nq, _ptr(pooled), cap,
+                                 _ptr(scores), ld, _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def qsa_topk_blocks(cfg: Config, batch: int, idx_q, q_begin: int, nq: int, pooled, cap: int,
+                    scores: Optional[torch.Tensor], ld: int, sel: torch.Tensor, nsel: torch.Tensor,
+                    ws: Optional[torch.Tensor], stream=None) -> None:
+    _check(_lib.qsa_topk_blocks(ctypes.byref(cfg.c()), batch, _ptr(idx_q), q_begin, nq, _ptr(pooled), cap,
+                                _ptr(scores), ld, _ptr(sel), _ptr(nsel), _ptr(ws),
+                                0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def qsa_sparse_attention(cfg: Config, batch: int, q: torch.Tensor, q_begin: int, nq: int,
+                         k_cache: torch.Tensor, v_cache: torch.Tensor, cap: int, sel: torch.Tensor,
+                         nsel: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                         ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(_lib.qsa_sparse_attention(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache),
+                                     _ptr(v_cache), cap, _ptr(sel), _ptr(nsel), _ptr(out), _ptr(lse),
+                                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def qsa_decode_step(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, idx_k, k_cache, v_cache,
+                    idx_k_cache, pooled, cap: int, rms_w, out, sel_out=None, nsel_out=None,
+                    ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(_lib.qsa_decode_step(ctypes.byref(cfg.c()), batch, _ptr(pos), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(idx_q), _ptr(idx_k), _ptr(k_cache), _ptr(v_cache), _ptr(idx_k_cache),
+                                _ptr(pooled), cap, _ptr(rms_w), _ptr(out), _ptr(sel_out), _ptr(nsel_out),
+                                _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def qsa_workspace_status(ws: torch.Tensor, stream=None) -> int:
+    out = ctypes.c_int32(0)
+    _check(_lib.qsa_workspace_status(_ptr(ws), _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def qsa_last_error() -> str:
+    return _lib.qsa_last_error().decode()

@@ -1,0 +1,322 @@
+// The C-ABI of libqsa.so (declared in include/qsa.h): host-side validation,
+// workspace layout and stream-ordered launches. No allocation, no sync except
+// in qsa_workspace_status.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/qsa.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+qsa_status fail(qsa_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+qsa_status cuda_check(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return QSA_OK;
+    return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+qsa_status make_dims(const qsa_config* c, qsa::LayerDims* L) {
+    if (!c) return fail(QSA_ERR_INVALID_ARG, "cfg is NULL");
+    if (c->r < 1 || c->r > 64) return fail(QSA_ERR_UNSUPPORTED, "r=%d outside [1, 64]", c->r);
+    if (c->K < 1) return fail(QSA_ERR_INVALID_ARG, "K=%d must be positive", c->K);
+    const int kB = (c->K + c->r - 1) / c->r;
+    if (kB > qsa::kMaxKB) return fail(QSA_ERR_UNSUPPORTED, "k_B=%d above %d", kB, qsa::kMaxKB);
+    if (c->idx_heads != qsa::kIdxHeads || c->idx_dim != qsa::kIdxDim)
+        return fail(QSA_ERR_UNSUPPORTED, "indexer must be 4 heads x 128 dims (got %d x %d)",
+                    c->idx_heads, c->idx_dim);
+    if (c->rope_dims < 0 || c->rope_dims > qsa::kIdxDim || c->rope_dims % 8 != 0)
+        return fail(QSA_ERR_UNSUPPORTED, "rope_dims=%d must be a multiple of 8 in [0, 128]",
+                    c->rope_dims);
+    if (!(c->rope_base > 0.0)) return fail(QSA_ERR_INVALID_ARG, "rope_base must be > 0");
+    if (!(c->rms_eps >= 0.0)) return fail(QSA_ERR_INVALID_ARG, "rms_eps must be >= 0");
+    if (c->head_dim != qsa::kHeadDim)
+        return fail(QSA_ERR_UNSUPPORTED, "head_dim=%d (only 128)", c->head_dim);
+    if (c->q_heads < 1 || c->kv_heads < 1 || c->q_heads % c->kv_heads != 0)
+        return fail(QSA_ERR_UNSUPPORTED, "q_heads=%d must be a multiple of kv_heads=%d",
+                    c->q_heads, c->kv_heads);
+    if (c->q_heads / c->kv_heads > 16)
+        return fail(QSA_ERR_UNSUPPORTED, "q_heads/kv_heads=%d above 16", c->q_heads / c->kv_heads);
+    if (!(c->kv_heads == 1 || c->kv_heads == 2 || c->kv_heads == 4 || c->kv_heads == 8))
+        return fail(QSA_ERR_UNSUPPORTED, "kv_heads=%d not in {1, 2, 4, 8}", c->kv_heads);
+    L->r = c->r;
+    L->K = c->K;
+    L->kB = kB;
+    L->rope_dims = c->rope_dims;
+    L->rope_base = c->rope_base;
+    L->rms_eps = c->rms_eps;
+    L->q_heads = c->q_heads;
+    L->kv_heads = c->kv_heads;
+    L->head_dim = c->head_dim;
+    L->sm_scale = c->sm_scale > 0.0 ? (float)c->sm_scale : (float)(1.0 / std::sqrt((double)c->head_dim));
+    L->rope.half = c->rope_dims / 2;
+    for (int j = 0; j < 64; ++j)
+        L->rope.theta[j] = j < L->rope.half ? std::pow(c->rope_base, -2.0 * j / c->rope_dims) : 0.0;
+    return QSA_OK;
+}
+
+// ---------------------------------------------------------------- workspaces
+// Every workspace: [0, 256) status header, then the op's regions (256-aligned).
+struct TopkWs {
+    size_t qrot, scores, total;
+    int64_t chunk_rows, ld;
+};
+
+int64_t visible_ld(const qsa::LayerDims& L, int64_t q_begin, int64_t nq) {
+    return std::max<int64_t>(1, (q_begin + nq - 1) / L.r);
+}
+
+// Row chunk of the materialised score matrix: at most ~1 GiB of fp32 scores.
+TopkWs topk_layout(const qsa::LayerDims& L, int batch, int64_t cap, int64_t nq) {
+    TopkWs w;
+    const int64_t ld = std::max<int64_t>(1, cap / L.r);
+    int64_t rows = std::max<int64_t>(32, ((int64_t)1 << 28) / std::max<int64_t>(1, (int64_t)batch * ld));
+    rows = std::min<int64_t>(rows, std::max<int64_t>(nq, 1));
+    rows = (rows + 31) / 32 * 32;
+    w.ld = ld;
+    w.chunk_rows = rows;
+    w.qrot = qsa::kWsHeader;
+    w.scores = w.qrot + align_up((size_t)batch * std::max<int64_t>(nq, 1) * qsa::kIdxHeads * qsa::kIdxDim * 2);
+    w.total = w.scores + align_up((size_t)batch * rows * ld * 4);
+    return w;
+}
+
+struct DecodeWs {
+    size_t qrot, scores, sel, nsel, part, total;
+};
+
+DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
+    DecodeWs w;
+    const int S = qsa::decode_attention_splits(L);
+    w.qrot = qsa::kWsHeader;
+    w.scores = w.qrot + align_up((size_t)batch * qsa::kIdxHeads * qsa::kIdxDim * 2);
+    w.sel = w.scores + align_up((size_t)batch * std::max<int64_t>(1, cap / L.r) * 4);
+    w.nsel = w.sel + align_up((size_t)batch * L.kB * 4);
+    w.part = w.nsel + align_up((size_t)batch * 4);
+    w.total = w.part + align_up((size_t)batch * L.q_heads * S * 132 * 4);
+    return w;
+}
+
+size_t index_scores_ws(int batch, int64_t nq) {
+    return qsa::kWsHeader + align_up((size_t)batch * std::max<int64_t>(nq, 1) * qsa::kIdxHeads * qsa::kIdxDim * 2);
+}
+
+qsa_status check_ws(void* ws, size_t have, size_t need) {
+    if (have < need)
+        return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", have, need);
+    if (need && !ws) return fail(QSA_ERR_WORKSPACE, "workspace is NULL");
+    if (ws && !aligned16(ws)) return fail(QSA_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+    return QSA_OK;
+}
+
+#define REQUIRE_PTR(p)                                                                   \
+    do {                                                                                 \
+        if (!(p)) return fail(QSA_ERR_INVALID_ARG, "%s is NULL", #p);                    \
+        if (!aligned16(p)) return fail(QSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+    } while (0)
+
+#define TRY(x)                              \
+    do {                                    \
+        qsa_status st_ = (x);               \
+        if (st_ != QSA_OK) return st_;      \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* qsa_last_error(void) { return g_err.c_str(); }
+
+qsa_status qsa_workspace_size(const qsa_config* cfg, int32_t op, int32_t batch, int64_t cap,
+                              int64_t nq, size_t* bytes) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    if (!bytes) return fail(QSA_ERR_INVALID_ARG, "bytes is NULL");
+    if (batch < 1 || cap < 1 || nq < 0) return fail(QSA_ERR_INVALID_ARG, "bad batch/cap/nq");
+    switch (op) {
+        case QSA_OP_INDEX_SCORES: *bytes = index_scores_ws(batch, nq); break;
+        case QSA_OP_TOPK_BLOCKS: *bytes = topk_layout(L, batch, cap, nq).total; break;
+        case QSA_OP_SPARSE_ATTENTION: *bytes = qsa::kWsHeader; break;
+        case QSA_OP_DECODE_STEP: *bytes = decode_layout(L, batch, cap).total; break;
+        default: return fail(QSA_ERR_INVALID_ARG, "unknown op %d", op);
+    }
+    return QSA_OK;
+}
+
+qsa_status qsa_compress_keys(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_k,
+                             int64_t cap, const float* rms_w, int64_t blk_begin, int64_t blk_end,
+                             qsa_bf16* pooled, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    REQUIRE_PTR(idx_k);
+    REQUIRE_PTR(pooled);
+    if (rms_w && !aligned16(rms_w)) return fail(QSA_ERR_INVALID_ARG, "rms_w not 16-byte aligned");
+    if (batch < 1 || cap < 1) return fail(QSA_ERR_INVALID_ARG, "batch=%d cap=%lld", batch, (long long)cap);
+    if (blk_begin < 0 || blk_end < blk_begin)
+        return fail(QSA_ERR_INVALID_ARG, "block range [%lld, %lld)", (long long)blk_begin, (long long)blk_end);
+    if (blk_end * L.r > cap)
+        return fail(QSA_ERR_CAPACITY, "block %lld needs %lld rows, cap=%lld", (long long)blk_end - 1,
+                    (long long)(blk_end * L.r), (long long)cap);
+    return cuda_check(qsa::launch_compress(L, batch, idx_k, cap, rms_w, blk_begin, blk_end, pooled,
+                                           (cudaStream_t)stream),
+                      "qsa_compress_keys launch");
+}
+
+qsa_status qsa_index_scores(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                            int64_t q_begin, int64_t nq, const qsa_bf16* pooled, int64_t cap,
+                            float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                            qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    REQUIRE_PTR(idx_q);
+    REQUIRE_PTR(pooled);
+    if (!scores || ((uintptr_t)scores & 3u)) return fail(QSA_ERR_INVALID_ARG, "scores NULL or misaligned");
+    if (batch < 1 || cap < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (q_begin + nq > cap) return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
+    if (nq == 0) return QSA_OK;
+    if (ld < visible_ld(L, q_begin, nq))
+        return fail(QSA_ERR_INVALID_ARG, "ld=%lld below %lld visible blocks", (long long)ld, (long long)visible_ld(L, q_begin, nq));
+    TRY(check_ws(ws, ws_bytes, index_scores_ws(batch, nq)));
+    uint16_t* qrot = reinterpret_cast<uint16_t*>((char*)ws + qsa::kWsHeader);
+    cudaStream_t st = (cudaStream_t)stream;
+    TRY(cuda_check(qsa::launch_rotate_queries(L, batch, idx_q, q_begin, nq, qrot, st), "rotate"));
+    return cuda_check(qsa::launch_index_scores(L, batch, qrot, nq, q_begin, 0, nq, pooled, cap,
+                                               scores, ld, true, st),
+                      "index scores");
+}
+
+qsa_status qsa_topk_blocks(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                           int64_t q_begin, int64_t nq, const qsa_bf16* pooled, int64_t cap,
+                           const float* scores, int64_t ld, int32_t* sel, int32_t* nsel, void* ws,
+                           size_t ws_bytes, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    REQUIRE_PTR(sel);
+    if (!nsel || ((uintptr_t)nsel & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel NULL or misaligned");
+    if (batch < 1 || cap < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (q_begin + nq > cap) return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
+    if (nq == 0) return QSA_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (scores) {
+        if ((uintptr_t)scores & 3u) return fail(QSA_ERR_INVALID_ARG, "scores misaligned");
+        if (ld < visible_ld(L, q_begin, nq)) return fail(QSA_ERR_INVALID_ARG, "ld below visible blocks");
+        return cuda_check(qsa::launch_select_rows(L, batch, scores, ld, q_begin, 0, nq, nq, sel, nsel, st),
+                          "select rows");
+    }
+    REQUIRE_PTR(idx_q);
+    REQUIRE_PTR(pooled);
+    const TopkWs w = topk_layout(L, batch, cap, nq);
+    TRY(check_ws(ws, ws_bytes, w.total));
+    uint16_t* qrot = reinterpret_cast<uint16_t*>((char*)ws + w.qrot);
+    float* chunk = reinterpret_cast<float*>((char*)ws + w.scores);
+    const int64_t vld = visible_ld(L, q_begin, nq);
+    TRY(cuda_check(qsa::launch_rotate_queries(L, batch, idx_q, q_begin, nq, qrot, st), "rotate"));
+    for (int64_t j0 = 0; j0 < nq; j0 += w.chunk_rows) {
+        const int64_t rows = std::min<int64_t>(w.chunk_rows, nq - j0);
+        TRY(cuda_check(qsa::launch_index_scores(L, batch, qrot, nq, q_begin, j0, rows, pooled, cap,
+                                                chunk, vld, false, st),
+                       "index scores (chunk)"));
+        TRY(cuda_check(qsa::launch_select_rows(L, batch, chunk, vld, q_begin, j0, rows, nq, sel, nsel, st),
+                       "select rows (chunk)"));
+    }
+    return QSA_OK;
+}
+
+qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_bf16* q,
+                                int64_t q_begin, int64_t nq, const qsa_bf16* k_cache,
+                                const qsa_bf16* v_cache, int64_t cap, const int32_t* sel,
+                                const int32_t* nsel, qsa_bf16* out, float* lse, void* ws,
+                                size_t ws_bytes, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(k_cache);
+    REQUIRE_PTR(v_cache);
+    REQUIRE_PTR(sel);
+    REQUIRE_PTR(out);
+    if (!nsel || ((uintptr_t)nsel & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel NULL or misaligned");
+    if (lse && ((uintptr_t)lse & 3u)) return fail(QSA_ERR_INVALID_ARG, "lse misaligned");
+    if (batch < 1 || cap < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (q_begin + nq > cap) return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
+    (void)ws;
+    (void)ws_bytes;
+    if (nq == 0) return QSA_OK;
+    return cuda_check(qsa::launch_sparse_attention(L, batch, q, q_begin, nq, k_cache, v_cache, cap,
+                                                   sel, nsel, out, lse, (cudaStream_t)stream),
+                      "sparse attention");
+}
+
+qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* pos,
+                           const qsa_bf16* q, const qsa_bf16* k, const qsa_bf16* v,
+                           const qsa_bf16* idx_q, const qsa_bf16* idx_k, qsa_bf16* k_cache,
+                           qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap,
+                           const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
+                           void* ws, size_t ws_bytes, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    REQUIRE_PTR(pos);
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(k);
+    REQUIRE_PTR(v);
+    REQUIRE_PTR(idx_q);
+    REQUIRE_PTR(idx_k);
+    REQUIRE_PTR(k_cache);
+    REQUIRE_PTR(v_cache);
+    REQUIRE_PTR(idx_k_cache);
+    REQUIRE_PTR(pooled);
+    REQUIRE_PTR(out);
+    if (rms_w && !aligned16(rms_w)) return fail(QSA_ERR_INVALID_ARG, "rms_w not 16-byte aligned");
+    if (sel_out && ((uintptr_t)sel_out & 3u)) return fail(QSA_ERR_INVALID_ARG, "sel_out misaligned");
+    if (nsel_out && ((uintptr_t)nsel_out & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel_out misaligned");
+    if (batch < 1 || cap < 1) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    const DecodeWs w = decode_layout(L, batch, cap);
+    TRY(check_ws(ws, ws_bytes, w.total));
+    char* base = (char*)ws;
+    int32_t* status = reinterpret_cast<int32_t*>(base);
+    uint16_t* qrot = reinterpret_cast<uint16_t*>(base + w.qrot);
+    float* scores = reinterpret_cast<float*>(base + w.scores);
+    int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + w.sel);
+    int32_t* nsel = nsel_out ? nsel_out : reinterpret_cast<int32_t*>(base + w.nsel);
+    float* part = reinterpret_cast<float*>(base + w.part);
+    cudaStream_t st = (cudaStream_t)stream;
+    TRY(cuda_check(qsa::launch_decode_prepare(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache,
+                                              idx_k_cache, pooled, cap, rms_w, qrot, status, st),
+                   "decode prepare"));
+    TRY(cuda_check(qsa::launch_decode_scores(L, batch, pos, qrot, pooled, cap, scores, st), "decode scores"));
+    TRY(cuda_check(qsa::launch_select_decode(L, batch, scores, std::max<int64_t>(1, cap / L.r), pos,
+                                             cap, sel, nsel, st),
+                   "decode select"));
+    return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel,
+                                                   nsel, part, out, st),
+                      "decode attention");
+}
+
+qsa_status qsa_workspace_status(void* ws, qsa_stream stream, int32_t* status) {
+    if (!ws || !status) return fail(QSA_ERR_INVALID_ARG, "ws or status is NULL");
+    cudaStream_t st = (cudaStream_t)stream;
+    TRY(cuda_check(cudaStreamSynchronize(st), "stream sync"));
+    int32_t v = 0;
+    TRY(cuda_check(cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost), "status read"));
+    TRY(cuda_check(cudaMemset(ws, 0, sizeof(v)), "status clear"));
+    *status = v;
+    return QSA_OK;
+}
+
+}  // extern "C"

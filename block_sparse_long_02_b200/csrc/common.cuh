@@ -1,0 +1,112 @@
+// Internal helpers shared by the QSA kernels (not part of the C-ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace qsa {
+
+constexpr int kIdxDim = 128;   // indexer head dim (one shared key head)
+constexpr int kIdxHeads = 4;   // indexer query heads
+constexpr int kHeadDim = 128;  // core head dim
+constexpr int kMaxKB = 4096;   // largest supported k_B
+constexpr int kWsHeader = 256; // every workspace starts with this many bytes of status
+
+// theta_j = base^(-2j/rope_dims) for j < half, computed on the host in fp64.
+struct RopeTable {
+    double theta[64];
+    int half;
+};
+
+// ---------------------------------------------------------------- bf16 / floats
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+// fp64 -> bf16 bits, round to nearest even in a single rounding: clear all but
+// the top 7 explicit significand bits of the double with RNE, then narrow
+// (exactly) to fp32 and keep the high half.
+__device__ __forceinline__ uint16_t f64_to_bf16(double x) {
+    unsigned long long u = (unsigned long long)__double_as_longlong(x);
+    const unsigned long long half_ulp = 1ull << 44, mask = (1ull << 45) - 1ull;
+    u = (u + (half_ulp - 1ull) + ((u >> 45) & 1ull)) & ~mask;
+    float f = __double2float_rn(__longlong_as_double((long long)u));
+    return (uint16_t)(__float_as_uint(f) >> 16);
+}
+
+// fp32 -> bf16 bits, round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f32_to_bf16(float x) {
+    uint32_t u = __float_as_uint(x);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return (uint32_t)f32_to_bf16(lo) | ((uint32_t)f32_to_bf16(hi) << 16);
+}
+
+// Order-preserving map of fp32 onto uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// First error wins.
+__device__ __forceinline__ void flag_status(int32_t* status, int32_t code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+// --------------------------------------------------------------- cp.async / mma
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid) {
+    int sz = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(sz));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                            uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                  uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte chunk `c` (0..15) of 256-byte row `row` in a
+// row-swizzled tile: conflict-free ldmatrix over 8 consecutive rows.
+__device__ __forceinline__ uint32_t swz256(int row, int c) {
+    return (uint32_t)(row * 256 + ((c ^ (row & 7)) << 4));
+}
+
+}  // namespace qsa

@@ -1,0 +1,70 @@
+// Internal launchers (host side) of the QSA kernels. The C-ABI in api.cu
+// validates arguments and calls these; each returns cudaGetLastError().
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace qsa {
+
+struct LayerDims {
+    int r, K, kB;
+    int rope_dims;
+    double rope_base, rms_eps;
+    int q_heads, kv_heads, head_dim;
+    float sm_scale;  // resolved (> 0)
+    RopeTable rope;
+};
+
+// compress.cu
+cudaError_t launch_compress(const LayerDims& L, int batch, const uint16_t* idx_k, int64_t cap,
+                            const float* rms_w, int64_t blk_begin, int64_t blk_end,
+                            uint16_t* pooled, cudaStream_t st);
+cudaError_t launch_rotate_queries(const LayerDims& L, int batch, const uint16_t* idx_q,
+                                  int64_t q_begin, int64_t nq, uint16_t* qrot, cudaStream_t st);
+
+// scores.cu: fp32 scores [batch][nq][ld] from rotated queries. Queries [j0, j0+nrows)
+// of each sequence are written to rows 0..nrows-1 of `scores` (per sequence stride
+// nrows*ld). Entries b >= floor(i/r) get -inf when fill_masked, else are left.
+cudaError_t launch_index_scores(const LayerDims& L, int batch, const uint16_t* qrot, int64_t nq,
+                                int64_t q_begin, int64_t j0, int64_t nrows, const uint16_t* pooled,
+                                int64_t cap, float* scores, int64_t ld, bool fill_masked,
+                                cudaStream_t st);
+
+// topk.cu: row selection. Row (s, j) has position i = q_begin + j0 + j and
+// floor(i/r) visible entries starting at scores + ((s*nrows + j) * ld).
+cudaError_t launch_select_rows(const LayerDims& L, int batch, const float* scores, int64_t ld,
+                               int64_t q_begin, int64_t j0, int64_t nrows, int64_t nq_total,
+                               int32_t* sel, int32_t* nsel, cudaStream_t st);
+// Variant for decode: position of sequence s is pos[s]; rows [batch][ld].
+cudaError_t launch_select_decode(const LayerDims& L, int batch, const float* scores, int64_t ld,
+                                 const int64_t* pos, int64_t cap, int32_t* sel, int32_t* nsel,
+                                 cudaStream_t st);
+
+// attention.cu
+cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_t* q,
+                                    int64_t q_begin, int64_t nq, const uint16_t* kc,
+                                    const uint16_t* vc, int64_t cap, const int32_t* sel,
+                                    const int32_t* nsel, uint16_t* out, float* lse,
+                                    cudaStream_t st);
+int decode_attention_splits(const LayerDims& L);
+cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
+                                    const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                                    int64_t cap, const int32_t* sel, const int32_t* nsel,
+                                    float* part, uint16_t* out, cudaStream_t st);
+
+// decode.cu
+cudaError_t launch_decode_prepare(const LayerDims& L, int batch, const int64_t* pos,
+                                  const uint16_t* k, const uint16_t* v, const uint16_t* idx_q,
+                                  const uint16_t* idx_k, uint16_t* kc, uint16_t* vc,
+                                  uint16_t* idx_k_cache, uint16_t* pooled, int64_t cap,
+                                  const float* rms_w, uint16_t* qrot, int32_t* status,
+                                  cudaStream_t st);
+cudaError_t launch_decode_scores(const LayerDims& L, int batch, const int64_t* pos,
+                                 const uint16_t* qrot, const uint16_t* pooled, int64_t cap,
+                                 float* scores, cudaStream_t st);
+
+}  // namespace qsa

@@ -1,0 +1,66 @@
+"""QSALayer: the layer's buffers plus the call sequence of the C-ABI.
+
+Holds the per-layer caches (core K/V, raw indexer keys, pooled indexer keys)
+and the workspaces, all allocated once with torch, and issues the library
+calls in the order the layer runs them:
+
+  prefill(q, idx_q, q_begin, nq):   qsa_compress_keys -> qsa_topk_blocks (fused)
+                                    -> qsa_sparse_attention
+  decode_step(pos, q, k, v, idx_q, idx_k): qsa_decode_step
+
+Every step of the computation runs in libqsa.so; this class only owns memory
+and marshals arguments.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step,
+               qsa_sparse_attention, qsa_topk_blocks, qsa_workspace_size)
+
+
+class QSALayer:
+    def __init__(self, cfg: Config, batch: int, cap: int, device="cuda", rms_w: Optional[torch.Tensor] = None):
+        self.cfg, self.batch, self.cap = cfg, batch, cap
+        self.device = torch.device(device)
+        bf = torch.bfloat16
+        self.k_cache = torch.zeros(batch, cap, cfg.kv_heads, cfg.head_dim, dtype=bf, device=self.device)
+        self.v_cache = torch.zeros_like(self.k_cache)
+        self.idx_k_cache = torch.zeros(batch, cap, cfg.idx_dim, dtype=bf, device=self.device)
+        self.pooled = torch.zeros(batch, cap // cfg.r, cfg.idx_dim, dtype=bf, device=self.device)
+        self.rms_w = rms_w
+        self._ws = {}
+
+    def workspace(self, op: int, nq: int = 0) -> torch.Tensor:
+        need = qsa_workspace_size(self.cfg, op, self.batch, self.cap, nq)
+        ws = self._ws.get(op)
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=self.device)
+            self._ws[op] = ws
+        return ws
+
+    def compress(self, blk_begin: int, blk_end: int, stream=None) -> None:
+        qsa_compress_keys(self.cfg, self.batch, self.idx_k_cache, self.cap, self.rms_w, blk_begin, blk_end,
+                          self.pooled, stream)
+
+    def prefill(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin: int, nq: int,
+                out: torch.Tensor, sel: torch.Tensor, nsel: torch.Tensor,
+                lse: Optional[torch.Tensor] = None, stream=None) -> None:
+        """Queries [q_begin, q_begin + nq) of every sequence, whose keys and values
+        (positions < q_begin + nq) are already in the caches."""
+        r = self.cfg.r
+        self.compress(q_begin // r, (q_begin + nq) // r, stream)
+        ws = self.workspace(OP_TOPK_BLOCKS, nq)
+        qsa_topk_blocks(self.cfg, self.batch, idx_q, q_begin, nq, self.pooled, self.cap, None, 0, sel, nsel,
+                        ws, stream)
+        qsa_sparse_attention(self.cfg, self.batch, q, q_begin, nq, self.k_cache, self.v_cache, self.cap, sel,
+                             nsel, out, lse, None, stream)
+
+    def decode_step(self, pos: torch.Tensor, q, k, v, idx_q, idx_k, out, sel_out=None, nsel_out=None,
+                    stream=None) -> None:
+        ws = self.workspace(OP_DECODE_STEP)
+        qsa_decode_step(self.cfg, self.batch, pos, q, k, v, idx_q, idx_k, self.k_cache, self.v_cache,
+                        self.idx_k_cache, self.pooled, self.cap, self.rms_w, out, sel_out, nsel_out, ws,
+                        stream)

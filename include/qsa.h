@@ -1,0 +1,193 @@
+/*
+ * qsa.h: C-ABI of libqsa.so, the B200 (sm_100a) hot path of the QSA (Qwen
+ * Sparse Attention) layer.
+ *
+ * The layer, as the pages state it:
+ *   "QSA (Qwen Sparse Attention)" concept page, "Key math / How it works":
+ *     (A) compressed lightweight indexer: 4 query heads + 1 shared key head of
+ *         128 dims; keys average-pooled into blocks of r tokens, RMSNorm'd,
+ *         partial RoPE on 64 of 128 dims after compression; block importance
+ *         I_ib = sum_h ReLU(<q_i^h, k_b>) under block-causal masking; keep the
+ *         k_B = ceil(K/r) best blocks, expand them to tokens, always add the
+ *         tail of the current block;
+ *     (B) sparse core attention: full scaled-dot-product attention restricted
+ *         to the selected tokens. "Config": K = 2048, r = 4.
+ *   "Qwen Sparse Attention" gallery page, "How block selection works": pooled
+ *     keys are normalised, then rotated at the first position of each block.
+ *
+ * Conventions (all entry points):
+ *   - bf16 tensors are passed as qsa_bf16 (the 16-bit pattern); all tensor
+ *     pointers are DEVICE pointers unless stated, 16-byte aligned, contiguous,
+ *     row-major in the layouts given. The caller owns every buffer.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream). Arguments are validated on the host before any launch;
+ *     a bad argument returns an error status and launches nothing.
+ *   - The library never allocates device memory: scratch comes from a caller
+ *     workspace sized by qsa_workspace_size(). The first 256 bytes of a
+ *     workspace hold a device status word and must be zero before first use
+ *     (qsa_workspace_status reads and re-clears it).
+ *   - No exceptions cross the ABI; qsa_last_error() returns a thread-local
+ *     message for the last non-OK status of the calling thread.
+ *   - Positions are 0-based. Query i sees complete blocks b < floor(i/r) and
+ *     the tail tokens r*floor(i/r) .. i. Prefill queries are the consecutive
+ *     positions [q_begin, q_begin + nq); every sequence of a batch shares them.
+ *   - Supported shapes: idx_heads = 4, idx_dim = 128, rope_dims even and
+ *     <= 128, head_dim = 128, q_heads % kv_heads == 0 with q_heads/kv_heads <= 16,
+ *     kv_heads <= 8, 1 <= r <= 64, k_B = ceil(K/r) <= 4096. Others return
+ *     QSA_ERR_UNSUPPORTED.
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t qsa_bf16; /* bfloat16 bit pattern */
+typedef void* qsa_stream;  /* cudaStream_t */
+
+typedef enum {
+    QSA_OK = 0,
+    QSA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative or inconsistent size */
+    QSA_ERR_UNSUPPORTED = 2,  /* shape outside the supported set above */
+    QSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than qsa_workspace_size() */
+    QSA_ERR_CAPACITY = 4,     /* a position does not fit the cache capacity */
+    QSA_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+    QSA_ERR_TIMEOUT = 6,      /* a bounded device wait expired */
+    QSA_ERR_DEVICE_CHECK = 7  /* a device-side check failed (see qsa_workspace_status) */
+} qsa_status;
+
+/* Layer configuration (the pages' statement of the layer). */
+typedef struct {
+    int32_t r;          /* block size (micro-block tokens), 4 */
+    int32_t K;          /* token budget, 2048; k_B = ceil(K / r) blocks */
+    int32_t idx_heads;  /* indexer query heads, 4 (one shared key head) */
+    int32_t idx_dim;    /* indexer head dim, 128 */
+    int32_t rope_dims;  /* dims [0, rope_dims) rotated, 64; pairs (j, j + rope_dims/2) */
+    double rope_base;   /* 10000 */
+    double rms_eps;     /* 1e-6 */
+    int32_t q_heads;    /* core query heads (32) */
+    int32_t kv_heads;   /* core kv heads (4); q head h reads kv head h / (q_heads/kv_heads) */
+    int32_t head_dim;   /* 128 */
+    double sm_scale;    /* softmax scale; <= 0 means 1/sqrt(head_dim) */
+} qsa_config;
+
+/* Operations that take a workspace. */
+typedef enum {
+    QSA_OP_INDEX_SCORES = 0,     /* qsa_index_scores */
+    QSA_OP_TOPK_BLOCKS = 1,      /* qsa_topk_blocks (both modes) */
+    QSA_OP_SPARSE_ATTENTION = 2, /* qsa_sparse_attention */
+    QSA_OP_DECODE_STEP = 3       /* qsa_decode_step */
+} qsa_op;
+
+/* Bytes of workspace `op` needs for `batch` sequences of capacity `cap` and
+ * `nq` queries per sequence (nq is ignored by QSA_OP_DECODE_STEP). Writes
+ * *bytes; never launches anything. */
+qsa_status qsa_workspace_size(const qsa_config* cfg, int32_t op, int32_t batch, int64_t cap,
+                              int64_t nq, size_t* bytes);
+
+/* a1-a3 (concept page (A) "Block compression" and "Partial RoPE"; gallery page
+ * "How block selection works"): for every sequence and every complete block b
+ * in [blk_begin, blk_end):
+ *   kbar = mean of idx_k rows r*b .. r*b+r-1;
+ *   kn   = kbar * (mean_j kbar_j^2 + rms_eps)^-1/2 * rms_w;
+ *   pooled[b] = RoPE at position r*b of kn on dims [0, rope_dims), as bf16 (RNE).
+ * idx_k:  [batch][cap][idx_dim] raw indexer keys.
+ * rms_w:  [idx_dim] fp32 RMSNorm weight, or NULL for all ones.
+ * pooled: [batch][cap / r][idx_dim], written for blocks [blk_begin, blk_end) only.
+ * Errors: blk_end * r > cap -> QSA_ERR_CAPACITY. */
+qsa_status qsa_compress_keys(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_k,
+                             int64_t cap, const float* rms_w, int64_t blk_begin, int64_t blk_end,
+                             qsa_bf16* pooled, qsa_stream stream);
+
+/* a3'+a4 materialised (concept page (A) "Block importance"): for query j of
+ * sequence s, at position i = q_begin + j, with q^h = RoPE_i(idx_q[s][j][h]) as bf16:
+ *   scores[s][j][b] = sum_h max(0, <q^h, pooled[s][b]>)  (fp32 accumulation)
+ *                                 for b < floor(i / r),
+ *   scores[s][j][b] = -inf        for floor(i / r) <= b < ld.
+ * idx_q:  [batch][nq][idx_heads][idx_dim] un-rotated indexer queries.
+ * pooled: [batch][cap / r][idx_dim] from qsa_compress_keys.
+ * scores: [batch][nq][ld] fp32; ld >= floor((q_begin + nq - 1) / r).
+ * ws:     qsa_workspace_size(QSA_OP_INDEX_SCORES, batch, cap, nq) bytes (holds the
+ *         rotated queries).
+ * Errors: q_begin + nq > cap -> QSA_ERR_CAPACITY. */
+qsa_status qsa_index_scores(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                            int64_t q_begin, int64_t nq, const qsa_bf16* pooled, int64_t cap,
+                            float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                            qsa_stream stream);
+
+/* a5 (concept page (A) "Top-k_B block selection"; gallery page pseudo-code
+ * top_k(scores, k=512)): for every query, the min(k_B, floor(i/r)) visible
+ * blocks ranked first by (score descending, block index ascending).
+ *   scores == NULL: fused a3'+a4+a5 from idx_q and pooled (the prefill path;
+ *                   the score matrix is never materialised in full);
+ *   scores != NULL: select from given scores laid out as qsa_index_scores
+ *                   writes them ([batch][nq][ld]); idx_q and pooled are unused.
+ * sel:  [batch][nq][k_B] int32, the selected blocks in ascending order; slots
+ *       past nsel hold -1.
+ * nsel: [batch][nq] int32.
+ * ws:   workspace of qsa_workspace_size(QSA_OP_TOPK_BLOCKS, batch, cap, nq). */
+qsa_status qsa_topk_blocks(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                           int64_t q_begin, int64_t nq, const qsa_bf16* pooled, int64_t cap,
+                           const float* scores, int64_t ld, int32_t* sel, int32_t* nsel, void* ws,
+                           size_t ws_bytes, qsa_stream stream);
+
+/* a6+a7 (concept page (B) "Sparse core attention"; gallery page
+ * attention_input = flatten(selected_blocks) + current_incomplete_block): for
+ * query i and core head h (kv head g = h / (q_heads / kv_heads)), over the
+ * tokens T_i = {r*b .. r*b+r-1 : b in sel} U {r*floor(i/r) .. i}:
+ *   out[h] = sum_t softmax_t(sm_scale * <q[h], k_cache[t][g]>) v_cache[t][g].
+ * Logits, softmax and accumulation are fp32; probabilities are rounded to bf16
+ * for the P.V product.
+ * q:       [batch][nq][q_heads][head_dim]  (already position-encoded)
+ * k_cache, v_cache: [batch][cap][kv_heads][head_dim]
+ * sel, nsel: as written by qsa_topk_blocks; entries outside [0, floor(i/r)) are
+ *          skipped (never read out of bounds).
+ * out:     [batch][nq][q_heads][head_dim] bf16.
+ * lse:     [batch][nq][q_heads] fp32 natural-log sum-exp of the scaled logits,
+ *          or NULL.
+ * ws:      qsa_workspace_size(QSA_OP_SPARSE_ATTENTION, ...) bytes (may be 0). */
+qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_bf16* q,
+                                int64_t q_begin, int64_t nq, const qsa_bf16* k_cache,
+                                const qsa_bf16* v_cache, int64_t cap, const int32_t* sel,
+                                const int32_t* nsel, qsa_bf16* out, float* lse, void* ws,
+                                size_t ws_bytes, qsa_stream stream);
+
+/* One decode step for every sequence s, at p = pos[s] (its current length):
+ *   a8: append k, v (-> k_cache/v_cache row p) and idx_k (-> idx_k_cache row p);
+ *   a3'..a7: the new token is query p: score blocks b < floor(p/r), select,
+ *       attend over the selection and the tail r*floor(p/r) .. p;
+ *   then, if (p + 1) % r == 0, pool block floor(p/r) into `pooled` (a1-a3), so
+ *       the next step sees it (gallery page: only the attention layers grow the
+ *       KV cache; the pooling time is a reading).
+ * pos:  DEVICE [batch] int64 (not modified; the caller advances it).
+ * q: [batch][q_heads][head_dim]; k, v: [batch][kv_heads][head_dim];
+ * idx_q: [batch][idx_heads][idx_dim]; idx_k: [batch][idx_dim].
+ * Caches as above with capacity cap; pooled [batch][cap/r][idx_dim].
+ * out: [batch][q_heads][head_dim] bf16; sel_out: [batch][k_B] int32 or NULL
+ * (ascending, -1 padded); nsel_out: [batch] int32 or NULL.
+ * A sequence with pos >= cap or pos < 0 is skipped and flags
+ * QSA_ERR_CAPACITY in the workspace status (qsa_workspace_status). */
+qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* pos,
+                           const qsa_bf16* q, const qsa_bf16* k, const qsa_bf16* v,
+                           const qsa_bf16* idx_q, const qsa_bf16* idx_k, qsa_bf16* k_cache,
+                           qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap,
+                           const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
+                           void* ws, size_t ws_bytes, qsa_stream stream);
+
+/* Device-side status recorded in a workspace by the calls that used it:
+ * QSA_OK, or the first error a kernel flagged (QSA_ERR_CAPACITY,
+ * QSA_ERR_DEVICE_CHECK, QSA_ERR_TIMEOUT). Synchronises `stream`, copies the
+ * word to *status and clears it. */
+qsa_status qsa_workspace_status(void* ws, qsa_stream stream, int32_t* status);
+
+/* Thread-local message describing the last non-OK status ("" if none). */
+const char* qsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QSA_H_ */

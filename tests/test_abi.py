@@ -1,0 +1,63 @@
+"""The C-ABI library loads and exports every symbol include/qsa.h declares, and
+its host-side validation answers without a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(qsa_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    from block_sparse_long_02_b200 import build
+
+    build.build()
+    import block_sparse_long_02_b200 as m
+
+    return m
+
+
+def test_every_declared_symbol_is_exported(qsa):
+    names = _declared()
+    assert "qsa_decode_step" in names and len(names) >= 8
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(qsa.EXPORTS) <= set(names)
+
+
+def test_workspace_sizes_and_config_validation(qsa):
+    cfg = qsa.Config()
+    n = qsa.qsa_workspace_size(cfg, qsa.OP_DECODE_STEP, 8, 262144 + 64)
+    assert n >= 8 * 65536 * 4  # at least the fp32 score row per sequence
+    assert qsa.qsa_workspace_size(cfg, qsa.OP_SPARSE_ATTENTION, 1, 1024, 1024) == 256
+    for bad, status in ((dict(idx_heads=8), 2), (dict(head_dim=64), 2), (dict(q_heads=30, kv_heads=4), 2),
+                        (dict(r=0), 2), (dict(K=0), 1), (dict(rope_dims=60), 2), (dict(kv_heads=3, q_heads=24), 2)):
+        c = qsa.Config(**bad)
+        with pytest.raises(qsa.QSAError) as e:
+            qsa.qsa_workspace_size(c, qsa.OP_TOPK_BLOCKS, 1, 1024, 16)
+        assert e.value.status == status, bad
+
+
+def test_null_and_capacity_errors_launch_nothing(qsa):
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    lib.qsa_compress_keys.restype = ctypes.c_int
+    cfg = qsa.Config().c()
+    # NULL idx_k -> INVALID_ARG before any CUDA call.
+    st = lib.qsa_compress_keys(ctypes.byref(cfg), 1, None, ctypes.c_int64(64), None, ctypes.c_int64(0),
+                               ctypes.c_int64(1), ctypes.c_void_p(256), None)
+    assert st == 1
+    # Block range past the capacity -> CAPACITY (fake, aligned, never dereferenced pointers).
+    st = lib.qsa_compress_keys(ctypes.byref(cfg), 1, ctypes.c_void_p(4096), ctypes.c_int64(64), None,
+                               ctypes.c_int64(0), ctypes.c_int64(17), ctypes.c_void_p(8192), None)
+    assert st == 4
+    lib.qsa_last_error.restype = ctypes.c_char_p
+    assert b"cap" in lib.qsa_last_error()

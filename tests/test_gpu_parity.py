@@ -1,0 +1,359 @@
+"""CUDA path (through the C-ABI) against the oracle, element by element, on the
+same seeded inputs. Sizes span several query/block tiles with ragged tails;
+each stage is fed the GPU's previous-stage output so tolerated differences do
+not cascade. Parity rules live in gpu_util."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import (bits, check_attention, check_scores, check_selection, dev_full, f32, score_tol,
+                      LSE_ATOL)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qsa():
+    import block_sparse_long_02_b200 as m
+
+    return m
+
+
+def _layer(qsa, w, cap, **over):
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    cfg = qsa.Config.of(w)
+    for k, v in over.items():
+        setattr(cfg, k, v)
+    return cfg, QSALayer(cfg, w.batch, cap)
+
+
+def _fill_caches(w, L, T):
+    w.device_fill("k", L.k_cache.view(w.batch, L.cap, -1), rows=(0, T))
+    w.device_fill("v", L.v_cache.view(w.batch, L.cap, -1), rows=(0, T))
+    w.device_fill("idx_k", L.idx_k_cache, rows=(0, T))
+
+
+def run_prefill(qsa, w, q_begin=0, nq=None, cap=None, lse=True, **over):
+    nq = w.n - q_begin if nq is None else nq
+    cap = cap or (q_begin + nq)
+    cfg, L = _layer(qsa, w, cap, **over)
+    _fill_caches(w, L, q_begin + nq)
+    iq = dev_full(w, "idx_q", cap, q_begin + nq)[:, q_begin:q_begin + nq].contiguous()
+    qq = dev_full(w, "q", cap, q_begin + nq)[:, q_begin:q_begin + nq].contiguous()
+    out = torch.empty(w.batch, nq, cfg.q_heads, cfg.head_dim, dtype=torch.bfloat16, device="cuda")
+    sel = torch.full((w.batch, nq, cfg.k_blocks), -7, dtype=torch.int32, device="cuda")
+    nsel = torch.full((w.batch, nq), -7, dtype=torch.int32, device="cuda")
+    lse_t = torch.empty(w.batch, nq, cfg.q_heads, dtype=torch.float32, device="cuda") if lse else None
+    if q_begin // cfg.r:
+        L.compress(0, q_begin // cfg.r)
+    L.prefill(qq, iq.view(w.batch, nq, 4, 128), q_begin, nq, out, sel, nsel, lse_t)
+    torch.cuda.synchronize()
+    return cfg, {"pooled": bits(L.pooled), "sel": sel.cpu().numpy(), "nsel": nsel.cpu().numpy(),
+                 "out": out.float().cpu().numpy(), "lse": None if lse_t is None else lse_t.cpu().numpy()}
+
+
+def _oracle(w, cfg):
+    return oracle.Oracle(r=cfg.r, K=cfg.K, q_heads=cfg.q_heads, kv_heads=cfg.kv_heads,
+                         rope_dims=cfg.rope_dims, rope_base=cfg.rope_base, rms_eps=cfg.rms_eps)
+
+
+def check_rows(w, cfg, res, rows, s=0, q_begin=0, attention=True):
+    o = _oracle(w, cfg)
+    T = q_begin + res["sel"].shape[1]
+    idx_q = w.host_full("idx_q", s, T).reshape(T, 4, 128)
+    q = w.host_full("q", s, T).reshape(T, cfg.q_heads, 128)
+    k = w.host_full("k", s, T).reshape(T, cfg.kv_heads, 128)
+    v = w.host_full("v", s, T).reshape(T, cfg.kv_heads, 128)
+    pooled = res["pooled"][s]
+    for i in rows:
+        j = i - q_begin
+        ref = o.row(i, idx_q[i], pooled)
+        tol = score_tol(o.rotate_query(idx_q[i], i), pooled, ref["scores"])
+        check_selection(res["sel"][s, j], res["nsel"][s, j], ref["scores"], tol, o.k_blocks, f"s{s} row {i}")
+        if attention:
+            n = res["nsel"][s, j]
+            toks = o.token_set(res["sel"][s, j, :n], i)
+            out_ref, lse_ref = o.attention(q[i], k, v, toks)
+            check_attention(res["out"][s, j], out_ref, f"s{s} row {i}")
+            if res["lse"] is not None:
+                assert np.abs(res["lse"][s, j] - lse_ref).max() <= LSE_ATOL, i
+
+
+# ----------------------------------------------------------------------------- a1-a3
+@pytest.mark.parametrize("n,batch", [(256, 1), (4096 + 12, 2), (1003, 1)])
+def test_compress_matches_oracle(qsa, n, batch):
+    w = synth.Workload(name="t", n=n, batch=batch, K=64, q_heads=8, kv_heads=2, base_seed=0xC0 + n)
+    cfg, L = _layer(qsa, w, n)
+    _fill_caches(w, L, n)
+    L.compress(0, n // 4)
+    torch.cuda.synchronize()
+    got = bits(L.pooled)
+    o = _oracle(w, cfg)
+    for s in range(batch):
+        ref = o.compress(w.host_full("idx_k", s), n // 4)
+        d = np.abs(got[s].astype(np.int32) - ref.astype(np.int32))
+        assert d.max() <= 1, f"pooled keys differ by {d.max()} bf16 ulp"
+        assert (d == 0).mean() > 0.9999
+
+
+def test_compress_subrange_and_weight(qsa):
+    w = synth.Workload(name="t", n=512, K=64, q_heads=4, kv_heads=1, base_seed=0xC1)
+    cfg, L = _layer(qsa, w, 512)
+    _fill_caches(w, L, 512)
+    L.rms_w = torch.linspace(0.5, 2.0, 128, device="cuda", dtype=torch.float32)
+    L.pooled.fill_(0)
+    L.compress(10, 50)
+    torch.cuda.synchronize()
+    got = bits(L.pooled)[0]
+    ref = _oracle(w, cfg).compress(w.host_full("idx_k", 0), 128, w=L.rms_w.cpu().numpy())
+    assert (got[:10] == 0).all() and (got[50:] == 0).all()
+    assert np.abs(got[10:50].astype(np.int32) - ref[10:50].astype(np.int32)).max() <= 1
+
+
+# ----------------------------------------------------------------------------- a4
+@pytest.mark.parametrize("n,q_begin", [(256, 0), (2003, 0), (2003, 1100)])
+def test_index_scores_match_oracle(qsa, n, q_begin):
+    w = synth.Workload(name="t", n=n, K=64, q_heads=4, kv_heads=1, base_seed=0xD0 + n + q_begin)
+    cfg, L = _layer(qsa, w, n)
+    _fill_caches(w, L, n)
+    L.compress(0, n // 4)
+    nq = n - q_begin
+    iq = dev_full(w, "idx_q", n)[:, q_begin:].contiguous()
+    ld = (n - 1) // 4 + 3
+    scores = torch.full((1, nq, ld), 7.0, device="cuda")
+    ws = qsa.workspace(cfg, qsa.OP_INDEX_SCORES, 1, n, nq)
+    qsa.qsa_index_scores(cfg, 1, iq, q_begin, nq, L.pooled, n, scores, ld, ws)
+    torch.cuda.synchronize()
+    got = scores.cpu().numpy()[0]
+    pooled = bits(L.pooled)[0]
+    o = _oracle(w, cfg)
+    idx_q = w.host_full("idx_q", 0).reshape(n, 4, 128)
+    for j in range(nq):
+        i = q_begin + j
+        c = i // 4
+        ref = o.scores(o.rotate_query(idx_q[i], i), pooled, c)
+        check_scores(got[j, :c], ref, score_tol(o.rotate_query(idx_q[i], i), pooled, ref), f"row {i}")
+        assert np.isneginf(got[j, c:]).all(), i
+
+
+# ----------------------------------------------------------------------------- a5
+def test_select_from_scores_is_exact(qsa):
+    """Selection is integer work: given the same scores it must equal the oracle's
+    selection exactly, including heavy ties (rounded and zero scores)."""
+    rng = np.random.default_rng(3)
+    cfg = qsa.Config(K=64, q_heads=4, kv_heads=1)  # k_B = 16
+    nq, q_begin = 300, 5000
+    ld = (q_begin + nq - 1) // 4
+    sc = np.round(rng.standard_normal((1, nq, ld)) * 3).astype(np.float32)
+    sc[:, : nq // 3] = 0.0                                # all-tie rows
+    sc[:, nq // 3: nq // 2] = np.abs(sc[:, nq // 3: nq // 2])  # many ties
+    sc[:, -5:] = rng.standard_normal((5, ld)).astype(np.float32)
+    scores = torch.from_numpy(sc).cuda()
+    sel = torch.empty(1, nq, 16, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(1, nq, dtype=torch.int32, device="cuda")
+    qsa.qsa_topk_blocks(cfg, 1, None, q_begin, nq, None, q_begin + nq, scores, ld, sel, nsel, None)
+    torch.cuda.synchronize()
+    o = oracle.Oracle(K=64, q_heads=4, kv_heads=1)
+    g = sel.cpu().numpy()[0]
+    for j in range(nq):
+        c = (q_begin + j) // 4
+        ref = o.select(sc[0, j, :c])
+        assert np.array_equal(g[j], ref), j
+    assert (nsel.cpu().numpy() == 16).all()
+
+
+def test_select_candidate_overflow_path(qsa):
+    """More than 4096 exactly equal scores at the threshold digit: the general path."""
+    cfg = qsa.Config(K=2048, q_heads=4, kv_heads=1)
+    ld = 60000
+    sc = np.zeros((1, 2, ld), dtype=np.float32)
+    sc[0, 1, ::7] = 1.0
+    scores = torch.from_numpy(sc).cuda()
+    sel = torch.empty(1, 2, 512, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(1, 2, dtype=torch.int32, device="cuda")
+    qsa.qsa_topk_blocks(cfg, 1, None, 4 * ld, 2, None, 4 * ld + 2, scores, ld, sel, nsel, None)
+    torch.cuda.synchronize()
+    o = oracle.Oracle(K=2048)
+    for j in range(2):
+        assert np.array_equal(sel.cpu().numpy()[0, j], o.select(sc[0, j, : (4 * ld + j) // 4]))
+
+
+# ----------------------------------------------------------------------------- a1..a7 prefill
+def test_tiny_prefill_all_rows(qsa):
+    w = synth.WORKLOADS["tiny_prefill_n256"]
+    cfg, res = run_prefill(qsa, w)
+    check_rows(w, cfg, res, range(w.n))
+
+
+@pytest.mark.parametrize("q_heads,kv_heads", [(32, 4), (8, 1), (16, 2), (64, 8), (16, 4)])
+def test_prefill_ragged_gqa(qsa, q_heads, kv_heads):
+    w = synth.Workload(name="t", n=2003, K=128, q_heads=q_heads, kv_heads=kv_heads,
+                       base_seed=0xE0 + q_heads, n_needles_prefill=6)
+    cfg, res = run_prefill(qsa, w)
+    rows = sorted(set(list(range(0, 40)) + list(range(1960, 2003)) +
+                      np.random.default_rng(1).integers(0, 2003, 40).tolist() + [p for _, p in w.needles(0)]))
+    check_rows(w, cfg, res, rows)
+
+
+def test_prefill_chunk_with_offset_and_batch(qsa):
+    w = synth.Workload(name="t", n=1500, batch=2, K=96, q_heads=8, kv_heads=2, base_seed=0xE7)
+    cfg, res = run_prefill(qsa, w, q_begin=701, nq=799)
+    rows = list(range(701, 740)) + list(range(1460, 1500))
+    for s in range(2):
+        check_rows(w, cfg, res, rows, s=s, q_begin=701)
+
+
+def test_budget_covering_all_blocks_is_dense(qsa):
+    """k_B >= visible blocks: every visible block is selected, in order."""
+    w = synth.Workload(name="t", n=600, K=4096, q_heads=8, kv_heads=2, base_seed=0xE8)
+    cfg, res = run_prefill(qsa, w)
+    for i in range(600):
+        c = i // 4
+        assert res["nsel"][0, i] == c and np.array_equal(res["sel"][0, i, :c], np.arange(c))
+    check_rows(w, cfg, res, [0, 1, 3, 4, 5, 77, 598, 599])
+
+
+@pytest.mark.parametrize("r", [1, 8])
+def test_generic_block_size(qsa, r):
+    w = synth.Workload(name="t", n=777, r=r, K=96, q_heads=8, kv_heads=2, base_seed=0xE9 + r)
+    cfg, res = run_prefill(qsa, w)
+    check_rows(w, cfg, res, list(range(0, 20)) + list(range(700, 777)))
+
+
+def test_invalid_selection_entries_are_skipped(qsa):
+    """Entries outside [0, floor(i/r)) never read memory; they drop out of the set."""
+    w = synth.Workload(name="t", n=512, K=64, q_heads=8, kv_heads=2, base_seed=0xEA)
+    cfg, L = _layer(qsa, w, 512)
+    _fill_caches(w, L, 512)
+    q = dev_full(w, "q", 512)
+    nq = 512
+    sel = torch.full((1, nq, 16), -1, dtype=torch.int32, device="cuda")
+    nsel = torch.full((1, nq), 16, dtype=torch.int32, device="cuda")
+    rng = np.random.default_rng(4)
+    raw = rng.integers(-5, 200, (nq, 16)).astype(np.int32)
+    raw[:, 0] = 10**9
+    sel.copy_(torch.from_numpy(raw)[None])
+    out = torch.empty(1, nq, 8, 128, dtype=torch.bfloat16, device="cuda")
+    qsa.qsa_sparse_attention(cfg, 1, q, 0, nq, L.k_cache, L.v_cache, 512, sel, nsel, out)
+    torch.cuda.synchronize()
+    o = _oracle(w, cfg)
+    qh = w.host_full("q", 0).reshape(512, 8, 128)
+    k = w.host_full("k", 0).reshape(512, 2, 128)
+    v = w.host_full("v", 0).reshape(512, 2, 128)
+    got = out.float().cpu().numpy()[0]
+    for i in [3, 50, 200, 511]:
+        valid = np.array([b for b in raw[i] if 0 <= b < i // 4], dtype=np.int32)
+        toks = np.concatenate([np.arange(4 * b, 4 * b + 4) for b in valid] +
+                              [np.arange(4 * (i // 4), i + 1)]).astype(np.int64)
+        ref, _ = o.attention(qh[i], k, v, toks)
+        check_attention(got[i], ref, f"row {i}")
+
+
+def test_host_errors(qsa):
+    cfg = qsa.Config()
+    t = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(qsa.QSAError) as e:
+        qsa.qsa_compress_keys(cfg, 1, t, 16, None, 0, 5, t)
+    assert e.value.status == 4
+    sel = torch.zeros(512, dtype=torch.int32, device="cuda")
+    with pytest.raises(qsa.QSAError) as e:
+        qsa.qsa_sparse_attention(cfg, 1, t, 10, 10, t, t, 15, sel, sel, t)
+    assert e.value.status == 4
+    with pytest.raises(qsa.QSAError) as e:
+        qsa.qsa_topk_blocks(cfg, 1, t, 0, 8, t, 64, None, 0, sel, sel, torch.zeros(8, dtype=torch.uint8,
+                                                                                  device="cuda"))
+    assert e.value.status == 3
+
+
+# ----------------------------------------------------------------------------- decode
+def _decode_run(qsa, w, starts, steps, check=True):
+    """Decode `steps` tokens per sequence starting at positions `starts` (one per
+    sequence); compare every step with the oracle's decode step."""
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    B = w.batch
+    cfg = qsa.Config.of(w)
+    cap = max(starts) + steps + 3
+    L = QSALayer(cfg, B, cap)
+    T = max(starts) + steps
+    full = {n: dev_full(w, n, cap, T) for n in ("q", "k", "v", "idx_q", "idx_k")}
+    for s in range(B):
+        for n, c in (("k", L.k_cache), ("v", L.v_cache), ("idx_k", L.idx_k_cache)):
+            c.view(B, cap, -1)[s, : starts[s]] = full[n][s, : starts[s]]
+    for s in range(B):
+        from block_sparse_long_02_b200 import qsa_compress_keys
+
+        qsa_compress_keys(cfg, 1, L.idx_k_cache[s:s + 1], cap, None, 0, starts[s] // cfg.r, L.pooled[s:s + 1])
+    o = _oracle(w, cfg)
+    host = [{n: w.host_full(n, s, T) for n in ("q", "k", "v", "idx_q", "idx_k")} for s in range(B)]
+    oc = []
+    for s in range(B):
+        kc = np.zeros((cap, cfg.kv_heads * 128), np.uint16)
+        vc = np.zeros_like(kc)
+        ik = np.zeros((cap, 128), np.uint16)
+        kc[: starts[s]] = host[s]["k"][: starts[s]]
+        vc[: starts[s]] = host[s]["v"][: starts[s]]
+        ik[: starts[s]] = host[s]["idx_k"][: starts[s]]
+        pooled = np.zeros((cap // cfg.r, 128), np.uint16)
+        pooled[: starts[s] // cfg.r] = o.compress(ik, starts[s] // cfg.r)
+        oc.append((kc, vc, ik, pooled))
+    pos = torch.tensor(starts, dtype=torch.int64, device="cuda")
+    out = torch.empty(B, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(B, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(B, dtype=torch.int32, device="cuda")
+    ar = torch.arange(B, device="cuda")
+    for step in range(steps):
+        p = pos.clone()
+        args = [full[n][ar, p].contiguous() for n in ("q", "k", "v", "idx_q", "idx_k")]
+        L.decode_step(pos, *args, out, sel, nsel)
+        torch.cuda.synchronize()
+        if check:
+            g_out, g_sel, g_nsel = out.float().cpu().numpy(), sel.cpu().numpy(), nsel.cpu().numpy()
+            g_pooled = bits(L.pooled)
+            for s in range(B):
+                ps = starts[s] + step
+                kc, vc, ik, pooled = oc[s]
+                hs = host[s]
+                # Scores of the oracle on the GPU's pooled keys (stage-by-stage feeding).
+                ref = o.row(ps, hs["idx_q"][ps].reshape(4, 128), g_pooled[s])
+                tol = score_tol(o.rotate_query(hs["idx_q"][ps].reshape(4, 128), ps), g_pooled[s], ref["scores"])
+                check_selection(g_sel[s], g_nsel[s], ref["scores"], tol, cfg.k_blocks, f"s{s} p{ps}")
+                res = o.decode_step(ps, hs["q"][ps], hs["k"][ps], hs["v"][ps], hs["idx_q"][ps], hs["idx_k"][ps],
+                                    kc, vc, ik, pooled)
+                toks = o.token_set(g_sel[s, : g_nsel[s]], ps)
+                out_ref, _ = o.attention(hs["q"][ps], kc, vc, toks)
+                check_attention(g_out[s], out_ref.reshape(cfg.q_heads, 128), f"s{s} p{ps}")
+                # Cache update: the GPU's pooled cache equals the oracle's (<= 1 ulp).
+                assert np.abs(g_pooled[s].astype(np.int32)[: (ps + 1) // cfg.r]
+                              - pooled.astype(np.int32)[: (ps + 1) // cfg.r]).max(initial=0) <= 1
+        pos += 1
+    return L
+
+
+def test_decode_steps_match_oracle(qsa):
+    w = synth.Workload(name="t", n=777, batch=2, decode_steps=12, prefill=False, K=128, q_heads=16,
+                       kv_heads=2, base_seed=0xF0, n_needles_decode=3)
+    _decode_run(qsa, w, [777, 782], 12)
+
+
+def test_decode_short_context_and_capacity_flag(qsa):
+    w = synth.Workload(name="t", n=0, batch=1, decode_steps=9, prefill=False, K=16, q_heads=8,
+                       kv_heads=2, base_seed=0xF1)
+    L = _decode_run(qsa, w, [0], 9)
+    # A position at or beyond the capacity is skipped and flagged in the workspace.
+    cfg = L.cfg
+    pos = torch.tensor([L.cap], dtype=torch.int64, device="cuda")
+    z = torch.zeros(1, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros(1, cfg.kv_heads, 128, dtype=torch.bfloat16, device="cuda")
+    iq = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
+    ik = torch.zeros(1, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(z)
+    L.decode_step(pos, z, kv, kv, iq, ik, out)
+    ws = L.workspace(qsa.OP_DECODE_STEP)
+    assert qsa.qsa_workspace_status(ws) == 4
+    assert qsa.qsa_workspace_status(ws) == 0
