@@ -1,0 +1,515 @@
+#!/usr/bin/env python
+"""QSA layer benchmark: prefill + decode tokens/s at 1M context on B200.
+
+One step = one pass of the whole hot path over the workload
+"prefill_n1m_decode64": key pooling, fused indexer score + top-k_B selection
+and sparse attention for all 1,048,576 prefill positions of one sequence, then
+64 decode steps (append, score, select, attend, pool). Inputs are synthetic
+(seeded), resident in HBM before timing; they are far larger than L2 (q 8.6 GB,
+K/V 2.1 GB), and decode steps run back to back as in real decoding.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun), every rank runs an
+independent replica (the layer has no cross-GPU exchange); time is the max
+over ranks and value counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "QSA layer prefill & decode tokens/s at 256K/1M ctx; % of HBM/tensor roofline"
+DEFAULT_WORKLOAD = "prefill_n1m_decode64"
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def algorithmic(w):
+    """Per-step algorithmic work (the units the roofline divides by)."""
+    r, kB, n = w.r, w.k_blocks, w.n
+    i = np.arange(n, dtype=np.int64)
+    vis = i // r
+    pairs = int(vis.sum()) if w.prefill else 0
+    tok = (r * np.minimum(kB, vis) + i % r + 1) if w.prefill else np.zeros(0, np.int64)
+    sum_t = int(tok.sum())
+    d = w.head_dim
+    out = {
+        "compress_bytes": (n * w.idx_dim * 2 + (n // r) * w.idx_dim * 2) if w.prefill else 0,
+        "index_flops": pairs * w.idx_heads * w.idx_dim * 2,
+        "attn_gather_bytes": sum_t * w.kv_heads * d * 2 * 2,
+        "attn_flops": sum_t * w.q_heads * d * 4,
+        "prefill_tokens": n if w.prefill else 0,
+    }
+    dec = 0
+    dec_tok = 0
+    for s in range(w.decode_steps):
+        p = w.n + s
+        nb = p // r
+        t = r * min(kB, nb) + p % r + 1
+        dec += nb * w.idx_dim * 2 + t * w.kv_heads * d * 2 * 2
+        dec_tok += 1
+    out["decode_bytes"] = dec * w.batch
+    out["decode_tokens"] = dec_tok * w.batch
+    out["prefill_tokens"] *= w.batch
+    for k in ("compress_bytes", "index_flops", "attn_gather_bytes", "attn_flops"):
+        out[k] *= w.batch
+    return out
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (clocks and throttle reasons)."""
+
+    Q = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.bus_id = bus_id if isinstance(bus_id, int) else None  # PCI bus number of our GPU
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except FileNotFoundError:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        try:
+            return self._stop()
+        except Exception as e:  # the sampler must never abort a measurement
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"sampler error: {e}"]}
+
+    def _stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) >= 10:
+                rows.append(f)
+
+        def bus(f):
+            try:
+                return int(f[1].split(":")[1], 16)
+            except (IndexError, ValueError):
+                return None
+
+        mine = [f for f in rows if self.bus_id is not None and bus(f) == self.bus_id]
+        if mine:
+            rows = mine
+        elif len({f[0] for f in rows}) > 1:
+            rows = [f for f in rows if f[0] == rows[0][0]]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(f[2]) for f in rows if f[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for f in rows:
+            for nm, v in zip(names, f[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(rows[0][3]) if rows[0][3].replace(".", "").isdigit() else None,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(float(f[4]) for f in rows if f[4].replace(".", "").isdigit())}
+
+
+def traffic_for(stage: str):
+    """DRAM bytes per launch of a stage from the committed ncu summary, or None
+    when that summary was taken on a different version of the kernel source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    for ln in open(p):
+        f = ln.split("#")[0].split()
+        if len(f) == 3 and f[0] == stage:
+            src = os.path.join(ROOT, "block_sparse_long_02_b200", "csrc")
+            h = hashlib.sha1()
+            for name in sorted(os.listdir(src)):
+                h.update(open(os.path.join(src, name), "rb").read())
+            return float(f[1]) if h.hexdigest()[:12] == f[2] else None
+    return None
+
+
+# ----------------------------------------------------------------------------- CUDA arm
+class Bench:
+    def __init__(self, w, device):
+        import block_sparse_long_02_b200 as qsa
+        from block_sparse_long_02_b200.layer import QSALayer
+
+        self.qsa, self.w, self.dev = qsa, w, device
+        cfg = qsa.Config.of(w)
+        self.cfg = cfg
+        B, n, S = w.batch, w.n, w.decode_steps
+        cap = -(-(n + S) // w.r) * w.r
+        self.L = L = QSALayer(cfg, B, cap, device=device)
+        bf = torch.bfloat16
+        w.device_fill("k", L.k_cache.view(B, cap, -1), rows=(0, n))
+        w.device_fill("v", L.v_cache.view(B, cap, -1), rows=(0, n))
+        w.device_fill("idx_k", L.idx_k_cache, rows=(0, n))
+        self.pre = None
+        if w.prefill:
+            q = torch.empty(B, n, cfg.q_heads, cfg.head_dim, dtype=bf, device=device)
+            iq = torch.empty(B, n, cfg.idx_heads, cfg.idx_dim, dtype=bf, device=device)
+            w.device_fill("q", q.view(B, n, -1), rows=(0, n))
+            w.device_fill("idx_q", iq.view(B, n, -1), rows=(0, n))
+            self.pre = {"q": q, "idx_q": iq,
+                        "out": torch.empty_like(q),
+                        "sel": torch.empty(B, n, cfg.k_blocks, dtype=torch.int32, device=device),
+                        "nsel": torch.empty(B, n, dtype=torch.int32, device=device)}
+        else:
+            L.compress(0, n // w.r)
+        self.dec = []
+        if S:
+            tmp = {}
+            for name in ("q", "k", "v", "idx_q", "idx_k"):
+                t = torch.empty(B, S, w.row_len(name), dtype=bf, device=device)
+                for s in range(B):
+                    synth.fill_device(w.seed(s), synth.TENSOR_IDS[name], n * w.row_len(name),
+                                      S * w.row_len(name), t[s].data_ptr())
+                tmp[name] = t
+            # Needle rows of decode positions are raw indexer keys of earlier blocks
+            # (already in the cache); the decode tokens themselves carry no needles.
+            for st in range(S):
+                self.dec.append({
+                    "pos": torch.full((B,), n + st, dtype=torch.int64, device=device),
+                    "q": tmp["q"][:, st].contiguous().view(B, cfg.q_heads, cfg.head_dim),
+                    "k": tmp["k"][:, st].contiguous().view(B, cfg.kv_heads, cfg.head_dim),
+                    "v": tmp["v"][:, st].contiguous().view(B, cfg.kv_heads, cfg.head_dim),
+                    "idx_q": tmp["idx_q"][:, st].contiguous().view(B, cfg.idx_heads, cfg.idx_dim),
+                    "idx_k": tmp["idx_k"][:, st].contiguous(),
+                    "out": torch.empty(B, cfg.q_heads, cfg.head_dim, dtype=bf, device=device),
+                })
+        # Workspaces allocated before timing.
+        if w.prefill:
+            L.workspace(qsa.OP_TOPK_BLOCKS, n)
+        if S:
+            L.workspace(qsa.OP_DECODE_STEP)
+        torch.cuda.synchronize()
+
+    def step(self, mark=None):
+        w, L = self.w, self.L
+        if self.pre is not None:
+            p = self.pre
+            L.prefill(p["q"], p["idx_q"], 0, w.n, p["out"], p["sel"], p["nsel"], mark=mark)
+        for d in self.dec:
+            L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+        if mark and self.dec:
+            mark("decode")
+
+    # -- end to end: host buffers in, host result out -----------------------------------
+    def e2e(self, steps, warmup):
+        w, L, B, n = self.w, self.L, self.w.batch, self.w.n
+        host_in, host_out = [], []
+
+        def pin_like(t):
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h.copy_(t)
+            return h
+
+        if self.pre is not None:
+            for dst in (self.pre["q"], self.pre["idx_q"]):
+                host_in.append((pin_like(dst), dst))
+            host_out.append((pin_like(self.pre["out"]), self.pre["out"]))
+        for c in (L.k_cache, L.v_cache, L.idx_k_cache):
+            for s in range(B):
+                dst = c[s, :n]
+                host_in.append((pin_like(dst), dst))
+        for d in self.dec:
+            for nm in ("q", "k", "v", "idx_q", "idx_k"):
+                host_in.append((pin_like(d[nm]), d[nm]))
+            host_out.append((pin_like(d["out"]), d["out"]))
+        h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
+        d2h = sum(h.numel() * h.element_size() for h, _ in host_out)
+        stream = torch.cuda.current_stream()
+
+        def one():
+            for h, dv in host_in:
+                dv.copy_(h, non_blocking=True)
+            self.step()
+            for h, dv in host_out:
+                h.copy_(dv, non_blocking=True)
+
+        for _ in range(warmup):
+            one()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def run_cuda(args, w, rank, world):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    b = Bench(w, dev)
+    qsa = b.qsa
+    for _ in range(args.warmup):
+        b.step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    bus = getattr(torch.cuda.get_device_properties(dev), "pci_bus_id", None)
+    clocks = ClockSampler(bus)
+    clocks.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    marks = []
+
+    def mark(name):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        marks.append((name, e))
+
+    launches0 = qsa.qsa_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        mark("start")
+        b.step(mark)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = qsa.qsa_launch_count() - launches0
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    stage_ms = {}
+    prev = None
+    for name, e in marks:
+        if name != "start" and prev is not None:
+            stage_ms[name] = stage_ms.get(name, 0.0) + prev.elapsed_time(e) / args.steps
+        prev = e
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    alg = algorithmic(w)
+    pk = peaks()
+    tokens = alg["prefill_tokens"] + alg["decode_tokens"]
+    stages = {}
+    defs = {"compress": ("hbm", alg["compress_bytes"]), "topk": ("tensor", alg["index_flops"]),
+            "attention": ("hbm", alg["attn_gather_bytes"]), "decode": ("hbm", alg["decode_bytes"])}
+    for name, t in stage_ms.items():
+        bound, amount = defs[name]
+        if bound == "hbm":
+            ach = amount / (t * 1e-3) / 1e9
+            peak = pk["hbm_gbs"]
+            unit = "GB/s"
+        else:
+            ach = amount / (t * 1e-3) / 1e12
+            peak = pk["bf16_tflops_sustained"]
+            unit = "TFLOP/s"
+        stages[name] = {"ms": round(t, 4), "bound": bound, "achieved": round(ach, 2), "unit": unit,
+                        "frac": round(ach / peak, 4)}
+    if "attention" in stages:
+        stages["attention"]["tensor_tflops"] = round(alg["attn_flops"] / (stage_ms["attention"] * 1e-3) / 1e12, 2)
+    dom = max(stage_ms, key=stage_ms.get)
+    ds = stages[dom]
+    roofline = {"bound": ds["bound"], "achieved": ds["achieved"],
+                "peak": pk["hbm_gbs"] if ds["bound"] == "hbm" else pk["bf16_tflops_sustained"],
+                "unit": ds["unit"], "frac": ds["frac"], "traffic": traffic_for(dom), "kernel": dom,
+                "peak_source": pk["source"] + (" (sustained bf16)" if ds["bound"] == "tensor" else " (copy)")}
+
+    res = {
+        "metric": METRIC, "value": round(tokens * world / (ms * 1e-3), 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded counter-based N(0,1) bf16 inputs with planted needle blocks",
+        "config": {"workload": w.name, "n": w.n, "batch": w.batch, "decode_steps": w.decode_steps, "r": w.r,
+                   "K": w.K, "k_B": w.k_blocks, "indexer": f"{w.idx_heads}x{w.idx_dim} MQA",
+                   "core": f"GQA {w.q_heads}q/{w.kv_heads}kv d={w.head_dim}",
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (K/V 2.1 GB, q 8.6 GB); decode steps back to back"},
+        "roofline": roofline, "stages": stages,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if alg["prefill_tokens"] and "decode" in stage_ms:
+        pre_ms = sum(stage_ms.get(k, 0.0) for k in ("compress", "topk", "attention"))
+        res["prefill_tokens_per_s"] = round(alg["prefill_tokens"] / (pre_ms * 1e-3), 1)
+        res["decode_tokens_per_s"] = round(alg["decode_tokens"] / (stage_ms["decode"] * 1e-3), 1)
+    if not args.no_e2e:
+        e_ms, h2d, d2h = b.e2e(max(1, min(args.steps, 2)), 1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        res["e2e"] = {"value": round(tokens * world / (e_ms * 1e-3), 2), "unit": "tokens/s",
+                      "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+class OracleTimer:
+    """Times the oracle (single-threaded C) on a bounded sample of the workload and
+    extrapolates one whole step: key pooling timed on `blocks` blocks, prefill
+    rows on `rows` positions stratified over [0, n) (fit t(i) = a + b*floor(i/r)),
+    and `dec` decode positions."""
+
+    def __init__(self, w):
+        import oracle
+
+        self.w = w
+        self.o = oracle.Oracle.for_workload(w)
+        n = w.n
+        self.idx_k = w.host_full("idx_k", 0, n + w.decode_steps)
+        t = time.perf_counter()
+        self.pooled = self.o.compress(self.idx_k, (n + w.decode_steps) // w.r)
+        self.t_compress_full = time.perf_counter() - t
+
+    def _row(self, i):
+        w, o = self.w, self.o
+        iq = w.host_rows("idx_q", 0, [i]).reshape(w.idx_heads, w.idx_dim)
+        qr = w.host_rows("q", 0, [i]).reshape(w.q_heads, w.head_dim)
+        t = time.perf_counter()
+        res = o.row(i, iq, self.pooled, want_scores=False)
+        t_sel = time.perf_counter() - t
+        toks = o.token_set(res["sel"], i)
+        kc = w.host_rows("k", 0, toks)
+        vc = w.host_rows("v", 0, toks)
+        t = time.perf_counter()
+        o.attention(qr, kc, vc, np.arange(toks.size, dtype=np.int64))
+        return t_sel + time.perf_counter() - t
+
+    def sample(self, rows, dec, blocks):
+        w = self.w
+        n, r = w.n, w.r
+        total = 0.0
+        parts = {}
+        if w.prefill:
+            nb = n // r
+            b = min(blocks, nb)
+            t = time.perf_counter()
+            self.o.compress(self.idx_k, b)
+            tc = (time.perf_counter() - t) * nb / max(b, 1)
+            pos = sorted(set([int((k + 0.5) * n / rows) for k in range(rows)] + [n - 1]))
+            ts = np.array([self._row(i) for i in pos])
+            x = np.array([i // r for i in pos], dtype=np.float64)
+            A = np.stack([np.ones_like(x), x], 1)
+            (a, bcoef), *_ = np.linalg.lstsq(A, ts, rcond=None)
+            pairs = float((np.arange(n) // r).sum())
+            tp = n * a + bcoef * pairs
+            resid = float(np.sqrt(np.mean((A @ np.array([a, bcoef]) - ts) ** 2)))
+            parts.update(compress_s=tc, prefill_rows_s=tp, fit={"a_s": a, "b_s": bcoef, "rms_resid_s": resid,
+                                                                 "rows": len(pos)})
+            total += tc + tp
+        if w.decode_steps:
+            ps = [n + int(k * w.decode_steps / dec) for k in range(dec)]
+            td = np.mean([self._row(p) for p in ps])
+            parts["decode_s_per_step"] = td
+            total += td * w.decode_steps
+        return total * w.batch, parts
+
+
+def cpu_baseline(w, rows=64, dec=2, blocks=65536):
+    ot = OracleTimer(w)
+    t, parts = ot.sample(rows, dec, blocks)
+    tokens = (w.n if w.prefill else 0) * w.batch + w.decode_steps * w.batch
+    return {"value": round(tokens / t, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": (f"{parts.get('fit', {}).get('rows', 0)} prefill rows stratified over [0,n) fitted by "
+                       f"t(i)=a+b*floor(i/r) and extrapolated over all n; key pooling timed on {blocks} blocks "
+                       f"and scaled; {dec} decode positions, scaled to {w.decode_steps} steps"),
+            "extrapolated_step_s": round(t, 3), "parts": {k: (round(v, 4) if isinstance(v, float) else v)
+                                                        for k, v in parts.items()}}
+
+
+def run_reference(args, w):
+    ot = OracleTimer(w)
+    times = []
+    for k in range(args.warmup + args.steps):
+        t, parts = ot.sample(rows=6, dec=1, blocks=8192)
+        if k >= args.warmup:
+            times.append(t)
+    t = float(np.mean(times))
+    tokens = (w.n if w.prefill else 0) * w.batch + w.decode_steps * w.batch
+    v = tokens / t
+    return {"metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "impl": "reference",
+            "data": "synthetic: seeded counter-based N(0,1) bf16 inputs with planted needle blocks",
+            "config": {"workload": w.name, "n": w.n, "batch": w.batch, "decode_steps": w.decode_steps,
+                       "r": w.r, "K": w.K},
+            "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "per step: 6 stratified prefill rows (fit t(i)=a+b*floor(i/r)), key "
+                                       "pooling on 8192 blocks, 1 decode position; extrapolated to the step"},
+            "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    res = run_cuda(args, w, rank, world)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

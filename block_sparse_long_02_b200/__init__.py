@@ -3,8 +3,8 @@
 Thin argument marshalling over the C-ABI of ``include/qsa.h``: every function
 below has the C entry point's name, takes torch tensors (device memory) and
 passes their pointers plus the current CUDA stream. All computation happens in
-the library's CUDA kernels; there is no fallback. Importing this module loads
-the library and raises if it has not been built (``python -m
+the library's CUDA kernels; there is no fallback. The library is loaded on the
+first call, which raises if it has not been built (``python -m
 block_sparse_long_02_b200.build``).
 """
 from __future__ import annotations
@@ -19,18 +19,14 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqsa.so")
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_long_02_b200.build`")
-
-_lib = ctypes.CDLL(LIB_PATH)
-
 QSA_OK = 0
 STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "QSA_ERR_WORKSPACE",
                 4: "QSA_ERR_CAPACITY", 5: "QSA_ERR_CUDA", 6: "QSA_ERR_TIMEOUT", 7: "QSA_ERR_DEVICE_CHECK"}
 OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 3
 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
-           "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error"]
+           "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
+           "qsa_launch_count"]
 
 
 class QSAError(RuntimeError):
@@ -88,17 +84,32 @@ _SIGS = {
                         _vp, _vp, _sz, _vp],
     "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
 }
-for _name, _args in _SIGS.items():
-    _f = getattr(_lib, _name)
-    _f.argtypes = _args
-    _f.restype = ctypes.c_int
-_lib.qsa_last_error.restype = ctypes.c_char_p
-_lib.qsa_last_error.argtypes = []
+_lib_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libqsa.so (loaded on first use). Raises if it was not built:
+    there is no other implementation to fall back to."""
+    global _lib_handle
+    if _lib_handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_long_02_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            f = getattr(h, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        h.qsa_last_error.restype = ctypes.c_char_p
+        h.qsa_last_error.argtypes = []
+        h.qsa_launch_count.restype = ctypes.c_uint64
+        h.qsa_launch_count.argtypes = []
+        _lib_handle = h
+    return _lib_handle
 
 
 def _check(status: int) -> None:
     if status != QSA_OK:
-        raise QSAError(status, _lib.qsa_last_error().decode())
+        raise QSAError(status, lib().qsa_last_error().decode())
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -119,7 +130,7 @@ def _stream(stream) -> ctypes.c_void_p:
 
 def qsa_workspace_size(cfg: Config, op: int, batch: int, cap: int, nq: int = 0) -> int:
     out = ctypes.c_size_t(0)
-    _check(_lib.qsa_workspace_size(ctypes.byref(cfg.c()), op, batch, cap, nq, ctypes.byref(out)))
+    _check(lib().qsa_workspace_size(ctypes.byref(cfg.c()), op, batch, cap, nq, ctypes.byref(out)))
     return out.value
 
 
@@ -131,21 +142,21 @@ def workspace(cfg: Config, op: int, batch: int, cap: int, nq: int = 0, device=No
 
 def qsa_compress_keys(cfg: Config, batch: int, idx_k: torch.Tensor, cap: int, rms_w, blk_begin: int,
                       blk_end: int, pooled: torch.Tensor, stream=None) -> None:
-    _check(_lib.qsa_compress_keys(ctypes.byref(cfg.c()), batch, _ptr(idx_k), cap, _ptr(rms_w), blk_begin,
+    _check(lib().qsa_compress_keys(ctypes.byref(cfg.c()), batch, _ptr(idx_k), cap, _ptr(rms_w), blk_begin,
                                   blk_end, _ptr(pooled), _stream(stream)))
 
 
 def qsa_index_scores(cfg: Config, batch: int, idx_q: torch.Tensor, q_begin: int, nq: int,
                      pooled: torch.Tensor, cap: int, scores: torch.Tensor, ld: int, ws: torch.Tensor,
                      stream=None) -> None:
-    _check(_lib.qsa_index_scores(ctypes.byref(cfg.c()), batch, _ptr(idx_q), q_begin, nq, _ptr(pooled), cap,
+    _check(lib().qsa_index_scores(ctypes.byref(cfg.c()), batch, _ptr(idx_q), q_begin, nq, _ptr(pooled), cap,
                                  _ptr(scores), ld, _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def qsa_topk_blocks(cfg: Config, batch: int, idx_q, q_begin: int, nq: int, pooled, cap: int,
                     scores: Optional[torch.Tensor], ld: int, sel: torch.Tensor, nsel: torch.Tensor,
                     ws: Optional[torch.Tensor], stream=None) -> None:
-    _check(_lib.qsa_topk_blocks(ctypes.byref(cfg.c()), batch, _ptr(idx_q), q_begin, nq, _ptr(pooled), cap,
+    _check(lib().qsa_topk_blocks(ctypes.byref(cfg.c()), batch, _ptr(idx_q), q_begin, nq, _ptr(pooled), cap,
                                 _ptr(scores), ld, _ptr(sel), _ptr(nsel), _ptr(ws),
                                 0 if ws is None else ws.numel(), _stream(stream)))
 
@@ -154,7 +165,7 @@ def qsa_sparse_attention(cfg: Config, batch: int, q: torch.Tensor, q_begin: int,
                          k_cache: torch.Tensor, v_cache: torch.Tensor, cap: int, sel: torch.Tensor,
                          nsel: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
                          ws: Optional[torch.Tensor] = None, stream=None) -> None:
-    _check(_lib.qsa_sparse_attention(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache),
+    _check(lib().qsa_sparse_attention(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache),
                                      _ptr(v_cache), cap, _ptr(sel), _ptr(nsel), _ptr(out), _ptr(lse),
                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
 
@@ -162,7 +173,7 @@ def qsa_sparse_attention(cfg: Config, batch: int, q: torch.Tensor, q_begin: int,
 def qsa_decode_step(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, idx_k, k_cache, v_cache,
                     idx_k_cache, pooled, cap: int, rms_w, out, sel_out=None, nsel_out=None,
                     ws: Optional[torch.Tensor] = None, stream=None) -> None:
-    _check(_lib.qsa_decode_step(ctypes.byref(cfg.c()), batch, _ptr(pos), _ptr(q), _ptr(k), _ptr(v),
+    _check(lib().qsa_decode_step(ctypes.byref(cfg.c()), batch, _ptr(pos), _ptr(q), _ptr(k), _ptr(v),
                                 _ptr(idx_q), _ptr(idx_k), _ptr(k_cache), _ptr(v_cache), _ptr(idx_k_cache),
                                 _ptr(pooled), cap, _ptr(rms_w), _ptr(out), _ptr(sel_out), _ptr(nsel_out),
                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
@@ -170,9 +181,14 @@ def qsa_decode_step(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, 
 
 def qsa_workspace_status(ws: torch.Tensor, stream=None) -> int:
     out = ctypes.c_int32(0)
-    _check(_lib.qsa_workspace_status(_ptr(ws), _stream(stream), ctypes.byref(out)))
+    _check(lib().qsa_workspace_status(_ptr(ws), _stream(stream), ctypes.byref(out)))
     return out.value
 
 
 def qsa_last_error() -> str:
-    return _lib.qsa_last_error().decode()
+    return lib().qsa_last_error().decode()
+
+
+def qsa_launch_count() -> int:
+    """Kernel launches issued by libqsa.so so far in this process."""
+    return int(lib().qsa_launch_count())

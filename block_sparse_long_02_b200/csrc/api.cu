@@ -2,6 +2,7 @@
 // workspace layout and stream-ordered launches. No allocation, no sync except
 // in qsa_workspace_status.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -9,6 +10,11 @@
 
 #include "../../include/qsa.h"
 #include "kernels.h"
+
+namespace qsa {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace qsa
 
 namespace {
 
@@ -143,6 +149,8 @@ qsa_status check_ws(void* ws, size_t have, size_t need) {
 extern "C" {
 
 const char* qsa_last_error(void) { return g_err.c_str(); }
+
+uint64_t qsa_launch_count(void) { return qsa::g_launches.load(std::memory_order_relaxed); }
 
 qsa_status qsa_workspace_size(const qsa_config* cfg, int32_t op, int32_t batch, int64_t cap,
                               int64_t nq, size_t* bytes) {

@@ -419,6 +419,7 @@ cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_
                          SMEM);
     const int GH = L.kv_heads < WARPS ? L.kv_heads : WARPS;
     dim3 grid((unsigned)nq, (unsigned)batch, (unsigned)(L.kv_heads / GH));
+    note_launch();
     prefill_attention_kernel<<<grid, WARPS * 32, SMEM, st>>>(
         q, q_begin, nq, kc, vc, cap, sel, nsel, out, lse, L.q_heads, L.kv_heads, L.r, L.kB,
         L.sm_scale * LOG2E);
@@ -440,12 +441,14 @@ cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t
                          SMEM);
     const int S = decode_attention_splits(L);
     const int64_t items = (int64_t)batch * L.kv_heads * S;
+    note_launch();
     decode_attention_kernel<<<(unsigned)((items + WARPS - 1) / WARPS), WARPS * 32, SMEM, st>>>(
         q, pos, kc, vc, cap, sel, nsel, part, batch, L.q_heads, L.kv_heads, L.r, L.kB, S,
         L.sm_scale * LOG2E);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int rows = batch * L.q_heads;
+    note_launch();
     decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(part, rows, S, out);
     return cudaGetLastError();
 }

@@ -58,6 +58,7 @@ cudaError_t launch_compress(const LayerDims& L, int batch, const uint16_t* idx_k
                             uint16_t* pooled, cudaStream_t st) {
     const int64_t nblk = blk_end - blk_begin;
     if (nblk <= 0 || batch <= 0) return cudaSuccess;
+    note_launch();
     compress_kernel<<<grid_for(nblk * batch), 256, 0, st>>>(idx_k, cap, batch, rms_w, blk_begin,
                                                             nblk, L.r, L.rms_eps, L.rope, pooled);
     return cudaGetLastError();
@@ -67,6 +68,7 @@ cudaError_t launch_rotate_queries(const LayerDims& L, int batch, const uint16_t*
                                   int64_t q_begin, int64_t nq, uint16_t* qrot, cudaStream_t st) {
     const int64_t total = (int64_t)batch * nq * kIdxHeads;
     if (total <= 0) return cudaSuccess;
+    note_launch();
     rotate_queries_kernel<<<grid_for(total), 256, 0, st>>>(idx_q, q_begin, nq, total, L.rope,
                                                            qrot);
     return cudaGetLastError();

@@ -111,6 +111,7 @@ cudaError_t launch_decode_prepare(const LayerDims& L, int batch, const int64_t* 
                                   uint16_t* idx_k_cache, uint16_t* pooled, int64_t cap,
                                   const float* rms_w, uint16_t* qrot, int32_t* status,
                                   cudaStream_t st) {
+    note_launch();
     decode_prepare_kernel<<<batch, 128, 0, st>>>(pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache,
                                                  pooled, cap, rms_w, L.kv_heads, L.r, L.rms_eps,
                                                  L.rope, qrot, status);
@@ -128,6 +129,7 @@ cudaError_t launch_decode_scores(const LayerDims& L, int batch, const int64_t* p
     int64_t x = (pcap + 15) / 16;
     const int64_t maxx = std::max<int64_t>(1, (int64_t)sms * 8 / batch);
     x = std::max<int64_t>(1, std::min<int64_t>(x, maxx));
+    note_launch();
     decode_scores_kernel<<<dim3((unsigned)x, (unsigned)batch), 256, 0, st>>>(pos, qrot, pooled, cap,
                                                                             L.r, scores);
     return cudaGetLastError();

@@ -10,6 +10,9 @@
 
 namespace qsa {
 
+// Counts one kernel launch (see qsa_launch_count).
+void note_launch(int n = 1);
+
 struct LayerDims {
     int r, K, kB;
     int rope_dims;

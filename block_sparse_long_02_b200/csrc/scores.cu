@@ -164,6 +164,7 @@ cudaError_t launch_index_scores(const LayerDims& L, int batch, const uint16_t* q
     z = std::max<int64_t>(1, std::min<int64_t>(z, ntiles));
     z = std::min<int64_t>(z, 65535);
     dim3 grid((unsigned)qtiles, (unsigned)batch, (unsigned)z);
+    note_launch();
     index_scores_kernel<<<grid, THREADS, SMEM, st>>>(qrot, nq, q_begin, j0, nrows, pooled,
                                                      cap / L.r, scores, ld, L.r, fill_masked);
     return cudaGetLastError();

@@ -281,6 +281,7 @@ cudaError_t launch_select_rows(const LayerDims& L, int batch, const float* score
     cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     const int64_t rows = (int64_t)batch * nrows;
     const int grid = (int)std::min<int64_t>(rows, (int64_t)sms() * 4);
+    note_launch();
     select_rows_kernel<<<grid, T, smem, st>>>(scores, ld, q_begin, j0, nrows, nq_total, batch, L.r,
                                               L.kB, sel, nsel);
     return cudaGetLastError();
@@ -292,6 +293,7 @@ cudaError_t launch_select_decode(const LayerDims& L, int batch, const float* sco
     if (batch <= 0) return cudaSuccess;
     const int smem = (int)sizeof(SelSmem);
     cudaFuncSetAttribute(select_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    note_launch();
     select_decode_kernel<<<batch, T, smem, st>>>(scores, ld, pos, cap, L.r, L.kB, sel, nsel);
     return cudaGetLastError();
 }

@@ -47,16 +47,23 @@ class QSALayer:
 
     def prefill(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin: int, nq: int,
                 out: torch.Tensor, sel: torch.Tensor, nsel: torch.Tensor,
-                lse: Optional[torch.Tensor] = None, stream=None) -> None:
+                lse: Optional[torch.Tensor] = None, stream=None, mark=None) -> None:
         """Queries [q_begin, q_begin + nq) of every sequence, whose keys and values
-        (positions < q_begin + nq) are already in the caches."""
+        (positions < q_begin + nq) are already in the caches. `mark(name)`, if
+        given, is called after each stage (e.g. to record a CUDA event)."""
         r = self.cfg.r
         self.compress(q_begin // r, (q_begin + nq) // r, stream)
+        if mark:
+            mark("compress")
         ws = self.workspace(OP_TOPK_BLOCKS, nq)
         qsa_topk_blocks(self.cfg, self.batch, idx_q, q_begin, nq, self.pooled, self.cap, None, 0, sel, nsel,
                         ws, stream)
+        if mark:
+            mark("topk")
         qsa_sparse_attention(self.cfg, self.batch, q, q_begin, nq, self.k_cache, self.v_cache, self.cap, sel,
                              nsel, out, lse, None, stream)
+        if mark:
+            mark("attention")
 
     def decode_step(self, pos: torch.Tensor, q, k, v, idx_q, idx_k, out, sel_out=None, nsel_out=None,
                     stream=None) -> None:

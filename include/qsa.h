@@ -187,6 +187,10 @@ qsa_status qsa_workspace_status(void* ws, qsa_stream stream, int32_t* status);
 /* Thread-local message describing the last non-OK status ("" if none). */
 const char* qsa_last_error(void);
 
+/* Number of kernel launches this library has issued in this process (all
+ * threads, all entry points). Used to count device work in benchmarks. */
+uint64_t qsa_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
