@@ -26,7 +26,7 @@ OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 
 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
-           "qsa_launch_count"]
+           "qsa_launch_count", "qsa_decode_step_noalloc"]
 
 
 class QSAError(RuntimeError):
@@ -83,6 +83,8 @@ _SIGS = {
     "qsa_decode_step": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
                         _vp, _vp, _sz, _vp],
     "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
+    "qsa_decode_step_noalloc": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp,
+                                _vp, _vp, _vp],
 }
 _lib_handle = None
 
@@ -177,6 +179,17 @@ def qsa_decode_step(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, 
                                 _ptr(idx_q), _ptr(idx_k), _ptr(k_cache), _ptr(v_cache), _ptr(idx_k_cache),
                                 _ptr(pooled), cap, _ptr(rms_w), _ptr(out), _ptr(sel_out), _ptr(nsel_out),
                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def qsa_decode_step_noalloc(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, idx_k, k_cache,
+                            v_cache, idx_k_cache, pooled, cap: int, rms_w, out, sel_out=None, nsel_out=None,
+                            stream=None) -> None:
+    """qsa_decode_step for callers that cannot allocate: no workspace argument;
+    the library's fixed 16 MiB device scratch is used instead (see qsa.h)."""
+    _check(lib().qsa_decode_step_noalloc(ctypes.byref(cfg.c()), batch, _ptr(pos), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(idx_q), _ptr(idx_k), _ptr(k_cache), _ptr(v_cache),
+                                         _ptr(idx_k_cache), _ptr(pooled), cap, _ptr(rms_w), _ptr(out),
+                                         _ptr(sel_out), _ptr(nsel_out), _stream(stream)))
 
 
 def qsa_workspace_status(ws: torch.Tensor, stream=None) -> int:

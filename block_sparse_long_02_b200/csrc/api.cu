@@ -30,6 +30,20 @@ qsa_status fail(qsa_status st, const char* fmt, ...) {
     return st;
 }
 
+}  // namespace
+
+int qsa::report_error(int status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return status;
+}
+
+namespace {
+
 qsa_status cuda_check(cudaError_t e, const char* what) {
     if (e == cudaSuccess) return QSA_OK;
     return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));

@@ -12,6 +12,8 @@ namespace qsa {
 
 // Counts one kernel launch (see qsa_launch_count).
 void note_launch(int n = 1);
+// Sets the calling thread's qsa_last_error message; returns `status`.
+int report_error(int status, const char* fmt, ...);
 
 struct LayerDims {
     int r, K, kB;

@@ -178,6 +178,41 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
                            const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
                            void* ws, size_t ws_bytes, qsa_stream stream);
 
+/* Bytes of the fixed device scratch array behind qsa_decode_step_noalloc. */
+#define QSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* qsa_decode_step without a workspace. The pages have no counterpart: this is
+ * a property of the library, not of the layer.
+ *
+ * For callers that cannot allocate device memory: serving engines that carve
+ * all device memory into their own pool and forbid allocations outside it,
+ * plugin hosts that pass a stream and tensors but no allocator or workspace,
+ * and latency-critical loops that cannot afford the device-wide
+ * synchronisation cudaMalloc/cudaFree may cause. It allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library routine). Its scratch is one
+ * fixed array of QSA_NOALLOC_SCRATCH_BYTES (16 MiB) in the library's device
+ * memory, which every GPU that loads the library holds until the process exits.
+ *
+ * Arguments and results are those of qsa_decode_step, minus ws/ws_bytes. The
+ * caller still owns and passes every input, output and cache.
+ * Limits and rules:
+ *   - If qsa_workspace_size(QSA_OP_DECODE_STEP, batch, cap) exceeds
+ *     QSA_NOALLOC_SCRATCH_BYTES the call returns QSA_ERR_WORKSPACE and launches
+ *     nothing (e.g. batch 8 x 256K cached tokens fits; batch 64 x 4M does not).
+ *   - The first call on each device does a one-time set-up (it looks up the
+ *     array's device address); make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents:
+ *     calls whose work overlaps on the GPU (other streams, other threads) race
+ *     and corrupt each other's results. Order them on one stream.
+ *   - The device status word is cleared at each call and cannot be read back:
+ *     a position outside [0, cap) is skipped without a report. */
+qsa_status qsa_decode_step_noalloc(const qsa_config* cfg, int32_t batch, const int64_t* pos,
+                                   const qsa_bf16* q, const qsa_bf16* k, const qsa_bf16* v,
+                                   const qsa_bf16* idx_q, const qsa_bf16* idx_k, qsa_bf16* k_cache,
+                                   qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled,
+                                   int64_t cap, const float* rms_w, qsa_bf16* out,
+                                   int32_t* sel_out, int32_t* nsel_out, qsa_stream stream);
+
 /* Device-side status recorded in a workspace by the calls that used it:
  * QSA_OK, or the first error a kernel flagged (QSA_ERR_CAPACITY,
  * QSA_ERR_DEVICE_CHECK, QSA_ERR_TIMEOUT). Synchronises `stream`, copies the
