@@ -97,6 +97,7 @@ qsa_status make_dims(const qsa_config* c, qsa::LayerDims* L) {
 struct TopkWs {
     size_t qrot, scores, total;
     int64_t chunk_rows, ld;
+    bool fused;
 };
 
 int64_t visible_ld(const qsa::LayerDims& L, int64_t q_begin, int64_t nq) {
@@ -114,7 +115,10 @@ TopkWs topk_layout(const qsa::LayerDims& L, int batch, int64_t cap, int64_t nq) 
     w.chunk_rows = rows;
     w.qrot = qsa::kWsHeader;
     w.scores = w.qrot + align_up((size_t)batch * std::max<int64_t>(nq, 1) * qsa::kIdxHeads * qsa::kIdxDim * 2);
-    w.total = w.scores + align_up((size_t)batch * rows * ld * 4);
+    w.fused = qsa::fused_topk_supported(L);
+    // Fused path: the region after the rotated queries holds the tile counter and
+    // candidate buffers; otherwise it holds one row chunk of materialised scores.
+    w.total = w.scores + align_up(w.fused ? qsa::fused_topk_ws_bytes(batch, nq) : (size_t)batch * rows * ld * 4);
     return w;
 }
 
@@ -250,6 +254,10 @@ qsa_status qsa_topk_blocks(const qsa_config* cfg, int32_t batch, const qsa_bf16*
     float* chunk = reinterpret_cast<float*>((char*)ws + w.scores);
     const int64_t vld = visible_ld(L, q_begin, nq);
     TRY(cuda_check(qsa::launch_rotate_queries(L, batch, idx_q, q_begin, nq, qrot, st), "rotate"));
+    if (w.fused)
+        return cuda_check(qsa::launch_fused_topk(L, batch, qrot, nq, q_begin, pooled, cap, sel, nsel,
+                                                 (char*)ws + w.scores, reinterpret_cast<int32_t*>(ws), st),
+                          "fused top-k");
     for (int64_t j0 = 0; j0 < nq; j0 += w.chunk_rows) {
         const int64_t rows = std::min<int64_t>(w.chunk_rows, nq - j0);
         TRY(cuda_check(qsa::launch_index_scores(L, batch, qrot, nq, q_begin, j0, rows, pooled, cap,

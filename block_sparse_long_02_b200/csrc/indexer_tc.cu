@@ -1,0 +1,610 @@
+// Fused prefill indexer: a3'..a5 ("QSA (Qwen Sparse Attention)" concept page,
+// (A) block importance I_ib = sum_h ReLU(<q_i^h, k_b>) under block-causal
+// masking, then top-k_B; "Qwen Sparse Attention" gallery page pseudo-code
+// scores = sum(relu(query_head @ block_key)), top_k(scores, k=512)).
+//
+// The score matrix (1.4e11 entries at 1M tokens) is never materialised. One
+// persistent CTA per SM owns a tile of 128 consecutive queries (512 rotated
+// indexer rows = 128 KB of bf16, resident in shared memory) and sweeps every
+// visible 128-block tile of pooled keys:
+//   warp 0      TMA producer: pooled-key tiles (SWIZZLE_128B) into a 3-stage ring;
+//   warp 1      MMA issuer: tcgen05.mma kind::f16, M = 128 blocks x N = 256
+//               (query, head) columns x K = 128, fp32 accumulators in TMEM; the
+//               512 TMEM columns hold two halves (queries 0-63 / 64-127) that
+//               are double-buffered against the epilogue;
+//   warps 2-9   epilogue: tcgen05.ld of 32 columns per thread-lane (a block
+//               row), ReLU-sum over the 4 heads in registers, block-causal
+//               mask, and a streaming top-k: a score enters the query's
+//               candidate buffer (global, 1024 entries) only if it beats the
+//               query's threshold tau; when a buffer could overflow, one warp
+//               keeps its k_B best entries (radix select over the 32-bit
+//               order-preserving keys, ties to the lower block index) and
+//               raises tau to the k_B-th score. Since blocks arrive in
+//               ascending order, a later block that ties tau loses the tie.
+// At the end of the sweep each query keeps exactly min(k_B, visible) entries,
+// which are sorted ascending and written out.
+//
+// Every wait is bounded (2 s of %globaltimer); on expiry the kernel records
+// QSA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "kernels.h"
+
+namespace qsa {
+namespace {
+
+constexpr int QT = 128;                // queries per CTA tile
+constexpr int BT = 128;                // pooled-key blocks per MMA tile (M)
+constexpr int NHALF = 256;             // TMEM columns per half = 64 queries x 4 heads
+constexpr int STAGES = 3;
+constexpr int CAP = 1024;              // candidate entries per query
+constexpr int KMAX_FUSED = 512;        // largest k_B handled here
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int THREADS = 64 + EPI_THREADS;
+constexpr int Q_BYTES = QT * kIdxHeads * 256;  // 131072
+constexpr int KT_BYTES = BT * 256;             // 32768
+constexpr uint64_t WAIT_NS = 2000000000ull;
+
+struct Ctl {
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t q_full, acc_full[2], acc_empty[2], epi_bar, cta_bar, mma_done;
+    uint32_t tmem_base;
+    int abort;
+    int tile[2];
+    float tau[QT];
+    int cnt[QT];
+    int cvis[QT];
+};
+constexpr int SMEM = Q_BYTES + STAGES * KT_BYTES + (int)sizeof(Ctl) + 1024;
+
+// ------------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint64_t gtime() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t a) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Waits for the phase of parity `parity` to complete. Returns false (and sets
+// the CTA's abort flag) after WAIT_NS, or at once if another warp aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try(a, parity)) return true;
+    const uint64_t t0 = gtime();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try(a, parity)) return true;
+        if ((it & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (gtime() - t0 > WAIT_NS) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t mbar,
+                                            int x, int y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"((uint64_t)map), "r"(mbar), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+
+// UMMA shared-memory descriptor: K-major, SWIZZLE_128B (rows of 128 bytes,
+// 8-row atoms of 1024 bytes).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;             // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024u >> 4) << 32;   // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1u << 46;             // descriptor version
+    d |= (uint64_t)2u << 61;             // SWIZZLE_128B
+    return d;
+}
+// Instruction descriptor: D f32, A/B bf16, both K-major, M = 128, N = 256.
+constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NHALF >> 3) << 17) |
+                           ((uint32_t)(BT >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc) {
+    const uint32_t z = 0;
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(IDESC), "r"(acc), "r"(z), "r"(z), "r"(z), "r"(z));
+}
+__device__ __forceinline__ void umma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+          "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+          "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(addr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// ------------------------------------------------------- candidate compaction
+// Keeps the k best of the n (k <= n <= CAP) entries of one query's candidate
+// buffer, ranked by (score desc, block asc), writing them to positions [0, k)
+// (in no particular order). Returns the smallest kept score. One warp.
+__device__ float warp_keep_best(float* sc, int32_t* id, int n, int k, int lane) {
+    uint32_t key[32];
+    uint32_t ix[32];
+    uint32_t valid = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int e = j * 32 + lane;
+        if (e < n) {
+            key[j] = float_key(sc[e]);
+            ix[j] = (uint32_t)id[e];
+            valid |= 1u << j;
+        } else {
+            key[j] = 0u;
+            ix[j] = 0xFFFFFFFFu;
+        }
+    }
+    // Radix select (one bit at a time) of the k-th largest key; stops as soon as
+    // every entry matching the prefix is needed.
+    uint32_t prefix = 0, mask = 0;
+    int need = k, rem = n;
+    for (int bit = 31; bit >= 0 && rem != need; --bit) {
+        const uint32_t m2 = mask | (1u << bit), c2 = prefix | (1u << bit);
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) c += (((valid >> j) & 1u) && ((key[j] & m2) == c2)) ? 1 : 0;
+        c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+        if (c >= need) {
+            prefix = c2;
+            rem = c;
+        } else {
+            need -= c;
+            rem -= c;
+        }
+        mask = m2;
+    }
+    // Ties at the threshold (only when the keys are exactly equal): the `need`
+    // lowest block indices among them.
+    uint32_t iprefix = 0xFFFFFFFFu, imask = 0;
+    if (rem != need) {
+        iprefix = 0;
+        int ineed = need, irem = rem;
+        for (int bit = 31; bit >= 0 && irem != ineed; --bit) {
+            const uint32_t m2 = imask | (1u << bit);
+            int c0 = 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                c0 += (((valid >> j) & 1u) && ((key[j] & mask) == prefix) && ((ix[j] & m2) == iprefix)) ? 1 : 0;
+            c0 = (int)__reduce_add_sync(0xffffffffu, (unsigned)c0);
+            if (c0 >= ineed) {
+                irem = c0;
+            } else {
+                ineed -= c0;
+                irem -= c0;
+                iprefix |= 1u << bit;
+            }
+            imask = m2;
+        }
+    }
+    uint32_t keep = 0, minkey = 0xFFFFFFFFu;
+    int kc = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const uint32_t km = key[j] & mask;
+        const bool tie_ok = (iprefix == 0xFFFFFFFFu && imask == 0) || ((ix[j] & imask) <= iprefix);
+        if (((valid >> j) & 1u) && (km > prefix || (km == prefix && tie_ok))) {
+            keep |= 1u << j;
+            ++kc;
+            minkey = min(minkey, key[j]);
+        }
+    }
+    // Exclusive prefix of the per-lane counts.
+    int incl = kc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int pos = incl - kc;
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if ((keep >> j) & 1u) {
+            sc[pos] = key_to_float(key[j]);
+            id[pos] = (int32_t)ix[j];
+            ++pos;
+        }
+    }
+    __syncwarp();
+    return key_to_float(__reduce_min_sync(0xffffffffu, minkey));
+}
+
+// Ascending bitonic sort of P (power of two, <= 512) ints in shared memory; one warp.
+__device__ void warp_sort(int32_t* a, int P, int lane) {
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = lane; i < P; i += 32) {
+                const int x = i ^ j;
+                if (x > i) {
+                    const int32_t u = a[i], w = a[x];
+                    if ((u > w) == ((i & k) == 0)) {
+                        a[i] = w;
+                        a[x] = u;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+// --------------------------------------------------------------------- kernel
+__global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int batch,
+    int64_t nq, int64_t q_begin, int64_t pcap, int r, int kB, int* __restrict__ tile_counter,
+    float* __restrict__ cand_score, int32_t* __restrict__ cand_idx, int32_t* __restrict__ sel,
+    int32_t* __restrict__ nsel, int32_t* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    uint8_t* base = smem_raw + (base_s - raw_s);
+    const uint32_t sQ = base_s;
+    const uint32_t sK = base_s + Q_BYTES;
+    Ctl& ctl = *reinterpret_cast<Ctl*>(base + Q_BYTES + STAGES * KT_BYTES);
+    volatile int* abort_flag = &ctl.abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t nqt = (nq + QT - 1) / QT;
+    const int64_t total_tiles = nqt * batch;
+
+    auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar(ctl.full[s]), 1);
+            mbar_init(bar(ctl.empty[s]), 1);
+        }
+        mbar_init(bar(ctl.q_full), 1);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(bar(ctl.acc_full[h]), 1);
+            mbar_init(bar(ctl.acc_empty[h]), EPI_THREADS);
+        }
+        mbar_init(bar(ctl.epi_bar), EPI_THREADS);
+        mbar_init(bar(ctl.cta_bar), THREADS);
+        mbar_init(bar(ctl.mma_done), 1);
+        ctl.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&ctl.tmem_base)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl.tmem_base;
+
+    // Per-role pipeline state (continues across query tiles).
+    uint32_t kring = 0;       // pooled-key tiles produced / consumed
+    uint32_t acc_iter = 0;    // MMA tiles (both halves) issued / drained
+    uint32_t q_iter = 0;      // query tiles with a sweep
+    uint32_t epi_phase = 0, cta_phase = 0;
+    uint32_t produced_last[STAGES] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+    const uint64_t pol_k = policy_evict_last();
+    const uint64_t pol_q = policy_evict_first();
+
+    for (int iter = 0;; ++iter) {
+        // ---- CTA-wide: next query tile (longest first) ----
+        if (tid == 0) ctl.tile[iter & 1] = atomicAdd(tile_counter, 1);
+        mbar_arrive(bar(ctl.cta_bar));
+        // Warp-uniform outcome: warp collectives follow.
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(ctl.cta_bar), cta_phase, abort_flag))) break;
+        cta_phase ^= 1;
+        const int64_t u = ctl.tile[iter & 1];
+        if (u >= total_tiles || *abort_flag) break;
+        const int s = (int)(u % batch);
+        const int64_t qt = nqt - 1 - u / batch;
+        const int64_t j0 = qt * QT;
+        const int nrows = (int)std::min<int64_t>(QT, nq - j0);
+        const int64_t c_min = (q_begin + j0) / r;
+        const int64_t c_max = (q_begin + j0 + nrows - 1) / r;
+        const int ntiles = c_max > kB ? (int)((c_max + BT - 1) / BT) : 0;
+
+        if (warp == 0) {
+            // ------------------------------------------------ TMA producer
+            if (lane == 0 && ntiles > 0) {
+                const uint32_t qb = bar(ctl.q_full);
+                mbar_expect_tx(qb, Q_BYTES);
+                const int qrow = (int)(((int64_t)s * nq + j0) * kIdxHeads);
+                for (int kh = 0; kh < 2; ++kh)
+                    for (int rh = 0; rh < 2; ++rh)
+                        tma_load_2d(sQ + kh * (Q_BYTES / 2) + rh * (Q_BYTES / 4), &tm_q, qb, kh * 64,
+                                    qrow + rh * 256, pol_q);
+                const int krow0 = (int)((int64_t)s * pcap);
+                for (int t = 0; t < ntiles; ++t, ++kring) {
+                    const int stg = (int)(kring % STAGES);
+                    const uint32_t round = kring / STAGES;
+                    if (!mbar_wait(bar(ctl.empty[stg]), (round & 1u) ^ 1u, abort_flag)) break;
+                    const uint32_t fb = bar(ctl.full[stg]);
+                    mbar_expect_tx(fb, KT_BYTES);
+                    for (int kh = 0; kh < 2; ++kh)
+                        tma_load_2d(sK + stg * KT_BYTES + kh * (KT_BYTES / 2), &tm_k, fb, kh * 64,
+                                    krow0 + t * BT, pol_k);
+                    produced_last[stg] = round;
+                }
+            }
+        } else if (warp == 1) {
+            // ------------------------------------------------ MMA issuer
+            if (lane == 0 && ntiles > 0) {
+                bool ok = mbar_wait(bar(ctl.q_full), q_iter & 1u, abort_flag);
+                for (int t = 0; ok && t < ntiles; ++t, ++kring, ++acc_iter) {
+                    const int stg = (int)(kring % STAGES);
+                    if (!(ok = mbar_wait(bar(ctl.full[stg]), (kring / STAGES) & 1u, abort_flag))) break;
+                    tc_fence_after();
+                    for (int h = 0; h < 2; ++h) {
+                        if (!(ok = mbar_wait(bar(ctl.acc_empty[h]), (acc_iter & 1u) ^ 1u, abort_flag))) break;
+                        tc_fence_after();
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t koff = (kk >> 2) * (KT_BYTES / 2) + (kk & 3) * 32;
+                            const uint32_t qoff = (kk >> 2) * (Q_BYTES / 2) + h * (NHALF * 128) + (kk & 3) * 32;
+                            umma_bf16(tmem + h * NHALF, desc_sw128(sK + stg * KT_BYTES + koff),
+                                      desc_sw128(sQ + qoff), kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(bar(ctl.acc_full[h]));
+                    }
+                    if (!ok) break;
+                    umma_commit(bar(ctl.empty[stg]));
+                }
+            }
+            if (ntiles > 0) ++q_iter;
+        } else {
+            // ------------------------------------------------ epilogue
+            const int et = tid - 64, ew = et >> 5;
+            const int qd = warp & 3;          // TMEM lane quadrant of this warp
+            const int ch = ew >> 2;           // which 128-column half of a TMEM half
+            for (int q = et; q < QT; q += EPI_THREADS) {
+                ctl.tau[q] = q < nrows ? -INFINITY : INFINITY;  // rows past nq never enter
+                ctl.cnt[q] = 0;
+                ctl.cvis[q] = q < nrows ? (int)((q_begin + j0 + q) / r) : 0;
+            }
+            mbar_arrive(bar(ctl.epi_bar));
+            bool ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.epi_bar), epi_phase, abort_flag));
+            epi_phase ^= 1;
+            const size_t slot0 = (size_t)blockIdx.x * QT;
+            for (int t = 0; ok && t < ntiles; ++t, ++acc_iter) {
+                const int b = t * BT + qd * 32 + lane;
+                const bool masked = (int64_t)(t + 1) * BT > c_min;
+                for (int h = 0; h < 2; ++h) {
+                    if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.acc_full[h]), acc_iter & 1u, abort_flag))))
+                        break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int g = 0; g < 4; ++g) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + ((uint32_t)(qd * 32) << 16) + h * NHALF + ch * 128 + g * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int qq = 0; qq < 8; ++qq) {
+                            const int q = h * 64 + ch * 32 + g * 8 + qq;
+                            const float sc = fmaxf(__uint_as_float(v[4 * qq]), 0.f) +
+                                             fmaxf(__uint_as_float(v[4 * qq + 1]), 0.f) +
+                                             fmaxf(__uint_as_float(v[4 * qq + 2]), 0.f) +
+                                             fmaxf(__uint_as_float(v[4 * qq + 3]), 0.f);
+                            const bool take = sc > ctl.tau[q] && (!masked || b < ctl.cvis[q]);
+                            const uint32_t bal = __ballot_sync(0xffffffffu, take);
+                            if (bal) {
+                                const int leader = __ffs(bal) - 1;
+                                int pos = 0;
+                                if (lane == leader) pos = atomicAdd(&ctl.cnt[q], __popc(bal));
+                                pos = __shfl_sync(0xffffffffu, pos, leader) + __popc(bal & ((1u << lane) - 1u));
+                                if (take) {
+                                    const size_t e = (slot0 + q) * CAP + pos;
+                                    cand_score[e] = sc;
+                                    cand_idx[e] = b;
+                                }
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(bar(ctl.acc_empty[h]));
+                }
+                if (!ok) break;
+                // All appends of tile t are in; shrink the buffers that could overflow.
+                mbar_arrive(bar(ctl.epi_bar));
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.epi_bar), epi_phase, abort_flag)))) break;
+                epi_phase ^= 1;
+                for (int q = ew; q < QT; q += EPI_WARPS) {
+                    const int n = ctl.cnt[q];
+                    if (n > CAP - BT) {
+                        const float tau = warp_keep_best(cand_score + (slot0 + q) * CAP,
+                                                         cand_idx + (slot0 + q) * CAP, n, kB, lane);
+                        if (lane == 0) {
+                            ctl.tau[q] = tau;
+                            ctl.cnt[q] = kB;
+                        }
+                    }
+                }
+                __syncwarp();
+                mbar_arrive(bar(ctl.epi_bar));
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.epi_bar), epi_phase, abort_flag)))) break;
+                epi_phase ^= 1;
+            }
+            // Final selection and ascending output (the pooled-key ring is idle now:
+            // use it as sort scratch, 2 KB per warp).
+            if (ok) {
+                int32_t* scratch = reinterpret_cast<int32_t*>(base + Q_BYTES) + ew * KMAX_FUSED;
+                for (int q = ew; q < nrows; q += EPI_WARPS) {
+                    const int cq = ctl.cvis[q];
+                    const int kq = cq < kB ? cq : kB;
+                    const size_t orow = (size_t)s * nq + j0 + q;
+                    int32_t* out = sel + orow * kB;
+                    if (ntiles == 0) {
+                        for (int k2 = lane; k2 < kB; k2 += 32) out[k2] = k2 < kq ? k2 : -1;
+                        if (lane == 0) nsel[orow] = kq;
+                        continue;
+                    }
+                    const int n = ctl.cnt[q];
+                    float* qs = cand_score + (slot0 + q) * CAP;
+                    int32_t* qi = cand_idx + (slot0 + q) * CAP;
+                    if (n > kq) warp_keep_best(qs, qi, n, kq, lane);
+                    const int m = n < kq ? n : kq;
+                    if (m != kq && lane == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
+                    int P = 1;
+                    while (P < m) P <<= 1;
+                    for (int k2 = lane; k2 < P; k2 += 32) scratch[k2] = k2 < m ? qi[k2] : 0x7fffffff;
+                    __syncwarp();
+                    warp_sort(scratch, P, lane);
+                    for (int k2 = lane; k2 < kB; k2 += 32) out[k2] = k2 < m ? scratch[k2] : -1;
+                    if (lane == 0) nsel[orow] = m;
+                    __syncwarp();
+                }
+            }
+        }
+        if (*abort_flag) break;
+    }
+
+    // ---- shutdown: drain what this CTA started, then free TMEM ----
+    if (!*abort_flag && warp == 0 && lane == 0) {
+        // The MMA warp's last commits release the ring stages; let them land
+        // before the CTA's shared memory goes away.
+        for (int stg = 0; stg < STAGES; ++stg)
+            if (produced_last[stg] != 0xFFFFFFFFu)
+                mbar_wait(smem_u32(&ctl.empty[stg]), produced_last[stg] & 1u, abort_flag);
+    }
+    if (*abort_flag) {
+        if (tid == 0) flag_status(status, 6 /* QSA_ERR_TIMEOUT */);
+        if (warp == 0 && lane == 0) {
+            // Outstanding TMA copies complete on their stage barriers.
+            volatile int no_abort = 0;
+            for (int stg = 0; stg < STAGES; ++stg)
+                if (produced_last[stg] != 0xFFFFFFFFu)
+                    mbar_wait(smem_u32(&ctl.full[stg]), produced_last[stg] & 1u, &no_abort);
+        }
+        if (warp == 1 && lane == 0) {
+            volatile int no_abort = 0;
+            umma_commit(smem_u32(&ctl.mma_done));
+            mbar_wait(smem_u32(&ctl.mma_done), 0, &no_abort);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2D bf16 map over `rows` rows of 128 elements, box = 64 elements x box_rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {256};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+}  // namespace
+
+bool fused_topk_supported(const LayerDims& L) { return L.kB <= KMAX_FUSED; }
+
+size_t fused_topk_ws_bytes(int /*batch*/, int64_t /*nq*/) {
+    // tile counter (256 B) + candidate buffers of one CTA per SM.
+    return 256 + (size_t)sm_count() * QT * CAP * (sizeof(float) + sizeof(int32_t));
+}
+
+cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qrot, int64_t nq,
+                              int64_t q_begin, const uint16_t* pooled, int64_t cap, int32_t* sel,
+                              int32_t* nsel, void* ws, int32_t* status, cudaStream_t st) {
+    if (nq <= 0 || batch <= 0) return cudaSuccess;
+    const int64_t pcap = cap / L.r;
+    CUtensorMap tm_q, tm_k;
+    if (!make_map(&tm_q, qrot, (uint64_t)batch * nq * kIdxHeads, 256) ||
+        !make_map(&tm_k, pooled, (uint64_t)batch * std::max<int64_t>(pcap, 1), BT))
+        return cudaErrorInvalidValue;
+    const int grid_max = sm_count();
+    const int64_t tiles = ((nq + QT - 1) / QT) * batch;
+    const int grid = (int)std::min<int64_t>(grid_max, tiles);
+    int* counter = reinterpret_cast<int*>(ws);
+    float* cand_score = reinterpret_cast<float*>((char*)ws + 256);
+    int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_score + (size_t)grid_max * QT * CAP);
+    cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    cudaFuncSetAttribute(fused_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    note_launch();
+    fused_topk_kernel<<<grid, THREADS, SMEM, st>>>(tm_q, tm_k, batch, nq, q_begin, pcap, L.r, L.kB, counter,
+                                                   cand_score, cand_idx, sel, nsel, status);
+    return cudaGetLastError();
+}
+
+}  // namespace qsa

@@ -39,6 +39,13 @@ cudaError_t launch_index_scores(const LayerDims& L, int batch, const uint16_t* q
                                 int64_t cap, float* scores, int64_t ld, bool fill_masked,
                                 cudaStream_t st);
 
+// indexer_tc.cu: fused tcgen05 score + streaming top-k (prefill), k_B <= 512.
+bool fused_topk_supported(const LayerDims& L);
+size_t fused_topk_ws_bytes(int batch, int64_t nq);
+cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qrot, int64_t nq,
+                              int64_t q_begin, const uint16_t* pooled, int64_t cap, int32_t* sel,
+                              int32_t* nsel, void* ws, int32_t* status, cudaStream_t st);
+
 // topk.cu: row selection. Row (s, j) has position i = q_begin + j0 + j and
 // floor(i/r) visible entries starting at scores + ((s*nrows + j) * ld).
 cudaError_t launch_select_rows(const LayerDims& L, int batch, const float* scores, int64_t ld,

@@ -357,3 +357,73 @@ def test_decode_short_context_and_capacity_flag(qsa):
     ws = L.workspace(qsa.OP_DECODE_STEP)
     assert qsa.qsa_workspace_status(ws) == 4
     assert qsa.qsa_workspace_status(ws) == 0
+
+
+# ----------------------------------------------------------------------------- fused top-k specifics
+@pytest.mark.parametrize("n,K", [(8192, 128), (8192, 2048), (6001, 2048)])
+def test_fused_topk_with_buffer_compaction(qsa, n, K):
+    """More than 896 visible blocks per query: candidate buffers are compacted
+    many times during the sweep (k_B = 32 and 512)."""
+    w = synth.Workload(name="t", n=n, K=K, q_heads=8, kv_heads=2, base_seed=0xB0 + n + K, n_needles_prefill=8)
+    cfg, res = run_prefill(qsa, w, lse=False)
+    rng = np.random.default_rng(n + K)
+    rows = sorted(set(rng.integers(0, n, 40).tolist() + list(range(n - 10, n)) + [p for _, p in w.needles(0)]
+                      + [4 * 513, 4 * 513 + 3, 4 * 897, 4 * 1024 + 1]))
+    check_rows(w, cfg, res, [i for i in rows if i < n], attention=False)
+    for b, p in w.needles(0):
+        assert b in set(res["sel"][0, p, : res["nsel"][0, p]].tolist()), (b, p)
+
+
+def test_fused_topk_exact_ties(qsa):
+    """rope_dims = 0 and a periodic key pattern make many pooled keys identical:
+    exactly equal scores must resolve to the lower block index, as in the oracle."""
+    n, period = 6000, 37
+    w = synth.Workload(name="t", n=n, K=256, rope_dims=0, q_heads=8, kv_heads=2, base_seed=0xB7)
+    cfg, L = _layer(qsa, w, n)
+    _fill_caches(w, L, n)
+    base_rows = L.idx_k_cache[:, : 4 * period].clone()
+    reps = -(-n // (4 * period))
+    L.idx_k_cache[:, :n] = base_rows.repeat(1, reps, 1)[:, :n]
+    iq = dev_full(w, "idx_q", n)
+    nq = n
+    sel = torch.empty(1, nq, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(1, nq, dtype=torch.int32, device="cuda")
+    L.compress(0, n // 4)
+    ws = L.workspace(qsa.OP_TOPK_BLOCKS, nq)
+    qsa.qsa_topk_blocks(cfg, 1, iq, 0, nq, L.pooled, n, None, 0, sel, nsel, ws)
+    torch.cuda.synchronize()
+    o = _oracle(w, cfg)
+    idx_k = bits(L.idx_k_cache)[0]
+    pooled = o.compress(idx_k, n // 4)
+    assert np.array_equal(pooled, bits(L.pooled)[0])
+    idx_q = w.host_full("idx_q", 0).reshape(n, 4, 128)
+    g_sel, g_n = sel.cpu().numpy()[0], nsel.cpu().numpy()[0]
+    for i in [300, 1999, 4000, 5555, 5999]:
+        ref = o.row(i, idx_q[i], pooled)
+        # Scores are bit-identical between equal blocks on both sides, so the set
+        # must match exactly (near-ties with other blocks are still tolerated).
+        tol = score_tol(o.rotate_query(idx_q[i], i), pooled, ref["scores"])
+        check_selection(g_sel[i], g_n[i], ref["scores"], tol, o.k_blocks, f"row {i}")
+        got = set(g_sel[i, : g_n[i]].tolist())
+        for b in got:  # every selected block's earlier twins with the same score are selected too
+            for b2 in range(b % period, b, period):
+                if ref["scores"][b2] == ref["scores"][b]:
+                    assert b2 in got, (i, b, b2)
+
+
+def test_fused_topk_all_zero_scores(qsa):
+    """Zero indexer queries make every score 0: the k_B lowest blocks win."""
+    n = 5000
+    w = synth.Workload(name="t", n=n, K=512, q_heads=8, kv_heads=2, base_seed=0xB8)
+    cfg, L = _layer(qsa, w, n)
+    _fill_caches(w, L, n)
+    L.compress(0, n // 4)
+    iq = torch.zeros(1, n, 4, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(1, n, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(1, n, dtype=torch.int32, device="cuda")
+    qsa.qsa_topk_blocks(cfg, 1, iq, 0, n, L.pooled, n, None, 0, sel, nsel, L.workspace(qsa.OP_TOPK_BLOCKS, n))
+    torch.cuda.synchronize()
+    g, gn = sel.cpu().numpy()[0], nsel.cpu().numpy()[0]
+    for i in range(0, n, 97):
+        m = min(128, i // 4)
+        assert gn[i] == m and np.array_equal(g[i, :m], np.arange(m)), i
