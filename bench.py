@@ -170,25 +170,30 @@ def traffic_for(stage: str):
 
 # ----------------------------------------------------------------------------- CUDA arm
 class Bench:
-    def __init__(self, w, device):
+    def __init__(self, w, device, stage="all"):
         import block_sparse_long_02_b200 as qsa
         from block_sparse_long_02_b200.layer import QSALayer
 
         self.qsa, self.w, self.dev = qsa, w, device
+        self.stage = stage
         cfg = qsa.Config.of(w)
         self.cfg = cfg
         B, n, S = w.batch, w.n, w.decode_steps
         cap = -(-(n + S) // w.r) * w.r
-        self.L = L = QSALayer(cfg, B, cap, device=device)
+        # stage "topk" (profiling): only what key pooling and the indexer need.
+        kv_cap = 1 if stage == "topk" else cap
+        self.L = L = QSALayer(cfg, B, cap, device=device, kv_cap=kv_cap)
         bf = torch.bfloat16
-        w.device_fill("k", L.k_cache.view(B, cap, -1), rows=(0, n))
-        w.device_fill("v", L.v_cache.view(B, cap, -1), rows=(0, n))
+        if stage != "topk":
+            w.device_fill("k", L.k_cache.view(B, cap, -1), rows=(0, n))
+            w.device_fill("v", L.v_cache.view(B, cap, -1), rows=(0, n))
         w.device_fill("idx_k", L.idx_k_cache, rows=(0, n))
         self.pre = None
         if w.prefill:
-            q = torch.empty(B, n, cfg.q_heads, cfg.head_dim, dtype=bf, device=device)
+            q = torch.empty(B, n if stage != "topk" else 1, cfg.q_heads, cfg.head_dim, dtype=bf, device=device)
             iq = torch.empty(B, n, cfg.idx_heads, cfg.idx_dim, dtype=bf, device=device)
-            w.device_fill("q", q.view(B, n, -1), rows=(0, n))
+            if stage != "topk":
+                w.device_fill("q", q.view(B, n, -1), rows=(0, n))
             w.device_fill("idx_q", iq.view(B, n, -1), rows=(0, n))
             self.pre = {"q": q, "idx_q": iq,
                         "out": torch.empty_like(q),
@@ -226,6 +231,18 @@ class Bench:
 
     def step(self, mark=None):
         w, L = self.w, self.L
+        if self.stage == "topk":
+            from block_sparse_long_02_b200 import OP_TOPK_BLOCKS, qsa_topk_blocks
+
+            p = self.pre
+            L.compress(0, w.n // w.r)
+            if mark:
+                mark("compress")
+            qsa_topk_blocks(self.cfg, w.batch, p["idx_q"], 0, w.n, L.pooled, L.cap, None, 0, p["sel"], p["nsel"],
+                            L.workspace(OP_TOPK_BLOCKS, w.n))
+            if mark:
+                mark("topk")
+            return
         if self.pre is not None:
             p = self.pre
             L.prefill(p["q"], p["idx_q"], 0, w.n, p["out"], p["sel"], p["nsel"], mark=mark)
@@ -281,7 +298,7 @@ class Bench:
 
 def run_cuda(args, w, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
-    b = Bench(w, dev)
+    b = Bench(w, dev, stage=args.stage)
     qsa = b.qsa
     for _ in range(args.warmup):
         b.step()
@@ -487,8 +504,19 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage", choices=["all", "topk"], default="all",
+                    help="topk: time only key pooling + the fused indexer (for profiling)")
+    ap.add_argument("--n", type=int, default=None, help="override the workload's sequence length")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.n is not None:
+        import dataclasses
+
+        w = dataclasses.replace(w, n=args.n, name=f"{w.name}@n={args.n}",
+                                n_needles_prefill=min(w.n_needles_prefill, args.n // 4096))
+    if args.stage == "topk":
+        args.no_e2e = True
+        args.no_cpu_baseline = True
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

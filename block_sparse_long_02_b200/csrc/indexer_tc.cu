@@ -24,7 +24,7 @@
 // At the end of the sweep each query keeps exactly min(k_B, visible) entries,
 // which are sorted ascending and written out.
 //
-// Every wait is bounded (2 s of %globaltimer); on expiry the kernel records
+// Every wait is bounded (10 s of %globaltimer); on expiry the kernel records
 // QSA_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -40,25 +40,28 @@ namespace {
 constexpr int QT = 128;                // queries per CTA tile
 constexpr int BT = 128;                // pooled-key blocks per MMA tile (M)
 constexpr int NHALF = 256;             // TMEM columns per half = 64 queries x 4 heads
-constexpr int STAGES = 3;
+constexpr int STAGES = 2;
 constexpr int CAP = 1024;              // candidate entries per query
+constexpr int NSEG = 4;                // one segment per TMEM lane quadrant (epilogue warp)
+constexpr int SEG = CAP / NSEG;        // entries per segment
 constexpr int KMAX_FUSED = 512;        // largest k_B handled here
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
 constexpr int THREADS = 64 + EPI_THREADS;
 constexpr int Q_BYTES = QT * kIdxHeads * 256;  // 131072
 constexpr int KT_BYTES = BT * 256;             // 32768
-constexpr uint64_t WAIT_NS = 2000000000ull;
+constexpr uint64_t WAIT_NS = 10000000000ull;  // 10 s
 
 struct Ctl {
     uint64_t full[STAGES], empty[STAGES];
-    uint64_t q_full, acc_full[2], acc_empty[2], epi_bar, cta_bar, mma_done;
+    uint64_t q_full, acc_full[2], acc_empty[2], cta_bar, mma_done;
     uint32_t tmem_base;
     int abort;
     int tile[2];
     float tau[QT];
-    int cnt[QT];
+    int seg[QT][NSEG];  // entries in each segment of a query's candidate buffer
     int cvis[QT];
+    uint32_t hist[EPI_WARPS][256];  // per-warp radix histogram of the compaction
 };
 constexpr int SMEM = Q_BYTES + STAGES * KT_BYTES + (int)sizeof(Ctl) + 1024;
 
@@ -102,6 +105,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile 
             }
         }
     }
+}
+
+// Barrier over the 256 epilogue threads (named barrier 1) that also ANDs a
+// predicate across them, so a timeout seen by any warp ends all of them alike.
+__device__ __forceinline__ bool epi_sync_and(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 256, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ uint64_t policy_evict_last() {
@@ -151,7 +167,7 @@ __device__ __forceinline__ void umma_commit(uint32_t mbar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&v)[32]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t* v) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
         "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -169,46 +185,99 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 }
 
 // ------------------------------------------------------- candidate compaction
-// Keeps the k best of the n (k <= n <= CAP) entries of one query's candidate
-// buffer, ranked by (score desc, block asc), writing them to positions [0, k)
-// (in no particular order). Returns the smallest kept score. One warp.
-__device__ float warp_keep_best(float* sc, int32_t* id, int n, int k, int lane) {
+// Keeps the k best of the n = sum(segn) (k <= n <= CAP) entries (score bits,
+// block) of one query's segmented candidate buffer, ranked by (score desc,
+// block asc). The kept entries are either written back spread over the
+// segments (ceil(k/4) per segment, in no particular order) or, if out_idx is
+// given, their block indices are written to out_idx[0, k). Returns the
+// order-preserving key of the smallest kept score. One warp; `hist` is its
+// 256-bin scratch.
+//
+// Radix select over the 32-bit keys with 8-bit digits, starting at the highest
+// bit where the buffer's keys differ (all keys above it are equal); each digit
+// level is one shared-memory histogram pass over the entries still tied with
+// the threshold prefix. It stops as soon as every entry matching the prefix is
+// needed; exact ties beyond that go to the lowest block indices.
+__device__ uint32_t warp_keep_best(uint2* qbuf, const int* segn, int k, int lane, uint32_t* hist,
+                                   int32_t* out_idx) {
     uint32_t key[32];
     uint32_t ix[32];
-    uint32_t valid = 0;
+    uint32_t valid = 0, kmin = 0xFFFFFFFFu, kmax = 0u;
+    int n = 0;
+#pragma unroll
+    for (int sg = 0; sg < NSEG; ++sg) n += segn[sg];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-        const int e = j * 32 + lane;
-        if (e < n) {
-            key[j] = float_key(sc[e]);
-            ix[j] = (uint32_t)id[e];
+        // Register slot j of this lane: segment j / 8, entry ((j % 8) * 32 + lane).
+        const int e = ((j & 7) << 5) | lane;
+        if (e < segn[j >> 3]) {
+            const uint2 v = qbuf[(j >> 3) * SEG + e];
+            key[j] = float_key(__uint_as_float(v.x));
+            ix[j] = v.y;
             valid |= 1u << j;
+            kmin = min(kmin, key[j]);
+            kmax = max(kmax, key[j]);
         } else {
             key[j] = 0u;
             ix[j] = 0xFFFFFFFFu;
         }
     }
-    // Radix select (one bit at a time) of the k-th largest key; stops as soon as
-    // every entry matching the prefix is needed.
-    uint32_t prefix = 0, mask = 0;
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const uint32_t diff = kmin ^ kmax;
+    int hi = diff ? 31 - __clz(diff) : -1;  // highest bit where keys differ
+    uint32_t mask = hi >= 0 ? ~((2u << hi) - 1u) : 0xFFFFFFFFu;
+    uint32_t prefix = kmin & mask;
     int need = k, rem = n;
-    for (int bit = 31; bit >= 0 && rem != need; --bit) {
-        const uint32_t m2 = mask | (1u << bit), c2 = prefix | (1u << bit);
-        int c = 0;
+    while (rem != need && hi >= 0) {
+        const int lo = hi >= 7 ? hi - 7 : 0;
+        const uint32_t dmask = (1u << (hi - lo + 1)) - 1u;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) c += (((valid >> j) & 1u) && ((key[j] & m2) == c2)) ? 1 : 0;
-        c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
-        if (c >= need) {
-            prefix = c2;
-            rem = c;
-        } else {
-            need -= c;
-            rem -= c;
+        for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0u;
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (((valid >> j) & 1u) && (key[j] & mask) == prefix) atomicAdd(&hist[(key[j] >> lo) & dmask], 1u);
+        __syncwarp();
+        uint32_t h[8], sum = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            h[t] = hist[lane * 8 + t];
+            sum += h[t];
         }
-        mask = m2;
+        uint32_t suf = sum;  // inclusive suffix sum over lanes (bins from the top)
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += v;
+        }
+        const uint32_t above = suf - sum;
+        const bool mine = above < (uint32_t)need && (uint32_t)need <= suf;
+        const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+        int digit = 0, acc_above = 0, dcount = 0;
+        if (mine) {
+            uint32_t acc = above;
+#pragma unroll
+            for (int t = 7; t >= 0; --t) {
+                if (acc + h[t] >= (uint32_t)need && digit == 0 && dcount == 0) {
+                    digit = lane * 8 + t;
+                    acc_above = (int)acc;
+                    dcount = (int)h[t];
+                }
+                acc += h[t];
+            }
+        }
+        digit = __shfl_sync(0xffffffffu, digit, src);
+        acc_above = __shfl_sync(0xffffffffu, acc_above, src);
+        dcount = __shfl_sync(0xffffffffu, dcount, src);
+        need -= acc_above;
+        rem = dcount;
+        prefix |= (uint32_t)digit << lo;
+        mask |= dmask << lo;
+        hi = lo - 1;
+        __syncwarp();
     }
-    // Ties at the threshold (only when the keys are exactly equal): the `need`
-    // lowest block indices among them.
+    // Ties at the threshold (keys exactly equal): the `need` lowest block indices.
     uint32_t iprefix = 0xFFFFFFFFu, imask = 0;
     if (rem != need) {
         iprefix = 0;
@@ -235,15 +304,14 @@ __device__ float warp_keep_best(float* sc, int32_t* id, int n, int k, int lane) 
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const uint32_t km = key[j] & mask;
-        const bool tie_ok = (iprefix == 0xFFFFFFFFu && imask == 0) || ((ix[j] & imask) <= iprefix);
+        const bool tie_ok = (imask == 0) || ((ix[j] & imask) <= iprefix);
         if (((valid >> j) & 1u) && (km > prefix || (km == prefix && tie_ok))) {
             keep |= 1u << j;
             ++kc;
             minkey = min(minkey, key[j]);
         }
     }
-    // Exclusive prefix of the per-lane counts.
-    int incl = kc;
+    int incl = kc;  // exclusive prefix of the per-lane counts
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -251,16 +319,57 @@ __device__ float warp_keep_best(float* sc, int32_t* id, int n, int k, int lane) 
     }
     int pos = incl - kc;
     __syncwarp();
+    const int per = (k + NSEG - 1) / NSEG;  // kept entries per segment after the rewrite
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         if ((keep >> j) & 1u) {
-            sc[pos] = key_to_float(key[j]);
-            id[pos] = (int32_t)ix[j];
+            if (out_idx) {
+                out_idx[pos] = (int32_t)ix[j];
+            } else {
+                const int sg = pos / per;
+                qbuf[sg * SEG + (pos - sg * per)] = make_uint2(__float_as_uint(key_to_float(key[j])), ix[j]);
+            }
             ++pos;
         }
     }
     __syncwarp();
-    return key_to_float(__reduce_min_sync(0xffffffffu, minkey));
+    return __reduce_min_sync(0xffffffffu, minkey);
+}
+
+// Scores of 16 queries x this lane's block from 64 accumulator words (4 heads
+// each) and the threshold test. Takers append to this warp's own segment of
+// each query's buffer: lane (sub*16 + qq) holds the segment fill of query qq in
+// `cnt`, so an append needs a shuffle, not an atomic.
+template <bool MASKED>
+__device__ __forceinline__ void score16(const uint32_t* v, int q0, int sub, int b, const Ctl& ctl,
+                                        uint2* seg_q0, int& cnt, int lane) {
+    float sc[16];
+    uint32_t takes = 0;
+#pragma unroll
+    for (int qq = 0; qq < 16; ++qq) {
+        sc[qq] = fmaxf(__uint_as_float(v[4 * qq]), 0.f) + fmaxf(__uint_as_float(v[4 * qq + 1]), 0.f) +
+                 fmaxf(__uint_as_float(v[4 * qq + 2]), 0.f) + fmaxf(__uint_as_float(v[4 * qq + 3]), 0.f);
+        bool t = sc[qq] > ctl.tau[q0 + qq];
+        if (MASKED) t = t && b < ctl.cvis[q0 + qq];
+        takes |= (uint32_t)t << qq;
+    }
+    const uint32_t any = __reduce_or_sync(0xffffffffu, takes);
+    if (!any) return;
+    const uint32_t lt = (1u << lane) - 1u;
+    // All positions come from the counters as they were on entry (independent
+    // shuffles); each lane then advances the counter of its own query once.
+    int add = 0;
+#pragma unroll
+    for (int qq = 0; qq < 16; ++qq) {
+        if ((any >> qq) & 1u) {
+            const bool mine = (takes >> qq) & 1u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, mine);
+            const int pos = __shfl_sync(0xffffffffu, cnt, sub * 16 + qq) + __popc(bal & lt);
+            if (mine) seg_q0[(size_t)qq * CAP + pos] = make_uint2(__float_as_uint(sc[qq]), (uint32_t)b);
+            if (lane == sub * 16 + qq) add = __popc(bal);
+        }
+    }
+    cnt += add;
 }
 
 // Ascending bitonic sort of P (power of two, <= 512) ints in shared memory; one warp.
@@ -286,8 +395,8 @@ __device__ void warp_sort(int32_t* a, int P, int lane) {
 __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int batch,
     int64_t nq, int64_t q_begin, int64_t pcap, int r, int kB, int* __restrict__ tile_counter,
-    float* __restrict__ cand_score, int32_t* __restrict__ cand_idx, int32_t* __restrict__ sel,
-    int32_t* __restrict__ nsel, int32_t* __restrict__ status) {
+    uint2* __restrict__ cand, int32_t* __restrict__ sel, int32_t* __restrict__ nsel,
+    int32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -311,9 +420,8 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         mbar_init(bar(ctl.q_full), 1);
         for (int h = 0; h < 2; ++h) {
             mbar_init(bar(ctl.acc_full[h]), 1);
-            mbar_init(bar(ctl.acc_empty[h]), EPI_THREADS);
+            mbar_init(bar(ctl.acc_empty[h]), EPI_WARPS);
         }
-        mbar_init(bar(ctl.epi_bar), EPI_THREADS);
         mbar_init(bar(ctl.cta_bar), THREADS);
         mbar_init(bar(ctl.mma_done), 1);
         ctl.abort = 0;
@@ -334,8 +442,10 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
     uint32_t kring = 0;       // pooled-key tiles produced / consumed
     uint32_t acc_iter = 0;    // MMA tiles (both halves) issued / drained
     uint32_t q_iter = 0;      // query tiles with a sweep
-    uint32_t epi_phase = 0, cta_phase = 0;
-    uint32_t produced_last[STAGES] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+    uint32_t cta_phase = 0;
+    uint32_t produced_last[STAGES];
+#pragma unroll
+    for (int i = 0; i < STAGES; ++i) produced_last[i] = 0xFFFFFFFFu;
     const uint64_t pol_k = policy_evict_last();
     const uint64_t pol_q = policy_evict_first();
 
@@ -343,11 +453,14 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         // ---- CTA-wide: next query tile (longest first) ----
         if (tid == 0) ctl.tile[iter & 1] = atomicAdd(tile_counter, 1);
         mbar_arrive(bar(ctl.cta_bar));
-        // Warp-uniform outcome: warp collectives follow.
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(ctl.cta_bar), cta_phase, abort_flag))) break;
+        // Warp-uniform outcome (warp collectives follow); for the epilogue warps
+        // also uniform across the group, which meets at named barriers.
+        const bool waited = __all_sync(0xffffffffu, mbar_wait(bar(ctl.cta_bar), cta_phase, abort_flag));
         cta_phase ^= 1;
-        const int64_t u = ctl.tile[iter & 1];
-        if (u >= total_tiles || *abort_flag) break;
+        const int64_t u = waited ? (int64_t)ctl.tile[iter & 1] : total_tiles;
+        bool go = waited && u < total_tiles && !*abort_flag;
+        if (warp >= 2) go = epi_sync_and(go);
+        if (!go) break;
         const int s = (int)(u % batch);
         const int64_t qt = nqt - 1 - u / batch;
         const int64_t j0 = qt * QT;
@@ -410,70 +523,74 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
             const int ch = ew >> 2;           // which 128-column half of a TMEM half
             for (int q = et; q < QT; q += EPI_THREADS) {
                 ctl.tau[q] = q < nrows ? -INFINITY : INFINITY;  // rows past nq never enter
-                ctl.cnt[q] = 0;
+                for (int sg = 0; sg < NSEG; ++sg) ctl.seg[q][sg] = 0;
                 ctl.cvis[q] = q < nrows ? (int)((q_begin + j0 + q) / r) : 0;
             }
-            mbar_arrive(bar(ctl.epi_bar));
-            bool ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.epi_bar), epi_phase, abort_flag));
-            epi_phase ^= 1;
+            bool ok = epi_sync_and(true);
             const size_t slot0 = (size_t)blockIdx.x * QT;
+            const uint32_t tlane = tmem + ((uint32_t)(qd * 32) << 16);
+            int cnt_h[2] = {0, 0};  // this lane's query (h*64 + ch*32 + lane): fill of segment qd
             for (int t = 0; ok && t < ntiles; ++t, ++acc_iter) {
                 const int b = t * BT + qd * 32 + lane;
                 const bool masked = (int64_t)(t + 1) * BT > c_min;
+                bool okt = true;
                 for (int h = 0; h < 2; ++h) {
-                    if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.acc_full[h]), acc_iter & 1u, abort_flag))))
-                        break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int g = 0; g < 4; ++g) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + ((uint32_t)(qd * 32) << 16) + h * NHALF + ch * 128 + g * 32, v);
+                    const bool okh =
+                        __all_sync(0xffffffffu, mbar_wait(bar(ctl.acc_full[h]), acc_iter & 1u, abort_flag));
+                    if (okh) {
+                        tc_fence_after();
+                        const int q0 = h * 64 + ch * 32;
+                        uint32_t v[128];
+                        const uint32_t col = tlane + h * NHALF + ch * 128;
+                        tmem_ld32(col, v);
+                        tmem_ld32(col + 32, v + 32);
+                        tmem_ld32(col + 64, v + 64);
+                        tmem_ld32(col + 96, v + 96);
                         tmem_wait_ld();
-#pragma unroll
-                        for (int qq = 0; qq < 8; ++qq) {
-                            const int q = h * 64 + ch * 32 + g * 8 + qq;
-                            const float sc = fmaxf(__uint_as_float(v[4 * qq]), 0.f) +
-                                             fmaxf(__uint_as_float(v[4 * qq + 1]), 0.f) +
-                                             fmaxf(__uint_as_float(v[4 * qq + 2]), 0.f) +
-                                             fmaxf(__uint_as_float(v[4 * qq + 3]), 0.f);
-                            const bool take = sc > ctl.tau[q] && (!masked || b < ctl.cvis[q]);
-                            const uint32_t bal = __ballot_sync(0xffffffffu, take);
-                            if (bal) {
-                                const int leader = __ffs(bal) - 1;
-                                int pos = 0;
-                                if (lane == leader) pos = atomicAdd(&ctl.cnt[q], __popc(bal));
-                                pos = __shfl_sync(0xffffffffu, pos, leader) + __popc(bal & ((1u << lane) - 1u));
-                                if (take) {
-                                    const size_t e = (slot0 + q) * CAP + pos;
-                                    cand_score[e] = sc;
-                                    cand_idx[e] = b;
-                                }
-                            }
+                        uint2* cq = cand + (slot0 + q0) * CAP + qd * SEG;
+                        int& cnt = cnt_h[h];
+                        if (masked) {
+                            score16<true>(v, q0, 0, b, ctl, cq, cnt, lane);
+                            score16<true>(v + 64, q0 + 16, 1, b, ctl, cq + (size_t)16 * CAP, cnt, lane);
+                        } else {
+                            score16<false>(v, q0, 0, b, ctl, cq, cnt, lane);
+                            score16<false>(v + 64, q0 + 16, 1, b, ctl, cq + (size_t)16 * CAP, cnt, lane);
                         }
+                        tc_fence_before();
                     }
-                    tc_fence_before();
-                    mbar_arrive(bar(ctl.acc_empty[h]));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(ctl.acc_empty[h]));
+                    okt = okt && okh;
                 }
-                if (!ok) break;
-                // All appends of tile t are in; shrink the buffers that could overflow.
-                mbar_arrive(bar(ctl.epi_bar));
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.epi_bar), epi_phase, abort_flag)))) break;
-                epi_phase ^= 1;
+                // All appends of tile t are in; shrink the buffers that could overflow
+                // (a tile adds at most 32 entries to a segment).
+                ctl.seg[ch * 32 + lane][qd] = cnt_h[0];
+                ctl.seg[64 + ch * 32 + lane][qd] = cnt_h[1];
+                if (!(ok = epi_sync_and(okt))) break;
+                bool changed = false;
                 for (int q = ew; q < QT; q += EPI_WARPS) {
-                    const int n = ctl.cnt[q];
-                    if (n > CAP - BT) {
-                        const float tau = warp_keep_best(cand_score + (slot0 + q) * CAP,
-                                                         cand_idx + (slot0 + q) * CAP, n, kB, lane);
+                    int* sq = ctl.seg[q];
+                    if (max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32) {
+                        // Keep the k_B best and raise tau to the smallest kept score. (With
+                        // fewer than k_B entries, only rebalance the segments.)
+                        const int n = sq[0] + sq[1] + sq[2] + sq[3];
+                        const int kk = n < kB ? n : kB;
+                        const uint32_t tk = warp_keep_best(cand + (slot0 + q) * CAP, sq, kk, lane, ctl.hist[ew],
+                                                           nullptr);
+                        __syncwarp();
                         if (lane == 0) {
-                            ctl.tau[q] = tau;
-                            ctl.cnt[q] = kB;
+                            if (kk == kB) ctl.tau[q] = key_to_float(tk);
+                            const int per = (kk + NSEG - 1) / NSEG;
+                            for (int sg = 0; sg < NSEG; ++sg) sq[sg] = max(0, min(per, kk - sg * per));
                         }
+                        changed = true;
                     }
                 }
                 __syncwarp();
-                mbar_arrive(bar(ctl.epi_bar));
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar(ctl.epi_bar), epi_phase, abort_flag)))) break;
-                epi_phase ^= 1;
+                if (!(ok = epi_sync_and(true))) break;
+                (void)changed;
+                cnt_h[0] = ctl.seg[ch * 32 + lane][qd];
+                cnt_h[1] = ctl.seg[64 + ch * 32 + lane][qd];
             }
             // Final selection and ascending output (the pooled-key ring is idle now:
             // use it as sort scratch, 2 KB per warp).
@@ -489,15 +606,14 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                         if (lane == 0) nsel[orow] = kq;
                         continue;
                     }
-                    const int n = ctl.cnt[q];
-                    float* qs = cand_score + (slot0 + q) * CAP;
-                    int32_t* qi = cand_idx + (slot0 + q) * CAP;
-                    if (n > kq) warp_keep_best(qs, qi, n, kq, lane);
+                    const int* sq = ctl.seg[q];
+                    const int n = sq[0] + sq[1] + sq[2] + sq[3];
                     const int m = n < kq ? n : kq;
                     if (m != kq && lane == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
+                    warp_keep_best(cand + (slot0 + q) * CAP, sq, m, lane, ctl.hist[ew], scratch);
                     int P = 1;
                     while (P < m) P <<= 1;
-                    for (int k2 = lane; k2 < P; k2 += 32) scratch[k2] = k2 < m ? qi[k2] : 0x7fffffff;
+                    for (int k2 = m + lane; k2 < P; k2 += 32) scratch[k2] = 0x7fffffff;
                     __syncwarp();
                     warp_sort(scratch, P, lane);
                     for (int k2 = lane; k2 < kB; k2 += 32) out[k2] = k2 < m ? scratch[k2] : -1;
@@ -506,7 +622,6 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                 }
             }
         }
-        if (*abort_flag) break;
     }
 
     // ---- shutdown: drain what this CTA started, then free TMEM ----
@@ -580,7 +695,7 @@ bool fused_topk_supported(const LayerDims& L) { return L.kB <= KMAX_FUSED; }
 
 size_t fused_topk_ws_bytes(int /*batch*/, int64_t /*nq*/) {
     // tile counter (256 B) + candidate buffers of one CTA per SM.
-    return 256 + (size_t)sm_count() * QT * CAP * (sizeof(float) + sizeof(int32_t));
+    return 256 + (size_t)sm_count() * QT * CAP * sizeof(uint2);
 }
 
 cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qrot, int64_t nq,
@@ -596,14 +711,13 @@ cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qro
     const int64_t tiles = ((nq + QT - 1) / QT) * batch;
     const int grid = (int)std::min<int64_t>(grid_max, tiles);
     int* counter = reinterpret_cast<int*>(ws);
-    float* cand_score = reinterpret_cast<float*>((char*)ws + 256);
-    int32_t* cand_idx = reinterpret_cast<int32_t*>(cand_score + (size_t)grid_max * QT * CAP);
+    uint2* cand = reinterpret_cast<uint2*>((char*)ws + 256);
     cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), st);
     if (e != cudaSuccess) return e;
     cudaFuncSetAttribute(fused_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     note_launch();
     fused_topk_kernel<<<grid, THREADS, SMEM, st>>>(tm_q, tm_k, batch, nq, q_begin, pcap, L.r, L.kB, counter,
-                                                   cand_score, cand_idx, sel, nsel, status);
+                                                   cand, sel, nsel, status);
     return cudaGetLastError();
 }
 

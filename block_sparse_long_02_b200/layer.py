@@ -22,11 +22,13 @@ from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_de
 
 
 class QSALayer:
-    def __init__(self, cfg: Config, batch: int, cap: int, device="cuda", rms_w: Optional[torch.Tensor] = None):
+    def __init__(self, cfg: Config, batch: int, cap: int, device="cuda", rms_w: Optional[torch.Tensor] = None,
+                 kv_cap: Optional[int] = None):
         self.cfg, self.batch, self.cap = cfg, batch, cap
         self.device = torch.device(device)
         bf = torch.bfloat16
-        self.k_cache = torch.zeros(batch, cap, cfg.kv_heads, cfg.head_dim, dtype=bf, device=self.device)
+        kv_cap = cap if kv_cap is None else kv_cap  # smaller only for indexer-only use
+        self.k_cache = torch.zeros(batch, kv_cap, cfg.kv_heads, cfg.head_dim, dtype=bf, device=self.device)
         self.v_cache = torch.zeros_like(self.k_cache)
         self.idx_k_cache = torch.zeros(batch, cap, cfg.idx_dim, dtype=bf, device=self.device)
         self.pooled = torch.zeros(batch, cap // cfg.r, cfg.idx_dim, dtype=bf, device=self.device)
