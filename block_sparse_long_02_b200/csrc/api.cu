@@ -123,7 +123,7 @@ TopkWs topk_layout(const qsa::LayerDims& L, int batch, int64_t cap, int64_t nq) 
 }
 
 struct DecodeWs {
-    size_t qrot, scores, sel, nsel, part, total;
+    size_t qrot, scores, sel, nsel, part, hist, counters, winners, cand, total;
 };
 
 DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
@@ -134,7 +134,11 @@ DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
     w.sel = w.scores + align_up((size_t)batch * std::max<int64_t>(1, cap / L.r) * 4);
     w.nsel = w.sel + align_up((size_t)batch * L.kB * 4);
     w.part = w.nsel + align_up((size_t)batch * 4);
-    w.total = w.part + align_up((size_t)batch * L.q_heads * S * 132 * 4);
+    w.hist = w.part + align_up((size_t)batch * L.q_heads * S * 132 * 4);
+    w.counters = w.hist + align_up((size_t)batch * 2048 * 4);
+    w.winners = w.counters + align_up((size_t)batch * 4 * 4);
+    w.cand = w.winners + align_up((size_t)batch * L.kB * 4);
+    w.total = w.cand + align_up((size_t)batch * qsa::kDecodeCand * 8);
     return w;
 }
 
@@ -325,14 +329,17 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + w.sel);
     int32_t* nsel = nsel_out ? nsel_out : reinterpret_cast<int32_t*>(base + w.nsel);
     float* part = reinterpret_cast<float*>(base + w.part);
+    qsa::DecodeSelWs sw;
+    sw.hist = reinterpret_cast<uint32_t*>(base + w.hist);
+    sw.counters = reinterpret_cast<int32_t*>(base + w.counters);
+    sw.winners = reinterpret_cast<int32_t*>(base + w.winners);
+    sw.cand = reinterpret_cast<uint2*>(base + w.cand);
     cudaStream_t st = (cudaStream_t)stream;
     TRY(cuda_check(qsa::launch_decode_prepare(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache,
-                                              idx_k_cache, pooled, cap, rms_w, qrot, status, st),
+                                              idx_k_cache, pooled, cap, rms_w, qrot, sw, status, st),
                    "decode prepare"));
-    TRY(cuda_check(qsa::launch_decode_scores(L, batch, pos, qrot, pooled, cap, scores, st), "decode scores"));
-    TRY(cuda_check(qsa::launch_select_decode(L, batch, scores, std::max<int64_t>(1, cap / L.r), pos,
-                                             cap, sel, nsel, st),
-                   "decode select"));
+    TRY(cuda_check(qsa::launch_decode_scores(L, batch, pos, qrot, pooled, cap, scores, sw, st), "decode scores"));
+    TRY(cuda_check(qsa::launch_decode_select(L, batch, pos, cap, scores, sw, sel, nsel, st), "decode select"));
     return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel,
                                                    nsel, part, out, st),
                       "decode attention");

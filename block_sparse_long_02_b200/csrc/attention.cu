@@ -383,28 +383,34 @@ __global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
     }
 }
 
-// Combine the S partials of each (sequence, head): one warp per head.
-__global__ void decode_combine_kernel(const float* __restrict__ part, int rows, int S,
-                                      uint16_t* __restrict__ out) {
-    const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (row >= rows) return;
+// Combine the S partials of each (sequence, head): one CTA of 128 threads per
+// head, thread d owns output dim d; the partials' maxima and sums are staged in
+// shared memory, the S partial rows are read coalesced.
+__global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part, int S,
+                                                            uint16_t* __restrict__ out) {
+    __shared__ float wgt[64];
+    __shared__ float inv_l;
+    const int row = blockIdx.x, d = threadIdx.x;
     const float* src = part + (size_t)row * S * 132;
-    float m = -INFINITY;
-    for (int k = 0; k < S; ++k) m = fmaxf(m, src[(size_t)k * 132 + 128]);
-    float l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < S; ++k) {
-        const float* pk = src + (size_t)k * 132;
-        const float c = (m == -INFINITY) ? 0.f : exp2f(pk[128] - m);
-        l += pk[129] * c;
+    if (d < 32) {
+        float m = -INFINITY;
+        for (int k = d; k < S; k += 32) m = fmaxf(m, src[(size_t)k * 132 + 128]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] += pk[lane * 4 + e] * c;
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        float l = 0.f;
+        for (int k = d; k < S; k += 32) {
+            const float c = (m == -INFINITY) ? 0.f : exp2f(src[(size_t)k * 132 + 128] - m);
+            wgt[k] = c;
+            l += src[(size_t)k * 132 + 129] * c;
+        }
+        l = warp_sum(l);
+        if (d == 0) inv_l = l > 0.f ? 1.f / l : 0.f;
     }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    uint2 v;
-    v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(out + (size_t)row * kHeadDim + lane * 4) = v;
+    __syncthreads();
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < S; ++k) acc = fmaf(src[(size_t)k * 132 + d], wgt[k], acc);
+    out[(size_t)row * kHeadDim + d] = f32_to_bf16(acc * inv_l);
 }
 
 }  // namespace
@@ -449,7 +455,7 @@ cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t
     if (e != cudaSuccess) return e;
     const int rows = batch * L.q_heads;
     note_launch();
-    decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(part, rows, S, out);
+    decode_combine_kernel<<<rows, 128, 0, st>>>(part, S, out);
     return cudaGetLastError();
 }
 

@@ -51,11 +51,6 @@ cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qro
 cudaError_t launch_select_rows(const LayerDims& L, int batch, const float* scores, int64_t ld,
                                int64_t q_begin, int64_t j0, int64_t nrows, int64_t nq_total,
                                int32_t* sel, int32_t* nsel, cudaStream_t st);
-// Variant for decode: position of sequence s is pos[s]; rows [batch][ld].
-cudaError_t launch_select_decode(const LayerDims& L, int batch, const float* scores, int64_t ld,
-                                 const int64_t* pos, int64_t cap, int32_t* sel, int32_t* nsel,
-                                 cudaStream_t st);
-
 // attention.cu
 cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_t* q,
                                     int64_t q_begin, int64_t nq, const uint16_t* kc,
@@ -68,15 +63,26 @@ cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
                                     float* part, uint16_t* out, cudaStream_t st);
 
-// decode.cu
+// decode.cu. Per-sequence selection state in the decode workspace.
+constexpr int kDecodeCand = 4096;  // candidates of the threshold digit kept for the final pick
+struct DecodeSelWs {
+    uint32_t* hist;     // [batch][2048] histogram of the top 11 key bits
+    int32_t* counters;  // [batch][4]: sure winners, candidates, finished CTAs
+    int32_t* winners;   // [batch][k_B]
+    uint2* cand;        // [batch][kDecodeCand] (key, block)
+};
+int decode_select_ctas(int batch);
 cudaError_t launch_decode_prepare(const LayerDims& L, int batch, const int64_t* pos,
                                   const uint16_t* k, const uint16_t* v, const uint16_t* idx_q,
                                   const uint16_t* idx_k, uint16_t* kc, uint16_t* vc,
                                   uint16_t* idx_k_cache, uint16_t* pooled, int64_t cap,
-                                  const float* rms_w, uint16_t* qrot, int32_t* status,
-                                  cudaStream_t st);
+                                  const float* rms_w, uint16_t* qrot, DecodeSelWs sw,
+                                  int32_t* status, cudaStream_t st);
 cudaError_t launch_decode_scores(const LayerDims& L, int batch, const int64_t* pos,
                                  const uint16_t* qrot, const uint16_t* pooled, int64_t cap,
-                                 float* scores, cudaStream_t st);
+                                 float* scores, DecodeSelWs sw, cudaStream_t st);
+cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
+                                 const float* scores, DecodeSelWs sw, int32_t* sel, int32_t* nsel,
+                                 cudaStream_t st);
 
 }  // namespace qsa

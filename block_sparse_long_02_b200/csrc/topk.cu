@@ -1,237 +1,14 @@
 // a5: top-k_B block selection over a materialised score row
 // ("QSA (Qwen Sparse Attention)" concept page, (A) "Top-k_B block selection";
 // "Qwen Sparse Attention" gallery page pseudo-code top_k(scores, k=512)).
-// Rank = (score descending, block index ascending); output ascending.
-//
-// One CTA per row. Scores map to order-preserving 32-bit keys; a radix select
-// finds the k-th key T in three digit levels (11, 11, 10 bits):
-//   pass 1 (global): 2048-bin shared-memory histogram of the top digit;
-//   pass 2 (global): entries above the threshold digit are taken outright,
-//                    entries equal to it become candidates in shared memory;
-//   levels 2-3 run on the candidates; ties at T take the lowest indices.
-// The selected indices are then bitonic-sorted in shared memory. If the
-// candidates overflow shared memory (e.g. thousands of exactly equal scores),
-// the digit levels re-read the row and an order-preserving compaction pass
-// writes the output directly.
+// One CTA per row; the exact selection routine is in select.cuh.
 #include <algorithm>
 
 #include "kernels.h"
+#include "select.cuh"
 
 namespace qsa {
 namespace {
-
-constexpr int T = 512;           // threads per CTA
-constexpr int NW = T / 32;
-constexpr int BINS = 2048;
-constexpr int CAND = 4096;
-
-struct SelSmem {
-    uint32_t hist[BINS];
-    uint32_t cand_key[CAND];
-    int32_t cand_idx[CAND];
-    int32_t out[kMaxKB];
-    uint32_t wsum[NW];
-    int32_t n_out, n_cand, bin, above, ties;
-};
-
-// Finds bin B (counting from the top) with above(B) < need <= above(B) + hist[B].
-// Result in sm.bin / sm.above. Must be called by all threads; nbins <= 2048.
-__device__ void find_bin(SelSmem& sm, int nbins, uint32_t need) {
-    __syncthreads();
-    const int tid = threadIdx.x;
-    if (tid < 32) {
-        const int per = nbins / 32;
-        uint32_t sum = 0;
-        for (int b = 0; b < per; ++b) sum += sm.hist[tid * per + b];
-        // Inclusive suffix sum over lanes (from lane 31 down).
-        uint32_t suf = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
-            if (tid + o < 32) suf += v;
-        }
-        const uint32_t above_lane = suf - sum;  // count in lanes > tid
-        const bool mine = above_lane < need && need <= suf;
-        if (mine) {
-            uint32_t acc = above_lane;
-            for (int b = per - 1; b >= 0; --b) {
-                const uint32_t h = sm.hist[tid * per + b];
-                if (acc + h >= need) {
-                    sm.bin = tid * per + b;
-                    sm.above = (int32_t)acc;
-                    break;
-                }
-                acc += h;
-            }
-        }
-    }
-    __syncthreads();
-}
-
-__device__ void clear_hist(SelSmem& sm) {
-    for (int b = threadIdx.x; b < BINS; b += T) sm.hist[b] = 0;
-    __syncthreads();
-}
-
-// Exclusive prefix of `flag` over the CTA in thread order; returns the CTA total.
-__device__ uint32_t cta_scan(SelSmem& sm, bool flag, uint32_t& prefix) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const uint32_t ballot = __ballot_sync(0xffffffffu, flag);
-    const uint32_t wpre = __popc(ballot & ((1u << lane) - 1u));
-    if (lane == 0) sm.wsum[w] = __popc(ballot);
-    __syncthreads();
-    uint32_t base = 0, total = 0;
-    for (int k = 0; k < NW; ++k) {
-        const uint32_t v = sm.wsum[k];
-        if (k < w) base += v;
-        total += v;
-    }
-    __syncthreads();
-    prefix = base + wpre;
-    return total;
-}
-
-// Slow general path: exact digits by re-reading the row, then an
-// order-preserving compaction that writes the sorted selection.
-__device__ void select_general(SelSmem& sm, const float* x, int64_t n, int kB, uint32_t b1,
-                               uint32_t need1, int32_t* sel) {
-    const int tid = threadIdx.x;
-    // Level 2.
-    clear_hist(sm);
-    for (int64_t i = tid; i < n; i += T) {
-        const uint32_t k = float_key(x[i]);
-        if ((k >> 21) == b1) atomicAdd(&sm.hist[(k >> 10) & 2047u], 1u);
-    }
-    find_bin(sm, 2048, need1);
-    const uint32_t b2 = sm.bin;
-    const uint32_t need2 = need1 - sm.above;
-    clear_hist(sm);
-    const uint32_t p2 = (b1 << 11) | b2;
-    for (int64_t i = tid; i < n; i += T) {
-        const uint32_t k = float_key(x[i]);
-        if ((k >> 10) == p2) atomicAdd(&sm.hist[k & 1023u], 1u);
-    }
-    find_bin(sm, 1024, need2);
-    const uint32_t key_t = (p2 << 10) | (uint32_t)sm.bin;
-    const uint32_t need_t = need2 - sm.above;  // ties at key_t to take, lowest index first
-    // Ordered compaction.
-    uint32_t taken = 0, ties = 0;
-    for (int64_t base = 0; base < n; base += T) {
-        const int64_t i = base + tid;
-        uint32_t k = 0;
-        if (i < n) k = float_key(x[i]);
-        const bool is_tie = i < n && k == key_t;
-        uint32_t tie_pre;
-        const uint32_t tie_tot = cta_scan(sm, is_tie, tie_pre);
-        const bool take = i < n && (k > key_t || (is_tie && ties + tie_pre < need_t));
-        uint32_t pre;
-        const uint32_t tot = cta_scan(sm, take, pre);
-        if (take) sel[taken + pre] = (int32_t)i;
-        taken += tot;
-        ties += tie_tot;
-    }
-    for (int k = (int)taken + tid; k < kB; k += T) sel[k] = -1;
-}
-
-__device__ void select_row(SelSmem& sm, const float* x, int64_t n, int kB, int32_t* sel,
-                           int32_t* nsel) {
-    const int tid = threadIdx.x;
-    if (n <= kB) {
-        for (int k = tid; k < kB; k += T) sel[k] = k < n ? k : -1;
-        if (tid == 0) *nsel = (int32_t)(n > 0 ? n : 0);
-        return;
-    }
-    if (tid == 0) *nsel = kB;
-    // Level 1.
-    clear_hist(sm);
-    for (int64_t i = tid; i < n; i += T) atomicAdd(&sm.hist[float_key(x[i]) >> 21], 1u);
-    find_bin(sm, BINS, (uint32_t)kB);
-    const uint32_t b1 = sm.bin;
-    const uint32_t need1 = (uint32_t)kB - (uint32_t)sm.above;
-    if (tid == 0) {
-        sm.n_out = 0;
-        sm.n_cand = 0;
-    }
-    __syncthreads();
-    for (int64_t i = tid; i < n; i += T) {
-        const uint32_t k = float_key(x[i]);
-        const uint32_t b = k >> 21;
-        if (b > b1) {
-            sm.out[atomicAdd(&sm.n_out, 1)] = (int32_t)i;
-        } else if (b == b1) {
-            const int p = atomicAdd(&sm.n_cand, 1);
-            if (p < CAND) {
-                sm.cand_key[p] = k;
-                sm.cand_idx[p] = (int32_t)i;
-            }
-        }
-    }
-    __syncthreads();
-    const int nc = sm.n_cand;
-    if (nc > CAND) {
-        select_general(sm, x, n, kB, b1, need1, sel);
-        return;
-    }
-    // Level 2 on the candidates.
-    clear_hist(sm);
-    for (int c = tid; c < nc; c += T) atomicAdd(&sm.hist[(sm.cand_key[c] >> 10) & 2047u], 1u);
-    find_bin(sm, 2048, need1);
-    const uint32_t b2 = sm.bin;
-    const uint32_t need2 = need1 - sm.above;
-    for (int c = tid; c < nc; c += T)
-        if (((sm.cand_key[c] >> 10) & 2047u) > b2) sm.out[atomicAdd(&sm.n_out, 1)] = sm.cand_idx[c];
-    // Level 3.
-    clear_hist(sm);
-    for (int c = tid; c < nc; c += T)
-        if (((sm.cand_key[c] >> 10) & 2047u) == b2) atomicAdd(&sm.hist[sm.cand_key[c] & 1023u], 1u);
-    find_bin(sm, 1024, need2);
-    const uint32_t key_t = (b1 << 21) | (b2 << 10) | (uint32_t)sm.bin;
-    const uint32_t need_t = need2 - sm.above;
-    if (tid == 0) sm.ties = 0;
-    __syncthreads();
-    for (int c = tid; c < nc; c += T) {
-        const uint32_t k = sm.cand_key[c];
-        if ((k >> 10) == (key_t >> 10) && k > key_t) sm.out[atomicAdd(&sm.n_out, 1)] = sm.cand_idx[c];
-        if (k == key_t) atomicAdd(&sm.ties, 1);
-    }
-    __syncthreads();
-    const int nties = sm.ties;
-    for (int c = tid; c < nc; c += T) {
-        if (sm.cand_key[c] != key_t) continue;
-        bool take = true;
-        if ((uint32_t)nties != need_t) {
-            const int32_t me = sm.cand_idx[c];
-            uint32_t rank = 0;
-            for (int d = 0; d < nc; ++d)
-                rank += (sm.cand_key[d] == key_t && sm.cand_idx[d] < me) ? 1u : 0u;
-            take = rank < need_t;
-        }
-        if (take) sm.out[atomicAdd(&sm.n_out, 1)] = sm.cand_idx[c];
-    }
-    __syncthreads();
-    // Bitonic sort of the kB selected indices (padded to a power of two).
-    int P = 1;
-    while (P < kB) P <<= 1;
-    for (int k = kB + tid; k < P; k += T) sm.out[k] = 0x7fffffff;
-    __syncthreads();
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < P; i += T) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const int32_t a = sm.out[i], b = sm.out[ixj];
-                    const bool up = (i & k) == 0;
-                    if ((a > b) == up) {
-                        sm.out[i] = b;
-                        sm.out[ixj] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
-    for (int k = tid; k < kB; k += T) sel[k] = sm.out[k];
-}
 
 __global__ void __launch_bounds__(T) select_rows_kernel(const float* __restrict__ scores, int64_t ld,
                                                         int64_t q_begin, int64_t j0, int64_t nrows,
@@ -249,19 +26,6 @@ __global__ void __launch_bounds__(T) select_rows_kernel(const float* __restrict_
                    nsel + out_row);
         __syncthreads();
     }
-}
-
-__global__ void __launch_bounds__(T) select_decode_kernel(const float* __restrict__ scores,
-                                                          int64_t ld, const int64_t* __restrict__ pos,
-                                                          int64_t cap, int r, int kB,
-                                                          int32_t* __restrict__ sel,
-                                                          int32_t* __restrict__ nsel) {
-    extern __shared__ __align__(16) uint8_t raw[];
-    SelSmem& sm = *reinterpret_cast<SelSmem*>(raw);
-    const int s = blockIdx.x;
-    const int64_t p = pos[s];
-    const int64_t n = (p >= 0 && p < cap) ? p / r : 0;
-    select_row(sm, scores + (size_t)s * ld, n, kB, sel + (size_t)s * kB, nsel + s);
 }
 
 int sms() {
@@ -284,17 +48,6 @@ cudaError_t launch_select_rows(const LayerDims& L, int batch, const float* score
     note_launch();
     select_rows_kernel<<<grid, T, smem, st>>>(scores, ld, q_begin, j0, nrows, nq_total, batch, L.r,
                                               L.kB, sel, nsel);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_select_decode(const LayerDims& L, int batch, const float* scores, int64_t ld,
-                                 const int64_t* pos, int64_t cap, int32_t* sel, int32_t* nsel,
-                                 cudaStream_t st) {
-    if (batch <= 0) return cudaSuccess;
-    const int smem = (int)sizeof(SelSmem);
-    cudaFuncSetAttribute(select_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    note_launch();
-    select_decode_kernel<<<batch, T, smem, st>>>(scores, ld, pos, cap, L.r, L.kB, sel, nsel);
     return cudaGetLastError();
 }
 
