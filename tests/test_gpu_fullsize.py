@@ -1,0 +1,213 @@
+"""Parity at the measured workloads' full sizes, in the launch configuration
+bench.py times (QSALayer: qsa_compress_keys -> fused qsa_topk_blocks ->
+qsa_sparse_attention for prefill; qsa_decode_step for decode).
+
+The oracle recomputes sampled rows one by one (scores over every visible block,
+selection, attention over the selected tokens, fetching only the K/V rows it
+needs); every row of the GPU output is checked against the invariants that
+hold at any size (selection count, range, order, padding; needle recall)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import bits, check_attention, check_selection, score_tol
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle(w):
+    return oracle.Oracle.for_workload(w)
+
+
+def check_all_rows_invariants(sel: torch.Tensor, nsel: torch.Tensor, q_begin: int, r: int, kB: int,
+                              chunk: int = 1 << 16):
+    """Every row: nsel = min(k_B, floor(i/r)); entries strictly ascending in
+    [0, floor(i/r)); -1 padding after nsel. (Checked in row chunks.)"""
+    for j0 in range(0, sel.shape[0], chunk):
+        _invariants(sel[j0:j0 + chunk].cpu().numpy(), nsel[j0:j0 + chunk].cpu().numpy(), q_begin + j0, r, kB)
+
+
+def _invariants(sel: np.ndarray, nsel: np.ndarray, q_begin: int, r: int, kB: int):
+    nq = sel.shape[0]
+    i = q_begin + np.arange(nq)
+    vis = i // r
+    want = np.minimum(kB, vis)
+    assert np.array_equal(nsel, want), np.nonzero(nsel != want)[0][:5]
+    cols = np.arange(kB)[None, :]
+    valid = cols < want[:, None]
+    assert (sel[~valid] == -1).all()
+    v = np.where(valid, sel, 0)
+    assert (v[valid] >= 0).all() and (np.where(valid, sel, -1) < vis[:, None]).all()
+    d = np.diff(np.where(valid, sel, np.iinfo(np.int32).max), axis=1)
+    both = valid[:, 1:] & valid[:, :-1]
+    assert (d[both] > 0).all()
+
+
+def oracle_row_check(w, o, s, i, idx_q_row, q_row, pooled_gpu, sel_row, nsel_i, out_row, what):
+    ref = o.row(i, idx_q_row, pooled_gpu)
+    tol = score_tol(o.rotate_query(idx_q_row, i), pooled_gpu, ref["scores"])
+    check_selection(sel_row, nsel_i, ref["scores"], tol, o.k_blocks, what)
+    toks = o.token_set(sel_row[:nsel_i], i)
+    kc = w.host_rows("k", s, toks)
+    vc = w.host_rows("v", s, toks)
+    out_ref, _ = o.attention(q_row, kc, vc, np.arange(toks.size, dtype=np.int64))
+    check_attention(out_row, out_ref, what)
+
+
+def _prefill(w, device="cuda"):
+    import block_sparse_long_02_b200 as qsa
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    cfg = qsa.Config.of(w)
+    B, n, S = w.batch, w.n, w.decode_steps
+    cap = -(-(n + S) // w.r) * w.r
+    L = QSALayer(cfg, B, cap, device=device)
+    w.device_fill("k", L.k_cache.view(B, cap, -1), rows=(0, n))
+    w.device_fill("v", L.v_cache.view(B, cap, -1), rows=(0, n))
+    w.device_fill("idx_k", L.idx_k_cache, rows=(0, n))
+    q = torch.empty(B, n, cfg.q_heads, cfg.head_dim, dtype=torch.bfloat16, device=device)
+    iq = torch.empty(B, n, cfg.idx_heads, cfg.idx_dim, dtype=torch.bfloat16, device=device)
+    w.device_fill("q", q.view(B, n, -1), rows=(0, n))
+    w.device_fill("idx_q", iq.view(B, n, -1), rows=(0, n))
+    out = torch.empty_like(q)
+    sel = torch.empty(B, n, cfg.k_blocks, dtype=torch.int32, device=device)
+    nsel = torch.empty(B, n, dtype=torch.int32, device=device)
+    L.prefill(q, iq, 0, n, out, sel, nsel)
+    torch.cuda.synchronize()
+    return cfg, L, q, iq, out, sel, nsel
+
+
+def _sample_rows(w, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.integers(w.r * (w.k_blocks + 1), w.n, count).tolist())
+    rows |= {w.n - 1, w.r * w.k_blocks, w.r * w.k_blocks + w.r - 1, 3, 4 * 37 + 2}
+    return sorted(rows)
+
+
+def _check_prefill(w, cfg, L, q, iq, out, sel, nsel, rows, needles):
+    o = _oracle(w)
+    s = 0
+    check_all_rows_invariants(sel[s], nsel[s], 0, w.r, cfg.k_blocks)
+    probe_rows = sorted(set(rows) | {p for _, p in needles if p < w.n})
+    pr = torch.tensor(probe_rows, device=sel.device)
+    g_sel = dict(zip(probe_rows, sel[s, pr].cpu().numpy()))
+    g_nsel = dict(zip(probe_rows, nsel[s, pr].cpu().numpy()))
+    # Needles: each probe selects its planted block.
+    for b, p in needles:
+        if p < w.n:
+            assert b in set(g_sel[p][: g_nsel[p]].tolist()), (b, p)
+    pooled = bits(L.pooled)[s, : w.n // w.r]
+    idx_q = w.host_rows("idx_q", s, rows).reshape(len(rows), 4, 128)
+    q_rows = w.host_rows("q", s, rows).reshape(len(rows), cfg.q_heads, 128)
+    out_rows = out[s, torch.tensor(rows, device=out.device)].float().cpu().numpy()
+    for k, i in enumerate(rows):
+        oracle_row_check(w, o, s, i, idx_q[k], q_rows[k], pooled, g_sel[i], int(g_nsel[i]), out_rows[k],
+                         f"{w.name} row {i}")
+    # The GPU's pooled keys match the oracle's on a sample of blocks (<= 1 ulp).
+    nb = w.n // w.r
+    blocks = np.unique(np.concatenate([np.arange(64), np.random.default_rng(5).integers(0, nb, 512), [nb - 1]]))
+    for b in blocks[::16]:
+        raw = w.host_rows("idx_k", s, np.arange(w.r * b, w.r * b + w.r))
+        ref = o.pool_block(raw, w.r * b)["out"]
+        assert np.abs(ref.astype(np.int32) - pooled[b].astype(np.int32)).max() <= 1, b
+    return o
+
+
+def test_prefill_128k_full_size():
+    w = synth.WORKLOADS["prefill_n128k"]
+    cfg, L, q, iq, out, sel, nsel = _prefill(w)
+    rows = _sample_rows(w, 24, 1) + sorted({p for _, p in w.needles(0)})[:16]
+    _check_prefill(w, cfg, L, q, iq, out, sel, nsel, sorted(set(rows)), w.needles(0))
+
+
+def _decode_inputs(w, L, s_idx, step):
+    """New-token tensors [batch][...] for decode step `step` (position n + step)."""
+    B = w.batch
+    p = w.n + step
+    out = {}
+    for name in ("q", "k", "v", "idx_q", "idx_k"):
+        t = torch.empty(B, w.row_len(name), dtype=torch.bfloat16, device="cuda")
+        for s in range(B):
+            synth.fill_device(w.seed(s), synth.TENSOR_IDS[name], p * w.row_len(name), w.row_len(name),
+                              t[s].data_ptr())
+        out[name] = t
+    return out
+
+
+def _check_decode_step(w, o, L, step, out, sel, nsel, seqs):
+    cfg = L.cfg
+    p = w.n + step
+    g_sel, g_nsel = sel.cpu().numpy(), nsel.cpu().numpy()
+    g_out = out.float().cpu().numpy()
+    for s in seqs:
+        pooled = bits(L.pooled[s, : p // w.r])
+        idx_q = w.host_rows("idx_q", s, [p]).reshape(4, 128)
+        q_row = w.host_rows("q", s, [p]).reshape(cfg.q_heads, 128)
+        m = int(g_nsel[s])
+        assert m == min(cfg.k_blocks, p // w.r)
+        assert (g_sel[s, m:] == -1).all() and np.all(np.diff(g_sel[s, :m]) > 0)
+        for b, pp in w.needles(s):
+            if pp == p:
+                assert b in set(g_sel[s, :m].tolist()), (s, b, p)
+        oracle_row_check(w, o, s, p, idx_q, q_row, pooled, g_sel[s], m, g_out[s].reshape(cfg.q_heads, 128),
+                         f"{w.name} seq {s} step {step}")
+
+
+def _decode_setup(w):
+    import block_sparse_long_02_b200 as qsa
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    cfg = qsa.Config.of(w)
+    B, n = w.batch, w.n
+    cap = -(-(n + w.decode_steps) // w.r) * w.r
+    L = QSALayer(cfg, B, cap)
+    w.device_fill("k", L.k_cache.view(B, cap, -1), rows=(0, n))
+    w.device_fill("v", L.v_cache.view(B, cap, -1), rows=(0, n))
+    w.device_fill("idx_k", L.idx_k_cache, rows=(0, n))
+    L.compress(0, n // w.r)
+    return cfg, L
+
+
+@pytest.mark.parametrize("name", ["decode_b1_n32k", "decode_b8_n256k"])
+def test_decode_full_size(name):
+    w = synth.WORKLOADS[name]
+    cfg, L = _decode_setup(w)
+    B = w.batch
+    o = _oracle(w)
+    pos = torch.full((B,), w.n, dtype=torch.int64, device="cuda")
+    inp = _decode_inputs(w, L, None, 0)
+    out = torch.empty(B, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(B, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(B, dtype=torch.int32, device="cuda")
+    L.decode_step(pos, inp["q"].view(B, -1, 128), inp["k"].view(B, -1, 128), inp["v"].view(B, -1, 128),
+                  inp["idx_q"].view(B, 4, 128), inp["idx_k"], out, sel, nsel)
+    torch.cuda.synchronize()
+    _check_decode_step(w, o, L, 0, out, sel, nsel, range(B))
+
+
+def test_prefill_1m_then_64_decode_steps_sampled():
+    """The benchmark's workload end to end: 1M-token prefill (sampled rows and all
+    row invariants), then 64 decode steps (4 of them checked against the oracle)."""
+    w = synth.WORKLOADS["prefill_n1m_decode64"]
+    cfg, L, q, iq, out, sel, nsel = _prefill(w)
+    needles = w.needles(0)
+    rows = _sample_rows(w, 6, 2) + sorted({p for _, p in needles if p < w.n})[:4]
+    o = _check_prefill(w, cfg, L, q, iq, out, sel, nsel, sorted(set(rows)), needles)
+    del q, iq, out, sel, nsel
+    torch.cuda.empty_cache()
+    B = w.batch
+    dout = torch.empty(B, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
+    dsel = torch.empty(B, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    dn = torch.empty(B, dtype=torch.int32, device="cuda")
+    for step in range(w.decode_steps):
+        pos = torch.full((B,), w.n + step, dtype=torch.int64, device="cuda")
+        inp = _decode_inputs(w, L, None, step)
+        L.decode_step(pos, inp["q"].view(B, -1, 128), inp["k"].view(B, -1, 128), inp["v"].view(B, -1, 128),
+                      inp["idx_q"].view(B, 4, 128), inp["idx_k"], dout, dsel, dn)
+        if step in (0, 3, 31, 63):
+            torch.cuda.synchronize()
+            _check_decode_step(w, o, L, step, dout, dsel, dn, range(B))
