@@ -43,6 +43,7 @@ constexpr int NHALF = 256;             // TMEM columns per half = 64 queries x 4
 constexpr int STAGES = 2;
 constexpr int CAP = 1024;              // candidate entries per query
 constexpr int NSEG = 4;                // one segment per TMEM lane quadrant (epilogue warp)
+constexpr int SAMPLE = 16;             // estimate phase: every SAMPLE-th pooled-key tile
 constexpr int SEG = CAP / NSEG;        // entries per segment
 constexpr int KMAX_FUSED = 512;        // largest k_B handled here
 constexpr int EPI_WARPS = 8;
@@ -57,7 +58,10 @@ struct Ctl {
     uint64_t q_full, acc_full[2], acc_empty[2], cta_bar, mma_done;
     uint32_t tmem_base;
     int abort;
-    int tile[2];
+    int tile[2];        // query tile of the next two iterations (double-buffered)
+    int redo[2];        // 1: repeat the tile in exact mode for the queries that failed
+    float tau_est[QT];  // threshold estimated from the sample phase (-inf: none)
+    uint8_t failed[QT]; // query's candidates did not prove the top-k in estimate mode
     float tau[QT];
     int seg[QT][NSEG];  // entries in each segment of a query's candidate buffer
     int cvis[QT];
@@ -336,6 +340,17 @@ __device__ uint32_t warp_keep_best(uint2* qbuf, const int* segn, int k, int lane
     return __reduce_min_sync(0xffffffffu, minkey);
 }
 
+// Number of entries of a segmented buffer whose score is strictly above thr.
+__device__ int warp_count_above(const uint2* qbuf, const int* segn, float thr, int lane) {
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int e = ((j & 7) << 5) | lane;
+        if (e < segn[j >> 3] && __uint_as_float(qbuf[(j >> 3) * SEG + e].x) > thr) ++c;
+    }
+    return (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+}
+
 // Scores of 16 queries x this lane's block from 64 accumulator words (4 heads
 // each) and the threshold test. Takers append to this warp's own segment of
 // each query's buffer: lane (sub*16 + qq) holds the segment fill of query qq in
@@ -349,7 +364,7 @@ __device__ __forceinline__ void score16(const uint32_t* v, int q0, int sub, int 
     for (int qq = 0; qq < 16; ++qq) {
         sc[qq] = fmaxf(__uint_as_float(v[4 * qq]), 0.f) + fmaxf(__uint_as_float(v[4 * qq + 1]), 0.f) +
                  fmaxf(__uint_as_float(v[4 * qq + 2]), 0.f) + fmaxf(__uint_as_float(v[4 * qq + 3]), 0.f);
-        bool t = sc[qq] > ctl.tau[q0 + qq];
+        bool t = sc[qq] >= ctl.tau[q0 + qq];
         if (MASKED) t = t && b < ctl.cvis[q0 + qq];
         takes |= (uint32_t)t << qq;
     }
@@ -391,6 +406,15 @@ __device__ void warp_sort(int32_t* a, int P, int lane) {
     }
 }
 
+// Sweep order of the pooled-key tiles: with nsamp > 0, first the sample tiles
+// 0, SAMPLE, 2*SAMPLE, ... then the others in ascending order.
+__device__ __forceinline__ int tile_at(int t, int nsamp) {
+    if (t < nsamp) return t * SAMPLE;
+    if (nsamp == 0) return t;
+    const int i = t - nsamp;
+    return i + i / (SAMPLE - 1) + 1;
+}
+
 // --------------------------------------------------------------------- kernel
 __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int batch,
@@ -425,6 +449,8 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         mbar_init(bar(ctl.cta_bar), THREADS);
         mbar_init(bar(ctl.mma_done), 1);
         ctl.abort = 0;
+        ctl.tile[0] = atomicAdd(tile_counter, 1);
+        ctl.redo[0] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -450,14 +476,14 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
     const uint64_t pol_q = policy_evict_first();
 
     for (int iter = 0;; ++iter) {
-        // ---- CTA-wide: next query tile (longest first) ----
-        if (tid == 0) ctl.tile[iter & 1] = atomicAdd(tile_counter, 1);
+        // ---- CTA-wide: this iteration's query tile (chosen by the previous one) ----
         mbar_arrive(bar(ctl.cta_bar));
         // Warp-uniform outcome (warp collectives follow); for the epilogue warps
         // also uniform across the group, which meets at named barriers.
         const bool waited = __all_sync(0xffffffffu, mbar_wait(bar(ctl.cta_bar), cta_phase, abort_flag));
         cta_phase ^= 1;
         const int64_t u = waited ? (int64_t)ctl.tile[iter & 1] : total_tiles;
+        const bool redo = waited && ctl.redo[iter & 1] != 0;
         bool go = waited && u < total_tiles && !*abort_flag;
         if (warp >= 2) go = epi_sync_and(go);
         if (!go) break;
@@ -468,6 +494,12 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         const int64_t c_min = (q_begin + j0) / r;
         const int64_t c_max = (q_begin + j0 + nrows - 1) / r;
         const int ntiles = c_max > kB ? (int)((c_max + BT - 1) / BT) : 0;
+        // Estimate mode (sample first) when the sweep is long enough to need it;
+        // exact mode (ascending sweep, running threshold) otherwise and on a redo.
+        const int nsamp = (!redo && c_max > CAP) ? (ntiles + SAMPLE - 1) / SAMPLE : 0;
+        // Sample entries kept: about 2 k_B candidates expected over the whole sweep.
+        int kA = nsamp ? (int)((2LL * kB * nsamp * BT + c_max - 1) / c_max) : kB;
+        kA = max(kA, min(16, kB));
 
         if (warp == 0) {
             // ------------------------------------------------ TMA producer
@@ -488,7 +520,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                     mbar_expect_tx(fb, KT_BYTES);
                     for (int kh = 0; kh < 2; ++kh)
                         tma_load_2d(sK + stg * KT_BYTES + kh * (KT_BYTES / 2), &tm_k, fb, kh * 64,
-                                    krow0 + t * BT, pol_k);
+                                    krow0 + tile_at(t, nsamp) * BT, pol_k);
                     produced_last[stg] = round;
                 }
             }
@@ -523,16 +555,19 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
             const int ch = ew >> 2;           // which 128-column half of a TMEM half
             for (int q = et; q < QT; q += EPI_THREADS) {
                 ctl.tau[q] = q < nrows ? -INFINITY : INFINITY;  // rows past nq never enter
+                ctl.tau_est[q] = -INFINITY;
                 for (int sg = 0; sg < NSEG; ++sg) ctl.seg[q][sg] = 0;
                 ctl.cvis[q] = q < nrows ? (int)((q_begin + j0 + q) / r) : 0;
+                if (!redo) ctl.failed[q] = 0;
             }
             bool ok = epi_sync_and(true);
             const size_t slot0 = (size_t)blockIdx.x * QT;
             const uint32_t tlane = tmem + ((uint32_t)(qd * 32) << 16);
             int cnt_h[2] = {0, 0};  // this lane's query (h*64 + ch*32 + lane): fill of segment qd
             for (int t = 0; ok && t < ntiles; ++t, ++acc_iter) {
-                const int b = t * BT + qd * 32 + lane;
-                const bool masked = (int64_t)(t + 1) * BT > c_min;
+                const int tt = tile_at(t, nsamp);
+                const int b = tt * BT + qd * 32 + lane;
+                const bool masked = (int64_t)(tt + 1) * BT > c_min;
                 bool okt = true;
                 for (int h = 0; h < 2; ++h) {
                     const bool okh =
@@ -567,28 +602,32 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                 ctl.seg[ch * 32 + lane][qd] = cnt_h[0];
                 ctl.seg[64 + ch * 32 + lane][qd] = cnt_h[1];
                 if (!(ok = epi_sync_and(okt))) break;
-                bool changed = false;
+                // Sample phase (t < nsamp): keep the k_A best; at its last tile every
+                // buffer is cut to k_A and tau becomes the estimate tau_est. Afterwards:
+                // keep the k_B best on overflow.
+                const bool boundary = t + 1 == nsamp;
+                const int target = t < nsamp ? kA : kB;
                 for (int q = ew; q < QT; q += EPI_WARPS) {
                     int* sq = ctl.seg[q];
-                    if (max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32) {
-                        // Keep the k_B best and raise tau to the smallest kept score. (With
-                        // fewer than k_B entries, only rebalance the segments.)
-                        const int n = sq[0] + sq[1] + sq[2] + sq[3];
-                        const int kk = n < kB ? n : kB;
+                    const int n = sq[0] + sq[1] + sq[2] + sq[3];
+                    if (max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32 || (boundary && n > target)) {
+                        // Keep the best `target` and raise tau to the smallest kept score.
+                        // (With fewer entries, only rebalance the segments.)
+                        const int kk = n < target ? n : target;
                         const uint32_t tk = warp_keep_best(cand + (slot0 + q) * CAP, sq, kk, lane, ctl.hist[ew],
                                                            nullptr);
                         __syncwarp();
                         if (lane == 0) {
-                            if (kk == kB) ctl.tau[q] = key_to_float(tk);
+                            if (kk == target) ctl.tau[q] = key_to_float(tk);
                             const int per = (kk + NSEG - 1) / NSEG;
                             for (int sg = 0; sg < NSEG; ++sg) sq[sg] = max(0, min(per, kk - sg * per));
                         }
-                        changed = true;
                     }
+                    __syncwarp();
+                    if (boundary && lane == 0) ctl.tau_est[q] = ctl.tau[q];
                 }
                 __syncwarp();
                 if (!(ok = epi_sync_and(true))) break;
-                (void)changed;
                 cnt_h[0] = ctl.seg[ch * 32 + lane][qd];
                 cnt_h[1] = ctl.seg[64 + ch * 32 + lane][qd];
             }
@@ -606,8 +645,22 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                         if (lane == 0) nsel[orow] = kq;
                         continue;
                     }
+                    if (redo && !ctl.failed[q]) continue;  // written by the estimate pass
                     const int* sq = ctl.seg[q];
                     const int n = sq[0] + sq[1] + sq[2] + sq[3];
+                    if (nsamp > 0) {
+                        // Every entry above tau_est was admitted and kept; if at least k_q
+                        // of them exist, the exact top k_q is among the candidates.
+                        // Otherwise this query is redone in exact mode.
+                        const float te = ctl.tau_est[q];
+                        const int above = te == -INFINITY ? n
+                                                          : warp_count_above(cand + (slot0 + q) * CAP, sq, te, lane);
+                        if (above < kq) {
+                            if (lane == 0) ctl.failed[q] = 1;
+                            __syncwarp();
+                            continue;
+                        }
+                    }
                     const int m = n < kq ? n : kq;
                     if (m != kq && lane == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
                     warp_keep_best(cand + (slot0 + q) * CAP, sq, m, lane, ctl.hist[ew], scratch);
@@ -620,6 +673,16 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                     if (lane == 0) nsel[orow] = m;
                     __syncwarp();
                 }
+            }
+            // Next iteration: this tile again in exact mode if a query failed its
+            // check, otherwise the next tile from the queue.
+            bool mine_ok = true;
+            for (int q = ew; q < nrows; q += EPI_WARPS) mine_ok = mine_ok && !ctl.failed[q];
+            const bool all_ok = epi_sync_and(mine_ok || redo);
+            if (et == 0) {
+                const int nx = (iter + 1) & 1;
+                ctl.redo[nx] = all_ok ? 0 : 1;
+                ctl.tile[nx] = all_ok ? atomicAdd(tile_counter, 1) : (int)u;
             }
         }
     }

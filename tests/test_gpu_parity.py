@@ -427,3 +427,36 @@ def test_fused_topk_all_zero_scores(qsa):
     for i in range(0, n, 97):
         m = min(128, i // 4)
         assert gn[i] == m and np.array_equal(g[i, :m], np.arange(m)), i
+
+
+def test_fused_topk_unrepresentative_sample_is_redone_exactly(qsa):
+    """Make the estimate phase fail on purpose: blocks of every 16th 128-block
+    tile (the sweep's sample) get keys along a direction all queries share, so the
+    threshold estimated from them admits too few candidates elsewhere. The check
+    must catch it and the exact redo must give the oracle's selection."""
+    n = 32768 + 40
+    w = synth.Workload(name="t", n=n, K=2048, q_heads=8, kv_heads=2, base_seed=0xB9)
+    cfg, L = _layer(qsa, w, n)
+    _fill_caches(w, L, n)
+    c = torch.zeros(128, device="cuda")
+    c[64:] = torch.randn(64, generator=torch.Generator().manual_seed(3)).cuda()
+    c = c / c.norm()
+    blk = torch.arange(n // 4, device="cuda")
+    sample_blocks = blk[(blk // 128) % 16 == 0]
+    rows = (sample_blocks[:, None] * 4 + torch.arange(4, device="cuda")[None, :]).reshape(-1)
+    L.idx_k_cache[0, rows] = (24.0 * c).to(torch.bfloat16)
+    iq = dev_full(w, "idx_q", n).view(1, n, 4, 128)
+    iq = (iq.float() + 3.0 * c).to(torch.bfloat16).contiguous()
+    L.compress(0, n // 4)
+    sel = torch.empty(1, n, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(1, n, dtype=torch.int32, device="cuda")
+    qsa.qsa_topk_blocks(cfg, 1, iq, 0, n, L.pooled, n, None, 0, sel, nsel, L.workspace(qsa.OP_TOPK_BLOCKS, n))
+    torch.cuda.synchronize()
+    o = _oracle(w, cfg)
+    pooled = bits(L.pooled)[0]
+    iq_bits = bits(iq)[0].reshape(n, 4, 128)
+    g, gn = sel.cpu().numpy()[0], nsel.cpu().numpy()[0]
+    for i in [4200, 9000, 20001, 32767, n - 1]:
+        ref = o.row(i, iq_bits[i], pooled)
+        tol = score_tol(o.rotate_query(iq_bits[i], i), pooled, ref["scores"])
+        check_selection(g[i], gn[i], ref["scores"], tol, o.k_blocks, f"row {i}")
