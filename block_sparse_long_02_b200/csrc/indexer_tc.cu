@@ -49,6 +49,7 @@ constexpr int KMAX_FUSED = 512;        // largest k_B handled here
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = EPI_WARPS * 32;
 constexpr int THREADS = 64 + EPI_THREADS;
+static_assert(QT / EPI_WARPS <= 32, "one lane per query of a warp in the compaction check");
 constexpr int Q_BYTES = QT * kIdxHeads * 256;  // 131072
 constexpr int KT_BYTES = BT * 256;             // 32768
 constexpr uint64_t WAIT_NS = 10000000000ull;  // 10 s
@@ -124,6 +125,18 @@ __device__ __forceinline__ bool epi_sync_and(bool v) {
     return r != 0;
 }
 
+// Barrier over the 256 epilogue threads that counts the threads whose
+// predicate is true.
+__device__ __forceinline__ int epi_sync_count(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.u32 p, %1, 0;\n bar.red.popc.u32 %0, 1, 256, p;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return (int)r;
+}
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -191,9 +204,10 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 // ------------------------------------------------------- candidate compaction
 // Keeps the k best of the n = sum(segn) (k <= n <= CAP) entries (score bits,
 // block) of one query's segmented candidate buffer, ranked by (score desc,
-// block asc). The kept entries are either written back spread over the
-// segments (ceil(k/4) per segment, in no particular order) or, if out_idx is
-// given, their block indices are written to out_idx[0, k). Returns the
+// block asc). The kept entries are either written back round-robin over the
+// segments (entry p of the kept list to segment p % 4, slot p / 4; in no
+// particular order) or, if out_idx is given, their block indices are written
+// to out_idx[0, k). Returns the
 // order-preserving key of the smallest kept score. One warp; `hist` is its
 // 256-bin scratch.
 //
@@ -323,16 +337,13 @@ __device__ uint32_t warp_keep_best(uint2* qbuf, const int* segn, int k, int lane
     }
     int pos = incl - kc;
     __syncwarp();
-    const int per = (k + NSEG - 1) / NSEG;  // kept entries per segment after the rewrite
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         if ((keep >> j) & 1u) {
-            if (out_idx) {
+            if (out_idx)
                 out_idx[pos] = (int32_t)ix[j];
-            } else {
-                const int sg = pos / per;
-                qbuf[sg * SEG + (pos - sg * per)] = make_uint2(__float_as_uint(key_to_float(key[j])), ix[j]);
-            }
+            else
+                qbuf[(pos % NSEG) * SEG + pos / NSEG] = make_uint2(__float_as_uint(key_to_float(key[j])), ix[j]);
             ++pos;
         }
     }
@@ -387,23 +398,75 @@ __device__ __forceinline__ void score16(const uint32_t* v, int q0, int sub, int 
     cnt += add;
 }
 
-// Ascending bitonic sort of P (power of two, <= 512) ints in shared memory; one warp.
-__device__ void warp_sort(int32_t* a, int P, int lane) {
-    for (int k = 2; k <= P; k <<= 1) {
+// Sorts a[0, m) (m <= 32 R, shared memory, 16-byte aligned) ascending in
+// place, one warp: bitonic network over 32 R values held in registers, element
+// lane * R + r in register r of `lane` (strides below R stay in a lane, larger
+// ones are shuffles); slots past m are padded with INT_MAX and come out last.
+template <int R>
+__device__ void warp_sort_regs(int32_t* a, int m, int lane) {
+    int32_t v[R];
+    if constexpr (R >= 4) {
+#pragma unroll
+        for (int r = 0; r < R; r += 4) {
+            const int4 x = *reinterpret_cast<const int4*>(a + lane * R + r);
+            v[r] = x.x, v[r + 1] = x.y, v[r + 2] = x.z, v[r + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r) v[r] = a[lane * R + r];
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+        if (lane * R + r >= m) v[r] = 0x7fffffff;
+#pragma unroll
+    for (int k = 2; k <= 32 * R; k <<= 1) {
+#pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = lane; i < P; i += 32) {
-                const int x = i ^ j;
-                if (x > i) {
-                    const int32_t u = a[i], w = a[x];
-                    if ((u > w) == ((i & k) == 0)) {
-                        a[i] = w;
-                        a[x] = u;
+            if (j >= R) {
+                const int lj = j / R;
+                const bool lower = (lane & lj) == 0;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const bool up = ((lane * R + r) & k) == 0;
+                    const int32_t o = __shfl_xor_sync(0xffffffffu, v[r], lj);
+                    v[r] = (lower == up) ? min(v[r], o) : max(v[r], o);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    if ((r & j) == 0) {
+                        const bool up = ((lane * R + r) & k) == 0;
+                        const int32_t x = v[r], y = v[r | j];
+                        v[r] = up ? min(x, y) : max(x, y);
+                        v[r | j] = up ? max(x, y) : min(x, y);
                     }
                 }
             }
-            __syncwarp();
         }
     }
+    __syncwarp();
+    if constexpr (R >= 4) {
+#pragma unroll
+        for (int r = 0; r < R; r += 4)
+            *reinterpret_cast<int4*>(a + lane * R + r) = make_int4(v[r], v[r + 1], v[r + 2], v[r + 3]);
+    } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r) a[lane * R + r] = v[r];
+    }
+    __syncwarp();
+}
+
+__device__ void warp_sort(int32_t* a, int m, int kB, int lane) {
+    if (kB <= 32)
+        warp_sort_regs<1>(a, m, lane);
+    else if (kB <= 64)
+        warp_sort_regs<2>(a, m, lane);
+    else if (kB <= 128)
+        warp_sort_regs<4>(a, m, lane);
+    else if (kB <= 256)
+        warp_sort_regs<8>(a, m, lane);
+    else
+        warp_sort_regs<16>(a, m, lane);
 }
 
 // Sweep order of the pooled-key tiles: with nsamp > 0, first the sample tiles
@@ -597,35 +660,42 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                     if (lane == 0) mbar_arrive(bar(ctl.acc_empty[h]));
                     okt = okt && okh;
                 }
-                // All appends of tile t are in; shrink the buffers that could overflow
-                // (a tile adds at most 32 entries to a segment).
+                // All appends of tile t are in. A buffer is compacted when one of its
+                // segments could overflow on the next tile (a tile adds at most 32
+                // entries to a segment), and at the end of the sample phase; the
+                // check and the second barrier run only when some warp needs them.
                 ctl.seg[ch * 32 + lane][qd] = cnt_h[0];
                 ctl.seg[64 + ch * 32 + lane][qd] = cnt_h[1];
+                const bool boundary = t + 1 == nsamp;
+                const bool near_full = cnt_h[0] > SEG - 32 || cnt_h[1] > SEG - 32;
+                if (epi_sync_count(near_full || !okt) == 0 && !boundary) continue;
                 if (!(ok = epi_sync_and(okt))) break;
                 // Sample phase (t < nsamp): keep the k_A best; at its last tile every
                 // buffer is cut to k_A and tau becomes the estimate tau_est. Afterwards:
-                // keep the k_B best on overflow.
-                const bool boundary = t + 1 == nsamp;
+                // keep the k_B best on overflow. Lane l < 16 checks query ew + 8 l.
                 const int target = t < nsamp ? kA : kB;
-                for (int q = ew; q < QT; q += EPI_WARPS) {
+                bool need = false;
+                if (lane < QT / EPI_WARPS) {
+                    const int* sq = ctl.seg[ew + EPI_WARPS * lane];
+                    const int n = sq[0] + sq[1] + sq[2] + sq[3];
+                    need = max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32 || (boundary && n > target);
+                }
+                for (uint32_t todo = __ballot_sync(0xffffffffu, need); todo; todo &= todo - 1) {
+                    const int q = ew + EPI_WARPS * (__ffs(todo) - 1);
                     int* sq = ctl.seg[q];
                     const int n = sq[0] + sq[1] + sq[2] + sq[3];
-                    if (max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32 || (boundary && n > target)) {
-                        // Keep the best `target` and raise tau to the smallest kept score.
-                        // (With fewer entries, only rebalance the segments.)
-                        const int kk = n < target ? n : target;
-                        const uint32_t tk = warp_keep_best(cand + (slot0 + q) * CAP, sq, kk, lane, ctl.hist[ew],
-                                                           nullptr);
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (kk == target) ctl.tau[q] = key_to_float(tk);
-                            const int per = (kk + NSEG - 1) / NSEG;
-                            for (int sg = 0; sg < NSEG; ++sg) sq[sg] = max(0, min(per, kk - sg * per));
-                        }
+                    // Keep the best `target` and raise tau to the smallest kept score.
+                    // (With fewer entries, only rebalance the segments.)
+                    const int kk = n < target ? n : target;
+                    const uint32_t tk = warp_keep_best(cand + (slot0 + q) * CAP, sq, kk, lane, ctl.hist[ew], nullptr);
+                    if (lane == 0) {
+                        if (kk == target) ctl.tau[q] = key_to_float(tk);
+                        for (int sg = 0; sg < NSEG; ++sg) sq[sg] = (kk + NSEG - 1 - sg) / NSEG;
                     }
                     __syncwarp();
-                    if (boundary && lane == 0) ctl.tau_est[q] = ctl.tau[q];
                 }
+                if (boundary && lane < QT / EPI_WARPS)
+                    ctl.tau_est[ew + EPI_WARPS * lane] = ctl.tau[ew + EPI_WARPS * lane];
                 __syncwarp();
                 if (!(ok = epi_sync_and(true))) break;
                 cnt_h[0] = ctl.seg[ch * 32 + lane][qd];
@@ -664,11 +734,8 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                     const int m = n < kq ? n : kq;
                     if (m != kq && lane == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
                     warp_keep_best(cand + (slot0 + q) * CAP, sq, m, lane, ctl.hist[ew], scratch);
-                    int P = 1;
-                    while (P < m) P <<= 1;
-                    for (int k2 = m + lane; k2 < P; k2 += 32) scratch[k2] = 0x7fffffff;
                     __syncwarp();
-                    warp_sort(scratch, P, lane);
+                    warp_sort(scratch, m, kB, lane);
                     for (int k2 = lane; k2 < kB; k2 += 32) out[k2] = k2 < m ? scratch[k2] : -1;
                     if (lane == 0) nsel[orow] = m;
                     __syncwarp();
