@@ -63,12 +63,16 @@ struct Ctl {
     int redo[2];        // 1: repeat the tile in exact mode for the queries that failed
     float tau_est[QT];  // threshold estimated from the sample phase (-inf: none)
     uint8_t failed[QT]; // query's candidates did not prove the top-k in estimate mode
-    float tau[QT];
+    alignas(16) float tau[QT];
     int seg[QT][NSEG];  // entries in each segment of a query's candidate buffer
-    int cvis[QT];
-    uint32_t hist[EPI_WARPS][256];  // per-warp radix histogram of the compaction
+    alignas(16) int cvis[QT];
 };
-constexpr int SMEM = Q_BYTES + STAGES * KT_BYTES + (int)sizeof(Ctl) + 1024;
+// Per epilogue warp: 16 scores x 32 lanes of append staging, which is also
+// the warp's 256-bin radix histogram while it compacts.
+constexpr int STAGE_FLOATS = 16 * 32;
+constexpr int STAGE_BYTES = EPI_WARPS * STAGE_FLOATS * 4;
+constexpr int SMEM = Q_BYTES + STAGES * KT_BYTES + STAGE_BYTES + (int)sizeof(Ctl) + 1024;
+static_assert(SMEM <= 232448, "shared memory per CTA");
 
 // ------------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint64_t gtime() {
@@ -362,40 +366,66 @@ __device__ int warp_count_above(const uint2* qbuf, const int* segn, float thr, i
     return (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
 }
 
-// Scores of 16 queries x this lane's block from 64 accumulator words (4 heads
-// each) and the threshold test. Takers append to this warp's own segment of
-// each query's buffer: lane (sub*16 + qq) holds the segment fill of query qq in
-// `cnt`, so an append needs a shuffle, not an atomic.
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+    float2 c;
+    asm("{\n .reg .b64 ra, rb, rc;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+        " add.rn.f32x2 rc, ra, rb;\n mov.b64 {%0, %1}, rc;\n}\n"
+        : "=f"(c.x), "=f"(c.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return c;
+}
+
+// Scores of 16 queries (q0 .. q0 + 15) x this lane's block b from 64
+// accumulator words (4 heads each). The kernel works with twice the score,
+// 2 s = sum_h (x_h + |x_h|): every term is exactly 2 ReLU(x_h), so the order
+// of all scores (and ties) is that of s, and the additions run on the FMA
+// pipe. A score enters query q's candidate segment of this warp if
+// 2 s >= tau[q] (tau is kept in the same units) and, on the diagonal tile,
+// b < cvis[q]. Lanes that take anything stage their 16 scores in shared
+// memory and append them one at a time (segment fill by shared atomics).
 template <bool MASKED>
-__device__ __forceinline__ void score16(const uint32_t* v, int q0, int sub, int b, const Ctl& ctl,
-                                        uint2* seg_q0, int& cnt, int lane) {
+__device__ __forceinline__ void score16(const uint32_t* v, int q0, uint32_t b, Ctl& ctl, int qd,
+                                        uint2* cand_q0, float* stage, int lane) {
     float sc[16];
-    uint32_t takes = 0;
+    uint32_t m = 0;
 #pragma unroll
-    for (int qq = 0; qq < 16; ++qq) {
-        sc[qq] = fmaxf(__uint_as_float(v[4 * qq]), 0.f) + fmaxf(__uint_as_float(v[4 * qq + 1]), 0.f) +
-                 fmaxf(__uint_as_float(v[4 * qq + 2]), 0.f) + fmaxf(__uint_as_float(v[4 * qq + 3]), 0.f);
-        bool t = sc[qq] >= ctl.tau[q0 + qq];
-        if (MASKED) t = t && b < ctl.cvis[q0 + qq];
-        takes |= (uint32_t)t << qq;
-    }
-    const uint32_t any = __reduce_or_sync(0xffffffffu, takes);
-    if (!any) return;
-    const uint32_t lt = (1u << lane) - 1u;
-    // All positions come from the counters as they were on entry (independent
-    // shuffles); each lane then advances the counter of its own query once.
-    int add = 0;
+    for (int g = 0; g < 4; ++g) {
+        const float4 t4 = *reinterpret_cast<const float4*>(&ctl.tau[q0 + 4 * g]);
+        const float tq[4] = {t4.x, t4.y, t4.z, t4.w};
+        int cq[4] = {0, 0, 0, 0};
+        if (MASKED) {
+            const int4 c4 = *reinterpret_cast<const int4*>(&ctl.cvis[q0 + 4 * g]);
+            cq[0] = c4.x, cq[1] = c4.y, cq[2] = c4.z, cq[3] = c4.w;
+        }
 #pragma unroll
-    for (int qq = 0; qq < 16; ++qq) {
-        if ((any >> qq) & 1u) {
-            const bool mine = (takes >> qq) & 1u;
-            const uint32_t bal = __ballot_sync(0xffffffffu, mine);
-            const int pos = __shfl_sync(0xffffffffu, cnt, sub * 16 + qq) + __popc(bal & lt);
-            if (mine) seg_q0[(size_t)qq * CAP + pos] = make_uint2(__float_as_uint(sc[qq]), (uint32_t)b);
-            if (lane == sub * 16 + qq) add = __popc(bal);
+        for (int i = 0; i < 4; ++i) {
+            const int qq = 4 * g + i;
+            const float x0 = __uint_as_float(v[4 * qq]), x1 = __uint_as_float(v[4 * qq + 1]);
+            const float x2 = __uint_as_float(v[4 * qq + 2]), x3 = __uint_as_float(v[4 * qq + 3]);
+            const float2 p = add_f32x2(make_float2(x0 + fabsf(x0), x1 + fabsf(x1)),
+                                       make_float2(x2 + fabsf(x2), x3 + fabsf(x3)));
+            sc[qq] = p.x + p.y;
+            bool t = sc[qq] >= tq[i];
+            if (MASKED) t = t && (int)b < cq[i];
+            if (t) m |= 1u << qq;
         }
     }
-    cnt += add;
+    if (!__any_sync(0xffffffffu, m != 0)) return;
+    if (m) {
+        // 16-byte chunks of the lane's 16 scores, rotated so that 8 consecutive
+        // lanes hit distinct bank groups.
+        const int rot = (lane >> 1) & 3;
+        float4* st = reinterpret_cast<float4*>(stage) + lane * 4;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) st[g ^ rot] = make_float4(sc[4 * g], sc[4 * g + 1], sc[4 * g + 2], sc[4 * g + 3]);
+        do {
+            const int qq = __ffs(m) - 1;
+            m &= m - 1;
+            const float val = stage[lane * 16 + (((qq >> 2) ^ rot) << 2) + (qq & 3)];
+            const int pos = atomicAdd(&ctl.seg[q0 + qq][qd], 1);
+            cand_q0[(size_t)qq * CAP + pos] = make_uint2(__float_as_uint(val), b);
+        } while (m);
+    }
 }
 
 // Sorts a[0, m) (m <= 32 R, shared memory, 16-byte aligned) ascending in
@@ -490,7 +520,8 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
     uint8_t* base = smem_raw + (base_s - raw_s);
     const uint32_t sQ = base_s;
     const uint32_t sK = base_s + Q_BYTES;
-    Ctl& ctl = *reinterpret_cast<Ctl*>(base + Q_BYTES + STAGES * KT_BYTES);
+    float* stage_all = reinterpret_cast<float*>(base + Q_BYTES + STAGES * KT_BYTES);
+    Ctl& ctl = *reinterpret_cast<Ctl*>(base + Q_BYTES + STAGES * KT_BYTES + STAGE_BYTES);
     volatile int* abort_flag = &ctl.abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -626,80 +657,90 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
             bool ok = epi_sync_and(true);
             const size_t slot0 = (size_t)blockIdx.x * QT;
             const uint32_t tlane = tmem + ((uint32_t)(qd * 32) << 16);
-            int cnt_h[2] = {0, 0};  // this lane's query (h*64 + ch*32 + lane): fill of segment qd
+            float* stage = stage_all + ew * STAGE_FLOATS;
+            uint32_t* hist = reinterpret_cast<uint32_t*>(stage);
             for (int t = 0; ok && t < ntiles; ++t, ++acc_iter) {
                 const int tt = tile_at(t, nsamp);
-                const int b = tt * BT + qd * 32 + lane;
+                const uint32_t b = (uint32_t)(tt * BT + qd * 32 + lane);
                 const bool masked = (int64_t)(tt + 1) * BT > c_min;
                 bool okt = true;
                 for (int h = 0; h < 2; ++h) {
                     const bool okh =
                         __all_sync(0xffffffffu, mbar_wait(bar(ctl.acc_full[h]), acc_iter & 1u, abort_flag));
-                    if (okh) {
-                        tc_fence_after();
-                        const int q0 = h * 64 + ch * 32;
+                    if (okh) {  // warp-uniform
                         uint32_t v[128];
+                        tc_fence_after();
                         const uint32_t col = tlane + h * NHALF + ch * 128;
                         tmem_ld32(col, v);
                         tmem_ld32(col + 32, v + 32);
                         tmem_ld32(col + 64, v + 64);
                         tmem_ld32(col + 96, v + 96);
                         tmem_wait_ld();
-                        uint2* cq = cand + (slot0 + q0) * CAP + qd * SEG;
-                        int& cnt = cnt_h[h];
-                        if (masked) {
-                            score16<true>(v, q0, 0, b, ctl, cq, cnt, lane);
-                            score16<true>(v + 64, q0 + 16, 1, b, ctl, cq + (size_t)16 * CAP, cnt, lane);
-                        } else {
-                            score16<false>(v, q0, 0, b, ctl, cq, cnt, lane);
-                            score16<false>(v + 64, q0 + 16, 1, b, ctl, cq + (size_t)16 * CAP, cnt, lane);
-                        }
                         tc_fence_before();
+                        // The accumulators are in registers: hand the TMEM half back to
+                        // the MMA warp before scoring.
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(ctl.acc_empty[h]));
+                        const int q0 = h * 64 + ch * 32;
+                        uint2* cq = cand + (slot0 + q0) * CAP + qd * SEG;
+                        if (masked) {
+                            score16<true>(v, q0, b, ctl, qd, cq, stage, lane);
+                            score16<true>(v + 64, q0 + 16, b, ctl, qd, cq + (size_t)16 * CAP, stage, lane);
+                        } else {
+                            score16<false>(v, q0, b, ctl, qd, cq, stage, lane);
+                            score16<false>(v + 64, q0 + 16, b, ctl, qd, cq + (size_t)16 * CAP, stage, lane);
+                        }
+                    } else {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(ctl.acc_empty[h]));
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(ctl.acc_empty[h]));
                     okt = okt && okh;
                 }
                 // All appends of tile t are in. A buffer is compacted when one of its
                 // segments could overflow on the next tile (a tile adds at most 32
                 // entries to a segment), and at the end of the sample phase; the
-                // check and the second barrier run only when some warp needs them.
-                ctl.seg[ch * 32 + lane][qd] = cnt_h[0];
-                ctl.seg[64 + ch * 32 + lane][qd] = cnt_h[1];
+                // check and the compaction barriers run only when some warp needs them.
+                __syncwarp();
                 const bool boundary = t + 1 == nsamp;
-                const bool near_full = cnt_h[0] > SEG - 32 || cnt_h[1] > SEG - 32;
+                const bool near_full =
+                    ctl.seg[ch * 32 + lane][qd] > SEG - 32 || ctl.seg[64 + ch * 32 + lane][qd] > SEG - 32;
                 if (epi_sync_count(near_full || !okt) == 0 && !boundary) continue;
-                if (!(ok = epi_sync_and(okt))) break;
                 // Sample phase (t < nsamp): keep the k_A best; at its last tile every
                 // buffer is cut to k_A and tau becomes the estimate tau_est. Afterwards:
-                // keep the k_B best on overflow. Lane l < 16 checks query ew + 8 l.
+                // keep the k_B best on overflow. Every warp reads the same counts and
+                // takes every 8th query that needs it, so the work is spread evenly.
                 const int target = t < nsamp ? kA : kB;
-                bool need = false;
-                if (lane < QT / EPI_WARPS) {
-                    const int* sq = ctl.seg[ew + EPI_WARPS * lane];
+                uint32_t needm[QT / 32];
+#pragma unroll
+                for (int wd = 0; wd < QT / 32; ++wd) {
+                    const int* sq = ctl.seg[wd * 32 + lane];
                     const int n = sq[0] + sq[1] + sq[2] + sq[3];
-                    need = max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32 || (boundary && n > target);
+                    needm[wd] = __ballot_sync(
+                        0xffffffffu, max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32 || (boundary && n > target));
                 }
-                for (uint32_t todo = __ballot_sync(0xffffffffu, need); todo; todo &= todo - 1) {
-                    const int q = ew + EPI_WARPS * (__ffs(todo) - 1);
-                    int* sq = ctl.seg[q];
-                    const int n = sq[0] + sq[1] + sq[2] + sq[3];
-                    // Keep the best `target` and raise tau to the smallest kept score.
-                    // (With fewer entries, only rebalance the segments.)
-                    const int kk = n < target ? n : target;
-                    const uint32_t tk = warp_keep_best(cand + (slot0 + q) * CAP, sq, kk, lane, ctl.hist[ew], nullptr);
-                    if (lane == 0) {
-                        if (kk == target) ctl.tau[q] = key_to_float(tk);
-                        for (int sg = 0; sg < NSEG; ++sg) sq[sg] = (kk + NSEG - 1 - sg) / NSEG;
+                if (!(ok = epi_sync_and(okt))) break;  // counts read by all before any changes
+                int rank = 0;
+#pragma unroll 1
+                for (int wd = 0; wd < QT / 32; ++wd) {
+                    for (uint32_t msk = needm[wd]; msk; msk &= msk - 1) {
+                        if ((rank++ & (EPI_WARPS - 1)) != ew) continue;
+                        const int q = wd * 32 + __ffs(msk) - 1;
+                        int* sq = ctl.seg[q];
+                        const int n = sq[0] + sq[1] + sq[2] + sq[3];
+                        // Keep the best `target` and raise tau to the smallest kept score.
+                        // (With fewer entries, only rebalance the segments.)
+                        const int kk = n < target ? n : target;
+                        const uint32_t tk = warp_keep_best(cand + (slot0 + q) * CAP, sq, kk, lane, hist, nullptr);
+                        if (lane == 0) {
+                            if (kk == target) ctl.tau[q] = key_to_float(tk);
+                            for (int sg = 0; sg < NSEG; ++sg) sq[sg] = (kk + NSEG - 1 - sg) / NSEG;
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
+                if (!(ok = epi_sync_and(true))) break;
                 if (boundary && lane < QT / EPI_WARPS)
                     ctl.tau_est[ew + EPI_WARPS * lane] = ctl.tau[ew + EPI_WARPS * lane];
-                __syncwarp();
-                if (!(ok = epi_sync_and(true))) break;
-                cnt_h[0] = ctl.seg[ch * 32 + lane][qd];
-                cnt_h[1] = ctl.seg[64 + ch * 32 + lane][qd];
             }
             // Final selection and ascending output (the pooled-key ring is idle now:
             // use it as sort scratch, 2 KB per warp).
@@ -733,7 +774,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                     }
                     const int m = n < kq ? n : kq;
                     if (m != kq && lane == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
-                    warp_keep_best(cand + (slot0 + q) * CAP, sq, m, lane, ctl.hist[ew], scratch);
+                    warp_keep_best(cand + (slot0 + q) * CAP, sq, m, lane, hist, scratch);
                     __syncwarp();
                     warp_sort(scratch, m, kB, lane);
                     for (int k2 = lane; k2 < kB; k2 += 32) out[k2] = k2 < m ? scratch[k2] : -1;
