@@ -375,17 +375,33 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
     return c;
 }
 
+// An append whose slot is reserved but whose store is still to be issued.
+struct Pending {
+    uint2* p;  // nullptr: none
+    float val;
+    uint32_t b;
+};
+__device__ __forceinline__ void retire(Pending& x) {
+    if (x.p) *x.p = make_uint2(__float_as_uint(x.val), x.b);
+    x.p = nullptr;
+}
+
 // Scores of 16 queries (q0 .. q0 + 15) x this lane's block b from 64
 // accumulator words (4 heads each). The kernel works with twice the score,
 // 2 s = sum_h (x_h + |x_h|): every term is exactly 2 ReLU(x_h), so the order
 // of all scores (and ties) is that of s, and the additions run on the FMA
 // pipe. A score enters query q's candidate segment of this warp if
 // 2 s >= tau[q] (tau is kept in the same units) and, on the diagonal tile,
-// b < cvis[q]. Lanes that take anything stage their 16 scores in shared
-// memory and append them one at a time (segment fill by shared atomics).
+// b < cvis[q].
+//
+// Appends are software-pipelined: a lane's first two takes of a call reserve
+// their slots (shared atomic on the segment fill) and fetch their values from
+// the lane's staging row now, and their stores are issued by the next call,
+// after its scoring has covered those latencies (`retire`); further takes of
+// the same call (only while tau is still low) are stored at once.
 template <bool MASKED>
 __device__ __forceinline__ void score16(const uint32_t* v, int q0, uint32_t b, Ctl& ctl, int qd,
-                                        uint2* cand_q0, float* stage, int lane) {
+                                        uint2* cand_q0, float* stage, int lane, Pending& pa, Pending& pb) {
     float sc[16];
     uint32_t m = 0;
 #pragma unroll
@@ -410,7 +426,8 @@ __device__ __forceinline__ void score16(const uint32_t* v, int q0, uint32_t b, C
             if (t) m |= 1u << qq;
         }
     }
-    if (!__any_sync(0xffffffffu, m != 0)) return;
+    retire(pa);
+    retire(pb);
     if (m) {
         // 16-byte chunks of the lane's 16 scores, rotated so that 8 consecutive
         // lanes hit distinct bank groups.
@@ -418,13 +435,25 @@ __device__ __forceinline__ void score16(const uint32_t* v, int q0, uint32_t b, C
         float4* st = reinterpret_cast<float4*>(stage) + lane * 4;
 #pragma unroll
         for (int g = 0; g < 4; ++g) st[g ^ rot] = make_float4(sc[4 * g], sc[4 * g + 1], sc[4 * g + 2], sc[4 * g + 3]);
-        do {
-            const int qq = __ffs(m) - 1;
+        int qq = __ffs(m) - 1;
+        m &= m - 1;
+        pa.val = stage[lane * 16 + (((qq >> 2) ^ rot) << 2) + (qq & 3)];
+        pa.b = b;
+        pa.p = cand_q0 + (size_t)qq * CAP + atomicAdd(&ctl.seg[q0 + qq][qd], 1);
+        if (m) {
+            qq = __ffs(m) - 1;
             m &= m - 1;
-            const float val = stage[lane * 16 + (((qq >> 2) ^ rot) << 2) + (qq & 3)];
-            const int pos = atomicAdd(&ctl.seg[q0 + qq][qd], 1);
-            cand_q0[(size_t)qq * CAP + pos] = make_uint2(__float_as_uint(val), b);
-        } while (m);
+            pb.val = stage[lane * 16 + (((qq >> 2) ^ rot) << 2) + (qq & 3)];
+            pb.b = b;
+            pb.p = cand_q0 + (size_t)qq * CAP + atomicAdd(&ctl.seg[q0 + qq][qd], 1);
+            while (m) {
+                qq = __ffs(m) - 1;
+                m &= m - 1;
+                const float val = stage[lane * 16 + (((qq >> 2) ^ rot) << 2) + (qq & 3)];
+                const int pos = atomicAdd(&ctl.seg[q0 + qq][qd], 1);
+                cand_q0[(size_t)qq * CAP + pos] = make_uint2(__float_as_uint(val), b);
+            }
+        }
     }
 }
 
@@ -659,6 +688,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
             const uint32_t tlane = tmem + ((uint32_t)(qd * 32) << 16);
             float* stage = stage_all + ew * STAGE_FLOATS;
             uint32_t* hist = reinterpret_cast<uint32_t*>(stage);
+            Pending pa{nullptr, 0.f, 0u}, pb{nullptr, 0.f, 0u};
             for (int t = 0; ok && t < ntiles; ++t, ++acc_iter) {
                 const int tt = tile_at(t, nsamp);
                 const uint32_t b = (uint32_t)(tt * BT + qd * 32 + lane);
@@ -684,11 +714,11 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                         const int q0 = h * 64 + ch * 32;
                         uint2* cq = cand + (slot0 + q0) * CAP + qd * SEG;
                         if (masked) {
-                            score16<true>(v, q0, b, ctl, qd, cq, stage, lane);
-                            score16<true>(v + 64, q0 + 16, b, ctl, qd, cq + (size_t)16 * CAP, stage, lane);
+                            score16<true>(v, q0, b, ctl, qd, cq, stage, lane, pa, pb);
+                            score16<true>(v + 64, q0 + 16, b, ctl, qd, cq + (size_t)16 * CAP, stage, lane, pa, pb);
                         } else {
-                            score16<false>(v, q0, b, ctl, qd, cq, stage, lane);
-                            score16<false>(v + 64, q0 + 16, b, ctl, qd, cq + (size_t)16 * CAP, stage, lane);
+                            score16<false>(v, q0, b, ctl, qd, cq, stage, lane, pa, pb);
+                            score16<false>(v + 64, q0 + 16, b, ctl, qd, cq + (size_t)16 * CAP, stage, lane, pa, pb);
                         }
                     } else {
                         __syncwarp();
@@ -705,18 +735,30 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                 const bool near_full =
                     ctl.seg[ch * 32 + lane][qd] > SEG - 32 || ctl.seg[64 + ch * 32 + lane][qd] > SEG - 32;
                 if (epi_sync_count(near_full || !okt) == 0 && !boundary) continue;
+                retire(pa);  // compaction reads every segment: all stores first
+                retire(pb);
                 // Sample phase (t < nsamp): keep the k_A best; at its last tile every
                 // buffer is cut to k_A and tau becomes the estimate tau_est. Afterwards:
                 // keep the k_B best on overflow. Every warp reads the same counts and
-                // takes every 8th query that needs it, so the work is spread evenly.
+                // takes every 8th query of the list, so the work is spread evenly; the
+                // list is topped up to a multiple of 8 with queries that are close to
+                // their own trigger (those warps would otherwise wait at the barrier).
                 const int target = t < nsamp ? kA : kB;
-                uint32_t needm[QT / 32];
+                uint32_t needm[QT / 32], optm[QT / 32];
+                int fill = 0;
 #pragma unroll
                 for (int wd = 0; wd < QT / 32; ++wd) {
                     const int* sq = ctl.seg[wd * 32 + lane];
                     const int n = sq[0] + sq[1] + sq[2] + sq[3];
-                    needm[wd] = __ballot_sync(
-                        0xffffffffu, max(max(sq[0], sq[1]), max(sq[2], sq[3])) > SEG - 32 || (boundary && n > target));
+                    const int mx = max(max(sq[0], sq[1]), max(sq[2], sq[3]));
+                    needm[wd] = __ballot_sync(0xffffffffu, mx > SEG - 32 || (boundary && n > target));
+                    optm[wd] = __ballot_sync(0xffffffffu, mx > SEG - 96 && n > target + 64) & ~needm[wd];
+                    fill -= __popc(needm[wd]);
+                }
+                fill &= EPI_WARPS - 1;
+#pragma unroll
+                for (int wd = 0; wd < QT / 32; ++wd) {
+                    for (uint32_t o = optm[wd]; fill > 0 && o; o &= o - 1, --fill) needm[wd] |= o & (0u - o);
                 }
                 if (!(ok = epi_sync_and(okt))) break;  // counts read by all before any changes
                 int rank = 0;
@@ -742,6 +784,10 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                 if (boundary && lane < QT / EPI_WARPS)
                     ctl.tau_est[ew + EPI_WARPS * lane] = ctl.tau[ew + EPI_WARPS * lane];
             }
+            // The last reserved appends, then every warp's stores before the reads.
+            retire(pa);
+            retire(pb);
+            if (ok) ok = epi_sync_and(true);
             // Final selection and ascending output (the pooled-key ring is idle now:
             // use it as sort scratch, 2 KB per warp).
             if (ok) {
