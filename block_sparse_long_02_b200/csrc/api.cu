@@ -123,20 +123,23 @@ TopkWs topk_layout(const qsa::LayerDims& L, int batch, int64_t cap, int64_t nq) 
 }
 
 struct DecodeWs {
-    size_t qrot, scores, sel, nsel, part, hist, counters, winners, cand, total;
+    size_t scores, sel, nsel, part, hist, counters, winners, cand, total;
 };
 
 DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
+    // The selection state (histograms, counters) comes first, right after the
+    // status header: it must be zero when a step starts, and every step leaves
+    // it zero.
     DecodeWs w;
     const int S = qsa::decode_attention_splits(L);
-    w.qrot = qsa::kWsHeader;
-    w.scores = w.qrot + align_up((size_t)batch * qsa::kIdxHeads * qsa::kIdxDim * 2);
+    w.hist = qsa::kWsHeader;
+    w.counters = w.hist + align_up((size_t)batch * 2048 * 4);
+    w.scores = w.counters + align_up((size_t)batch * 4 * 4);
+    // (w.scores == qsa::decode_state_bytes(batch))
     w.sel = w.scores + align_up((size_t)batch * std::max<int64_t>(1, cap / L.r) * 4);
     w.nsel = w.sel + align_up((size_t)batch * L.kB * 4);
     w.part = w.nsel + align_up((size_t)batch * 4);
-    w.hist = w.part + align_up((size_t)batch * L.q_heads * S * 132 * 4);
-    w.counters = w.hist + align_up((size_t)batch * 2048 * 4);
-    w.winners = w.counters + align_up((size_t)batch * 4 * 4);
+    w.winners = w.part + align_up((size_t)batch * L.q_heads * S * 132 * 4);
     w.cand = w.winners + align_up((size_t)batch * L.kB * 4);
     w.total = w.cand + align_up((size_t)batch * qsa::kDecodeCand * 8);
     return w;
@@ -324,7 +327,6 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     TRY(check_ws(ws, ws_bytes, w.total));
     char* base = (char*)ws;
     int32_t* status = reinterpret_cast<int32_t*>(base);
-    uint16_t* qrot = reinterpret_cast<uint16_t*>(base + w.qrot);
     float* scores = reinterpret_cast<float*>(base + w.scores);
     int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + w.sel);
     int32_t* nsel = nsel_out ? nsel_out : reinterpret_cast<int32_t*>(base + w.nsel);
@@ -335,10 +337,9 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     sw.winners = reinterpret_cast<int32_t*>(base + w.winners);
     sw.cand = reinterpret_cast<uint2*>(base + w.cand);
     cudaStream_t st = (cudaStream_t)stream;
-    TRY(cuda_check(qsa::launch_decode_prepare(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache,
-                                              idx_k_cache, pooled, cap, rms_w, qrot, sw, status, st),
-                   "decode prepare"));
-    TRY(cuda_check(qsa::launch_decode_scores(L, batch, pos, qrot, pooled, cap, scores, sw, st), "decode scores"));
+    TRY(cuda_check(qsa::launch_decode_score(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
+                                            pooled, cap, rms_w, scores, sw, status, st),
+                   "decode score"));
     TRY(cuda_check(qsa::launch_decode_select(L, batch, pos, cap, scores, sw, sel, nsel, st), "decode select"));
     return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel,
                                                    nsel, part, out, st),
@@ -357,3 +358,9 @@ qsa_status qsa_workspace_status(void* ws, qsa_stream stream, int32_t* status) {
 }
 
 }  // extern "C"
+
+namespace qsa {
+size_t decode_state_bytes(int batch) {
+    return kWsHeader + align_up((size_t)batch * 2048 * 4) + align_up((size_t)batch * 4 * 4);
+}
+}  // namespace qsa

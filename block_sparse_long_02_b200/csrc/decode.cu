@@ -26,47 +26,8 @@ namespace {
 constexpr int SC_THREADS = 512;  // score and select CTAs
 constexpr int SC_WARPS = SC_THREADS / 32;
 
-__global__ void __launch_bounds__(128) decode_prepare_kernel(
-    const int64_t* __restrict__ pos, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
-    const uint16_t* __restrict__ idx_q, const uint16_t* __restrict__ idx_k, uint16_t* __restrict__ kc,
-    uint16_t* __restrict__ vc, uint16_t* __restrict__ idx_k_cache, uint16_t* __restrict__ pooled,
-    int64_t cap, const float* __restrict__ rms_w, int kv_heads, int r, double eps, RopeTable rt,
-    uint16_t* __restrict__ qrot, DecodeSelWs sw, int32_t* __restrict__ status) {
-    const int s = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // Selection state of this step starts empty.
-    for (int b = tid; b < 2048; b += blockDim.x) sw.hist[(size_t)s * 2048 + b] = 0u;
-    if (tid < 4) sw.counters[s * 4 + tid] = 0;
-    const int64_t p = pos[s];
-    if (p < 0 || p >= cap) {
-        if (tid == 0) flag_status(status, 4 /* QSA_ERR_CAPACITY */);
-        return;
-    }
-    const int row16 = kv_heads * kHeadDim / 8;  // 16-byte chunks per kv row
-    const uint4* ks = reinterpret_cast<const uint4*>(k + (size_t)s * kv_heads * kHeadDim);
-    const uint4* vs = reinterpret_cast<const uint4*>(v + (size_t)s * kv_heads * kHeadDim);
-    uint4* kd = reinterpret_cast<uint4*>(kc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
-    uint4* vd = reinterpret_cast<uint4*>(vc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
-    for (int c = tid; c < row16; c += blockDim.x) {
-        kd[c] = ks[c];
-        vd[c] = vs[c];
-    }
-    if (tid < kIdxDim / 8)
-        reinterpret_cast<uint4*>(idx_k_cache + ((size_t)s * cap + p) * kIdxDim)[tid] =
-            reinterpret_cast<const uint4*>(idx_k + (size_t)s * kIdxDim)[tid];
-    // a3': the new indexer query, rotated at its own position.
-    rotate_head_warp(idx_q + ((size_t)s * kIdxHeads + warp) * kIdxDim, p, rt,
-                     qrot + ((size_t)s * kIdxHeads + warp) * kIdxDim, lane);
-    // a8: the token closes its block -> pool it for the following steps. The
-    // block's last raw key is read from the input (the append above is by
-    // other threads of this CTA).
-    if (warp == 0 && (p + 1) % r == 0) {
-        const int64_t b = p / r;
-        pool_block_warp(idx_k_cache + ((size_t)s * cap + (size_t)b * r) * kIdxDim,
-                        idx_k + (size_t)s * kIdxDim, r, rms_w, eps, b * r, rt,
-                        pooled + ((size_t)s * (cap / r) + b) * kIdxDim, lane);
-    }
-}
+constexpr int DS_THREADS = 256;  // fused score CTAs
+constexpr int DS_WARPS = DS_THREADS / 32;
 
 // Blocks [lo, hi) of a sequence's nvis visible blocks handled by CTA x of X.
 __device__ __forceinline__ void cta_range(int64_t nvis, int x, int X, int64_t& lo, int64_t& hi) {
@@ -75,93 +36,135 @@ __device__ __forceinline__ void cta_range(int64_t nvis, int x, int X, int64_t& l
     hi = min(nvis, lo + chunk);
 }
 
-__device__ __forceinline__ void load4(const uint16_t* ks, int64_t b0, int64_t hi, int hl, uint4 (&w)[4]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t b = b0 + i;
-        w[i] = b < hi ? *reinterpret_cast<const uint4*>(ks + (size_t)b * kIdxDim + hl * 8)
-                      : make_uint4(0u, 0u, 0u, 0u);
-    }
-}
-
-__global__ void __launch_bounds__(SC_THREADS) decode_scores_kernel(
-    const int64_t* __restrict__ pos, const uint16_t* __restrict__ qrot,
-    const uint16_t* __restrict__ pooled, int64_t cap, int r, float* __restrict__ scores,
-    uint32_t* __restrict__ hist_g) {
+// One decode step's cache update, query rotation and score stream, fused.
+//
+// CTA (0, s) appends the new token's K, V and raw indexer key to the caches
+// and, when the token closes its block, pools that block for later steps (a8;
+// the block is not visible at this position, so no CTA of this step reads
+// it). Every CTA rotates the new indexer query itself (a3', 4 warps, fp64)
+// and scores its slice of the visible pooled keys (a4) on the tensor cores:
+// mma.sync m16n8k16 with A = 16 pooled keys x 16 dims and B = 16 dims x
+// (4 heads + 4 zero columns). The 128 dims are taken in a fixed permutation
+// (the same for keys and query, so every dot product is unchanged) chosen so
+// that lane (g, t) of a warp reads its A fragments for all 8 k-steps of rows
+// g and g + 8 with four 16-byte loads per row: chunk i of lane t is bytes
+// [64 i + 16 t, +16) of the row, and k-step j uses its pairs 2 (j % 2) and
+// 2 (j % 2) + 1 of chunk j / 2 as the low and high column pairs. The ReLU
+// head sum takes one shuffle; the scores go to `scores` and their top 11 key
+// bits to the sequence's histogram (zeroed by the selection after use).
+__global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
+    const int64_t* __restrict__ pos, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+    const uint16_t* __restrict__ idx_q, const uint16_t* __restrict__ idx_k, uint16_t* __restrict__ kc,
+    uint16_t* __restrict__ vc, uint16_t* __restrict__ idx_k_cache, uint16_t* __restrict__ pooled,
+    int64_t cap, const float* __restrict__ rms_w, int kv_heads, int r, int kB, double eps, RopeTable rt,
+    float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status) {
     __shared__ uint32_t hist[2048];
+    __shared__ __align__(16) uint16_t qs[kIdxHeads * kIdxDim];
     const int s = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int hl = lane & 15, half = lane >> 4;
     const int64_t p = pos[s];
-    if (p < 0 || p >= cap) return;
+    if (p < 0 || p >= cap) {
+        if (blockIdx.x == 0 && tid == 0) flag_status(status, 4 /* QSA_ERR_CAPACITY */);
+        return;
+    }
+    if (blockIdx.x == 0) {
+        const int row16 = kv_heads * kHeadDim / 8;  // 16-byte chunks per kv row
+        const uint4* ks = reinterpret_cast<const uint4*>(k + (size_t)s * kv_heads * kHeadDim);
+        const uint4* vs = reinterpret_cast<const uint4*>(v + (size_t)s * kv_heads * kHeadDim);
+        uint4* kd = reinterpret_cast<uint4*>(kc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
+        uint4* vd = reinterpret_cast<uint4*>(vc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
+        for (int c = tid; c < row16; c += DS_THREADS) {
+            kd[c] = ks[c];
+            vd[c] = vs[c];
+        }
+        if (tid < kIdxDim / 8)
+            reinterpret_cast<uint4*>(idx_k_cache + ((size_t)s * cap + p) * kIdxDim)[tid] =
+                reinterpret_cast<const uint4*>(idx_k + (size_t)s * kIdxDim)[tid];
+        // The block's last raw key is read from the input (its cache row is
+        // written by another thread of this CTA).
+        if (warp == kIdxHeads && (p + 1) % r == 0) {
+            const int64_t b = p / r;
+            pool_block_warp(idx_k_cache + ((size_t)s * cap + (size_t)b * r) * kIdxDim,
+                            idx_k + (size_t)s * kIdxDim, r, rms_w, eps, b * r, rt,
+                            pooled + ((size_t)s * (cap / r) + b) * kIdxDim, lane);
+        }
+    }
     const int64_t pcap = cap / r;
+    if (p / r <= kB) return;  // every visible block is selected: no scores needed
     int64_t lo, hi;
     cta_range(p / r, blockIdx.x, gridDim.x, lo, hi);
     if (lo >= hi) return;
-    for (int b = tid; b < 2048; b += SC_THREADS) hist[b] = 0u;
-    // This lane's 8 dims of the 4 rotated query heads.
-    float qv[kIdxHeads][8];
-#pragma unroll
-    for (int h = 0; h < kIdxHeads; ++h) {
-        const uint4 w = *reinterpret_cast<const uint4*>(qrot + ((size_t)s * kIdxHeads + h) * kIdxDim + hl * 8);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            qv[h][2 * e] = bf16_lo(ws[e]);
-            qv[h][2 * e + 1] = bf16_hi(ws[e]);
-        }
-    }
+    if (warp < kIdxHeads)
+        rotate_head_warp(idx_q + ((size_t)s * kIdxHeads + warp) * kIdxDim, p, rt, qs + warp * kIdxDim, lane);
+    for (int b = tid; b < 2048; b += DS_THREADS) hist[b] = 0u;
     __syncthreads();
-    const uint16_t* ks = pooled + (size_t)s * pcap * kIdxDim;
+    const int g = lane >> 2, t = lane & 3;
+    // B fragments: column g (head g, zero for g >= 4), k-step j.
+    uint32_t bq0[8], bq1[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int d = 32 * (j >> 1) + 8 * t + 4 * (j & 1);
+        bq0[j] = g < kIdxHeads ? *reinterpret_cast<const uint32_t*>(qs + g * kIdxDim + d) : 0u;
+        bq1[j] = g < kIdxHeads ? *reinterpret_cast<const uint32_t*>(qs + g * kIdxDim + d + 2) : 0u;
+    }
+    const uint16_t* keys = pooled + (size_t)s * pcap * kIdxDim;
     float* dst = scores + (size_t)s * pcap;
-    // Warp step: 8 blocks, half-warp `half` takes blocks b0 + 4*half + (0..3).
-    const int64_t stride = (int64_t)SC_WARPS * 8;
-    int64_t b0 = lo + (int64_t)warp * 8;
-    uint4 cur[4];
-    load4(ks, b0 + half * 4, hi, hl, cur);
-    for (; b0 < hi; b0 += stride) {
-        uint4 nxt[4];
-        load4(ks, b0 + stride + half * 4, hi, hl, nxt);  // prefetch the next step
-        float v[16];  // v[4*i + h]: block i, head h (partial over this lane's 8 dims)
+    auto load = [&](int64_t base, uint4 (&ra)[4], uint4 (&rb)[4]) {
+        const int64_t b0 = base + g, b1 = b0 + 8;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t ws[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+            ra[i] = b0 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b0 * kIdxDim + 32 * i + 8 * t))
+                            : make_uint4(0u, 0u, 0u, 0u);
+            rb[i] = b1 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b1 * kIdxDim + 32 * i + 8 * t))
+                            : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    const int64_t step = 16 * DS_WARPS;
+    int64_t base = lo + 16 * warp;
+    uint4 ca[4], cb[4];
+    load(base, ca, cb);
+    for (; base < hi; base += step) {
+        uint4 na[4], nb[4];
+        load(base + step, na, nb);  // the next group, in flight during this one
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int h = 0; h < kIdxHeads; ++h) {
-                float a = 0.f;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    a = fmaf(qv[h][2 * e], bf16_lo(ws[e]), a);
-                    a = fmaf(qv[h][2 * e + 1], bf16_hi(ws[e]), a);
-                }
-                v[4 * i + h] = a;
+        for (int i = 0; i < 4; ++i) {
+            mma_bf16_16816(c, ca[i].x, cb[i].x, ca[i].y, cb[i].y, bq0[2 * i], bq1[2 * i]);
+            mma_bf16_16816(c, ca[i].z, cb[i].z, ca[i].w, cb[i].w, bq0[2 * i + 1], bq1[2 * i + 1]);
+        }
+        // Lane t = 0 holds heads 0, 1 and lane t = 1 heads 2, 3 of rows g, g + 8.
+        float sa = fmaxf(c[0], 0.f) + fmaxf(c[1], 0.f);
+        float sb = fmaxf(c[2], 0.f) + fmaxf(c[3], 0.f);
+        sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+        sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+        if (t == 0) {
+            const int64_t b0 = base + g, b1 = b0 + 8;
+            if (b0 < hi) {
+                dst[b0] = sa;
+                atomicAdd(&hist[float_key(sa) >> 21], 1u);
+            }
+            if (b1 < hi) {
+                dst[b1] = sb;
+                atomicAdd(&hist[float_key(sb) >> 21], 1u);
             }
         }
-        // Transpose reduction over the 16 lanes: lane hl ends with sum index hl.
 #pragma unroll
-        for (int m = 8, n = 8; m >= 1; m >>= 1, n >>= 1) {
-            const bool up = (hl & m) != 0;
-#pragma unroll
-            for (int j = 0; j < n; ++j) {
-                const float send = up ? v[j] : v[j + n];
-                const float keep = up ? v[j + n] : v[j];
-                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-            }
+        for (int i = 0; i < 4; ++i) {
+            ca[i] = na[i];
+            cb[i] = nb[i];
         }
-        float sc = fmaxf(v[0], 0.f);  // block hl >> 2, head hl & 3
-        sc += __shfl_xor_sync(0xffffffffu, sc, 1);
-        sc += __shfl_xor_sync(0xffffffffu, sc, 2);
-        const int64_t b = b0 + half * 4 + (hl >> 2);
-        if ((hl & 3) == 0 && b < hi) {
-            dst[b] = sc;
-            atomicAdd(&hist[float_key(sc) >> 21], 1u);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
     }
     __syncthreads();
-    for (int b = tid; b < 2048; b += SC_THREADS)
+    for (int b = tid; b < 2048; b += DS_THREADS)
         if (hist[b]) atomicAdd(&hist_g[(size_t)s * 2048 + b], hist[b]);
+}
+
+// The sequence's histogram and counters back to zero for the next step (the
+// score kernel only adds to them). Called by the last CTA, after every CTA
+// of the sequence has read them.
+__device__ __forceinline__ void reset_state(DecodeSelWs& sw, int s) {
+    for (int b = threadIdx.x; b < 2048; b += blockDim.x) sw.hist[(size_t)s * 2048 + b] = 0u;
+    if (threadIdx.x < 4) sw.counters[s * 4 + threadIdx.x] = 0;
 }
 
 // Block-aggregated append: the CTA's flagged entries get consecutive slots of a
@@ -228,6 +231,7 @@ __global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
     if (n_win != (int)(kB - need1) || nc > CAND || nc > kDecodeCand) {
         // Candidates overflow (e.g. thousands of equal scores): exact pick from the row.
         select_row(sm, row, nvis, kB, out, nsel + s);
+        reset_state(sw, s);
         return;
     }
     for (int k2 = tid; k2 < n_win; k2 += SC_THREADS) sm.out[k2] = __ldcg(winners + k2);
@@ -238,6 +242,8 @@ __global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
     }
     if (tid == 0) sm.n_out = n_win;
     __syncthreads();
+    __syncthreads();  // counters read by every thread before the reset
+    reset_state(sw, s);
     finish_from_candidates(sm, nc, b1, need1, kB, out);
     if (tid == 0) nsel[s] = kB;
 }
@@ -251,25 +257,22 @@ int decode_select_ctas(int batch) {
     return std::max(1, 2 * sms / std::max(batch, 1));
 }
 
-cudaError_t launch_decode_prepare(const LayerDims& L, int batch, const int64_t* pos,
-                                  const uint16_t* k, const uint16_t* v, const uint16_t* idx_q,
-                                  const uint16_t* idx_k, uint16_t* kc, uint16_t* vc,
-                                  uint16_t* idx_k_cache, uint16_t* pooled, int64_t cap,
-                                  const float* rms_w, uint16_t* qrot, DecodeSelWs sw,
-                                  int32_t* status, cudaStream_t st) {
-    note_launch();
-    decode_prepare_kernel<<<batch, 128, 0, st>>>(pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache,
-                                                 pooled, cap, rms_w, L.kv_heads, L.r, L.rms_eps,
-                                                 L.rope, qrot, sw, status);
-    return cudaGetLastError();
+int decode_score_ctas(int batch) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return std::max(1, 4 * sms / std::max(batch, 1));
 }
 
-cudaError_t launch_decode_scores(const LayerDims& L, int batch, const int64_t* pos,
-                                 const uint16_t* qrot, const uint16_t* pooled, int64_t cap,
-                                 float* scores, DecodeSelWs sw, cudaStream_t st) {
+cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* pos, const uint16_t* k,
+                                const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
+                                uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,
+                                int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
+                                int32_t* status, cudaStream_t st) {
     note_launch();
-    decode_scores_kernel<<<dim3((unsigned)decode_select_ctas(batch), (unsigned)batch), SC_THREADS, 0, st>>>(
-        pos, qrot, pooled, cap, L.r, scores, sw.hist);
+    decode_score_kernel<<<dim3((unsigned)decode_score_ctas(batch), (unsigned)batch), DS_THREADS, 0, st>>>(
+        pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps,
+        L.rope, scores, sw.hist, status);
     return cudaGetLastError();
 }
 

@@ -72,15 +72,15 @@ struct DecodeSelWs {
     uint2* cand;        // [batch][kDecodeCand] (key, block)
 };
 int decode_select_ctas(int batch);
-cudaError_t launch_decode_prepare(const LayerDims& L, int batch, const int64_t* pos,
-                                  const uint16_t* k, const uint16_t* v, const uint16_t* idx_q,
-                                  const uint16_t* idx_k, uint16_t* kc, uint16_t* vc,
-                                  uint16_t* idx_k_cache, uint16_t* pooled, int64_t cap,
-                                  const float* rms_w, uint16_t* qrot, DecodeSelWs sw,
-                                  int32_t* status, cudaStream_t st);
-cudaError_t launch_decode_scores(const LayerDims& L, int batch, const int64_t* pos,
-                                 const uint16_t* qrot, const uint16_t* pooled, int64_t cap,
-                                 float* scores, DecodeSelWs sw, cudaStream_t st);
+// Bytes at the start of a decode workspace (status header, histograms,
+// counters) that must be zero when a decode step starts; each step leaves
+// them zero.
+size_t decode_state_bytes(int batch);
+cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* pos, const uint16_t* k,
+                                const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
+                                uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,
+                                int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
+                                int32_t* status, cudaStream_t st);
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
                                  const float* scores, DecodeSelWs sw, int32_t* sel, int32_t* nsel,
                                  cudaStream_t st);

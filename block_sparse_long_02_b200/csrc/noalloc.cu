@@ -71,8 +71,9 @@ extern "C" qsa_status qsa_decode_step_noalloc(const qsa_config* cfg, int32_t bat
     if (e != cudaSuccess)
         return (qsa_status)qsa::report_error(QSA_ERR_CUDA, "qsa_decode_step_noalloc set-up: %s",
                                              cudaGetErrorString(e));
-    // The status header must start at zero for every call.
-    e = cudaMemsetAsync(ws, 0, qsa::kWsHeader, (cudaStream_t)stream);
+    // The status header and the selection state must start at zero; the array
+    // may hold another batch size's layout from an earlier call.
+    e = cudaMemsetAsync(ws, 0, qsa::decode_state_bytes(batch), (cudaStream_t)stream);
     if (e != cudaSuccess)
         return (qsa_status)qsa::report_error(QSA_ERR_CUDA, "qsa_decode_step_noalloc: %s",
                                              cudaGetErrorString(e));

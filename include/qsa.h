@@ -25,7 +25,9 @@
  *   - The library never allocates device memory: scratch comes from a caller
  *     workspace sized by qsa_workspace_size(). The first 256 bytes of a
  *     workspace hold a device status word and must be zero before first use
- *     (qsa_workspace_status reads and re-clears it).
+ *     (qsa_workspace_status reads and re-clears it). A decode-step workspace
+ *     must be all zero before its first use, and again whenever batch or cap
+ *     change; each step leaves it ready for the next.
  *   - No exceptions cross the ABI; qsa_last_error() returns a thread-local
  *     message for the last non-OK status of the calling thread.
  *   - Positions are 0-based. Query i sees complete blocks b < floor(i/r) and
