@@ -167,17 +167,27 @@ __device__ __forceinline__ void reset_state(DecodeSelWs& sw, int s) {
     if (threadIdx.x < 4) sw.counters[s * 4 + threadIdx.x] = 0;
 }
 
-// Block-aggregated append: the CTA's flagged entries get consecutive slots of a
-// per-sequence global list (one atomic per CTA round). Returns this thread's
-// slot or -1. All threads must call it.
-__device__ __forceinline__ int cta_append(SelSmem& sm, bool flag, int32_t* counter, int* base_slot) {
-    uint32_t pre;
-    const uint32_t tot = cta_scan(sm, flag, pre);
-    if (threadIdx.x == 0) *base_slot = tot ? atomicAdd(counter, (int)tot) : 0;
+// Exclusive prefix over the CTA (thread order) of a per-thread packed count;
+// returns the CTA total. All threads must call it.
+__device__ __forceinline__ uint32_t cta_prefix(SelSmem& sm, uint32_t v, uint32_t& prefix) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    if (lane == 31) sm.wsum[w] = inc;
     __syncthreads();
-    const int slot = flag ? *base_slot + (int)pre : -1;
+    uint32_t base = 0, total = 0;
+    for (int k = 0; k < NW; ++k) {
+        const uint32_t x = sm.wsum[k];
+        if (k < w) base += x;
+        total += x;
+    }
     __syncthreads();
-    return slot;
+    prefix = base + inc - v;
+    return total;
 }
 
 __global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
@@ -185,7 +195,8 @@ __global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
     DecodeSelWs sw, int32_t* __restrict__ sel, int32_t* __restrict__ nsel) {
     extern __shared__ __align__(16) uint8_t raw[];
     SelSmem& sm = *reinterpret_cast<SelSmem*>(raw);
-    __shared__ int base_slot, last;
+    __shared__ unsigned long long slot_base;  // (candidates << 32) | winners before this round
+    __shared__ int last;
     const int s = blockIdx.y;
     const int tid = threadIdx.x;
     const int64_t p = pos[s];
@@ -200,24 +211,53 @@ __global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
     }
     const float* row = scores + (size_t)s * (cap / r);
     // Threshold digit from the sequence's histogram.
-    for (int b = tid; b < 2048; b += SC_THREADS) sm.hist[b] = __ldcg(&sw.hist[(size_t)s * 2048 + b]);
+    reinterpret_cast<uint4*>(sm.hist)[tid] = __ldcg(reinterpret_cast<const uint4*>(sw.hist + (size_t)s * 2048) + tid);
     find_bin(sm, 2048, (uint32_t)kB);
     const uint32_t b1 = sm.bin;
     const uint32_t need1 = (uint32_t)kB - (uint32_t)sm.above;
     int32_t* cnt = sw.counters + s * 4;
     int32_t* winners = sw.winners + (size_t)s * kB;
     uint2* cand = sw.cand + (size_t)s * kDecodeCand;
+    // Sure winners (digit above b1) and candidates (digit b1) of this CTA's
+    // slice, 8 entries per thread per round (coalesced: entry e of thread t
+    // is r0 + e T + t); one scan and one 64-bit atomic on (winners,
+    // candidates) place a round's entries.
     int64_t lo, hi;
     cta_range(nvis, blockIdx.x, gridDim.x, lo, hi);
-    for (int64_t b0 = lo; b0 < hi; b0 += SC_THREADS) {
-        const int64_t b = b0 + tid;
-        const uint32_t key = b < hi ? float_key(__ldcg(row + b)) : 0u;
-        const bool win = b < hi && (key >> 21) > b1;
-        const bool tie = b < hi && (key >> 21) == b1;
-        const int ws = cta_append(sm, win, cnt + 0, &base_slot);
-        if (ws >= 0) winners[ws] = (int32_t)b;
-        const int cs = cta_append(sm, tie, cnt + 1, &base_slot);
-        if (cs >= 0 && cs < kDecodeCand) cand[cs] = make_uint2(key, (uint32_t)b);
+    constexpr int E = 8;
+    for (int64_t r0 = lo; r0 < hi; r0 += (int64_t)E * SC_THREADS) {
+        uint32_t key[E];
+        uint32_t nw = 0, ncand = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int64_t b = r0 + (int64_t)e * SC_THREADS + tid;
+            key[e] = b < hi ? float_key(__ldcg(row + b)) : 0u;
+            nw += (b < hi && (key[e] >> 21) > b1) ? 1u : 0u;
+            ncand += (b < hi && (key[e] >> 21) == b1) ? 1u : 0u;
+        }
+        uint32_t pre;
+        const uint32_t tot = cta_prefix(sm, (ncand << 16) | nw, pre);
+        if (tid == 0) {
+            const unsigned long long add = ((unsigned long long)(tot >> 16) << 32) | (tot & 0xFFFFu);
+            slot_base = tot ? atomicAdd(reinterpret_cast<unsigned long long*>(cnt), add) : 0ull;
+        }
+        __syncthreads();
+        int ws_ = (int)(uint32_t)slot_base + (int)(pre & 0xFFFFu);
+        int cs = (int)(uint32_t)(slot_base >> 32) + (int)(pre >> 16);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const int64_t b = r0 + (int64_t)e * SC_THREADS + tid;
+            if (b >= hi) break;
+            const uint32_t d = key[e] >> 21;
+            if (d > b1) {
+                if (ws_ < kB) winners[ws_] = (int32_t)b;  // < k_B by the histogram
+                ++ws_;
+            } else if (d == b1) {
+                if (cs < kDecodeCand) cand[cs] = make_uint2(key[e], (uint32_t)b);
+                ++cs;
+            }
+        }
+        __syncthreads();
     }
     // The last CTA of the sequence finishes the pick.
     __threadfence();
@@ -241,8 +281,7 @@ __global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
         sm.cand_idx[c] = (int32_t)e.y;
     }
     if (tid == 0) sm.n_out = n_win;
-    __syncthreads();
-    __syncthreads();  // counters read by every thread before the reset
+    __syncthreads();  // (counters read by every thread before the reset)
     reset_state(sw, s);
     finish_from_candidates(sm, nc, b1, need1, kB, out);
     if (tid == 0) nsel[s] = kB;

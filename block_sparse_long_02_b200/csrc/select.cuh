@@ -18,6 +18,7 @@ constexpr int T = 512;           // threads per CTA of the select routines
 constexpr int NW = T / 32;
 constexpr int BINS = 2048;
 constexpr int CAND = 4096;
+static_assert(T * 4 == BINS, "find_bin: 4 bins per thread");
 
 struct SelSmem {
     uint32_t hist[BINS];
@@ -29,37 +30,56 @@ struct SelSmem {
 };
 
 // Finds bin B (counting from the top) with above(B) < need <= above(B) + hist[B].
-// Result in sm.bin / sm.above. Must be called by all threads; nbins <= 2048.
-__device__ void find_bin(SelSmem& sm, int nbins, uint32_t need) {
-    __syncthreads();
-    const int tid = threadIdx.x;
-    if (tid < 32) {
-        const int per = nbins / 32;
-        uint32_t sum = 0;
-        for (int b = 0; b < per; ++b) sum += sm.hist[tid * per + b];
-        // Inclusive suffix sum over lanes (from lane 31 down).
-        uint32_t suf = sum;
+// Result in sm.bin / sm.above. Must be called by all T threads; nbins is 1024
+// or 2048. Thread t owns bins [t * per, (t + 1) * per) (one vector load, no
+// bank conflicts); a suffix scan over the threads gives every thread the
+// count above its bins, and the one thread whose bins hold the need-th key
+// walks them.
+template <int PER>
+__device__ __forceinline__ void find_bin_per(SelSmem& sm, uint32_t need) {
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    uint32_t h[4];
+    if (PER == 4) {
+        const uint4 x = reinterpret_cast<const uint4*>(sm.hist)[tid];
+        h[0] = x.x, h[1] = x.y, h[2] = x.z, h[3] = x.w;
+    } else {
+        const uint2 x = reinterpret_cast<const uint2*>(sm.hist)[tid];
+        h[0] = x.x, h[1] = x.y, h[2] = 0u, h[3] = 0u;
+    }
+    const uint32_t sum = h[0] + h[1] + h[2] + h[3];
+    uint32_t suf = sum;  // inclusive suffix over this warp's lanes
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
-            if (tid + o < 32) suf += v;
-        }
-        const uint32_t above_lane = suf - sum;  // count in lanes > tid
-        const bool mine = above_lane < need && need <= suf;
-        if (mine) {
-            uint32_t acc = above_lane;
-            for (int b = per - 1; b >= 0; --b) {
-                const uint32_t h = sm.hist[tid * per + b];
-                if (acc + h >= need) {
-                    sm.bin = tid * per + b;
-                    sm.above = (int32_t)acc;
-                    break;
-                }
-                acc += h;
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += v;
+    }
+    if (lane == 0) sm.wsum[w] = suf;
+    __syncthreads();
+    uint32_t above_w = 0;
+    for (int k = w + 1; k < NW; ++k) above_w += sm.wsum[k];
+    const uint32_t incl = suf + above_w;  // keys in bins >= my first bin
+    const uint32_t above = incl - sum;    // keys in bins above mine
+    if (above < need && need <= incl) {
+        uint32_t acc = above;
+#pragma unroll
+        for (int b = PER - 1; b >= 0; --b) {
+            if (acc + h[b] >= need) {
+                sm.bin = tid * PER + b;
+                sm.above = (int32_t)acc;
+                break;
             }
+            acc += h[b];
         }
     }
     __syncthreads();
+}
+
+__device__ void find_bin(SelSmem& sm, int nbins, uint32_t need) {
+    __syncthreads();
+    if (nbins == 2048)
+        find_bin_per<4>(sm, need);
+    else
+        find_bin_per<2>(sm, need);
 }
 
 __device__ void clear_hist(SelSmem& sm) {
@@ -130,8 +150,58 @@ __device__ void select_general(SelSmem& sm, const float* x, int64_t n, int kB, u
 __device__ void finish_from_candidates(SelSmem& sm, int nc, uint32_t b1, uint32_t need1, int kB,
                                        int32_t* sel);
 
+// Sorts sm.out[0, kB) ascending (bitonic network, padded with INT_MAX to a
+// power of two). For up to T keys each thread holds one key; compare-exchange
+// steps with a partner in the same warp use shuffles, the others go through
+// shared memory.
+__device__ void sort_out(SelSmem& sm, int kB) {
+    const int tid = threadIdx.x;
+    int P = 1;
+    while (P < kB) P <<= 1;
+    if (P <= T) {
+        int32_t v = tid < kB ? sm.out[tid] : 0x7fffffff;
+        for (int k = 2; k <= T; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                int32_t o;
+                if (j >= 32) {
+                    __syncthreads();
+                    sm.out[tid] = v;
+                    __syncthreads();
+                    o = sm.out[tid ^ j];
+                } else {
+                    o = __shfl_xor_sync(0xffffffffu, v, j);
+                }
+                const bool up = (tid & k) == 0, lower = (tid & j) == 0;
+                v = (lower == up) ? min(v, o) : max(v, o);
+            }
+        }
+        __syncthreads();
+        sm.out[tid] = v;
+        __syncthreads();
+        return;
+    }
+    for (int k = kB + tid; k < P; k += T) sm.out[k] = 0x7fffffff;
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += T) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const int32_t a = sm.out[i], b = sm.out[ixj];
+                    const bool up = (i & k) == 0;
+                    if ((a > b) == up) {
+                        sm.out[i] = b;
+                        sm.out[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
 // Exact top-k_B of one row of n scores (x[i] = score of block i), written
-// ascending to sel, nsel = min(n, k_B). One CTA of SEL_T threads.
+// ascending to sel, nsel = min(n, k_B). One CTA of T threads.
 __device__ void select_row(SelSmem& sm, const float* x, int64_t n, int kB, int32_t* sel,
                            int32_t* nsel) {
     const int tid = threadIdx.x;
@@ -219,27 +289,7 @@ __device__ void finish_from_candidates(SelSmem& sm, int nc, uint32_t b1, uint32_
         if (take) sm.out[atomicAdd(&sm.n_out, 1)] = sm.cand_idx[c];
     }
     __syncthreads();
-    // Bitonic sort of the kB selected indices (padded to a power of two).
-    int P = 1;
-    while (P < kB) P <<= 1;
-    for (int k = kB + tid; k < P; k += T) sm.out[k] = 0x7fffffff;
-    __syncthreads();
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < P; i += T) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const int32_t a = sm.out[i], b = sm.out[ixj];
-                    const bool up = (i & k) == 0;
-                    if ((a > b) == up) {
-                        sm.out[i] = b;
-                        sm.out[ixj] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
+    sort_out(sm, kB);
     for (int k = tid; k < kB; k += T) sel[k] = sm.out[k];
 }
 
