@@ -249,17 +249,32 @@ __device__ void select_row(SelSmem& sm, const float* x, int64_t n, int kB, int32
 // digit b1) are in sm.cand_key / sm.cand_idx: refines the threshold on the
 // remaining 21 key bits, takes ties at the threshold by lowest index, sorts the
 // k_B winners ascending and writes them to sel. need1 = k_B - sm.n_out.
+// Warp-aggregated append to a shared-memory list: one atomic per warp.
+// Every lane of the warp must call it.
+__device__ __forceinline__ void warp_push(SelSmem& sm, bool flag, int32_t value) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t bal = __ballot_sync(0xffffffffu, flag);
+    int base = 0;
+    if (lane == 0 && bal) base = atomicAdd(&sm.n_out, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (flag) sm.out[base + __popc(bal & ((1u << lane) - 1u))] = value;
+}
+
 __device__ void finish_from_candidates(SelSmem& sm, int nc, uint32_t b1, uint32_t need1, int kB,
                                        int32_t* sel) {
     const int tid = threadIdx.x;
-    // Level 2 on the candidates.
+    // Level 2 on the candidates. (Loops run the same trip count in every
+    // thread, so the warp-wide appends see full warps.)
     clear_hist(sm);
     for (int c = tid; c < nc; c += T) atomicAdd(&sm.hist[(sm.cand_key[c] >> 10) & 2047u], 1u);
     find_bin(sm, 2048, need1);
     const uint32_t b2 = sm.bin;
     const uint32_t need2 = need1 - sm.above;
-    for (int c = tid; c < nc; c += T)
-        if (((sm.cand_key[c] >> 10) & 2047u) > b2) sm.out[atomicAdd(&sm.n_out, 1)] = sm.cand_idx[c];
+    for (int c0 = 0; c0 < nc; c0 += T) {
+        const int c = c0 + tid;
+        const bool f = c < nc && ((sm.cand_key[c] >> 10) & 2047u) > b2;
+        warp_push(sm, f, f ? sm.cand_idx[c] : 0);
+    }
     // Level 3.
     clear_hist(sm);
     for (int c = tid; c < nc; c += T)
@@ -269,24 +284,29 @@ __device__ void finish_from_candidates(SelSmem& sm, int nc, uint32_t b1, uint32_
     const uint32_t need_t = need2 - sm.above;
     if (tid == 0) sm.ties = 0;
     __syncthreads();
-    for (int c = tid; c < nc; c += T) {
-        const uint32_t k = sm.cand_key[c];
-        if ((k >> 10) == (key_t >> 10) && k > key_t) sm.out[atomicAdd(&sm.n_out, 1)] = sm.cand_idx[c];
-        if (k == key_t) atomicAdd(&sm.ties, 1);
+    int my_ties = 0;
+    for (int c0 = 0; c0 < nc; c0 += T) {
+        const int c = c0 + tid;
+        const uint32_t k = c < nc ? sm.cand_key[c] : 0u;
+        const bool f = c < nc && (k >> 10) == (key_t >> 10) && k > key_t;
+        warp_push(sm, f, f ? sm.cand_idx[c] : 0);
+        my_ties += (c < nc && k == key_t) ? 1 : 0;
     }
+    my_ties = (int)warp_sum((uint32_t)my_ties);
+    if ((tid & 31) == 0 && my_ties) atomicAdd(&sm.ties, my_ties);
     __syncthreads();
     const int nties = sm.ties;
-    for (int c = tid; c < nc; c += T) {
-        if (sm.cand_key[c] != key_t) continue;
-        bool take = true;
-        if ((uint32_t)nties != need_t) {
+    for (int c0 = 0; c0 < nc; c0 += T) {
+        const int c = c0 + tid;
+        bool take = c < nc && sm.cand_key[c] == key_t;
+        if (take && (uint32_t)nties != need_t) {
             const int32_t me = sm.cand_idx[c];
             uint32_t rank = 0;
             for (int d = 0; d < nc; ++d)
                 rank += (sm.cand_key[d] == key_t && sm.cand_idx[d] < me) ? 1u : 0u;
             take = rank < need_t;
         }
-        if (take) sm.out[atomicAdd(&sm.n_out, 1)] = sm.cand_idx[c];
+        warp_push(sm, take, take ? sm.cand_idx[c] : 0);
     }
     __syncthreads();
     sort_out(sm, kB);
