@@ -81,24 +81,28 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
     const int nchunks = (int)((ntok + CT - 1) / CT);
     const int64_t cur = w.i / w.r;
     const int64_t row_stride = (int64_t)w.kv_heads * kHeadDim;
+    // The warp's first 32 selection entries in one round trip (lane u holds
+    // unit u0 + u); later units, if any, are read when their chunk is issued.
+    const int32_t sel_lane = (w.u0 + lane < w.u1 && w.u0 + lane < w.nsel) ? w.sel[w.u0 + lane] : -1;
 
     auto issue = [&](int c) {
         const int stg = c % STAGES;
-        if (lane < CT) {
-            const int64_t p = (int64_t)c * CT + lane;
+        {
+            const int64_t p = (int64_t)c * CT + (lane & (CT - 1));  // lanes >= CT mirror lanes < CT
+            const int u = w.u0 + (int)(p / w.r);
+            const int32_t b_pre = __shfl_sync(0xffffffffu, sel_lane, (u - w.u0) & 31);
             int64_t t = -1;
             if (p < ntok) {
-                const int u = w.u0 + (int)(p / w.r);
                 const int e = (int)(p % w.r);
                 if (u < w.nsel) {
-                    const int32_t b = w.sel[u];
+                    const int32_t b = u - w.u0 < 32 ? b_pre : w.sel[u];
                     if (b >= 0 && (int64_t)b < cur) t = (int64_t)b * w.r + e;
                 } else {
                     const int64_t tt = cur * w.r + e;
                     if (tt <= w.i) t = tt;
                 }
             }
-            tok[stg * CT + lane] = t;
+            if (lane < CT) tok[stg * CT + lane] = t;
         }
         __syncwarp();
         if (lane == 0) {
@@ -383,34 +387,38 @@ __global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
     }
 }
 
-// Combine the S partials of each (sequence, head): one CTA of 128 threads per
-// head, thread d owns output dim d; the partials' maxima and sums are staged in
-// shared memory, the S partial rows are read coalesced.
+// Combine the S partials of each (sequence, head): one CTA of 4 warps per
+// head; every warp finds the partials' maximum itself (two loads per lane),
+// warp w sums partials w, w + 4, ... for all 128 dims (lane: dims lane + 32 j),
+// with every load of the warp issued before the first use, and the four warp
+// sums meet in shared memory.
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part, int S,
                                                             uint16_t* __restrict__ out) {
-    __shared__ float wgt[64];
-    __shared__ float inv_l;
-    const int row = blockIdx.x, d = threadIdx.x;
+    __shared__ float so[4][128];
+    __shared__ float sl[4];
+    const int row = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const float* src = part + (size_t)row * S * 132;
-    if (d < 32) {
-        float m = -INFINITY;
-        for (int k = d; k < S; k += 32) m = fmaxf(m, src[(size_t)k * 132 + 128]);
+    float m = -INFINITY;
+    for (int k = lane; k < S; k += 32) m = fmaxf(m, src[(size_t)k * 132 + 128]);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
-        for (int k = d; k < S; k += 32) {
-            const float c = (m == -INFINITY) ? 0.f : exp2f(src[(size_t)k * 132 + 128] - m);
-            wgt[k] = c;
-            l += src[(size_t)k * 132 + 129] * c;
-        }
-        l = warp_sum(l);
-        if (d == 0) inv_l = l > 0.f ? 1.f / l : 0.f;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
+#pragma unroll 4
+    for (int k = w; k < S; k += 4) {
+        const float* pk = src + (size_t)k * 132;
+        const float c = (m == -INFINITY) ? 0.f : exp2f(pk[128] - m);
+        l = fmaf(pk[129], c, l);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = fmaf(pk[lane + 32 * j], c, acc[j]);
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) so[w][lane + 32 * j] = acc[j];
+    if (lane == 0) sl[w] = l;
     __syncthreads();
-    float acc = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < S; ++k) acc = fmaf(src[(size_t)k * 132 + d], wgt[k], acc);
-    out[(size_t)row * kHeadDim + d] = f32_to_bf16(acc * inv_l);
+    const int d = threadIdx.x;
+    const float lt = sl[0] + sl[1] + sl[2] + sl[3];
+    const float o = so[0][d] + so[1][d] + so[2][d] + so[3][d];
+    out[(size_t)row * kHeadDim + d] = f32_to_bf16(lt > 0.f ? o / lt : 0.f);
 }
 
 }  // namespace
