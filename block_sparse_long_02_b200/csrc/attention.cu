@@ -332,6 +332,8 @@ __global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
     const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc, int64_t cap,
     const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel, float* __restrict__ part,
     int batch, int q_heads, int kv_heads, int r, int kB, int S, float scale_log2) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t item = (int64_t)blockIdx.x * WARPS + warp;
@@ -394,6 +396,8 @@ __global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
 // sums meet in shared memory.
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part, int S,
                                                             uint16_t* __restrict__ out) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float so[4][128];
     __shared__ float sl[4];
     const int row = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -456,15 +460,13 @@ cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t
     const int S = decode_attention_splits(L);
     const int64_t items = (int64_t)batch * L.kv_heads * S;
     note_launch();
-    decode_attention_kernel<<<(unsigned)((items + WARPS - 1) / WARPS), WARPS * 32, SMEM, st>>>(
-        q, pos, kc, vc, cap, sel, nsel, part, batch, L.q_heads, L.kv_heads, L.r, L.kB, S,
-        L.sm_scale * LOG2E);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(decode_attention_kernel, dim3((unsigned)((items + WARPS - 1) / WARPS)),
+                               dim3(WARPS * 32), (size_t)SMEM, st, q, pos, kc, vc, cap, sel, nsel, part, batch,
+                               L.q_heads, L.kv_heads, L.r, L.kB, S, L.sm_scale * LOG2E);
     if (e != cudaSuccess) return e;
     const int rows = batch * L.q_heads;
     note_launch();
-    decode_combine_kernel<<<rows, 128, 0, st>>>(part, S, out);
-    return cudaGetLastError();
+    return launch_pdl(decode_combine_kernel, dim3((unsigned)rows), dim3(128), 0, st, (const float*)part, S, out);
 }
 
 }  // namespace qsa

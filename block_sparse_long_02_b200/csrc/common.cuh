@@ -63,6 +63,15 @@ __device__ __forceinline__ void flag_status(int32_t* status, int32_t code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before
+// the previous kernel in the stream has finished; pdl_wait() blocks until
+// every earlier grid has completed and its writes are visible (a no-op for a
+// normal launch), and pdl_trigger() lets the next such kernel start launching.
+// Decode kernels call both first thing, so they read nothing early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // --------------------------------------------------------------- cp.async / mma
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);

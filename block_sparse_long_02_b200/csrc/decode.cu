@@ -24,7 +24,6 @@ namespace qsa {
 namespace {
 
 constexpr int SC_THREADS = 512;  // score and select CTAs
-constexpr int SC_WARPS = SC_THREADS / 32;
 
 constexpr int DS_THREADS = 256;  // fused score CTAs
 constexpr int DS_WARPS = DS_THREADS / 32;
@@ -60,6 +59,8 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status) {
     __shared__ uint32_t hist[2048];
     __shared__ __align__(16) uint16_t qs[kIdxHeads * kIdxDim];
+    pdl_wait();
+    pdl_trigger();
     const int s = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t p = pos[s];
@@ -197,6 +198,8 @@ __global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
     SelSmem& sm = *reinterpret_cast<SelSmem*>(raw);
     __shared__ unsigned long long slot_base;  // (candidates << 32) | winners before this round
     __shared__ int last;
+    pdl_wait();
+    pdl_trigger();
     const int s = blockIdx.y;
     const int tid = threadIdx.x;
     const int64_t p = pos[s];
@@ -309,10 +312,9 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
                                 int32_t* status, cudaStream_t st) {
     note_launch();
-    decode_score_kernel<<<dim3((unsigned)decode_score_ctas(batch), (unsigned)batch), DS_THREADS, 0, st>>>(
-        pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps,
-        L.rope, scores, sw.hist, status);
-    return cudaGetLastError();
+    return launch_pdl(decode_score_kernel, dim3((unsigned)decode_score_ctas(batch), (unsigned)batch),
+                      dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache, pooled, cap, rms_w,
+                      L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist, status);
 }
 
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
@@ -321,9 +323,8 @@ cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* p
     const int smem = (int)sizeof(SelSmem);
     cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     note_launch();
-    decode_select_kernel<<<dim3((unsigned)decode_select_ctas(batch), (unsigned)batch), SC_THREADS, smem, st>>>(
-        pos, cap, L.r, L.kB, scores, sw, sel, nsel);
-    return cudaGetLastError();
+    return launch_pdl(decode_select_kernel, dim3((unsigned)decode_select_ctas(batch), (unsigned)batch),
+                      dim3(SC_THREADS), (size_t)smem, st, pos, cap, L.r, L.kB, scores, sw, sel, nsel);
 }
 
 }  // namespace qsa

@@ -2,6 +2,8 @@
 // validates arguments and calls these; each returns cudaGetLastError().
 #pragma once
 
+#include <utility>
+
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -9,6 +11,25 @@
 #include "common.cuh"
 
 namespace qsa {
+
+// Launch with programmatic stream serialization: the kernel may begin
+// launching while the previous kernel in the stream finishes; it must call
+// pdl_wait() before touching memory (the decode kernels do so first thing).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Counts one kernel launch (see qsa_launch_count).
 void note_launch(int n = 1);
