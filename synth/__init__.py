@@ -239,6 +239,9 @@ class Workload:
         L = self.row_len(name)
         t = tensor.view(tensor.shape[0], -1, L) if tensor.dim() != 3 or tensor.shape[-1] != L else tensor
         assert t.is_contiguous() and t.dtype == torch.bfloat16
+        # Rows are absolute: the tensor must hold rows [0, r1) of each sequence.
+        if not 0 <= r0 <= r1 <= t.shape[1]:
+            raise ValueError(f"rows [{r0}, {r1}) outside a tensor of {t.shape[1]} rows")
         for s in range(t.shape[0]):
             dst = t[s, r0:r1]
             fill_device(self.seed(s), TENSOR_IDS[name], r0 * L, (r1 - r0) * L, dst.data_ptr(), stream)

@@ -58,3 +58,14 @@ def test_device_generator_matches_host_bit_for_bit():
     got = big.view(torch.int16).cpu().numpy().view(np.uint16)[idx]
     want = np.array([synth.fill_host(99, 3, (1 << 30) + int(i), 1)[0] for i in idx])
     assert np.array_equal(got, want)
+
+
+def test_device_fill_rejects_rows_outside_the_tensor():
+    """Rows are absolute positions: a buffer that holds fewer rows is refused
+    on the host, before any device write."""
+    import torch
+
+    w = synth.WORKLOADS["tiny_prefill_n256"]
+    t = torch.empty(1, 16, w.row_len("q"), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        w.device_fill("q", t, rows=(200, 216))
