@@ -4,13 +4,17 @@
 // page: attention_input = flatten(selected_blocks) + current_incomplete_block).
 //
 // The stage is a gather: per query and kv head, ~2K random 256-byte key and
-// value rows feed 8 query heads (8 flop per byte), so it is bound by memory,
-// not by the tensor pipe. One warp owns one (query, kv head) pair (or a slice
-// of its units): the G = q_heads/kv_heads query heads are the rows of an
-// m16n8k16 tile (padded to 16), tokens stream through a 3-stage cp.async ring
-// of 16-token chunks in row-swizzled shared memory, logits/softmax/accumulation
-// are fp32 with an online (running max) softmax, and probabilities are rounded
-// to bf16 for the P.V product. Invalid selections are skipped, never read.
+// value rows feed G = q_heads/kv_heads query heads (8 flop per byte). One warp
+// owns one (query, kv head) pair (or a slice of its units); tokens stream
+// through a 3-stage cp.async ring of 16-token chunks in row-swizzled shared
+// memory. The tiles are transposed so that no row is padding: in
+// S^T = K Q^T the 16 tokens of a chunk are the m16 rows and the query heads
+// the n8 columns (one n8 tile per 8 heads), and in O^T += V^T P^T the 128
+// dims are eight m16 tiles and the heads again the columns; the probabilities
+// move from the S^T accumulator to the P^T operand with one movmatrix
+// transpose per 8x8 block. Logits, the online (running max) softmax and the
+// accumulation are fp32; probabilities are rounded to bf16 for the P.V
+// product. Invalid selections are skipped, never read.
 #include <algorithm>
 
 #include "kernels.h"
@@ -42,40 +46,58 @@ struct Work {
     float scale_log2;      // sm_scale * log2(e)
 };
 
+// Per-warp attention state for NT tiles of 8 query heads. Lane (g, t) =
+// (lane / 4, lane % 4) holds, for head h = 8 nt + 2 t + e (e = 0, 1):
+// o[nt][i][e] and o[nt][i][2 + e] = unnormalised output dims 16 i + g and
+// 16 i + g + 8; m[nt][e] = running maximum (log2 domain), l[nt][e] = sum of
+// probabilities (after warp_attend: over the whole warp).
+template <int NT>
 struct WarpState {
-    float o[16][4];
-    float m[2], l[2];
+    float o[NT][8][4];
+    float m[NT][2], l[NT][2];
 };
+template <int NT>
+constexpr int park_floats() {
+    return NT * 36;  // o (32), m (2), l (2) per n8 tile
+}
 
-__device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lane, WarpState& st) {
+// 8x8 b16 matrix transpose in the mma fragment layout (lane l holds row l/4,
+// columns 2 (l % 4) and 2 (l % 4) + 1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(d) : "r"(a));
+    return d;
+}
+
+template <int NT>
+__device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lane, WarpState<NT>& st) {
     uint16_t* ring = reinterpret_cast<uint16_t*>(wsm);
     int64_t* tok = reinterpret_cast<int64_t*>(wsm + STAGES * STAGE_BYTES);  // [STAGES][CT]
     uint32_t* vmask = reinterpret_cast<uint32_t*>(wsm + STAGES * STAGE_BYTES + STAGES * CT * 8);
     const uint32_t ring_s = smem_u32(ring);
-    const int gq = lane >> 2, tig = lane & 3;
+    const int g = lane >> 2, t = lane & 3;
 
-    // Query fragments (A operand, rows = query heads of the group).
-    uint32_t qa[8][4];
+    // Query fragments (B operand of S^T = K Q^T): column = head 8 nt + g,
+    // k rows = dims 16 ks + 2 t (+1) and 16 ks + 8 + 2 t (+1).
+    uint32_t qb[NT][8][2];
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = 8 * nt + g;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-            for (int kh = 0; kh < 2; ++kh) {
-                const int row = gq + hf * 8;
-                const int col = ks * 16 + kh * 8 + 2 * tig;
-                uint32_t v = 0;
-                if (row < w.G) v = *reinterpret_cast<const uint32_t*>(w.q + row * kHeadDim + col);
-                qa[ks][kh * 2 + hf] = v;
-            }
+        for (int ks = 0; ks < 8; ++ks) {
+            qb[nt][ks][0] = h < w.G ? *reinterpret_cast<const uint32_t*>(w.q + h * kHeadDim + ks * 16 + 2 * t) : 0u;
+            qb[nt][ks][1] = h < w.G ? *reinterpret_cast<const uint32_t*>(w.q + h * kHeadDim + ks * 16 + 8 + 2 * t) : 0u;
         }
     }
 #pragma unroll
-    for (int nd = 0; nd < 16; ++nd)
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) st.o[nd][e] = 0.f;
-    st.m[0] = st.m[1] = -INFINITY;
-    st.l[0] = st.l[1] = 0.f;
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st.o[nt][i][e] = 0.f;
+        st.m[nt][0] = st.m[nt][1] = -INFINITY;
+        st.l[nt][0] = st.l[nt][1] = 0.f;
+    }
 
     const int64_t ntok = (int64_t)(w.u1 - w.u0) * w.r;
     const int nchunks = (int)((ntok + CT - 1) / CT);
@@ -91,18 +113,18 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
             const int64_t p = (int64_t)c * CT + (lane & (CT - 1));  // lanes >= CT mirror lanes < CT
             const int u = w.u0 + (int)(p / w.r);
             const int32_t b_pre = __shfl_sync(0xffffffffu, sel_lane, (u - w.u0) & 31);
-            int64_t t = -1;
+            int64_t tk = -1;
             if (p < ntok) {
                 const int e = (int)(p % w.r);
                 if (u < w.nsel) {
                     const int32_t b = u - w.u0 < 32 ? b_pre : w.sel[u];
-                    if (b >= 0 && (int64_t)b < cur) t = (int64_t)b * w.r + e;
+                    if (b >= 0 && (int64_t)b < cur) tk = (int64_t)b * w.r + e;
                 } else {
                     const int64_t tt = cur * w.r + e;
-                    if (tt <= w.i) t = tt;
+                    if (tt <= w.i) tk = tt;
                 }
             }
-            if (lane < CT) tok[stg * CT + lane] = t;
+            if (lane < CT) tok[stg * CT + lane] = tk;
         }
         __syncwarp();
         if (lane == 0) {
@@ -116,9 +138,9 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         for (int k = 0; k < (CT * 16) / 32; ++k) {
             const int idx = lane + k * 32;
             const int row = idx >> 4, ch = idx & 15;
-            const int64_t t = tok[stg * CT + row];
-            const bool ok = t >= 0;
-            const size_t off = (size_t)(ok ? t : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 8;
+            const int64_t tk = tok[stg * CT + row];
+            const bool ok = tk >= 0;
+            const size_t off = (size_t)(ok ? tk : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 8;
             cp_async16_zfill(kbase + swz256(row, ch), w.kc + off, ok);
             cp_async16_zfill(vbase + swz256(row, ch), w.vc + off, ok);
         }
@@ -129,6 +151,10 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         if (c < nchunks) issue(c);
         cp_async_commit();
     }
+    // ldmatrix row addresses: K as the A operand (token rows, dims in chunk
+    // pairs), V^T as the A operand (transposed 8x8 loads of token rows).
+    const int krow = (lane & 7) + ((lane >> 3) & 1) * 8, kch = lane >> 4;
+    const int vrow = (lane & 7) + ((lane >> 4) & 1) * 8, vch = (lane >> 3) & 1;
     for (int c = 0; c < nchunks; ++c) {
         if (c + STAGES - 1 < nchunks) issue(c + STAGES - 1);
         cp_async_commit();
@@ -139,119 +165,137 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         const uint32_t vbase = kbase + CT * 256;
         const uint32_t valid = vmask[stg];
 
-        // S = Q K^T over 16 tokens (two n8 tiles).
-        float s[2][4];
+        // S^T = K Q^T: rows = tokens g, g + 8; columns = heads 8 nt + 2 t (+1).
+        float s[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            uint32_t b00, b01, b10, b11;
-            const int nrow = (lane & 7) + ((lane >> 4) & 1) * 8;
-            const int ch = ks * 2 + ((lane >> 3) & 1);
-            ldmatrix_x4(kbase + swz256(nrow, ch), b00, b01, b10, b11);
-            mma_bf16_16816(s[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
-            mma_bf16_16816(s[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(kbase + swz256(krow, ks * 2 + kch), a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
         }
-        // Online softmax (log2 domain), rows gq (hf=0) and gq+8 (hf=1).
+        // Online softmax per head (log2 domain); a head's 16 tokens sit in the
+        // 8 lanes with the same t.
+        const bool v0 = (valid >> g) & 1u, v1 = (valid >> (g + 8)) & 1u;
+        uint32_t pb[NT][2];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            float mx = -INFINITY;
+        for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int e = 0; e < 2; ++e) {
+                const float x0 = v0 ? s[nt][e] * w.scale_log2 : -INFINITY;
+                const float x1 = v1 ? s[nt][2 + e] * w.scale_log2 : -INFINITY;
+                float mx = fmaxf(x0, x1);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float m_new = fmaxf(st.m[nt][e], mx);
+                const float corr = (m_new == -INFINITY) ? 1.f : exp2f(st.m[nt][e] - m_new);
+                const float p0 = (x0 == -INFINITY) ? 0.f : exp2f(x0 - m_new);
+                const float p1 = (x1 == -INFINITY) ? 0.f : exp2f(x1 - m_new);
+                st.l[nt][e] = st.l[nt][e] * corr + (p0 + p1);
+                st.m[nt][e] = m_new;
+                s[nt][e] = p0;
+                s[nt][2 + e] = p1;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int col = nt * 8 + 2 * tig + e;
-                    float v = s[nt][hf * 2 + e] * w.scale_log2;
-                    v = ((valid >> col) & 1u) ? v : -INFINITY;
-                    s[nt][hf * 2 + e] = v;
-                    mx = fmaxf(mx, v);
+                for (int i = 0; i < 8; ++i) {
+                    st.o[nt][i][e] *= corr;
+                    st.o[nt][i][2 + e] *= corr;
                 }
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(st.m[hf], mx);
-            const float corr = (m_new == -INFINITY) ? 1.f : exp2f(st.m[hf] - m_new);
-            float psum = 0.f;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float v = s[nt][hf * 2 + e];
-                    const float p = (v == -INFINITY) ? 0.f : exp2f(v - m_new);
-                    s[nt][hf * 2 + e] = p;
-                    psum += p;
-                }
-            st.l[hf] = st.l[hf] * corr + psum;
-            st.m[hf] = m_new;
-#pragma unroll
-            for (int nd = 0; nd < 16; ++nd) {
-                st.o[nd][hf * 2] *= corr;
-                st.o[nd][hf * 2 + 1] *= corr;
             }
+            // P^T operand: the two 8x8 blocks (tokens 0-7, 8-15) of this tile,
+            // rounded to bf16 and transposed.
+            pb[nt][0] = movmatrix_trans(pack_bf16x2(s[nt][0], s[nt][1]));
+            pb[nt][1] = movmatrix_trans(pack_bf16x2(s[nt][2], s[nt][3]));
         }
-        // O += P V (P rounded to bf16).
-        const uint32_t pa0 = pack_bf16x2(s[0][0], s[0][1]);
-        const uint32_t pa1 = pack_bf16x2(s[0][2], s[0][3]);
-        const uint32_t pa2 = pack_bf16x2(s[1][0], s[1][1]);
-        const uint32_t pa3 = pack_bf16x2(s[1][2], s[1][3]);
+        // O^T += V^T P^T: rows = dims 16 i + g (+8), columns = heads.
 #pragma unroll
-        for (int np = 0; np < 8; ++np) {
-            uint32_t b0, b1, b2, b3;
-            const int trow = (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int ch = np * 2 + (lane >> 4);
-            ldmatrix_x4_trans(vbase + swz256(trow, ch), b0, b1, b2, b3);
-            mma_bf16_16816(st.o[2 * np], pa0, pa1, pa2, pa3, b0, b1);
-            mma_bf16_16816(st.o[2 * np + 1], pa0, pa1, pa2, pa3, b2, b3);
+        for (int i = 0; i < 8; ++i) {
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(vbase + swz256(vrow, 2 * i + vch), a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(st.o[nt][i], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
         }
         __syncwarp();
     }
     cp_async_wait<0>();
-    // Full row sums across the quad.
+    // Full sums over the 16-token rows (the 8 lanes with the same t).
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        st.l[hf] += __shfl_xor_sync(0xffffffffu, st.l[hf], 1);
-        st.l[hf] += __shfl_xor_sync(0xffffffffu, st.l[hf], 2);
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            st.l[nt][e] += __shfl_xor_sync(0xffffffffu, st.l[nt][e], 4);
+            st.l[nt][e] += __shfl_xor_sync(0xffffffffu, st.l[nt][e], 8);
+            st.l[nt][e] += __shfl_xor_sync(0xffffffffu, st.l[nt][e], 16);
+        }
+}
+
+// Parks a state in the lane-strided layout: slot k of lane l at k * 32 + l.
+template <int NT>
+__device__ __forceinline__ void park_state(const WarpState<NT>& st, float* dst, int lane) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[(nt * 36 + i * 4 + e) * 32 + lane] = st.o[nt][i][e];
+        dst[(nt * 36 + 32) * 32 + lane] = st.m[nt][0];
+        dst[(nt * 36 + 33) * 32 + lane] = st.m[nt][1];
+        dst[(nt * 36 + 34) * 32 + lane] = st.l[nt][0];
+        dst[(nt * 36 + 35) * 32 + lane] = st.l[nt][1];
     }
 }
 
-// Merge state `b` into `a` (same rows).
-__device__ __forceinline__ void merge_state(WarpState& a, const float* bo, const float* bm,
-                                            const float* bl) {
+// Merges a parked state (same lanes, same heads) into `a`.
+template <int NT>
+__device__ __forceinline__ void merge_parked(WarpState<NT>& a, const float* src, int lane) {
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        const float m = fmaxf(a.m[hf], bm[hf]);
-        const float ca = (m == -INFINITY) ? 0.f : exp2f(a.m[hf] - m);
-        const float cb = (m == -INFINITY) ? 0.f : exp2f(bm[hf] - m);
-        a.l[hf] = a.l[hf] * ca + bl[hf] * cb;
-        a.m[hf] = m;
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-        for (int nd = 0; nd < 16; ++nd) {
-            a.o[nd][hf * 2] = a.o[nd][hf * 2] * ca + bo[nd * 4 + hf * 2] * cb;
-            a.o[nd][hf * 2 + 1] = a.o[nd][hf * 2 + 1] * ca + bo[nd * 4 + hf * 2 + 1] * cb;
+        for (int e = 0; e < 2; ++e) {
+            const float bm = src[(nt * 36 + 32 + e) * 32 + lane];
+            const float bl = src[(nt * 36 + 34 + e) * 32 + lane];
+            const float m = fmaxf(a.m[nt][e], bm);
+            const float ca = (m == -INFINITY) ? 0.f : exp2f(a.m[nt][e] - m);
+            const float cb = (m == -INFINITY) ? 0.f : exp2f(bm - m);
+            a.l[nt][e] = a.l[nt][e] * ca + bl * cb;
+            a.m[nt][e] = m;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                a.o[nt][i][e] = a.o[nt][i][e] * ca + src[(nt * 36 + i * 4 + e) * 32 + lane] * cb;
+                a.o[nt][i][2 + e] = a.o[nt][i][2 + e] * ca + src[(nt * 36 + i * 4 + 2 + e) * 32 + lane] * cb;
+            }
         }
     }
 }
 
-__device__ __forceinline__ void write_out(const WarpState& st, int G, uint16_t* out_rows,
-                                          float* lse_rows, int lane) {
-    const int gq = lane >> 2, tig = lane & 3;
+// Writes the G normalised output rows (bf16) and, if asked, their LSE.
+template <int NT>
+__device__ __forceinline__ void write_out(const WarpState<NT>& st, int G, uint16_t* out_rows, float* lse_rows,
+                                          int lane) {
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        const int row = gq + hf * 8;
-        if (row >= G) continue;
-        const float inv = st.l[hf] > 0.f ? 1.f / st.l[hf] : 0.f;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nd = 0; nd < 16; ++nd) {
-            const uint32_t v = pack_bf16x2(st.o[nd][hf * 2] * inv, st.o[nd][hf * 2 + 1] * inv);
-            *reinterpret_cast<uint32_t*>(out_rows + row * kHeadDim + nd * 8 + 2 * tig) = v;
+        for (int e = 0; e < 2; ++e) {
+            const int h = 8 * nt + 2 * t + e;
+            if (h >= G) continue;
+            const float inv = st.l[nt][e] > 0.f ? 1.f / st.l[nt][e] : 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                out_rows[h * kHeadDim + 16 * i + g] = f32_to_bf16(st.o[nt][i][e] * inv);
+                out_rows[h * kHeadDim + 16 * i + g + 8] = f32_to_bf16(st.o[nt][i][2 + e] * inv);
+            }
+            if (lse_rows && g == 0)
+                lse_rows[h] = st.l[nt][e] > 0.f ? (st.m[nt][e] + log2f(st.l[nt][e])) * LN2 : -INFINITY;
         }
-        if (lse_rows && tig == 0)
-            lse_rows[row] = st.l[hf] > 0.f ? (st.m[hf] + log2f(st.l[hf])) * LN2 : -INFINITY;
-    }
 }
 
 // Prefill: CTA = one query; warp w -> kv head kv0 + (w % GH), unit split w / GH.
+template <int NT>
 __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
     const uint16_t* __restrict__ q, int64_t q_begin, int64_t nq, const uint16_t* __restrict__ kc,
     const uint16_t* __restrict__ vc, int64_t cap, const int32_t* __restrict__ sel,
@@ -288,45 +332,26 @@ __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
     w.scale_log2 = scale_log2;
 
     uint8_t* wsm = smem + warp * WARP_SMEM;
-    WarpState st;
-    warp_attend(w, wsm, lane, st);
+    WarpState<NT> st;
+    warp_attend<NT>(w, wsm, lane, st);
 
     if (NS > 1) {
         // Splits > 0 park their state in their own smem; split 0 merges.
-        float* park = reinterpret_cast<float*>(wsm);
         __syncthreads();
-        if (split > 0) {
-#pragma unroll
-            for (int nd = 0; nd < 16; ++nd)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) park[(nd * 4 + e) * 32 + lane] = st.o[nd][e];
-            park[64 * 32 + lane] = st.m[0];
-            park[65 * 32 + lane] = st.m[1];
-            park[66 * 32 + lane] = st.l[0];
-            park[67 * 32 + lane] = st.l[1];
-        }
+        if (split > 0) park_state<NT>(st, reinterpret_cast<float*>(wsm), lane);
         __syncthreads();
-        if (split == 0) {
-            for (int sp = 1; sp < NS; ++sp) {
-                const float* src = reinterpret_cast<const float*>(smem + (warp + sp * GH) * WARP_SMEM);
-                float bo[64], bm[2], bl[2];
-#pragma unroll
-                for (int k = 0; k < 64; ++k) bo[k] = src[k * 32 + lane];
-                bm[0] = src[64 * 32 + lane];
-                bm[1] = src[65 * 32 + lane];
-                bl[0] = src[66 * 32 + lane];
-                bl[1] = src[67 * 32 + lane];
-                merge_state(st, bo, bm, bl);
-            }
-        }
+        if (split == 0)
+            for (int sp = 1; sp < NS; ++sp)
+                merge_parked<NT>(st, reinterpret_cast<const float*>(smem + (warp + sp * GH) * WARP_SMEM), lane);
     }
     if (split == 0)
-        write_out(st, G, out + ((size_t)row * q_heads + (size_t)g * G) * kHeadDim,
-                  lse ? lse + (size_t)row * q_heads + (size_t)g * G : nullptr, lane);
+        write_out<NT>(st, G, out + ((size_t)row * q_heads + (size_t)g * G) * kHeadDim,
+                      lse ? lse + (size_t)row * q_heads + (size_t)g * G : nullptr, lane);
 }
 
 // Decode: one warp per (sequence, kv head, split); partial states to `part`
 // laid out [batch][q_heads][S][132] = (o[128], m, l, pad, pad), log2 domain.
+template <int NT>
 __global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
     const uint16_t* __restrict__ q, const int64_t* __restrict__ pos,
     const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc, int64_t cap,
@@ -369,24 +394,26 @@ __global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
     w.kv_heads = kv_heads;
     w.r = r;
     w.scale_log2 = scale_log2;
-    WarpState st;
-    warp_attend(w, smem + warp * WARP_SMEM, lane, st);
-    const int gq = lane >> 2, tig = lane & 3;
+    WarpState<NT> st;
+    warp_attend<NT>(w, smem + warp * WARP_SMEM, lane, st);
+    const int gq = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        const int row = gq + hf * 8;
-        if (row >= G) continue;
-        float* d = dst + (size_t)row * S * 132;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nd = 0; nd < 16; ++nd) {
-            d[nd * 8 + 2 * tig] = st.o[nd][hf * 2];
-            d[nd * 8 + 2 * tig + 1] = st.o[nd][hf * 2 + 1];
+        for (int e = 0; e < 2; ++e) {
+            const int h = 8 * nt + 2 * t + e;
+            if (h >= G) continue;
+            float* d = dst + (size_t)h * S * 132;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                d[16 * i + gq] = st.o[nt][i][e];
+                d[16 * i + gq + 8] = st.o[nt][i][2 + e];
+            }
+            if (gq == 0) {
+                d[128] = st.m[nt][e];
+                d[129] = st.l[nt][e];
+            }
         }
-        if (tig == 0) {
-            d[128] = st.m[hf];
-            d[129] = st.l[hf];
-        }
-    }
 }
 
 // Combine the S partials of each (sequence, head): one CTA of 4 warps per
@@ -433,14 +460,14 @@ cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_
                                     const int32_t* nsel, uint16_t* out, float* lse,
                                     cudaStream_t st) {
     if (nq <= 0 || batch <= 0) return cudaSuccess;
-    cudaFuncSetAttribute(prefill_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         SMEM);
     const int GH = L.kv_heads < WARPS ? L.kv_heads : WARPS;
     dim3 grid((unsigned)nq, (unsigned)batch, (unsigned)(L.kv_heads / GH));
+    const int G = L.q_heads / L.kv_heads;
+    auto kern = G > 8 ? prefill_attention_kernel<2> : prefill_attention_kernel<1>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     note_launch();
-    prefill_attention_kernel<<<grid, WARPS * 32, SMEM, st>>>(
-        q, q_begin, nq, kc, vc, cap, sel, nsel, out, lse, L.q_heads, L.kv_heads, L.r, L.kB,
-        L.sm_scale * LOG2E);
+    kern<<<grid, WARPS * 32, SMEM, st>>>(q, q_begin, nq, kc, vc, cap, sel, nsel, out, lse, L.q_heads, L.kv_heads,
+                                         L.r, L.kB, L.sm_scale * LOG2E);
     return cudaGetLastError();
 }
 
@@ -455,14 +482,15 @@ cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
                                     float* part, uint16_t* out, cudaStream_t st) {
     if (batch <= 0) return cudaSuccess;
-    cudaFuncSetAttribute(decode_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         SMEM);
+    const int G = L.q_heads / L.kv_heads;
+    auto kern = G > 8 ? decode_attention_kernel<2> : decode_attention_kernel<1>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     const int S = decode_attention_splits(L);
     const int64_t items = (int64_t)batch * L.kv_heads * S;
     note_launch();
-    cudaError_t e = launch_pdl(decode_attention_kernel, dim3((unsigned)((items + WARPS - 1) / WARPS)),
-                               dim3(WARPS * 32), (size_t)SMEM, st, q, pos, kc, vc, cap, sel, nsel, part, batch,
-                               L.q_heads, L.kv_heads, L.r, L.kB, S, L.sm_scale * LOG2E);
+    cudaError_t e = launch_pdl(kern, dim3((unsigned)((items + WARPS - 1) / WARPS)), dim3(WARPS * 32), (size_t)SMEM,
+                               st, q, pos, kc, vc, cap, sel, nsel, part, batch, L.q_heads, L.kv_heads, L.r, L.kB,
+                               S, L.sm_scale * LOG2E);
     if (e != cudaSuccess) return e;
     const int rows = batch * L.q_heads;
     note_launch();
