@@ -6,13 +6,14 @@
 // The stage is a gather: per query and kv head, ~2K random 256-byte key and
 // value rows feed G = q_heads/kv_heads query heads (8 flop per byte). One warp
 // owns one (query, kv head) pair (or a slice of its units); tokens stream
-// through a 3-stage cp.async ring of 16-token chunks in row-swizzled shared
-// memory. The tiles are transposed so that no row is padding: in
-// S^T = K Q^T the 16 tokens of a chunk are the m16 rows and the query heads
-// the n8 columns (one n8 tile per 8 heads), and in O^T += V^T P^T the 128
-// dims are eight m16 tiles and the heads again the columns; the probabilities
-// move from the S^T accumulator to the P^T operand with one movmatrix
-// transpose per 8x8 block. Logits, the online (running max) softmax and the
+// through a 2-stage cp.async ring of 16-token chunks in row-swizzled shared
+// memory (two stages leave room for three 4-warp CTAs per SM, which hides the
+// gather latency better than a deeper ring). The tiles are transposed so that
+// no row is padding: in S^T = K Q^T the 16 tokens of a chunk are the m16 rows
+// and the query heads the n8 columns (one n8 tile per 8 heads), and in
+// O^T += V^T P^T the 128 dims are eight m16 tiles and the heads again the
+// columns; the probabilities move from the S^T accumulator to the P^T operand
+// with one movmatrix transpose per 8x8 block. Logits, the online (running max) softmax and the
 // accumulation are fp32; probabilities are rounded to bf16 for the P.V
 // product. Invalid selections are skipped, never read.
 #include <algorithm>
@@ -24,7 +25,7 @@ namespace {
 
 constexpr int WARPS = 4;
 constexpr int CT = 16;                    // tokens per chunk
-constexpr int STAGES = 3;
+constexpr int STAGES = 2;
 constexpr int STAGE_BYTES = CT * 256 * 2; // K and V rows
 constexpr int WARP_SMEM = STAGES * STAGE_BYTES + STAGES * CT * 8 + 64;
 constexpr int SMEM = WARPS * WARP_SMEM;
