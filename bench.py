@@ -363,6 +363,25 @@ def run_cuda(args, w, rank, world):
     if "attention" in stages:
         stages["attention"]["tensor_tflops"] = round(alg["attn_flops"] / (stage_ms["attention"] * 1e-3) / 1e12, 2)
     dom = max(stage_ms, key=stage_ms.get)
+    if b.dec and args.stage == "all":
+        # Cold decode: the same steps again (re-writing the same cache rows), each
+        # after a 256 MB write that evicts L2; only the decode calls are timed.
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        evs = []
+        for d in b.dec:
+            flush.fill_(len(evs) & 0xFF)
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            b.L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+            a1.record(stream)
+            evs.append((a0, a1))
+        torch.cuda.synchronize()
+        cold = sum(x.elapsed_time(y) for x, y in evs)
+        del flush
+        ach = alg["decode_bytes"] / (cold * 1e-3) / 1e9
+        stages["decode_cold"] = {"ms": round(cold, 4), "bound": "hbm", "achieved": round(ach, 2), "unit": "GB/s",
+                                 "frac": round(ach / pk["hbm_gbs"], 4),
+                                 "note": "each step after a 256 MB L2-evicting write"}
     ds = stages[dom]
     roofline = {"bound": ds["bound"], "achieved": ds["achieved"],
                 "peak": pk["hbm_gbs"] if ds["bound"] == "hbm" else pk["bf16_tflops_sustained"],
@@ -460,11 +479,39 @@ class OracleTimer:
         return total * w.batch, parts
 
 
+def host_cpu():
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return model, os.cpu_count()
+
+
+class one_core:
+    """Pins the calling process to one CPU (the oracle is single-threaded) and
+    restores the previous affinity on exit."""
+
+    def __enter__(self):
+        self.prev = os.sched_getaffinity(0)
+        os.sched_setaffinity(0, {min(self.prev)})
+        return self
+
+    def __exit__(self, *exc):
+        os.sched_setaffinity(0, self.prev)
+
+
 def cpu_baseline(w, rows=64, dec=2, blocks=65536):
-    ot = OracleTimer(w)
-    t, parts = ot.sample(rows, dec, blocks)
+    with one_core():
+        ot = OracleTimer(w)
+        t, parts = ot.sample(rows, dec, blocks)
     tokens = (w.n if w.prefill else 0) * w.batch + w.decode_steps * w.batch
+    model, ncpu = host_cpu()
     return {"value": round(tokens / t, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "cpu_model": model, "host_cores": ncpu,
             "sample": (f"{parts.get('fit', {}).get('rows', 0)} prefill rows stratified over [0,n) fitted by "
                        f"t(i)=a+b*floor(i/r) and extrapolated over all n; key pooling timed on {blocks} blocks "
                        f"and scaled; {dec} decode positions, scaled to {w.decode_steps} steps"),
@@ -473,12 +520,14 @@ def cpu_baseline(w, rows=64, dec=2, blocks=65536):
 
 
 def run_reference(args, w):
-    ot = OracleTimer(w)
     times = []
-    for k in range(args.warmup + args.steps):
-        t, parts = ot.sample(rows=6, dec=1, blocks=8192)
-        if k >= args.warmup:
-            times.append(t)
+    with one_core():
+        ot = OracleTimer(w)
+        for k in range(args.warmup + args.steps):
+            t, parts = ot.sample(rows=6, dec=1, blocks=8192)
+            if k >= args.warmup:
+                times.append(t)
+    model, ncpu = host_cpu()
     t = float(np.mean(times))
     tokens = (w.n if w.prefill else 0) * w.batch + w.decode_steps * w.batch
     v = tokens / t
@@ -489,6 +538,7 @@ def run_reference(args, w):
             "config": {"workload": w.name, "n": w.n, "batch": w.batch, "decode_steps": w.decode_steps,
                        "r": w.r, "K": w.K},
             "cpu_baseline": {"value": round(v, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "cpu_model": model, "host_cores": ncpu,
                              "sample": "per step: 6 stratified prefill rows (fit t(i)=a+b*floor(i/r)), key "
                                        "pooling on 8192 blocks, 1 decode position; extrapolated to the step"},
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
