@@ -40,8 +40,11 @@ __device__ __forceinline__ void cta_range(int64_t nvis, int x, int X, int64_t& l
 // CTA (0, s) appends the new token's K, V and raw indexer key to the caches
 // and, when the token closes its block, pools that block for later steps (a8;
 // the block is not visible at this position, so no CTA of this step reads
-// it). Every CTA rotates the new indexer query itself (a3', 4 warps, fp64)
-// and scores its slice of the visible pooled keys (a4) on the tensor cores:
+// it); with more than one CTA per sequence it scores nothing, so the slow
+// fp64 rotation of the pooling never delays a score slice. The other CTAs
+// rotate the new indexer query themselves (a3', fp64, from one shared table
+// of the position's angles) and score their slices of the visible pooled
+// keys (a4) on the tensor cores:
 // mma.sync m16n8k16 with A = 16 pooled keys x 16 dims and B = 16 dims x
 // (4 heads + 4 zero columns). The 128 dims are taken in a fixed permutation
 // (the same for keys and query, so every dot product is unchanged) chosen so
@@ -59,6 +62,7 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status) {
     __shared__ uint32_t hist[2048];
     __shared__ __align__(16) uint16_t qs[kIdxHeads * kIdxDim];
+    __shared__ double2 cs[kIdxDim / 2];  // (sin, cos) of the query position's angles
     pdl_wait();
     pdl_trigger();
     const int s = blockIdx.y;
@@ -92,12 +96,24 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     }
     const int64_t pcap = cap / r;
     if (p / r <= kB) return;  // every visible block is selected: no scores needed
+    const int X = gridDim.x > 1 ? (int)gridDim.x - 1 : 1;  // scoring CTAs
+    const int x = gridDim.x > 1 ? (int)blockIdx.x - 1 : 0;
+    if (x < 0) return;                                     // CTA 0 only appends and pools
     int64_t lo, hi;
-    cta_range(p / r, blockIdx.x, gridDim.x, lo, hi);
+    cta_range(p / r, x, X, lo, hi);
     if (lo >= hi) return;
-    if (warp < kIdxHeads)
-        rotate_head_warp(idx_q + ((size_t)s * kIdxHeads + warp) * kIdxDim, p, rt, qs + warp * kIdxDim, lane);
+    // The rope_dims / 2 angles of position p once per CTA (an fp64 sincos of a
+    // large argument is slow), then the 4 heads rotate from the table.
+    if (tid < rt.half) {
+        double sn, cn;
+        sincos(__dmul_rn((double)p, rt.theta[tid]), &sn, &cn);
+        cs[tid] = make_double2(sn, cn);
+    }
     for (int b = tid; b < 2048; b += DS_THREADS) hist[b] = 0u;
+    __syncthreads();
+    if (warp < kIdxHeads)
+        rotate_head_warp_tab(idx_q + ((size_t)s * kIdxHeads + warp) * kIdxDim, rt.half, cs, qs + warp * kIdxDim,
+                             lane);
     __syncthreads();
     const int g = lane >> 2, t = lane & 3;
     // B fragments: column g (head g, zero for g >= 4), k-step j.
@@ -299,11 +315,15 @@ int decode_select_ctas(int batch) {
     return std::max(1, 2 * sms / std::max(batch, 1));
 }
 
+// One wave: as many CTAs as fit on the GPU at once, split over the batch.
 int decode_score_ctas(int batch) {
-    int dev = 0, sms = 148;
+    int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return std::max(1, 4 * sms / std::max(batch, 1));
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel, DS_THREADS, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    return std::max(1, per_sm * sms / std::max(batch, 1));
 }
 
 cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* pos, const uint16_t* k,

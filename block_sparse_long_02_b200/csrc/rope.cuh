@@ -44,6 +44,28 @@ __device__ __forceinline__ void rope_lane4(double (&x)[4], int lane, int64_t pos
     }
 }
 
+// rope_lane4 with the sines and cosines of the position's angles precomputed
+// (cs[j] = (sin, cos) of pos * theta[j], j < half, the same operations as
+// rope_lane4 uses, so the results are identical).
+__device__ __forceinline__ void rope_lane4_tab(double (&x)[4], int lane, int half, const double2* cs) {
+    const int d0 = lane * 4;
+    const int qh = half >> 2;
+    const int src = (d0 < half) ? lane + qh : (d0 < 2 * half ? lane - qh : lane);
+    double y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = __shfl_sync(0xffffffffu, x[e], src);
+    if (d0 < 2 * half) {
+        const bool first = d0 < half;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int j = first ? d0 + e : d0 + e - half;
+            const double s = cs[j].x, c = cs[j].y;
+            x[e] = first ? __dsub_rn(__dmul_rn(x[e], c), __dmul_rn(y[e], s))
+                         : __dadd_rn(__dmul_rn(y[e], s), __dmul_rn(x[e], c));
+        }
+    }
+}
+
 // Loads 4 bf16 dims (8 bytes) of a row as fp64.
 __device__ __forceinline__ void load4(const uint16_t* p, double (&v)[4]) {
     const uint2 w = *reinterpret_cast<const uint2*>(p);
@@ -96,6 +118,15 @@ __device__ __forceinline__ void rotate_head_warp(const uint16_t* in, int64_t pos
     double x[4];
     load4(in + lane * 4, x);
     rope_lane4(x, lane, pos, rt);
+    store4(out + lane * 4, x);
+}
+
+// rotate_head_warp with a precomputed (sin, cos) table of the position.
+__device__ __forceinline__ void rotate_head_warp_tab(const uint16_t* in, int half, const double2* cs,
+                                                     uint16_t* out, int lane) {
+    double x[4];
+    load4(in + lane * 4, x);
+    rope_lane4_tab(x, lane, half, cs);
     store4(out + lane * 4, x);
 }
 
