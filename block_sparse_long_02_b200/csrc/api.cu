@@ -118,7 +118,7 @@ TopkWs topk_layout(const qsa::LayerDims& L, int batch, int64_t cap, int64_t nq) 
     w.fused = qsa::fused_topk_supported(L);
     // Fused path: the region after the rotated queries holds the tile counter and
     // candidate buffers; otherwise it holds one row chunk of materialised scores.
-    w.total = w.scores + align_up(w.fused ? qsa::fused_topk_ws_bytes(batch, nq) : (size_t)batch * rows * ld * 4);
+    w.total = w.scores + align_up(w.fused ? qsa::fused_topk_ws_bytes(batch, nq, L.kB) : (size_t)batch * rows * ld * 4);
     return w;
 }
 

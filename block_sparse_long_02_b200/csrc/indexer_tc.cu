@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int batch,
     int64_t nq, int64_t q_begin, int64_t pcap, int r, int kB, int* __restrict__ tile_counter,
     uint2* __restrict__ cand, int32_t* __restrict__ sel, int32_t* __restrict__ nsel,
-    int32_t* __restrict__ status) {
+    int32_t* __restrict__ status, int splits, uint2* __restrict__ split_out, int32_t* __restrict__ split_cnt) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t nqt = (nq + QT - 1) / QT;
-    const int64_t total_tiles = nqt * batch;
+    const int64_t total_tiles = nqt * batch * splits;  // work units: (query tile, key split)
 
     auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
 
@@ -610,18 +610,25 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         bool go = waited && u < total_tiles && !*abort_flag;
         if (warp >= 2) go = epi_sync_and(go);
         if (!go) break;
-        const int s = (int)(u % batch);
-        const int64_t qt = nqt - 1 - u / batch;
+        // Unit u: query tile tu = u / splits (deepest first) and key split sp, the
+        // pooled-key tiles [kt0, kt0 + ntiles) of the tile's visible range.
+        const int64_t tu = u / splits;
+        const int sp = (int)(u % splits);
+        const int s = (int)(tu % batch);
+        const int64_t qt = nqt - 1 - tu / batch;
         const int64_t j0 = qt * QT;
         const int nrows = (int)std::min<int64_t>(QT, nq - j0);
         const int64_t c_min = (q_begin + j0) / r;
         const int64_t c_max = (q_begin + j0 + nrows - 1) / r;
-        const int ntiles = c_max > kB ? (int)((c_max + BT - 1) / BT) : 0;
+        const int ntiles_all = c_max > kB ? (int)((c_max + BT - 1) / BT) : 0;
+        const int kt0 = (int)((int64_t)ntiles_all * sp / splits);
+        const int ntiles = (int)((int64_t)ntiles_all * (sp + 1) / splits) - kt0;
+        const int64_t c_range = std::min<int64_t>((int64_t)(kt0 + ntiles) * BT, c_max) - (int64_t)kt0 * BT;
         // Estimate mode (sample first) when the sweep is long enough to need it;
         // exact mode (ascending sweep, running threshold) otherwise and on a redo.
-        const int nsamp = (!redo && c_max > CAP) ? (ntiles + SAMPLE - 1) / SAMPLE : 0;
+        const int nsamp = (!redo && c_range > CAP) ? (ntiles + SAMPLE - 1) / SAMPLE : 0;
         // Sample entries kept: about 2 k_B candidates expected over the whole sweep.
-        int kA = nsamp ? (int)((2LL * kB * nsamp * BT + c_max - 1) / c_max) : kB;
+        int kA = nsamp ? (int)((2LL * kB * nsamp * BT + c_range - 1) / c_range) : kB;
         kA = max(kA, min(16, kB));
 
         if (warp == 0) {
@@ -643,7 +650,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                     mbar_expect_tx(fb, KT_BYTES);
                     for (int kh = 0; kh < 2; ++kh)
                         tma_load_2d(sK + stg * KT_BYTES + kh * (KT_BYTES / 2), &tm_k, fb, kh * 64,
-                                    krow0 + tile_at(t, nsamp) * BT, pol_k);
+                                    krow0 + (kt0 + tile_at(t, nsamp)) * BT, pol_k);
                     produced_last[stg] = round;
                 }
             }
@@ -690,7 +697,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
             uint32_t* hist = reinterpret_cast<uint32_t*>(stage);
             Pending pa{nullptr, 0.f, 0u}, pb{nullptr, 0.f, 0u};
             for (int t = 0; ok && t < ntiles; ++t, ++acc_iter) {
-                const int tt = tile_at(t, nsamp);
+                const int tt = kt0 + tile_at(t, nsamp);
                 const uint32_t b = (uint32_t)(tt * BT + qd * 32 + lane);
                 const bool masked = (int64_t)(tt + 1) * BT > c_min;
                 bool okt = true;
@@ -793,13 +800,20 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
             if (ok) {
                 int32_t* scratch = reinterpret_cast<int32_t*>(base + Q_BYTES) + ew * KMAX_FUSED;
                 for (int q = ew; q < nrows; q += EPI_WARPS) {
-                    const int cq = ctl.cvis[q];
+                    // Visible blocks of query q inside this unit's key range.
+                    const int cq = max(0, min(ctl.cvis[q], (kt0 + ntiles) * BT) - kt0 * BT);
                     const int kq = cq < kB ? cq : kB;
                     const size_t orow = (size_t)s * nq + j0 + q;
                     int32_t* out = sel + orow * kB;
-                    if (ntiles == 0) {
-                        for (int k2 = lane; k2 < kB; k2 += 32) out[k2] = k2 < kq ? k2 : -1;
-                        if (lane == 0) nsel[orow] = kq;
+                    const size_t slot = ((size_t)tu * splits + sp) * QT + q;  // split result slot
+                    if (splits > 1 && ntiles == 0) {
+                        if (lane == 0) split_cnt[slot] = 0;
+                        continue;
+                    }
+                    if (ntiles == 0) {  // every visible block is selected
+                        const int kv = min(ctl.cvis[q], kB);
+                        for (int k2 = lane; k2 < kB; k2 += 32) out[k2] = k2 < kv ? k2 : -1;
+                        if (lane == 0) nsel[orow] = kv;
                         continue;
                     }
                     if (redo && !ctl.failed[q]) continue;  // written by the estimate pass
@@ -820,6 +834,17 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                     }
                     const int m = n < kq ? n : kq;
                     if (m != kq && lane == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
+                    if (splits > 1) {
+                        // The exact top k_q of this key range, with scores, for the merge.
+                        uint2* qb = cand + (slot0 + q) * CAP;
+                        warp_keep_best(qb, sq, m, lane, hist, nullptr);
+                        __syncwarp();
+                        uint2* dst = split_out + slot * kB;
+                        for (int k2 = lane; k2 < m; k2 += 32) dst[k2] = qb[(k2 % NSEG) * SEG + k2 / NSEG];
+                        if (lane == 0) split_cnt[slot] = m;
+                        __syncwarp();
+                        continue;
+                    }
                     warp_keep_best(cand + (slot0 + q) * CAP, sq, m, lane, hist, scratch);
                     __syncwarp();
                     warp_sort(scratch, m, kB, lane);
@@ -910,9 +935,29 @@ int sm_count() {
 
 bool fused_topk_supported(const LayerDims& L) { return L.kB <= KMAX_FUSED; }
 
-size_t fused_topk_ws_bytes(int /*batch*/, int64_t /*nq*/) {
-    // tile counter (256 B) + candidate buffers of one CTA per SM.
-    return 256 + (size_t)sm_count() * QT * CAP * sizeof(uint2);
+// When there are fewer query tiles than SMs (a short chunk against a long
+// context), each tile's key range is split over several CTAs; every split
+// keeps the exact top-k of its range (with scores) and a merge selects the
+// top k_B of their union, which is the top k_B of the whole range: an entry
+// of the overall top k_B is beaten by fewer than k_B entries in its own split.
+constexpr int kMaxSplits = 8;
+
+int fused_topk_max_splits(int batch, int64_t nq) {
+    const int64_t tiles = ((nq + QT - 1) / QT) * batch;
+    const int sms = sm_count();
+    if (tiles >= sms) return 1;
+    return (int)std::min<int64_t>(kMaxSplits, (sms + tiles - 1) / tiles);
+}
+
+static size_t split_slots(int batch, int64_t nq) {
+    return (size_t)((nq + QT - 1) / QT) * batch * fused_topk_max_splits(batch, nq) * QT;
+}
+
+size_t fused_topk_ws_bytes(int batch, int64_t nq, int kB) {
+    // tile counter (256 B) + candidate buffers of one CTA per SM (+ split results).
+    size_t bytes = 256 + (size_t)sm_count() * QT * CAP * sizeof(uint2);
+    if (fused_topk_max_splits(batch, nq) > 1) bytes += split_slots(batch, nq) * ((size_t)kB * sizeof(uint2) + 4);
+    return bytes;
 }
 
 cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qrot, int64_t nq,
@@ -926,16 +971,41 @@ cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qro
         return cudaErrorInvalidValue;
     const int grid_max = sm_count();
     const int64_t tiles = ((nq + QT - 1) / QT) * batch;
-    const int grid = (int)std::min<int64_t>(grid_max, tiles);
+    // Splits: the count that minimises the makespan estimate (rounds of units
+    // over the CTAs) x (key tiles per unit of the deepest query tile), fewer
+    // splits on a tie, at least 16 key tiles per split.
+    int splits = 1;
+    const int smax = fused_topk_max_splits(batch, nq);
+    if (smax > 1) {
+        const int64_t cdeep = (q_begin + nq - 1) / L.r;
+        const int64_t kt = cdeep > L.kB ? (cdeep + BT - 1) / BT : 0;
+        int64_t best = -1;
+        for (int S = 1; S <= smax && (S == 1 || kt / S >= 16); ++S) {
+            const int64_t est = ((tiles * S + grid_max - 1) / grid_max) * ((kt + S - 1) / S);
+            if (best < 0 || est < best) {
+                best = est;
+                splits = S;
+            }
+        }
+    }
+    const int grid = (int)std::min<int64_t>(grid_max, tiles * splits);
     int* counter = reinterpret_cast<int*>(ws);
     uint2* cand = reinterpret_cast<uint2*>((char*)ws + 256);
+    uint2* split_out = nullptr;
+    int32_t* split_cnt = nullptr;
+    if (splits > 1) {
+        split_out = cand + (size_t)grid_max * QT * CAP;
+        split_cnt = reinterpret_cast<int32_t*>(split_out + split_slots(batch, nq) * L.kB);
+    }
     cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), st);
     if (e != cudaSuccess) return e;
     cudaFuncSetAttribute(fused_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     note_launch();
     fused_topk_kernel<<<grid, THREADS, SMEM, st>>>(tm_q, tm_k, batch, nq, q_begin, pcap, L.r, L.kB, counter,
-                                                   cand, sel, nsel, status);
-    return cudaGetLastError();
+                                                   cand, sel, nsel, status, splits, split_out, split_cnt);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || splits == 1) return e;
+    return launch_split_merge(L, batch, nq, q_begin, QT, splits, split_out, split_cnt, sel, nsel, st);
 }
 
 }  // namespace qsa

@@ -62,7 +62,15 @@ cudaError_t launch_index_scores(const LayerDims& L, int batch, const uint16_t* q
 
 // indexer_tc.cu: fused tcgen05 score + streaming top-k (prefill), k_B <= 512.
 bool fused_topk_supported(const LayerDims& L);
-size_t fused_topk_ws_bytes(int batch, int64_t nq);
+size_t fused_topk_ws_bytes(int batch, int64_t nq, int kB);
+// Merge of the per-split top-k lists of the fused indexer (topk.cu): for query
+// j of sequence s, the lists of its query tile's `splits` key ranges hold
+// (score bits, block) entries in split_out[(unit * QT + j % QT) * k_B ...],
+// unit = ((nqt - 1 - j / QT) * batch + s) * splits + split, with counts in
+// split_cnt; the top k_B of their union goes to sel/nsel, ascending.
+cudaError_t launch_split_merge(const LayerDims& L, int batch, int64_t nq, int64_t q_begin, int qt_rows,
+                               int splits, const uint2* split_out, const int32_t* split_cnt, int32_t* sel,
+                               int32_t* nsel, cudaStream_t st);
 cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qrot, int64_t nq,
                               int64_t q_begin, const uint16_t* pooled, int64_t cap, int32_t* sel,
                               int32_t* nsel, void* ws, int32_t* status, cudaStream_t st);

@@ -460,3 +460,17 @@ def test_fused_topk_unrepresentative_sample_is_redone_exactly(qsa):
         ref = o.row(i, iq_bits[i], pooled)
         tol = score_tol(o.rotate_query(iq_bits[i], i), pooled, ref["scores"])
         check_selection(g[i], gn[i], ref["scores"], tol, o.k_blocks, f"row {i}")
+
+
+def test_fused_topk_split_key_ranges(qsa):
+    """A short chunk against a long context (6 query tiles, ~15K visible blocks):
+    the fused indexer splits each tile's key range over several CTAs and merges
+    the per-split top-k lists; every row must still be the exact selection."""
+    w = synth.Workload(name="t", n=60300, batch=2, K=2048, q_heads=4, kv_heads=1, base_seed=0x5B1)
+    n0 = qsa.qsa_launch_count()
+    cfg, res = run_prefill(qsa, w, q_begin=60000, nq=300)
+    # prefix compress, compress, rotate, fused indexer, split merge, attention
+    assert qsa.qsa_launch_count() - n0 == 6
+    for s in range(w.batch):
+        check_rows(w, cfg, res, range(60000, 60300), s=s, q_begin=60000, attention=False)
+        check_rows(w, cfg, res, [60000, 60001, 60150, 60299], s=s, q_begin=60000)
