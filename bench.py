@@ -168,6 +168,21 @@ def traffic_for(stage: str):
     return None
 
 
+# ----------------------------------------------------------------------------- replicas
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (the job's time is its slowest replica's)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(tokens_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
+
+
 # ----------------------------------------------------------------------------- CUDA arm
 class Bench:
     def __init__(self, w, device, stage="all"):
@@ -337,10 +352,7 @@ def run_cuda(args, w, rank, world):
         if name != "start" and prev is not None:
             stage_ms[name] = stage_ms.get(name, 0.0) + prev.elapsed_time(e) / args.steps
         prev = e
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
 
     alg = algorithmic(w)
     pk = peaks()
@@ -389,7 +401,7 @@ def run_cuda(args, w, rank, world):
                 "peak_source": pk["source"] + (" (sustained bf16)" if ds["bound"] == "tensor" else " (copy)")}
 
     res = {
-        "metric": METRIC, "value": round(tokens * world / (ms * 1e-3), 2), "unit": "tokens/s",
+        "metric": METRIC, "value": round(job_value(tokens, ms, world), 2), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded counter-based N(0,1) bf16 inputs with planted needle blocks",
@@ -408,11 +420,8 @@ def run_cuda(args, w, rank, world):
         res["decode_tokens_per_s"] = round(alg["decode_tokens"] / (stage_ms["decode"] * 1e-3), 1)
     if not args.no_e2e:
         e_ms, h2d, d2h = b.e2e(max(1, min(args.steps, 2)), 1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        res["e2e"] = {"value": round(tokens * world / (e_ms * 1e-3), 2), "unit": "tokens/s",
+        e_ms = max_over_ranks(e_ms, world, dev)
+        res["e2e"] = {"value": round(job_value(tokens, e_ms, world), 2), "unit": "tokens/s",
                       "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     return res
 
