@@ -26,7 +26,7 @@ OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 
 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
-           "qsa_launch_count", "qsa_decode_step_noalloc"]
+           "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection"]
 
 
 class QSAError(RuntimeError):
@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
         h.qsa_last_error.argtypes = []
         h.qsa_launch_count.restype = ctypes.c_uint64
         h.qsa_launch_count.argtypes = []
+        h.qsa_set_fault_injection.restype = ctypes.c_int
+        h.qsa_set_fault_injection.argtypes = [ctypes.c_int32, ctypes.c_double]
         _lib_handle = h
     return _lib_handle
 
@@ -205,3 +207,9 @@ def qsa_last_error() -> str:
 def qsa_launch_count() -> int:
     """Kernel launches issued by libqsa.so so far in this process."""
     return int(lib().qsa_launch_count())
+
+
+def qsa_set_fault_injection(mode: int, wait_seconds: float = 0.0) -> None:
+    """Tests of the failure path only (see include/qsa.h): mode 1 makes the fused
+    top-k's bounded wait run out after wait_seconds; mode 0 restores normal use."""
+    _check(lib().qsa_set_fault_injection(int(mode), float(wait_seconds)))

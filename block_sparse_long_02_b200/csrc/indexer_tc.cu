@@ -30,6 +30,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "kernels.h"
@@ -52,7 +53,7 @@ constexpr int THREADS = 64 + EPI_THREADS;
 static_assert(QT / EPI_WARPS <= 32, "one lane per query of a warp in the compaction check");
 constexpr int Q_BYTES = QT * kIdxHeads * 256;  // 131072
 constexpr int KT_BYTES = BT * 256;             // 32768
-constexpr uint64_t WAIT_NS = 10000000000ull;  // 10 s
+constexpr uint64_t WAIT_NS = 10000000000ull;  // 10 s: the limit of every wait in normal use
 
 struct Ctl {
     uint64_t full[STAGES], empty[STAGES];
@@ -100,15 +101,16 @@ __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
     return ok != 0;
 }
 // Waits for the phase of parity `parity` to complete. Returns false (and sets
-// the CTA's abort flag) after WAIT_NS, or at once if another warp aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag) {
+// the CTA's abort flag) after limit_ns, or at once if another warp aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
     if (mbar_try(a, parity)) return true;
     const uint64_t t0 = gtime();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try(a, parity)) return true;
         if ((it & 63u) == 0u) {
             if (*abort_flag) return false;
-            if (gtime() - t0 > WAIT_NS) {
+            if (gtime() - t0 > limit_ns) {
                 *abort_flag = 1;
                 return false;
             }
@@ -542,7 +544,8 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int batch,
     int64_t nq, int64_t q_begin, int64_t pcap, int r, int kB, int* __restrict__ tile_counter,
     uint2* __restrict__ cand, int32_t* __restrict__ sel, int32_t* __restrict__ nsel,
-    int32_t* __restrict__ status, int splits, uint2* __restrict__ split_out, int32_t* __restrict__ split_cnt) {
+    int32_t* __restrict__ status, int splits, uint2* __restrict__ split_out, int32_t* __restrict__ split_cnt,
+    uint64_t wait_ns, int fault_mode) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
@@ -603,7 +606,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         mbar_arrive(bar(ctl.cta_bar));
         // Warp-uniform outcome (warp collectives follow); for the epilogue warps
         // also uniform across the group, which meets at named barriers.
-        const bool waited = __all_sync(0xffffffffu, mbar_wait(bar(ctl.cta_bar), cta_phase, abort_flag));
+        const bool waited = __all_sync(0xffffffffu, mbar_wait(bar(ctl.cta_bar), cta_phase, abort_flag, wait_ns));
         cta_phase ^= 1;
         const int64_t u = waited ? (int64_t)ctl.tile[iter & 1] : total_tiles;
         const bool redo = waited && ctl.redo[iter & 1] != 0;
@@ -642,10 +645,14 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                         tma_load_2d(sQ + kh * (Q_BYTES / 2) + rh * (Q_BYTES / 4), &tm_q, qb, kh * 64,
                                     qrow + rh * 256, pol_q);
                 const int krow0 = (int)((int64_t)s * pcap);
+                // Fault injection (tests of the failure path only): the CTA's first
+                // unit gets no key tiles, so the MMA warp's wait runs out.
+                const bool withhold = fault_mode == 1 && iter == 0;
                 for (int t = 0; t < ntiles; ++t, ++kring) {
                     const int stg = (int)(kring % STAGES);
                     const uint32_t round = kring / STAGES;
-                    if (!mbar_wait(bar(ctl.empty[stg]), (round & 1u) ^ 1u, abort_flag)) break;
+                    if (!mbar_wait(bar(ctl.empty[stg]), (round & 1u) ^ 1u, abort_flag, wait_ns)) break;
+                    if (withhold) continue;
                     const uint32_t fb = bar(ctl.full[stg]);
                     mbar_expect_tx(fb, KT_BYTES);
                     for (int kh = 0; kh < 2; ++kh)
@@ -657,13 +664,13 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         } else if (warp == 1) {
             // ------------------------------------------------ MMA issuer
             if (lane == 0 && ntiles > 0) {
-                bool ok = mbar_wait(bar(ctl.q_full), q_iter & 1u, abort_flag);
+                bool ok = mbar_wait(bar(ctl.q_full), q_iter & 1u, abort_flag, wait_ns);
                 for (int t = 0; ok && t < ntiles; ++t, ++kring, ++acc_iter) {
                     const int stg = (int)(kring % STAGES);
-                    if (!(ok = mbar_wait(bar(ctl.full[stg]), (kring / STAGES) & 1u, abort_flag))) break;
+                    if (!(ok = mbar_wait(bar(ctl.full[stg]), (kring / STAGES) & 1u, abort_flag, wait_ns))) break;
                     tc_fence_after();
                     for (int h = 0; h < 2; ++h) {
-                        if (!(ok = mbar_wait(bar(ctl.acc_empty[h]), (acc_iter & 1u) ^ 1u, abort_flag))) break;
+                        if (!(ok = mbar_wait(bar(ctl.acc_empty[h]), (acc_iter & 1u) ^ 1u, abort_flag, wait_ns))) break;
                         tc_fence_after();
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t koff = (kk >> 2) * (KT_BYTES / 2) + (kk & 3) * 32;
@@ -703,7 +710,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
                 bool okt = true;
                 for (int h = 0; h < 2; ++h) {
                     const bool okh =
-                        __all_sync(0xffffffffu, mbar_wait(bar(ctl.acc_full[h]), acc_iter & 1u, abort_flag));
+                        __all_sync(0xffffffffu, mbar_wait(bar(ctl.acc_full[h]), acc_iter & 1u, abort_flag, wait_ns));
                     if (okh) {  // warp-uniform
                         uint32_t v[128];
                         tc_fence_after();
@@ -872,7 +879,7 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
         // before the CTA's shared memory goes away.
         for (int stg = 0; stg < STAGES; ++stg)
             if (produced_last[stg] != 0xFFFFFFFFu)
-                mbar_wait(smem_u32(&ctl.empty[stg]), produced_last[stg] & 1u, abort_flag);
+                mbar_wait(smem_u32(&ctl.empty[stg]), produced_last[stg] & 1u, abort_flag, wait_ns);
     }
     if (*abort_flag) {
         if (tid == 0) flag_status(status, 6 /* QSA_ERR_TIMEOUT */);
@@ -881,12 +888,12 @@ __global__ void __launch_bounds__(THREADS, 1) fused_topk_kernel(
             volatile int no_abort = 0;
             for (int stg = 0; stg < STAGES; ++stg)
                 if (produced_last[stg] != 0xFFFFFFFFu)
-                    mbar_wait(smem_u32(&ctl.full[stg]), produced_last[stg] & 1u, &no_abort);
+                    mbar_wait(smem_u32(&ctl.full[stg]), produced_last[stg] & 1u, &no_abort, wait_ns);
         }
         if (warp == 1 && lane == 0) {
             volatile int no_abort = 0;
             umma_commit(smem_u32(&ctl.mma_done));
-            mbar_wait(smem_u32(&ctl.mma_done), 0, &no_abort);
+            mbar_wait(smem_u32(&ctl.mma_done), 0, &no_abort, wait_ns);
         }
     }
     tc_fence_before();
@@ -941,6 +948,15 @@ bool fused_topk_supported(const LayerDims& L) { return L.kB <= KMAX_FUSED; }
 // top k_B of their union, which is the top k_B of the whole range: an entry
 // of the overall top k_B is beaten by fewer than k_B entries in its own split.
 constexpr int kMaxSplits = 8;
+
+// Fault injection for tests of the failure path (off unless a test sets it).
+std::atomic<int> g_fault_mode{0};
+std::atomic<uint64_t> g_fault_wait_ns{WAIT_NS};
+
+void set_fault_injection(int mode, uint64_t wait_ns) {
+    g_fault_wait_ns.store(wait_ns, std::memory_order_relaxed);
+    g_fault_mode.store(mode, std::memory_order_relaxed);
+}
 
 int fused_topk_max_splits(int batch, int64_t nq) {
     const int64_t tiles = ((nq + QT - 1) / QT) * batch;
@@ -1001,8 +1017,11 @@ cudaError_t launch_fused_topk(const LayerDims& L, int batch, const uint16_t* qro
     if (e != cudaSuccess) return e;
     cudaFuncSetAttribute(fused_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     note_launch();
+    const int fmode = g_fault_mode.load(std::memory_order_relaxed);
+    const uint64_t wait_ns = fmode ? g_fault_wait_ns.load(std::memory_order_relaxed) : WAIT_NS;
     fused_topk_kernel<<<grid, THREADS, SMEM, st>>>(tm_q, tm_k, batch, nq, q_begin, pcap, L.r, L.kB, counter,
-                                                   cand, sel, nsel, status, splits, split_out, split_cnt);
+                                                   cand, sel, nsel, status, splits, split_out, split_cnt, wait_ns,
+                                                   fmode);
     e = cudaGetLastError();
     if (e != cudaSuccess || splits == 1) return e;
     return launch_split_merge(L, batch, nq, q_begin, QT, splits, split_out, split_cnt, sel, nsel, st);

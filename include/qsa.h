@@ -228,6 +228,19 @@ const char* qsa_last_error(void);
  * threads, all entry points). Used to count device work in benchmarks. */
 uint64_t qsa_launch_count(void);
 
+/* Fault injection, for tests of the failure path (the pages have no
+ * counterpart; SURVEY-style host-side fault tests need a wait that runs out
+ * without faulting the GPU). Process-wide, off by default.
+ *   mode 0: normal operation (every bounded device wait gives up after 10 s).
+ *   mode 1: the fused qsa_topk_blocks path (k_B <= 512) withholds the pooled-key
+ *           tiles of each CTA's first unit of work, so the MMA's bounded wait
+ *           runs out after wait_seconds (0 < wait_seconds <= 10): the kernel
+ *           records QSA_ERR_TIMEOUT in the workspace status, drains its own
+ *           copies and MMAs, frees its tensor memory and returns; the selection
+ *           it leaves is incomplete, and the CUDA context stays usable.
+ * Returns QSA_ERR_INVALID_ARG for another mode or wait. */
+qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds);
+
 #ifdef __cplusplus
 }
 #endif

@@ -61,3 +61,16 @@ def test_null_and_capacity_errors_launch_nothing(qsa):
     assert st == 4
     lib.qsa_last_error.restype = ctypes.c_char_p
     assert b"cap" in lib.qsa_last_error()
+
+
+def test_fault_injection_arguments_are_validated(qsa):
+    """Host-side checks of the failure-path switch (no device work)."""
+    for mode, wait, ok in [(2, 0.1, False), (-1, 0.1, False), (1, 0.0, False), (1, 11.0, False),
+                           (1, float("nan"), False), (1, 0.5, True), (0, 0.0, True)]:
+        if ok:
+            qsa.qsa_set_fault_injection(mode, wait)
+        else:
+            with pytest.raises(qsa.QSAError) as e:
+                qsa.qsa_set_fault_injection(mode, wait)
+            assert e.value.status == 1, (mode, wait)
+    qsa.qsa_set_fault_injection(0)

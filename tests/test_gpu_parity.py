@@ -474,3 +474,43 @@ def test_fused_topk_split_key_ranges(qsa):
     for s in range(w.batch):
         check_rows(w, cfg, res, range(60000, 60300), s=s, q_begin=60000, attention=False)
         check_rows(w, cfg, res, [60000, 60001, 60150, 60299], s=s, q_begin=60000)
+
+
+def test_forced_timeout_is_reported_and_the_context_survives(qsa):
+    """Failure path of the fused indexer, without a GPU fault: with fault
+    injection the key tiles of each CTA's first unit are withheld, the MMA
+    warp's bounded wait runs out (0.25 s), the kernel reports QSA_ERR_TIMEOUT
+    in the workspace status, drains and returns; the next call is normal."""
+    import time
+
+    n = 4096 + 8
+    w = synth.Workload(name="t", n=n, K=2048, q_heads=4, kv_heads=1, base_seed=0xE1)
+    cfg, L = _layer(qsa, w, n)
+    _fill_caches(w, L, n)
+    L.compress(0, n // 4)
+    iq = dev_full(w, "idx_q", n).view(1, n, 4, 128).contiguous()
+    sel = torch.empty(1, n, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(1, n, dtype=torch.int32, device="cuda")
+    ws = L.workspace(qsa.OP_TOPK_BLOCKS, n)
+    assert qsa.qsa_workspace_status(ws) == 0
+    qsa.qsa_set_fault_injection(1, 0.25)
+    try:
+        t0 = time.time()
+        qsa.qsa_topk_blocks(cfg, 1, iq, 0, n, L.pooled, n, None, 0, sel, nsel, ws)
+        torch.cuda.synchronize()
+        elapsed = time.time() - t0
+    finally:
+        qsa.qsa_set_fault_injection(0)
+    assert qsa.qsa_workspace_status(ws) == 6  # QSA_ERR_TIMEOUT (read and cleared)
+    assert elapsed >= 0.2
+    qsa.qsa_topk_blocks(cfg, 1, iq, 0, n, L.pooled, n, None, 0, sel, nsel, ws)
+    torch.cuda.synchronize()
+    assert qsa.qsa_workspace_status(ws) == 0
+    o = _oracle(w, cfg)
+    pooled = bits(L.pooled)[0]
+    iq_bits = bits(iq)[0].reshape(n, 4, 128)
+    g, gn = sel.cpu().numpy()[0], nsel.cpu().numpy()[0]
+    for i in [100, 2051, 3000, n - 1]:
+        ref = o.row(i, iq_bits[i], pooled)
+        tol = score_tol(o.rotate_query(iq_bits[i], i), pooled, ref["scores"])
+        check_selection(g[i], gn[i], ref["scores"], tol, o.k_blocks, f"row {i}")
