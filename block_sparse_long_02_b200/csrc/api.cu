@@ -123,7 +123,7 @@ TopkWs topk_layout(const qsa::LayerDims& L, int batch, int64_t cap, int64_t nq) 
 }
 
 struct DecodeWs {
-    size_t scores, sel, nsel, part, hist, counters, winners, cand, total;
+    size_t scores, sel, nsel, hist, counters, winners, cand, total;
 };
 
 DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
@@ -131,15 +131,13 @@ DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
     // status header: it must be zero when a step starts, and every step leaves
     // it zero.
     DecodeWs w;
-    const int S = qsa::decode_attention_splits(L);
     w.hist = qsa::kWsHeader;
     w.counters = w.hist + align_up((size_t)batch * 2048 * 4);
     w.scores = w.counters + align_up((size_t)batch * 4 * 4);
     // (w.scores == qsa::decode_state_bytes(batch))
     w.sel = w.scores + align_up((size_t)batch * std::max<int64_t>(1, cap / L.r) * 4);
     w.nsel = w.sel + align_up((size_t)batch * L.kB * 4);
-    w.part = w.nsel + align_up((size_t)batch * 4);
-    w.winners = w.part + align_up((size_t)batch * L.q_heads * S * 132 * 4);
+    w.winners = w.nsel + align_up((size_t)batch * 4);
     w.cand = w.winners + align_up((size_t)batch * L.kB * 4);
     w.total = w.cand + align_up((size_t)batch * qsa::kDecodeCand * 8);
     return w;
@@ -338,7 +336,6 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     float* scores = reinterpret_cast<float*>(base + w.scores);
     int32_t* sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(base + w.sel);
     int32_t* nsel = nsel_out ? nsel_out : reinterpret_cast<int32_t*>(base + w.nsel);
-    float* part = reinterpret_cast<float*>(base + w.part);
     qsa::DecodeSelWs sw;
     sw.hist = reinterpret_cast<uint32_t*>(base + w.hist);
     sw.counters = reinterpret_cast<int32_t*>(base + w.counters);
@@ -348,9 +345,10 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     TRY(cuda_check(qsa::launch_decode_score(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
                                             pooled, cap, rms_w, scores, sw, status, st),
                    "decode score"));
-    TRY(cuda_check(qsa::launch_decode_select(L, batch, pos, cap, scores, sw, sel, nsel, st), "decode select"));
+    TRY(cuda_check(qsa::launch_decode_select(L, batch, pos, cap, scores, sw, sel, nsel, status, st),
+                   "decode select"));
     return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel,
-                                                   nsel, part, out, st),
+                                                   nsel, out, st),
                       "decode attention");
 }
 

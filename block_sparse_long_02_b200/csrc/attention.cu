@@ -29,6 +29,7 @@ constexpr int STAGES = 2;
 constexpr int STAGE_BYTES = CT * 256 * 2; // K and V rows
 constexpr int WARP_SMEM = STAGES * STAGE_BYTES + STAGES * CT * 8 + 64;
 constexpr int SMEM = WARPS * WARP_SMEM;
+constexpr int kMaxCluster = 16;           // decode CTAs per (sequence, kv head)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -38,8 +39,10 @@ struct Work {
     const uint16_t* vc;
     const int32_t* sel;    // selection row
     int64_t i;             // query position
-    int nsel;              // valid count (clamped)
-    int u0, u1;            // unit range, units [0, nsel) = selected blocks, nsel = tail
+    int64_t cur;           // its block, i / r
+    int nsel;              // valid selection entries (clamped)
+    int tail_unit;         // the unit that stands for the current block's tail
+    int u0, u1;            // unit range; unit u != tail_unit is selection entry u if u < nsel, else empty
     int g;                 // kv head
     int G;                 // query heads per kv head
     int kv_heads;
@@ -70,26 +73,32 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
     return d;
 }
 
+// Query fragments (B operand of S^T = K Q^T) of the G heads at q: column =
+// head 8 nt + g, k rows = dims 16 ks + 2 t (+1) and 16 ks + 8 + 2 t (+1).
 template <int NT>
-__device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lane, WarpState<NT>& st) {
-    uint16_t* ring = reinterpret_cast<uint16_t*>(wsm);
-    int64_t* tok = reinterpret_cast<int64_t*>(wsm + STAGES * STAGE_BYTES);  // [STAGES][CT]
-    uint32_t* vmask = reinterpret_cast<uint32_t*>(wsm + STAGES * STAGE_BYTES + STAGES * CT * 8);
-    const uint32_t ring_s = smem_u32(ring);
+__device__ __forceinline__ void load_q_frags(const uint16_t* q, int G, int lane, uint32_t (&qb)[NT][8][2]) {
     const int g = lane >> 2, t = lane & 3;
-
-    // Query fragments (B operand of S^T = K Q^T): column = head 8 nt + g,
-    // k rows = dims 16 ks + 2 t (+1) and 16 ks + 8 + 2 t (+1).
-    uint32_t qb[NT][8][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int h = 8 * nt + g;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-            qb[nt][ks][0] = h < w.G ? *reinterpret_cast<const uint32_t*>(w.q + h * kHeadDim + ks * 16 + 2 * t) : 0u;
-            qb[nt][ks][1] = h < w.G ? *reinterpret_cast<const uint32_t*>(w.q + h * kHeadDim + ks * 16 + 8 + 2 * t) : 0u;
+            qb[nt][ks][0] = h < G ? *reinterpret_cast<const uint32_t*>(q + h * kHeadDim + ks * 16 + 2 * t) : 0u;
+            qb[nt][ks][1] = h < G ? *reinterpret_cast<const uint32_t*>(q + h * kHeadDim + ks * 16 + 8 + 2 * t) : 0u;
         }
     }
+}
+
+// The warp's units [u0, u1) against the query fragments qb. sel_lane: lane l
+// holds selection entry u0 + l when that unit is a selection entry (any
+// value otherwise); later entries are read when their chunk is issued.
+template <int NT>
+__device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lane, const uint32_t (&qb)[NT][8][2],
+                                            int32_t sel_lane, WarpState<NT>& st) {
+    uint16_t* ring = reinterpret_cast<uint16_t*>(wsm);
+    uint32_t* vmask = reinterpret_cast<uint32_t*>(wsm + STAGES * STAGE_BYTES + STAGES * CT * 8);
+    const uint32_t ring_s = smem_u32(ring);
+    const int g = lane >> 2;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -102,46 +111,39 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
 
     const int64_t ntok = (int64_t)(w.u1 - w.u0) * w.r;
     const int nchunks = (int)((ntok + CT - 1) / CT);
-    const int64_t cur = w.i / w.r;
+    const int64_t cur = w.cur;
     const int64_t row_stride = (int64_t)w.kv_heads * kHeadDim;
-    // The warp's first 32 selection entries in one round trip (lane u holds
-    // unit u0 + u); later units, if any, are read when their chunk is issued.
-    const int32_t sel_lane = (w.u0 + lane < w.u1 && w.u0 + lane < w.nsel) ? w.sel[w.u0 + lane] : -1;
 
+    const int ntok_i = (int)ntok;
+    // Chunk c: lane l (and l + 16) resolves token l of the chunk; the valid
+    // mask is a ballot and the row addresses come by shuffle.
     auto issue = [&](int c) {
         const int stg = c % STAGES;
-        {
-            const int64_t p = (int64_t)c * CT + (lane & (CT - 1));  // lanes >= CT mirror lanes < CT
-            const int u = w.u0 + (int)(p / w.r);
-            const int32_t b_pre = __shfl_sync(0xffffffffu, sel_lane, (u - w.u0) & 31);
-            int64_t tk = -1;
-            if (p < ntok) {
-                const int e = (int)(p % w.r);
-                if (u < w.nsel) {
-                    const int32_t b = u - w.u0 < 32 ? b_pre : w.sel[u];
-                    if (b >= 0 && (int64_t)b < cur) tk = (int64_t)b * w.r + e;
-                } else {
-                    const int64_t tt = cur * w.r + e;
-                    if (tt <= w.i) tk = tt;
-                }
+        const int pl = c * CT + (lane & (CT - 1));  // lanes >= CT mirror lanes < CT
+        const int u = w.u0 + pl / w.r;
+        const int32_t b_pre = __shfl_sync(0xffffffffu, sel_lane, (u - w.u0) & 31);
+        int32_t tk = -1;  // token (the cache capacity is below 2^31 tokens)
+        if (pl < ntok_i) {
+            const int e = pl % w.r;
+            if (u == w.tail_unit) {
+                const int64_t tt = cur * w.r + e;
+                if (tt <= w.i) tk = (int32_t)tt;
+            } else if (u < w.nsel) {
+                const int32_t b = u - w.u0 < 32 ? b_pre : w.sel[u];
+                if (b >= 0 && (int64_t)b < cur) tk = b * w.r + e;
             }
-            if (lane < CT) tok[stg * CT + lane] = tk;
         }
-        __syncwarp();
-        if (lane == 0) {
-            uint32_t m = 0;
-            for (int k = 0; k < CT; ++k) m |= (tok[stg * CT + k] >= 0 ? 1u : 0u) << k;
-            vmask[stg] = m;
-        }
+        const uint32_t valid = __ballot_sync(0xffffffffu, tk >= 0) & ((1u << CT) - 1u);
+        if (lane == 0) vmask[stg] = valid;
         const uint32_t kbase = ring_s + stg * STAGE_BYTES;
         const uint32_t vbase = kbase + CT * 256;
 #pragma unroll
         for (int k = 0; k < (CT * 16) / 32; ++k) {
             const int idx = lane + k * 32;
             const int row = idx >> 4, ch = idx & 15;
-            const int64_t tk = tok[stg * CT + row];
-            const bool ok = tk >= 0;
-            const size_t off = (size_t)(ok ? tk : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 8;
+            const int32_t tkr = __shfl_sync(0xffffffffu, tk, row);
+            const bool ok = tkr >= 0;
+            const size_t off = (size_t)(ok ? tkr : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 8;
             cp_async16_zfill(kbase + swz256(row, ch), w.kc + off, ok);
             cp_async16_zfill(vbase + swz256(row, ch), w.vc + off, ok);
         }
@@ -173,12 +175,24 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
 #pragma unroll
+        // (two independent accumulation chains over the k-steps, summed after)
+        float s2[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s2[nt][e] = 0.f;
+#pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4(kbase + swz256(krow, ks * 2 + kch), a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+            for (int nt = 0; nt < NT; ++nt)
+                mma_bf16_16816((ks & 1) ? s2[nt] : s[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
         // Online softmax per head (log2 domain); a head's 16 tokens sit in the
         // 8 lanes with the same t.
         const bool v0 = (valid >> g) & 1u, v1 = (valid >> (g + 8)) & 1u;
@@ -194,9 +208,9 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                 const float m_new = fmaxf(st.m[nt][e], mx);
-                const float corr = (m_new == -INFINITY) ? 1.f : exp2f(st.m[nt][e] - m_new);
-                const float p0 = (x0 == -INFINITY) ? 0.f : exp2f(x0 - m_new);
-                const float p1 = (x1 == -INFINITY) ? 0.f : exp2f(x1 - m_new);
+                const float corr = (m_new == -INFINITY) ? 1.f : ex2_approx(st.m[nt][e] - m_new);
+                const float p0 = (x0 == -INFINITY) ? 0.f : ex2_approx(x0 - m_new);
+                const float p1 = (x1 == -INFINITY) ? 0.f : ex2_approx(x1 - m_new);
                 st.l[nt][e] = st.l[nt][e] * corr + (p0 + p1);
                 st.m[nt][e] = m_new;
                 s[nt][e] = p0;
@@ -323,7 +337,9 @@ __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
     w.vc = vc + (size_t)s * cap * kv_heads * kHeadDim;
     w.sel = sel + (size_t)row * kB;
     w.i = i;
+    w.cur = i / r;
     w.nsel = ns;
+    w.tail_unit = ns;
     w.u0 = (int)((int64_t)units * split / NS);
     w.u1 = (int)((int64_t)units * (split + 1) / NS);
     w.g = g;
@@ -333,8 +349,11 @@ __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
     w.scale_log2 = scale_log2;
 
     uint8_t* wsm = smem + warp * WARP_SMEM;
+    uint32_t qb[NT][8][2];
+    load_q_frags<NT>(w.q, G, lane, qb);
+    const int32_t sel_lane = (w.u0 + lane < w.u1 && w.u0 + lane < ns) ? w.sel[w.u0 + lane] : -1;
     WarpState<NT> st;
-    warp_attend<NT>(w, wsm, lane, st);
+    warp_attend<NT>(w, wsm, lane, qb, sel_lane, st);
 
     if (NS > 1) {
         // Splits > 0 park their state in their own smem; split 0 merges.
@@ -350,53 +369,10 @@ __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
                       lse ? lse + (size_t)row * q_heads + (size_t)g * G : nullptr, lane);
 }
 
-// Decode: one warp per (sequence, kv head, split); partial states to `part`
-// laid out [batch][q_heads][S][132] = (o[128], m, l, pad, pad), log2 domain.
+// Writes a warp state in the head-major layout: o[h][128] (unnormalised),
+// then m[h], then l[h] (log2 domain), heads h < G.
 template <int NT>
-__global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
-    const uint16_t* __restrict__ q, const int64_t* __restrict__ pos,
-    const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc, int64_t cap,
-    const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel, float* __restrict__ part,
-    int batch, int q_heads, int kv_heads, int r, int kB, int S, float scale_log2) {
-    pdl_wait();
-    pdl_trigger();
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t item = (int64_t)blockIdx.x * WARPS + warp;
-    if (item >= (int64_t)batch * kv_heads * S) return;
-    const int split = (int)(item % S);
-    const int g = (int)((item / S) % kv_heads);
-    const int s = (int)(item / ((int64_t)S * kv_heads));
-    const int G = q_heads / kv_heads;
-    const int64_t p = pos[s];
-    float* dst = part + (((size_t)s * q_heads + (size_t)g * G) * S + split) * 132;
-    if (p < 0 || p >= cap) {
-        // Skipped sequence: an empty partial (m = -inf, l = 0).
-        for (int row = 0; row < G; ++row) {
-            float* d = dst + (size_t)row * S * 132;
-            for (int k = lane; k < 132; k += 32) d[k] = k == 128 ? -INFINITY : 0.f;
-        }
-        return;
-    }
-    int ns = nsel[s];
-    ns = ns < 0 ? 0 : (ns > kB ? kB : ns);
-    const int units = ns + 1;
-    Work w;
-    w.q = q + ((size_t)s * q_heads + (size_t)g * G) * kHeadDim;
-    w.kc = kc + (size_t)s * cap * kv_heads * kHeadDim;
-    w.vc = vc + (size_t)s * cap * kv_heads * kHeadDim;
-    w.sel = sel + (size_t)s * kB;
-    w.i = p;
-    w.nsel = ns;
-    w.u0 = (int)((int64_t)units * split / S);
-    w.u1 = (int)((int64_t)units * (split + 1) / S);
-    w.g = g;
-    w.G = G;
-    w.kv_heads = kv_heads;
-    w.r = r;
-    w.scale_log2 = scale_log2;
-    WarpState<NT> st;
-    warp_attend<NT>(w, smem + warp * WARP_SMEM, lane, st);
+__device__ __forceinline__ void store_state_hd(const WarpState<NT>& st, int G, float* dst, int lane) {
     const int gq = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -404,53 +380,130 @@ __global__ void __launch_bounds__(WARPS * 32) decode_attention_kernel(
         for (int e = 0; e < 2; ++e) {
             const int h = 8 * nt + 2 * t + e;
             if (h >= G) continue;
-            float* d = dst + (size_t)h * S * 132;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                d[16 * i + gq] = st.o[nt][i][e];
-                d[16 * i + gq + 8] = st.o[nt][i][2 + e];
+                dst[h * kHeadDim + 16 * i + gq] = st.o[nt][i][e];
+                dst[h * kHeadDim + 16 * i + gq + 8] = st.o[nt][i][2 + e];
             }
             if (gq == 0) {
-                d[128] = st.m[nt][e];
-                d[129] = st.l[nt][e];
+                dst[G * kHeadDim + h] = st.m[nt][e];
+                dst[G * kHeadDim + G + h] = st.l[nt][e];
             }
         }
 }
 
-// Combine the S partials of each (sequence, head): one CTA of 4 warps per
-// head; every warp finds the partials' maximum itself (two loads per lane),
-// warp w sums partials w, w + 4, ... for all 128 dims (lane: dims lane + 32 j),
-// with every load of the warp issued before the first use, and the four warp
-// sums meet in shared memory.
-__global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ part, int S,
-                                                            uint16_t* __restrict__ out) {
+// Bytes of the decode kernel's receive area: C slices of the G x 128 outputs
+// plus every CTA's m and l per head.
+__host__ __device__ constexpr int decode_recv_bytes(int G, int C) { return (G * kHeadDim + 2 * G * C) * 4; }
+
+// Decode: one thread-block cluster of C CTAs of DW warps per (sequence, kv
+// head); warp w of CTA c takes unit split DW c + w of S = DW C. The units are the k_B
+// selection entries (entry u counts if u < nsel) and, as unit k_B, the tail,
+// so a split's entries are known before nsel is: the query and the position
+// (inputs of the step) are read before the dependency wait, and nsel and the
+// selection entries right after it, in one round trip. The four warp states
+// of a CTA are merged element-wise by all its threads; CTA c then owns the
+// outputs [c E / C, (c + 1) E / C) of the E = G x 128 and every CTA pushes its
+// merged slice for them into c's shared memory (remote stores, no remote
+// loads); after one cluster barrier each CTA finishes its slice locally.
+template <int NT, int DW>
+__global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
+    const uint16_t* __restrict__ q, const int64_t* __restrict__ pos,
+    const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc, int64_t cap,
+    const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel, uint16_t* __restrict__ out,
+    int q_heads, int kv_heads, int r, int kB, float scale_log2) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    cluster_arrive_relaxed();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int C = (int)gridDim.x;        // the cluster spans the grid's x dimension
+    const int rank = (int)blockIdx.x;    // = rank in the cluster
+    const int g = (int)blockIdx.y, s = (int)blockIdx.z;
+    const int G = q_heads / kv_heads;
+    const int S = C * DW, split = rank * DW + warp;
+    const int units = kB + 1;
+    Work w;
+    w.q = q + ((size_t)s * q_heads + (size_t)g * G) * kHeadDim;
+    w.kc = kc + (size_t)s * cap * kv_heads * kHeadDim;
+    w.vc = vc + (size_t)s * cap * kv_heads * kHeadDim;
+    w.sel = sel + (size_t)s * kB;
+    w.tail_unit = kB;
+    w.u0 = (int)((int64_t)units * split / S);
+    w.u1 = (int)((int64_t)units * (split + 1) / S);
+    w.g = g;
+    w.G = G;
+    w.kv_heads = kv_heads;
+    w.r = r;
+    w.scale_log2 = scale_log2;
+    // Inputs of the step: the kernels before this one in the step do not
+    // write them, and they were complete before the step's first kernel ran.
+    const int64_t p = pos[s];
+    uint32_t qb[NT][8][2];
+    load_q_frags<NT>(w.q, G, lane, qb);
+    uint8_t* wsm = smem + warp * WARP_SMEM;
+    WarpState<NT> st;
+    w.cur = p / r;
     pdl_wait();
     pdl_trigger();
-    __shared__ float so[4][128];
-    __shared__ float sl[4];
-    const int row = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const float* src = part + (size_t)row * S * 132;
-    float m = -INFINITY;
-    for (int k = lane; k < S; k += 32) m = fmaxf(m, src[(size_t)k * 132 + 128]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
-#pragma unroll 4
-    for (int k = w; k < S; k += 4) {
-        const float* pk = src + (size_t)k * 132;
-        const float c = (m == -INFINITY) ? 0.f : exp2f(pk[128] - m);
-        l = fmaf(pk[129], c, l);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[j] = fmaf(pk[lane + 32 * j], c, acc[j]);
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) so[w][lane + 32 * j] = acc[j];
-    if (lane == 0) sl[w] = l;
+    const int u_sel = w.u0 + lane;
+    const int32_t sel_lane = (u_sel < w.u1 && u_sel < kB) ? __ldcg(w.sel + u_sel) : -1;
+    int ns = __ldcg(nsel + s);
+    ns = ns < 0 ? 0 : (ns > kB ? kB : ns);
+    w.nsel = ns;
+    w.i = p;
+    if (p < 0 || p >= cap) w.u1 = w.u0;  // skipped sequence: zero output
+
+    warp_attend<NT>(w, wsm, lane, qb, sel_lane, st);
+
+    const int E = G * kHeadDim, per = E / C;
+    store_state_hd<NT>(st, G, reinterpret_cast<float*>(wsm), lane);
     __syncthreads();
-    const int d = threadIdx.x;
-    const float lt = sl[0] + sl[1] + sl[2] + sl[3];
-    const float o = so[0][d] + so[1][d] + so[2][d] + so[3][d];
-    out[(size_t)row * kHeadDim + d] = f32_to_bf16(lt > 0.f ? o / lt : 0.f);
+    float* recv = reinterpret_cast<float*>(smem + DW * WARP_SMEM);  // [C][per] o, [C][G] m, [C][G] l
+    const uint32_t recv_s = smem_u32(recv);
+    cluster_wait();  // every CTA of the cluster runs: its receive area exists
+    for (int x = threadIdx.x; x < E; x += DW * 32) {
+        const int h = x / kHeadDim;
+        float mw[DW], M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < DW; ++k) {
+            mw[k] = reinterpret_cast<const float*>(smem + k * WARP_SMEM)[E + h];
+            M = fmaxf(M, mw[k]);
+        }
+        float o = 0.f;
+#pragma unroll
+        for (int k = 0; k < DW; ++k)
+            o = fmaf(reinterpret_cast<const float*>(smem + k * WARP_SMEM)[x], M == -INFINITY ? 0.f : exp2f(mw[k] - M), o);
+        const int owner = x / per;
+        st_dsmem(dsmem_addr(recv_s + (uint32_t)(rank * per + x - owner * per) * 4u, (uint32_t)owner), o);
+    }
+    for (int h = threadIdx.x; h < G; h += DW * 32) {
+        float mw[DW], M = -INFINITY, L = 0.f;
+#pragma unroll
+        for (int k = 0; k < DW; ++k) {
+            mw[k] = reinterpret_cast<const float*>(smem + k * WARP_SMEM)[E + h];
+            M = fmaxf(M, mw[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < DW; ++k)
+            L = fmaf(reinterpret_cast<const float*>(smem + k * WARP_SMEM)[E + G + h],
+                     M == -INFINITY ? 0.f : exp2f(mw[k] - M), L);
+        for (int c2 = 0; c2 < C; ++c2) {
+            st_dsmem(dsmem_addr(recv_s + (uint32_t)(E + rank * G + h) * 4u, (uint32_t)c2), M);
+            st_dsmem(dsmem_addr(recv_s + (uint32_t)(E + C * G + rank * G + h) * 4u, (uint32_t)c2), L);
+        }
+    }
+    cluster_sync();  // every push has landed
+    for (int xi = threadIdx.x; xi < per; xi += DW * 32) {
+        const int x = rank * per + xi, h = x / kHeadDim;
+        float M = -INFINITY;
+        for (int j = 0; j < C; ++j) M = fmaxf(M, recv[E + j * G + h]);
+        float num = 0.f, den = 0.f;
+        for (int j = 0; j < C; ++j) {
+            const float c = M == -INFINITY ? 0.f : exp2f(recv[E + j * G + h] - M);
+            num = fmaf(recv[j * per + xi], c, num);
+            den = fmaf(recv[E + C * G + j * G + h], c, den);
+        }
+        out[((size_t)s * q_heads + (size_t)g * G) * kHeadDim + x] = f32_to_bf16(den > 0.f ? num / den : 0.f);
+    }
 }
 
 }  // namespace
@@ -472,30 +525,112 @@ cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_
     return cudaGetLastError();
 }
 
-int decode_attention_splits(const LayerDims& L) {
-    const int units = L.kB + 1;
-    int S = (units + 7) / 8;
-    return S < 1 ? 1 : (S > 64 ? 64 : S);
+// Launch shape of the decode attention: DW warps per CTA and C CTAs per
+// cluster (one cluster per (sequence, kv head)). More warps per CTA shorten the
+// per-warp chain of chunks when the batch leaves SMs idle; otherwise the
+// largest of 16, 8, 4, 2, 1 CTAs per cluster whose grid runs in one wave and
+// whose cluster the device can place.
+namespace {
+
+struct DecodeShape {
+    int dw, c;
+};
+
+template <int NT, int DW>
+int decode_cluster_for(const LayerDims& L, int batch, int G) {
+    auto kern = decode_attention_kernel<NT, DW>;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int base = DW * WARP_SMEM;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, base + decode_recv_bytes(G, kMaxCluster));
+    cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    for (int C = kMaxCluster; C > 1; C >>= 1) {
+        const int smem = base + decode_recv_bytes(G, C);
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DW * 32, smem) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        if ((int64_t)batch * L.kv_heads * C > (int64_t)sms * per_sm) continue;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)C, (unsigned)L.kv_heads, (unsigned)batch);
+        cfg.blockDim = dim3(DW * 32);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0) return C;
+        cudaGetLastError();  // clear a refused size
+    }
+    return 1;
 }
+
+template <int NT>
+DecodeShape decode_shape(const LayerDims& L, int batch, int G) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if ((int64_t)batch * L.kv_heads * kMaxCluster <= sms) {
+        const int c = decode_cluster_for<NT, 8>(L, batch, G);
+        if (c == kMaxCluster) return {8, c};
+    }
+    return {4, decode_cluster_for<NT, 4>(L, batch, G)};
+}
+
+template <int NT, int DW>
+cudaError_t launch_decode_attention_t(const LayerDims& L, int batch, int C, const int64_t* pos, const uint16_t* q,
+                                      const uint16_t* kc, const uint16_t* vc, int64_t cap, const int32_t* sel,
+                                      const int32_t* nsel, uint16_t* out, cudaStream_t st) {
+    auto kern = decode_attention_kernel<NT, DW>;
+    const int G = L.q_heads / L.kv_heads;
+    const int smem = DW * WARP_SMEM + decode_recv_bytes(G, C);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (C > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)C, (unsigned)L.kv_heads, (unsigned)batch);
+    cfg.blockDim = dim3(DW * 32);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    note_launch();
+    return cudaLaunchKernelEx(&cfg, kern, q, pos, kc, vc, cap, sel, nsel, out, L.q_heads, L.kv_heads, L.r, L.kB,
+                              L.sm_scale * LOG2E);
+}
+
+}  // namespace
 
 cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
                                     const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
-                                    float* part, uint16_t* out, cudaStream_t st) {
+                                    uint16_t* out, cudaStream_t st) {
     if (batch <= 0) return cudaSuccess;
     const int G = L.q_heads / L.kv_heads;
-    auto kern = G > 8 ? decode_attention_kernel<2> : decode_attention_kernel<1>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    const int S = decode_attention_splits(L);
-    const int64_t items = (int64_t)batch * L.kv_heads * S;
-    note_launch();
-    cudaError_t e = launch_pdl(kern, dim3((unsigned)((items + WARPS - 1) / WARPS)), dim3(WARPS * 32), (size_t)SMEM,
-                               st, q, pos, kc, vc, cap, sel, nsel, part, batch, L.q_heads, L.kv_heads, L.r, L.kB,
-                               S, L.sm_scale * LOG2E);
-    if (e != cudaSuccess) return e;
-    const int rows = batch * L.q_heads;
-    note_launch();
-    return launch_pdl(decode_combine_kernel, dim3((unsigned)rows), dim3(128), 0, st, (const float*)part, S, out);
+    // The launch shape is chosen once per problem shape (and thread).
+    static thread_local int cached_key[4] = {-1, -1, -1, -1};
+    static thread_local DecodeShape cached = {4, 1};
+    const int key[4] = {batch, L.q_heads, L.kv_heads, L.kB};
+    if (!std::equal(key, key + 4, cached_key)) {
+        cached = G > 8 ? decode_shape<2>(L, batch, G) : decode_shape<1>(L, batch, G);
+        std::copy(key, key + 4, cached_key);
+    }
+    const DecodeShape sh = cached;
+    if (G > 8)
+        return sh.dw == 8 ? launch_decode_attention_t<2, 8>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st)
+                          : launch_decode_attention_t<2, 4>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st);
+    return sh.dw == 8 ? launch_decode_attention_t<1, 8>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st)
+                      : launch_decode_attention_t<1, 4>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st);
 }
 
 }  // namespace qsa

@@ -4,16 +4,15 @@
 // a5 selection.
 //
 // The score stream is the hot spot: 256 bytes of pooled key per block and
-// 4 x 128 multiply-adds, an L2/HBM stream. A half-warp scores four blocks per
-// step from 16-byte loads (prefetched one step ahead); the 16 per-lane partial
-// sums (4 blocks x 4 heads) are reduced across the half-warp with a transpose
-// reduction (15 shuffles for 16 sums), then ReLU and the head sum take two more.
-// The same pass builds a histogram of the scores' top 11 key bits per sequence,
-// so the selection needs one more pass over the score row, not a sort:
-// every CTA finds the threshold digit from the histogram, appends the sure
-// winners and the threshold-digit candidates, and the last CTA of the sequence
-// finishes the exact pick among the candidates (ties to the lower block index)
-// and sorts the k_B winners (select.cuh).
+// 4 x 128 multiply-adds, an L2/HBM stream spread over one wave of CTAs, each
+// scoring its slice on the tensor cores (mma.sync) from 16-byte loads issued a
+// group ahead. The same pass builds a per-sequence histogram of a level-1 key
+// digit of the scores, so the selection reads the score row once more and never
+// sorts it: one thread-block cluster per sequence finds the threshold digit,
+// collects the sure winners and the threshold-digit candidates of each CTA's
+// slice in shared memory, resolves the exact pick among all candidates over
+// distributed shared memory (ties to the lower block index), and writes the
+// k_B winners in ascending order.
 #include <algorithm>
 
 #include "kernels.h"
@@ -22,8 +21,6 @@
 
 namespace qsa {
 namespace {
-
-constexpr int SC_THREADS = 512;  // score and select CTAs
 
 constexpr int DS_THREADS = 256;  // fused score CTAs
 constexpr int DS_WARPS = DS_THREADS / 32;
@@ -34,6 +31,16 @@ __device__ __forceinline__ void cta_range(int64_t nvis, int x, int X, int64_t& l
     lo = min(nvis, (int64_t)x * chunk);
     hi = min(nvis, lo + chunk);
 }
+
+// Level-1 digit of a decode score's key: bits 30..20 (8 exponent and 3
+// mantissa bits). Decode scores are sums of ReLUs, never negative, so the sign
+// bit carries nothing; a negative key (impossible here) maps to digit 0, which
+// the selection treats as "refine from the row".
+__device__ __forceinline__ uint32_t dec_digit1(uint32_t key) {
+    return key >= 0x80000000u ? (key >> 20) & 2047u : 0u;
+}
+// Level-2 digit inside a level-1 bin: bits 19..9.
+__device__ __forceinline__ uint32_t dec_digit2(uint32_t key) { return (key >> 9) & 2047u; }
 
 // One decode step's cache update, query rotation and score stream, fused.
 //
@@ -63,12 +70,36 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     __shared__ uint32_t hist[2048];
     __shared__ __align__(16) uint16_t qs[kIdxHeads * kIdxDim];
     __shared__ double2 cs[kIdxDim / 2];  // (sin, cos) of the query position's angles
-    pdl_wait();
-    pdl_trigger();
     const int s = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // The position and the indexer query are inputs of the step (complete
+    // before the step's first kernel could start), so the query rotation runs
+    // before the dependency wait, overlapping the end of the previous step.
     const int64_t p = pos[s];
-    if (p < 0 || p >= cap) {
+    const bool valid = p >= 0 && p < cap;
+    const int X = gridDim.x > 1 ? (int)gridDim.x - 1 : 1;  // scoring CTAs
+    const int x = gridDim.x > 1 ? (int)blockIdx.x - 1 : 0;  // CTA 0 only appends and pools
+    int64_t lo = 0, hi = 0;
+    if (valid && p / r > kB && x >= 0) cta_range(p / r, x, X, lo, hi);
+    const bool scoring = lo < hi;  // (uniform over the CTA)
+    if (scoring) {
+        // The rope_dims / 2 angles of position p once per CTA (an fp64 sincos of
+        // a large argument is slow), then the 4 heads rotate from the table.
+        if (tid < rt.half) {
+            double sn, cn;
+            sincos(__dmul_rn((double)p, rt.theta[tid]), &sn, &cn);
+            cs[tid] = make_double2(sn, cn);
+        }
+        for (int b = tid; b < 2048; b += DS_THREADS) hist[b] = 0u;
+        __syncthreads();
+        if (warp < kIdxHeads)
+            rotate_head_warp_tab(idx_q + ((size_t)s * kIdxHeads + warp) * kIdxDim, rt.half, cs,
+                                 qs + warp * kIdxDim, lane);
+        __syncthreads();
+    }
+    pdl_wait();
+    pdl_trigger();
+    if (!valid) {
         if (blockIdx.x == 0 && tid == 0) flag_status(status, 4 /* QSA_ERR_CAPACITY */);
         return;
     }
@@ -94,27 +125,8 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
                             pooled + ((size_t)s * (cap / r) + b) * kIdxDim, lane);
         }
     }
+    if (!scoring) return;  // (also: every visible block is selected, no scores needed)
     const int64_t pcap = cap / r;
-    if (p / r <= kB) return;  // every visible block is selected: no scores needed
-    const int X = gridDim.x > 1 ? (int)gridDim.x - 1 : 1;  // scoring CTAs
-    const int x = gridDim.x > 1 ? (int)blockIdx.x - 1 : 0;
-    if (x < 0) return;                                     // CTA 0 only appends and pools
-    int64_t lo, hi;
-    cta_range(p / r, x, X, lo, hi);
-    if (lo >= hi) return;
-    // The rope_dims / 2 angles of position p once per CTA (an fp64 sincos of a
-    // large argument is slow), then the 4 heads rotate from the table.
-    if (tid < rt.half) {
-        double sn, cn;
-        sincos(__dmul_rn((double)p, rt.theta[tid]), &sn, &cn);
-        cs[tid] = make_double2(sn, cn);
-    }
-    for (int b = tid; b < 2048; b += DS_THREADS) hist[b] = 0u;
-    __syncthreads();
-    if (warp < kIdxHeads)
-        rotate_head_warp_tab(idx_q + ((size_t)s * kIdxHeads + warp) * kIdxDim, rt.half, cs, qs + warp * kIdxDim,
-                             lane);
-    __syncthreads();
     const int g = lane >> 2, t = lane & 3;
     // B fragments: column g (head g, zero for g >= 4), k-step j.
     uint32_t bq0[8], bq1[8];
@@ -158,11 +170,11 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
             const int64_t b0 = base + g, b1 = b0 + 8;
             if (b0 < hi) {
                 dst[b0] = sa;
-                atomicAdd(&hist[float_key(sa) >> 21], 1u);
+                atomicAdd(&hist[dec_digit1(float_key(sa))], 1u);
             }
             if (b1 < hi) {
                 dst[b1] = sb;
-                atomicAdd(&hist[float_key(sb) >> 21], 1u);
+                atomicAdd(&hist[dec_digit1(float_key(sb))], 1u);
             }
         }
 #pragma unroll
@@ -176,17 +188,27 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
         if (hist[b]) atomicAdd(&hist_g[(size_t)s * 2048 + b], hist[b]);
 }
 
-// The sequence's histogram and counters back to zero for the next step (the
-// score kernel only adds to them). Called by the last CTA, after every CTA
-// of the sequence has read them.
-__device__ __forceinline__ void reset_state(DecodeSelWs& sw, int s) {
-    for (int b = threadIdx.x; b < 2048; b += blockDim.x) sw.hist[(size_t)s * 2048 + b] = 0u;
-    if (threadIdx.x < 4) sw.counters[s * 4 + threadIdx.x] = 0;
-}
+constexpr int SEL_E = 8;                 // scores per thread per round of the scan
+constexpr int SEL_BITMAP_WORDS = 10240;  // ordered output by bitmap for up to 327680 blocks
 
-// Exclusive prefix over the CTA (thread order) of a per-thread packed count;
-// returns the CTA total. All threads must call it.
-__device__ __forceinline__ uint32_t cta_prefix(SelSmem& sm, uint32_t v, uint32_t& prefix) {
+struct DecSelSmem {
+    uint32_t hist[BINS];     // level-1, then level-2 histogram
+    uint32_t cand_key[CAND]; // candidates (threshold digit): this CTA's, then all
+    int32_t cand_idx[CAND];
+    int32_t l3[T];           // candidate slots in the level-2 threshold bin
+    union {
+        int32_t out[kMaxKB];                // winners as a list
+        uint32_t bitmap[SEL_BITMAP_WORDS];  // winners as a bitmap over the blocks
+    } u;
+    uint32_t wsum[NW];
+    unsigned long long base;
+    int32_t n_win, n_cand, n_l3, bin, above, last;
+};
+static_assert(sizeof(SelSmem) <= sizeof(DecSelSmem), "the row-selection fallback reuses this shared memory");
+
+// Exclusive prefix of v over the CTA in thread order; returns the total.
+template <typename Sm>
+__device__ __forceinline__ uint32_t cta_prefix(Sm& sm, uint32_t v, uint32_t& prefix) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     uint32_t inc = v;
 #pragma unroll
@@ -207,112 +229,243 @@ __device__ __forceinline__ uint32_t cta_prefix(SelSmem& sm, uint32_t v, uint32_t
     return total;
 }
 
-__global__ void __launch_bounds__(SC_THREADS) decode_select_kernel(
+// Warp-aggregated append of `value` to list[*count] (every lane calls it).
+__device__ __forceinline__ void warp_append(int32_t* count, bool flag, int32_t* list, int32_t value, int cap) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t bal = __ballot_sync(0xffffffffu, flag);
+    int base = 0;
+    if (lane == 0 && bal) base = atomicAdd(count, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const int at = base + __popc(bal & ((1u << lane) - 1u));
+    if (flag && at < cap) list[at] = value;
+}
+
+// The sequence's histogram and counters back to zero for the next step.
+__device__ __forceinline__ void reset_state(DecodeSelWs sw, int s) {
+    for (int b = threadIdx.x; b < BINS; b += T) sw.hist[(size_t)s * BINS + b] = 0u;
+    if (threadIdx.x < 4) sw.counters[s * 4 + threadIdx.x] = 0;
+}
+
+// Exact selection from the whole row (degenerate inputs only), in the last CTA.
+__device__ __noinline__ void decode_select_fallback(uint8_t* raw, const float* row, int64_t nvis, int kB,
+                                                    int32_t* out, int32_t* nsel_s) {
+    select_row(*reinterpret_cast<SelSmem*>(raw), row, nvis, kB, out, nsel_s);
+}
+
+// The decode selection (a5) of each sequence by X CTAs: every CTA reads the
+// sequence's level-1 histogram (built by the score pass) and finds the
+// threshold digit b1 with above(b1) < k_B <= above(b1) + hist[b1], scans its
+// slice of the scores into shared-memory lists of sure winners (digit > b1)
+// and candidates (digit == b1), reserves room in the sequence's global lists
+// with one atomic and copies them there. The last CTA to finish resolves the
+// exact pick among the candidates (a level-2 histogram on the next 11 key
+// bits, then a rank by (key descending, block ascending) inside the level-2
+// threshold bin) and writes the k_B winners in ascending block order through a
+// bitmap over the blocks. The code is kept small and nearly barrier-free: it
+// runs once per step on cold instruction caches.
+__global__ void __launch_bounds__(T) decode_select_kernel(
     const int64_t* __restrict__ pos, int64_t cap, int r, int kB, const float* __restrict__ scores,
-    DecodeSelWs sw, int32_t* __restrict__ sel, int32_t* __restrict__ nsel) {
+    DecodeSelWs sw, int32_t* __restrict__ sel, int32_t* __restrict__ nsel, int32_t* __restrict__ status) {
     extern __shared__ __align__(16) uint8_t raw[];
-    SelSmem& sm = *reinterpret_cast<SelSmem*>(raw);
-    __shared__ unsigned long long slot_base;  // (candidates << 32) | winners before this round
-    __shared__ int last;
+    DecSelSmem& sm = *reinterpret_cast<DecSelSmem*>(raw);
+    const int s = blockIdx.y, tid = threadIdx.x;
+    const int64_t p = pos[s];  // an input of the step
     pdl_wait();
     pdl_trigger();
-    const int s = blockIdx.y;
-    const int tid = threadIdx.x;
-    const int64_t p = pos[s];
     const int64_t nvis = (p >= 0 && p < cap) ? p / r : 0;
     int32_t* out = sel + (size_t)s * kB;
     if (nvis <= kB) {  // every visible block is selected
         if (blockIdx.x == 0) {
-            for (int k2 = tid; k2 < kB; k2 += SC_THREADS) out[k2] = k2 < nvis ? k2 : -1;
+            for (int k2 = tid; k2 < kB; k2 += T) out[k2] = k2 < nvis ? k2 : -1;
             if (tid == 0) nsel[s] = (int32_t)nvis;
         }
         return;
     }
     const float* row = scores + (size_t)s * (cap / r);
-    // Threshold digit from the sequence's histogram.
-    reinterpret_cast<uint4*>(sm.hist)[tid] = __ldcg(reinterpret_cast<const uint4*>(sw.hist + (size_t)s * 2048) + tid);
-    find_bin(sm, 2048, (uint32_t)kB);
+    reinterpret_cast<uint4*>(sm.hist)[tid] = __ldcg(reinterpret_cast<const uint4*>(sw.hist + (size_t)s * BINS) + tid);
+    if (tid == 0) {
+        sm.n_win = 0;
+        sm.n_cand = 0;
+        sm.n_l3 = 0;
+    }
+    find_bin(sm, BINS, (uint32_t)kB);
     const uint32_t b1 = sm.bin;
     const uint32_t need1 = (uint32_t)kB - (uint32_t)sm.above;
-    int32_t* cnt = sw.counters + s * 4;
-    int32_t* winners = sw.winners + (size_t)s * kB;
-    uint2* cand = sw.cand + (size_t)s * kDecodeCand;
-    // Sure winners (digit above b1) and candidates (digit b1) of this CTA's
-    // slice, 8 entries per thread per round (coalesced: entry e of thread t
-    // is r0 + e T + t); one scan and one 64-bit atomic on (winners,
-    // candidates) place a round's entries.
+
+    // Scan this CTA's slice; hits are rare, so their appends sit behind a vote.
     int64_t lo, hi;
     cta_range(nvis, blockIdx.x, gridDim.x, lo, hi);
-    constexpr int E = 8;
-    for (int64_t r0 = lo; r0 < hi; r0 += (int64_t)E * SC_THREADS) {
-        uint32_t key[E];
-        uint32_t nw = 0, ncand = 0;
+    for (int64_t r0 = lo; r0 < hi; r0 += (int64_t)SEL_E * T) {
+        uint32_t key[SEL_E];
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int64_t b = r0 + (int64_t)e * SC_THREADS + tid;
+        for (int e = 0; e < SEL_E; ++e) {
+            const int64_t b = r0 + (int64_t)e * T + tid;
             key[e] = b < hi ? float_key(__ldcg(row + b)) : 0u;
-            nw += (b < hi && (key[e] >> 21) > b1) ? 1u : 0u;
-            ncand += (b < hi && (key[e] >> 21) == b1) ? 1u : 0u;
         }
-        uint32_t pre;
-        const uint32_t tot = cta_prefix(sm, (ncand << 16) | nw, pre);
-        if (tid == 0) {
-            const unsigned long long add = ((unsigned long long)(tot >> 16) << 32) | (tot & 0xFFFFu);
-            slot_base = tot ? atomicAdd(reinterpret_cast<unsigned long long*>(cnt), add) : 0ull;
-        }
-        __syncthreads();
-        int ws_ = (int)(uint32_t)slot_base + (int)(pre & 0xFFFFu);
-        int cs = (int)(uint32_t)(slot_base >> 32) + (int)(pre >> 16);
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const int64_t b = r0 + (int64_t)e * SC_THREADS + tid;
-            if (b >= hi) break;
-            const uint32_t d = key[e] >> 21;
-            if (d > b1) {
-                if (ws_ < kB) winners[ws_] = (int32_t)b;  // < k_B by the histogram
-                ++ws_;
-            } else if (d == b1) {
-                if (cs < kDecodeCand) cand[cs] = make_uint2(key[e], (uint32_t)b);
-                ++cs;
+        for (int e = 0; e < SEL_E; ++e) {
+            const int64_t b = r0 + (int64_t)e * T + tid;
+            const uint32_t d = dec_digit1(key[e]);
+            const bool w = b < hi && d > b1, c = b < hi && d == b1;
+            if (__any_sync(0xffffffffu, w || c)) {
+                warp_append(&sm.n_win, w, sm.u.out, (int32_t)b, kMaxKB);
+                const uint32_t bal = __ballot_sync(0xffffffffu, c);
+                int cb = 0;
+                if ((tid & 31) == 0 && bal) cb = atomicAdd(&sm.n_cand, __popc(bal));
+                cb = __shfl_sync(0xffffffffu, cb, 0) + __popc(bal & ((1u << (tid & 31)) - 1u));
+                if (c && cb < CAND) {
+                    sm.cand_key[cb] = key[e];
+                    sm.cand_idx[cb] = (int32_t)b;
+                }
             }
         }
-        __syncthreads();
     }
-    // The last CTA of the sequence finishes the pick.
+    __syncthreads();
+    int32_t* cnt = sw.counters + s * 4;  // [0] sure winners, [1] candidates, [2] finished CTAs
+    if (tid == 0) {
+        const unsigned long long add = ((unsigned long long)(uint32_t)sm.n_cand << 32) | (uint32_t)sm.n_win;
+        sm.base = add ? atomicAdd(reinterpret_cast<unsigned long long*>(cnt), add) : 0ull;
+    }
+    __syncthreads();
+    {
+        const int wb = (int)(uint32_t)sm.base, cb = (int)(uint32_t)(sm.base >> 32);
+        const int nw = sm.n_win, nc = min(sm.n_cand, CAND);
+        int32_t* winners = sw.winners + (size_t)s * kB;
+        uint2* cand = sw.cand + (size_t)s * kDecodeCand;
+        for (int k = tid; k < nw; k += T)
+            if (wb + k < kB) winners[wb + k] = sm.u.out[k];  // (< k_B by the histogram)
+        for (int k = tid; k < nc; k += T)
+            if (cb + k < kDecodeCand) cand[cb + k] = make_uint2(sm.cand_key[k], (uint32_t)sm.cand_idx[k]);
+    }
     __threadfence();
     __syncthreads();
-    if (tid == 0) last = atomicAdd(cnt + 2, 1) == (int)gridDim.x - 1;
+    if (tid == 0) sm.last = atomicAdd(cnt + 2, 1) == (int)gridDim.x - 1;
     __syncthreads();
-    if (!last) return;
+    if (!sm.last) return;
+
+    // ---- the last CTA of the sequence ----
     __threadfence();
-    const int n_win = __ldcg(cnt + 0);
-    const int nc = __ldcg(cnt + 1);
-    if (n_win != (int)(kB - need1) || nc > CAND || nc > kDecodeCand) {
-        // Candidates overflow (e.g. thousands of equal scores): exact pick from the row.
-        select_row(sm, row, nvis, kB, out, nsel + s);
+    const int n_win = __ldcg(cnt + 0), nc = __ldcg(cnt + 1);
+    if (b1 == 0u || nc > kDecodeCand || nc > CAND || n_win != kB - (int)need1) {
+        __syncthreads();
+        decode_select_fallback(raw, row, nvis, kB, out, nsel + s);
+        __syncthreads();
         reset_state(sw, s);
         return;
     }
-    for (int k2 = tid; k2 < n_win; k2 += SC_THREADS) sm.out[k2] = __ldcg(winners + k2);
-    for (int c = tid; c < nc; c += SC_THREADS) {
+    const bool use_bm = nvis <= (int64_t)SEL_BITMAP_WORDS * 32;
+    const int words = use_bm ? (int)((nvis + 31) / 32) : 0;
+    for (int b = tid; b < BINS; b += T) sm.hist[b] = 0u;
+    for (int w = tid; w < words; w += T) sm.u.bitmap[w] = 0u;
+    if (tid == 0) {
+        sm.n_l3 = 0;
+        sm.n_win = n_win;
+    }
+    const uint2* cand = sw.cand + (size_t)s * kDecodeCand;
+    for (int c = tid; c < nc; c += T) {
         const uint2 e = __ldcg(cand + c);
         sm.cand_key[c] = e.x;
         sm.cand_idx[c] = (int32_t)e.y;
     }
-    if (tid == 0) sm.n_out = n_win;
-    __syncthreads();  // (counters read by every thread before the reset)
-    reset_state(sw, s);
-    finish_from_candidates(sm, nc, b1, need1, kB, out);
+    __syncthreads();
+    const int32_t* winners = sw.winners + (size_t)s * kB;
+    for (int k = tid; k < n_win; k += T) {
+        const int32_t id = __ldcg(winners + k);
+        if (use_bm)
+            atomicOr(&sm.u.bitmap[id >> 5], 1u << (id & 31));
+        else
+            sm.u.out[k] = id;
+    }
+    for (int c = tid; c < nc; c += T) atomicAdd(&sm.hist[dec_digit2(sm.cand_key[c])], 1u);
+    find_bin(sm, BINS, need1);
+    const uint32_t b2 = sm.bin;
+    const uint32_t need2 = need1 - (uint32_t)sm.above;
+    for (int c0 = 0; c0 < nc; c0 += T) {
+        const int c = c0 + tid;
+        const uint32_t d2 = c < nc ? dec_digit2(sm.cand_key[c]) : 0u;
+        if (c < nc && d2 > b2) {
+            const int32_t id = sm.cand_idx[c];
+            if (use_bm) {
+                atomicOr(&sm.u.bitmap[id >> 5], 1u << (id & 31));
+            } else {
+                const int at = atomicAdd(&sm.n_win, 1);
+                if (at < kMaxKB) sm.u.out[at] = id;
+            }
+        }
+        warp_append(&sm.n_l3, c < nc && d2 == b2, sm.l3, c, T);
+    }
+    __syncthreads();
+    const int n3 = sm.n_l3;
+    if (n3 > T) {  // thousands of equal keys
+        decode_select_fallback(raw, row, nvis, kB, out, nsel + s);
+        __syncthreads();
+        reset_state(sw, s);
+        return;
+    }
+    if (tid < n3) {  // rank inside the level-2 threshold bin: (key desc, block asc)
+        const int x = sm.l3[tid];
+        const uint32_t kx = sm.cand_key[x];
+        const int32_t ix = sm.cand_idx[x];
+        uint32_t rk = 0;
+        for (int u = 0; u < n3; ++u) {
+            const int y = sm.l3[u];
+            const uint32_t ky = sm.cand_key[y];
+            rk += (ky > kx || (ky == kx && sm.cand_idx[y] < ix)) ? 1u : 0u;
+        }
+        if (rk < need2) {
+            if (use_bm) {
+                atomicOr(&sm.u.bitmap[ix >> 5], 1u << (ix & 31));
+            } else {
+                const int at = atomicAdd(&sm.n_win, 1);
+                if (at < kMaxKB) sm.u.out[at] = ix;
+            }
+        }
+    }
+    __syncthreads();
+    if (use_bm) {
+        // Ordered compaction: thread t owns words [t per, (t + 1) per).
+        const int per = (words + T - 1) / T;
+        const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+        uint32_t n = 0;
+        for (int w = w0; w < w1; ++w) n += __popc(sm.u.bitmap[w]);
+        uint32_t at;
+        const uint32_t total = cta_prefix(sm, n, at);
+        if (total != (uint32_t)kB && tid == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
+        for (int w = w0; w < w1; ++w) {
+            uint32_t m = sm.u.bitmap[w];
+            while (m) {
+                const int bit = __ffs(m) - 1;
+                m &= m - 1;
+                if (at < (uint32_t)kB) out[at] = w * 32 + bit;
+                ++at;
+            }
+        }
+    } else {
+        if (sm.n_win != kB && tid == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
+        sort_ints(sm.u.out, kB);
+        for (int k2 = tid; k2 < kB; k2 += T) out[k2] = sm.u.out[k2];
+    }
     if (tid == 0) nsel[s] = kB;
+    reset_state(sw, s);
 }
 
 }  // namespace
 
+// CTAs per sequence of the decode selection: one wave over the batch.
 int decode_select_ctas(int batch) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    return std::max(1, 2 * sms / std::max(batch, 1));
+    static thread_local int cached = -1;
+    if (cached < 0) {
+        const int smem = (int)sizeof(DecSelSmem);
+        cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        int dev = 0, sms = 148, per_sm = 1;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_select_kernel, T, smem) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        cached = sms * per_sm;
+    }
+    return std::max(1, cached / std::max(batch, 1));
 }
 
 // One wave: as many CTAs as fit on the GPU at once, split over the batch.
@@ -339,12 +492,13 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
 
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
                                  const float* scores, DecodeSelWs sw, int32_t* sel, int32_t* nsel,
-                                 cudaStream_t st) {
-    const int smem = (int)sizeof(SelSmem);
+                                 int32_t* status, cudaStream_t st) {
+    const int smem = (int)sizeof(DecSelSmem);
+    const int X = decode_select_ctas(batch);
     cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     note_launch();
-    return launch_pdl(decode_select_kernel, dim3((unsigned)decode_select_ctas(batch), (unsigned)batch),
-                      dim3(SC_THREADS), (size_t)smem, st, pos, cap, L.r, L.kB, scores, sw, sel, nsel);
+    return launch_pdl(decode_select_kernel, dim3((unsigned)X, (unsigned)batch), dim3(T), (size_t)smem, st, pos, cap,
+                      L.r, L.kB, scores, sw, sel, nsel, status);
 }
 
 }  // namespace qsa

@@ -90,16 +90,15 @@ cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_
                                     const uint16_t* vc, int64_t cap, const int32_t* sel,
                                     const int32_t* nsel, uint16_t* out, float* lse,
                                     cudaStream_t st);
-int decode_attention_splits(const LayerDims& L);
 cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
                                     const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
-                                    float* part, uint16_t* out, cudaStream_t st);
+                                    uint16_t* out, cudaStream_t st);
 
 // decode.cu. Per-sequence selection state in the decode workspace.
 constexpr int kDecodeCand = 4096;  // candidates of the threshold digit kept for the final pick
 struct DecodeSelWs {
-    uint32_t* hist;     // [batch][2048] histogram of the top 11 key bits
+    uint32_t* hist;     // [batch][2048] histogram of the scores' level-1 key digit
     int32_t* counters;  // [batch][4]: sure winners, candidates, finished CTAs
     int32_t* winners;   // [batch][k_B]
     uint2* cand;        // [batch][kDecodeCand] (key, block)
@@ -116,6 +115,6 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 int32_t* status, cudaStream_t st);
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
                                  const float* scores, DecodeSelWs sw, int32_t* sel, int32_t* nsel,
-                                 cudaStream_t st);
+                                 int32_t* status, cudaStream_t st);
 
 }  // namespace qsa

@@ -35,8 +35,8 @@ struct SelSmem {
 // bank conflicts); a suffix scan over the threads gives every thread the
 // count above its bins, and the one thread whose bins hold the need-th key
 // walks them.
-template <int PER>
-__device__ __forceinline__ void find_bin_per(SelSmem& sm, uint32_t need) {
+template <int PER, typename Sm>
+__device__ __forceinline__ void find_bin_per(Sm& sm, uint32_t need) {
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     uint32_t h[4];
     if (PER == 4) {
@@ -74,7 +74,8 @@ __device__ __forceinline__ void find_bin_per(SelSmem& sm, uint32_t need) {
     __syncthreads();
 }
 
-__device__ void find_bin(SelSmem& sm, int nbins, uint32_t need) {
+template <typename Sm>
+__device__ void find_bin(Sm& sm, int nbins, uint32_t need) {
     __syncthreads();
     if (nbins == 2048)
         find_bin_per<4>(sm, need);
@@ -82,7 +83,8 @@ __device__ void find_bin(SelSmem& sm, int nbins, uint32_t need) {
         find_bin_per<2>(sm, need);
 }
 
-__device__ void clear_hist(SelSmem& sm) {
+template <typename Sm>
+__device__ void clear_hist(Sm& sm) {
     for (int b = threadIdx.x; b < BINS; b += T) sm.hist[b] = 0;
     __syncthreads();
 }
@@ -192,6 +194,54 @@ __device__ void sort_out(SelSmem& sm, int kB) {
                     if ((a > b) == up) {
                         sm.out[i] = b;
                         sm.out[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// Sorts a[0, n) (shared memory, room for max(n, T) entries) ascending: the
+// bitonic network of sort_out over the next power of two above n only.
+__device__ void sort_ints(int32_t* a, int n) {
+    const int tid = threadIdx.x;
+    int P = 1;
+    while (P < n) P <<= 1;
+    if (P <= T) {
+        int32_t v = tid < n ? a[tid] : 0x7fffffff;
+        for (int k = 2; k <= P; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                int32_t o;
+                if (j >= 32) {
+                    __syncthreads();
+                    a[tid] = v;
+                    __syncthreads();
+                    o = a[tid ^ j];
+                } else {
+                    o = __shfl_xor_sync(0xffffffffu, v, j);
+                }
+                const bool up = (tid & k) == 0, lower = (tid & j) == 0;
+                v = (lower == up) ? min(v, o) : max(v, o);
+            }
+        }
+        __syncthreads();
+        if (tid < n) a[tid] = v;
+        __syncthreads();
+        return;
+    }
+    for (int k = n + tid; k < P; k += T) a[k] = 0x7fffffff;
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += T) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const int32_t x = a[i], y = a[ixj];
+                    const bool up = (i & k) == 0;
+                    if ((x > y) == up) {
+                        a[i] = y;
+                        a[ixj] = x;
                     }
                 }
             }
