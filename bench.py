@@ -242,6 +242,21 @@ class Bench:
             L.workspace(qsa.OP_TOPK_BLOCKS, n)
         if S:
             L.workspace(qsa.OP_DECODE_STEP)
+        self.dec_graph, self.dec_graphs_1, self.graph_kernels = None, [], 0
+        self.graph_launches = 0  # kernels launched by graph replays so far
+        torch.cuda.synchronize()
+
+    def capture(self):
+        """The decode steps as CUDA graphs (after an eager warm-up step): one
+        graph for the back-to-back steps and one per step for the cold pass.
+        Replays launch the same kernels as the eager calls."""
+        if not self.dec or self.dec_graph is not None:
+            return
+        qsa = self.qsa
+        n0 = qsa.qsa_launch_count()
+        self.dec_graph = self.L.capture_decode(self.dec)
+        self.graph_kernels = qsa.qsa_launch_count() - n0
+        self.dec_graphs_1 = [self.L.capture_decode([d]) for d in self.dec]
         torch.cuda.synchronize()
 
     def step(self, mark=None):
@@ -261,8 +276,12 @@ class Bench:
         if self.pre is not None:
             p = self.pre
             L.prefill(p["q"], p["idx_q"], 0, w.n, p["out"], p["sel"], p["nsel"], mark=mark)
-        for d in self.dec:
-            L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+        if self.dec_graph is not None:
+            self.dec_graph.replay()
+            self.graph_launches += self.graph_kernels
+        else:
+            for d in self.dec:
+                L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
         if mark and self.dec:
             mark("decode")
 
@@ -315,8 +334,10 @@ def run_cuda(args, w, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
     b = Bench(w, dev, stage=args.stage)
     qsa = b.qsa
-    for _ in range(args.warmup):
+    for k in range(args.warmup):
         b.step()
+        if k == 0 and not args.no_graph:
+            b.capture()  # decode steps replayed from CUDA graphs from here on
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -332,7 +353,7 @@ def run_cuda(args, w, rank, world):
         e.record(stream)
         marks.append((name, e))
 
-    launches0 = qsa.qsa_launch_count()
+    launches0 = qsa.qsa_launch_count() + b.graph_launches
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     t0.record(stream)
@@ -343,7 +364,7 @@ def run_cuda(args, w, rank, world):
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    launches = qsa.qsa_launch_count() - launches0
+    launches = qsa.qsa_launch_count() + b.graph_launches - launches0
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / args.steps
     stage_ms = {}
@@ -380,11 +401,14 @@ def run_cuda(args, w, rank, world):
         # after a 256 MB write that evicts L2; only the decode calls are timed.
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         evs = []
-        for d in b.dec:
+        for k, d in enumerate(b.dec):
             flush.fill_(len(evs) & 0xFF)
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a0.record(stream)
-            b.L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+            if b.dec_graphs_1:
+                b.dec_graphs_1[k].replay()
+            else:
+                b.L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
             a1.record(stream)
             evs.append((a0, a1))
         torch.cuda.synchronize()
@@ -409,7 +433,8 @@ def run_cuda(args, w, rank, world):
                    "K": w.K, "k_B": w.k_blocks, "indexer": f"{w.idx_heads}x{w.idx_dim} MQA",
                    "core": f"GQA {w.q_heads}q/{w.kv_heads}kv d={w.head_dim}",
                    "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (K/V 2.1 GB, q 8.6 GB); decode steps back to back"},
+                   "l2": "inputs larger than L2 (K/V 2.1 GB, q 8.6 GB); decode steps back to back",
+                   "decode_launch": "eager calls" if b.dec_graph is None else "CUDA graph replay of the steps"},
         "roofline": roofline, "stages": stages,
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -563,6 +588,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="decode steps as eager calls, not CUDA graph replays")
     ap.add_argument("--stage", choices=["all", "topk"], default="all",
                     help="topk: time only key pooling + the fused indexer (for profiling)")
     ap.add_argument("--n", type=int, default=None, help="override the workload's sequence length")

@@ -73,3 +73,21 @@ class QSALayer:
         qsa_decode_step(self.cfg, self.batch, pos, q, k, v, idx_q, idx_k, self.k_cache, self.v_cache,
                         self.idx_k_cache, self.pooled, self.cap, self.rms_w, out, sel_out, nsel_out, ws,
                         stream)
+
+    def capture_decode(self, steps) -> "torch.cuda.CUDAGraph":
+        """Captures the decode steps `steps` (a list of dicts with the
+        decode_step arguments pos, q, k, v, idx_q, idx_k, out) into one CUDA
+        graph, run by `graph.replay()`: one launch for the whole sequence of
+        steps, with the kernels' programmatic dependencies kept as graph edges.
+        The graph holds the tensors' addresses: refill the same tensors
+        between replays. The workspace is allocated (and warmed) first, so
+        nothing is allocated during capture."""
+        self.workspace(OP_DECODE_STEP)
+        side = torch.cuda.Stream(device=self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
+            for d in steps:
+                self.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        return graph

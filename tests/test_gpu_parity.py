@@ -514,3 +514,43 @@ def test_forced_timeout_is_reported_and_the_context_survives(qsa):
         ref = o.row(i, iq_bits[i], pooled)
         tol = score_tol(o.rotate_query(iq_bits[i], i), pooled, ref["scores"])
         check_selection(g[i], gn[i], ref["scores"], tol, o.k_blocks, f"row {i}")
+
+
+def test_decode_graph_replay_matches_eager(qsa):
+    """Decode steps captured into one CUDA graph and replayed give the same
+    outputs, bit for bit, and the same caches as the eager calls (the kernels'
+    programmatic dependencies become graph edges)."""
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    n, S = 9000, 6
+    w = synth.Workload(name="t", n=n, batch=2, decode_steps=S, prefill=False, K=2048, q_heads=32, kv_heads=4,
+                       base_seed=0xF7)
+    B = w.batch
+    cfg = qsa.Config.of(w)
+    cap = n + S + 4
+    full = {nm: dev_full(w, nm, cap, n + S) for nm in ("q", "k", "v", "idx_q", "idx_k")}
+
+    def make():
+        L = QSALayer(cfg, B, cap)
+        _fill_caches(w, L, n)
+        L.compress(0, n // cfg.r)
+        return L
+
+    def steps():
+        return [{"pos": torch.full((B,), n + k, dtype=torch.int64, device="cuda"),
+                 **{nm: full[nm][:, n + k].contiguous() for nm in ("q", "k", "v", "idx_q", "idx_k")},
+                 "out": torch.empty(B, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")} for k in range(S)]
+
+    La, Lb = make(), make()
+    sa, sb = steps(), steps()
+    for d in sa:
+        La.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+    g = Lb.capture_decode(sb)
+    g.replay()
+    torch.cuda.synchronize()
+    for k in range(S):
+        assert torch.equal(sa[k]["out"], sb[k]["out"]), k
+    for name in ("k_cache", "v_cache", "idx_k_cache", "pooled"):
+        assert torch.equal(getattr(La, name), getattr(Lb, name)), name
+    assert qsa.qsa_workspace_status(La.workspace(qsa.OP_DECODE_STEP)) == 0
+    assert qsa.qsa_workspace_status(Lb.workspace(qsa.OP_DECODE_STEP)) == 0
