@@ -49,19 +49,20 @@ def peaks():
 
 def algorithmic(w):
     """Per-step algorithmic work (the units the roofline divides by)."""
-    r, kB, n = w.r, w.k_blocks, w.n
-    i = np.arange(n, dtype=np.int64)
+    r, kB, n, q0 = w.r, w.k_blocks, w.n, w.q_begin
+    i = np.arange(q0, n, dtype=np.int64)
     vis = i // r
     pairs = int(vis.sum()) if w.prefill else 0
     tok = (r * np.minimum(kB, vis) + i % r + 1) if w.prefill else np.zeros(0, np.int64)
     sum_t = int(tok.sum())
     d = w.head_dim
+    nb = n // r - q0 // r  # blocks pooled by the prefill
     out = {
-        "compress_bytes": (n * w.idx_dim * 2 + (n // r) * w.idx_dim * 2) if w.prefill else 0,
+        "compress_bytes": (nb * r * w.idx_dim * 2 + nb * w.idx_dim * 2) if w.prefill else 0,
         "index_flops": pairs * w.idx_heads * w.idx_dim * 2,
         "attn_gather_bytes": sum_t * w.kv_heads * d * 2 * 2,
         "attn_flops": sum_t * w.q_heads * d * 4,
-        "prefill_tokens": n if w.prefill else 0,
+        "prefill_tokens": (n - q0) if w.prefill else 0,
     }
     dec = 0
     dec_tok = 0
@@ -151,15 +152,17 @@ class ClockSampler:
                 "power_w_max": max(float(f[4]) for f in rows if f[4].replace(".", "").isdigit())}
 
 
-def traffic_for(stage: str):
-    """DRAM bytes per launch of a stage from the committed ncu summary, or None
-    when that summary was taken on a different version of the kernel source."""
+def traffic_for(workload: str, stage: str):
+    """DRAM bytes per launch of a stage of a workload from the committed ncu
+    summary, or None when there is none or it was taken on a different version
+    of the kernel source."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
     for ln in open(p):
         f = ln.split("#")[0].split()
-        if len(f) == 3 and f[0] == stage:
+        if len(f) == 4 and f[0] == workload and f[1] == stage:
+            f = f[1:]
             src = os.path.join(ROOT, "block_sparse_long_02_b200", "csrc")
             h = hashlib.sha1()
             for name in sorted(os.listdir(src)):
@@ -205,15 +208,21 @@ class Bench:
         w.device_fill("idx_k", L.idx_k_cache, rows=(0, n))
         self.pre = None
         if w.prefill:
-            q = torch.empty(B, n if stage != "topk" else 1, cfg.q_heads, cfg.head_dim, dtype=bf, device=device)
-            iq = torch.empty(B, n, cfg.idx_heads, cfg.idx_dim, dtype=bf, device=device)
-            if stage != "topk":
-                w.device_fill("q", q.view(B, n, -1), rows=(0, n))
-            w.device_fill("idx_q", iq.view(B, n, -1), rows=(0, n))
+            q0, nq = w.q_begin, n - w.q_begin
+            q = torch.empty(B, nq if stage != "topk" else 1, cfg.q_heads, cfg.head_dim, dtype=bf, device=device)
+            iq = torch.empty(B, nq, cfg.idx_heads, cfg.idx_dim, dtype=bf, device=device)
+            for s in range(B):  # rows [q0, n) of each sequence
+                for name, t in (("q", q), ("idx_q", iq)):
+                    if name == "q" and stage == "topk":
+                        continue
+                    L_ = w.row_len(name)
+                    synth.fill_device(w.seed(s), synth.TENSOR_IDS[name], q0 * L_, nq * L_, t[s].data_ptr())
             self.pre = {"q": q, "idx_q": iq,
                         "out": torch.empty_like(q),
-                        "sel": torch.empty(B, n, cfg.k_blocks, dtype=torch.int32, device=device),
-                        "nsel": torch.empty(B, n, dtype=torch.int32, device=device)}
+                        "sel": torch.empty(B, nq, cfg.k_blocks, dtype=torch.int32, device=device),
+                        "nsel": torch.empty(B, nq, dtype=torch.int32, device=device)}
+            if q0:
+                L.compress(0, q0 // w.r)  # the existing cache's pooled keys
         else:
             L.compress(0, n // w.r)
         self.dec = []
@@ -239,7 +248,7 @@ class Bench:
                 })
         # Workspaces allocated before timing.
         if w.prefill:
-            L.workspace(qsa.OP_TOPK_BLOCKS, n)
+            L.workspace(qsa.OP_TOPK_BLOCKS, n - w.q_begin)
         if S:
             L.workspace(qsa.OP_DECODE_STEP)
         self.dec_graph, self.dec_graphs_1, self.graph_kernels = None, [], 0
@@ -265,17 +274,18 @@ class Bench:
             from block_sparse_long_02_b200 import OP_TOPK_BLOCKS, qsa_topk_blocks
 
             p = self.pre
-            L.compress(0, w.n // w.r)
+            nq = w.n - w.q_begin
+            L.compress(w.q_begin // w.r, w.n // w.r)
             if mark:
                 mark("compress")
-            qsa_topk_blocks(self.cfg, w.batch, p["idx_q"], 0, w.n, L.pooled, L.cap, None, 0, p["sel"], p["nsel"],
-                            L.workspace(OP_TOPK_BLOCKS, w.n))
+            qsa_topk_blocks(self.cfg, w.batch, p["idx_q"], w.q_begin, nq, L.pooled, L.cap, None, 0, p["sel"],
+                            p["nsel"], L.workspace(OP_TOPK_BLOCKS, nq))
             if mark:
                 mark("topk")
             return
         if self.pre is not None:
             p = self.pre
-            L.prefill(p["q"], p["idx_q"], 0, w.n, p["out"], p["sel"], p["nsel"], mark=mark)
+            L.prefill(p["q"], p["idx_q"], w.q_begin, w.n - w.q_begin, p["out"], p["sel"], p["nsel"], mark=mark)
         if self.dec_graph is not None:
             self.dec_graph.replay()
             self.graph_launches += self.graph_kernels
@@ -301,7 +311,8 @@ class Bench:
             host_out.append((pin_like(self.pre["out"]), self.pre["out"]))
         for c in (L.k_cache, L.v_cache, L.idx_k_cache):
             for s in range(B):
-                dst = c[s, :n]
+                # the step's new rows (a chunked prefill's earlier rows are cache state)
+                dst = c[s, w.q_begin if w.prefill else 0:n]
                 host_in.append((pin_like(dst), dst))
         for d in self.dec:
             for nm in ("q", "k", "v", "idx_q", "idx_k"):
@@ -421,7 +432,7 @@ def run_cuda(args, w, rank, world):
     ds = stages[dom]
     roofline = {"bound": ds["bound"], "achieved": ds["achieved"],
                 "peak": pk["hbm_gbs"] if ds["bound"] == "hbm" else pk["bf16_tflops_sustained"],
-                "unit": ds["unit"], "frac": ds["frac"], "traffic": traffic_for(dom), "kernel": dom,
+                "unit": ds["unit"], "frac": ds["frac"], "traffic": traffic_for(w.name, dom), "kernel": dom,
                 "peak_source": pk["source"] + (" (sustained bf16)" if ds["bound"] == "tensor" else " (copy)")}
 
     res = {
@@ -429,11 +440,14 @@ def run_cuda(args, w, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded counter-based N(0,1) bf16 inputs with planted needle blocks",
-        "config": {"workload": w.name, "n": w.n, "batch": w.batch, "decode_steps": w.decode_steps, "r": w.r,
+        "config": {"workload": w.name, "n": w.n, "q_begin": w.q_begin, "batch": w.batch,
+                   "decode_steps": w.decode_steps, "r": w.r,
                    "K": w.K, "k_B": w.k_blocks, "indexer": f"{w.idx_heads}x{w.idx_dim} MQA",
                    "core": f"GQA {w.q_heads}q/{w.kv_heads}kv d={w.head_dim}",
                    "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (K/V 2.1 GB, q 8.6 GB); decode steps back to back",
+                   "l2": (f"inputs larger than L2 (K/V cache {2 * w.batch * w.total * w.kv_heads * w.head_dim * 2 / 1e9:.1f} GB"
+                          f" gathered, q {w.batch * (w.n - w.q_begin) * w.q_heads * w.head_dim * 2 / 1e9:.2f} GB);"
+                          " decode steps back to back"),
                    "decode_launch": "eager calls" if b.dec_graph is None else "CUDA graph replay of the steps"},
         "roofline": roofline, "stages": stages,
         "gpu_launches": int(launches),
@@ -489,18 +503,22 @@ class OracleTimer:
         total = 0.0
         parts = {}
         if w.prefill:
-            nb = n // r
+            q0 = w.q_begin
+            nb = n // r - q0 // r
             b = min(blocks, nb)
             t = time.perf_counter()
             self.o.compress(self.idx_k, b)
             tc = (time.perf_counter() - t) * nb / max(b, 1)
-            pos = sorted(set([int((k + 0.5) * n / rows) for k in range(rows)] + [n - 1]))
+            pos = sorted(set([q0 + int((k + 0.5) * (n - q0) / rows) for k in range(rows)] + [n - 1]))
             ts = np.array([self._row(i) for i in pos])
             x = np.array([i // r for i in pos], dtype=np.float64)
             A = np.stack([np.ones_like(x), x], 1)
-            (a, bcoef), *_ = np.linalg.lstsq(A, ts, rcond=None)
-            pairs = float((np.arange(n) // r).sum())
-            tp = n * a + bcoef * pairs
+            if len(set(x.tolist())) < 2:  # (a chunk inside one block range: constant work)
+                a, bcoef = float(ts.mean()), 0.0
+            else:
+                (a, bcoef), *_ = np.linalg.lstsq(A, ts, rcond=None)
+            pairs = float((np.arange(q0, n) // r).sum())
+            tp = (n - q0) * a + bcoef * pairs
             resid = float(np.sqrt(np.mean((A @ np.array([a, bcoef]) - ts) ** 2)))
             parts.update(compress_s=tc, prefill_rows_s=tp, fit={"a_s": a, "b_s": bcoef, "rms_resid_s": resid,
                                                                  "rows": len(pos)})
@@ -542,11 +560,11 @@ def cpu_baseline(w, rows=64, dec=2, blocks=65536):
     with one_core():
         ot = OracleTimer(w)
         t, parts = ot.sample(rows, dec, blocks)
-    tokens = (w.n if w.prefill else 0) * w.batch + w.decode_steps * w.batch
+    tokens = ((w.n - w.q_begin) if w.prefill else 0) * w.batch + w.decode_steps * w.batch
     model, ncpu = host_cpu()
     return {"value": round(tokens / t, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "cpu_model": model, "host_cores": ncpu,
-            "sample": (f"{parts.get('fit', {}).get('rows', 0)} prefill rows stratified over [0,n) fitted by "
+            "sample": (f"{parts.get('fit', {}).get('rows', 0)} prefill rows stratified over [q_begin,n) fitted by "
                        f"t(i)=a+b*floor(i/r) and extrapolated over all n; key pooling timed on {blocks} blocks "
                        f"and scaled; {dec} decode positions, scaled to {w.decode_steps} steps"),
             "extrapolated_step_s": round(t, 3), "parts": {k: (round(v, 4) if isinstance(v, float) else v)
@@ -563,7 +581,7 @@ def run_reference(args, w):
                 times.append(t)
     model, ncpu = host_cpu()
     t = float(np.mean(times))
-    tokens = (w.n if w.prefill else 0) * w.batch + w.decode_steps * w.batch
+    tokens = ((w.n - w.q_begin) if w.prefill else 0) * w.batch + w.decode_steps * w.batch
     v = tokens / t
     return {"metric": METRIC, "value": round(v, 3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(t * 1e3, 1), "higher_is_better": True,

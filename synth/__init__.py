@@ -130,7 +130,8 @@ class Workload:
     n: int                      # prefill length, or tokens already cached before decoding
     batch: int = 1
     decode_steps: int = 0       # new tokens decoded after the first n positions
-    prefill: bool = True        # every position < n is a query
+    prefill: bool = True        # every position in [q_begin, n) is a query
+    q_begin: int = 0            # positions before it form an existing cache (chunked prefill)
     r: int = 4
     K: int = 2048
     idx_heads: int = 4
@@ -269,4 +270,7 @@ WORKLOADS: Dict[str, Workload] = {
                           base_seed=0x51534104, n_needles_decode=32),
     "prefill_n1m_decode64": _w(name="prefill_n1m_decode64", n=1048576, decode_steps=64,
                                base_seed=0x51534105, n_needles_prefill=64, n_needles_decode=64),
+    # Chunked prefill against an existing cache: the last 8192 positions of a 1M context.
+    "prefill_chunk8k_n1m": _w(name="prefill_chunk8k_n1m", n=1048576, q_begin=1048576 - 8192,
+                              base_seed=0x51534106),
 }

@@ -1,0 +1,38 @@
+"""The bench's algorithmic work counts (the roofline numerators), checked against
+closed forms; host logic only."""
+from __future__ import annotations
+
+import dataclasses
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def test_full_prefill_counts_match_the_closed_forms():
+    w = dataclasses.replace(synth.WORKLOADS["prefill_n1m_decode64"], n=4096, decode_steps=0)
+    a = bench.algorithmic(w)
+    nb = w.n // w.r
+    # sum_i floor(i / r) over [0, n) = r * nb * (nb - 1) / 2 = 2 nb (nb - 1) at r = 4
+    assert a["index_flops"] == 2 * nb * (nb - 1) * w.idx_heads * w.idx_dim * 2
+    assert a["prefill_tokens"] == w.n
+    # every query attends r * min(k_B, i // r) + i % r + 1 tokens
+    tokens = sum(w.r * min(w.k_blocks, i // w.r) + i % w.r + 1 for i in range(w.n))
+    assert a["attn_gather_bytes"] == tokens * w.kv_heads * w.head_dim * 4
+    assert a["compress_bytes"] == nb * w.r * w.idx_dim * 2 + nb * w.idx_dim * 2
+
+
+def test_chunked_prefill_counts_only_the_chunk():
+    full = dataclasses.replace(synth.WORKLOADS["prefill_n1m_decode64"], n=8192, decode_steps=0)
+    chunk = dataclasses.replace(full, q_begin=8192 - 1024)
+    head = dataclasses.replace(full, n=8192 - 1024)
+    a, b, c = bench.algorithmic(full), bench.algorithmic(chunk), bench.algorithmic(head)
+    # The chunk's work is the full prefill's minus the prefix's (queries are independent).
+    for k in ("index_flops", "attn_gather_bytes", "attn_flops", "prefill_tokens", "compress_bytes"):
+        assert b[k] == a[k] - c[k], k
+    assert b["prefill_tokens"] == 1024
+    assert synth.WORKLOADS["prefill_chunk8k_n1m"].n - synth.WORKLOADS["prefill_chunk8k_n1m"].q_begin == 8192
