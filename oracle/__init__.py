@@ -82,6 +82,13 @@ class Oracle:
         L.qsa_oracle_row.argtypes = [vp, ctypes.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.qsa_oracle_decode_step.restype = ctypes.c_int64
         L.qsa_oracle_decode_step.argtypes = [vp, ctypes.c_int64] + [vp] * 13
+        L.qsa_oracle_e4m3_value.restype = ctypes.c_double
+        L.qsa_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.qsa_oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.qsa_oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.qsa_oracle_quant_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int, vp, vp]
+        L.qsa_oracle_attention_q8.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp]
+        L.qsa_oracle_scores_q8.argtypes = [vp, vp, vp, vp, ctypes.c_int64, vp]
 
     @classmethod
     def for_workload(cls, w, **kw) -> "Oracle":
@@ -193,3 +200,46 @@ class Oracle:
             _p(_u16(idx_k_new)), _p(kc), _p(vc), _p(idx_k_cache), _p(pooled), _p(w), _p(sel),
             _p(out), _p(lse))
         return {"sel": sel[:m].copy(), "nsel": int(m), "out": out, "lse": lse}
+
+    # ------------------------------------------------ low-precision (fp8) caches
+    def e4m3_value(self, code: int) -> float:
+        return float(self.lib.qsa_oracle_e4m3_value(int(code) & 0xFF))
+
+    def e4m3_encode(self, y: float) -> int:
+        return int(self.lib.qsa_oracle_e4m3_encode(float(y)))
+
+    def quant_rows(self, x: np.ndarray):
+        """bf16 rows [..., dim] -> (E4M3 codes uint8 [..., dim], fp32 scales [...])."""
+        x = _u16(x)
+        dim = x.shape[-1]
+        rows = x.size // dim
+        codes = np.empty(x.shape, dtype=np.uint8)
+        scales = np.empty(x.shape[:-1], dtype=np.float32)
+        self.lib.qsa_oracle_quant_rows(_p(x), rows, dim, _p(codes), _p(scales))
+        return codes, scales
+
+    def dequant(self, codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+        """E4M3(code) * scale in fp64, [..., dim]."""
+        table = np.array([self.e4m3_value(c) for c in range(256)])
+        return table[codes] * scales.astype(np.float64)[..., None]
+
+    def attention_q8(self, q, kc, ks, vc, vs, tokens):
+        q = _u16(q)
+        kc, vc = (np.ascontiguousarray(a, dtype=np.uint8) for a in (kc, vc))
+        ks, vs = (np.ascontiguousarray(a, dtype=np.float32) for a in (ks, vs))
+        tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+        c = self.cfg
+        out = np.empty((c.q_heads, c.head_dim))
+        lse = np.empty(c.q_heads)
+        self.lib.qsa_oracle_attention_q8(self._c, _p(q), _p(kc), _p(ks), _p(vc), _p(vs), _p(tokens), tokens.size,
+                                         _p(out), _p(lse))
+        return out, lse
+
+    def scores_q8(self, qrot, pooled_codes, pooled_scales, n_vis: int) -> np.ndarray:
+        qrot = _u16(qrot)
+        pc = np.ascontiguousarray(pooled_codes, dtype=np.uint8)
+        ps = np.ascontiguousarray(pooled_scales, dtype=np.float32)
+        assert pc.size >= n_vis * self.cfg.idx_dim and ps.size >= n_vis
+        out = np.empty(n_vis, dtype=np.float32)
+        self.lib.qsa_oracle_scores_q8(self._c, _p(qrot), _p(pc), _p(ps), n_vis, _p(out))
+        return out

@@ -312,3 +312,118 @@ int64_t qsa_oracle_decode_step(const qsa_oracle_cfg* c, int64_t p, const uint16_
     }
     return nsel;
 }
+
+/* ================================================ low-precision (fp8) caches */
+/* Reading (the "Community Quantized Version" section of the "Qwen Sparse
+ * Attention" gallery page reports a quantized variant but not its format): K,
+ * V and pooled-key rows stored as FP8 E4M3 codes (the OCP 8-bit format: 1 sign
+ * bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest
+ * finite 448, code S.1111.111 = NaN) with one fp32 scale per row:
+ *   scale = fl32(max_j |x_j| / 448),  code_j = E4M3_rne_sat(fl32(x_j / scale)),
+ *   value_j = E4M3(code_j) * scale;  an all-zero row has scale 0 and codes 0.
+ * Both divisions are done in fp64 and rounded once to fp32; since the quotient
+ * of two fp32 values rounded to 53 bits and then to 24 bits equals the
+ * correctly rounded fp32 quotient (53 >= 2*24 + 2), this is the fp32 division. */
+
+/* The value of an E4M3 code, from the format definition. */
+double qsa_oracle_e4m3_value(uint8_t code) {
+    const int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6); /* subnormal: 0.m * 2^(1 - 7) */
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* The E4M3 code nearest to y (ties to the even code, i.e. even mantissa),
+ * magnitudes above 448 saturating to 448. y must not be NaN. */
+uint8_t qsa_oracle_e4m3_encode(double y) {
+    const uint8_t sign = y < 0.0 ? 0x80 : 0x00;
+    const double a = fabs(y);
+    /* Walk the 127 non-negative finite codes (values increase with the code). */
+    uint8_t best = 0;
+    for (int c = 1; c <= 126; ++c) {
+        const double lo = qsa_oracle_e4m3_value((uint8_t)(c - 1)), hi = qsa_oracle_e4m3_value((uint8_t)c);
+        if (a >= hi) {
+            best = (uint8_t)c;
+            continue;
+        }
+        /* lo <= a < hi */
+        const double mid = 0.5 * (lo + hi);
+        if (a > mid || (a == mid && (c & 1) == 0)) best = (uint8_t)c;
+        else best = (uint8_t)(c - 1);
+        return sign | best;
+    }
+    return sign | best; /* a >= 448: saturate */
+}
+
+static float fl32_div(double a, double b) { return (float)(a / b); }
+
+/* Quantizes `rows` rows of `dim` bf16 values. codes: [rows][dim]; scales: [rows]. */
+void qsa_oracle_quant_rows(const uint16_t* x, int64_t rows, int dim, uint8_t* codes, float* scales) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + (size_t)r * dim;
+        double amax = 0.0;
+        for (int j = 0; j < dim; ++j) {
+            const double a = fabs(bf(xr[j]));
+            if (a > amax) amax = a;
+        }
+        const float scale = amax > 0.0 ? fl32_div(amax, 448.0) : 0.0f;
+        scales[r] = scale;
+        for (int j = 0; j < dim; ++j)
+            codes[(size_t)r * dim + j] = scale > 0.0f ? qsa_oracle_e4m3_encode(fl32_div(bf(xr[j]), scale)) : 0;
+    }
+}
+
+/* a7 on fp8 caches: as qsa_oracle_attention with K and V values
+ * E4M3(code) * scale (exact in fp64). kc, vc: codes [tokens][kv_heads][d];
+ * ks, vs: scales [tokens][kv_heads]. */
+void qsa_oracle_attention_q8(const qsa_oracle_cfg* c, const uint16_t* q, const uint8_t* kc, const float* ks,
+                             const uint8_t* vc, const float* vs, const int64_t* tokens, int64_t ntok,
+                             double* out, double* lse) {
+    const int d = c->head_dim, hkv = c->kv_heads, group = c->q_heads / c->kv_heads;
+    const double sm = c->sm_scale > 0.0 ? c->sm_scale : 1.0 / sqrt((double)d);
+    double* lg = (double*)malloc(sizeof(double) * (size_t)(ntok > 0 ? ntok : 1));
+    for (int h = 0; h < c->q_heads; ++h) {
+        const int kv = h / group;  /* GQA: contiguous groups of q heads */
+        double mx = -INFINITY;
+        for (int64_t t = 0; t < ntok; ++t) {
+            const size_t row = (size_t)tokens[t] * hkv + kv;
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j)
+                acc += (qsa_oracle_e4m3_value(kc[row * d + j]) * ks[row]) * bf(q[(size_t)h * d + j]);
+            lg[t] = sm * acc;
+            if (lg[t] > mx) mx = lg[t];
+        }
+        double z = 0.0;
+        double* o = out + (size_t)h * d;
+        for (int j = 0; j < d; ++j) o[j] = 0.0;
+        for (int64_t t = 0; t < ntok; ++t) {
+            const double w = exp(lg[t] - mx);
+            z += w;
+            const size_t row = (size_t)tokens[t] * hkv + kv;
+            for (int j = 0; j < d; ++j) o[j] += w * (qsa_oracle_e4m3_value(vc[row * d + j]) * vs[row]);
+        }
+        for (int j = 0; j < d; ++j) o[j] /= z;
+        if (lse) lse[h] = mx + log(z);
+    }
+    free(lg);
+}
+
+/* a4 on fp8 pooled keys: I_ib = sum_h ReLU(<q_i^h, E4M3(code_b) * scale_b>). */
+void qsa_oracle_scores_q8(const qsa_oracle_cfg* c, const uint16_t* qrot, const uint8_t* pooled,
+                          const float* pscale, int64_t n_vis, float* scores) {
+    const int dim = c->idx_dim;
+    for (int64_t b = 0; b < n_vis; ++b) {
+        double sum = 0.0;
+        for (int h = 0; h < c->idx_heads; ++h) {
+            double acc = 0.0;
+            for (int j = 0; j < dim; ++j)
+                acc += (qsa_oracle_e4m3_value(pooled[(size_t)b * dim + j]) * pscale[b]) * bf(qrot[(size_t)h * dim + j]);
+            sum += acc > 0.0 ? acc : 0.0; /* ReLU */
+        }
+        scores[b] = (float)sum;
+    }
+}

@@ -327,4 +327,95 @@ def pin_decode_matches_prefill_row(make):
     assert np.array_equal(pooled, full_pooled)
 
 
+# ---------------------------------------------------------------- fp8 caches
+# Reading (the pages name a quantized variant but not its format): OCP FP8 E4M3
+# codes with one fp32 scale per row, scale = fl32(max|x| / 448).
+
+def pin_e4m3_codec_matches_library(make):
+    """Every code decodes, and every fp32 value within the finite range encodes,
+    as torch's float8_e4m3fn (an independent implementation of the OCP format
+    with round-to-nearest-even) does."""
+    import torch
+
+    o = make()
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([o.e4m3_value(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert (np.isnan(mine) == nan).all() and (mine[~nan] == ref[~nan]).all()
+    rng = np.random.default_rng(8)
+    grid = ref[~nan]
+    mids = (np.sort(np.unique(grid))[1:] + np.sort(np.unique(grid))[:-1]) / 2  # exact ties
+    ys = np.concatenate([rng.uniform(-448, 448, 3000), rng.uniform(-0.02, 0.02, 3000),
+                         np.exp(rng.uniform(-12, 6, 2000)) * rng.choice([-1, 1], 2000), mids, grid])
+    ys = ys.astype(np.float32)
+    lib = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    enc = np.array([o.e4m3_encode(float(y)) for y in ys], dtype=np.uint8)
+    # (+0 and -0 are both fine for a zero input)
+    same = (enc == lib) | ((ys == 0) & ((enc & 0x7F) == 0) & ((lib & 0x7F) == 0))
+    assert same.all(), ys[~same][:5]
+    # Saturation beyond the largest finite value (448, code 0x7E).
+    assert o.e4m3_encode(1000.0) == 0x7E and o.e4m3_encode(-1e30) == 0xFE and o.e4m3_encode(464.0) == 0x7E
+
+
+def pin_quant_rows_closed_forms(make):
+    """scale = max|x| / 448 (fp32); a row already on the scaled E4M3 grid comes
+    back exactly; an all-zero row has scale 0 and codes 0; the round trip error
+    is at most half a unit in the last place of the code."""
+    o = make()
+    rng = np.random.default_rng(9)
+    grid = np.array([o.e4m3_value(c) for c in range(127)])  # non-negative finite values
+    x = np.zeros((4, 128))
+    for r in range(3):
+        v = rng.choice(grid, 128) * rng.choice([-1, 1], 128)
+        v[rng.integers(128)] = 448.0 * (1 if r % 2 else -1)
+        x[r] = v * 2.0 ** (r - 3)  # exact in bf16 (at most 4 significant bits)
+    xb = _bits(x.astype(np.float32))
+    codes, scales = o.quant_rows(xb)
+    assert scales[0] == np.float32(2.0 ** -3) and scales[1] == np.float32(2.0 ** -2) and scales[3] == 0.0
+    back = o.dequant(codes, scales)
+    assert np.array_equal(back[:3], x[:3]) and (codes[3] == 0).all()
+    # Random rows: |x - E4M3(code) * scale| <= 2^-4 |x| (normal codes) or 2^-10 scale (subnormal).
+    y = rng.standard_normal((64, 128)).astype(np.float32) * np.exp(rng.uniform(-8, 8, (64, 1))).astype(np.float32)
+    yb = _bits(y)
+    yv = np.array([[float(np.uint32(int(v) << 16).view(np.float32)) for v in row] for row in yb])
+    c2, s2 = o.quant_rows(yb)
+    err = np.abs(o.dequant(c2, s2) - yv)
+    amax = np.abs(yv).max(axis=1)
+    assert np.allclose(s2, (amax / 448.0).astype(np.float32), rtol=0, atol=0)
+    bound = np.maximum(2.0 ** -4 * np.abs(yv), 2.0 ** -10 * s2[:, None].astype(np.float64)) * (1 + 2.0 ** -20)
+    assert (err <= bound).all()
+
+
+def pin_q8_attention_and_scores_on_exact_values(make):
+    """On K, V and pooled-key rows that the format holds exactly, the fp8-cache
+    attention and scores equal the bf16 ones (same values, same arithmetic)."""
+    w = GQA
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    rng = np.random.default_rng(10)
+    grid = np.array([o.e4m3_value(c) for c in range(127)])
+    n, hk, d = 40, w.kv_heads, w.head_dim
+
+    def exact_rows(shape):
+        v = rng.choice(grid, shape) * rng.choice([-1, 1], shape)
+        v[..., 0] = 448.0
+        return (v * 2.0 ** rng.integers(-9, -5, shape[:-1] + (1,))).astype(np.float32)
+
+    k = exact_rows((n, hk, d))
+    v = exact_rows((n, hk, d))
+    kb, vb = _bits(k), _bits(v)
+    kc, ks = o.quant_rows(kb)
+    vc, vs = o.quant_rows(vb)
+    q = _bits(rng.standard_normal((w.q_heads, d)).astype(np.float32))
+    toks = np.array([0, 3, 4, 5, 17, 30, 31, 39], dtype=np.int64)
+    out, lse = o.attention(q, kb.reshape(n, -1), vb.reshape(n, -1), toks)
+    out8, lse8 = o.attention_q8(q, kc, ks, vc, vs, toks)
+    assert np.abs(out8 - out).max() < 1e-12 and np.abs(lse8 - lse).max() < 1e-12
+    pk = exact_rows((12, d))
+    pb = _bits(pk)
+    pc, ps = o.quant_rows(pb)
+    qr = _bits(rng.standard_normal((w.idx_heads, d)).astype(np.float32))
+    assert np.array_equal(o.scores_q8(qr, pc, ps, 12), o.scores(qr, pb, 12))
+
+
 ALL_PINS = [v for kname, v in sorted(globals().items()) if kname.startswith("pin_")]

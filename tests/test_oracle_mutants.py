@@ -34,6 +34,11 @@ MUTANTS = {
     "gqa_modulo": ("const int kvh = h / g;", "const int kvh = h % c->kv_heads;"),
     "values_from_keys": ("const uint16_t* vr = vc +", "const uint16_t* vr = kc +"),
     "decode_pool_early": ("if ((p + 1) % c->r == 0) {", "if (p % c->r == 0) {"),
+    "e4m3_bias_8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_ties_up": ("if (a > mid || (a == mid && (c & 1) == 0)) best", "if (a >= mid) best"),
+    "quant_scale_max_normal_240": ("fl32_div(amax, 448.0)", "fl32_div(amax, 240.0)"),
+    "q8_value_scale_dropped": ("o[j] += w * (qsa_oracle_e4m3_value(vc[row * d + j]) * vs[row]);",
+                               "o[j] += w * qsa_oracle_e4m3_value(vc[row * d + j]);"),
 }
 
 
