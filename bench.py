@@ -47,8 +47,11 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def algorithmic(w):
-    """Per-step algorithmic work (the units the roofline divides by)."""
+def algorithmic(w, kv="bf16"):
+    """Per-step algorithmic work (the units the roofline divides by). kv="fp8":
+    the prefill attention gathers 128-byte E4M3 code rows plus a 4-byte scale
+    per row, and the step quantizes the prefill's K/V rows (2 bytes read, 1
+    written per value, 4 bytes per row scale)."""
     r, kB, n, q0 = w.r, w.k_blocks, w.n, w.q_begin
     i = np.arange(q0, n, dtype=np.int64)
     vis = i // r
@@ -60,7 +63,8 @@ def algorithmic(w):
     out = {
         "compress_bytes": (nb * r * w.idx_dim * 2 + nb * w.idx_dim * 2) if w.prefill else 0,
         "index_flops": pairs * w.idx_heads * w.idx_dim * 2,
-        "attn_gather_bytes": sum_t * w.kv_heads * d * 2 * 2,
+        "attn_gather_bytes": sum_t * w.kv_heads * (d * 2 * 2 if kv == "bf16" else (d + 4) * 2),
+        "quantize_bytes": ((n - q0) * w.kv_heads * 2 * (d * 3 + 4)) if (w.prefill and kv == "fp8") else 0,
         "attn_flops": sum_t * w.q_heads * d * 4,
         "prefill_tokens": (n - q0) if w.prefill else 0,
     }
@@ -75,7 +79,7 @@ def algorithmic(w):
     out["decode_bytes"] = dec * w.batch
     out["decode_tokens"] = dec_tok * w.batch
     out["prefill_tokens"] *= w.batch
-    for k in ("compress_bytes", "index_flops", "attn_gather_bytes", "attn_flops"):
+    for k in ("compress_bytes", "index_flops", "attn_gather_bytes", "attn_flops", "quantize_bytes"):
         out[k] *= w.batch
     return out
 
@@ -188,12 +192,13 @@ def job_value(tokens_per_rank: float, ms_max: float, world: int) -> float:
 
 # ----------------------------------------------------------------------------- CUDA arm
 class Bench:
-    def __init__(self, w, device, stage="all"):
+    def __init__(self, w, device, stage="all", kv="bf16"):
         import block_sparse_long_02_b200 as qsa
         from block_sparse_long_02_b200.layer import QSALayer
 
         self.qsa, self.w, self.dev = qsa, w, device
         self.stage = stage
+        self.kv = kv
         cfg = qsa.Config.of(w)
         self.cfg = cfg
         B, n, S = w.batch, w.n, w.decode_steps
@@ -251,6 +256,8 @@ class Bench:
             L.workspace(qsa.OP_TOPK_BLOCKS, n - w.q_begin)
         if S:
             L.workspace(qsa.OP_DECODE_STEP)
+        if kv == "fp8" and w.prefill and w.q_begin:
+            L.quantize_kv(0, w.q_begin)  # the existing cache is held in fp8
         self.dec_graph, self.dec_graphs_1, self.graph_kernels = None, [], 0
         self.graph_launches = 0  # kernels launched by graph replays so far
         torch.cuda.synchronize()
@@ -285,7 +292,17 @@ class Bench:
             return
         if self.pre is not None:
             p = self.pre
-            L.prefill(p["q"], p["idx_q"], w.q_begin, w.n - w.q_begin, p["out"], p["sel"], p["nsel"], mark=mark)
+            if self.kv == "fp8":
+                # The prefill's new K/V rows to E4M3 codes (the caches' other rows
+                # were quantized in set-up), then the prefill on the fp8 caches.
+                L.quantize_kv(w.q_begin, w.n)
+                if mark:
+                    mark("quantize")
+                L.prefill_q8(p["q"], p["idx_q"], w.q_begin, w.n - w.q_begin, p["out"], p["sel"], p["nsel"],
+                             mark=mark)
+            else:
+                L.prefill(p["q"], p["idx_q"], w.q_begin, w.n - w.q_begin, p["out"], p["sel"], p["nsel"],
+                          mark=mark)
         if self.dec_graph is not None:
             self.dec_graph.replay()
             self.graph_launches += self.graph_kernels
@@ -343,7 +360,7 @@ class Bench:
 
 def run_cuda(args, w, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
-    b = Bench(w, dev, stage=args.stage)
+    b = Bench(w, dev, stage=args.stage, kv=args.kv)
     qsa = b.qsa
     for k in range(args.warmup):
         b.step()
@@ -386,11 +403,12 @@ def run_cuda(args, w, rank, world):
         prev = e
     ms = max_over_ranks(ms, world, dev)
 
-    alg = algorithmic(w)
+    alg = algorithmic(w, args.kv)
     pk = peaks()
     tokens = alg["prefill_tokens"] + alg["decode_tokens"]
     stages = {}
     defs = {"compress": ("hbm", alg["compress_bytes"]), "topk": ("tensor", alg["index_flops"]),
+            "quantize": ("hbm", alg["quantize_bytes"]),
             "attention": ("hbm", alg["attn_gather_bytes"]), "decode": ("hbm", alg["decode_bytes"])}
     for name, t in stage_ms.items():
         bound, amount = defs[name]
@@ -432,13 +450,14 @@ def run_cuda(args, w, rank, world):
     ds = stages[dom]
     roofline = {"bound": ds["bound"], "achieved": ds["achieved"],
                 "peak": pk["hbm_gbs"] if ds["bound"] == "hbm" else pk["bf16_tflops_sustained"],
-                "unit": ds["unit"], "frac": ds["frac"], "traffic": traffic_for(w.name, dom), "kernel": dom,
+                "unit": ds["unit"], "frac": ds["frac"], "traffic": traffic_for(w.name + ("" if args.kv == "bf16" else "+fp8"), dom), "kernel": dom,
                 "peak_source": pk["source"] + (" (sustained bf16)" if ds["bound"] == "tensor" else " (copy)")}
 
     res = {
         "metric": METRIC, "value": round(job_value(tokens, ms, world), 2), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if args.kv == "bf16" else "bf16 (K/V caches fp8 E4M3)",
         "data": "synthetic: seeded counter-based N(0,1) bf16 inputs with planted needle blocks",
         "config": {"workload": w.name, "n": w.n, "q_begin": w.q_begin, "batch": w.batch,
                    "decode_steps": w.decode_steps, "r": w.r,
@@ -448,7 +467,9 @@ def run_cuda(args, w, rank, world):
                    "l2": (f"inputs larger than L2 (K/V cache {2 * w.batch * w.total * w.kv_heads * w.head_dim * 2 / 1e9:.1f} GB"
                           f" gathered, q {w.batch * (w.n - w.q_begin) * w.q_heads * w.head_dim * 2 / 1e9:.2f} GB);"
                           " decode steps back to back"),
-                   "decode_launch": "eager calls" if b.dec_graph is None else "CUDA graph replay of the steps"},
+                   "decode_launch": "eager calls" if b.dec_graph is None else "CUDA graph replay of the steps",
+                   "kv_cache": ("bf16" if args.kv == "bf16" else
+                                "fp8 E4M3 + per-row fp32 scale for the prefill attention (decode on bf16 caches)")},
         "roofline": roofline, "stages": stages,
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -607,6 +628,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="decode steps as eager calls, not CUDA graph replays")
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
+                    help="core K/V cache format of the prefill attention (fp8: E4M3 codes, per-row scales)")
     ap.add_argument("--stage", choices=["all", "topk"], default="all",
                     help="topk: time only key pooling + the fused indexer (for profiling)")
     ap.add_argument("--n", type=int, default=None, help="override the workload's sequence length")

@@ -26,7 +26,8 @@ OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 
 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
-           "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection"]
+           "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection", "qsa_quantize_rows",
+           "qsa_sparse_attention_q8"]
 
 
 class QSAError(RuntimeError):
@@ -83,6 +84,9 @@ _SIGS = {
     "qsa_decode_step": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
                         _vp, _vp, _sz, _vp],
     "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
+    "qsa_quantize_rows": [_vp, _i64, _i32, _vp, _vp, _vp],
+    "qsa_sparse_attention_q8": [_CFG, _i32, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
+                                _sz, _vp],
     "qsa_decode_step_noalloc": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp,
                                 _vp, _vp, _vp],
 }
@@ -172,6 +176,23 @@ def qsa_sparse_attention(cfg: Config, batch: int, q: torch.Tensor, q_begin: int,
     _check(lib().qsa_sparse_attention(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache),
                                      _ptr(v_cache), cap, _ptr(sel), _ptr(nsel), _ptr(out), _ptr(lse),
                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def qsa_quantize_rows(x: torch.Tensor, rows: int, dim: int, codes: torch.Tensor, scales: torch.Tensor,
+                      stream=None) -> None:
+    """FP8 E4M3 rows with one fp32 scale per row (see include/qsa.h)."""
+    _check(lib().qsa_quantize_rows(_ptr(x), rows, dim, _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def qsa_sparse_attention_q8(cfg: Config, batch: int, q: torch.Tensor, q_begin: int, nq: int,
+                            k_codes: torch.Tensor, k_scales: torch.Tensor, v_codes: torch.Tensor,
+                            v_scales: torch.Tensor, cap: int, sel: torch.Tensor, nsel: torch.Tensor,
+                            out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                            ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().qsa_sparse_attention_q8(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_codes),
+                                        _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), cap, _ptr(sel), _ptr(nsel),
+                                        _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
+                                        _stream(stream)))
 
 
 def qsa_decode_step(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, idx_k, k_cache, v_cache,

@@ -306,6 +306,44 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
                       "sparse attention");
 }
 
+qsa_status qsa_quantize_rows(const qsa_bf16* x, int64_t rows, int32_t dim, uint8_t* codes, float* scales,
+                             qsa_stream stream) {
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(codes);
+    if (!scales || ((uintptr_t)scales & 3u)) return fail(QSA_ERR_INVALID_ARG, "scales NULL or misaligned");
+    if (rows < 0) return fail(QSA_ERR_INVALID_ARG, "rows=%lld", (long long)rows);
+    if (dim != 64 && dim != 128 && dim != 256) return fail(QSA_ERR_UNSUPPORTED, "dim=%d (64, 128 or 256)", dim);
+    if (rows == 0) return QSA_OK;
+    return cuda_check(qsa::launch_quantize_rows(x, rows, dim, codes, scales, (cudaStream_t)stream),
+                      "quantize rows");
+}
+
+qsa_status qsa_sparse_attention_q8(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin,
+                                   int64_t nq, const uint8_t* k_codes, const float* k_scales,
+                                   const uint8_t* v_codes, const float* v_scales, int64_t cap,
+                                   const int32_t* sel, const int32_t* nsel, qsa_bf16* out, float* lse,
+                                   void* ws, size_t ws_bytes, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(k_codes);
+    REQUIRE_PTR(v_codes);
+    REQUIRE_PTR(sel);
+    REQUIRE_PTR(out);
+    if (!k_scales || !v_scales || ((uintptr_t)k_scales & 3u) || ((uintptr_t)v_scales & 3u))
+        return fail(QSA_ERR_INVALID_ARG, "k_scales/v_scales NULL or misaligned");
+    if (!nsel || ((uintptr_t)nsel & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel NULL or misaligned");
+    if (lse && ((uintptr_t)lse & 3u)) return fail(QSA_ERR_INVALID_ARG, "lse misaligned");
+    if (batch < 1 || cap < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (q_begin + nq > cap) return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
+    (void)ws;
+    (void)ws_bytes;
+    if (nq == 0) return QSA_OK;
+    return cuda_check(qsa::launch_sparse_attention_q8(L, batch, q, q_begin, nq, k_codes, k_scales, v_codes,
+                                                      v_scales, cap, sel, nsel, out, lse, (cudaStream_t)stream),
+                      "sparse attention (fp8 caches)");
+}
+
 qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* pos,
                            const qsa_bf16* q, const qsa_bf16* k, const qsa_bf16* v,
                            const qsa_bf16* idx_q, const qsa_bf16* idx_k, qsa_bf16* k_cache,

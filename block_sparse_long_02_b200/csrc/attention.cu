@@ -35,8 +35,10 @@ constexpr float LN2 = 0.6931471805599453f;
 
 struct Work {
     const uint16_t* q;     // first query head of the group: [G][128]
-    const uint16_t* kc;    // sequence base of k_cache
-    const uint16_t* vc;
+    const void* kc;        // sequence base of the K cache (bf16, or fp8 codes)
+    const void* vc;
+    const float* ks;       // fp8 caches: sequence base of the row scales [cap][kv_heads]
+    const float* vs;
     const int32_t* sel;    // selection row
     int64_t i;             // query position
     int64_t cur;           // its block, i / r
@@ -89,15 +91,39 @@ __device__ __forceinline__ void load_q_frags(const uint16_t* q, int G, int lane,
     }
 }
 
+// As load_q_frags, converted to f16 (exact while |q| < 65504, the f16 range).
+template <int NT>
+__device__ __forceinline__ void load_q_frags_f16(const uint16_t* q, int G, int lane, uint32_t (&qb)[NT][8][2]) {
+    load_q_frags<NT>(q, G, lane, qb);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) qb[nt][ks][k] = pack_f16x2(bf16_lo(qb[nt][ks][k]), bf16_hi(qb[nt][ks][k]));
+}
+
+// fp8 caches, per warp: an f16 tile (K rows then V rows, 256-byte swizzled
+// rows as in the bf16 ring) and STAGES staging slots of codes and scales.
+constexpr int Q8_TILE = CT * 256 * 2;
+constexpr int Q8_STAGE = CT * 128 * 2 + CT * 8;  // K codes, V codes, K scales, V scales
+static_assert(Q8_TILE + STAGES * Q8_STAGE + 8 <= WARP_SMEM, "fp8 layout fits the warp's area");
+
 // The warp's units [u0, u1) against the query fragments qb. sel_lane: lane l
 // holds selection entry u0 + l when that unit is a selection entry (any
 // value otherwise); later entries are read when their chunk is issued.
-template <int NT>
+// Q8: the caches hold FP8 E4M3 codes with per-row scales; each chunk is
+// gathered as codes, then converted into the warp's f16 tile (values times
+// their row scale), the logits take the key rows' scales, and both products
+// run in f16 (qb then holds f16 fragments).
+template <int NT, bool Q8 = false>
 __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lane, const uint32_t (&qb)[NT][8][2],
                                             int32_t sel_lane, WarpState<NT>& st) {
     uint16_t* ring = reinterpret_cast<uint16_t*>(wsm);
-    uint32_t* vmask = reinterpret_cast<uint32_t*>(wsm + STAGES * STAGE_BYTES + STAGES * CT * 8);
+    uint32_t* vmask = reinterpret_cast<uint32_t*>(
+        Q8 ? wsm + Q8_TILE + STAGES * Q8_STAGE : wsm + STAGES * STAGE_BYTES + STAGES * CT * 8);
     const uint32_t ring_s = smem_u32(ring);
+    const uint32_t q8_stage_s = ring_s + Q8_TILE;  // stage k at q8_stage_s + k * Q8_STAGE
     const int g = lane >> 2;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -135,17 +161,42 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         }
         const uint32_t valid = __ballot_sync(0xffffffffu, tk >= 0) & ((1u << CT) - 1u);
         if (lane == 0) vmask[stg] = valid;
-        const uint32_t kbase = ring_s + stg * STAGE_BYTES;
-        const uint32_t vbase = kbase + CT * 256;
+        if (Q8) {
+            // Codes: 16 rows x 128 bytes per cache, 16-byte pieces; scales: lanes
+            // 0-15 fetch the K row scales, lanes 16-31 the V row scales.
+            const uint32_t kb8 = q8_stage_s + stg * Q8_STAGE, vb8 = kb8 + CT * 128;
+            const uint8_t* kc8 = static_cast<const uint8_t*>(w.kc);
+            const uint8_t* vc8 = static_cast<const uint8_t*>(w.vc);
 #pragma unroll
-        for (int k = 0; k < (CT * 16) / 32; ++k) {
-            const int idx = lane + k * 32;
-            const int row = idx >> 4, ch = idx & 15;
+            for (int k = 0; k < (CT * 8) / 32; ++k) {
+                const int idx = lane + k * 32;
+                const int row = idx >> 3, ch = idx & 7;
+                const int32_t tkr = __shfl_sync(0xffffffffu, tk, row);
+                const bool ok = tkr >= 0;
+                const size_t off = (size_t)(ok ? tkr : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 16;
+                cp_async16_zfill(kb8 + row * 128 + ch * 16, kc8 + off, ok);
+                cp_async16_zfill(vb8 + row * 128 + ch * 16, vc8 + off, ok);
+            }
+            const int row = lane & (CT - 1);
             const int32_t tkr = __shfl_sync(0xffffffffu, tk, row);
             const bool ok = tkr >= 0;
-            const size_t off = (size_t)(ok ? tkr : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 8;
-            cp_async16_zfill(kbase + swz256(row, ch), w.kc + off, ok);
-            cp_async16_zfill(vbase + swz256(row, ch), w.vc + off, ok);
+            const size_t so = (size_t)(ok ? tkr : 0) * w.kv_heads + w.g;
+            cp_async4_zfill(kb8 + 2 * CT * 128 + (lane < CT ? 0 : CT * 4) + row * 4, (lane < CT ? w.ks : w.vs) + so, ok);
+        } else {
+            const uint32_t kbase = ring_s + stg * STAGE_BYTES;
+            const uint32_t vbase = kbase + CT * 256;
+            const uint16_t* kc16 = static_cast<const uint16_t*>(w.kc);
+            const uint16_t* vc16 = static_cast<const uint16_t*>(w.vc);
+#pragma unroll
+            for (int k = 0; k < (CT * 16) / 32; ++k) {
+                const int idx = lane + k * 32;
+                const int row = idx >> 4, ch = idx & 15;
+                const int32_t tkr = __shfl_sync(0xffffffffu, tk, row);
+                const bool ok = tkr >= 0;
+                const size_t off = (size_t)(ok ? tkr : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 8;
+                cp_async16_zfill(kbase + swz256(row, ch), kc16 + off, ok);
+                cp_async16_zfill(vbase + swz256(row, ch), vc16 + off, ok);
+            }
         }
     };
 
@@ -164,7 +215,43 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         cp_async_wait<STAGES - 1>();
         __syncwarp();
         const int stg = c % STAGES;
-        const uint32_t kbase = ring_s + stg * STAGE_BYTES;
+        uint32_t kbase = ring_s + stg * STAGE_BYTES;
+        float ksc0 = 1.f, ksc1 = 1.f;  // fp8: the key rows' scales of tokens g, g + 8
+        if (Q8) {
+            // Codes -> f16 tiles: K exact, V times its row scale (rounded to
+            // f16); lane handles 16-byte code pieces (16 values) of rows idx / 8.
+            kbase = ring_s;
+            const uint8_t* st8 = wsm + Q8_TILE + stg * Q8_STAGE;
+            const float* ksc = reinterpret_cast<const float*>(st8 + 2 * CT * 128);
+            const float* vsc = ksc + CT;
+#pragma unroll
+            for (int k = 0; k < (CT * 8) / 32; ++k) {
+                const int idx = lane + k * 32;
+                const int row = idx >> 3, ch = idx & 7;
+#pragma unroll
+                for (int kv = 0; kv < 2; ++kv) {
+                    const uint4 c16 = *reinterpret_cast<const uint4*>(st8 + kv * CT * 128 + row * 128 + ch * 16);
+                    const uint32_t w4[4] = {c16.x, c16.y, c16.z, c16.w};
+                    uint32_t h[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        h[2 * j] = e4m3x2_to_f16x2((uint16_t)(w4[j] & 0xFFFFu));
+                        h[2 * j + 1] = e4m3x2_to_f16x2((uint16_t)(w4[j] >> 16));
+                    }
+                    if (kv == 1) {  // V: times the row's scale, in f16
+                        const uint32_t s2 = pack_f16x2(vsc[row], vsc[row]);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) h[j] = hmul2(h[j], s2);
+                    }
+                    uint8_t* tile = wsm + kv * CT * 256;
+                    *reinterpret_cast<uint4*>(tile + swz256(row, 2 * ch)) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4*>(tile + swz256(row, 2 * ch + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
+                }
+            }
+            ksc0 = ksc[g];
+            ksc1 = ksc[g + 8];
+            __syncwarp();
+        }
         const uint32_t vbase = kbase + CT * 256;
         const uint32_t valid = vmask[stg];
 
@@ -174,7 +261,6 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-#pragma unroll
         // (two independent accumulation chains over the k-steps, summed after)
         float s2[NT][4];
 #pragma unroll
@@ -186,8 +272,12 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4(kbase + swz256(krow, ks * 2 + kch), a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                mma_bf16_16816((ks & 1) ? s2[nt] : s[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                if (Q8)
+                    mma_f16_16816((ks & 1) ? s2[nt] : s[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+                else
+                    mma_bf16_16816((ks & 1) ? s2[nt] : s[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+            }
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -201,8 +291,8 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const float x0 = v0 ? s[nt][e] * w.scale_log2 : -INFINITY;
-                const float x1 = v1 ? s[nt][2 + e] * w.scale_log2 : -INFINITY;
+                const float x0 = v0 ? s[nt][e] * ksc0 * w.scale_log2 : -INFINITY;
+                const float x1 = v1 ? s[nt][2 + e] * ksc1 * w.scale_log2 : -INFINITY;
                 float mx = fmaxf(x0, x1);
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -223,8 +313,8 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
             }
             // P^T operand: the two 8x8 blocks (tokens 0-7, 8-15) of this tile,
             // rounded to bf16 and transposed.
-            pb[nt][0] = movmatrix_trans(pack_bf16x2(s[nt][0], s[nt][1]));
-            pb[nt][1] = movmatrix_trans(pack_bf16x2(s[nt][2], s[nt][3]));
+            pb[nt][0] = movmatrix_trans(Q8 ? pack_f16x2(s[nt][0], s[nt][1]) : pack_bf16x2(s[nt][0], s[nt][1]));
+            pb[nt][1] = movmatrix_trans(Q8 ? pack_f16x2(s[nt][2], s[nt][3]) : pack_bf16x2(s[nt][2], s[nt][3]));
         }
         // O^T += V^T P^T: rows = dims 16 i + g (+8), columns = heads.
 #pragma unroll
@@ -232,7 +322,12 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4_trans(vbase + swz256(vrow, 2 * i + vch), a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(st.o[nt][i], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                if (Q8)
+                    mma_f16_16816(st.o[nt][i], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+                else
+                    mma_bf16_16816(st.o[nt][i], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            }
         }
         __syncwarp();
     }
@@ -310,12 +405,13 @@ __device__ __forceinline__ void write_out(const WarpState<NT>& st, int G, uint16
 }
 
 // Prefill: CTA = one query; warp w -> kv head kv0 + (w % GH), unit split w / GH.
-template <int NT>
+// Q8: fp8 caches (codes with row scales ks, vs [batch][cap][kv_heads]).
+template <int NT, bool Q8>
 __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
-    const uint16_t* __restrict__ q, int64_t q_begin, int64_t nq, const uint16_t* __restrict__ kc,
-    const uint16_t* __restrict__ vc, int64_t cap, const int32_t* __restrict__ sel,
-    const int32_t* __restrict__ nsel, uint16_t* __restrict__ out, float* __restrict__ lse,
-    int q_heads, int kv_heads, int r, int kB, float scale_log2) {
+    const uint16_t* __restrict__ q, int64_t q_begin, int64_t nq, const void* __restrict__ kc,
+    const void* __restrict__ vc, const float* __restrict__ ks, const float* __restrict__ vs, int64_t cap,
+    const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel, uint16_t* __restrict__ out,
+    float* __restrict__ lse, int q_heads, int kv_heads, int r, int kB, float scale_log2) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t j = blockIdx.x;
@@ -333,8 +429,13 @@ __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
     const int units = ns + 1;
     Work w;
     w.q = q + ((size_t)row * q_heads + (size_t)g * G) * kHeadDim;
-    w.kc = kc + (size_t)s * cap * kv_heads * kHeadDim;
-    w.vc = vc + (size_t)s * cap * kv_heads * kHeadDim;
+    const size_t seq_elems = (size_t)s * cap * kv_heads * kHeadDim;  // elements (bf16) or bytes (fp8)
+    w.kc = Q8 ? (const void*)(static_cast<const uint8_t*>(kc) + seq_elems)
+              : (const void*)(static_cast<const uint16_t*>(kc) + seq_elems);
+    w.vc = Q8 ? (const void*)(static_cast<const uint8_t*>(vc) + seq_elems)
+              : (const void*)(static_cast<const uint16_t*>(vc) + seq_elems);
+    w.ks = Q8 ? ks + (size_t)s * cap * kv_heads : nullptr;
+    w.vs = Q8 ? vs + (size_t)s * cap * kv_heads : nullptr;
     w.sel = sel + (size_t)row * kB;
     w.i = i;
     w.cur = i / r;
@@ -350,10 +451,13 @@ __global__ void __launch_bounds__(WARPS * 32) prefill_attention_kernel(
 
     uint8_t* wsm = smem + warp * WARP_SMEM;
     uint32_t qb[NT][8][2];
-    load_q_frags<NT>(w.q, G, lane, qb);
+    if (Q8)
+        load_q_frags_f16<NT>(w.q, G, lane, qb);
+    else
+        load_q_frags<NT>(w.q, G, lane, qb);
     const int32_t sel_lane = (w.u0 + lane < w.u1 && w.u0 + lane < ns) ? w.sel[w.u0 + lane] : -1;
     WarpState<NT> st;
-    warp_attend<NT>(w, wsm, lane, qb, sel_lane, st);
+    warp_attend<NT, Q8>(w, wsm, lane, qb, sel_lane, st);
 
     if (NS > 1) {
         // Splits > 0 park their state in their own smem; split 0 merges.
@@ -425,6 +529,7 @@ __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
     w.q = q + ((size_t)s * q_heads + (size_t)g * G) * kHeadDim;
     w.kc = kc + (size_t)s * cap * kv_heads * kHeadDim;
     w.vc = vc + (size_t)s * cap * kv_heads * kHeadDim;
+    w.ks = w.vs = nullptr;
     w.sel = sel + (size_t)s * kB;
     w.tail_unit = kB;
     w.u0 = (int)((int64_t)units * split / S);
@@ -517,11 +622,27 @@ cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_
     const int GH = L.kv_heads < WARPS ? L.kv_heads : WARPS;
     dim3 grid((unsigned)nq, (unsigned)batch, (unsigned)(L.kv_heads / GH));
     const int G = L.q_heads / L.kv_heads;
-    auto kern = G > 8 ? prefill_attention_kernel<2> : prefill_attention_kernel<1>;
+    auto kern = G > 8 ? prefill_attention_kernel<2, false> : prefill_attention_kernel<1, false>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     note_launch();
-    kern<<<grid, WARPS * 32, SMEM, st>>>(q, q_begin, nq, kc, vc, cap, sel, nsel, out, lse, L.q_heads, L.kv_heads,
-                                         L.r, L.kB, L.sm_scale * LOG2E);
+    kern<<<grid, WARPS * 32, SMEM, st>>>(q, q_begin, nq, kc, vc, nullptr, nullptr, cap, sel, nsel, out, lse,
+                                         L.q_heads, L.kv_heads, L.r, L.kB, L.sm_scale * LOG2E);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sparse_attention_q8(const LayerDims& L, int batch, const uint16_t* q, int64_t q_begin,
+                                       int64_t nq, const uint8_t* k8, const float* ks, const uint8_t* v8,
+                                       const float* vs, int64_t cap, const int32_t* sel, const int32_t* nsel,
+                                       uint16_t* out, float* lse, cudaStream_t st) {
+    if (nq <= 0 || batch <= 0) return cudaSuccess;
+    const int GH = L.kv_heads < WARPS ? L.kv_heads : WARPS;
+    dim3 grid((unsigned)nq, (unsigned)batch, (unsigned)(L.kv_heads / GH));
+    const int G = L.q_heads / L.kv_heads;
+    auto kern = G > 8 ? prefill_attention_kernel<2, true> : prefill_attention_kernel<1, true>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    note_launch();
+    kern<<<grid, WARPS * 32, SMEM, st>>>(q, q_begin, nq, k8, v8, ks, vs, cap, sel, nsel, out, lse, L.q_heads,
+                                         L.kv_heads, L.r, L.kB, L.sm_scale * LOG2E);
     return cudaGetLastError();
 }
 

@@ -90,10 +90,18 @@ cudaError_t launch_sparse_attention(const LayerDims& L, int batch, const uint16_
                                     const uint16_t* vc, int64_t cap, const int32_t* sel,
                                     const int32_t* nsel, uint16_t* out, float* lse,
                                     cudaStream_t st);
+cudaError_t launch_sparse_attention_q8(const LayerDims& L, int batch, const uint16_t* q, int64_t q_begin,
+                                       int64_t nq, const uint8_t* k8, const float* ks, const uint8_t* v8,
+                                       const float* vs, int64_t cap, const int32_t* sel, const int32_t* nsel,
+                                       uint16_t* out, float* lse, cudaStream_t st);
 cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
                                     const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
                                     uint16_t* out, cudaStream_t st);
+
+// quant.cu: FP8 E4M3 rows with one fp32 scale per row (dim 64, 128 or 256).
+cudaError_t launch_quantize_rows(const uint16_t* x, int64_t rows, int dim, uint8_t* codes, float* scales,
+                                 cudaStream_t st);
 
 // decode.cu. Per-sequence selection state in the decode workspace.
 constexpr int kDecodeCand = 4096;  // candidates of the threshold digit kept for the final pick

@@ -17,8 +17,8 @@ from typing import Optional
 
 import torch
 
-from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step,
-               qsa_sparse_attention, qsa_topk_blocks, qsa_workspace_size)
+from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step, qsa_quantize_rows,
+               qsa_sparse_attention, qsa_sparse_attention_q8, qsa_topk_blocks, qsa_workspace_size)
 
 
 class QSALayer:
@@ -64,6 +64,42 @@ class QSALayer:
             mark("topk")
         qsa_sparse_attention(self.cfg, self.batch, q, q_begin, nq, self.k_cache, self.v_cache, self.cap, sel,
                              nsel, out, lse, None, stream)
+        if mark:
+            mark("attention")
+
+    # ------------------------------------------------ fp8 (E4M3) core K/V caches
+    def quantize_kv(self, begin: int, end: int, stream=None) -> None:
+        """FP8 copies of the core K/V cache rows [begin, end) of every sequence
+        (allocated on first use: codes [batch][cap][kv_heads][head_dim] uint8,
+        scales [batch][cap][kv_heads] fp32), read by prefill_q8."""
+        if getattr(self, "k8", None) is None:
+            shape = self.k_cache.shape
+            self.k8 = torch.zeros(shape, dtype=torch.uint8, device=self.device)
+            self.v8 = torch.zeros_like(self.k8)
+            self.ks = torch.zeros(shape[:3], dtype=torch.float32, device=self.device)
+            self.vs = torch.zeros_like(self.ks)
+        h, d = self.cfg.kv_heads, self.cfg.head_dim
+        for s in range(self.batch):
+            for src, codes, scales in ((self.k_cache, self.k8, self.ks), (self.v_cache, self.v8, self.vs)):
+                qsa_quantize_rows(src[s, begin:end], (end - begin) * h, d, codes[s, begin:end], scales[s, begin:end],
+                                  stream)
+
+    def prefill_q8(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin: int, nq: int, out: torch.Tensor,
+                   sel: torch.Tensor, nsel: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None,
+                   mark=None) -> None:
+        """As prefill, with the sparse attention reading the fp8 K/V caches
+        (quantize_kv must cover positions < q_begin + nq)."""
+        r = self.cfg.r
+        self.compress(q_begin // r, (q_begin + nq) // r, stream)
+        if mark:
+            mark("compress")
+        ws = self.workspace(OP_TOPK_BLOCKS, nq)
+        qsa_topk_blocks(self.cfg, self.batch, idx_q, q_begin, nq, self.pooled, self.cap, None, 0, sel, nsel,
+                        ws, stream)
+        if mark:
+            mark("topk")
+        qsa_sparse_attention_q8(self.cfg, self.batch, q, q_begin, nq, self.k8, self.ks, self.v8, self.vs, self.cap,
+                                sel, nsel, out, lse, None, stream)
         if mark:
             mark("attention")
 

@@ -158,6 +158,39 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
                                 const int32_t* nsel, qsa_bf16* out, float* lse, void* ws,
                                 size_t ws_bytes, qsa_stream stream);
 
+/* ---- Low-precision (fp8) caches ----
+ * The "Qwen Sparse Attention" gallery page ("Community Quantized Version")
+ * reports a quantized variant but not its format. This library's reading: a
+ * row of dim bf16 values is stored as dim FP8 E4M3 codes (the OCP format: 1
+ * sign bit, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448)
+ * and one fp32 scale,
+ *   scale = fl32(max|x| / 448),  code = E4M3(fl32(x / scale)) rounded to
+ *   nearest even, magnitudes beyond 448 saturating,  value = E4M3(code)*scale;
+ * an all-zero row has scale 0 and codes 0. */
+
+/* Quantizes rows: x [rows][dim] bf16 -> codes [rows][dim] uint8 and scales
+ * [rows] fp32. dim is 64, 128 or 256 (QSA_ERR_UNSUPPORTED otherwise). Device
+ * pointers; x and codes 16-byte aligned, scales 4-byte aligned. Asynchronous
+ * on `stream`. Used for the core K/V cache rows (one row per token and kv
+ * head) and for the pooled keys (one row per block). */
+qsa_status qsa_quantize_rows(const qsa_bf16* x, int64_t rows, int32_t dim, uint8_t* codes, float* scales,
+                             qsa_stream stream);
+
+/* a6+a7 as qsa_sparse_attention, on fp8 core K/V caches:
+ * k_codes, v_codes: [batch][cap][kv_heads][head_dim] uint8, 16-byte aligned;
+ * k_scales, v_scales: [batch][cap][kv_heads] fp32, one per (token, kv head) row.
+ * The key codes enter the logit product exactly (as f16, with the query
+ * converted to f16: exact for |q| below 65504) and each logit is multiplied by
+ * its key row's scale in fp32; the values enter the P.V product as f16
+ * (code times its row's scale, rounded to f16: full precision between 6e-5 and
+ * 65504 in magnitude) with the probabilities as f16. Other arguments, errors
+ * and the workspace as for qsa_sparse_attention. */
+qsa_status qsa_sparse_attention_q8(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin,
+                                   int64_t nq, const uint8_t* k_codes, const float* k_scales,
+                                   const uint8_t* v_codes, const float* v_scales, int64_t cap,
+                                   const int32_t* sel, const int32_t* nsel, qsa_bf16* out, float* lse,
+                                   void* ws, size_t ws_bytes, qsa_stream stream);
+
 /* One decode step for every sequence s, at p = pos[s] (its current length):
  *   a8: append k, v (-> k_cache/v_cache row p) and idx_k (-> idx_k_cache row p);
  *   a3'..a7: the new token is query p: score blocks b < floor(p/r), select,
@@ -229,8 +262,8 @@ const char* qsa_last_error(void);
 uint64_t qsa_launch_count(void);
 
 /* Fault injection, for tests of the failure path (the pages have no
- * counterpart; SURVEY-style host-side fault tests need a wait that runs out
- * without faulting the GPU). Process-wide, off by default.
+ * counterpart; such a test needs a bounded device wait that runs out without
+ * faulting the GPU). Process-wide, off by default.
  *   mode 0: normal operation (every bounded device wait gives up after 10 s).
  *   mode 1: the fused qsa_topk_blocks path (k_B <= 512) withholds the pooled-key
  *           tiles of each CTA's first unit of work, so the MMA's bounded wait

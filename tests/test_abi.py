@@ -12,7 +12,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared():
     src = open(os.path.join(ROOT, "include", "qsa.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(qsa_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(qsa_[a-z0-9_]+)\s*\(", src)))
 
 
 @pytest.fixture(scope="module")
@@ -74,3 +74,15 @@ def test_fault_injection_arguments_are_validated(qsa):
                 qsa.qsa_set_fault_injection(mode, wait)
             assert e.value.status == 1, (mode, wait)
     qsa.qsa_set_fault_injection(0)
+
+
+def test_quantize_rows_validation_launches_nothing(qsa):
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    lib.qsa_quantize_rows.restype = ctypes.c_int
+    lib.qsa_quantize_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p]
+    p = ctypes.c_void_p(4096)  # aligned, never dereferenced
+    assert lib.qsa_quantize_rows(p, 10, 96, p, p, None) == 2  # dim not 64/128/256: unsupported
+    assert lib.qsa_quantize_rows(None, 10, 128, p, p, None) == 1
+    assert lib.qsa_quantize_rows(p, 10, 128, p, ctypes.c_void_p(4098), None) == 1  # scales misaligned
+    assert lib.qsa_quantize_rows(p, 0, 128, p, p, None) == 0  # nothing to do

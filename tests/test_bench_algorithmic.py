@@ -36,3 +36,12 @@ def test_chunked_prefill_counts_only_the_chunk():
         assert b[k] == a[k] - c[k], k
     assert b["prefill_tokens"] == 1024
     assert synth.WORKLOADS["prefill_chunk8k_n1m"].n - synth.WORKLOADS["prefill_chunk8k_n1m"].q_begin == 8192
+
+
+def test_fp8_caches_count_code_rows_and_scales():
+    w = dataclasses.replace(synth.WORKLOADS["prefill_n1m_decode64"], n=4096, decode_steps=0)
+    a, b = bench.algorithmic(w), bench.algorithmic(w, "fp8")
+    rows = a["attn_gather_bytes"] // (w.head_dim * 2)  # gathered (token, kv head, K or V) rows
+    assert b["attn_gather_bytes"] == rows * (w.head_dim + 4)
+    assert b["quantize_bytes"] == w.n * w.kv_heads * 2 * (w.head_dim * 3 + 4) and a["quantize_bytes"] == 0
+    assert b["index_flops"] == a["index_flops"] and b["attn_flops"] == a["attn_flops"]

@@ -554,3 +554,68 @@ def test_decode_graph_replay_matches_eager(qsa):
         assert torch.equal(getattr(La, name), getattr(Lb, name)), name
     assert qsa.qsa_workspace_status(La.workspace(qsa.OP_DECODE_STEP)) == 0
     assert qsa.qsa_workspace_status(Lb.workspace(qsa.OP_DECODE_STEP)) == 0
+
+
+# ----------------------------------------------------------------------------- fp8 (E4M3) caches
+def test_quantize_rows_matches_oracle_bit_for_bit(qsa):
+    """Codes and scales of the row quantizer equal the oracle's: random rows
+    over many magnitudes, a zero row, rows on the scaled E4M3 grid (exact ties
+    between codes) and rows whose values saturate."""
+    rng = np.random.default_rng(81)
+    rows = 3000
+    x = (rng.standard_normal((rows, 128)) * np.exp(rng.uniform(-12, 12, (rows, 1)))).astype(np.float32)
+    x[5] = 0.0
+    o = oracle.Oracle()
+    grid = np.array([o.e4m3_value(c) for c in range(127)])
+    for r in range(10, 60):  # midpoints between adjacent codes, times a power of two
+        a = rng.integers(0, 125, 128)
+        x[r] = ((grid[a] + grid[a + 1]) / 2 * rng.choice([-1, 1], 128) * 2.0 ** int(rng.integers(-8, 8))).astype(
+            np.float32)
+        x[r, 0] = 448.0 * 2.0 ** int(rng.integers(-8, 8))
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    ref_codes, ref_scales = o.quant_rows(xb.view(torch.int16).numpy().view(np.uint16))
+    codes = torch.full((rows, 128), 7, dtype=torch.uint8, device="cuda")
+    scales = torch.full((rows,), -1.0, dtype=torch.float32, device="cuda")
+    qsa.qsa_quantize_rows(xb.cuda(), rows, 128, codes, scales)
+    torch.cuda.synchronize()
+    assert np.array_equal(scales.cpu().numpy(), ref_scales)
+    g = codes.cpu().numpy()
+    # +0 and -0 codes of a zero value are the same value
+    same = (g == ref_codes) | (((g & 0x7F) == 0) & ((ref_codes & 0x7F) == 0))
+    assert same.all(), np.argwhere(~same)[:5]
+
+
+@pytest.mark.parametrize("q_heads,kv_heads", [(32, 4), (16, 1)])
+def test_prefill_with_fp8_caches_matches_oracle(qsa, q_heads, kv_heads):
+    """Prefill with the attention on fp8 K/V caches: the selection is the
+    bf16 path's; each output row matches the oracle's fp8-cache attention on
+    the GPU's own codes, scales and selection (several tiles, ragged tail)."""
+    n = 3000 + 37
+    w = synth.Workload(name="t", n=n, K=512, q_heads=q_heads, kv_heads=kv_heads, base_seed=0xF8 + q_heads)
+    cfg, L = _layer(qsa, w, n)
+    _fill_caches(w, L, n)
+    L.quantize_kv(0, n)
+    iq = dev_full(w, "idx_q", n).view(1, n, 4, 128).contiguous()
+    qq = dev_full(w, "q", n).view(1, n, q_heads, 128).contiguous()
+    out = torch.empty(1, n, q_heads, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(1, n, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(1, n, dtype=torch.int32, device="cuda")
+    lse = torch.empty(1, n, q_heads, dtype=torch.float32, device="cuda")
+    L.prefill_q8(qq, iq, 0, n, out, sel, nsel, lse)
+    torch.cuda.synchronize()
+    o = _oracle(w, cfg)
+    k8, v8 = L.k8[0].cpu().numpy(), L.v8[0].cpu().numpy()
+    ks, vs = L.ks[0].cpu().numpy(), L.vs[0].cpu().numpy()
+    # The GPU's quantized caches are the oracle's quantization of the bf16 caches.
+    rk, rks = o.quant_rows(bits(L.k_cache)[0, :n].reshape(n, kv_heads, 128))
+    assert np.array_equal(rks, ks[:n])
+    assert (((rk == k8[:n]) | (((rk & 0x7F) == 0) & ((k8[:n] & 0x7F) == 0)))).all()
+    q_bits = bits(qq)[0].reshape(n, q_heads, 128)
+    g_out, g_lse = out.float().cpu().numpy()[0], lse.cpu().numpy()[0]
+    g_sel, g_n = sel.cpu().numpy()[0], nsel.cpu().numpy()[0]
+    rng = np.random.default_rng(n)
+    for i in sorted(set(rng.integers(0, n, 24).tolist() + [0, 1, 3, 2047, 2048, n - 1])):
+        toks = o.token_set(g_sel[i, : g_n[i]], i)
+        ref, ref_lse = o.attention_q8(q_bits[i], k8, ks, v8, vs, toks)
+        check_attention(g_out[i], ref, f"row {i}")
+        assert np.abs(g_lse[i] - ref_lse).max() <= LSE_ATOL, i
