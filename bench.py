@@ -64,7 +64,9 @@ def algorithmic(w, kv="bf16"):
         "compress_bytes": (nb * r * w.idx_dim * 2 + nb * w.idx_dim * 2) if w.prefill else 0,
         "index_flops": pairs * w.idx_heads * w.idx_dim * 2,
         "attn_gather_bytes": sum_t * w.kv_heads * (d * 2 * 2 if kv == "bf16" else (d + 4) * 2),
-        "quantize_bytes": ((n - q0) * w.kv_heads * 2 * (d * 3 + 4)) if (w.prefill and kv == "fp8") else 0,
+        "quantize_bytes": (((n - q0) * w.kv_heads * 2 * (d * 3 + 4))
+                           + ((n // r - q0 // r) * (w.idx_dim * 3 + 4) if w.decode_steps else 0))
+                          if (w.prefill and kv == "fp8") else 0,
         "attn_flops": sum_t * w.q_heads * d * 4,
         "prefill_tokens": (n - q0) if w.prefill else 0,
     }
@@ -74,7 +76,10 @@ def algorithmic(w, kv="bf16"):
         p = w.n + s
         nb = p // r
         t = r * min(kB, nb) + p % r + 1
-        dec += nb * w.idx_dim * 2 + t * w.kv_heads * d * 2 * 2
+        if kv == "fp8":  # code rows plus 4-byte scales
+            dec += nb * (w.idx_dim + 4) + t * w.kv_heads * (d + 4) * 2
+        else:
+            dec += nb * w.idx_dim * 2 + t * w.kv_heads * d * 2 * 2
         dec_tok += 1
     out["decode_bytes"] = dec * w.batch
     out["decode_tokens"] = dec_tok * w.batch
@@ -256,8 +261,12 @@ class Bench:
             L.workspace(qsa.OP_TOPK_BLOCKS, n - w.q_begin)
         if S:
             L.workspace(qsa.OP_DECODE_STEP)
-        if kv == "fp8" and w.prefill and w.q_begin:
-            L.quantize_kv(0, w.q_begin)  # the existing cache is held in fp8
+        if kv == "fp8":
+            # The caches already present before the timed step are held in fp8.
+            cached = w.q_begin if w.prefill else n
+            if cached:
+                L.quantize_kv(0, cached)
+                L.quantize_pooled(0, cached // w.r)
         self.dec_graph, self.dec_graphs_1, self.graph_kernels = None, [], 0
         self.graph_launches = 0  # kernels launched by graph replays so far
         torch.cuda.synchronize()
@@ -270,9 +279,10 @@ class Bench:
             return
         qsa = self.qsa
         n0 = qsa.qsa_launch_count()
-        self.dec_graph = self.L.capture_decode(self.dec)
+        q8 = self.kv == "fp8"
+        self.dec_graph = self.L.capture_decode(self.dec, q8)
         self.graph_kernels = qsa.qsa_launch_count() - n0
-        self.dec_graphs_1 = [self.L.capture_decode([d]) for d in self.dec]
+        self.dec_graphs_1 = [self.L.capture_decode([d], q8) for d in self.dec]
         torch.cuda.synchronize()
 
     def step(self, mark=None):
@@ -300,6 +310,10 @@ class Bench:
                     mark("quantize")
                 L.prefill_q8(p["q"], p["idx_q"], w.q_begin, w.n - w.q_begin, p["out"], p["sel"], p["nsel"],
                              mark=mark)
+                if self.dec:  # the decode score stream reads fp8 pooled keys
+                    L.quantize_pooled(w.q_begin // w.r, w.n // w.r)
+                    if mark:
+                        mark("quantize")
             else:
                 L.prefill(p["q"], p["idx_q"], w.q_begin, w.n - w.q_begin, p["out"], p["sel"], p["nsel"],
                           mark=mark)
@@ -307,8 +321,9 @@ class Bench:
             self.dec_graph.replay()
             self.graph_launches += self.graph_kernels
         else:
+            dstep = L.decode_step_q8 if self.kv == "fp8" else L.decode_step
             for d in self.dec:
-                L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+                dstep(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
         if mark and self.dec:
             mark("decode")
 
@@ -437,7 +452,8 @@ def run_cuda(args, w, rank, world):
             if b.dec_graphs_1:
                 b.dec_graphs_1[k].replay()
             else:
-                b.L.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+                (b.L.decode_step_q8 if b.kv == "fp8" else b.L.decode_step)(
+                    d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
             a1.record(stream)
             evs.append((a0, a1))
         torch.cuda.synchronize()
@@ -469,7 +485,7 @@ def run_cuda(args, w, rank, world):
                           " decode steps back to back"),
                    "decode_launch": "eager calls" if b.dec_graph is None else "CUDA graph replay of the steps",
                    "kv_cache": ("bf16" if args.kv == "bf16" else
-                                "fp8 E4M3 + per-row fp32 scale for the prefill attention (decode on bf16 caches)")},
+                                "fp8 E4M3 codes + one fp32 scale per row: core K/V, and pooled keys for decode")},
         "roofline": roofline, "stages": stages,
         "gpu_launches": int(launches),
         "clocks": clk,

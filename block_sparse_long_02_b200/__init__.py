@@ -27,7 +27,7 @@ OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
            "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection", "qsa_quantize_rows",
-           "qsa_sparse_attention_q8"]
+           "qsa_sparse_attention_q8", "qsa_decode_step_q8"]
 
 
 class QSAError(RuntimeError):
@@ -85,6 +85,7 @@ _SIGS = {
                         _vp, _vp, _sz, _vp],
     "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
     "qsa_quantize_rows": [_vp, _i64, _i32, _vp, _vp, _vp],
+    "qsa_decode_step_q8": [_CFG, _i32] + [_vp] * 14 + [_i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "qsa_sparse_attention_q8": [_CFG, _i32, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
                                 _sz, _vp],
     "qsa_decode_step_noalloc": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp,
@@ -193,6 +194,16 @@ def qsa_sparse_attention_q8(cfg: Config, batch: int, q: torch.Tensor, q_begin: i
                                         _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), cap, _ptr(sel), _ptr(nsel),
                                         _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
                                         _stream(stream)))
+
+
+def qsa_decode_step_q8(cfg: Config, batch: int, pos, q, k, v, idx_q, idx_k, k_codes, k_scales, v_codes, v_scales,
+                       idx_k_cache, pooled, pooled_codes, pooled_scales, cap: int, rms_w, out, sel_out=None,
+                       nsel_out=None, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().qsa_decode_step_q8(ctypes.byref(cfg.c()), batch, _ptr(pos), _ptr(q), _ptr(k), _ptr(v), _ptr(idx_q),
+                                   _ptr(idx_k), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+                                   _ptr(idx_k_cache), _ptr(pooled), _ptr(pooled_codes), _ptr(pooled_scales), cap,
+                                   _ptr(rms_w), _ptr(out), _ptr(sel_out), _ptr(nsel_out), _ptr(ws),
+                                   0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def qsa_decode_step(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, idx_k, k_cache, v_cache,

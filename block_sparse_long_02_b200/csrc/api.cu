@@ -344,12 +344,15 @@ qsa_status qsa_sparse_attention_q8(const qsa_config* cfg, int32_t batch, const q
                       "sparse attention (fp8 caches)");
 }
 
-qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* pos,
-                           const qsa_bf16* q, const qsa_bf16* k, const qsa_bf16* v,
-                           const qsa_bf16* idx_q, const qsa_bf16* idx_k, qsa_bf16* k_cache,
-                           qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap,
-                           const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
-                           void* ws, size_t ws_bytes, qsa_stream stream) {
+}  // extern "C"
+
+namespace {
+// The decode step's launches; q8 non-null: fp8 K/V and pooled-key caches.
+qsa_status decode_step_impl(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,
+                            const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q, const qsa_bf16* idx_k,
+                            qsa_bf16* k_cache, qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled,
+                            int64_t cap, const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
+                            void* ws, size_t ws_bytes, qsa_stream stream, const qsa::Q8Caches* q8) {
     qsa::LayerDims L;
     TRY(make_dims(cfg, &L));
     REQUIRE_PTR(pos);
@@ -358,8 +361,10 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     REQUIRE_PTR(v);
     REQUIRE_PTR(idx_q);
     REQUIRE_PTR(idx_k);
-    REQUIRE_PTR(k_cache);
-    REQUIRE_PTR(v_cache);
+    if (!q8) {
+        REQUIRE_PTR(k_cache);
+        REQUIRE_PTR(v_cache);
+    }
     REQUIRE_PTR(idx_k_cache);
     REQUIRE_PTR(pooled);
     REQUIRE_PTR(out);
@@ -367,6 +372,7 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     if (sel_out && ((uintptr_t)sel_out & 3u)) return fail(QSA_ERR_INVALID_ARG, "sel_out misaligned");
     if (nsel_out && ((uintptr_t)nsel_out & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel_out misaligned");
     if (batch < 1 || cap < 1) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (q8 && L.head_dim != 128) return fail(QSA_ERR_UNSUPPORTED, "fp8 caches need head_dim 128");
     const DecodeWs w = decode_layout(L, batch, cap);
     TRY(check_ws(ws, ws_bytes, w.total));
     char* base = (char*)ws;
@@ -381,13 +387,41 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
     sw.cand = reinterpret_cast<uint2*>(base + w.cand);
     cudaStream_t st = (cudaStream_t)stream;
     TRY(cuda_check(qsa::launch_decode_score(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
-                                            pooled, cap, rms_w, scores, sw, status, st),
+                                            pooled, cap, rms_w, scores, sw, status, q8, st),
                    "decode score"));
     TRY(cuda_check(qsa::launch_decode_select(L, batch, pos, cap, scores, sw, sel, nsel, status, st),
                    "decode select"));
-    return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel,
-                                                   nsel, out, st),
+    return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel, nsel, out, q8, st),
                       "decode attention");
+}
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* pos,
+                           const qsa_bf16* q, const qsa_bf16* k, const qsa_bf16* v,
+                           const qsa_bf16* idx_q, const qsa_bf16* idx_k, qsa_bf16* k_cache,
+                           qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap,
+                           const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
+                           void* ws, size_t ws_bytes, qsa_stream stream) {
+    return decode_step_impl(cfg, batch, pos, q, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache, pooled, cap,
+                            rms_w, out, sel_out, nsel_out, ws, ws_bytes, stream, nullptr);
+}
+
+qsa_status qsa_decode_step_q8(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,
+                              const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q, const qsa_bf16* idx_k,
+                              uint8_t* k_codes, float* k_scales, uint8_t* v_codes, float* v_scales,
+                              qsa_bf16* idx_k_cache, qsa_bf16* pooled, uint8_t* pooled_codes,
+                              float* pooled_scales, int64_t cap, const float* rms_w, qsa_bf16* out,
+                              int32_t* sel_out, int32_t* nsel_out, void* ws, size_t ws_bytes, qsa_stream stream) {
+    REQUIRE_PTR(k_codes);
+    REQUIRE_PTR(v_codes);
+    REQUIRE_PTR(pooled_codes);
+    for (const float* p : {k_scales, v_scales, pooled_scales})
+        if (!p || ((uintptr_t)p & 3u)) return fail(QSA_ERR_INVALID_ARG, "a scale array is NULL or misaligned");
+    const qsa::Q8Caches q8{k_codes, k_scales, v_codes, v_scales, pooled_codes, pooled_scales};
+    return decode_step_impl(cfg, batch, pos, q, k, v, idx_q, idx_k, nullptr, nullptr, idx_k_cache, pooled, cap,
+                            rms_w, out, sel_out, nsel_out, ws, ws_bytes, stream, &q8);
 }
 
 qsa_status qsa_workspace_status(void* ws, qsa_stream stream, int32_t* status) {

@@ -510,10 +510,12 @@ __host__ __device__ constexpr int decode_recv_bytes(int G, int C) { return (G * 
 // outputs [c E / C, (c + 1) E / C) of the E = G x 128 and every CTA pushes its
 // merged slice for them into c's shared memory (remote stores, no remote
 // loads); after one cluster barrier each CTA finishes its slice locally.
-template <int NT, int DW>
+// Q8: fp8 K/V caches (codes kc, vc with row scales ks, vs).
+template <int NT, int DW, bool Q8>
 __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
     const uint16_t* __restrict__ q, const int64_t* __restrict__ pos,
-    const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc, int64_t cap,
+    const void* __restrict__ kc, const void* __restrict__ vc, const float* __restrict__ ks,
+    const float* __restrict__ vs, int64_t cap,
     const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel, uint16_t* __restrict__ out,
     int q_heads, int kv_heads, int r, int kB, float scale_log2) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -527,9 +529,13 @@ __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
     const int units = kB + 1;
     Work w;
     w.q = q + ((size_t)s * q_heads + (size_t)g * G) * kHeadDim;
-    w.kc = kc + (size_t)s * cap * kv_heads * kHeadDim;
-    w.vc = vc + (size_t)s * cap * kv_heads * kHeadDim;
-    w.ks = w.vs = nullptr;
+    const size_t seq_elems = (size_t)s * cap * kv_heads * kHeadDim;  // elements (bf16) or bytes (fp8)
+    w.kc = Q8 ? (const void*)(static_cast<const uint8_t*>(kc) + seq_elems)
+              : (const void*)(static_cast<const uint16_t*>(kc) + seq_elems);
+    w.vc = Q8 ? (const void*)(static_cast<const uint8_t*>(vc) + seq_elems)
+              : (const void*)(static_cast<const uint16_t*>(vc) + seq_elems);
+    w.ks = Q8 ? ks + (size_t)s * cap * kv_heads : nullptr;
+    w.vs = Q8 ? vs + (size_t)s * cap * kv_heads : nullptr;
     w.sel = sel + (size_t)s * kB;
     w.tail_unit = kB;
     w.u0 = (int)((int64_t)units * split / S);
@@ -543,7 +549,10 @@ __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
     // write them, and they were complete before the step's first kernel ran.
     const int64_t p = pos[s];
     uint32_t qb[NT][8][2];
-    load_q_frags<NT>(w.q, G, lane, qb);
+    if (Q8)
+        load_q_frags_f16<NT>(w.q, G, lane, qb);
+    else
+        load_q_frags<NT>(w.q, G, lane, qb);
     uint8_t* wsm = smem + warp * WARP_SMEM;
     WarpState<NT> st;
     w.cur = p / r;
@@ -557,7 +566,7 @@ __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
     w.i = p;
     if (p < 0 || p >= cap) w.u1 = w.u0;  // skipped sequence: zero output
 
-    warp_attend<NT>(w, wsm, lane, qb, sel_lane, st);
+    warp_attend<NT, Q8>(w, wsm, lane, qb, sel_lane, st);
 
     const int E = G * kHeadDim, per = E / C;
     store_state_hd<NT>(st, G, reinterpret_cast<float*>(wsm), lane);
@@ -659,7 +668,7 @@ struct DecodeShape {
 
 template <int NT, int DW>
 int decode_cluster_for(const LayerDims& L, int batch, int G) {
-    auto kern = decode_attention_kernel<NT, DW>;
+    auto kern = decode_attention_kernel<NT, DW, false>;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -702,11 +711,11 @@ DecodeShape decode_shape(const LayerDims& L, int batch, int G) {
     return {4, decode_cluster_for<NT, 4>(L, batch, G)};
 }
 
-template <int NT, int DW>
+template <int NT, int DW, bool Q8>
 cudaError_t launch_decode_attention_t(const LayerDims& L, int batch, int C, const int64_t* pos, const uint16_t* q,
-                                      const uint16_t* kc, const uint16_t* vc, int64_t cap, const int32_t* sel,
-                                      const int32_t* nsel, uint16_t* out, cudaStream_t st) {
-    auto kern = decode_attention_kernel<NT, DW>;
+                                      const void* kc, const void* vc, const float* ks, const float* vs, int64_t cap,
+                                      const int32_t* sel, const int32_t* nsel, uint16_t* out, cudaStream_t st) {
+    auto kern = decode_attention_kernel<NT, DW, Q8>;
     const int G = L.q_heads / L.kv_heads;
     const int smem = DW * WARP_SMEM + decode_recv_bytes(G, C);
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -726,8 +735,22 @@ cudaError_t launch_decode_attention_t(const LayerDims& L, int batch, int C, cons
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     note_launch();
-    return cudaLaunchKernelEx(&cfg, kern, q, pos, kc, vc, cap, sel, nsel, out, L.q_heads, L.kv_heads, L.r, L.kB,
-                              L.sm_scale * LOG2E);
+    return cudaLaunchKernelEx(&cfg, kern, q, pos, kc, vc, ks, vs, cap, sel, nsel, out, L.q_heads, L.kv_heads, L.r,
+                              L.kB, L.sm_scale * LOG2E);
+}
+
+template <int NT>
+cudaError_t launch_decode_attention_nt(const LayerDims& L, int batch, const DecodeShape& sh, const int64_t* pos,
+                                       const uint16_t* q, const void* kc, const void* vc, const float* ks,
+                                       const float* vs, bool q8, int64_t cap, const int32_t* sel, const int32_t* nsel,
+                                       uint16_t* out, cudaStream_t st) {
+    if (q8)
+        return sh.dw == 8
+                   ? launch_decode_attention_t<NT, 8, true>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st)
+                   : launch_decode_attention_t<NT, 4, true>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st);
+    return sh.dw == 8
+               ? launch_decode_attention_t<NT, 8, false>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st)
+               : launch_decode_attention_t<NT, 4, false>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st);
 }
 
 }  // namespace
@@ -735,7 +758,7 @@ cudaError_t launch_decode_attention_t(const LayerDims& L, int batch, int C, cons
 cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
                                     const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
-                                    uint16_t* out, cudaStream_t st) {
+                                    uint16_t* out, const Q8Caches* q8, cudaStream_t st) {
     if (batch <= 0) return cudaSuccess;
     const int G = L.q_heads / L.kv_heads;
     // The launch shape is chosen once per problem shape (and thread).
@@ -747,11 +770,12 @@ cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t
         std::copy(key, key + 4, cached_key);
     }
     const DecodeShape sh = cached;
-    if (G > 8)
-        return sh.dw == 8 ? launch_decode_attention_t<2, 8>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st)
-                          : launch_decode_attention_t<2, 4>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st);
-    return sh.dw == 8 ? launch_decode_attention_t<1, 8>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st)
-                      : launch_decode_attention_t<1, 4>(L, batch, sh.c, pos, q, kc, vc, cap, sel, nsel, out, st);
+    const void* k = q8 ? (const void*)q8->k8 : (const void*)kc;
+    const void* v = q8 ? (const void*)q8->v8 : (const void*)vc;
+    const float* ks = q8 ? q8->ks : nullptr;
+    const float* vs = q8 ? q8->vs : nullptr;
+    if (G > 8) return launch_decode_attention_nt<2>(L, batch, sh, pos, q, k, v, ks, vs, q8 != nullptr, cap, sel, nsel, out, st);
+    return launch_decode_attention_nt<1>(L, batch, sh, pos, q, k, v, ks, vs, q8 != nullptr, cap, sel, nsel, out, st);
 }
 
 }  // namespace qsa

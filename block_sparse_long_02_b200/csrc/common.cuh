@@ -194,6 +194,26 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
     return d;
 }
 
+// One warp quantizes a 128-value bf16 row to FP8 E4M3 codes and an fp32
+// scale: scale = fl32(max|x| / 448) (0 for an all-zero row), code =
+// E4M3(fl32(x / scale)) rounded to nearest even, saturating. Lane l handles
+// values 4 l .. 4 l + 3.
+__device__ __forceinline__ void quantize_row128_warp(const uint16_t* x, uint8_t* codes, float* scale_out,
+                                                     int lane) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(x + lane * 4);
+    const float v[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
+    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 0.f;
+    uint32_t packed = 0u;
+    if (scale > 0.f)
+        packed = (uint32_t)f32x2_to_e4m3x2(__fdiv_rn(v[0], scale), __fdiv_rn(v[1], scale)) |
+                 ((uint32_t)f32x2_to_e4m3x2(__fdiv_rn(v[2], scale), __fdiv_rn(v[3], scale)) << 16);
+    *reinterpret_cast<uint32_t*>(codes + lane * 4) = packed;
+    if (lane == 0) *scale_out = scale;
+}
+
 // Byte offset of 16-byte chunk `c` (0..15) of 256-byte row `row` in a
 // row-swizzled tile: conflict-free ldmatrix over 8 consecutive rows.
 __device__ __forceinline__ uint32_t swz256(int row, int c) {

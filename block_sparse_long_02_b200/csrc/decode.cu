@@ -61,12 +61,21 @@ __device__ __forceinline__ uint32_t dec_digit2(uint32_t key) { return (key >> 9)
 // 2 (j % 2) + 1 of chunk j / 2 as the low and high column pairs. The ReLU
 // head sum takes one shuffle; the scores go to `scores` and their top 11 key
 // bits to the sequence's histogram (zeroed by the selection after use).
+//
+// Q8 (fp8 caches): the appended K and V rows are quantized (one warp per row),
+// a block closed by the token is pooled into the bf16 pooled keys and then
+// quantized into the fp8 pooled keys, and the stream reads those: 128-byte
+// code rows (each lane's 16-byte pieces hold 16 dims, so the fixed dimension
+// permutation maps virtual chunk 2 i' + c of lane t to dims 64 i' + 16 t + 8 c),
+// converted to f16 (exact) for an f16 mma.sync; a block's ReLU head sum is
+// multiplied by its scale (scales are non-negative, so ReLU commutes).
+template <bool Q8>
 __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     const int64_t* __restrict__ pos, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
     const uint16_t* __restrict__ idx_q, const uint16_t* __restrict__ idx_k, uint16_t* __restrict__ kc,
     uint16_t* __restrict__ vc, uint16_t* __restrict__ idx_k_cache, uint16_t* __restrict__ pooled,
     int64_t cap, const float* __restrict__ rms_w, int kv_heads, int r, int kB, double eps, RopeTable rt,
-    float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status) {
+    float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status, Q8Caches q8) {
     __shared__ uint32_t hist[2048];
     __shared__ __align__(16) uint16_t qs[kIdxHeads * kIdxDim];
     __shared__ double2 cs[kIdxDim / 2];  // (sin, cos) of the query position's angles
@@ -104,14 +113,24 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
         return;
     }
     if (blockIdx.x == 0) {
-        const int row16 = kv_heads * kHeadDim / 8;  // 16-byte chunks per kv row
-        const uint4* ks = reinterpret_cast<const uint4*>(k + (size_t)s * kv_heads * kHeadDim);
-        const uint4* vs = reinterpret_cast<const uint4*>(v + (size_t)s * kv_heads * kHeadDim);
-        uint4* kd = reinterpret_cast<uint4*>(kc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
-        uint4* vd = reinterpret_cast<uint4*>(vc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
-        for (int c = tid; c < row16; c += DS_THREADS) {
-            kd[c] = ks[c];
-            vd[c] = vs[c];
+        if constexpr (Q8) {
+            for (int row = warp; row < 2 * kv_heads; row += DS_WARPS) {  // K rows, then V rows
+                const bool isk = row < kv_heads;
+                const int h = isk ? row : row - kv_heads;
+                const size_t cr = ((size_t)s * cap + p) * kv_heads + h;  // (token, kv head) row of the cache
+                quantize_row128_warp((isk ? k : v) + ((size_t)s * kv_heads + h) * kHeadDim,
+                                     (isk ? q8.k8 : q8.v8) + cr * kHeadDim, (isk ? q8.ks : q8.vs) + cr, lane);
+            }
+        } else {
+            const int row16 = kv_heads * kHeadDim / 8;  // 16-byte chunks per kv row
+            const uint4* ks = reinterpret_cast<const uint4*>(k + (size_t)s * kv_heads * kHeadDim);
+            const uint4* vs = reinterpret_cast<const uint4*>(v + (size_t)s * kv_heads * kHeadDim);
+            uint4* kd = reinterpret_cast<uint4*>(kc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
+            uint4* vd = reinterpret_cast<uint4*>(vc + ((size_t)s * cap + p) * kv_heads * kHeadDim);
+            for (int c = tid; c < row16; c += DS_THREADS) {
+                kd[c] = ks[c];
+                vd[c] = vs[c];
+            }
         }
         if (tid < kIdxDim / 8)
             reinterpret_cast<uint4*>(idx_k_cache + ((size_t)s * cap + p) * kIdxDim)[tid] =
@@ -120,9 +139,14 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
         // written by another thread of this CTA).
         if (warp == kIdxHeads && (p + 1) % r == 0) {
             const int64_t b = p / r;
+            uint16_t* prow = pooled + ((size_t)s * (cap / r) + b) * kIdxDim;
             pool_block_warp(idx_k_cache + ((size_t)s * cap + (size_t)b * r) * kIdxDim,
-                            idx_k + (size_t)s * kIdxDim, r, rms_w, eps, b * r, rt,
-                            pooled + ((size_t)s * (cap / r) + b) * kIdxDim, lane);
+                            idx_k + (size_t)s * kIdxDim, r, rms_w, eps, b * r, rt, prow, lane);
+            if constexpr (Q8) {
+                __syncwarp();  // each lane reads back the values it stored
+                const size_t pr = (size_t)s * (cap / r) + b;
+                quantize_row128_warp(prow, q8.pooled8 + pr * kIdxDim, q8.pscale + pr, lane);
+            }
         }
     }
     if (!scoring) return;  // (also: every visible block is selected, no scores needed)
@@ -132,40 +156,94 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     uint32_t bq0[8], bq1[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const int d = 32 * (j >> 1) + 8 * t + 4 * (j & 1);
+        const int i = j >> 1;
+        const int d = Q8 ? 64 * (i >> 1) + 16 * t + 8 * (i & 1) + 4 * (j & 1) : 32 * i + 8 * t + 4 * (j & 1);
         bq0[j] = g < kIdxHeads ? *reinterpret_cast<const uint32_t*>(qs + g * kIdxDim + d) : 0u;
         bq1[j] = g < kIdxHeads ? *reinterpret_cast<const uint32_t*>(qs + g * kIdxDim + d + 2) : 0u;
+        if (Q8) {  // the query in f16 (exact for its bf16 values inside the f16 range)
+            bq0[j] = pack_f16x2(bf16_lo(bq0[j]), bf16_hi(bq0[j]));
+            bq1[j] = pack_f16x2(bf16_lo(bq1[j]), bf16_hi(bq1[j]));
+        }
     }
     const uint16_t* keys = pooled + (size_t)s * pcap * kIdxDim;
+    const uint8_t* keys8 = Q8 ? q8.pooled8 + (size_t)s * pcap * kIdxDim : nullptr;
+    const float* kscale = Q8 ? q8.pscale + (size_t)s * pcap : nullptr;
     float* dst = scores + (size_t)s * pcap;
-    auto load = [&](int64_t base, uint4 (&ra)[4], uint4 (&rb)[4]) {
+    // bf16: four 16-byte pieces of each row; fp8: two (16 codes each), and the
+    // rows' scales.
+    auto load = [&](int64_t base, uint4 (&ra)[4], uint4 (&rb)[4], float& sa_, float& sb_) {
         const int64_t b0 = base + g, b1 = b0 + 8;
+        if constexpr (Q8) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            ra[i] = b0 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b0 * kIdxDim + 32 * i + 8 * t))
-                            : make_uint4(0u, 0u, 0u, 0u);
-            rb[i] = b1 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b1 * kIdxDim + 32 * i + 8 * t))
-                            : make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < 2; ++i) {
+                ra[i] = b0 < hi ? __ldg(reinterpret_cast<const uint4*>(keys8 + (size_t)b0 * kIdxDim + 64 * i + 16 * t))
+                                : make_uint4(0u, 0u, 0u, 0u);
+                rb[i] = b1 < hi ? __ldg(reinterpret_cast<const uint4*>(keys8 + (size_t)b1 * kIdxDim + 64 * i + 16 * t))
+                                : make_uint4(0u, 0u, 0u, 0u);
+            }
+            sa_ = (t == 0 && b0 < hi) ? __ldg(kscale + b0) : 0.f;
+            sb_ = (t == 0 && b1 < hi) ? __ldg(kscale + b1) : 0.f;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                ra[i] = b0 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b0 * kIdxDim + 32 * i + 8 * t))
+                                : make_uint4(0u, 0u, 0u, 0u);
+                rb[i] = b1 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b1 * kIdxDim + 32 * i + 8 * t))
+                                : make_uint4(0u, 0u, 0u, 0u);
+            }
         }
+    };
+    // fp8: 16 codes -> two virtual bf16-layout pieces of f16 pairs.
+    auto widen = [&](const uint4& c, uint4& lo4, uint4& hi4) {
+        const uint32_t w4[4] = {c.x, c.y, c.z, c.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            h[2 * j] = e4m3x2_to_f16x2((uint16_t)(w4[j] & 0xFFFFu));
+            h[2 * j + 1] = e4m3x2_to_f16x2((uint16_t)(w4[j] >> 16));
+        }
+        lo4 = make_uint4(h[0], h[1], h[2], h[3]);
+        hi4 = make_uint4(h[4], h[5], h[6], h[7]);
     };
     const int64_t step = 16 * DS_WARPS;
     int64_t base = lo + 16 * warp;
     uint4 ca[4], cb[4];
-    load(base, ca, cb);
+    float psa = 0.f, psb = 0.f;
+    load(base, ca, cb, psa, psb);
     for (; base < hi; base += step) {
         uint4 na[4], nb[4];
-        load(base + step, na, nb);  // the next group, in flight during this one
+        float nsa = 0.f, nsb = 0.f;
+        load(base + step, na, nb, nsa, nsb);  // the next group, in flight during this one
         float c[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (Q8) {
+            uint4 wa[4], wb[4];
+            widen(ca[0], wa[0], wa[1]);
+            widen(ca[1], wa[2], wa[3]);
+            widen(cb[0], wb[0], wb[1]);
+            widen(cb[1], wb[2], wb[3]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            mma_bf16_16816(c, ca[i].x, cb[i].x, ca[i].y, cb[i].y, bq0[2 * i], bq1[2 * i]);
-            mma_bf16_16816(c, ca[i].z, cb[i].z, ca[i].w, cb[i].w, bq0[2 * i + 1], bq1[2 * i + 1]);
+            for (int i = 0; i < 4; ++i) {
+                mma_f16_16816(c, wa[i].x, wb[i].x, wa[i].y, wb[i].y, bq0[2 * i], bq1[2 * i]);
+                mma_f16_16816(c, wa[i].z, wb[i].z, wa[i].w, wb[i].w, bq0[2 * i + 1], bq1[2 * i + 1]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                mma_bf16_16816(c, ca[i].x, cb[i].x, ca[i].y, cb[i].y, bq0[2 * i], bq1[2 * i]);
+                mma_bf16_16816(c, ca[i].z, cb[i].z, ca[i].w, cb[i].w, bq0[2 * i + 1], bq1[2 * i + 1]);
+            }
         }
         // Lane t = 0 holds heads 0, 1 and lane t = 1 heads 2, 3 of rows g, g + 8.
         float sa = fmaxf(c[0], 0.f) + fmaxf(c[1], 0.f);
         float sb = fmaxf(c[2], 0.f) + fmaxf(c[3], 0.f);
         sa += __shfl_xor_sync(0xffffffffu, sa, 1);
         sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+        if constexpr (Q8) {
+            sa *= psa;
+            sb *= psb;
+            psa = nsa;
+            psb = nsb;
+        }
         if (t == 0) {
             const int64_t b0 = base + g, b1 = b0 + 8;
             if (b0 < hi) {
@@ -473,7 +551,7 @@ int decode_score_ctas(int batch) {
     int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel, DS_THREADS, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<true>, DS_THREADS, 0) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     return std::max(1, per_sm * sms / std::max(batch, 1));
@@ -483,11 +561,15 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
                                 uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,
                                 int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
-                                int32_t* status, cudaStream_t st) {
-    note_launch();
-    return launch_pdl(decode_score_kernel, dim3((unsigned)decode_score_ctas(batch), (unsigned)batch),
-                      dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache, pooled, cap, rms_w,
-                      L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist, status);
+                                int32_t* status, const Q8Caches* q8, cudaStream_t st) {
+    const dim3 grid((unsigned)decode_score_ctas(batch), (unsigned)batch);
+    if (q8)
+        return launch_pdl(decode_score_kernel<true>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,
+                          idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist,
+                          status, *q8);
+    return launch_pdl(decode_score_kernel<false>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,
+                      idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist,
+                      status, Q8Caches{});
 }
 
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,

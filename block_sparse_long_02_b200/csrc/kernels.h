@@ -94,14 +94,27 @@ cudaError_t launch_sparse_attention_q8(const LayerDims& L, int batch, const uint
                                        int64_t nq, const uint8_t* k8, const float* ks, const uint8_t* v8,
                                        const float* vs, int64_t cap, const int32_t* sel, const int32_t* nsel,
                                        uint16_t* out, float* lse, cudaStream_t st);
+// q8 non-null: the K/V caches are q8's fp8 codes and scales (kc, vc unused).
 cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
                                     const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
-                                    uint16_t* out, cudaStream_t st);
+                                    uint16_t* out, const struct Q8Caches* q8, cudaStream_t st);
 
 // quant.cu: FP8 E4M3 rows with one fp32 scale per row (dim 64, 128 or 256).
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t rows, int dim, uint8_t* codes, float* scales,
                                  cudaStream_t st);
+
+// fp8 decode caches: core K/V codes [batch][cap][kv_heads][128] with row scales
+// [batch][cap][kv_heads], and the pooled keys' codes [batch][cap/r][128] with
+// block scales [batch][cap/r].
+struct Q8Caches {
+    uint8_t* k8;
+    float* ks;
+    uint8_t* v8;
+    float* vs;
+    uint8_t* pooled8;
+    float* pscale;
+};
 
 // decode.cu. Per-sequence selection state in the decode workspace.
 constexpr int kDecodeCand = 4096;  // candidates of the threshold digit kept for the final pick
@@ -120,7 +133,7 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
                                 uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,
                                 int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
-                                int32_t* status, cudaStream_t st);
+                                int32_t* status, const Q8Caches* q8, cudaStream_t st);
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
                                  const float* scores, DecodeSelWs sw, int32_t* sel, int32_t* nsel,
                                  int32_t* status, cudaStream_t st);

@@ -17,7 +17,8 @@ from typing import Optional
 
 import torch
 
-from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step, qsa_quantize_rows,
+from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step, qsa_decode_step_q8,
+               qsa_quantize_rows,
                qsa_sparse_attention, qsa_sparse_attention_q8, qsa_topk_blocks, qsa_workspace_size)
 
 
@@ -84,6 +85,26 @@ class QSALayer:
                 qsa_quantize_rows(src[s, begin:end], (end - begin) * h, d, codes[s, begin:end], scales[s, begin:end],
                                   stream)
 
+    def quantize_pooled(self, blk_begin: int, blk_end: int, stream=None) -> None:
+        """FP8 copies of the pooled keys of blocks [blk_begin, blk_end) of every
+        sequence (codes [batch][cap/r][128] uint8, scales [batch][cap/r] fp32),
+        read by decode_step_q8's score stream."""
+        if getattr(self, "pooled8", None) is None:
+            self.pooled8 = torch.zeros(self.pooled.shape, dtype=torch.uint8, device=self.device)
+            self.pscale = torch.zeros(self.pooled.shape[:2], dtype=torch.float32, device=self.device)
+        for s in range(self.batch):
+            qsa_quantize_rows(self.pooled[s, blk_begin:blk_end], blk_end - blk_begin, self.cfg.idx_dim,
+                              self.pooled8[s, blk_begin:blk_end], self.pscale[s, blk_begin:blk_end], stream)
+
+    def decode_step_q8(self, pos: torch.Tensor, q, k, v, idx_q, idx_k, out, sel_out=None, nsel_out=None,
+                       stream=None) -> None:
+        """decode_step on the fp8 caches (quantize_kv and quantize_pooled must
+        cover the cached positions and blocks)."""
+        ws = self.workspace(OP_DECODE_STEP)
+        qsa_decode_step_q8(self.cfg, self.batch, pos, q, k, v, idx_q, idx_k, self.k8, self.ks, self.v8, self.vs,
+                           self.idx_k_cache, self.pooled, self.pooled8, self.pscale, self.cap, self.rms_w, out,
+                           sel_out, nsel_out, ws, stream)
+
     def prefill_q8(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin: int, nq: int, out: torch.Tensor,
                    sel: torch.Tensor, nsel: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None,
                    mark=None) -> None:
@@ -110,7 +131,7 @@ class QSALayer:
                         self.idx_k_cache, self.pooled, self.cap, self.rms_w, out, sel_out, nsel_out, ws,
                         stream)
 
-    def capture_decode(self, steps) -> "torch.cuda.CUDAGraph":
+    def capture_decode(self, steps, q8: bool = False) -> "torch.cuda.CUDAGraph":
         """Captures the decode steps `steps` (a list of dicts with the
         decode_step arguments pos, q, k, v, idx_q, idx_k, out) into one CUDA
         graph, run by `graph.replay()`: one launch for the whole sequence of
@@ -123,7 +144,8 @@ class QSALayer:
         side.wait_stream(torch.cuda.current_stream(self.device))
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
+            step = self.decode_step_q8 if q8 else self.decode_step
             for d in steps:
-                self.decode_step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
+                step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
         torch.cuda.current_stream(self.device).wait_stream(side)
         return graph

@@ -191,6 +191,23 @@ qsa_status qsa_sparse_attention_q8(const qsa_config* cfg, int32_t batch, const q
                                    const int32_t* sel, const int32_t* nsel, qsa_bf16* out, float* lse,
                                    void* ws, size_t ws_bytes, qsa_stream stream);
 
+/* qsa_decode_step on fp8 caches: the core K/V caches are k_codes/k_scales and
+ * v_codes/v_scales (layouts as for qsa_sparse_attention_q8; the appended
+ * token's rows are quantized as qsa_quantize_rows would), and the decode score
+ * stream reads pooled_codes [batch][cap/r][128] uint8 (16-byte aligned) with
+ * pooled_scales [batch][cap/r] fp32: I_b = scale_b * sum_h ReLU(<q_h, codes_b>)
+ * in fp32 (the query in f16, exact for its bf16 values inside the f16 range).
+ * A block the token completes is pooled into `pooled` (bf16, as in
+ * qsa_decode_step) and quantized from it into pooled_codes/pooled_scales. The
+ * attention is that of qsa_sparse_attention_q8. Other arguments, the workspace
+ * and the errors as for qsa_decode_step; head_dim must be 128. */
+qsa_status qsa_decode_step_q8(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,
+                              const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q, const qsa_bf16* idx_k,
+                              uint8_t* k_codes, float* k_scales, uint8_t* v_codes, float* v_scales,
+                              qsa_bf16* idx_k_cache, qsa_bf16* pooled, uint8_t* pooled_codes,
+                              float* pooled_scales, int64_t cap, const float* rms_w, qsa_bf16* out,
+                              int32_t* sel_out, int32_t* nsel_out, void* ws, size_t ws_bytes, qsa_stream stream);
+
 /* One decode step for every sequence s, at p = pos[s] (its current length):
  *   a8: append k, v (-> k_cache/v_cache row p) and idx_k (-> idx_k_cache row p);
  *   a3'..a7: the new token is query p: score blocks b < floor(p/r), select,

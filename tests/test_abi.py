@@ -86,3 +86,15 @@ def test_quantize_rows_validation_launches_nothing(qsa):
     assert lib.qsa_quantize_rows(None, 10, 128, p, p, None) == 1
     assert lib.qsa_quantize_rows(p, 10, 128, p, ctypes.c_void_p(4098), None) == 1  # scales misaligned
     assert lib.qsa_quantize_rows(p, 0, 128, p, p, None) == 0  # nothing to do
+
+
+def test_binding_argument_counts_match_the_header(qsa):
+    """Every ctypes signature of the binding has as many arguments as the
+    declaration in include/qsa.h."""
+    src = open(os.path.join(ROOT, "include", "qsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    decls = {m.group(1): m.group(2) for m in re.finditer(r"\b(qsa_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src)}
+    for name, args in qsa._SIGS.items():
+        assert name in decls, name
+        params = [p for p in decls[name].split(",") if p.strip() and p.strip() != "void"]
+        assert len(args) == len(params), (name, len(args), len(params))

@@ -619,3 +619,60 @@ def test_prefill_with_fp8_caches_matches_oracle(qsa, q_heads, kv_heads):
         ref, ref_lse = o.attention_q8(q_bits[i], k8, ks, v8, vs, toks)
         check_attention(g_out[i], ref, f"row {i}")
         assert np.abs(g_lse[i] - ref_lse).max() <= LSE_ATOL, i
+
+
+def test_decode_steps_with_fp8_caches_match_oracle(qsa):
+    """Decode on fp8 caches, step by step across block boundaries: the appended
+    K/V rows and each newly pooled block are quantized exactly as the oracle
+    does; the selection is the oracle's on the fp8 pooled keys (near-ties
+    aside); the output matches the oracle's fp8-cache attention."""
+    from gpu_util import SCORE_COND_ATOL, SCORE_RTOL
+
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    n0, S = 3001, 9
+    w = synth.Workload(name="t", n=n0, batch=2, decode_steps=S, prefill=False, K=512, q_heads=32, kv_heads=4,
+                       base_seed=0xF9)
+    B = w.batch
+    cfg = qsa.Config.of(w)
+    cap = n0 + S + 3
+    L = QSALayer(cfg, B, cap)
+    _fill_caches(w, L, n0)
+    L.compress(0, n0 // cfg.r)
+    L.quantize_kv(0, n0)
+    L.quantize_pooled(0, n0 // cfg.r)
+    full = {nm: dev_full(w, nm, cap, n0 + S) for nm in ("q", "k", "v", "idx_q", "idx_k")}
+    o = _oracle(w, cfg)
+    out = torch.empty(B, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(B, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(B, dtype=torch.int32, device="cuda")
+    for step in range(S):
+        p = n0 + step
+        pos = torch.full((B,), p, dtype=torch.int64, device="cuda")
+        args = [full[nm][:, p].contiguous() for nm in ("q", "k", "v", "idx_q", "idx_k")]
+        L.decode_step_q8(pos, *args, out, sel, nsel)
+        torch.cuda.synchronize()
+        assert qsa.qsa_workspace_status(L.workspace(qsa.OP_DECODE_STEP)) == 0
+        k8, v8, ks, vs = (t.cpu().numpy() for t in (L.k8, L.v8, L.ks, L.vs))
+        p8, ps = L.pooled8.cpu().numpy(), L.pscale.cpu().numpy()
+        pooled = bits(L.pooled)
+        g_out, g_sel, g_n = out.float().cpu().numpy(), sel.cpu().numpy(), nsel.cpu().numpy()
+        for s in range(B):
+            hs = {nm: w.host_full(nm, s, n0 + S) for nm in ("q", "k", "v", "idx_q")}
+            for src, c8, sc in ((hs["k"], k8, ks), (hs["v"], v8, vs)):  # appended rows
+                rc, rs = o.quant_rows(src[p].reshape(cfg.kv_heads, 128))
+                assert np.array_equal(rs, sc[s, p]) and np.array_equal(rc, c8[s, p]), (s, p)
+            if (p + 1) % cfg.r == 0:  # the block the token closed
+                b = p // cfg.r
+                rc, rs = o.quant_rows(pooled[s, b:b + 1])
+                assert np.array_equal(rs, ps[s, b:b + 1]) and np.array_equal(rc, p8[s, b:b + 1]), (s, b)
+            nvis = p // cfg.r
+            qrot = o.rotate_query(hs["idx_q"][p].reshape(4, 128), p)
+            ref = o.scores_q8(qrot, p8[s], ps[s], nvis)
+            kd = o.dequant(p8[s, :nvis], ps[s, :nvis])
+            tol = SCORE_RTOL * np.abs(ref.astype(np.float64)) + SCORE_COND_ATOL * (
+                np.abs(kd) @ np.abs(f32(qrot).astype(np.float64)).T).sum(axis=1)
+            check_selection(g_sel[s], g_n[s], ref, tol, o.k_blocks, f"s{s} p{p}")
+            toks = o.token_set(g_sel[s, : g_n[s]], p)
+            ref_out, _ = o.attention_q8(hs["q"][p], k8[s], ks[s], v8[s], vs[s], toks)
+            check_attention(g_out[s], ref_out.reshape(cfg.q_heads, 128), f"s{s} p{p}")
