@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
 
 constexpr int SEL_E = 8;                 // scores per thread per round of the scan
 constexpr int SEL_BITMAP_WORDS = 10240;  // ordered output by bitmap for up to 327680 blocks
+static_assert(SEL_BITMAP_WORDS % (4 * 512) == 0, "T threads x 4-word multiples cover the bitmap exactly");
 
 struct DecSelSmem {
     uint32_t hist[BINS];     // level-1, then level-2 histogram
@@ -433,8 +434,11 @@ __global__ void __launch_bounds__(T) decode_select_kernel(
     }
     const bool use_bm = nvis <= (int64_t)SEL_BITMAP_WORDS * 32;
     const int words = use_bm ? (int)((nvis + 31) / 32) : 0;
+    // Bitmap words per thread for the ordered output, a multiple of 4 (read as
+    // 16-byte vectors); every word a thread reads is cleared here.
+    const int per = (((words + T - 1) / T) + 3) & ~3;
     for (int b = tid; b < BINS; b += T) sm.hist[b] = 0u;
-    for (int w = tid; w < words; w += T) sm.u.bitmap[w] = 0u;
+    for (int w = tid; w < T * per; w += T) sm.u.bitmap[w] = 0u;
     if (tid == 0) {
         sm.n_l3 = 0;
         sm.n_win = n_win;
@@ -501,21 +505,29 @@ __global__ void __launch_bounds__(T) decode_select_kernel(
     }
     __syncthreads();
     if (use_bm) {
-        // Ordered compaction: thread t owns words [t per, (t + 1) per).
-        const int per = (words + T - 1) / T;
-        const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+        // Ordered compaction: thread t owns words [t per, (t + 1) per), read
+        // as 16-byte vectors.
+        const int w0 = tid * per;
         uint32_t n = 0;
-        for (int w = w0; w < w1; ++w) n += __popc(sm.u.bitmap[w]);
+        for (int w = w0; w < w0 + per; w += 4) {
+            const uint4 x = *reinterpret_cast<const uint4*>(&sm.u.bitmap[w]);
+            n += __popc(x.x) + __popc(x.y) + __popc(x.z) + __popc(x.w);
+        }
         uint32_t at;
         const uint32_t total = cta_prefix(sm, n, at);
         if (total != (uint32_t)kB && tid == 0) flag_status(status, 7 /* QSA_ERR_DEVICE_CHECK */);
-        for (int w = w0; w < w1; ++w) {
-            uint32_t m = sm.u.bitmap[w];
-            while (m) {
-                const int bit = __ffs(m) - 1;
-                m &= m - 1;
-                if (at < (uint32_t)kB) out[at] = w * 32 + bit;
-                ++at;
+        for (int w = w0; n && w < w0 + per; w += 4) {
+            const uint4 x = *reinterpret_cast<const uint4*>(&sm.u.bitmap[w]);
+            const uint32_t m4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t m = m4[j];
+                while (m) {
+                    const int bit = __ffs(m) - 1;
+                    m &= m - 1;
+                    if (at < (uint32_t)kB) out[at] = (w + j) * 32 + bit;
+                    ++at;
+                }
             }
         }
     } else {
