@@ -16,6 +16,11 @@
 // with one movmatrix transpose per 8x8 block. Logits, the online (running max) softmax and the
 // accumulation are fp32; probabilities are rounded to bf16 for the P.V
 // product. Invalid selections are skipped, never read.
+//
+// Variants: on fp8 caches (Q8) each chunk is gathered as E4M3 code rows with
+// their row scales and converted into f16 tiles before the same tile products
+// (in f16); the decode kernel runs one thread-block cluster per (sequence, kv
+// head) and merges its split states over distributed shared memory.
 #include <algorithm>
 
 #include "kernels.h"
@@ -62,10 +67,6 @@ struct WarpState {
     float o[NT][8][4];
     float m[NT][2], l[NT][2];
 };
-template <int NT>
-constexpr int park_floats() {
-    return NT * 36;  // o (32), m (2), l (2) per n8 tile
-}
 
 // 8x8 b16 matrix transpose in the mma fragment layout (lane l holds row l/4,
 // columns 2 (l % 4) and 2 (l % 4) + 1).
