@@ -82,6 +82,9 @@ def algorithmic(w, kv="bf16"):
             dec += nb * w.idx_dim * 2 + t * w.kv_heads * d * 2 * 2
         dec_tok += 1
     out["decode_bytes"] = dec * w.batch
+    out["decode_gather_bytes"] = sum(
+        (r * min(kB, (w.n + s) // r) + (w.n + s) % r + 1) * w.kv_heads * d * 2 * 2 for s in range(w.decode_steps)
+    ) * w.batch
     out["decode_tokens"] = dec_tok * w.batch
     out["prefill_tokens"] *= w.batch
     for k in ("compress_bytes", "index_flops", "attn_gather_bytes", "attn_flops", "quantize_bytes"):
@@ -197,13 +200,14 @@ def job_value(tokens_per_rank: float, ms_max: float, world: int) -> float:
 
 # ----------------------------------------------------------------------------- CUDA arm
 class Bench:
-    def __init__(self, w, device, stage="all", kv="bf16"):
+    def __init__(self, w, device, stage="all", kv="bf16", offload=0):
         import block_sparse_long_02_b200 as qsa
         from block_sparse_long_02_b200.layer import QSALayer
 
         self.qsa, self.w, self.dev = qsa, w, device
         self.stage = stage
         self.kv = kv
+        self.offload = offload  # hot-cache blocks per sequence (0: K/V caches in HBM)
         cfg = qsa.Config.of(w)
         self.cfg = cfg
         B, n, S = w.batch, w.n, w.decode_steps
@@ -267,6 +271,10 @@ class Bench:
             if cached:
                 L.quantize_kv(0, cached)
                 L.quantize_pooled(0, cached // w.r)
+        if offload:
+            if w.prefill:
+                raise SystemExit("--offload applies to the decode-only workloads")
+            L.offload_kv(offload)
         self.dec_graph, self.dec_graphs_1, self.graph_kernels = None, [], 0
         self.graph_launches = 0  # kernels launched by graph replays so far
         torch.cuda.synchronize()
@@ -279,10 +287,10 @@ class Bench:
             return
         qsa = self.qsa
         n0 = qsa.qsa_launch_count()
-        q8 = self.kv == "fp8"
-        self.dec_graph = self.L.capture_decode(self.dec, q8)
+        q8, off = self.kv == "fp8", bool(self.offload)
+        self.dec_graph = self.L.capture_decode(self.dec, q8, off)
         self.graph_kernels = qsa.qsa_launch_count() - n0
-        self.dec_graphs_1 = [self.L.capture_decode([d], q8) for d in self.dec]
+        self.dec_graphs_1 = [self.L.capture_decode([d], q8, off) for d in self.dec]
         torch.cuda.synchronize()
 
     def step(self, mark=None):
@@ -321,7 +329,8 @@ class Bench:
             self.dec_graph.replay()
             self.graph_launches += self.graph_kernels
         else:
-            dstep = L.decode_step_q8 if self.kv == "fp8" else L.decode_step
+            dstep = (L.decode_step_q8 if self.kv == "fp8" else
+                     L.decode_step_offload if self.offload else L.decode_step)
             for d in self.dec:
                 dstep(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
         if mark and self.dec:
@@ -375,7 +384,7 @@ class Bench:
 
 def run_cuda(args, w, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
-    b = Bench(w, dev, stage=args.stage, kv=args.kv)
+    b = Bench(w, dev, stage=args.stage, kv=args.kv, offload=args.offload)
     qsa = b.qsa
     for k in range(args.warmup):
         b.step()
@@ -447,6 +456,8 @@ def run_cuda(args, w, rank, world):
         evs = []
         for k, d in enumerate(b.dec):
             flush.fill_(len(evs) & 0xFF)
+            if b.offload:
+                b.L.hot_tags.fill_(-1)  # every selected block misses: read over the host link
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a0.record(stream)
             if b.dec_graphs_1:
@@ -463,6 +474,11 @@ def run_cuda(args, w, rank, world):
         stages["decode_cold"] = {"ms": round(cold, 4), "bound": "hbm", "achieved": round(ach, 2), "unit": "GB/s",
                                  "frac": round(ach / pk["hbm_gbs"], 4),
                                  "note": "each step after a 256 MB L2-evicting write"}
+        if b.offload:
+            host = alg["decode_gather_bytes"] / (cold * 1e-3) / 1e9
+            stages["decode_cold"]["note"] += ("; hot cache emptied before each step, so every selected block and the "
+                                              "tail are read from host memory")
+            stages["decode_cold"]["host_gbs"] = round(host, 2)
     ds = stages[dom]
     roofline = {"bound": ds["bound"], "achieved": ds["achieved"],
                 "peak": pk["hbm_gbs"] if ds["bound"] == "hbm" else pk["bf16_tflops_sustained"],
@@ -484,6 +500,8 @@ def run_cuda(args, w, rank, world):
                           f" gathered, q {w.batch * (w.n - w.q_begin) * w.q_heads * w.head_dim * 2 / 1e9:.2f} GB);"
                           " decode steps back to back"),
                    "decode_launch": "eager calls" if b.dec_graph is None else "CUDA graph replay of the steps",
+                   "kv_location": ("HBM" if not args.offload else
+                                   f"pinned host memory, {args.offload} hot blocks per sequence in HBM"),
                    "kv_cache": ("bf16" if args.kv == "bf16" else
                                 "fp8 E4M3 codes + one fp32 scale per row: core K/V, and pooled keys for decode")},
         "roofline": roofline, "stages": stages,
@@ -644,6 +662,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="decode steps as eager calls, not CUDA graph replays")
+    ap.add_argument("--offload", type=int, default=0, metavar="SLOTS",
+                    help="decode with the K/V caches in pinned host memory and SLOTS hot blocks per sequence in HBM")
     ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
                     help="core K/V cache format of the prefill attention (fp8: E4M3 codes, per-row scales)")
     ap.add_argument("--stage", choices=["all", "topk"], default="all",

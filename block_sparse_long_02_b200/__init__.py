@@ -27,7 +27,7 @@ OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
            "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection", "qsa_quantize_rows",
-           "qsa_sparse_attention_q8", "qsa_decode_step_q8"]
+           "qsa_sparse_attention_q8", "qsa_decode_step_q8", "qsa_decode_step_offload"]
 
 
 class QSAError(RuntimeError):
@@ -86,6 +86,8 @@ _SIGS = {
     "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
     "qsa_quantize_rows": [_vp, _i64, _i32, _vp, _vp, _vp],
     "qsa_decode_step_q8": [_CFG, _i32] + [_vp] * 14 + [_i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "qsa_decode_step_offload": [_CFG, _i32] + [_vp] * 11 + [_i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz,
+                                                           _vp],
     "qsa_sparse_attention_q8": [_CFG, _i32, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
                                 _sz, _vp],
     "qsa_decode_step_noalloc": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp,
@@ -128,6 +130,14 @@ def _ptr(t: Optional[torch.Tensor]):
         raise ValueError("tensors passed to libqsa must live on a CUDA device")
     if not t.is_contiguous():
         raise ValueError("tensors passed to libqsa must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host_ptr(t: torch.Tensor):
+    """Address of a pinned host tensor (the library checks that it is mapped
+    into the device address space)."""
+    if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+        raise ValueError("host caches must be contiguous pinned CPU tensors")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -204,6 +214,17 @@ def qsa_decode_step_q8(cfg: Config, batch: int, pos, q, k, v, idx_q, idx_k, k_co
                                    _ptr(idx_k_cache), _ptr(pooled), _ptr(pooled_codes), _ptr(pooled_scales), cap,
                                    _ptr(rms_w), _ptr(out), _ptr(sel_out), _ptr(nsel_out), _ptr(ws),
                                    0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def qsa_decode_step_offload(cfg: Config, batch: int, pos, q, k, v, idx_q, idx_k, host_k_cache, host_v_cache,
+                            hot_k, hot_v, hot_tags, hot_blocks: int, idx_k_cache, pooled, cap: int, rms_w, out,
+                            sel_out=None, nsel_out=None, ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().qsa_decode_step_offload(ctypes.byref(cfg.c()), batch, _ptr(pos), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(idx_q), _ptr(idx_k), _host_ptr(host_k_cache), _host_ptr(host_v_cache),
+                                        _ptr(hot_k),
+                                        _ptr(hot_v), _ptr(hot_tags), hot_blocks, _ptr(idx_k_cache), _ptr(pooled), cap,
+                                        _ptr(rms_w), _ptr(out), _ptr(sel_out), _ptr(nsel_out), _ptr(ws),
+                                        0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def qsa_decode_step(cfg: Config, batch: int, pos: torch.Tensor, q, k, v, idx_q, idx_k, k_cache, v_cache,

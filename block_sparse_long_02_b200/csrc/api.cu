@@ -352,7 +352,8 @@ qsa_status decode_step_impl(const qsa_config* cfg, int32_t batch, const int64_t*
                             const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q, const qsa_bf16* idx_k,
                             qsa_bf16* k_cache, qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled,
                             int64_t cap, const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
-                            void* ws, size_t ws_bytes, qsa_stream stream, const qsa::Q8Caches* q8) {
+                            void* ws, size_t ws_bytes, qsa_stream stream, const qsa::Q8Caches* q8,
+                            qsa::HotCache* hot = nullptr) {
     qsa::LayerDims L;
     TRY(make_dims(cfg, &L));
     REQUIRE_PTR(pos);
@@ -387,12 +388,32 @@ qsa_status decode_step_impl(const qsa_config* cfg, int32_t batch, const int64_t*
     sw.cand = reinterpret_cast<uint2*>(base + w.cand);
     cudaStream_t st = (cudaStream_t)stream;
     TRY(cuda_check(qsa::launch_decode_score(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
-                                            pooled, cap, rms_w, scores, sw, status, q8, st),
+                                            pooled, cap, rms_w, scores, sw, status, q8, hot, st),
                    "decode score"));
     TRY(cuda_check(qsa::launch_decode_select(L, batch, pos, cap, scores, sw, sel, nsel, status, st),
                    "decode select"));
-    return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel, nsel, out, q8, st),
-                      "decode attention");
+    if (!hot)
+        return cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel, nsel, out, q8,
+                                                       nullptr, st),
+                          "decode attention");
+    TRY(cuda_check(qsa::launch_decode_attention(L, batch, pos, q, k_cache, v_cache, cap, sel, nsel, out, nullptr, hot,
+                                                st),
+                   "decode attention"));
+    return cuda_check(qsa::launch_install_hot(L, batch, pos, cap, sel, nsel, k_cache, v_cache, hot->k, hot->v,
+                                              hot->tags, hot->blocks, st),
+                      "hot-cache install");
+}
+
+// The device address of pinned host memory that is mapped into the device's
+// address space, or NULL (then the caller returns an error: the library never
+// hands a kernel a host pointer it cannot read).
+void* mapped_host(void* p) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
 }
 }  // namespace
 
@@ -406,6 +427,30 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
                            void* ws, size_t ws_bytes, qsa_stream stream) {
     return decode_step_impl(cfg, batch, pos, q, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache, pooled, cap,
                             rms_w, out, sel_out, nsel_out, ws, ws_bytes, stream, nullptr);
+}
+
+qsa_status qsa_decode_step_offload(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,
+                                   const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q,
+                                   const qsa_bf16* idx_k, qsa_bf16* host_k_cache, qsa_bf16* host_v_cache,
+                                   qsa_bf16* hot_k, qsa_bf16* hot_v, int32_t* hot_tags, int64_t hot_blocks,
+                                   qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap, const float* rms_w,
+                                   qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out, void* ws, size_t ws_bytes,
+                                   qsa_stream stream) {
+    REQUIRE_PTR(host_k_cache);
+    REQUIRE_PTR(host_v_cache);
+    REQUIRE_PTR(hot_k);
+    REQUIRE_PTR(hot_v);
+    if (!hot_tags || ((uintptr_t)hot_tags & 3u)) return fail(QSA_ERR_INVALID_ARG, "hot_tags NULL or misaligned");
+    if (hot_blocks < 1 || hot_blocks >= INT32_MAX)
+        return fail(QSA_ERR_INVALID_ARG, "hot_blocks=%lld", (long long)hot_blocks);
+    void* hk = mapped_host(host_k_cache);
+    void* hv = mapped_host(host_v_cache);
+    if (!hk || !hv)
+        return fail(QSA_ERR_INVALID_ARG, "host K/V caches must be pinned host memory mapped into the device");
+    qsa::HotCache hot{reinterpret_cast<uint16_t*>(hot_k), reinterpret_cast<uint16_t*>(hot_v), hot_tags, hot_blocks};
+    return decode_step_impl(cfg, batch, pos, q, k, v, idx_q, idx_k, static_cast<qsa_bf16*>(hk),
+                            static_cast<qsa_bf16*>(hv), idx_k_cache, pooled, cap, rms_w, out, sel_out, nsel_out, ws,
+                            ws_bytes, stream, nullptr, &hot);
 }
 
 qsa_status qsa_decode_step_q8(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,

@@ -44,6 +44,11 @@ struct Work {
     const void* vc;
     const float* ks;       // fp8 caches: sequence base of the row scales [cap][kv_heads]
     const float* vs;
+    const uint16_t* hot_k; // host-offloaded caches: sequence base of the HBM hot blocks
+    const uint16_t* hot_v; //   [hot_blocks + 1][r][kv_heads][128] (the last one the tail slot)
+    const int32_t* tags;   //   and of their tags [hot_blocks + 1]
+    int32_t hot_blocks;
+    int32_t tail_hrow0;    //   first hot row of the tail slot when it holds the tail, else -1
     const int32_t* sel;    // selection row
     int64_t i;             // query position
     int64_t cur;           // its block, i / r
@@ -117,9 +122,14 @@ static_assert(Q8_TILE + STAGES * Q8_STAGE + 8 <= WARP_SMEM, "fp8 layout fits the
 // gathered as codes, then converted into the warp's f16 tile (values times
 // their row scale), the logits take the key rows' scales, and both products
 // run in f16 (qb then holds f16 fragments).
-template <int NT, bool Q8 = false>
+// HOT: the caches kc, vc are in host memory and the HBM hot cache holds some
+// blocks: hot_lane (lane l, for the warp's unit u0 + l) is the hot slot of that
+// selection entry's block, or -1 (read from host memory); entries past the
+// warp's first 32 units look their slot's tag up when issued, and the tail
+// comes from the tail slot when w.tail_hrow0 >= 0.
+template <int NT, bool Q8 = false, bool HOT = false>
 __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lane, const uint32_t (&qb)[NT][8][2],
-                                            int32_t sel_lane, WarpState<NT>& st) {
+                                            int32_t sel_lane, WarpState<NT>& st, int32_t hot_lane = -1) {
     uint16_t* ring = reinterpret_cast<uint16_t*>(wsm);
     uint32_t* vmask = reinterpret_cast<uint32_t*>(
         Q8 ? wsm + Q8_TILE + STAGES * Q8_STAGE : wsm + STAGES * STAGE_BYTES + STAGES * CT * 8);
@@ -149,15 +159,30 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
         const int pl = c * CT + (lane & (CT - 1));  // lanes >= CT mirror lanes < CT
         const int u = w.u0 + pl / w.r;
         const int32_t b_pre = __shfl_sync(0xffffffffu, sel_lane, (u - w.u0) & 31);
+        const int32_t hot_pre = HOT ? __shfl_sync(0xffffffffu, hot_lane, (u - w.u0) & 31) : -1;
         int32_t tk = -1;  // token (the cache capacity is below 2^31 tokens)
+        int32_t hrow = -1;  // HOT: the token's row in the hot cache, or -1
         if (pl < ntok_i) {
             const int e = pl % w.r;
             if (u == w.tail_unit) {
                 const int64_t tt = cur * w.r + e;
-                if (tt <= w.i) tk = (int32_t)tt;
+                if (tt <= w.i) {
+                    tk = (int32_t)tt;
+                    if (HOT && w.tail_hrow0 >= 0) hrow = w.tail_hrow0 + e;
+                }
             } else if (u < w.nsel) {
                 const int32_t b = u - w.u0 < 32 ? b_pre : w.sel[u];
-                if (b >= 0 && (int64_t)b < cur) tk = b * w.r + e;
+                if (b >= 0 && (int64_t)b < cur) {
+                    tk = b * w.r + e;
+                    if (HOT) {
+                        int32_t slot = hot_pre;
+                        if (u - w.u0 >= 32) {
+                            slot = b % w.hot_blocks;
+                            if (__ldcg(w.tags + slot) != b) slot = -1;
+                        }
+                        if (slot >= 0) hrow = slot * w.r + e;
+                    }
+                }
             }
         }
         const uint32_t valid = __ballot_sync(0xffffffffu, tk >= 0) & ((1u << CT) - 1u);
@@ -194,9 +219,20 @@ __device__ __forceinline__ void warp_attend(const Work& w, uint8_t* wsm, int lan
                 const int row = idx >> 4, ch = idx & 15;
                 const int32_t tkr = __shfl_sync(0xffffffffu, tk, row);
                 const bool ok = tkr >= 0;
-                const size_t off = (size_t)(ok ? tkr : 0) * row_stride + (size_t)w.g * kHeadDim + ch * 8;
-                cp_async16_zfill(kbase + swz256(row, ch), kc16 + off, ok);
-                cp_async16_zfill(vbase + swz256(row, ch), vc16 + off, ok);
+                const uint16_t* ksrc = kc16;
+                const uint16_t* vsrc = vc16;
+                int32_t src_row = ok ? tkr : 0;
+                if (HOT) {
+                    const int32_t hr = __shfl_sync(0xffffffffu, hrow, row);
+                    if (hr >= 0) {
+                        ksrc = w.hot_k;
+                        vsrc = w.hot_v;
+                        src_row = hr;
+                    }
+                }
+                const size_t off = (size_t)src_row * row_stride + (size_t)w.g * kHeadDim + ch * 8;
+                cp_async16_zfill(kbase + swz256(row, ch), ksrc + off, ok);
+                cp_async16_zfill(vbase + swz256(row, ch), vsrc + off, ok);
             }
         }
     };
@@ -511,14 +547,15 @@ __host__ __device__ constexpr int decode_recv_bytes(int G, int C) { return (G * 
 // outputs [c E / C, (c + 1) E / C) of the E = G x 128 and every CTA pushes its
 // merged slice for them into c's shared memory (remote stores, no remote
 // loads); after one cluster barrier each CTA finishes its slice locally.
-// Q8: fp8 K/V caches (codes kc, vc with row scales ks, vs).
-template <int NT, int DW, bool Q8>
+// Q8: fp8 K/V caches (codes kc, vc with row scales ks, vs). HOT: kc, vc are
+// host memory and hot holds an HBM cache of blocks (see HotCache).
+template <int NT, int DW, bool Q8, bool HOT = false>
 __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
     const uint16_t* __restrict__ q, const int64_t* __restrict__ pos,
     const void* __restrict__ kc, const void* __restrict__ vc, const float* __restrict__ ks,
     const float* __restrict__ vs, int64_t cap,
     const int32_t* __restrict__ sel, const int32_t* __restrict__ nsel, uint16_t* __restrict__ out,
-    int q_heads, int kv_heads, int r, int kB, float scale_log2) {
+    int q_heads, int kv_heads, int r, int kB, float scale_log2, HotCache hot) {
     extern __shared__ __align__(128) uint8_t smem[];
     cluster_arrive_relaxed();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -537,6 +574,12 @@ __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
               : (const void*)(static_cast<const uint16_t*>(vc) + seq_elems);
     w.ks = Q8 ? ks + (size_t)s * cap * kv_heads : nullptr;
     w.vs = Q8 ? vs + (size_t)s * cap * kv_heads : nullptr;
+    const size_t hot_seq = (size_t)s * (hot.blocks + 1) * r * kv_heads * kHeadDim;
+    w.hot_k = HOT ? hot.k + hot_seq : nullptr;
+    w.hot_v = HOT ? hot.v + hot_seq : nullptr;
+    w.tags = HOT ? hot.tags + (size_t)s * (hot.blocks + 1) : nullptr;
+    w.hot_blocks = (int32_t)hot.blocks;
+    w.tail_hrow0 = -1;
     w.sel = sel + (size_t)s * kB;
     w.tail_unit = kB;
     w.u0 = (int)((int64_t)units * split / S);
@@ -566,8 +609,16 @@ __global__ void __launch_bounds__(DW * 32) decode_attention_kernel(
     w.nsel = ns;
     w.i = p;
     if (p < 0 || p >= cap) w.u1 = w.u0;  // skipped sequence: zero output
+    int32_t hot_lane = -1;  // HOT: the hot slot holding this lane's selected block
+    if (HOT) {
+        if (sel_lane >= 0) {
+            const int32_t slot = sel_lane % w.hot_blocks;
+            if (__ldcg(w.tags + slot) == sel_lane) hot_lane = slot;
+        }
+        if (__ldcg(w.tags + w.hot_blocks) == (int32_t)w.cur) w.tail_hrow0 = w.hot_blocks * r;
+    }
 
-    warp_attend<NT, Q8>(w, wsm, lane, qb, sel_lane, st);
+    warp_attend<NT, Q8, HOT>(w, wsm, lane, qb, sel_lane, st, hot_lane);
 
     const int E = G * kHeadDim, per = E / C;
     store_state_hd<NT>(st, G, reinterpret_cast<float*>(wsm), lane);
@@ -712,11 +763,12 @@ DecodeShape decode_shape(const LayerDims& L, int batch, int G) {
     return {4, decode_cluster_for<NT, 4>(L, batch, G)};
 }
 
-template <int NT, int DW, bool Q8>
+template <int NT, int DW, bool Q8, bool HOT>
 cudaError_t launch_decode_attention_t(const LayerDims& L, int batch, int C, const int64_t* pos, const uint16_t* q,
                                       const void* kc, const void* vc, const float* ks, const float* vs, int64_t cap,
-                                      const int32_t* sel, const int32_t* nsel, uint16_t* out, cudaStream_t st) {
-    auto kern = decode_attention_kernel<NT, DW, Q8>;
+                                      const int32_t* sel, const int32_t* nsel, uint16_t* out, const HotCache& hot,
+                                      cudaStream_t st) {
+    auto kern = decode_attention_kernel<NT, DW, Q8, HOT>;
     const int G = L.q_heads / L.kv_heads;
     const int smem = DW * WARP_SMEM + decode_recv_bytes(G, C);
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -737,21 +789,20 @@ cudaError_t launch_decode_attention_t(const LayerDims& L, int batch, int C, cons
     cfg.numAttrs = 2;
     note_launch();
     return cudaLaunchKernelEx(&cfg, kern, q, pos, kc, vc, ks, vs, cap, sel, nsel, out, L.q_heads, L.kv_heads, L.r,
-                              L.kB, L.sm_scale * LOG2E);
+                              L.kB, L.sm_scale * LOG2E, hot);
 }
 
 template <int NT>
 cudaError_t launch_decode_attention_nt(const LayerDims& L, int batch, const DecodeShape& sh, const int64_t* pos,
                                        const uint16_t* q, const void* kc, const void* vc, const float* ks,
                                        const float* vs, bool q8, int64_t cap, const int32_t* sel, const int32_t* nsel,
-                                       uint16_t* out, cudaStream_t st) {
-    if (q8)
-        return sh.dw == 8
-                   ? launch_decode_attention_t<NT, 8, true>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st)
-                   : launch_decode_attention_t<NT, 4, true>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st);
-    return sh.dw == 8
-               ? launch_decode_attention_t<NT, 8, false>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st)
-               : launch_decode_attention_t<NT, 4, false>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, st);
+                                       uint16_t* out, const HotCache& hot, cudaStream_t st) {
+#define QSA_DA(DW_, Q8_, HOT_) \
+    launch_decode_attention_t<NT, DW_, Q8_, HOT_>(L, batch, sh.c, pos, q, kc, vc, ks, vs, cap, sel, nsel, out, hot, st)
+    if (hot.k) return sh.dw == 8 ? QSA_DA(8, false, true) : QSA_DA(4, false, true);
+    if (q8) return sh.dw == 8 ? QSA_DA(8, true, false) : QSA_DA(4, true, false);
+    return sh.dw == 8 ? QSA_DA(8, false, false) : QSA_DA(4, false, false);
+#undef QSA_DA
 }
 
 }  // namespace
@@ -759,7 +810,7 @@ cudaError_t launch_decode_attention_nt(const LayerDims& L, int batch, const Deco
 cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
                                     const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
-                                    uint16_t* out, const Q8Caches* q8, cudaStream_t st) {
+                                    uint16_t* out, const Q8Caches* q8, const HotCache* hot, cudaStream_t st) {
     if (batch <= 0) return cudaSuccess;
     const int G = L.q_heads / L.kv_heads;
     // The launch shape is chosen once per problem shape (and thread).
@@ -775,8 +826,12 @@ cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t
     const void* v = q8 ? (const void*)q8->v8 : (const void*)vc;
     const float* ks = q8 ? q8->ks : nullptr;
     const float* vs = q8 ? q8->vs : nullptr;
-    if (G > 8) return launch_decode_attention_nt<2>(L, batch, sh, pos, q, k, v, ks, vs, q8 != nullptr, cap, sel, nsel, out, st);
-    return launch_decode_attention_nt<1>(L, batch, sh, pos, q, k, v, ks, vs, q8 != nullptr, cap, sel, nsel, out, st);
+    const HotCache hc = hot ? *hot : HotCache{nullptr, nullptr, nullptr, 1};
+    if (G > 8)
+        return launch_decode_attention_nt<2>(L, batch, sh, pos, q, k, v, ks, vs, q8 != nullptr, cap, sel, nsel, out, hc,
+                                             st);
+    return launch_decode_attention_nt<1>(L, batch, sh, pos, q, k, v, ks, vs, q8 != nullptr, cap, sel, nsel, out, hc,
+                                         st);
 }
 
 }  // namespace qsa

@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     const uint16_t* __restrict__ idx_q, const uint16_t* __restrict__ idx_k, uint16_t* __restrict__ kc,
     uint16_t* __restrict__ vc, uint16_t* __restrict__ idx_k_cache, uint16_t* __restrict__ pooled,
     int64_t cap, const float* __restrict__ rms_w, int kv_heads, int r, int kB, double eps, RopeTable rt,
-    float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status, Q8Caches q8) {
+    float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status, Q8Caches q8,
+    HotCache hot) {
     __shared__ uint32_t hist[2048];
     __shared__ __align__(16) uint16_t qs[kIdxHeads * kIdxDim];
     __shared__ double2 cs[kIdxDim / 2];  // (sin, cos) of the query position's angles
@@ -130,6 +131,23 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
             for (int c = tid; c < row16; c += DS_THREADS) {
                 kd[c] = ks[c];
                 vd[c] = vs[c];
+            }
+            if (hot.k) {
+                // Host caches: the token also goes to row p % r of the tail slot,
+                // which holds the current block's tokens once its tag names it.
+                const size_t tail = (((size_t)s * (hot.blocks + 1) + hot.blocks) * r + p % r) * row16;
+                uint4* tk = reinterpret_cast<uint4*>(hot.k) + tail;
+                uint4* tv = reinterpret_cast<uint4*>(hot.v) + tail;
+                for (int c = tid; c < row16; c += DS_THREADS) {
+                    tk[c] = ks[c];
+                    tv[c] = vs[c];
+                }
+                if (tid == 0) {
+                    int32_t* tag = hot.tags + (size_t)s * (hot.blocks + 1) + hot.blocks;
+                    const int32_t cur = (int32_t)(p / r);
+                    // Rows before p are there when the tag already names the block.
+                    *tag = (p % r == 0 || *tag == cur) ? cur : -1;
+                }
             }
         }
         if (tid < kIdxDim / 8)
@@ -573,15 +591,15 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
                                 uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,
                                 int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
-                                int32_t* status, const Q8Caches* q8, cudaStream_t st) {
+                                int32_t* status, const Q8Caches* q8, const HotCache* hot, cudaStream_t st) {
     const dim3 grid((unsigned)decode_score_ctas(batch), (unsigned)batch);
     if (q8)
         return launch_pdl(decode_score_kernel<true>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,
                           idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist,
-                          status, *q8);
+                          status, *q8, HotCache{});
     return launch_pdl(decode_score_kernel<false>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,
                       idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist,
-                      status, Q8Caches{});
+                      status, Q8Caches{}, hot ? *hot : HotCache{});
 }
 
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,

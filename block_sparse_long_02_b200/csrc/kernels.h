@@ -94,11 +94,31 @@ cudaError_t launch_sparse_attention_q8(const LayerDims& L, int batch, const uint
                                        int64_t nq, const uint8_t* k8, const float* ks, const uint8_t* v8,
                                        const float* vs, int64_t cap, const int32_t* sel, const int32_t* nsel,
                                        uint16_t* out, float* lse, cudaStream_t st);
+// An HBM cache of K/V blocks in front of caches held in host memory:
+// k, v [batch][blocks + 1][r][kv_heads][128] bf16; tags [batch][blocks + 1] =
+// the block a slot holds, or -1; block b may only sit in slot b % blocks.
+// Slot `blocks` is the tail slot: when its tag is the current block, its rows
+// hold that block's tokens up to the step's position (each step appends its
+// token there as well, and claims the slot when its token opens a block).
+struct HotCache {
+    uint16_t* k;
+    uint16_t* v;
+    int32_t* tags;
+    int64_t blocks;
+};
 // q8 non-null: the K/V caches are q8's fp8 codes and scales (kc, vc unused).
+// hot non-null: kc, vc are (device-mapped) host memory with hot in front.
 cudaError_t launch_decode_attention(const LayerDims& L, int batch, const int64_t* pos,
                                     const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
                                     int64_t cap, const int32_t* sel, const int32_t* nsel,
-                                    uint16_t* out, const struct Q8Caches* q8, cudaStream_t st);
+                                    uint16_t* out, const struct Q8Caches* q8, const HotCache* hot,
+                                    cudaStream_t st);
+// offload.cu: after the attention, installs each selected block that missed
+// into its hot slot (the lowest selected block of a slot wins); blocks is the
+// number of slots before the tail slot.
+cudaError_t launch_install_hot(const LayerDims& L, int batch, const int64_t* pos, int64_t cap, const int32_t* sel,
+                               const int32_t* nsel, const uint16_t* host_k, const uint16_t* host_v, uint16_t* hot_k,
+                               uint16_t* hot_v, int32_t* tags, int64_t blocks, cudaStream_t st);
 
 // quant.cu: FP8 E4M3 rows with one fp32 scale per row (dim 64, 128 or 256).
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t rows, int dim, uint8_t* codes, float* scales,
@@ -133,7 +153,7 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
                                 uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,
                                 int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
-                                int32_t* status, const Q8Caches* q8, cudaStream_t st);
+                                int32_t* status, const Q8Caches* q8, const HotCache* hot, cudaStream_t st);
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
                                  const float* scores, DecodeSelWs sw, int32_t* sel, int32_t* nsel,
                                  int32_t* status, cudaStream_t st);

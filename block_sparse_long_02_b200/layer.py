@@ -17,8 +17,8 @@ from typing import Optional
 
 import torch
 
-from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step, qsa_decode_step_q8,
-               qsa_quantize_rows,
+from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step,
+               qsa_decode_step_offload, qsa_decode_step_q8, qsa_quantize_rows,
                qsa_sparse_attention, qsa_sparse_attention_q8, qsa_topk_blocks, qsa_workspace_size)
 
 
@@ -105,6 +105,30 @@ class QSALayer:
                            self.idx_k_cache, self.pooled, self.pooled8, self.pscale, self.cap, self.rms_w, out,
                            sel_out, nsel_out, ws, stream)
 
+    # ------------------------------------------------ host-offloaded K/V caches
+    def offload_kv(self, hot_blocks: int) -> None:
+        """Moves the core K/V caches to pinned host memory (copying their
+        contents) and puts an HBM cache of hot_blocks blocks per sequence
+        (plus the tail slot) in front of them, initially empty;
+        decode_step_offload uses them."""
+        self.host_k = torch.empty(self.k_cache.shape, dtype=self.k_cache.dtype, pin_memory=True)
+        self.host_v = torch.empty_like(self.host_k, pin_memory=True)
+        self.host_k.copy_(self.k_cache)
+        self.host_v.copy_(self.v_cache)
+        c = self.cfg
+        self.hot_blocks = hot_blocks
+        self.hot_k = torch.zeros(self.batch, hot_blocks + 1, c.r, c.kv_heads, c.head_dim, dtype=torch.bfloat16,
+                                 device=self.device)
+        self.hot_v = torch.zeros_like(self.hot_k)
+        self.hot_tags = torch.full((self.batch, hot_blocks + 1), -1, dtype=torch.int32, device=self.device)
+
+    def decode_step_offload(self, pos: torch.Tensor, q, k, v, idx_q, idx_k, out, sel_out=None, nsel_out=None,
+                            stream=None) -> None:
+        ws = self.workspace(OP_DECODE_STEP)
+        qsa_decode_step_offload(self.cfg, self.batch, pos, q, k, v, idx_q, idx_k, self.host_k, self.host_v,
+                                self.hot_k, self.hot_v, self.hot_tags, self.hot_blocks, self.idx_k_cache, self.pooled,
+                                self.cap, self.rms_w, out, sel_out, nsel_out, ws, stream)
+
     def prefill_q8(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin: int, nq: int, out: torch.Tensor,
                    sel: torch.Tensor, nsel: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None,
                    mark=None) -> None:
@@ -131,7 +155,7 @@ class QSALayer:
                         self.idx_k_cache, self.pooled, self.cap, self.rms_w, out, sel_out, nsel_out, ws,
                         stream)
 
-    def capture_decode(self, steps, q8: bool = False) -> "torch.cuda.CUDAGraph":
+    def capture_decode(self, steps, q8: bool = False, offload: bool = False) -> "torch.cuda.CUDAGraph":
         """Captures the decode steps `steps` (a list of dicts with the
         decode_step arguments pos, q, k, v, idx_q, idx_k, out) into one CUDA
         graph, run by `graph.replay()`: one launch for the whole sequence of
@@ -144,7 +168,7 @@ class QSALayer:
         side.wait_stream(torch.cuda.current_stream(self.device))
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
-            step = self.decode_step_q8 if q8 else self.decode_step
+            step = self.decode_step_q8 if q8 else (self.decode_step_offload if offload else self.decode_step)
             for d in steps:
                 step(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
         torch.cuda.current_stream(self.device).wait_stream(side)

@@ -208,6 +208,36 @@ qsa_status qsa_decode_step_q8(const qsa_config* cfg, int32_t batch, const int64_
                               float* pooled_scales, int64_t cap, const float* rms_w, qsa_bf16* out,
                               int32_t* sel_out, int32_t* nsel_out, void* ws, size_t ws_bytes, qsa_stream stream);
 
+/* qsa_decode_step with the core K/V caches in host memory. A step reads only
+ * the selected blocks' tokens and the tail (concept page, (B)), so the cache
+ * can outgrow HBM when each step fetches just those blocks.
+ * host_k_cache, host_v_cache: [batch][cap][kv_heads][head_dim] bf16 in pinned
+ *   host memory mapped into the device address space (cudaHostAlloc or a
+ *   torch pinned tensor); anything else returns QSA_ERR_INVALID_ARG. The
+ *   step appends the new token's K/V there and reads the tail and the blocks
+ *   missing from the hot cache from there (over the host link).
+ * hot_k, hot_v: [batch][hot_blocks + 1][r][kv_heads][head_dim] bf16 (HBM),
+ *   an HBM cache of blocks; hot_tags [batch][hot_blocks + 1] int32: the block
+ *   each slot holds, or -1 (initialise to -1, and again whenever the host
+ *   caches change other than by these steps). Block b may only sit in slot
+ *   b % hot_blocks; 1 <= hot_blocks < INT32_MAX, else QSA_ERR_INVALID_ARG.
+ *   After the attention, every selected block that missed is installed (of
+ *   several selected blocks sharing a slot, the lowest). Slot hot_blocks is
+ *   the tail slot: the step writes its token to row p % r there as well and
+ *   tags the slot with block p / r when p opens that block or the tag already
+ *   names it (else -1); the tail is read from there when the tag names the
+ *   current block, from host memory otherwise.
+ * The outputs equal qsa_decode_step's on the same caches bit for bit (the
+ * same arithmetic on the same values). Other arguments and the workspace as
+ * for qsa_decode_step. */
+qsa_status qsa_decode_step_offload(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,
+                                   const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q,
+                                   const qsa_bf16* idx_k, qsa_bf16* host_k_cache, qsa_bf16* host_v_cache,
+                                   qsa_bf16* hot_k, qsa_bf16* hot_v, int32_t* hot_tags, int64_t hot_blocks,
+                                   qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap, const float* rms_w,
+                                   qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out, void* ws, size_t ws_bytes,
+                                   qsa_stream stream);
+
 /* One decode step for every sequence s, at p = pos[s] (its current length):
  *   a8: append k, v (-> k_cache/v_cache row p) and idx_k (-> idx_k_cache row p);
  *   a3'..a7: the new token is query p: score blocks b < floor(p/r), select,

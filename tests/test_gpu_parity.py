@@ -676,3 +676,85 @@ def test_decode_steps_with_fp8_caches_match_oracle(qsa):
             toks = o.token_set(g_sel[s, : g_n[s]], p)
             ref_out, _ = o.attention_q8(hs["q"][p], k8[s], ks[s], v8[s], vs[s], toks)
             check_attention(g_out[s], ref_out.reshape(cfg.q_heads, 128), f"s{s} p{p}")
+
+
+# ----------------------------------------------------------------------------- host-offloaded K/V
+@pytest.mark.parametrize("n0,S,H,batch", [(9002, 8, 97, 2), (4097, 6, 61, 24)])
+def test_decode_offload_matches_hbm_decode_bit_for_bit(qsa, n0, S, H, batch):
+    """K/V caches in pinned host memory with a small direct-mapped HBM hot
+    cache (a prime number of slots, so selected blocks collide): every step's
+    output and selection equal the all-HBM decode's bit for bit; the appended
+    rows reach host memory; every tagged hot slot holds a copy of its block.
+    The same query for every step makes later steps hit blocks installed by
+    earlier ones. The larger batch runs fewer warps per sequence, so a warp
+    holds more than 32 selection entries (their tags are looked up when
+    their chunks are issued)."""
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    # n0 inside a block: the first steps read the tail from host memory
+    w = synth.Workload(name="t", n=n0, batch=batch, decode_steps=S, prefill=False, K=2048, q_heads=32, kv_heads=4,
+                       base_seed=0xFA)
+    B = w.batch
+    cfg = qsa.Config.of(w)
+    cap = -(-(n0 + S + 8) // cfg.r) * cfg.r  # a multiple of r
+    full = {nm: dev_full(w, nm, cap, n0 + S) for nm in ("q", "k", "v", "idx_q", "idx_k")}
+
+    def make():
+        L = QSALayer(cfg, B, cap)
+        _fill_caches(w, L, n0)
+        L.compress(0, n0 // cfg.r)
+        return L
+
+    La, Lb = make(), make()
+    Lb.offload_kv(H)
+    hits_seen = False
+    for step in range(S):
+        p = n0 + step
+        pos = torch.full((B,), p, dtype=torch.int64, device="cuda")
+        q = full["q"][:, n0].contiguous()          # the same query every step
+        iq = full["idx_q"][:, n0].contiguous()
+        k, v, ik = (full[nm][:, p].contiguous() for nm in ("k", "v", "idx_k"))
+        outs, sels = [], []
+        for L, fn in ((La, La.decode_step), (Lb, Lb.decode_step_offload)):
+            out = torch.empty(B, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
+            sel = torch.empty(B, cfg.k_blocks, dtype=torch.int32, device="cuda")
+            nsel = torch.empty(B, dtype=torch.int32, device="cuda")
+            tags_before = Lb.hot_tags.clone()
+            fn(pos, q, k, v, iq, ik, out, sel, nsel)
+            torch.cuda.synchronize()
+            outs.append(out)
+            sels.append(sel)
+        assert torch.equal(outs[0], outs[1]), step
+        assert torch.equal(sels[0], sels[1]), step
+        # blocks this step found in the hot cache
+        sb = sels[1].long()
+        slot = sb.clamp(min=0) % H
+        hit = (tags_before.gather(1, slot) == sels[1]) & (sels[1] >= 0)
+        hits_seen = hits_seen or bool(hit.any())
+        assert qsa.qsa_workspace_status(Lb.workspace(qsa.OP_DECODE_STEP)) == 0
+    assert hits_seen
+    assert torch.equal(Lb.host_k.cuda(), La.k_cache) and torch.equal(Lb.host_v.cuda(), La.v_cache)
+    tags = Lb.hot_tags.cpu().numpy()
+    hk, hv = Lb.hot_k.cpu(), Lb.hot_v.cpu()
+    ck, cv = Lb.host_k.view(B, cap // cfg.r, cfg.r, cfg.kv_heads, 128), Lb.host_v.view(B, cap // cfg.r, cfg.r,
+                                                                                       cfg.kv_heads, 128)
+    n_tagged = 0
+    for s in range(B):
+        for sl in range(H):
+            b = int(tags[s, sl])
+            if b < 0:
+                continue
+            n_tagged += 1
+            assert b % H == sl
+            assert torch.equal(hk[s, sl], ck[s, b]) and torch.equal(hv[s, sl], cv[s, b]), (s, sl, b)
+        # the tail slot: the last step's block, rows up to its position (the
+        # steps ran from n0, so they opened that block when n0 + S - 1 crossed
+        # a block boundary after n0)
+        p_last = n0 + S - 1
+        cur = p_last // cfg.r
+        expect = cur if cur * cfg.r >= n0 else -1
+        assert int(tags[s, H]) == expect, (s, int(tags[s, H]), expect)
+        if expect >= 0:
+            e = p_last % cfg.r + 1
+            assert torch.equal(hk[s, H, :e], ck[s, cur, :e]) and torch.equal(hv[s, H, :e], cv[s, cur, :e])
+    assert n_tagged > 0
