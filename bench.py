@@ -164,22 +164,48 @@ class ClockSampler:
                 "power_w_max": max(float(f[4]) for f in rows if f[4].replace(".", "").isdigit())}
 
 
+def host_copy_gbs(dev, stream) -> float:
+    """Pinned host -> HBM copy rate (256 MB copies), the host link's reference."""
+    hb = torch.empty(256 << 20, dtype=torch.uint8, pin_memory=True)
+    db = torch.empty(hb.shape, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            db.copy_(hb, non_blocking=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            db.copy_(hb, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return 5 * hb.numel() / (e0.elapsed_time(e1) * 1e-3) / 1e9
+
+
+# The sources that define each stage's kernels (their code and launch shape).
+STAGE_SOURCES = {
+    "attention": ("attention.cu", "common.cuh"),
+    "topk": ("indexer_tc.cu", "topk.cu", "select.cuh", "common.cuh"),
+}
+
+
+def stage_source_sha1(stage: str) -> str:
+    src = os.path.join(ROOT, "block_sparse_long_02_b200", "csrc")
+    h = hashlib.sha1()
+    for name in STAGE_SOURCES[stage]:
+        h.update(open(os.path.join(src, name), "rb").read())
+    return h.hexdigest()[:12]
+
+
 def traffic_for(workload: str, stage: str):
     """DRAM bytes per launch of a stage of a workload from the committed ncu
     summary, or None when there is none or it was taken on a different version
-    of the kernel source."""
+    of the stage's kernel sources."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or stage not in STAGE_SOURCES:
         return None
     for ln in open(p):
         f = ln.split("#")[0].split()
         if len(f) == 4 and f[0] == workload and f[1] == stage:
-            f = f[1:]
-            src = os.path.join(ROOT, "block_sparse_long_02_b200", "csrc")
-            h = hashlib.sha1()
-            for name in sorted(os.listdir(src)):
-                h.update(open(os.path.join(src, name), "rb").read())
-            return float(f[1]) if h.hexdigest()[:12] == f[2] else None
+            return float(f[2]) if stage_source_sha1(stage) == f[3] else None
     return None
 
 
@@ -477,8 +503,10 @@ def run_cuda(args, w, rank, world):
         if b.offload:
             host = alg["decode_gather_bytes"] / (cold * 1e-3) / 1e9
             stages["decode_cold"]["note"] += ("; hot cache emptied before each step, so every selected block and the "
-                                              "tail are read from host memory")
+                                              "tail are read from host memory by the attention (host_gbs counts "
+                                              "these bytes), and the install kernel reads the blocks once more")
             stages["decode_cold"]["host_gbs"] = round(host, 2)
+            stages["decode_cold"]["host_copy_gbs"] = round(host_copy_gbs(dev, stream), 2)
     ds = stages[dom]
     roofline = {"bound": ds["bound"], "achieved": ds["achieved"],
                 "peak": pk["hbm_gbs"] if ds["bound"] == "hbm" else pk["bf16_tflops_sustained"],

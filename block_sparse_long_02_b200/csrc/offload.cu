@@ -2,7 +2,9 @@
 // selected blocks and the tail of each sequence ("QSA (Qwen Sparse Attention)"
 // concept page, (B): attention restricted to the selected blocks' tokens), so
 // the core K/V caches can live in host memory (pinned, mapped into the device
-// address space) with an HBM cache of blocks in front of them. The decode
+// address space) with an HBM cache of blocks in front of them, as the
+// community KV-offloading port on the "QSA" knowledge page (kongchang) does:
+// history in host memory, hot data and the indexer's caches on the GPU. The decode
 // attention reads a block from its hot slot when the slot's tag names it and
 // from host memory otherwise; this kernel then installs the step's missed
 // blocks for the steps that follow.

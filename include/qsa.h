@@ -210,7 +210,9 @@ qsa_status qsa_decode_step_q8(const qsa_config* cfg, int32_t batch, const int64_
 
 /* qsa_decode_step with the core K/V caches in host memory. A step reads only
  * the selected blocks' tokens and the tail (concept page, (B)), so the cache
- * can outgrow HBM when each step fetches just those blocks.
+ * can outgrow HBM when each step fetches just those blocks (the KV-offloading
+ * port on the "QSA" knowledge page: history in host memory, hot data and the
+ * indexer's caches on the GPU).
  * host_k_cache, host_v_cache: [batch][cap][kv_heads][head_dim] bf16 in pinned
  *   host memory mapped into the device address space (cudaHostAlloc or a
  *   torch pinned tensor); anything else returns QSA_ERR_INVALID_ARG. The
