@@ -6,8 +6,10 @@ slow, single-threaded statement of the layer (pool -> RMSNorm -> partial RoPE ->
 ReLU-sum indexer score -> top-k_B blocks -> expand + tail -> attention), written
 from the "QSA (Qwen Sparse Attention)" concept page, section "Key math / How it
 works", and the "Qwen Sparse Attention" gallery page, section "How block
-selection works". Every function is pinned by ``tests/test_oracle_pins.py``;
-none is "parity unpinned".
+selection works"; plus the training pieces of the concept page's "Native
+trainability" section (the gradient of the sparse attention, the stage-1
+block-max-pooled dense target and its KL loss). Every function is pinned by
+``tests/test_oracle_pins.py``; none is "parity unpinned".
 
 Arrays are numpy: bf16 values travel as their uint16 bit patterns.
 """
@@ -89,6 +91,12 @@ class Oracle:
         L.qsa_oracle_quant_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int, vp, vp]
         L.qsa_oracle_attention_q8.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp]
         L.qsa_oracle_scores_q8.argtypes = [vp, vp, vp, vp, ctypes.c_int64, vp]
+        L.qsa_oracle_attention_f64.argtypes = [vp, vp, vp, vp, ctypes.c_int64, vp, vp]
+        L.qsa_oracle_attention_backward_f64.argtypes = [vp, vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp]
+        L.qsa_oracle_attention_backward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp]
+        L.qsa_oracle_distill_target.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
+        L.qsa_oracle_distill_kl.restype = ctypes.c_double
+        L.qsa_oracle_distill_kl.argtypes = [vp, vp, ctypes.c_int64, vp]
 
     @classmethod
     def for_workload(cls, w, **kw) -> "Oracle":
@@ -243,3 +251,61 @@ class Oracle:
         out = np.empty(n_vis, dtype=np.float32)
         self.lib.qsa_oracle_scores_q8(self._c, _p(qrot), _p(pc), _p(ps), n_vis, _p(out))
         return out
+
+    # ------------------------------------------------------------ training (f3)
+    def attention_f64(self, q, kt, vt):
+        """Sparse attention on fp64 operands: q [q_heads][d], kt, vt [ntok][kv_heads][d]
+        (the listed tokens' rows in order) -> (out [q_heads][d], lse [q_heads])."""
+        c = self.cfg
+        q, kt, vt = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, kt, vt))
+        ntok = kt.size // (c.kv_heads * c.head_dim)
+        out = np.empty((c.q_heads, c.head_dim))
+        lse = np.empty(c.q_heads)
+        self.lib.qsa_oracle_attention_f64(self._c, _p(q), _p(kt), _p(vt), ntok, _p(out), _p(lse))
+        return out, lse
+
+    def attention_backward_f64(self, q, kt, vt, dout):
+        """Gradient of attention_f64 for the upstream gradient dout [q_heads][d]:
+        (dq [q_heads][d], dk [ntok][kv_heads][d], dv [ntok][kv_heads][d])."""
+        c = self.cfg
+        q, kt, vt, dout = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, kt, vt, dout))
+        ntok = kt.size // (c.kv_heads * c.head_dim)
+        dq = np.empty((c.q_heads, c.head_dim))
+        dk = np.empty((ntok, c.kv_heads, c.head_dim))
+        dv = np.empty((ntok, c.kv_heads, c.head_dim))
+        self.lib.qsa_oracle_attention_backward_f64(self._c, _p(q), _p(kt), _p(vt), ntok, _p(dout), _p(dq),
+                                                   _p(dk), _p(dv))
+        return dq, dk, dv
+
+    def attention_backward(self, q, kc, vc, tokens, dout):
+        """The gradient on bf16 operands (as ``attention`` takes them); dk, dv hold
+        one row per listed token."""
+        c = self.cfg
+        q, kc, vc, dout = _u16(q), _u16(kc), _u16(vc), _u16(dout)
+        tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+        dq = np.empty((c.q_heads, c.head_dim))
+        dk = np.empty((tokens.size, c.kv_heads, c.head_dim))
+        dv = np.empty((tokens.size, c.kv_heads, c.head_dim))
+        self.lib.qsa_oracle_attention_backward(self._c, _p(q), _p(kc), _p(vc), _p(tokens), tokens.size,
+                                               _p(dout), _p(dq), _p(dk), _p(dv))
+        return dq, dk, dv
+
+    def distill_target(self, i: int, q, kc) -> np.ndarray:
+        """Stage-1 target of query i over its floor(i/r) visible blocks (fp64)."""
+        c = self.cfg
+        n_vis = i // c.r
+        q, kc = _u16(q), _u16(kc)
+        assert kc.size >= (i + 1) * c.kv_heads * c.head_dim
+        # Padded with a sentinel: writing past the visible blocks is reported.
+        t = np.full(n_vis + c.r + 1, -7.0)
+        self.lib.qsa_oracle_distill_target(self._c, i, _p(q), _p(kc), _p(t))
+        assert (t[n_vis:] == -7.0).all(), "target written beyond floor(i/r)"
+        return t[:n_vis].copy()
+
+    def distill_kl(self, t, scores):
+        """(KL(t || softmax(scores)), d KL / d scores) over the given blocks."""
+        t = np.ascontiguousarray(t, dtype=np.float64)
+        s = np.ascontiguousarray(scores, dtype=np.float32)
+        ds = np.empty(t.size)
+        kl = self.lib.qsa_oracle_distill_kl(_p(t), _p(s), t.size, _p(ds))
+        return float(kl), ds

@@ -8,7 +8,8 @@
  *
  * Sources (page title, section):
  *   [P1] "QSA (Qwen Sparse Attention)" concept page, "Key math / How it works":
- *        (A) compressed lightweight indexer, (B) sparse core attention, "Config".
+ *        (A) compressed lightweight indexer, (B) sparse core attention, "Config";
+ *        "Native trainability via 2-stage continued pretraining" (training section).
  *   [P2] "Qwen Sparse Attention" (LLM architecture gallery), "How block selection
  *        works" (prose and pseudo-code) and the selection-unit / budget table.
  *
@@ -426,4 +427,188 @@ void qsa_oracle_scores_q8(const qsa_oracle_cfg* c, const uint16_t* qrot, const u
         }
         scores[b] = (float)sum;
     }
+}
+
+/* ============================================================ training (f3) */
+/* [P1] "Native trainability via 2-stage continued pretraining": stage 1 trains
+ * the indexer scores to match a block-max-pooled version of the dense teacher
+ * attention distribution through a KL loss; stage 2 trains the model and the
+ * indexer together under the sparse selection, which needs the gradient of the
+ * sparse core attention. Readings (the page names the pieces, not their
+ * arithmetic):
+ *   - the teacher distribution of query i is the dense causal attention
+ *     probability of every token j <= i, averaged over the core heads;
+ *   - block-max-pooling keeps, for each block the indexer scores (b < floor(i/r)),
+ *     the largest probability among its r tokens; the kept values are then
+ *     normalised to sum to 1 so that they form a distribution;
+ *   - the loss of query i is KL(target || softmax of the indexer scores over
+ *     the same blocks).                                                       */
+
+/* Sparse attention of one query on fp64 operands: q [q_heads][d]; kt, vt
+ * [ntok][kv_heads][d] are the rows of the listed tokens in list order. The
+ * same arithmetic as qsa_oracle_attention (which widens bf16 exactly). */
+void qsa_oracle_attention_f64(const qsa_oracle_cfg* c, const double* q, const double* kt, const double* vt,
+                              int64_t ntok, double* out, double* lse) {
+    const int d = c->head_dim, hkv = c->kv_heads, g = c->q_heads / c->kv_heads;
+    const double scale = c->sm_scale > 0.0 ? c->sm_scale : 1.0 / sqrt((double)d);
+    double* z = (double*)malloc(sizeof(double) * (size_t)(ntok > 0 ? ntok : 1));
+    for (int h = 0; h < c->q_heads; ++h) {
+        const int kvh = h / g;
+        double mx = -INFINITY;
+        for (int64_t t = 0; t < ntok; ++t) {
+            double dot = 0.0;
+            for (int j = 0; j < d; ++j) dot += q[(size_t)h * d + j] * kt[((size_t)t * hkv + kvh) * d + j];
+            z[t] = dot * scale;
+            if (z[t] > mx) mx = z[t];
+        }
+        double den = 0.0;
+        for (int j = 0; j < d; ++j) out[(size_t)h * d + j] = 0.0;
+        for (int64_t t = 0; t < ntok; ++t) {
+            const double e = exp(z[t] - mx);
+            den += e;
+            for (int j = 0; j < d; ++j) out[(size_t)h * d + j] += e * vt[((size_t)t * hkv + kvh) * d + j];
+        }
+        for (int j = 0; j < d; ++j) out[(size_t)h * d + j] /= den;
+        if (lse) lse[h] = mx + log(den);
+    }
+    free(z);
+}
+
+/* Gradient of that attention for the upstream gradient dout [q_heads][d], i.e.
+ * of L = sum_h <dout_h, out_h>, from out_h = sum_t p_ht v_t, p_ht = softmax over
+ * t of z_ht, z_ht = scale <q_h, k_t>:
+ *   dL/dv_t   = sum over the heads h of v_t's group of p_ht dout_h;
+ *   dL/dz_ht  = p_ht (<dout_h, v_t> - <dout_h, out_h>)   (softmax Jacobian);
+ *   dL/dq_h   = scale sum_t dL/dz_ht k_t;
+ *   dL/dk_t   = scale sum over the group's heads of dL/dz_ht q_h.
+ * dq: [q_heads][d]; dk, dv: [ntok][kv_heads][d], one row per listed token (a
+ * token listed twice gets two rows; the caller adds rows of the same token). */
+void qsa_oracle_attention_backward_f64(const qsa_oracle_cfg* c, const double* q, const double* kt,
+                                       const double* vt, int64_t ntok, const double* dout, double* dq,
+                                       double* dk, double* dv) {
+    const int d = c->head_dim, hkv = c->kv_heads, g = c->q_heads / c->kv_heads;
+    const double scale = c->sm_scale > 0.0 ? c->sm_scale : 1.0 / sqrt((double)d);
+    const size_t n_out = (size_t)c->q_heads * d;
+    double* out = (double*)malloc(sizeof(double) * n_out);
+    double* lse = (double*)malloc(sizeof(double) * (size_t)c->q_heads);
+    qsa_oracle_attention_f64(c, q, kt, vt, ntok, out, lse);
+    memset(dq, 0, sizeof(double) * n_out);
+    memset(dk, 0, sizeof(double) * (size_t)(ntok > 0 ? ntok : 0) * hkv * d);
+    memset(dv, 0, sizeof(double) * (size_t)(ntok > 0 ? ntok : 0) * hkv * d);
+    for (int h = 0; h < c->q_heads; ++h) {
+        const int kvh = h / g;
+        const double* qh = q + (size_t)h * d;
+        const double* gh = dout + (size_t)h * d;
+        double delta = 0.0; /* <dout_h, out_h> */
+        for (int j = 0; j < d; ++j) delta += gh[j] * out[(size_t)h * d + j];
+        for (int64_t t = 0; t < ntok; ++t) {
+            const double* kr = kt + ((size_t)t * hkv + kvh) * d;
+            const double* vr = vt + ((size_t)t * hkv + kvh) * d;
+            double qk = 0.0, gv = 0.0;
+            for (int j = 0; j < d; ++j) {
+                qk += qh[j] * kr[j];
+                gv += gh[j] * vr[j];
+            }
+            const double p = exp(qk * scale - lse[h]);
+            const double dz = p * (gv - delta);
+            double* dkr = dk + ((size_t)t * hkv + kvh) * d;
+            double* dvr = dv + ((size_t)t * hkv + kvh) * d;
+            for (int j = 0; j < d; ++j) {
+                dvr[j] += p * gh[j];
+                dq[(size_t)h * d + j] += scale * dz * kr[j];
+                dkr[j] += scale * dz * qh[j];
+            }
+        }
+    }
+    free(out);
+    free(lse);
+}
+
+/* The same gradient on the layer's bf16 operands: q, dout [q_heads][d]; kc, vc
+ * [>= max token + 1][kv_heads][d]; tokens as for qsa_oracle_attention. */
+void qsa_oracle_attention_backward(const qsa_oracle_cfg* c, const uint16_t* q, const uint16_t* kc,
+                                   const uint16_t* vc, const int64_t* tokens, int64_t ntok, const uint16_t* dout,
+                                   double* dq, double* dk, double* dv) {
+    const int d = c->head_dim, hkv = c->kv_heads;
+    const size_t row = (size_t)hkv * d, nq = (size_t)c->q_heads * d;
+    double* qd = (double*)malloc(sizeof(double) * nq);
+    double* gd = (double*)malloc(sizeof(double) * nq);
+    double* kt = (double*)malloc(sizeof(double) * (size_t)(ntok > 0 ? ntok : 1) * row);
+    double* vt = (double*)malloc(sizeof(double) * (size_t)(ntok > 0 ? ntok : 1) * row);
+    for (size_t j = 0; j < nq; ++j) {
+        qd[j] = bf(q[j]);
+        gd[j] = bf(dout[j]);
+    }
+    for (int64_t t = 0; t < ntok; ++t)
+        for (size_t j = 0; j < row; ++j) {
+            kt[(size_t)t * row + j] = bf(kc[(size_t)tokens[t] * row + j]);
+            vt[(size_t)t * row + j] = bf(vc[(size_t)tokens[t] * row + j]);
+        }
+    qsa_oracle_attention_backward_f64(c, qd, kt, vt, ntok, gd, dq, dk, dv);
+    free(qd);
+    free(gd);
+    free(kt);
+    free(vt);
+}
+
+/* Stage-1 target of query i: q [q_heads][d] (position-encoded, as the core
+ * attention takes it), kc [>= i + 1][kv_heads][d]. Writes t[b] for the
+ * floor(i/r) blocks the indexer scores (nothing when there are none). */
+void qsa_oracle_distill_target(const qsa_oracle_cfg* c, int64_t i, const uint16_t* q, const uint16_t* kc,
+                               double* t) {
+    const int64_t n_vis = i / c->r;
+    if (n_vis <= 0) return;
+    const int d = c->head_dim, hkv = c->kv_heads, g = c->q_heads / c->kv_heads;
+    const double scale = c->sm_scale > 0.0 ? c->sm_scale : 1.0 / sqrt((double)d);
+    double* avg = (double*)calloc((size_t)(i + 1), sizeof(double));
+    double* z = (double*)malloc(sizeof(double) * (size_t)(i + 1));
+    for (int h = 0; h < c->q_heads; ++h) {
+        /* dense causal softmax of head h over tokens 0..i */
+        double mx = -INFINITY;
+        for (int64_t j = 0; j <= i; ++j) {
+            const uint16_t* kr = kc + ((size_t)j * hkv + h / g) * d;
+            double dot = 0.0;
+            for (int e = 0; e < d; ++e) dot += bf(q[(size_t)h * d + e]) * bf(kr[e]);
+            z[j] = dot * scale;
+            if (z[j] > mx) mx = z[j];
+        }
+        double den = 0.0;
+        for (int64_t j = 0; j <= i; ++j) den += exp(z[j] - mx);
+        for (int64_t j = 0; j <= i; ++j) avg[j] += exp(z[j] - mx) / den;
+    }
+    for (int64_t j = 0; j <= i; ++j) avg[j] /= (double)c->q_heads;
+    double mass = 0.0;
+    for (int64_t b = 0; b < n_vis; ++b) {
+        double best = avg[b * c->r];
+        for (int e = 1; e < c->r; ++e)
+            if (avg[b * c->r + e] > best) best = avg[b * c->r + e];
+        t[b] = best;
+        mass += best;
+    }
+    for (int64_t b = 0; b < n_vis; ++b) t[b] /= mass;
+    free(avg);
+    free(z);
+}
+
+/* KL(t || softmax(s)) over n blocks, with 0 log 0 = 0, and its gradient with
+ * respect to the scores: d/ds_b = (sum_b' t_b') softmax(s)_b - t_b. ds may be
+ * NULL. Returns 0 for n = 0. */
+double qsa_oracle_distill_kl(const double* t, const float* s, int64_t n, double* ds) {
+    if (n <= 0) return 0.0;
+    double mx = -INFINITY;
+    for (int64_t b = 0; b < n; ++b)
+        if ((double)s[b] > mx) mx = (double)s[b];
+    double den = 0.0, tsum = 0.0;
+    for (int64_t b = 0; b < n; ++b) {
+        den += exp((double)s[b] - mx);
+        tsum += t[b];
+    }
+    const double log_den = mx + log(den);
+    double kl = 0.0;
+    for (int64_t b = 0; b < n; ++b) {
+        const double log_soft = (double)s[b] - log_den;
+        if (t[b] > 0.0) kl += t[b] * (log(t[b]) - log_soft);
+        if (ds) ds[b] = tsum * exp(log_soft) - t[b];
+    }
+    return kl;
 }

@@ -418,4 +418,173 @@ def pin_q8_attention_and_scores_on_exact_values(make):
     assert np.array_equal(o.scores_q8(qr, pc, ps, 12), o.scores(qr, pb, 12))
 
 
+# ----------------------------------------------------------------------------- training (f3)
+# "QSA (Qwen Sparse Attention)" concept page, "Native trainability via 2-stage
+# continued pretraining": stage 1 fits the indexer to a block-max-pooled dense
+# teacher distribution by KL; stage 2 trains through the sparse attention.
+def _f3_oracle(make, q_heads=4, kv_heads=2, head_dim=16):
+    return make(r=4, K=16, q_heads=q_heads, kv_heads=kv_heads, head_dim=head_dim)
+
+
+def pin_attention_f64_is_the_bf16_attention(make):
+    """The fp64-operand attention used for the gradient checks is the pinned
+    bf16 attention: the same outputs bit for bit on widened bf16 operands."""
+    w = GQA
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    _, _, q, k, v = _inputs(w)
+    i = 61
+    toks = np.array([0, 1, 2, 3, 20, 21, 22, 23, 36, 37, 38, 39, 60, 61], dtype=np.int64)
+    out, lse = o.attention(q[i], k.reshape(w.total, -1), v.reshape(w.total, -1), toks)
+    wid = bfm.bf16_to_f64
+    out2, lse2 = o.attention_f64(wid(q[i]), wid(k[toks]), wid(v[toks]))
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
+def pin_attention_backward_finite_differences(make):
+    """Every entry of dq, dk, dv matches a central difference of the loss
+    sum_h <dout_h, out_h> computed with the forward attention."""
+    o = _f3_oracle(make)
+    c = o.cfg
+    rng = np.random.default_rng(31)
+    ntok = 7
+    q = rng.standard_normal((c.q_heads, c.head_dim))
+    kt = rng.standard_normal((ntok, c.kv_heads, c.head_dim))
+    vt = rng.standard_normal((ntok, c.kv_heads, c.head_dim))
+    dout = rng.standard_normal((c.q_heads, c.head_dim))
+    grads = o.attention_backward_f64(q, kt, vt, dout)
+    base = [q, kt, vt]
+    h = 1e-6
+
+    def loss(args):
+        out, _ = o.attention_f64(*args)
+        return float((out * dout).sum())
+
+    for which in range(3):
+        for idx in np.ndindex(base[which].shape):
+            plus = [a.copy() for a in base]
+            minus = [a.copy() for a in base]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            fd = (loss(plus) - loss(minus)) / (2 * h)
+            g = grads[which][idx]
+            assert abs(fd - g) <= 1e-6 * (1.0 + abs(g)), (which, idx, fd, g)
+
+
+def pin_attention_backward_matches_autograd(make):
+    """The gradient equals torch autograd's (float64) through a plain GQA
+    softmax attention over the same tokens."""
+    import torch
+
+    o = _f3_oracle(make, q_heads=8, kv_heads=2, head_dim=32)
+    c = o.cfg
+    rng = np.random.default_rng(32)
+    ntok, G = 11, c.q_heads // c.kv_heads
+    q = rng.standard_normal((c.q_heads, c.head_dim))
+    kt = rng.standard_normal((ntok, c.kv_heads, c.head_dim))
+    vt = rng.standard_normal((ntok, c.kv_heads, c.head_dim))
+    dout = rng.standard_normal((c.q_heads, c.head_dim))
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, kt, vt))
+    kx, vx = tk.repeat_interleave(G, dim=1), tv.repeat_interleave(G, dim=1)
+    p = torch.softmax(torch.einsum("hd,thd->ht", tq, kx) / np.sqrt(c.head_dim), dim=1)
+    out = torch.einsum("ht,thd->hd", p, vx)
+    out.backward(torch.tensor(dout))
+    dq, dk, dv = o.attention_backward_f64(q, kt, vt, dout)
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(mine - ref.numpy()).max() < 1e-12
+
+
+def pin_attention_backward_bf16_gather(make):
+    """The bf16-operand gradient is the fp64 one on the listed tokens' widened
+    rows (one row per listed token, in list order)."""
+    w = GQA
+    o = make(r=w.r, K=w.K, q_heads=w.q_heads, kv_heads=w.kv_heads)
+    _, _, q, k, v = _inputs(w)
+    i = 50
+    toks = np.array([4, 5, 6, 7, 28, 29, 30, 31, 48, 49, 50], dtype=np.int64)
+    dout = _bits(np.random.default_rng(33).standard_normal((w.q_heads, w.head_dim)))
+    got = o.attention_backward(q[i], k.reshape(w.total, -1), v.reshape(w.total, -1), toks, dout)
+    wid = bfm.bf16_to_f64
+    ref = o.attention_backward_f64(wid(q[i]), wid(k[toks]), wid(v[toks]), wid(dout))
+    for a, b in zip(got, ref):
+        assert np.array_equal(a, b)
+
+
+def pin_distill_target_closed_forms(make):
+    """Closed forms of the stage-1 target. (1) Identical keys: every head is
+    uniform, so the target is uniform over the visible blocks. (2) Dominant
+    tokens: heads of kv head 0 put 1/4 on each of tokens 5, 6, 13 and the tail
+    token 20, heads of kv head 1 put everything on token 13; the head average
+    is 1/8, 1/8, 5/8, 1/8, block 1's maximum is 1/8 and block 3's 5/8, so the
+    target over blocks 0..4 is (0, 1/6, 0, 5/6, 0) (a mean pool, or a maximum
+    over heads, gives other values). Keys after the query (here a dominant
+    one and NaNs) are never read. (3) One key with logit L = 1 among zeros:
+    the target over blocks 0, 1 of query 8 is (e/(e+1), 1/(e+1))."""
+    o = _f3_oracle(make)
+    c = o.cfg
+    rng = np.random.default_rng(34)
+    d, hk = c.head_dim, c.kv_heads
+    nan = np.uint16(0x7FC0)
+    # (1)
+    i = 37
+    kc = np.full((i + 9, hk, d), _bits(np.float32(0.5)), dtype=np.uint16)
+    kc[i + 1:] = nan
+    q = _bits(rng.standard_normal((c.q_heads, d)).astype(np.float32))
+    t = o.distill_target(i, q, kc)
+    assert t.size == i // c.r and np.abs(t - 1.0 / t.size).max() < 1e-15
+    # (2)
+    i = 20
+    k = np.zeros((i + 9, hk, d), dtype=np.float32)
+    for j in (5, 6, 13, 20):
+        k[j, 0, 0] = 16.0
+    k[13, 1, 0] = 16.0
+    k[22, :, 0] = 64.0
+    kc = _bits(k)
+    kc[i + 3:] = nan
+    qf = np.zeros((c.q_heads, d), dtype=np.float32)
+    qf[:, 0] = 16.0
+    t = o.distill_target(i, _bits(qf), kc)
+    assert np.abs(t - np.array([0.0, 1 / 6, 0.0, 5 / 6, 0.0])).max() < 1e-12, t
+    # (3)
+    i = 8
+    k = np.zeros((i + 1, hk, d), dtype=np.float32)
+    k[1, :, 0] = 2.0
+    qf = np.zeros((c.q_heads, d), dtype=np.float32)
+    qf[:, 0] = 2.0  # logit 2 * 2 / sqrt(16) = 1
+    t = o.distill_target(i, _bits(qf), _bits(k))
+    e = np.e
+    assert np.abs(t - np.array([e / (e + 1), 1 / (e + 1)])).max() < 1e-14, t
+    # no visible block: nothing
+    assert o.distill_target(3, _bits(qf), _bits(k)).size == 0
+
+
+def pin_distill_kl_library_and_gradient(make):
+    """KL(t || softmax(s)) equals scipy's relative entropy (zero target entries
+    included); it is 0 with a zero gradient at s = log t + const; its gradient
+    matches central differences on exactly representable fp32 scores; no
+    blocks gives 0."""
+    from scipy.special import softmax
+    from scipy.stats import entropy
+
+    o = _f3_oracle(make)
+    rng = np.random.default_rng(35)
+    t = rng.random(50)
+    t[[3, 17, 40]] = 0.0
+    t /= t.sum()
+    s = (np.round(rng.standard_normal(50) * 3 * 256) / 256).astype(np.float32)
+    kl, ds = o.distill_kl(t, s)
+    assert abs(kl - entropy(t, softmax(s.astype(np.float64)))) < 1e-12
+    t2 = rng.random(20) + 0.1
+    t2 /= t2.sum()
+    kl0, ds0 = o.distill_kl(t2, (np.log(t2) + 3.0).astype(np.float32))
+    assert abs(kl0) < 1e-12 and np.abs(ds0).max() < 1e-6
+    h = 2.0 ** -12
+    for b in range(0, 50, 7):
+        sp, sm = s.copy(), s.copy()
+        sp[b] += np.float32(h)
+        sm[b] -= np.float32(h)
+        fd = (o.distill_kl(t, sp)[0] - o.distill_kl(t, sm)[0]) / (2 * h)
+        assert abs(fd - ds[b]) < 1e-6, (b, fd, ds[b])
+    assert o.distill_kl(np.zeros(0), np.zeros(0, dtype=np.float32))[0] == 0.0
+
+
 ALL_PINS = [v for kname, v in sorted(globals().items()) if kname.startswith("pin_")]

@@ -25,13 +25,18 @@ MUTANTS = {
     "rms_no_sqrt": ("const double rms = sqrt(ms + c->rms_eps);", "const double rms = ms + c->rms_eps;"),
     "relu_dropped": ("if (dot > 0.0) I += dot;", "I += dot;"),
     "score_one_head": ("dot += bf(qrot[(size_t)h * dim + j])", "dot += bf(qrot[(size_t)0 * dim + j])"),
-    "mask_includes_own_block": ("const int64_t n_vis = i / c->r;", "const int64_t n_vis = (i + 1) / c->r;"),
+    "mask_includes_own_block": ("const int64_t n_vis = i / c->r;\n    const int64_t k_b",
+                                "const int64_t n_vis = (i + 1) / c->r;\n    const int64_t k_b"),
+    "target_includes_own_block": ("const int64_t n_vis = i / c->r;\n    if (n_vis <= 0) return;",
+                                  "const int64_t n_vis = (i + 1) / c->r;\n    if (n_vis <= 0) return;"),
     "tie_to_higher_index": ("return (a->b > b->b) - (a->b < b->b);", "return (a->b < b->b) - (a->b > b->b);"),
     "budget_off_by_one": ("const int64_t m = n_vis < k_b ? n_vis : k_b;",
                           "const int64_t m = n_vis < k_b ? n_vis : k_b - 1;"),
     "tail_excludes_query": ("for (int64_t t = cur * c->r; t <= i; ++t)", "for (int64_t t = cur * c->r; t < i; ++t)"),
     "no_softmax_scale": ("logit[t] = dot * scale;", "logit[t] = dot;"),
-    "gqa_modulo": ("const int kvh = h / g;", "const int kvh = h % c->kv_heads;"),
+    "gqa_modulo": ("const int kvh = h / g;\n        double m = -INFINITY;",
+                   "const int kvh = h % c->kv_heads;\n        double m = -INFINITY;"),
+    "bwd_gqa_modulo": ("const int kvh = h / g;\n        const double* qh", "const int kvh = h % c->kv_heads;\n        const double* qh"),
     "values_from_keys": ("const uint16_t* vr = vc +", "const uint16_t* vr = kc +"),
     "decode_pool_early": ("if ((p + 1) % c->r == 0) {", "if (p % c->r == 0) {"),
     "e4m3_bias_8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
@@ -39,6 +44,20 @@ MUTANTS = {
     "quant_scale_max_normal_240": ("fl32_div(amax, 448.0)", "fl32_div(amax, 240.0)"),
     "q8_value_scale_dropped": ("o[j] += w * (qsa_oracle_e4m3_value(vc[row * d + j]) * vs[row]);",
                                "o[j] += w * qsa_oracle_e4m3_value(vc[row * d + j]);"),
+    "bwd_softmax_jacobian_no_delta": ("const double dz = p * (gv - delta);", "const double dz = p * gv;"),
+    "bwd_dk_unscaled": ("dkr[j] += scale * dz * qh[j];", "dkr[j] += dz * qh[j];"),
+    "bwd_dv_from_dz": ("dvr[j] += p * gh[j];", "dvr[j] += dz * gh[j];"),
+    "bwd_gather_first_token": ("kt[(size_t)t * row + j] = bf(kc[(size_t)tokens[t] * row + j]);",
+                               "kt[(size_t)t * row + j] = bf(kc[(size_t)tokens[0] * row + j]);"),
+    "target_mean_pool": ("if (avg[b * c->r + e] > best) best = avg[b * c->r + e];", "best += avg[b * c->r + e];"),
+    "target_max_over_heads": ("avg[j] += exp(z[j] - mx) / den;", "avg[j] = fmax(avg[j], exp(z[j] - mx) / den);"),
+    "target_not_normalised": ("for (int64_t b = 0; b < n_vis; ++b) t[b] /= mass;", ";"),
+    "target_unscaled_logits": ("z[j] = dot * scale;", "z[j] = dot;"),
+    "target_keys_shifted_past_query": ("const uint16_t* kr = kc + ((size_t)j * hkv + h / g) * d;",
+                                       "const uint16_t* kr = kc + ((size_t)(j + 1) * hkv + h / g) * d;"),
+    "kl_gradient_sign": ("if (ds) ds[b] = tsum * exp(log_soft) - t[b];", "if (ds) ds[b] = t[b] - tsum * exp(log_soft);"),
+    "kl_reversed": ("if (t[b] > 0.0) kl += t[b] * (log(t[b]) - log_soft);",
+                    "if (t[b] > 0.0) kl += exp(log_soft) * (log_soft - log(t[b]));"),
 }
 
 
