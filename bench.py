@@ -87,7 +87,21 @@ def algorithmic(w, kv="bf16"):
     ) * w.batch
     out["decode_tokens"] = dec_tok * w.batch
     out["prefill_tokens"] *= w.batch
-    for k in ("compress_bytes", "index_flops", "attn_gather_bytes", "attn_flops", "quantize_bytes"):
+    # Training kernels (zero unless the workload trains).
+    nq = n - q0
+    ld = (n - 1) // r
+    train = bool(getattr(w, "train", False)) and w.prefill
+    # backward: the forward's gather again, every (token, kv head) row's dK and
+    # dV added once per query that holds it (fp32), q / dout / out read, dq written.
+    out["bwd_bytes"] = (sum_t * w.kv_heads * (d * 2 * 2 + d * 4 * 2) + nq * w.q_heads * d * (2 * 3 + 4)) if train else 0
+    out["bwd_flops"] = sum_t * w.q_heads * d * 2 * 5 if train else 0  # S, dP, dQ, dK, dV products
+    # target: every head's logits over tokens <= i (log-sum-exp), then over the
+    # visible blocks' tokens (probabilities).
+    out["target_flops"] = int((i + 1 + r * vis).sum()) * w.q_heads * d * 2 if train else 0
+    out["scores_bytes"] = nq * (ld * 4 + w.idx_heads * w.idx_dim * 2) if train else 0
+    out["kl_bytes"] = (pairs * 4 * 2 + nq * ld * 4 + nq * 4) if train else 0  # target + scores read, dscores written
+    for k in ("compress_bytes", "index_flops", "attn_gather_bytes", "attn_flops", "quantize_bytes", "bwd_bytes",
+              "bwd_flops", "target_flops", "scores_bytes", "kl_bytes"):
         out[k] *= w.batch
     return out
 
@@ -263,6 +277,25 @@ class Bench:
                         "nsel": torch.empty(B, nq, dtype=torch.int32, device=device)}
             if q0:
                 L.compress(0, q0 // w.r)  # the existing cache's pooled keys
+            if w.train:
+                # Training step: the forward's LSE, a seeded upstream gradient, the
+                # gradients, and the stage-1 target / scores / loss rows.
+                dout = torch.empty_like(q)
+                for s in range(B):
+                    L_ = w.row_len("dout")
+                    synth.fill_device(w.seed(s), synth.TENSOR_IDS["dout"], q0 * L_, nq * L_, dout[s].data_ptr())
+                ld = (n - 1) // w.r
+                f32 = torch.float32
+                self.pre.update({
+                    "lse": torch.empty(B, nq, cfg.q_heads, dtype=f32, device=device), "dout": dout,
+                    "dq": torch.empty(B, nq, cfg.q_heads, cfg.head_dim, dtype=f32, device=device),
+                    "dk": torch.empty(B, cap, cfg.kv_heads, cfg.head_dim, dtype=f32, device=device),
+                    "dv": torch.empty(B, cap, cfg.kv_heads, cfg.head_dim, dtype=f32, device=device),
+                    "ld": ld, "target": torch.empty(B, nq, ld, dtype=f32, device=device),
+                    "scores": torch.empty(B, nq, ld, dtype=f32, device=device),
+                    "dscores": torch.empty(B, nq, ld, dtype=f32, device=device),
+                    "kl": torch.empty(B, nq, dtype=f32, device=device)})
+                L.workspace(qsa.OP_INDEX_SCORES, nq)
         else:
             L.compress(0, n // w.r)
         self.dec = []
@@ -350,7 +383,9 @@ class Bench:
                         mark("quantize")
             else:
                 L.prefill(p["q"], p["idx_q"], w.q_begin, w.n - w.q_begin, p["out"], p["sel"], p["nsel"],
-                          mark=mark)
+                          lse=p.get("lse"), mark=mark)
+            if w.train:
+                self.train_step(mark)
         if self.dec_graph is not None:
             self.dec_graph.replay()
             self.graph_launches += self.graph_kernels
@@ -361,6 +396,29 @@ class Bench:
                 dstep(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"])
         if mark and self.dec:
             mark("decode")
+
+    def train_step(self, mark=None):
+        """The training kernels after the forward: the sparse-attention gradient
+        (dk, dv accumulate, so they are cleared first), the stage-1 target, the
+        materialised indexer scores and the KL loss with its gradient."""
+        qsa, w, L, p, cfg = self.qsa, self.w, self.L, self.pre, self.cfg
+        q0, nq, B = w.q_begin, w.n - w.q_begin, w.batch
+        p["dk"].zero_()
+        p["dv"].zero_()
+        qsa.qsa_sparse_attention_backward(cfg, B, p["q"], q0, nq, L.k_cache, L.v_cache, L.cap, p["sel"], p["nsel"],
+                                          p["out"], p["lse"], p["dout"], p["dq"], p["dk"], p["dv"])
+        if mark:
+            mark("backward")
+        qsa.qsa_distill_target(cfg, B, p["q"], q0, nq, L.k_cache, L.cap, p["target"], p["ld"])
+        if mark:
+            mark("target")
+        qsa.qsa_index_scores(cfg, B, p["idx_q"], q0, nq, L.pooled, L.cap, p["scores"], p["ld"],
+                             L.workspace(qsa.OP_INDEX_SCORES, nq))
+        if mark:
+            mark("scores")
+        qsa.qsa_distill_kl(cfg, B, q0, nq, p["target"], p["scores"], p["ld"], p["kl"], p["dscores"])
+        if mark:
+            mark("kl")
 
     # -- end to end: host buffers in, host result out -----------------------------------
     def e2e(self, steps, warmup):
@@ -373,9 +431,11 @@ class Bench:
             return h
 
         if self.pre is not None:
-            for dst in (self.pre["q"], self.pre["idx_q"]):
+            for dst in (self.pre["q"], self.pre["idx_q"]) + ((self.pre["dout"],) if w.train else ()):
                 host_in.append((pin_like(dst), dst))
-            host_out.append((pin_like(self.pre["out"]), self.pre["out"]))
+            for src in (self.pre["out"],) + ((self.pre["kl"], self.pre["dq"], self.pre["dk"], self.pre["dv"])
+                                             if w.train else ()):
+                host_out.append((pin_like(src), src))
         for c in (L.k_cache, L.v_cache, L.idx_k_cache):
             for s in range(B):
                 # the step's new rows (a chunked prefill's earlier rows are cache state)
@@ -459,7 +519,9 @@ def run_cuda(args, w, rank, world):
     stages = {}
     defs = {"compress": ("hbm", alg["compress_bytes"]), "topk": ("tensor", alg["index_flops"]),
             "quantize": ("hbm", alg["quantize_bytes"]),
-            "attention": ("hbm", alg["attn_gather_bytes"]), "decode": ("hbm", alg["decode_bytes"])}
+            "attention": ("hbm", alg["attn_gather_bytes"]), "decode": ("hbm", alg["decode_bytes"]),
+            "backward": ("hbm", alg["bwd_bytes"]), "target": ("tensor", alg["target_flops"]),
+            "scores": ("hbm", alg["scores_bytes"]), "kl": ("hbm", alg["kl_bytes"])}
     for name, t in stage_ms.items():
         bound, amount = defs[name]
         if bound == "hbm":
@@ -474,6 +536,8 @@ def run_cuda(args, w, rank, world):
                         "frac": round(ach / peak, 4)}
     if "attention" in stages:
         stages["attention"]["tensor_tflops"] = round(alg["attn_flops"] / (stage_ms["attention"] * 1e-3) / 1e12, 2)
+    if "backward" in stages:
+        stages["backward"]["tensor_tflops"] = round(alg["bwd_flops"] / (stage_ms["backward"] * 1e-3) / 1e12, 2)
     dom = max(stage_ms, key=stage_ms.get)
     if b.dec and args.stage == "all":
         # Cold decode: the same steps again (re-writing the same cache rows), each
@@ -568,17 +632,29 @@ class OracleTimer:
 
     def _row(self, i):
         w, o = self.w, self.o
+        train = w.train and i < w.n
         iq = w.host_rows("idx_q", 0, [i]).reshape(w.idx_heads, w.idx_dim)
         qr = w.host_rows("q", 0, [i]).reshape(w.q_heads, w.head_dim)
         t = time.perf_counter()
-        res = o.row(i, iq, self.pooled, want_scores=False)
+        res = o.row(i, iq, self.pooled, want_scores=train)
         t_sel = time.perf_counter() - t
         toks = o.token_set(res["sel"], i)
         kc = w.host_rows("k", 0, toks)
         vc = w.host_rows("v", 0, toks)
         t = time.perf_counter()
         o.attention(qr, kc, vc, np.arange(toks.size, dtype=np.int64))
-        return t_sel + time.perf_counter() - t
+        t_att = time.perf_counter() - t
+        if not train:
+            return t_sel + t_att
+        # The training kernels' work for this row: the attention gradient, the
+        # stage-1 target over tokens <= i, and the KL with its gradient.
+        g = w.host_rows("dout", 0, [i]).reshape(w.q_heads, w.head_dim)
+        k_all = w.host_rows("k", 0, np.arange(i + 1))
+        t = time.perf_counter()
+        o.attention_backward(qr, kc, vc, np.arange(toks.size, dtype=np.int64), g)
+        tgt = o.distill_target(i, qr, k_all)
+        o.distill_kl(tgt, res["scores"])
+        return t_sel + t_att + time.perf_counter() - t
 
     def sample(self, rows, dec, blocks):
         w = self.w
@@ -640,6 +716,8 @@ class one_core:
 
 
 def cpu_baseline(w, rows=64, dec=2, blocks=65536):
+    if w.train:
+        rows = 16  # each row also runs the dense stage-1 target over tokens <= i
     with one_core():
         ot = OracleTimer(w)
         t, parts = ot.sample(rows, dec, blocks)

@@ -27,7 +27,8 @@ OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
            "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection", "qsa_quantize_rows",
-           "qsa_sparse_attention_q8", "qsa_decode_step_q8", "qsa_decode_step_offload"]
+           "qsa_sparse_attention_q8", "qsa_decode_step_q8", "qsa_decode_step_offload",
+           "qsa_sparse_attention_backward", "qsa_distill_target", "qsa_distill_kl"]
 
 
 class QSAError(RuntimeError):
@@ -84,6 +85,10 @@ _SIGS = {
     "qsa_decode_step": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp,
                         _vp, _vp, _sz, _vp],
     "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
+    "qsa_sparse_attention_backward": [_CFG, _i32, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _vp, _vp, _vp],
+    "qsa_distill_target": [_CFG, _i32, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp],
+    "qsa_distill_kl": [_CFG, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp],
     "qsa_quantize_rows": [_vp, _i64, _i32, _vp, _vp, _vp],
     "qsa_decode_step_q8": [_CFG, _i32] + [_vp] * 14 + [_i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "qsa_decode_step_offload": [_CFG, _i32] + [_vp] * 11 + [_i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz,
@@ -187,6 +192,30 @@ def qsa_sparse_attention(cfg: Config, batch: int, q: torch.Tensor, q_begin: int,
     _check(lib().qsa_sparse_attention(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache),
                                      _ptr(v_cache), cap, _ptr(sel), _ptr(nsel), _ptr(out), _ptr(lse),
                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def qsa_sparse_attention_backward(cfg: Config, batch: int, q: torch.Tensor, q_begin: int, nq: int,
+                                  k_cache: torch.Tensor, v_cache: torch.Tensor, cap: int, sel: torch.Tensor,
+                                  nsel: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, dout: torch.Tensor,
+                                  dq: torch.Tensor, dk: torch.Tensor, dv: torch.Tensor, stream=None) -> None:
+    """Gradient of qsa_sparse_attention: dq written, dk and dv added to (see include/qsa.h)."""
+    _check(lib().qsa_sparse_attention_backward(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache),
+                                              _ptr(v_cache), cap, _ptr(sel), _ptr(nsel), _ptr(out), _ptr(lse),
+                                              _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)))
+
+
+def qsa_distill_target(cfg: Config, batch: int, q: torch.Tensor, q_begin: int, nq: int, k_cache: torch.Tensor,
+                       cap: int, target: torch.Tensor, ld: int, stream=None) -> None:
+    """Stage-1 distillation target (see include/qsa.h)."""
+    _check(lib().qsa_distill_target(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache), cap,
+                                   _ptr(target), ld, _stream(stream)))
+
+
+def qsa_distill_kl(cfg: Config, batch: int, q_begin: int, nq: int, target: torch.Tensor, scores: torch.Tensor,
+                   ld: int, kl: torch.Tensor, dscores: Optional[torch.Tensor] = None, stream=None) -> None:
+    """KL(target || softmax(scores)) per query and its gradient (see include/qsa.h)."""
+    _check(lib().qsa_distill_kl(ctypes.byref(cfg.c()), batch, q_begin, nq, _ptr(target), _ptr(scores), ld,
+                               _ptr(kl), _ptr(dscores), _stream(stream)))
 
 
 def qsa_quantize_rows(x: torch.Tensor, rows: int, dim: int, codes: torch.Tensor, scales: torch.Tensor,

@@ -306,6 +306,71 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
                       "sparse attention");
 }
 
+qsa_status qsa_sparse_attention_backward(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin,
+                                         int64_t nq, const qsa_bf16* k_cache, const qsa_bf16* v_cache, int64_t cap,
+                                         const int32_t* sel, const int32_t* nsel, const qsa_bf16* out,
+                                         const float* lse, const qsa_bf16* dout, float* dq, float* dk, float* dv,
+                                         qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(k_cache);
+    REQUIRE_PTR(v_cache);
+    REQUIRE_PTR(sel);
+    REQUIRE_PTR(out);
+    REQUIRE_PTR(dout);
+    REQUIRE_PTR(dq);
+    REQUIRE_PTR(dk);
+    REQUIRE_PTR(dv);
+    if (!nsel || ((uintptr_t)nsel & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel NULL or misaligned");
+    if (!lse || ((uintptr_t)lse & 3u)) return fail(QSA_ERR_INVALID_ARG, "lse NULL or misaligned");
+    if (batch < 1 || cap < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (q_begin + nq > cap)
+        return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
+    if (nq == 0) return QSA_OK;
+    return cuda_check(qsa::launch_attention_backward(L, batch, q, q_begin, nq, k_cache, v_cache, cap, sel, nsel, out,
+                                                     lse, dout, dq, dk, dv, (cudaStream_t)stream),
+                      "sparse attention backward");
+}
+
+qsa_status qsa_distill_target(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin, int64_t nq,
+                              const qsa_bf16* k_cache, int64_t cap, float* target, int64_t ld, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    if (!qsa::distill_target_supported(L))
+        return fail(QSA_ERR_UNSUPPORTED, "distillation target: q_heads <= 32, q_heads/kv_heads dividing or "
+                                         "divisible by 8, r in {1, 2, 4, 8, 16}");
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(k_cache);
+    if (!target || ((uintptr_t)target & 3u)) return fail(QSA_ERR_INVALID_ARG, "target NULL or misaligned");
+    if (batch < 1 || cap < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (q_begin + nq > cap)
+        return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
+    if (nq > 0 && ld < (q_begin + nq - 1) / L.r)
+        return fail(QSA_ERR_INVALID_ARG, "ld=%lld < floor((q_begin + nq - 1) / r)", (long long)ld);
+    if (nq == 0) return QSA_OK;
+    return cuda_check(qsa::launch_distill_target(L, batch, q, q_begin, nq, k_cache, cap, target, ld,
+                                                 (cudaStream_t)stream),
+                      "distillation target");
+}
+
+qsa_status qsa_distill_kl(const qsa_config* cfg, int32_t batch, int64_t q_begin, int64_t nq, const float* target,
+                          const float* scores, int64_t ld, float* kl, float* dscores, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    if (!target || ((uintptr_t)target & 3u)) return fail(QSA_ERR_INVALID_ARG, "target NULL or misaligned");
+    if (!scores || ((uintptr_t)scores & 3u)) return fail(QSA_ERR_INVALID_ARG, "scores NULL or misaligned");
+    if (!kl || ((uintptr_t)kl & 3u)) return fail(QSA_ERR_INVALID_ARG, "kl NULL or misaligned");
+    if (dscores && ((uintptr_t)dscores & 3u)) return fail(QSA_ERR_INVALID_ARG, "dscores misaligned");
+    if (batch < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
+    if (nq > 0 && ld < (q_begin + nq - 1) / L.r)
+        return fail(QSA_ERR_INVALID_ARG, "ld=%lld < floor((q_begin + nq - 1) / r)", (long long)ld);
+    if (nq == 0) return QSA_OK;
+    return cuda_check(qsa::launch_distill_kl(L, batch, q_begin, nq, target, scores, ld, kl, dscores,
+                                             (cudaStream_t)stream),
+                      "distillation KL");
+}
+
 qsa_status qsa_quantize_rows(const qsa_bf16* x, int64_t rows, int32_t dim, uint8_t* codes, float* scales,
                              qsa_stream stream) {
     REQUIRE_PTR(x);

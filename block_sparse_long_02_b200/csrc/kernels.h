@@ -120,6 +120,22 @@ cudaError_t launch_install_hot(const LayerDims& L, int batch, const int64_t* pos
                                const int32_t* nsel, const uint16_t* host_k, const uint16_t* host_v, uint16_t* hot_k,
                                uint16_t* hot_v, int32_t* tags, int64_t blocks, cudaStream_t st);
 
+// attention_bwd.cu: gradient of launch_sparse_attention (dq written; dk, dv
+// accumulated with atomics).
+cudaError_t launch_attention_backward(const LayerDims& L, int batch, const uint16_t* q, int64_t q_begin, int64_t nq,
+                                      const uint16_t* kc, const uint16_t* vc, int64_t cap, const int32_t* sel,
+                                      const int32_t* nsel, const uint16_t* out, const float* lse,
+                                      const uint16_t* dout, float* dq, float* dk, float* dv, cudaStream_t st);
+
+// distill.cu: stage-1 distillation target (block-max-pooled, head-averaged
+// dense attention distribution over the visible blocks, normalised; zero from
+// floor(i/r) to ld) and the KL loss with its gradient w.r.t. the scores.
+bool distill_target_supported(const LayerDims& L);
+cudaError_t launch_distill_target(const LayerDims& L, int batch, const uint16_t* q, int64_t q_begin, int64_t nq,
+                                  const uint16_t* kc, int64_t cap, float* target, int64_t ld, cudaStream_t st);
+cudaError_t launch_distill_kl(const LayerDims& L, int batch, int64_t q_begin, int64_t nq, const float* target,
+                              const float* scores, int64_t ld, float* kl, float* dscores, cudaStream_t st);
+
 // quant.cu: FP8 E4M3 rows with one fp32 scale per row (dim 64, 128 or 256).
 cudaError_t launch_quantize_rows(const uint16_t* x, int64_t rows, int dim, uint8_t* codes, float* scales,
                                  cudaStream_t st);

@@ -158,6 +158,67 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
                                 const int32_t* nsel, qsa_bf16* out, float* lse, void* ws,
                                 size_t ws_bytes, qsa_stream stream);
 
+/* Gradient of qsa_sparse_attention (concept page, "Native trainability via
+ * 2-stage continued pretraining": stage 2 trains the model and the indexer
+ * together under the sparse selection, so the attention over the selected
+ * tokens is differentiated). For query i, core head h (kv head g) and the
+ * forward's token set T_i, with L = sum <dout, out>:
+ *   P[h][t]   = exp(sm_scale <q[h], k_cache[t][g]> - lse[h]);
+ *   dv[t][g] += sum over g's heads h of P[h][t] dout[h];
+ *   dS[h][t]  = P[h][t] (<dout[h], v_cache[t][g]> - <dout[h], out[h]>);
+ *   dq[h]     = sm_scale sum_t dS[h][t] k_cache[t][g];
+ *   dk[t][g] += sm_scale sum over g's heads h of dS[h][t] q[h].
+ * q, k_cache, v_cache, sel, nsel: as given to qsa_sparse_attention.
+ * out, lse: its outputs for them (lse is required here).
+ * dout: [batch][nq][q_heads][head_dim] bf16, the loss gradient w.r.t. out.
+ * dq:   [batch][nq][q_heads][head_dim] fp32, written.
+ * dk, dv: [batch][cap][kv_heads][head_dim] fp32, ADDED to (zero them before
+ *       the first call; calls over several query ranges accumulate).
+ * Probabilities are recomputed in fp32; P and dS are rounded to bf16 for the
+ * tile products, which accumulate in fp32; dk and dv take fp32 atomic adds, so
+ * their summation order (and last bits) may differ from run to run.
+ * Errors: q_begin + nq > cap -> QSA_ERR_CAPACITY. No workspace. */
+qsa_status qsa_sparse_attention_backward(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin,
+                                         int64_t nq, const qsa_bf16* k_cache, const qsa_bf16* v_cache, int64_t cap,
+                                         const int32_t* sel, const int32_t* nsel, const qsa_bf16* out,
+                                         const float* lse, const qsa_bf16* dout, float* dq, float* dk, float* dv,
+                                         qsa_stream stream);
+
+/* ---- Stage-1 indexer distillation ----
+ * Concept page, "Native trainability via 2-stage continued pretraining",
+ * stage 1: the indexer scores are trained to match a block-max-pooled version
+ * of the dense teacher attention distribution through a KL loss, while the
+ * model still runs dense attention. The page names the pieces, not their
+ * arithmetic; this library's reading: the teacher distribution of query i is
+ * the dense causal softmax of every core head over tokens j <= i, averaged
+ * over the heads; block b's pooled value is the largest of its r tokens'
+ * probabilities; only the blocks the indexer scores (b < floor(i/r)) are kept,
+ * normalised to sum to 1; the loss is KL(target || softmax of the scores). */
+
+/* target[s][j][b] = max over j' in block b of p_i(j') / sum over b' < floor(i/r)
+ *                   of the same maximum, for b < floor(i/r); 0 for
+ *                   floor(i/r) <= b < ld  (i = q_begin + j);
+ *   p_i(j') = (1/q_heads) sum_h softmax over j'' <= i of sm_scale <q[h], k_cache[j''][g(h)]>.
+ * q:       [batch][nq][q_heads][head_dim] bf16 (position-encoded, as the core
+ *          attention takes it); k_cache: [batch][cap][kv_heads][head_dim].
+ * target:  [batch][nq][ld] fp32; ld >= floor((q_begin + nq - 1) / r).
+ * Logits and softmax in fp32 (two sweeps over the keys: the heads' log-sum-exp,
+ * then the probabilities). Supported: q_heads <= 32, q_heads/kv_heads dividing
+ * or divisible by 8, r in {1, 2, 4, 8, 16}; else QSA_ERR_UNSUPPORTED. */
+qsa_status qsa_distill_target(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin, int64_t nq,
+                              const qsa_bf16* k_cache, int64_t cap, float* target, int64_t ld, qsa_stream stream);
+
+/* Per query i = q_begin + j, over its n = floor(i/r) visible blocks:
+ *   kl[s][j]         = sum_b t_b (log t_b - log softmax_b(scores)), 0 log 0 = 0
+ *                      (0 when n = 0);
+ *   dscores[s][j][b] = (sum_b' t_b') softmax_b(scores) - t_b for b < n, 0 for
+ *                      n <= b < ld (the gradient of kl; may be NULL).
+ * target: as qsa_distill_target writes it; scores: as qsa_index_scores writes
+ * them ([batch][nq][ld] fp32; entries from n on are not read).
+ * kl: [batch][nq] fp32. fp32 arithmetic. */
+qsa_status qsa_distill_kl(const qsa_config* cfg, int32_t batch, int64_t q_begin, int64_t nq, const float* target,
+                          const float* scores, int64_t ld, float* kl, float* dscores, qsa_stream stream);
+
 /* ---- Low-precision (fp8) caches ----
  * The "Qwen Sparse Attention" gallery page ("Community Quantized Version")
  * reports a quantized variant but not its format. This library's reading: a

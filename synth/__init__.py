@@ -40,7 +40,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _HOST_SO = os.path.join(_HERE, "libsynth_host.so")
 _DEV_SO = os.path.join(_HERE, "libsynth_device.so")
 
-TENSOR_IDS = {"idx_q": 1, "idx_k": 2, "q": 3, "k": 4, "v": 5}
+TENSOR_IDS = {"idx_q": 1, "idx_k": 2, "q": 3, "k": 4, "v": 5, "dout": 6}  # dout: an upstream gradient of out
 
 
 # ----------------------------------------------------------------------------- build / load
@@ -145,6 +145,7 @@ class Workload:
     base_seed: int = 0
     n_needles_prefill: int = 0  # per sequence, probes drawn among prefill positions
     n_needles_decode: int = 0   # per sequence; probes are decode positions (cycled)
+    train: bool = False         # the prefill also runs the training kernels (upstream gradient "dout")
 
     @property
     def k_blocks(self) -> int:
@@ -160,7 +161,7 @@ class Workload:
     def row_len(self, name: str) -> int:
         return {"idx_q": self.idx_heads * self.idx_dim, "idx_k": self.idx_dim,
                 "q": self.q_heads * self.head_dim, "k": self.kv_heads * self.head_dim,
-                "v": self.kv_heads * self.head_dim}[name]
+                "v": self.kv_heads * self.head_dim, "dout": self.q_heads * self.head_dim}[name]
 
     # -- needles ---------------------------------------------------------------
     def needles(self, seq: int) -> List[Tuple[int, int]]:
@@ -259,7 +260,7 @@ def _w(**kw) -> Workload:
     return Workload(**kw)
 
 
-# The five workloads the layer is measured on (contexts of 32K, ~261K and 1M tokens).
+# The workloads the layer is measured on (contexts of 32K, ~261K and 1M tokens).
 WORKLOADS: Dict[str, Workload] = {
     "tiny_prefill_n256": _w(name="tiny_prefill_n256", n=256, K=32, q_heads=4, kv_heads=1,
                             base_seed=0x51534101),
@@ -273,4 +274,7 @@ WORKLOADS: Dict[str, Workload] = {
     # Chunked prefill against an existing cache: the last 8192 positions of a 1M context.
     "prefill_chunk8k_n1m": _w(name="prefill_chunk8k_n1m", n=1048576, q_begin=1048576 - 8192,
                               base_seed=0x51534106),
+    # One training step of the layer on a 32K sequence: the prefill forward, the
+    # sparse-attention gradient and the stage-1 distillation target and loss.
+    "train_n32k": _w(name="train_n32k", n=32768, base_seed=0x51534107, train=True),
 }

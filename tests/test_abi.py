@@ -98,3 +98,29 @@ def test_binding_argument_counts_match_the_header(qsa):
         assert name in decls, name
         params = [p for p in decls[name].split(",") if p.strip() and p.strip() != "void"]
         assert len(args) == len(params), (name, len(args), len(params))
+
+
+def test_training_entry_points_validate_before_launching(qsa):
+    """The backward, distillation-target and KL calls reject bad arguments with
+    a status and launch nothing (fake, aligned, never dereferenced pointers)."""
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    for name in ("qsa_sparse_attention_backward", "qsa_distill_target", "qsa_distill_kl"):
+        getattr(lib, name).restype = ctypes.c_int
+        getattr(lib, name).argtypes = qsa._SIGS[name]
+    cfg = ctypes.byref(qsa.Config().c())
+    p = ctypes.c_void_p(4096)
+    bwd = lib.qsa_sparse_attention_backward
+    assert bwd(cfg, 1, p, 0, 16, p, p, 64, p, p, p, None, p, p, p, p, None) == 1  # lse is required
+    assert bwd(cfg, 1, p, 60, 16, p, p, 64, p, p, p, p, p, p, p, p, None) == 4  # queries past cap
+    assert bwd(cfg, 1, p, 0, 16, p, p, 64, p, p, p, p, p, None, p, p, None) == 1  # dq NULL
+    assert bwd(cfg, 1, p, 0, 0, p, p, 64, p, p, p, p, p, p, p, p, None) == 0  # nothing to do
+    tgt = lib.qsa_distill_target
+    assert tgt(cfg, 1, p, 0, 64, p, 64, p, 8, None) == 1  # ld < floor(63 / 4)
+    assert tgt(cfg, 1, p, 0, 64, p, 32, p, 16, None) == 4  # queries past cap
+    assert tgt(ctypes.byref(qsa.Config(r=3).c()), 1, p, 0, 8, p, 64, p, 16, None) == 2  # r outside {1,2,4,8,16}
+    assert tgt(ctypes.byref(qsa.Config(q_heads=64, kv_heads=4).c()), 1, p, 0, 8, p, 64, p, 16, None) == 2
+    assert tgt(cfg, 1, p, 0, 0, p, 64, p, 0, None) == 0
+    kl = lib.qsa_distill_kl
+    assert kl(cfg, 1, 0, 64, p, p, 8, p, None, None) == 1  # ld too small
+    assert kl(cfg, 1, 0, 64, p, p, 16, ctypes.c_void_p(4098), None, None) == 1  # kl misaligned
+    assert kl(cfg, 1, 0, 0, p, p, 0, p, None, None) == 0
