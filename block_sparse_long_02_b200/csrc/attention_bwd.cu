@@ -19,8 +19,8 @@
 //                                    layout is already the A-operand layout).
 // P and dS are rounded to bf16 for the products. dQ rows belong to one warp and
 // are written once; dK and dV rows are shared by every query that selected the
-// token, so each chunk's tiles are added with fp32 vector atomics (the order of
-// the additions is not fixed).
+// token, so each chunk's tiles are added with 16-byte fp32 vector atomics (the
+// order of the additions is not fixed).
 #include <algorithm>
 
 #include "kernels.h"
@@ -245,10 +245,13 @@ __global__ void __launch_bounds__(BW * 32) attention_backward_kernel(
         const uint32_t sa0 = pack_bf16x2(dp[0][0], dp[0][1]), sa1 = pack_bf16x2(dp[0][2], dp[0][3]);
         const uint32_t sa2 = NT > 1 ? pack_bf16x2(dp[NT - 1][0], dp[NT - 1][1]) : 0u;
         const uint32_t sa3 = NT > 1 ? pack_bf16x2(dp[NT - 1][2], dp[NT - 1][3]) : 0u;
-        float* dv0 = dv_seq + (size_t)(tk0 >= 0 ? tk0 : 0) * row_stride;
-        float* dv1 = dv_seq + (size_t)(tk1 >= 0 ? tk1 : 0) * row_stride;
-        float* dk0 = dk_seq + (size_t)(tk0 >= 0 ? tk0 : 0) * row_stride;
-        float* dk1 = dk_seq + (size_t)(tk1 >= 0 ? tk1 : 0) * row_stride;
+        // Atomics as float4: lanes t and t ^ 1 swap halves so that an even-t
+        // lane owns dims 2 t .. 2 t + 3 of row gq and an odd-t lane dims
+        // 2 t - 2 .. 2 t + 1 of row gq + 8.
+        const bool odd = t & 1;
+        const int32_t tkm = odd ? tk1 : tk0;
+        float* dvm = dv_seq + (size_t)(tkm >= 0 ? tkm : 0) * row_stride + 2 * (t & ~1);
+        float* dkm = dk_seq + (size_t)(tkm >= 0 ? tkm : 0) * row_stride + 2 * (t & ~1);
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {  // dims 16 jj .. 16 jj + 15 (two n8 tiles)
             uint32_t g0, g1, g2, g3, q0, q1, q2, q3;
@@ -259,14 +262,17 @@ __global__ void __launch_bounds__(BW * 32) attention_backward_kernel(
                 float vt[4] = {0.f, 0.f, 0.f, 0.f}, kt[4] = {0.f, 0.f, 0.f, 0.f};
                 mma_bf16_16816(vt, pa0, pa1, pa2, pa3, half ? g2 : g0, half ? g3 : g1);
                 mma_bf16_16816(kt, sa0, sa1, sa2, sa3, half ? q2 : q0, half ? q3 : q1);
-                const int dim = 16 * jj + 8 * half + 2 * t;
-                if (tk0 >= 0) {
-                    atomicAdd(reinterpret_cast<float2*>(dv0 + dim), make_float2(vt[0], vt[1]));
-                    atomicAdd(reinterpret_cast<float2*>(dk0 + dim), make_float2(kt[0] * scale, kt[1] * scale));
-                }
-                if (tk1 >= 0) {
-                    atomicAdd(reinterpret_cast<float2*>(dv1 + dim), make_float2(vt[2], vt[3]));
-                    atomicAdd(reinterpret_cast<float2*>(dk1 + dim), make_float2(kt[2] * scale, kt[3] * scale));
+                const int dim = 16 * jj + 8 * half;
+                const float v0 = __shfl_xor_sync(0xffffffffu, odd ? vt[0] : vt[2], 1);
+                const float v1 = __shfl_xor_sync(0xffffffffu, odd ? vt[1] : vt[3], 1);
+                const float k0 = __shfl_xor_sync(0xffffffffu, odd ? kt[0] : kt[2], 1);
+                const float k1 = __shfl_xor_sync(0xffffffffu, odd ? kt[1] : kt[3], 1);
+                if (tkm >= 0) {
+                    atomicAdd(reinterpret_cast<float4*>(dvm + dim),
+                              odd ? make_float4(v0, v1, vt[2], vt[3]) : make_float4(vt[0], vt[1], v0, v1));
+                    atomicAdd(reinterpret_cast<float4*>(dkm + dim),
+                              odd ? make_float4(k0 * scale, k1 * scale, kt[2] * scale, kt[3] * scale)
+                                  : make_float4(kt[0] * scale, kt[1] * scale, k0 * scale, k1 * scale));
                 }
             }
         }

@@ -15,7 +15,7 @@
 // S^T = K Q^T on the tensor cores (mma.sync m16n8k16: the chunk's 16 tokens as
 // the m16 rows, its query's heads as the n8 columns, query fragments held in
 // registers for the whole sweep), so the head average of a token is a sum over
-// the warp's own columns. Sweep 1 keeps the online maximum and sum of every
+// the warp's own columns. Sweep 1 keeps a running sum of exponentials of every
 // head over tokens <= i (its log-sum-exp); sweep 2 recomputes the logits,
 // averages the probabilities over the heads, takes each block's maximum with
 // shuffles, writes it and sums it; the warp then normalises its row.
@@ -146,6 +146,10 @@ __global__ void __launch_bounds__(DQ * 32) distill_target_kernel(
         float sc[NTQ][4];
         scores(c & 1, sc);
         const int64_t t0 = (int64_t)c * DCT + gq, t1 = t0 + 8;
+        // Lane-local running sums (merged over the 8 lanes of a column after
+        // the sweep). The reference maximum is raised only when a logit exceeds
+        // it by more than 8 (log2 units), so terms stay below 2^8 and most
+        // chunks take one exponential per logit and no rescaling.
 #pragma unroll
         for (int k = 0; k < NTQ; ++k)
 #pragma unroll
@@ -153,33 +157,31 @@ __global__ void __launch_bounds__(DQ * 32) distill_target_kernel(
                 const bool hv = 8 * k + 2 * t + e < q_heads;
                 const float x0 = (hv && t0 <= i) ? sc[k][e] * scale_log2 : -INFINITY;
                 const float x1 = (hv && t1 <= i) ? sc[k][2 + e] * scale_log2 : -INFINITY;
-                float mx = fmaxf(x0, x1);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                const float mn = fmaxf(m[k][e], mx);
-                if (mn != -INFINITY) {
-                    const float corr = ex2_approx(m[k][e] - mn);
-                    const float p0 = x0 == -INFINITY ? 0.f : ex2_approx(x0 - mn);
-                    const float p1 = x1 == -INFINITY ? 0.f : ex2_approx(x1 - mn);
-                    l[k][e] = l[k][e] * corr + p0 + p1;
-                    m[k][e] = mn;
+                const float mx = fmaxf(x0, x1);
+                if (mx > m[k][e] + 8.f) {
+                    l[k][e] *= ex2_approx(m[k][e] - mx);  // (0 while m is -inf)
+                    m[k][e] = mx;
                 }
+                if (mx != -INFINITY) l[k][e] += ex2_approx(x0 - m[k][e]) + ex2_approx(x1 - m[k][e]);
             }
         __syncthreads();  // the stage is refilled next iteration
     }
     cp_async_wait<0>();
-    // lse per column (log2 domain), over the 8 lanes that share t.
+    // lse per column (log2 domain): merge the 8 lanes that share t.
     float lse2[NTQ][2];
 #pragma unroll
     for (int k = 0; k < NTQ; ++k)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            float sum = l[k][e];
+            float mc = m[k][e];
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, 4));
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, 8));
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, 16));
+            float sum = m[k][e] == -INFINITY ? 0.f : l[k][e] * ex2_approx(m[k][e] - mc);
             sum += __shfl_xor_sync(0xffffffffu, sum, 4);
             sum += __shfl_xor_sync(0xffffffffu, sum, 8);
             sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-            lse2[k][e] = m[k][e] + log2f(sum);
+            lse2[k][e] = mc + log2f(sum);
         }
 
     // Sweep 2: head-averaged probabilities, block maxima, their sum.
