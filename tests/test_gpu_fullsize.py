@@ -211,3 +211,62 @@ def test_prefill_1m_then_64_decode_steps_sampled():
         if step in (0, 3, 31, 63):
             torch.cuda.synchronize()
             _check_decode_step(w, o, L, step, dout, dsel, dn, range(B))
+
+
+def test_train_32k_full_size():
+    """The training step bench.py times on train_n32k (forward, sparse-attention
+    gradient, stage-1 target, indexer scores, KL), through bench's own Bench.
+    Sampled rows against the oracle (dq, target, KL and its gradient); every
+    row and token against identities that hold at any size: target rows are
+    distributions over the visible blocks, KL >= 0 with a gradient summing to
+    0, the dv rows of a kv head sum to the sum of its heads' upstream gradients
+    (every P row sums to 1) and the dk rows to 0 (every dS row sums to 0)."""
+    import bench
+
+    w = synth.WORKLOADS["train_n32k"]
+    b = bench.Bench(w, torch.device("cuda", 0))
+    b.step()
+    torch.cuda.synchronize()
+    p, cfg, n, r = b.pre, b.cfg, w.n, w.r
+    o = _oracle(w)
+    G, hk = cfg.q_heads // cfg.kv_heads, cfg.kv_heads
+    # every row: distributions, zeros past the visible blocks, KL >= 0, sum of dKL/dI = 0
+    tgt = p["target"][0]
+    vis = torch.arange(n, device="cuda") // r
+    cols = torch.arange(p["ld"], device="cuda")[None, :]
+    inside = cols < vis[:, None]
+    assert (tgt[~inside] == 0).all() and (tgt >= 0).all()
+    sums = tgt.double().sum(1)
+    assert ((sums - 1).abs()[vis > 0] < 1e-4).all() and (sums[vis == 0] == 0).all()
+    assert (p["kl"][0] > -1e-5).all()
+    ds_sum = p["dscores"][0].double().sum(1)
+    assert (ds_sum.abs() < 1e-4).all()
+    # dv / dk column identities per kv head
+    dv = p["dv"][0, :n].double().sum(0)                      # [kv][128]
+    dk = p["dk"][0, :n].double().sum(0)
+    dout = p["dout"][0].double().view(n, hk, G, 128).sum(dim=(0, 2))
+    scale_v = p["dout"][0].double().abs().view(n, hk, G, 128).sum(dim=(0, 2))
+    assert ((dv - dout).abs() <= 1e-2 * scale_v).all(), (dv - dout).abs().max().item()
+    scale_k = p["dk"][0, :n].double().abs().sum(0)
+    assert (dk.abs() <= 2e-2 * scale_k + 1e-6).all(), (dk.abs() / scale_k).max().item()
+    # sampled rows against the oracle
+    rows = _sample_rows(w, 5, 0x7A)
+    sel, nsel = p["sel"][0].cpu().numpy(), p["nsel"][0].cpu().numpy()
+    dq = p["dq"][0]
+    k_all = w.host_full("k", 0, n)
+    for i in rows:
+        qi = w.host_rows("q", 0, [i]).reshape(cfg.q_heads, 128)
+        gi = w.host_rows("dout", 0, [i]).reshape(cfg.q_heads, 128)
+        toks = o.token_set(sel[i, :nsel[i]], i)
+        kc, vc = w.host_rows("k", 0, toks), w.host_rows("v", 0, toks)
+        ref_dq, _, _ = o.attention_backward(qi, kc, vc, np.arange(toks.size, dtype=np.int64), gi)
+        got = dq[i].cpu().numpy()
+        assert np.abs(got - ref_dq).max() <= 1e-2 * np.abs(ref_dq).max(), f"dq row {i}"
+        ref_t = o.distill_target(i, qi, k_all)
+        got_t = tgt[i, : i // r].cpu().numpy()
+        assert (np.abs(got_t - ref_t) <= 2e-3 * ref_t + 1e-7).all(), f"target row {i}"
+        ref_kl, ref_ds = o.distill_kl(got_t.astype(np.float64), p["scores"][0, i, : i // r].cpu().numpy())
+        assert abs(p["kl"][0, i].item() - ref_kl) <= 1e-4 * (1 + abs(ref_kl)), f"kl row {i}"
+        got_ds = p["dscores"][0, i, : i // r].cpu().numpy()
+        big = np.abs(ref_ds).max() if ref_ds.size else 0.0
+        assert (np.abs(got_ds - ref_ds) <= 1e-4 * np.abs(ref_ds) + 1e-6 * big + 1e-9).all(), f"dscores row {i}"
