@@ -296,6 +296,7 @@ class Bench:
                     "dscores": torch.empty(B, nq, ld, dtype=f32, device=device),
                     "kl": torch.empty(B, nq, dtype=f32, device=device)})
                 L.workspace(qsa.OP_INDEX_SCORES, nq)
+                L.workspace(qsa.OP_DISTILL_TARGET, nq)
         else:
             L.compress(0, n // w.r)
         self.dec = []
@@ -409,7 +410,8 @@ class Bench:
                                           p["out"], p["lse"], p["dout"], p["dq"], p["dk"], p["dv"])
         if mark:
             mark("backward")
-        qsa.qsa_distill_target(cfg, B, p["q"], q0, nq, L.k_cache, L.cap, p["target"], p["ld"])
+        qsa.qsa_distill_target(cfg, B, p["q"], q0, nq, L.k_cache, L.cap, p["target"], p["ld"],
+                               L.workspace(qsa.OP_DISTILL_TARGET, nq))
         if mark:
             mark("target")
         qsa.qsa_index_scores(cfg, B, p["idx_q"], q0, nq, L.pooled, L.cap, p["scores"], p["ld"],

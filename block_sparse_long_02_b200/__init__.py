@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libqsa.so")
 QSA_OK = 0
 STATUS_NAMES = {0: "QSA_OK", 1: "QSA_ERR_INVALID_ARG", 2: "QSA_ERR_UNSUPPORTED", 3: "QSA_ERR_WORKSPACE",
                 4: "QSA_ERR_CAPACITY", 5: "QSA_ERR_CUDA", 6: "QSA_ERR_TIMEOUT", 7: "QSA_ERR_DEVICE_CHECK"}
-OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP = 0, 1, 2, 3
+OP_INDEX_SCORES, OP_TOPK_BLOCKS, OP_SPARSE_ATTENTION, OP_DECODE_STEP, OP_DISTILL_TARGET = 0, 1, 2, 3, 4
 
 EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_topk_blocks",
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
@@ -87,7 +87,7 @@ _SIGS = {
     "qsa_workspace_status": [_vp, _vp, ctypes.POINTER(_i32)],
     "qsa_sparse_attention_backward": [_CFG, _i32, _vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                                       _vp, _vp, _vp],
-    "qsa_distill_target": [_CFG, _i32, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp],
+    "qsa_distill_target": [_CFG, _i32, _vp, _i64, _i64, _vp, _i64, _vp, _i64, _vp, _sz, _vp],
     "qsa_distill_kl": [_CFG, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp],
     "qsa_quantize_rows": [_vp, _i64, _i32, _vp, _vp, _vp],
     "qsa_decode_step_q8": [_CFG, _i32] + [_vp] * 14 + [_i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
@@ -205,10 +205,10 @@ def qsa_sparse_attention_backward(cfg: Config, batch: int, q: torch.Tensor, q_be
 
 
 def qsa_distill_target(cfg: Config, batch: int, q: torch.Tensor, q_begin: int, nq: int, k_cache: torch.Tensor,
-                       cap: int, target: torch.Tensor, ld: int, stream=None) -> None:
+                       cap: int, target: torch.Tensor, ld: int, ws: torch.Tensor, stream=None) -> None:
     """Stage-1 distillation target (see include/qsa.h)."""
     _check(lib().qsa_distill_target(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache), cap,
-                                   _ptr(target), ld, _stream(stream)))
+                                   _ptr(target), ld, _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def qsa_distill_kl(cfg: Config, batch: int, q_begin: int, nq: int, target: torch.Tensor, scores: torch.Tensor,

@@ -194,6 +194,7 @@ qsa_status qsa_workspace_size(const qsa_config* cfg, int32_t op, int32_t batch, 
         case QSA_OP_TOPK_BLOCKS: *bytes = topk_layout(L, batch, cap, nq).total; break;
         case QSA_OP_SPARSE_ATTENTION: *bytes = qsa::kWsHeader; break;
         case QSA_OP_DECODE_STEP: *bytes = decode_layout(L, batch, cap).total; break;
+        case QSA_OP_DISTILL_TARGET: *bytes = qsa::distill_target_ws_bytes(batch, nq, L.q_heads); break;
         default: return fail(QSA_ERR_INVALID_ARG, "unknown op %d", op);
     }
     return QSA_OK;
@@ -334,7 +335,8 @@ qsa_status qsa_sparse_attention_backward(const qsa_config* cfg, int32_t batch, c
 }
 
 qsa_status qsa_distill_target(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin, int64_t nq,
-                              const qsa_bf16* k_cache, int64_t cap, float* target, int64_t ld, qsa_stream stream) {
+                              const qsa_bf16* k_cache, int64_t cap, float* target, int64_t ld, void* ws,
+                              size_t ws_bytes, qsa_stream stream) {
     qsa::LayerDims L;
     TRY(make_dims(cfg, &L));
     if (!qsa::distill_target_supported(L))
@@ -349,7 +351,10 @@ qsa_status qsa_distill_target(const qsa_config* cfg, int32_t batch, const qsa_bf
     if (nq > 0 && ld < (q_begin + nq - 1) / L.r)
         return fail(QSA_ERR_INVALID_ARG, "ld=%lld < floor((q_begin + nq - 1) / r)", (long long)ld);
     if (nq == 0) return QSA_OK;
-    return cuda_check(qsa::launch_distill_target(L, batch, q, q_begin, nq, k_cache, cap, target, ld,
+    const size_t need = qsa::distill_target_ws_bytes(batch, nq, L.q_heads);
+    if (!ws || !aligned16(ws) || ws_bytes < need)
+        return fail(QSA_ERR_WORKSPACE, "workspace %zu bytes < %zu (or NULL / misaligned)", ws_bytes, need);
+    return cuda_check(qsa::launch_distill_target(L, batch, q, q_begin, nq, k_cache, cap, target, ld, ws,
                                                  (cudaStream_t)stream),
                       "distillation target");
 }

@@ -131,8 +131,12 @@ cudaError_t launch_attention_backward(const LayerDims& L, int batch, const uint1
 // dense attention distribution over the visible blocks, normalised; zero from
 // floor(i/r) to ld) and the KL loss with its gradient w.r.t. the scores.
 bool distill_target_supported(const LayerDims& L);
+// distill_tc.cu: the target on tcgen05; ws = status header + the heads'
+// log-sum-exps [batch][nq][q_heads] fp32.
+size_t distill_target_ws_bytes(int batch, int64_t nq, int q_heads);
 cudaError_t launch_distill_target(const LayerDims& L, int batch, const uint16_t* q, int64_t q_begin, int64_t nq,
-                                  const uint16_t* kc, int64_t cap, float* target, int64_t ld, cudaStream_t st);
+                                  const uint16_t* kc, int64_t cap, float* target, int64_t ld, void* ws,
+                                  cudaStream_t st);
 cudaError_t launch_distill_kl(const LayerDims& L, int batch, int64_t q_begin, int64_t nq, const float* target,
                               const float* scores, int64_t ld, float* kl, float* dscores, cudaStream_t st);
 

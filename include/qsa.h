@@ -82,7 +82,8 @@ typedef enum {
     QSA_OP_INDEX_SCORES = 0,     /* qsa_index_scores */
     QSA_OP_TOPK_BLOCKS = 1,      /* qsa_topk_blocks (both modes) */
     QSA_OP_SPARSE_ATTENTION = 2, /* qsa_sparse_attention */
-    QSA_OP_DECODE_STEP = 3       /* qsa_decode_step */
+    QSA_OP_DECODE_STEP = 3,      /* qsa_decode_step */
+    QSA_OP_DISTILL_TARGET = 4    /* qsa_distill_target */
 } qsa_op;
 
 /* Bytes of workspace `op` needs for `batch` sequences of capacity `cap` and
@@ -202,11 +203,15 @@ qsa_status qsa_sparse_attention_backward(const qsa_config* cfg, int32_t batch, c
  * q:       [batch][nq][q_heads][head_dim] bf16 (position-encoded, as the core
  *          attention takes it); k_cache: [batch][cap][kv_heads][head_dim].
  * target:  [batch][nq][ld] fp32; ld >= floor((q_begin + nq - 1) / r).
- * Logits and softmax in fp32 (two sweeps over the keys: the heads' log-sum-exp,
- * then the probabilities). Supported: q_heads <= 32, q_heads/kv_heads dividing
- * or divisible by 8, r in {1, 2, 4, 8, 16}; else QSA_ERR_UNSUPPORTED. */
+ * ws:      qsa_workspace_size(QSA_OP_DISTILL_TARGET, batch, cap, nq) bytes (the
+ *          heads' log-sum-exps); a smaller one returns QSA_ERR_WORKSPACE.
+ * Logits on the tensor cores (bf16 in, fp32 accumulate), softmax in fp32: two
+ * passes over the keys (every head's log-sum-exp, then the probabilities).
+ * Supported: q_heads <= 32, q_heads/kv_heads in {1, 2, 4, 8, 16}, r in
+ * {1, 2, 4, 8, 16}; else QSA_ERR_UNSUPPORTED. */
 qsa_status qsa_distill_target(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin, int64_t nq,
-                              const qsa_bf16* k_cache, int64_t cap, float* target, int64_t ld, qsa_stream stream);
+                              const qsa_bf16* k_cache, int64_t cap, float* target, int64_t ld, void* ws,
+                              size_t ws_bytes, qsa_stream stream);
 
 /* Per query i = q_begin + j, over its n = floor(i/r) visible blocks:
  *   kl[s][j]         = sum_b t_b (log t_b - log softmax_b(scores)), 0 log 0 = 0

@@ -115,11 +115,14 @@ def test_training_entry_points_validate_before_launching(qsa):
     assert bwd(cfg, 1, p, 0, 16, p, p, 64, p, p, p, p, p, None, p, p, None) == 1  # dq NULL
     assert bwd(cfg, 1, p, 0, 0, p, p, 64, p, p, p, p, p, p, p, p, None) == 0  # nothing to do
     tgt = lib.qsa_distill_target
-    assert tgt(cfg, 1, p, 0, 64, p, 64, p, 8, None) == 1  # ld < floor(63 / 4)
-    assert tgt(cfg, 1, p, 0, 64, p, 32, p, 16, None) == 4  # queries past cap
-    assert tgt(ctypes.byref(qsa.Config(r=3).c()), 1, p, 0, 8, p, 64, p, 16, None) == 2  # r outside {1,2,4,8,16}
-    assert tgt(ctypes.byref(qsa.Config(q_heads=64, kv_heads=4).c()), 1, p, 0, 8, p, 64, p, 16, None) == 2
-    assert tgt(cfg, 1, p, 0, 0, p, 64, p, 0, None) == 0
+    big = 1 << 20
+    assert tgt(cfg, 1, p, 0, 64, p, 64, p, 8, p, big, None) == 1  # ld < floor(63 / 4)
+    assert tgt(cfg, 1, p, 0, 64, p, 32, p, 16, p, big, None) == 4  # queries past cap
+    assert tgt(ctypes.byref(qsa.Config(r=3).c()), 1, p, 0, 8, p, 64, p, 16, p, big, None) == 2  # r not in {1..16}
+    assert tgt(ctypes.byref(qsa.Config(q_heads=64, kv_heads=4).c()), 1, p, 0, 8, p, 64, p, 16, p, big, None) == 2
+    assert tgt(cfg, 1, p, 0, 64, p, 64, p, 16, p, 256, None) == 3  # workspace without the lse rows
+    assert tgt(cfg, 1, p, 0, 0, p, 64, p, 0, None, 0, None) == 0
+    assert qsa.qsa_workspace_size(qsa.Config(), qsa.OP_DISTILL_TARGET, 2, 64, 10) == 256 + 2 * 10 * 32 * 4
     kl = lib.qsa_distill_kl
     assert kl(cfg, 1, 0, 64, p, p, 8, p, None, None) == 1  # ld too small
     assert kl(cfg, 1, 0, 64, p, p, 16, ctypes.c_void_p(4098), None, None) == 1  # kl misaligned

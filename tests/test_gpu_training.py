@@ -103,14 +103,18 @@ def _target_case(qsa, w, cfg, cap, q_begin, nq):
     q = dev_full(w, "q", cap, q_begin + nq)[:, q_begin:q_begin + nq].contiguous()
     ld = (q_begin + nq - 1) // cfg.r + 3
     target = torch.full((w.batch, nq, ld), float("nan"), dtype=torch.float32, device="cuda")
-    qsa.qsa_distill_target(cfg, w.batch, q, q_begin, nq, kc, cap, target, ld)
+    ws = torch.zeros(qsa.qsa_workspace_size(cfg, qsa.OP_DISTILL_TARGET, w.batch, cap, nq), dtype=torch.uint8,
+                     device="cuda")
+    qsa.qsa_distill_target(cfg, w.batch, q, q_begin, nq, kc, cap, target, ld, ws)
     torch.cuda.synchronize()
+    assert qsa.qsa_workspace_status(ws) == 0
     return target.cpu().numpy(), ld
 
 
 @pytest.mark.parametrize("n,q_begin,r,q_heads,kv_heads,batch",
                          [(700, 0, 4, 32, 4, 2), (611, 250, 4, 32, 4, 1), (300, 0, 1, 8, 8, 1),
-                          (530, 0, 16, 16, 1, 1)])
+                          (530, 0, 16, 16, 1, 1), (401, 0, 2, 16, 8, 1), (333, 0, 8, 16, 4, 1),
+                          (290, 0, 4, 32, 2, 1)])
 def test_distill_target_matches_oracle(qsa, n, q_begin, r, q_heads, kv_heads, batch):
     """Every entry of every row: the oracle's block-max-pooled, head-averaged
     dense distribution over the visible blocks; zeros from floor(i/r) to ld."""
