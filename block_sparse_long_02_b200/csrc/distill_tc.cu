@@ -6,16 +6,19 @@
 // Two passes over the keys, each a tcgen05 kernel with the same roles: warp 0
 // issues TMA tile loads (SWIZZLE_128B) into a 4-stage key ring, warp 1 issues
 // tcgen05.mma (kind::f16, fp32 accumulators in TMEM, double-buffered against
-// the epilogue) and warps 2-5 are the epilogue (one TMEM lane each).
+// the epilogue) and warps 2-9 are the epilogue (two warps per TMEM lane
+// quadrant, each taking half of the quadrant's columns).
 //   distill_lse_kernel:  rows (M = 128) = the query heads of one kv head for
 //     128 / G queries, columns (N = 128) = keys. Each epilogue thread owns one
-//     (query, head) row and keeps a running sum of exponentials of its logits
-//     over keys <= i (raising its reference maximum only when a logit exceeds
-//     it by more than 2^8): the head's log-sum-exp, written to the workspace.
+//     (query, head) row for half the key columns and keeps a running sum of
+//     exponentials of its logits over keys <= i (raising its reference maximum
+//     only when a logit exceeds it by more than 2^8); the two halves merge
+//     into the head's log-sum-exp, written to the workspace.
 //   distill_pool_kernel: rows (M = 128) = keys, columns = (query, head) for
 //     8 queries (16 when G = 1) and every head, one MMA per kv head. Each
-//     thread owns one key: the head average of its probabilities for each
-//     query is a sum over its own columns, the block maximum a shuffle over
+//     thread owns one key and half of the queries: the head average of its
+//     probabilities for a query is a sum over its own columns, the block
+//     maximum a shuffle over
 //     the r lanes of the block; the block values are written and summed, and
 //     each row is normalised at the end.
 // Every wait is bounded (10 s of %globaltimer); on expiry the kernel records
@@ -30,8 +33,8 @@
 namespace qsa {
 namespace {
 
-constexpr int TC_THREADS = 192;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int EPI = 128;             // epilogue threads (one TMEM lane each)
+constexpr int TC_THREADS = 320;      // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int EPI = 256;             // epilogue threads: two warps per TMEM lane quadrant
 constexpr int KT = 128;              // keys per tile
 constexpr int HALF = 128 * 128;      // one 64-dim half of a 128-row bf16 tile
 constexpr int TILE = 2 * HALF;       // 128 rows x 128 dims
@@ -150,7 +153,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_lse_kernel(
             }
         }
     } else {
-        // Epilogue: thread = TMEM lane = row (query qi, head h) of the tile.
+        // Epilogue: thread = TMEM lane = row (query qi, head h) of the tile; the
+        // two warps of a quadrant take key columns [0, 64) and [64, 128).
+        const int ew = warp - 2, hc = ew >> 2;
         const int qd = warp & 3;
         const int row = qd * 32 + lane;
         const int qi = row / G, h = row % G;
@@ -163,36 +168,55 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_lse_kernel(
                                        tc::mbar_wait(bar_s(bars.acc_full[buf]), (t >> 1) & 1, abort_flag, WAIT_NS));
             if (!ok) break;
             tc::fence_after();
-            float v[KT];
-            const uint32_t a = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * KT);
+            constexpr int HC = KT / 2;
+            float v[HC];
+            const uint32_t a = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * KT + hc * HC);
 #pragma unroll
-            for (int c = 0; c < KT / 16; ++c) tc::tmem_ld16(a + c * 16, v + c * 16);
+            for (int c = 0; c < HC / 16; ++c) tc::tmem_ld16(a + c * 16, v + c * 16);
             tc::tmem_wait_ld();
             tc::fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar_s(bars.acc_empty[buf]));
-            const int64_t nvalid = i - (int64_t)t * KT + 1;  // keys of this tile that are <= i
+            const int64_t nvalid = i - ((int64_t)t * KT + hc * HC) + 1;  // columns whose key is <= i
             if (!live || nvalid <= 0) continue;
-            float tmax = -INFINITY;
+            float vmax = -INFINITY;
+            if (nvalid >= HC) {
 #pragma unroll
-            for (int c = 0; c < KT; ++c) {
-                v[c] = c < nvalid ? v[c] * scale_log2 : -INFINITY;
-                tmax = fmaxf(tmax, v[c]);
+                for (int c = 0; c < HC; ++c) vmax = fmaxf(vmax, v[c]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < HC; ++c) {
+                    v[c] = c < nvalid ? v[c] : -INFINITY;
+                    vmax = fmaxf(vmax, v[c]);
+                }
             }
+            const float tmax = vmax * scale_log2;  // (the scale is positive)
             if (tmax > m + 8.f) {
                 l *= ex2_approx(m - tmax);  // (0 while m is -inf)
                 m = tmax;
             }
             float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < KT; c += 2) {
-                acc0 += ex2_approx(v[c] - m);
-                acc1 += ex2_approx(v[c + 1] - m);
+            for (int c = 0; c < HC; c += 2) {
+                acc0 += ex2_approx(fmaf(v[c], scale_log2, -m));
+                acc1 += ex2_approx(fmaf(v[c + 1], scale_log2, -m));
             }
             l += acc0 + acc1;
         }
-        if (live && !*abort_flag)
-            lse2_out[((size_t)s * nq + (size_t)(j0 + qi)) * q_heads + (size_t)g * G + h] = m + log2f(l);
+        // Merge the two column halves of each row.
+        __shared__ float red_m[128], red_l[128];
+        if (hc == 1) {
+            red_m[row] = m;
+            red_l[row] = l;
+        }
+        tc::named_sync(1, EPI);
+        if (hc == 0 && live && !*abort_flag) {
+            const float m1 = red_m[row], l1 = red_l[row];
+            const float mm = fmaxf(m, m1);
+            const float ll = (m == -INFINITY ? 0.f : l * ex2_approx(m - mm)) +
+                             (m1 == -INFINITY ? 0.f : l1 * ex2_approx(m1 - mm));
+            lse2_out[((size_t)s * nq + (size_t)(j0 + qi)) * q_heads + (size_t)g * G + h] = mm + log2f(ll);
+        }
     }
 
     if (!*abort_flag && warp == 0 && lane == 0)
@@ -300,69 +324,79 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_pool_kernel(
             }
         }
     } else {
-        // Epilogue: thread = TMEM lane = key row of the tile.
-        const int et = tid - 64;
+        // Epilogue: thread = TMEM lane = key row of the tile; the two warps of a
+        // quadrant take queries [0, QB / 2) and [QB / 2, QB).
+        constexpr int QH = QB / 2;       // queries per thread
+        constexpr int NH = QH * G;       // columns per kv head and thread (a multiple of 8)
+        const int et = tid - 64, ew = warp - 2, qh = ew >> 2;
         const int qd = warp & 3;
         const int row = qd * 32 + lane;
         for (int x = et; x < QB * q_heads; x += EPI) {
             const int q = x / q_heads;
             lse_s[x] = q < nrows ? lse2[((size_t)s * nq + (size_t)(j0 + q)) * q_heads + x % q_heads] : 0.f;
         }
-        int64_t nvis[QB];
-        float mass[QB];
+        int64_t nvis[QH];
+        float mass[QH];
 #pragma unroll
-        for (int q = 0; q < QB; ++q) {
-            nvis[q] = q < nrows ? (q_begin + j0 + q) / r : 0;
+        for (int q = 0; q < QH; ++q) {
+            const int qq = qh * QH + q;
+            nvis[q] = qq < nrows ? (q_begin + j0 + qq) / r : 0;
             mass[q] = 0.f;
         }
         tc::named_sync(1, EPI);
         const float inv_h = 1.f / (float)q_heads;
-        bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
             const int buf = t & 1;
-            ok = __all_sync(0xffffffffu, tc::mbar_wait(bar_s(bars.acc_full[buf]), (t >> 1) & 1, abort_flag, WAIT_NS));
+            const bool ok =
+                __all_sync(0xffffffffu, tc::mbar_wait(bar_s(bars.acc_full[buf]), (t >> 1) & 1, abort_flag, WAIT_NS));
             if (!ok) break;
             tc::fence_after();
-            float sum[QB];
+            float sum[QH];
 #pragma unroll
-            for (int q = 0; q < QB; ++q) sum[q] = 0.f;
-            const uint32_t a = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * bstride);
+            for (int q = 0; q < QH; ++q) sum[q] = 0.f;
+            const uint32_t a = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(buf * bstride + qh * NH);
             for (int gg = 0; gg < kv_heads; ++gg) {
-                float v[NG];
+                float v[NH];
+                if constexpr (NH % 16 == 0) {
 #pragma unroll
-                for (int c = 0; c < NG / 16; ++c) tc::tmem_ld16(a + gg * NG + c * 16, v + c * 16);
+                    for (int c = 0; c < NH / 16; ++c) tc::tmem_ld16(a + gg * NG + c * 16, v + c * 16);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NH / 8; ++c) tc::tmem_ld8(a + gg * NG + c * 8, v + c * 8);
+                }
                 tc::tmem_wait_ld();
-                const float* lg = lse_s + gg * G;
+                const float* lg = lse_s + (qh * QH) * q_heads + gg * G;
 #pragma unroll
-                for (int c = 0; c < NG; ++c)
-                    sum[c / G] += ex2_approx(v[c] * scale_log2 - lg[(c / G) * q_heads + c % G]);
+                for (int c = 0; c < NH; ++c)
+                    sum[c / G] += ex2_approx(fmaf(v[c], scale_log2, -lg[(c / G) * q_heads + c % G]));
             }
             tc::fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar_s(bars.acc_empty[buf]));
             const int64_t b = ((int64_t)t * KT + row) / r;
 #pragma unroll
-            for (int q = 0; q < QB; ++q) {
+            for (int q = 0; q < QH; ++q) {
                 const bool vis = b < nvis[q];
                 float val = vis ? sum[q] * inv_h : -INFINITY;
                 for (int o = 1; o < r; o <<= 1) val = fmaxf(val, __shfl_xor_sync(0xffffffffu, val, o));
                 if (vis && (lane & (r - 1)) == 0) {
-                    trow0[(size_t)q * ld + b] = val;
+                    trow0[(size_t)(qh * QH + q) * ld + b] = val;
                     mass[q] += val;
                 }
             }
         }
 #pragma unroll
-        for (int q = 0; q < QB; ++q) {
+        for (int q = 0; q < QH; ++q) {
             const float w = warp_sum(mass[q]);
-            if (lane == 0) atomicAdd(&bars.mass[q], w);
+            if (lane == 0) atomicAdd(&bars.mass[qh * QH + q], w);
         }
         tc::named_sync(1, EPI);
         if (!*abort_flag)
             for (int q = 0; q < nrows; ++q) {
                 const float inv = bars.mass[q] > 0.f ? 1.f / bars.mass[q] : 0.f;
+                const int64_t nv = (q_begin + j0 + q) / r;
                 float* tr = trow0 + (size_t)q * ld;
-                for (int64_t bb = et; bb < ld; bb += EPI) tr[bb] = bb < nvis[q] ? tr[bb] * inv : 0.f;
+                for (int64_t bb = et; bb < ld; bb += EPI) tr[bb] = bb < nv ? tr[bb] * inv : 0.f;
             }
     }
 
