@@ -176,8 +176,8 @@ const char* qsa_last_error(void) { return g_err.c_str(); }
 uint64_t qsa_launch_count(void) { return qsa::g_launches.load(std::memory_order_relaxed); }
 
 qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds) {
-    if (mode < 0 || mode > 1) return fail(QSA_ERR_INVALID_ARG, "fault injection mode %d", mode);
-    if (mode == 1 && !(wait_seconds > 0.0 && wait_seconds <= 10.0))
+    if (mode < 0 || mode > 2) return fail(QSA_ERR_INVALID_ARG, "fault injection mode %d", mode);
+    if (mode != 0 && !(wait_seconds > 0.0 && wait_seconds <= 10.0))
         return fail(QSA_ERR_INVALID_ARG, "fault injection wait of %g s (want (0, 10])", wait_seconds);
     qsa::set_fault_injection(mode, mode ? (uint64_t)(wait_seconds * 1e9) : 0);
     return QSA_OK;

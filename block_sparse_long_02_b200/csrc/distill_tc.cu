@@ -84,7 +84,7 @@ template <int G>
 __global__ void __launch_bounds__(TC_THREADS, 1) distill_lse_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int64_t q_begin, int64_t nq,
     int64_t cap, int batch, int q_heads, int kv_heads, float scale_log2, float* __restrict__ lse2_out,
-    int32_t* __restrict__ status) {
+    int32_t* __restrict__ status, uint64_t wait_ns, int fault_mode) {
     constexpr int QA = 128 / G;  // queries per tile
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_lse_kernel(
             const int kz0 = (int)(s * cap);
             for (int t = 0; t < ntiles; ++t) {
                 const int stg = t % RING;
-                if (!tc::mbar_wait(bar_s(bars.empty[stg]), ((t / RING) & 1) ^ 1, abort_flag, WAIT_NS)) break;
+                if (!tc::mbar_wait(bar_s(bars.empty[stg]), ((t / RING) & 1) ^ 1, abort_flag, wait_ns)) break;
+                if (fault_mode == 2) continue;  // tests of the failure path: the tile never arrives
                 tc::mbar_expect_tx(bar_s(bars.full[stg]), TILE);
                 for (int hf = 0; hf < 2; ++hf)
                     tc::tma_load_3d(sK + stg * TILE + hf * HALF, &tm_k, bar_s(bars.full[stg]), hf * 64, g,
@@ -135,11 +136,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_lse_kernel(
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t ID = tc::idesc_bf16(128, KT);
-            bool ok = tc::mbar_wait(bar_s(bars.q_full), 0, abort_flag, WAIT_NS);
+            bool ok = tc::mbar_wait(bar_s(bars.q_full), 0, abort_flag, wait_ns);
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int stg = t % RING, buf = t & 1;
-                if (!(ok = tc::mbar_wait(bar_s(bars.full[stg]), (t / RING) & 1, abort_flag, WAIT_NS))) break;
-                if (!(ok = tc::mbar_wait(bar_s(bars.acc_empty[buf]), ((t >> 1) & 1) ^ 1, abort_flag, WAIT_NS)))
+                if (!(ok = tc::mbar_wait(bar_s(bars.full[stg]), (t / RING) & 1, abort_flag, wait_ns))) break;
+                if (!(ok = tc::mbar_wait(bar_s(bars.acc_empty[buf]), ((t >> 1) & 1) ^ 1, abort_flag, wait_ns)))
                     break;
                 tc::fence_after();
 #pragma unroll
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_lse_kernel(
         for (int t = 0; t < ntiles; ++t) {
             const int buf = t & 1;
             const bool ok = __all_sync(0xffffffffu,
-                                       tc::mbar_wait(bar_s(bars.acc_full[buf]), (t >> 1) & 1, abort_flag, WAIT_NS));
+                                       tc::mbar_wait(bar_s(bars.acc_full[buf]), (t >> 1) & 1, abort_flag, wait_ns));
             if (!ok) break;
             tc::fence_after();
             constexpr int HC = KT / 2;
@@ -221,7 +222,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_lse_kernel(
 
     if (!*abort_flag && warp == 0 && lane == 0)
         for (int k = 0; k < RING; ++k)  // the last commits on the ring land before shared memory goes away
-            if (issued[k] >= 0) tc::mbar_wait(bar_s(bars.empty[k]), issued[k] & 1, abort_flag, WAIT_NS);
+            if (issued[k] >= 0) tc::mbar_wait(bar_s(bars.empty[k]), issued[k] & 1, abort_flag, wait_ns);
     if (*abort_flag) {
         if (tid == 0) flag_status(status, 6 /* QSA_ERR_TIMEOUT */);
         drain(bars, warp, lane, issued);
@@ -236,7 +237,7 @@ template <int G>
 __global__ void __launch_bounds__(TC_THREADS, 1) distill_pool_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, int64_t q_begin, int64_t nq,
     int64_t cap, int batch, int q_heads, int kv_heads, int r, float scale_log2, const float* __restrict__ lse2,
-    float* __restrict__ target, int64_t ld, int32_t* __restrict__ status) {
+    float* __restrict__ target, int64_t ld, int32_t* __restrict__ status, uint64_t wait_ns, int fault_mode) {
     constexpr int QB = G == 1 ? 16 : 8;  // queries per tile
     constexpr int NG = QB * G;           // columns per kv head (a multiple of 16)
     extern __shared__ uint8_t smem_raw[];
@@ -287,10 +288,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_pool_kernel(
             for (int t = 0, idx = 0; t < ntiles; ++t)
                 for (int gg = 0; gg < kv_heads; ++gg, ++idx) {
                     const int stg = idx % RING;
-                    if (!tc::mbar_wait(bar_s(bars.empty[stg]), ((idx / RING) & 1) ^ 1, abort_flag, WAIT_NS)) {
+                    if (!tc::mbar_wait(bar_s(bars.empty[stg]), ((idx / RING) & 1) ^ 1, abort_flag, wait_ns)) {
                         t = ntiles;
                         break;
                     }
+                    if (fault_mode == 2) continue;  // tests of the failure path: the tile never arrives
                     tc::mbar_expect_tx(bar_s(bars.full[stg]), TILE);
                     for (int hf = 0; hf < 2; ++hf)
                         tc::tma_load_3d(sK + stg * TILE + hf * HALF, &tm_k, bar_s(bars.full[stg]), hf * 64, gg,
@@ -301,14 +303,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_pool_kernel(
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t ID = tc::idesc_bf16(128, NG);
-            bool ok = tc::mbar_wait(bar_s(bars.q_full), 0, abort_flag, WAIT_NS);
+            bool ok = tc::mbar_wait(bar_s(bars.q_full), 0, abort_flag, wait_ns);
             for (int t = 0, idx = 0; ok && t < ntiles; ++t) {
                 const int buf = t & 1;
-                if (!(ok = tc::mbar_wait(bar_s(bars.acc_empty[buf]), ((t >> 1) & 1) ^ 1, abort_flag, WAIT_NS)))
+                if (!(ok = tc::mbar_wait(bar_s(bars.acc_empty[buf]), ((t >> 1) & 1) ^ 1, abort_flag, wait_ns)))
                     break;
                 for (int gg = 0; gg < kv_heads; ++gg, ++idx) {
                     const int stg = idx % RING;
-                    if (!(ok = tc::mbar_wait(bar_s(bars.full[stg]), (idx / RING) & 1, abort_flag, WAIT_NS))) break;
+                    if (!(ok = tc::mbar_wait(bar_s(bars.full[stg]), (idx / RING) & 1, abort_flag, wait_ns))) break;
                     tc::fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_pool_kernel(
         for (int t = 0; t < ntiles; ++t) {
             const int buf = t & 1;
             const bool ok =
-                __all_sync(0xffffffffu, tc::mbar_wait(bar_s(bars.acc_full[buf]), (t >> 1) & 1, abort_flag, WAIT_NS));
+                __all_sync(0xffffffffu, tc::mbar_wait(bar_s(bars.acc_full[buf]), (t >> 1) & 1, abort_flag, wait_ns));
             if (!ok) break;
             tc::fence_after();
             float sum[QH];
@@ -402,7 +404,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) distill_pool_kernel(
 
     if (!*abort_flag && warp == 0 && lane == 0)
         for (int k = 0; k < RING; ++k)  // the last commits on the ring land before shared memory goes away
-            if (issued[k] >= 0) tc::mbar_wait(bar_s(bars.empty[k]), issued[k] & 1, abort_flag, WAIT_NS);
+            if (issued[k] >= 0) tc::mbar_wait(bar_s(bars.empty[k]), issued[k] & 1, abort_flag, wait_ns);
     if (*abort_flag) {
         if (tid == 0) flag_status(status, 6 /* QSA_ERR_TIMEOUT */);
         drain(bars, warp, lane, issued);
@@ -458,8 +460,10 @@ cudaError_t launch_target_tc_g(const LayerDims& L, int batch, const uint16_t* q,
     cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a);
     const int64_t grid_a = ((nq + QA - 1) / QA) * L.kv_heads * batch;
     note_launch();
+    const int fmode = g_fault_mode.load(std::memory_order_relaxed);
+    const uint64_t wait_ns = fmode == 2 ? g_fault_wait_ns.load(std::memory_order_relaxed) : WAIT_NS;
     ka<<<(unsigned)grid_a, TC_THREADS, smem_a, st>>>(tq_a, tk, q_begin, nq, cap, batch, L.q_heads, L.kv_heads, sl2,
-                                                     lse2, status);
+                                                     lse2, status, wait_ns, fmode);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int smem_b = L.kv_heads * QB * G * 256 + RING * TILE + QB * 32 * 4 + (int)sizeof(Bars) + 1024;
@@ -468,7 +472,7 @@ cudaError_t launch_target_tc_g(const LayerDims& L, int batch, const uint16_t* q,
     const int64_t grid_b = ((nq + QB - 1) / QB) * batch;
     note_launch();
     kb<<<(unsigned)grid_b, TC_THREADS, smem_b, st>>>(tq_b, tk, q_begin, nq, cap, batch, L.q_heads, L.kv_heads, L.r,
-                                                     sl2, lse2, target, ld, status);
+                                                     sl2, lse2, target, ld, status, wait_ns, fmode);
     return cudaGetLastError();
 }
 

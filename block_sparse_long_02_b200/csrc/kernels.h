@@ -2,6 +2,7 @@
 // validates arguments and calls these; each returns cudaGetLastError().
 #pragma once
 
+#include <atomic>
 #include <utility>
 
 #include <cuda_runtime.h>
@@ -64,9 +65,13 @@ cudaError_t launch_index_scores(const LayerDims& L, int batch, const uint16_t* q
 bool fused_topk_supported(const LayerDims& L);
 size_t fused_topk_ws_bytes(int batch, int64_t nq, int kB);
 // Tests of the failure path: mode 1 makes the fused indexer's TMA producer
-// withhold the key tiles of each CTA's first unit, so the MMA warp's bounded
-// wait runs out after wait_ns; mode 0 restores normal operation.
+// withhold the key tiles of each CTA's first unit, mode 2 the stage-1 target
+// kernels' producers their key tiles, so the MMA warp's bounded wait runs out
+// after wait_ns; mode 0 restores normal operation. The state (defined with the
+// fused indexer) is read by the kernels' launchers.
 void set_fault_injection(int mode, uint64_t wait_ns);
+extern std::atomic<int> g_fault_mode;
+extern std::atomic<uint64_t> g_fault_wait_ns;
 // Merge of the per-split top-k lists of the fused indexer (topk.cu): for query
 // j of sequence s, the lists of its query tile's `splits` key ranges hold
 // (score bits, block) entries in split_out[(unit * QT + j % QT) * k_B ...],

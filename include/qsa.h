@@ -386,6 +386,10 @@ uint64_t qsa_launch_count(void);
  *           records QSA_ERR_TIMEOUT in the workspace status, drains its own
  *           copies and MMAs, frees its tensor memory and returns; the selection
  *           it leaves is incomplete, and the CUDA context stays usable.
+ *   mode 2: the same for qsa_distill_target: both of its kernels withhold
+ *           every key tile; each CTA records QSA_ERR_TIMEOUT after
+ *           wait_seconds, drains, frees its tensor memory and returns (the
+ *           target it leaves is incomplete).
  * Returns QSA_ERR_INVALID_ARG for another mode or wait. */
 qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds);
 

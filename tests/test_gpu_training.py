@@ -186,3 +186,42 @@ def test_distill_kl_is_zero_at_its_target(qsa):
     qsa.qsa_distill_kl(cfg, 1, 0, 300, t, scores, ld, kl, ds)
     torch.cuda.synchronize()
     assert kl.abs().max().item() < 1e-5 and ds.abs().max().item() < 1e-5
+
+
+def test_target_forced_timeout_is_reported_and_the_context_survives(qsa):
+    """Failure path of the tcgen05 target kernels, without a GPU fault: with
+    fault injection their producers withhold every key tile, the MMA warps'
+    bounded waits run out (0.1 s), each CTA records QSA_ERR_TIMEOUT in the
+    workspace status, drains, frees its tensor memory and returns; the next
+    call is normal and matches the oracle."""
+    import time
+
+    w = synth.Workload(name="tto", n=300, K=64, q_heads=32, kv_heads=4, batch=1, base_seed=0xE3)
+    cfg = qsa.Config.of(w)
+    cap, nq = 304, 300
+    kc = dev_full(w, "k", cap, nq).view(1, cap, cfg.kv_heads, 128)
+    q = dev_full(w, "q", cap, nq)[:, :nq].contiguous()
+    ld = (nq - 1) // cfg.r
+    target = torch.zeros(1, nq, ld, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(qsa.qsa_workspace_size(cfg, qsa.OP_DISTILL_TARGET, 1, cap, nq), dtype=torch.uint8,
+                     device="cuda")
+    qsa.qsa_set_fault_injection(2, 0.1)
+    try:
+        t0 = time.time()
+        qsa.qsa_distill_target(cfg, 1, q, 0, nq, kc, cap, target, ld, ws)
+        torch.cuda.synchronize()
+        elapsed = time.time() - t0
+    finally:
+        qsa.qsa_set_fault_injection(0)
+    assert qsa.qsa_workspace_status(ws) == 6  # QSA_ERR_TIMEOUT (read and cleared)
+    assert elapsed >= 0.1
+    qsa.qsa_distill_target(cfg, 1, q, 0, nq, kc, cap, target, ld, ws)
+    torch.cuda.synchronize()
+    assert qsa.qsa_workspace_status(ws) == 0
+    o = _oracle(cfg)
+    qh = w.host_full("q", 0, nq).reshape(nq, cfg.q_heads, 128)
+    kh = w.host_full("k", 0, nq)
+    got = target.cpu().numpy()[0]
+    for i in (5, 150, nq - 1):
+        ref = o.distill_target(i, qh[i], kh)
+        assert (np.abs(got[i, : i // cfg.r] - ref) <= TARGET_RTOL * ref + TARGET_ATOL).all(), i
