@@ -18,7 +18,7 @@
  * rotated indexer queries are stored as bf16 (round-to-nearest-even, directly
  * from fp64), indexer scores are returned as fp32. Attention is fp64 end to end.
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent:
  *   - order pool -> RMSNorm -> RoPE; RMSNorm is x * (mean x^2 + eps)^-1/2 * w;
  *   - RoPE pairs dim j with dim j + rope_dims/2 for j < rope_dims/2 ("rotate
  *     half"), theta_j = base^(-2j/rope_dims), angle = pos * theta_j;
