@@ -270,3 +270,28 @@ def test_train_32k_full_size():
         got_ds = p["dscores"][0, i, : i // r].cpu().numpy()
         big = np.abs(ref_ds).max() if ref_ds.size else 0.0
         assert (np.abs(got_ds - ref_ds) <= 1e-4 * np.abs(ref_ds) + 1e-6 * big + 1e-9).all(), f"dscores row {i}"
+
+
+def test_decode_offload_full_size():
+    """decode_b8_n256k with the K/V caches in pinned host memory behind a
+    16384-block hot cache (the configuration bench.py --offload 16384 times),
+    through bench's own Bench: the step's outputs equal the all-HBM step's bit
+    for bit, on a first step (every block misses) and on the same step again
+    (the selected blocks are then hot), and the appended rows reach host memory."""
+    import bench
+
+    w = synth.WORKLOADS["decode_b8_n256k"]
+    dev = torch.device("cuda", 0)
+    ha = bench.Bench(w, dev)
+    hb = bench.Bench(w, dev, offload=16384)
+    d_a, d_b = ha.dec[0], hb.dec[0]
+    for it in range(2):
+        ha.L.decode_step(d_a["pos"], d_a["q"], d_a["k"], d_a["v"], d_a["idx_q"], d_a["idx_k"], d_a["out"])
+        hb.L.decode_step_offload(d_b["pos"], d_b["q"], d_b["k"], d_b["v"], d_b["idx_q"], d_b["idx_k"], d_b["out"])
+        torch.cuda.synchronize()
+        assert torch.equal(d_a["out"], d_b["out"]), it
+        if it == 0:
+            assert (hb.L.hot_tags[:, :16384] >= 0).sum().item() > 0  # the first step installed blocks
+    p = w.n
+    assert torch.equal(hb.L.host_k[:, p].cuda(), ha.L.k_cache[:, p])
+    assert torch.equal(hb.L.host_v[:, p].cuda(), ha.L.v_cache[:, p])
