@@ -295,3 +295,42 @@ def test_decode_offload_full_size():
     p = w.n
     assert torch.equal(hb.L.host_k[:, p].cuda(), ha.L.k_cache[:, p])
     assert torch.equal(hb.L.host_v[:, p].cuda(), ha.L.v_cache[:, p])
+
+
+def test_decode_fp8_full_size():
+    """decode_b8_n256k on fp8 caches (the configuration bench.py --kv fp8
+    times), through bench's own Bench: for sampled sequences, the appended
+    rows are quantized exactly as the oracle does, the selection is the
+    oracle's on the fp8 pooled keys (near-ties aside) and the output matches
+    the oracle's fp8-cache attention."""
+    import bench
+    from gpu_util import SCORE_COND_ATOL, SCORE_RTOL, f32
+
+    w = synth.WORKLOADS["decode_b8_n256k"]
+    b = bench.Bench(w, torch.device("cuda", 0), kv="fp8")
+    cfg, L, d = b.cfg, b.L, b.dec[0]
+    sel = torch.empty(w.batch, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(w.batch, dtype=torch.int32, device="cuda")
+    L.decode_step_q8(d["pos"], d["q"], d["k"], d["v"], d["idx_q"], d["idx_k"], d["out"], sel, nsel)
+    torch.cuda.synchronize()
+    o = _oracle(w)
+    p = w.n
+    nvis = p // cfg.r
+    g_out, g_sel, g_n = d["out"].float().cpu().numpy(), sel.cpu().numpy(), nsel.cpu().numpy()
+    for s in (0, 5):
+        k8, v8 = L.k8[s].cpu().numpy(), L.v8[s].cpu().numpy()
+        ks, vs = L.ks[s].cpu().numpy(), L.vs[s].cpu().numpy()
+        p8, ps = L.pooled8[s].cpu().numpy(), L.pscale[s].cpu().numpy()
+        for name, c8, sc in (("k", k8, ks), ("v", v8, vs)):  # the appended row
+            row = w.host_rows(name, s, [p]).reshape(cfg.kv_heads, 128)
+            rc, rs = o.quant_rows(row)
+            assert np.array_equal(rs, sc[p]) and np.array_equal(rc, c8[p]), (s, name)
+        qrot = o.rotate_query(w.host_rows("idx_q", s, [p]).reshape(4, 128), p)
+        ref = o.scores_q8(qrot, p8, ps, nvis)
+        kd = o.dequant(p8[:nvis], ps[:nvis])
+        tol = SCORE_RTOL * np.abs(ref.astype(np.float64)) + SCORE_COND_ATOL * (
+            np.abs(kd) @ np.abs(f32(qrot).astype(np.float64)).T).sum(axis=1)
+        check_selection(g_sel[s], g_n[s], ref, tol, o.k_blocks, f"s{s}")
+        toks = o.token_set(g_sel[s, : g_n[s]], p)
+        ref_out, _ = o.attention_q8(w.host_rows("q", s, [p])[0], k8, ks, v8, vs, toks)
+        check_attention(g_out[s], ref_out.reshape(cfg.q_heads, 128), f"s{s}")
