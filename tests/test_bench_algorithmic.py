@@ -45,3 +45,22 @@ def test_fp8_caches_count_code_rows_and_scales():
     assert b["attn_gather_bytes"] == rows * (w.head_dim + 4)
     assert b["quantize_bytes"] == w.n * w.kv_heads * 2 * (w.head_dim * 3 + 4) and a["quantize_bytes"] == 0
     assert b["index_flops"] == a["index_flops"] and b["attn_flops"] == a["attn_flops"]
+
+
+def test_training_counts_match_the_closed_forms():
+    w = dataclasses.replace(synth.WORKLOADS["train_n32k"], n=2048)
+    a = bench.algorithmic(w)
+    n, r, d, H, hk = w.n, w.r, w.head_dim, w.q_heads, w.kv_heads
+    tokens = sum(r * min(w.k_blocks, i // r) + i % r + 1 for i in range(n))
+    # the five products of the gradient over the forward's token sets
+    assert a["bwd_flops"] == 5 * tokens * H * d * 2
+    # the forward's gather, an fp32 dK and dV row per gathered (token, kv head), q / dout / out read, dq written
+    assert a["bwd_bytes"] == tokens * hk * (d * 4 + d * 8) + n * H * d * (6 + 4)
+    # the target: logits over tokens <= i (log-sum-exp), then over the visible blocks' tokens
+    assert a["target_flops"] == sum(i + 1 + r * (i // r) for i in range(n)) * H * d * 2
+    ld = (n - 1) // r
+    assert a["scores_bytes"] == n * (ld * 4 + w.idx_heads * w.idx_dim * 2)
+    assert a["kl_bytes"] == sum(i // r for i in range(n)) * 8 + n * ld * 4 + n * 4
+    # a workload without training counts none of it
+    b = bench.algorithmic(dataclasses.replace(w, train=False))
+    assert b["bwd_bytes"] == b["bwd_flops"] == b["target_flops"] == b["scores_bytes"] == b["kl_bytes"] == 0
