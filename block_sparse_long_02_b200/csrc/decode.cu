@@ -577,13 +577,17 @@ int decode_select_ctas(int batch) {
 }
 
 // One wave: as many CTAs as fit on the GPU at once, split over the batch.
-int decode_score_ctas(int batch) {
+// CTAs per sequence: one wave of the variant that runs (the bf16 and fp8
+// variants use different register counts, so their occupancies differ).
+int decode_score_ctas(int batch, bool q8) {
     int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<true>, DS_THREADS, 0) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
+    const cudaError_t e = q8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<true>,
+                                                                             DS_THREADS, 0)
+                             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<false>,
+                                                                             DS_THREADS, 0);
+    if (e != cudaSuccess || per_sm < 1) per_sm = 1;
     return std::max(1, per_sm * sms / std::max(batch, 1));
 }
 
@@ -592,7 +596,7 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,
                                 int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
                                 int32_t* status, const Q8Caches* q8, const HotCache* hot, cudaStream_t st) {
-    const dim3 grid((unsigned)decode_score_ctas(batch), (unsigned)batch);
+    const dim3 grid((unsigned)decode_score_ctas(batch, q8 != nullptr), (unsigned)batch);
     if (q8)
         return launch_pdl(decode_score_kernel<true>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,
                           idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist,
