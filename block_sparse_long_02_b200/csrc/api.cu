@@ -350,6 +350,8 @@ qsa_status qsa_distill_target(const qsa_config* cfg, int32_t batch, const qsa_bf
         return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
     if (nq > 0 && ld < (q_begin + nq - 1) / L.r)
         return fail(QSA_ERR_INVALID_ARG, "ld=%lld < floor((q_begin + nq - 1) / r)", (long long)ld);
+    if ((int64_t)batch * cap >= INT32_MAX || (int64_t)batch * nq >= INT32_MAX)  // 32-bit TMA row coordinates
+        return fail(QSA_ERR_UNSUPPORTED, "batch x cap and batch x nq must stay below 2^31");
     if (nq == 0) return QSA_OK;
     const size_t need = qsa::distill_target_ws_bytes(batch, nq, L.q_heads);
     if (!ws || !aligned16(ws) || ws_bytes < need)

@@ -208,7 +208,8 @@ qsa_status qsa_sparse_attention_backward(const qsa_config* cfg, int32_t batch, c
  * Logits on the tensor cores (bf16 in, fp32 accumulate), softmax in fp32: two
  * passes over the keys (every head's log-sum-exp, then the probabilities).
  * Supported: q_heads <= 32, q_heads/kv_heads in {1, 2, 4, 8, 16}, r in
- * {1, 2, 4, 8, 16}; else QSA_ERR_UNSUPPORTED. */
+ * {1, 2, 4, 8, 16}, batch x cap and batch x nq below 2^31; else
+ * QSA_ERR_UNSUPPORTED. */
 qsa_status qsa_distill_target(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin, int64_t nq,
                               const qsa_bf16* k_cache, int64_t cap, float* target, int64_t ld, void* ws,
                               size_t ws_bytes, qsa_stream stream);

@@ -122,6 +122,7 @@ def test_training_entry_points_validate_before_launching(qsa):
     assert tgt(ctypes.byref(qsa.Config(r=3).c()), 1, p, 0, 8, p, 64, p, 16, p, big, None) == 2  # r not in {1..16}
     assert tgt(ctypes.byref(qsa.Config(q_heads=64, kv_heads=4).c()), 1, p, 0, 8, p, 64, p, 16, p, big, None) == 2
     assert tgt(cfg, 1, p, 0, 64, p, 64, p, 16, p, 256, None) == 3  # workspace without the lse rows
+    assert tgt(cfg, 4096, p, 0, 64, p, 1 << 20, p, 16, p, big, None) == 2  # batch x cap past 32-bit rows
     assert tgt(cfg, 1, p, 0, 0, p, 64, p, 0, None, 0, None) == 0
     assert qsa.qsa_workspace_size(qsa.Config(), qsa.OP_DISTILL_TARGET, 2, 64, 10) == 256 + 2 * 10 * 32 * 4
     kl = lib.qsa_distill_kl
