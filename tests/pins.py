@@ -557,6 +557,72 @@ def pin_distill_target_closed_forms(make):
     assert o.distill_target(3, _bits(qf), _bits(k)).size == 0
 
 
+def pin_distill_target_other_block_sizes(make):
+    """For r = 1 and r = 16 as for r = 4: identical keys give a uniform target
+    over the floor(i/r) visible blocks; with r = 1 and one dominant token j
+    below i, the target is the one-hot vector of block j."""
+    rng = np.random.default_rng(36)
+    for r in (1, 16):
+        o = make(r=r, K=64, q_heads=4, kv_heads=2, head_dim=16)
+        c = o.cfg
+        i = 70
+        kc = np.full((i + 1, c.kv_heads, c.head_dim), _bits(np.float32(0.25)), dtype=np.uint16)
+        q = _bits(rng.standard_normal((c.q_heads, c.head_dim)).astype(np.float32))
+        t = o.distill_target(i, q, kc)
+        assert t.size == i // r and np.abs(t - 1.0 / t.size).max() < 1e-15, r
+    o = make(r=1, K=64, q_heads=4, kv_heads=2, head_dim=16)
+    c = o.cfg
+    i, j = 40, 17
+    k = np.zeros((i + 1, c.kv_heads, c.head_dim), dtype=np.float32)
+    k[j, :, 0] = 32.0
+    qf = np.zeros((c.q_heads, c.head_dim), dtype=np.float32)
+    qf[:, 0] = 32.0  # logit 256 for token j, 0 elsewhere
+    t = o.distill_target(i, _bits(qf), _bits(k))
+    want = np.zeros(i)
+    want[j] = 1.0
+    assert np.abs(t - want).max() < 1e-12
+
+
+def pin_attention_backward_properties(make):
+    """The gradient is linear in dout (doubling dout doubles dq, dk, dv; a sum
+    of two upstream gradients gives the sum of the gradients), and the rows of
+    dS sum to zero, so sum_t dk_t = 0 for every kv head (the softmax is
+    invariant to a shift of a head's logits)."""
+    o = _f3_oracle(make, q_heads=8, kv_heads=2, head_dim=16)
+    c = o.cfg
+    rng = np.random.default_rng(37)
+    ntok = 9
+    q = rng.standard_normal((c.q_heads, c.head_dim))
+    kt = rng.standard_normal((ntok, c.kv_heads, c.head_dim))
+    vt = rng.standard_normal((ntok, c.kv_heads, c.head_dim))
+    g1 = rng.standard_normal((c.q_heads, c.head_dim))
+    g2 = rng.standard_normal((c.q_heads, c.head_dim))
+    a = o.attention_backward_f64(q, kt, vt, g1)
+    b = o.attention_backward_f64(q, kt, vt, g2)
+    ab = o.attention_backward_f64(q, kt, vt, g1 + g2)
+    a2 = o.attention_backward_f64(q, kt, vt, 2.0 * g1)
+    for x, y, xy, x2 in zip(a, b, ab, a2):
+        assert np.abs(xy - (x + y)).max() < 1e-12 and np.abs(x2 - 2.0 * x).max() < 1e-12
+    assert np.abs(a[1].sum(axis=0)).max() < 1e-12
+
+
+def pin_distill_kl_properties(make):
+    """KL >= 0 on random targets and scores; its gradient sums to zero over the
+    blocks (a normalised target); adding a constant to every score changes
+    neither the KL nor its gradient."""
+    o = _f3_oracle(make)
+    rng = np.random.default_rng(38)
+    for _ in range(20):
+        n = int(rng.integers(1, 60))
+        t = rng.random(n)
+        t /= t.sum()
+        s = (np.round(rng.standard_normal(n) * 4 * 256) / 256).astype(np.float32)  # + 8 stays exact
+        kl, ds = o.distill_kl(t, s)
+        assert kl >= -1e-12 and abs(ds.sum()) < 1e-12
+        kl2, ds2 = o.distill_kl(t, s + np.float32(8.0))
+        assert abs(kl2 - kl) < 1e-9 and np.abs(ds2 - ds).max() < 1e-9
+
+
 def pin_distill_kl_library_and_gradient(make):
     """KL(t || softmax(s)) equals scipy's relative entropy (zero target entries
     included); it is 0 with a zero gradient at s = log t + const; its gradient
