@@ -15,6 +15,8 @@ def test_host_draws_are_reproducible_and_row_addressable():
     assert np.array_equal(rows[2], a[7 * 512:8 * 512])
     assert not np.array_equal(synth.fill_host(124, 4, 0, 64), a[:64])
     assert not np.array_equal(synth.fill_host(123, 5, 0, 64), a[:64])
+    # every tensor of a workload has its own stream (distinct ids)
+    assert len(set(synth.TENSOR_IDS.values())) == len(synth.TENSOR_IDS)
 
 
 def test_host_draws_look_standard_normal():
@@ -45,7 +47,7 @@ def test_device_generator_matches_host_bit_for_bit():
     import torch
 
     w = synth.WORKLOADS["tiny_prefill_n256"]
-    for name in ("idx_q", "idx_k", "q", "k", "v"):
+    for name in ("idx_q", "idx_k", "q", "k", "v", "dout"):
         t = torch.zeros(1, w.total, w.row_len(name), dtype=torch.bfloat16, device="cuda")
         w.device_fill(name, t)
         torch.cuda.synchronize()
