@@ -727,9 +727,12 @@ def cpu_baseline(w, rows=64, dec=2, blocks=65536):
     model, ncpu = host_cpu()
     return {"value": round(tokens / t, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "cpu_model": model, "host_cores": ncpu,
-            "sample": (f"{parts.get('fit', {}).get('rows', 0)} prefill rows stratified over [q_begin,n) fitted by "
-                       f"t(i)=a+b*floor(i/r) and extrapolated over all n; key pooling timed on {blocks} blocks "
-                       f"and scaled; {dec} decode positions, scaled to {w.decode_steps} steps"),
+            "sample": (f"{parts.get('fit', {}).get('rows', 0)} prefill rows stratified over [q_begin,n)"
+                       + (" (each also running the attention gradient, the stage-1 target and the KL)"
+                          if w.train else "")
+                       + f" fitted by t(i)=a+b*floor(i/r) and extrapolated over all n; key pooling timed on "
+                       f"{blocks} blocks and scaled"
+                       + (f"; {dec} decode positions, scaled to {w.decode_steps} steps" if w.decode_steps else "")),
             "extrapolated_step_s": round(t, 3), "parts": {k: (round(v, 4) if isinstance(v, float) else v)
                                                         for k, v in parts.items()}}
 
