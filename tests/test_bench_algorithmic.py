@@ -64,3 +64,23 @@ def test_training_counts_match_the_closed_forms():
     # a workload without training counts none of it
     b = bench.algorithmic(dataclasses.replace(w, train=False))
     assert b["bwd_bytes"] == b["bwd_flops"] == b["target_flops"] == b["scores_bytes"] == b["kl_bytes"] == 0
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the oracle on the host) prints one JSON line
+    with the contract's keys, the reference marker, a cpu_baseline that
+    describes the run and an e2e object with zero copied bytes."""
+    import json
+    import subprocess
+
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny_prefill_n256", "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
+                         timeout=600, check=True).stdout.strip().splitlines()
+    d = json.loads(out[-1])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["config"]["workload"] == "tiny_prefill_n256"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["value"] == d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
