@@ -129,3 +129,29 @@ def test_training_entry_points_validate_before_launching(qsa):
     assert kl(cfg, 1, 0, 64, p, p, 8, p, None, None) == 1  # ld too small
     assert kl(cfg, 1, 0, 64, p, p, 16, ctypes.c_void_p(4098), None, None) == 1  # kl misaligned
     assert kl(cfg, 1, 0, 0, p, p, 0, p, None, None) == 0
+
+
+def test_offload_decode_validates_before_launching(qsa):
+    """qsa_decode_step_offload rejects a bad hot-cache size and host caches that
+    are not pinned, mapped host memory (fake, aligned, never dereferenced
+    pointers), with a status and no launch."""
+    lib = ctypes.CDLL(qsa.LIB_PATH)
+    f = lib.qsa_decode_step_offload
+    f.restype = ctypes.c_int
+    f.argtypes = qsa._SIGS["qsa_decode_step_offload"]
+    cfg = ctypes.byref(qsa.Config().c())
+    p = ctypes.c_void_p(4096)
+    lib.qsa_last_error.restype = ctypes.c_char_p
+    lib.qsa_launch_count.restype = ctypes.c_uint64
+    n0 = lib.qsa_launch_count()
+
+    def call(hot_blocks):
+        # cfg, batch, pos, q, k, v, idx_q, idx_k, host_k, host_v, hot_k, hot_v, hot_tags, hot_blocks,
+        # idx_k_cache, pooled, cap, rms_w, out, sel, nsel, ws, ws_bytes, stream
+        return f(cfg, 1, p, p, p, p, p, p, p, p, p, p, p, hot_blocks, p, p, 4096, None, p, None, None, p,
+                 1 << 20, None)
+
+    assert call(0) == 1 and call(2 ** 31 - 1) == 1  # hot_blocks outside [1, INT32_MAX)
+    assert call(64) == 1                            # the host caches are not mapped host memory
+    assert b"host" in lib.qsa_last_error()
+    assert lib.qsa_launch_count() == n0
