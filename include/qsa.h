@@ -204,7 +204,9 @@ qsa_status qsa_sparse_attention_backward(const qsa_config* cfg, int32_t batch, c
  *          attention takes it); k_cache: [batch][cap][kv_heads][head_dim].
  * target:  [batch][nq][ld] fp32; ld >= floor((q_begin + nq - 1) / r).
  * ws:      qsa_workspace_size(QSA_OP_DISTILL_TARGET, batch, cap, nq) bytes (the
- *          heads' log-sum-exps); a smaller one returns QSA_ERR_WORKSPACE.
+ *          heads' log-sum-exps); a smaller one returns QSA_ERR_WORKSPACE. A
+ *          bounded device wait that runs out records QSA_ERR_TIMEOUT in its
+ *          status word (qsa_workspace_status); the target is then incomplete.
  * Logits on the tensor cores (bf16 in, fp32 accumulate), softmax in fp32: two
  * passes over the keys (every head's log-sum-exp, then the probabilities).
  * Supported: q_heads <= 32, q_heads/kv_heads in {1, 2, 4, 8, 16}, r in
