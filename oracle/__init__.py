@@ -97,6 +97,7 @@ class Oracle:
         L.qsa_oracle_distill_target.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
         L.qsa_oracle_distill_kl.restype = ctypes.c_double
         L.qsa_oracle_distill_kl.argtypes = [vp, vp, ctypes.c_int64, vp]
+        L.qsa_oracle_round_bf16.argtypes = [vp, ctypes.c_int64, vp]
 
     @classmethod
     def for_workload(cls, w, **kw) -> "Oracle":
@@ -108,6 +109,13 @@ class Oracle:
     @property
     def k_blocks(self) -> int:
         return int(self.lib.qsa_oracle_k_blocks(self._c))
+
+    def round_bf16(self, x) -> np.ndarray:
+        """The storage rounding (fp64 -> bf16 bits, nearest even)."""
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        out = np.empty(x.shape, dtype=np.uint16)
+        self.lib.qsa_oracle_round_bf16(_p(x), x.size, _p(out))
+        return out
 
     def rope(self, x: np.ndarray, pos: int) -> np.ndarray:
         x = np.ascontiguousarray(x, dtype=np.float64)

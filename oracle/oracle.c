@@ -53,21 +53,34 @@ static double bf(uint16_t h) {
     return (double)f;
 }
 
-/* fp64 -> bf16 bits, round to nearest, ties to even, in one step: keep the top
- * 7 explicit significand bits of the double, then narrow (exact) to fp32. */
+/* fp64 -> bf16 bits: the bf16 value nearest to x, ties to the even significand
+ * (IEEE round-to-nearest-even), in one rounding from the exact value.
+ * bf16 keeps 8 significant bits with fp32's exponent range: a normal value in
+ * [2^e, 2^(e+1)) sits on the grid 2^(e-7); below 2^-126 the grid is the
+ * subnormal step 2^-133. A result beyond the largest finite bf16
+ * ((2 - 2^-7) * 2^127) is an infinity. */
 static uint16_t to_bf16(double x) {
-    uint64_t u;
-    memcpy(&u, &x, 8);
-    const uint64_t drop = 45; /* 52 - 7 */
-    uint64_t lsb = (u >> drop) & 1u;
-    u += ((1ull << (drop - 1)) - 1u) + lsb;
-    u &= ~((1ull << drop) - 1u);
-    double y;
-    memcpy(&y, &u, 8);
-    float f = (float)y;
+    const uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    if (isnan(x)) return (uint16_t)(sign | 0x7FC0u);
+    const double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e); /* a = m * 2^e, m in [0.5, 1): a lies in [2^(e-1), 2^e) */
+    const int q = (e - 1 >= -126) ? (e - 1) - 7 : -133;
+    const double k = ldexp(a, -q);        /* exact: a scaled by a power of two */
+    const double kr = nearbyint(k);       /* nearest integer, ties to even */
+    const double y = ldexp(kr, q);        /* exact: at most 9 significant bits */
+    if (y > ldexp(255.0, 120)) return (uint16_t)(sign | 0x7F80u);
+    const float f = (float)y; /* exact: y is on the bf16 grid, inside fp32's range */
     uint32_t v;
     memcpy(&v, &f, 4);
-    return (uint16_t)(v >> 16);
+    return (uint16_t)(sign | ((v >> 16) & 0x7FFFu));
+}
+
+/* The storage rounding above, exposed for the pins. */
+void qsa_oracle_round_bf16(const double* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = to_bf16(x[i]);
 }
 
 int64_t qsa_oracle_k_blocks(const qsa_oracle_cfg* c) {

@@ -20,12 +20,37 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
+_BF16_TABLE = None
+
+
+def _bf16_table():
+    """Every non-negative bf16 pattern 0x0000 .. 0x7F80 (+inf) and its value,
+    increasing. The value used for +inf is 2^128, the grid point one step
+    past the largest finite bf16, so that rounding to it means overflow."""
+    global _BF16_TABLE
+    if _BF16_TABLE is None:
+        pat = np.arange(0x7F81, dtype=np.uint32)
+        val = (pat << np.uint32(16)).view(np.float32).astype(np.float64)
+        val[-1] = 2.0 ** 128
+        _BF16_TABLE = (pat.astype(np.uint16), val)
+    return _BF16_TABLE
+
+
 def f64_to_bf16(x: np.ndarray) -> np.ndarray:
-    """Round fp64 directly to bf16 bits (nearest, ties to even)."""
-    u = np.ascontiguousarray(x, dtype=np.float64).view(np.uint64)
-    lsb = (u >> np.uint64(45)) & np.uint64(1)
-    u = (u + np.uint64((1 << 44) - 1) + lsb) & ~np.uint64((1 << 45) - 1)
-    return (u.view(np.float64).astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    """Round fp64 to bf16 bits as the nearest bf16 value, ties to the even
+    pattern: a search over the table of all bf16 values (no bit tricks)."""
+    x = np.asarray(x, dtype=np.float64)
+    pat, val = _bf16_table()
+    a = np.abs(x).ravel()
+    hi = np.clip(np.searchsorted(val, a, side="left"), 0, val.size - 1)
+    lo = np.clip(hi - 1, 0, None)
+    mid = val[lo] + val[hi]          # exact: two 8-bit significands
+    twice = 2.0 * a                  # exact
+    pick = np.where(twice < mid, lo, np.where(twice > mid, hi, np.where(pat[lo] % 2 == 0, lo, hi)))
+    pick = np.where(val[hi] == a, hi, pick)
+    out = pat[pick].astype(np.uint16)
+    out = np.where(np.signbit(x.ravel()), out | np.uint16(0x8000), out).astype(np.uint16)
+    return out.reshape(x.shape)
 
 
 def rope_complex(x: np.ndarray, pos: np.ndarray, rope_dims: int, base: float) -> np.ndarray:

@@ -57,6 +57,55 @@ def pin_budget_golden(make):
     assert o.select(s).size == 512
 
 
+# ----------------------------------------------------------------------------- bf16 storage
+def _f32_patterns_to_f64(bits32):
+    with np.errstate(invalid="ignore"):  # NaN patterns are dropped by the caller
+        return np.asarray(bits32, dtype=np.uint32).view(np.float32).astype(np.float64)
+
+
+def pin_bf16_rounding(make):
+    """Pooled keys and rotated indexer queries are stored as bf16, rounded once
+    to nearest with ties to even. Inputs that fp32 holds exactly are checked
+    against torch's float32 -> bfloat16 conversion (a library rounding);
+    every input, fp32-exact or not, against a nearest-value search over the
+    table of all bf16 values. Cases: exact halfway ties with odd and even last
+    kept bits, ties and near-ties that carry into the exponent, signed zeros,
+    the subnormal range, the largest finite values and the overflow edge, and
+    fp64 values one hair off a tie (fp32 would first round them onto it)."""
+    import torch
+
+    o = make()
+    rng = np.random.default_rng(16)
+    pats = [rng.integers(0, 2 ** 32, 60000, dtype=np.uint64).astype(np.uint32)]
+    h = rng.integers(0, 0x7F7F, 4000).astype(np.uint32)
+    for low in (0x8000, 0x7FFF, 0x8001, 0x0000, 0xFFFF):
+        pats.append((h << 16) | low)
+    pats.append(np.array([0x3F7F8000, 0x3F7FFFFF, 0x3FFF8000, 0x3F808000, 0x3F818000,  # carries / ties
+                          0x00000000, 0x80000000, 0x00008000, 0x00018000, 0x00017FFF,   # zeros, subnormals
+                          0x00000001, 0x007F8000, 0x007FFFFF, 0x00800000,
+                          0x7F7F7FFF, 0x7F7F8000, 0x7F7EFFFF, 0x7F7F0000, 0x7F7FFFFF], dtype=np.uint32))
+    p32 = np.concatenate(pats)
+    p32 = np.concatenate([p32, p32 | np.uint32(0x80000000)])
+    x32 = _f32_patterns_to_f64(p32)
+    x32 = x32[np.isfinite(x32)]
+    got = o.round_bf16(x32)
+    lib = torch.from_numpy(x32.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    bad = np.nonzero(got != lib)[0]
+    assert bad.size == 0, (x32[bad[:4]], got[bad[:4]], lib[bad[:4]])
+    assert np.array_equal(got, bfm.f64_to_bf16(x32))
+    # fp64 inputs: random magnitudes over the whole range, and ties shifted by
+    # less than fp32's last bit.
+    mag = rng.uniform(-140.0, 128.5, 40000)
+    x64 = rng.choice([-1.0, 1.0], mag.size) * np.exp2(mag) * (1.0 + rng.random(mag.size) * 2.0 ** -30)
+    ties = _f32_patterns_to_f64((h << 16) | np.uint32(0x8000))
+    x64 = np.concatenate([x64, ties * (1 + 2.0 ** -40), ties * (1 - 2.0 ** -40), -ties * (1 + 2.0 ** -40)])
+    x64 = x64[np.isfinite(x64)]
+    assert np.array_equal(o.round_bf16(x64), bfm.f64_to_bf16(x64))
+    # a tie nudged up rounds up although its fp32 rounding is the tie itself
+    t = float(_f32_patterns_to_f64(np.array([0x3F808000], dtype=np.uint32))[0]) * (1 + 2.0 ** -40)
+    assert int(o.round_bf16(np.array([t]))[0]) == 0x3F81
+
+
 # ----------------------------------------------------------------------------- RoPE
 def pin_rope_textbook(make):
     """RoPE = complex rotation z_j * e^{i pos theta_j}, theta_j = base^(-2j/64),

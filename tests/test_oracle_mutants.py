@@ -12,6 +12,8 @@ import pins
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
 MUTANTS = {
+    "bf16_truncation": ("const double kr = nearbyint(k);", "const double kr = trunc(k);"),
+    "bf16_ties_away_from_zero": ("const double kr = nearbyint(k);", "const double kr = round(k);"),
     "rope_sign": ("out[j] = x[j] * c - x[j + half] * s;", "out[j] = x[j] * c + x[j + half] * s;"),
     "rope_freq_full_dim": ("-2.0 * (double)j / (double)rope_dims", "-2.0 * (double)j / (double)dim"),
     "rope_interleaved_pairs": ("out[j] = x[j] * c - x[j + half] * s;\n        out[j + half] = x[j] * s + x[j + half] * c;",
