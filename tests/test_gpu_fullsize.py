@@ -275,9 +275,10 @@ def test_train_32k_full_size():
 def test_decode_offload_full_size():
     """decode_b8_n256k with the K/V caches in pinned host memory behind a
     16384-block hot cache (the configuration bench.py --offload 16384 times),
-    through bench's own Bench: the step's outputs equal the all-HBM step's bit
-    for bit, on a first step (every block misses) and on the same step again
-    (the selected blocks are then hot), and the appended rows reach host memory."""
+    through bench's own Bench: on a first step (every block misses) and on the
+    same step again (the selected blocks are then hot), the offloaded step's
+    selection and output match the oracle on sampled sequences, and equal the
+    all-HBM step's bit for bit; the appended rows reach host memory."""
     import bench
 
     w = synth.WORKLOADS["decode_b8_n256k"]
@@ -285,13 +286,21 @@ def test_decode_offload_full_size():
     ha = bench.Bench(w, dev)
     hb = bench.Bench(w, dev, offload=16384)
     d_a, d_b = ha.dec[0], hb.dec[0]
+    cfg = hb.cfg
+    o = _oracle(w)
+    sels = [torch.empty(w.batch, cfg.k_blocks, dtype=torch.int32, device="cuda") for _ in range(2)]
+    nsels = [torch.empty(w.batch, dtype=torch.int32, device="cuda") for _ in range(2)]
     for it in range(2):
-        ha.L.decode_step(d_a["pos"], d_a["q"], d_a["k"], d_a["v"], d_a["idx_q"], d_a["idx_k"], d_a["out"])
-        hb.L.decode_step_offload(d_b["pos"], d_b["q"], d_b["k"], d_b["v"], d_b["idx_q"], d_b["idx_k"], d_b["out"])
+        ha.L.decode_step(d_a["pos"], d_a["q"], d_a["k"], d_a["v"], d_a["idx_q"], d_a["idx_k"], d_a["out"],
+                         sels[0], nsels[0])
+        hb.L.decode_step_offload(d_b["pos"], d_b["q"], d_b["k"], d_b["v"], d_b["idx_q"], d_b["idx_k"], d_b["out"],
+                                 sels[1], nsels[1])
         torch.cuda.synchronize()
         assert torch.equal(d_a["out"], d_b["out"]), it
+        assert torch.equal(sels[0], sels[1]) and torch.equal(nsels[0], nsels[1]), it
         if it == 0:
             assert (hb.L.hot_tags[:, :16384] >= 0).sum().item() > 0  # the first step installed blocks
+        _check_decode_step(w, o, hb.L, 0, d_b["out"], sels[1], nsels[1], (0, 3, 7))
     p = w.n
     assert torch.equal(hb.L.host_k[:, p].cuda(), ha.L.k_cache[:, p])
     assert torch.equal(hb.L.host_v[:, p].cuda(), ha.L.v_cache[:, p])

@@ -374,10 +374,14 @@ def test_fused_topk_with_buffer_compaction(qsa, n, K):
         assert b in set(res["sel"][0, p, : res["nsel"][0, p]].tolist()), (b, p)
 
 
-def test_fused_topk_exact_ties(qsa):
+@pytest.mark.parametrize("n", [6000, 36000])
+def test_fused_topk_exact_ties(qsa, n):
     """rope_dims = 0 and a periodic key pattern make many pooled keys identical:
-    exactly equal scores must resolve to the lower block index, as in the oracle."""
-    n, period = 6000, 37
+    exactly equal scores must resolve to the lower block index, as in the oracle.
+    At n = 36000 a query sees up to 71 key tiles, so the sweep visits the sample
+    tiles 0, 16, 32, ... before tiles 1-15: equal-score blocks of lower index
+    then arrive after higher-index ones and must still win."""
+    period = 37
     w = synth.Workload(name="t", n=n, K=256, rope_dims=0, q_heads=8, kv_heads=2, base_seed=0xB7)
     cfg, L = _layer(qsa, w, n)
     _fill_caches(w, L, n)
@@ -398,7 +402,8 @@ def test_fused_topk_exact_ties(qsa):
     assert np.array_equal(pooled, bits(L.pooled)[0])
     idx_q = w.host_full("idx_q", 0).reshape(n, 4, 128)
     g_sel, g_n = sel.cpu().numpy()[0], nsel.cpu().numpy()[0]
-    for i in [300, 1999, 4000, 5555, 5999]:
+    rows = [300, 1999, 4000, 5555, 5999] + ([9000, 17777, 26000, 35999] if n > 6000 else [])
+    for i in rows:
         ref = o.row(i, idx_q[i], pooled)
         # Scores are bit-identical between equal blocks on both sides, so the set
         # must match exactly (near-ties with other blocks are still tolerated).
@@ -683,7 +688,8 @@ def test_decode_steps_with_fp8_caches_match_oracle(qsa):
 def test_decode_offload_matches_hbm_decode_bit_for_bit(qsa, n0, S, H, batch):
     """K/V caches in pinned host memory with a small direct-mapped HBM hot
     cache (a prime number of slots, so selected blocks collide): every step's
-    output and selection equal the all-HBM decode's bit for bit; the appended
+    selection and output match the oracle on sampled sequences and equal the
+    all-HBM decode's bit for bit; the appended
     rows reach host memory; every tagged hot slot holds a copy of its block.
     The same query for every step makes later steps hit blocks installed by
     earlier ones. The larger batch runs fewer warps per sequence, so a warp
@@ -707,6 +713,10 @@ def test_decode_offload_matches_hbm_decode_bit_for_bit(qsa, n0, S, H, batch):
 
     La, Lb = make(), make()
     Lb.offload_kv(H)
+    o = _oracle(w, cfg)
+    seqs = sorted({0, B // 2, B - 1})
+    T = n0 + S
+    host = {s: {nm: w.host_full(nm, s, T) for nm in ("q", "k", "v", "idx_q")} for s in seqs}
     hits_seen = False
     for step in range(S):
         p = n0 + step
@@ -714,7 +724,7 @@ def test_decode_offload_matches_hbm_decode_bit_for_bit(qsa, n0, S, H, batch):
         q = full["q"][:, n0].contiguous()          # the same query every step
         iq = full["idx_q"][:, n0].contiguous()
         k, v, ik = (full[nm][:, p].contiguous() for nm in ("k", "v", "idx_k"))
-        outs, sels = [], []
+        outs, sels, nsels = [], [], []
         for L, fn in ((La, La.decode_step), (Lb, Lb.decode_step_offload)):
             out = torch.empty(B, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
             sel = torch.empty(B, cfg.k_blocks, dtype=torch.int32, device="cuda")
@@ -724,8 +734,23 @@ def test_decode_offload_matches_hbm_decode_bit_for_bit(qsa, n0, S, H, batch):
             torch.cuda.synchronize()
             outs.append(out)
             sels.append(sel)
+            nsels.append(nsel)
         assert torch.equal(outs[0], outs[1]), step
+        assert torch.equal(nsels[0], nsels[1]), step
         assert torch.equal(sels[0], sels[1]), step
+        # The offloaded step against the oracle: the selection on the GPU's
+        # pooled keys, the attention on the caches' values over that selection.
+        g_sel, g_out, g_pooled = sels[1].cpu().numpy(), outs[1].float().cpu().numpy(), bits(Lb.pooled)
+        for s in seqs:
+            hs = host[s]
+            iq_row = hs["idx_q"][n0].reshape(4, 128)
+            ref = o.row(p, iq_row, g_pooled[s])
+            tol = score_tol(o.rotate_query(iq_row, p), g_pooled[s], ref["scores"])
+            m = int(nsels[1][s].item())
+            check_selection(g_sel[s], m, ref["scores"], tol, cfg.k_blocks, f"offload s{s} p{p}")
+            toks = o.token_set(g_sel[s, :m], p)
+            out_ref, _ = o.attention(hs["q"][n0], hs["k"], hs["v"], toks)
+            check_attention(g_out[s], out_ref.reshape(cfg.q_heads, 128), f"offload s{s} p{p}")
         # blocks this step found in the hot cache
         sb = sels[1].long()
         slot = sb.clamp(min=0) % H
