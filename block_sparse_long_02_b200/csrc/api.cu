@@ -425,7 +425,7 @@ qsa_status decode_step_impl(const qsa_config* cfg, int32_t batch, const int64_t*
                             qsa_bf16* k_cache, qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled,
                             int64_t cap, const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
                             void* ws, size_t ws_bytes, qsa_stream stream, const qsa::Q8Caches* q8,
-                            qsa::HotCache* hot = nullptr) {
+                            qsa::HotCache* hot = nullptr, bool clear_state = false) {
     qsa::LayerDims L;
     TRY(make_dims(cfg, &L));
     REQUIRE_PTR(pos);
@@ -459,6 +459,11 @@ qsa_status decode_step_impl(const qsa_config* cfg, int32_t batch, const int64_t*
     sw.winners = reinterpret_cast<int32_t*>(base + w.winners);
     sw.cand = reinterpret_cast<uint2*>(base + w.cand);
     cudaStream_t st = (cudaStream_t)stream;
+    // Every argument is valid from here on. A caller whose scratch may hold
+    // another call's state asks for the status header and the selection state
+    // to be cleared first.
+    if (clear_state)
+        TRY(cuda_check(cudaMemsetAsync(ws, 0, qsa::decode_state_bytes(batch), st), "decode state clear"));
     TRY(cuda_check(qsa::launch_decode_score(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
                                             pooled, cap, rms_w, scores, sw, status, q8, hot, st),
                    "decode score"));
@@ -555,6 +560,15 @@ qsa_status qsa_workspace_status(void* ws, qsa_stream stream, int32_t* status) {
 }  // extern "C"
 
 namespace qsa {
+int decode_step_cleared(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,
+                        const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q, const qsa_bf16* idx_k,
+                        qsa_bf16* k_cache, qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap,
+                        const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out, void* ws,
+                        size_t ws_bytes, void* stream) {
+    return decode_step_impl(cfg, batch, pos, q, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache, pooled, cap,
+                            rms_w, out, sel_out, nsel_out, ws, ws_bytes, stream, nullptr, nullptr, true);
+}
+
 size_t decode_state_bytes(int batch) {
     return kWsHeader + align_up((size_t)batch * 2048 * 4) + align_up((size_t)batch * 4 * 4);
 }

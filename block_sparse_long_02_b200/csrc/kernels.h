@@ -9,6 +9,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include "../../include/qsa.h"
 #include "common.cuh"
 
 namespace qsa {
@@ -174,6 +175,15 @@ int decode_select_ctas(int batch);
 // counters) that must be zero when a decode step starts; each step leaves
 // them zero.
 size_t decode_state_bytes(int batch);
+// qsa_decode_step on a workspace whose state bytes may hold anything (another
+// call's leftovers): checks every argument first, then clears the state bytes
+// on `stream`, then launches the step. A bad argument returns its error status
+// and queues nothing.
+int decode_step_cleared(const qsa_config* cfg, int32_t batch, const int64_t* pos, const qsa_bf16* q,
+                        const qsa_bf16* k, const qsa_bf16* v, const qsa_bf16* idx_q, const qsa_bf16* idx_k,
+                        qsa_bf16* k_cache, qsa_bf16* v_cache, qsa_bf16* idx_k_cache, qsa_bf16* pooled, int64_t cap,
+                        const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out, void* ws,
+                        size_t ws_bytes, void* stream);
 cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* pos, const uint16_t* k,
                                 const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
                                 uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled,

@@ -11,8 +11,6 @@
 // GPU, and held until the process exits) instead of a caller workspace.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "../../include/qsa.h"
 #include "kernels.h"
 
@@ -23,26 +21,18 @@ namespace {
 constexpr size_t kScratchBytes = (size_t)QSA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_decode_scratch on the current device (set up once per
-// device). In host code the array's name is only a host-side stand-in; its
-// device address comes from cudaGetSymbolAddress.
+// Device address of g_decode_scratch in the current context. In host code the
+// array's name is only a host-side stand-in; its device address comes from
+// cudaGetSymbolAddress, asked on every call: the address belongs to the
+// context that loaded the library's device code, and a context that is
+// destroyed and created again (cudaDeviceReset) may load it elsewhere. The
+// first call in a context loads that code, so it must not fall inside a
+// stream capture.
 cudaError_t scratch_ptr(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -72,11 +62,9 @@ extern "C" qsa_status qsa_decode_step_noalloc(const qsa_config* cfg, int32_t bat
         return (qsa_status)qsa::report_error(QSA_ERR_CUDA, "qsa_decode_step_noalloc set-up: %s",
                                              cudaGetErrorString(e));
     // The status header and the selection state must start at zero; the array
-    // may hold another batch size's layout from an earlier call.
-    e = cudaMemsetAsync(ws, 0, qsa::decode_state_bytes(batch), (cudaStream_t)stream);
-    if (e != cudaSuccess)
-        return (qsa_status)qsa::report_error(QSA_ERR_CUDA, "qsa_decode_step_noalloc: %s",
-                                             cudaGetErrorString(e));
-    return qsa_decode_step(cfg, batch, pos, q, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
-                           pooled, cap, rms_w, out, sel_out, nsel_out, ws, kScratchBytes, stream);
+    // may hold another batch size's layout from an earlier call. The step
+    // checks every argument before it clears them and launches.
+    return (qsa_status)qsa::decode_step_cleared(cfg, batch, pos, q, k, v, idx_q, idx_k, k_cache, v_cache,
+                                                idx_k_cache, pooled, cap, rms_w, out, sel_out, nsel_out, ws,
+                                                kScratchBytes, stream);
 }

@@ -352,13 +352,20 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
  *   - If qsa_workspace_size(QSA_OP_DECODE_STEP, batch, cap) exceeds
  *     QSA_NOALLOC_SCRATCH_BYTES the call returns QSA_ERR_WORKSPACE and launches
  *     nothing (e.g. batch 8 x 256K cached tokens fits; batch 64 x 4M does not).
- *   - The first call on each device does a one-time set-up (it looks up the
- *     array's device address); make that first call before any stream capture.
+ *   - Every call looks up the array's device address in the current context;
+ *     the first call in a context also loads the library's device code there,
+ *     so make that first call before any stream capture.
+ *   - Every argument is checked before anything is queued: a bad argument
+ *     returns its error status and leaves the stream untouched.
  *   - Every call shares the one array and it keeps the last call's contents:
  *     calls whose work overlaps on the GPU (other streams, other threads) race
  *     and corrupt each other's results. Order them on one stream.
- *   - The device status word is cleared at each call and cannot be read back:
- *     a position outside [0, cap) is skipped without a report. */
+ *   - The device status word lives in the array, is cleared at each call and
+ *     cannot be read back, so every status the step can flag on the device is
+ *     lost: QSA_ERR_CAPACITY (a position outside [0, cap) is skipped) and
+ *     QSA_ERR_DEVICE_CHECK (the selection's internal consistency check; out
+ *     and sel_out may then be wrong). Callers that need them use
+ *     qsa_decode_step with a workspace. */
 qsa_status qsa_decode_step_noalloc(const qsa_config* cfg, int32_t batch, const int64_t* pos,
                                    const qsa_bf16* q, const qsa_bf16* k, const qsa_bf16* v,
                                    const qsa_bf16* idx_q, const qsa_bf16* idx_k, qsa_bf16* k_cache,
