@@ -14,6 +14,7 @@
 // distributed shared memory (ties to the lower block index), and writes the
 // k_B winners in ascending order.
 #include <algorithm>
+#include <atomic>
 
 #include "kernels.h"
 #include "rope.cuh"
@@ -559,21 +560,26 @@ __global__ void __launch_bounds__(T) decode_select_kernel(
 
 }  // namespace
 
-// CTAs per sequence of the decode selection: one wave over the batch.
+// CTAs per sequence of the decode selection: one wave over the batch, on the
+// current device (each device's figure is computed once).
 int decode_select_ctas(int batch) {
-    static thread_local int cached = -1;
-    if (cached < 0) {
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> cached[kMaxDev];  // 0: not yet known
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int wave = (dev >= 0 && dev < kMaxDev) ? cached[dev].load(std::memory_order_relaxed) : 0;
+    if (wave <= 0) {
         const int smem = (int)sizeof(DecSelSmem);
         cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        int dev = 0, sms = 148, per_sm = 1;
-        cudaGetDevice(&dev);
+        int sms = 148, per_sm = 1;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_select_kernel, T, smem) != cudaSuccess ||
             per_sm < 1)
             per_sm = 1;
-        cached = sms * per_sm;
+        wave = sms * per_sm;
+        if (dev >= 0 && dev < kMaxDev) cached[dev].store(wave, std::memory_order_relaxed);
     }
-    return std::max(1, cached / std::max(batch, 1));
+    return std::max(1, wave / std::max(batch, 1));
 }
 
 // One wave: as many CTAs as fit on the GPU at once, split over the batch.
