@@ -176,10 +176,12 @@ const char* qsa_last_error(void) { return g_err.c_str(); }
 uint64_t qsa_launch_count(void) { return qsa::g_launches.load(std::memory_order_relaxed); }
 
 qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds) {
-    if (mode < 0 || mode > 2) return fail(QSA_ERR_INVALID_ARG, "fault injection mode %d", mode);
+    if (mode < 0 || mode > 3) return fail(QSA_ERR_INVALID_ARG, "fault injection mode %d", mode);
     if (mode != 0 && !(wait_seconds > 0.0 && wait_seconds <= 10.0))
         return fail(QSA_ERR_INVALID_ARG, "fault injection wait of %g s (want (0, 10])", wait_seconds);
-    qsa::set_fault_injection(mode, mode ? (uint64_t)(wait_seconds * 1e9) : 0);
+    const uint64_t ns = mode ? (uint64_t)(wait_seconds * 1e9) : 0;
+    qsa::set_fault_injection(mode == 3 ? 0 : mode, ns);
+    qsa::set_attention_fault_injection(mode == 3 ? 3 : 0, ns);
     return QSA_OK;
 }
 
@@ -299,9 +301,14 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
     if (lse && ((uintptr_t)lse & 3u)) return fail(QSA_ERR_INVALID_ARG, "lse misaligned");
     if (batch < 1 || cap < 1 || nq < 0 || q_begin < 0) return fail(QSA_ERR_INVALID_ARG, "bad sizes");
     if (q_begin + nq > cap) return fail(QSA_ERR_CAPACITY, "queries end at %lld > cap %lld", (long long)(q_begin + nq), (long long)cap);
-    (void)ws;
-    (void)ws_bytes;
+    if (ws && (ws_bytes < (size_t)qsa::kWsHeader || !aligned16(ws)))
+        return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes (%d needed) or misaligned", ws_bytes, qsa::kWsHeader);
     if (nq == 0) return QSA_OK;
+    if (qsa::attention_tc_supported(L, batch, cap, nq))
+        return cuda_check(qsa::launch_sparse_attention_tc(L, batch, q, q_begin, nq, k_cache, v_cache, cap, sel, nsel,
+                                                          out, lse, reinterpret_cast<int32_t*>(ws),
+                                                          (cudaStream_t)stream),
+                          "sparse attention");
     return cuda_check(qsa::launch_sparse_attention(L, batch, q, q_begin, nq, k_cache, v_cache, cap,
                                                    sel, nsel, out, lse, (cudaStream_t)stream),
                       "sparse attention");

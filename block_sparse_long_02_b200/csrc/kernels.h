@@ -171,6 +171,15 @@ struct DecodeSelWs {
     uint2* cand;        // [batch][kDecodeCand] (key, block)
 };
 int decode_select_ctas(int batch);
+// Sparse attention (a6 + a7) on tcgen05 with TMA block gathers; `status` (a
+// workspace header, may be NULL) receives QSA_ERR_TIMEOUT if a bounded wait
+// runs out.
+bool attention_tc_supported(const LayerDims& L, int batch, int64_t cap, int64_t nq);
+cudaError_t launch_sparse_attention_tc(const LayerDims& L, int batch, const uint16_t* q, int64_t q_begin, int64_t nq,
+                                       const uint16_t* kc, const uint16_t* vc, int64_t cap, const int32_t* sel,
+                                       const int32_t* nsel, uint16_t* out, float* lse, int32_t* status,
+                                       cudaStream_t st);
+void set_attention_fault_injection(int mode, uint64_t wait_ns);
 // Bytes at the start of a decode workspace (status header, histograms,
 // counters) that must be zero when a decode step starts; each step leaves
 // them zero.

@@ -17,7 +17,7 @@ from typing import Optional
 
 import torch
 
-from . import (OP_DECODE_STEP, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step,
+from . import (OP_DECODE_STEP, OP_SPARSE_ATTENTION, OP_TOPK_BLOCKS, Config, qsa_compress_keys, qsa_decode_step,
                qsa_decode_step_offload, qsa_decode_step_q8, qsa_quantize_rows,
                qsa_sparse_attention, qsa_sparse_attention_q8, qsa_topk_blocks, qsa_workspace_size)
 
@@ -64,7 +64,7 @@ class QSALayer:
         if mark:
             mark("topk")
         qsa_sparse_attention(self.cfg, self.batch, q, q_begin, nq, self.k_cache, self.v_cache, self.cap, sel,
-                             nsel, out, lse, None, stream)
+                             nsel, out, lse, self.workspace(OP_SPARSE_ATTENTION), stream)
         if mark:
             mark("attention")
 

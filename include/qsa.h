@@ -152,7 +152,14 @@ qsa_status qsa_topk_blocks(const qsa_config* cfg, int32_t batch, const qsa_bf16*
  * out:     [batch][nq][q_heads][head_dim] bf16.
  * lse:     [batch][nq][q_heads] fp32 natural-log sum-exp of the scaled logits,
  *          or NULL.
- * ws:      qsa_workspace_size(QSA_OP_SPARSE_ATTENTION, ...) bytes (may be 0). */
+ * ws:      qsa_workspace_size(QSA_OP_SPARSE_ATTENTION, ...) bytes (its status
+ *          header), or NULL. The tensor-core kernel's bounded waits record
+ *          QSA_ERR_TIMEOUT there (qsa_workspace_status); without a workspace a
+ *          timeout goes unreported.
+ * Kernels: q_heads / kv_heads in {1, 2, 4, 8, 16} (and batch x cap, batch x
+ * nq x q_heads below 2^31) run on the tensor cores, with whole blocks of every
+ * kv head gathered by TMA; other groups run on the warp-level kernel. Both
+ * compute the same values up to fp32 summation order. */
 qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_bf16* q,
                                 int64_t q_begin, int64_t nq, const qsa_bf16* k_cache,
                                 const qsa_bf16* v_cache, int64_t cap, const int32_t* sel,
@@ -400,6 +407,10 @@ uint64_t qsa_launch_count(void);
  *           every key tile; each CTA records QSA_ERR_TIMEOUT after
  *           wait_seconds, drains, frees its tensor memory and returns (the
  *           target it leaves is incomplete).
+ *   mode 3: the same for qsa_sparse_attention (its tensor-core kernel): the
+ *           key tiles of each CTA's first group of queries are withheld; the
+ *           timeout is recorded in the workspace passed to that call (none is
+ *           recorded without one) and the outputs it leaves are incomplete.
  * Returns QSA_ERR_INVALID_ARG for another mode or wait. */
 qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds);
 

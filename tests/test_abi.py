@@ -65,9 +65,9 @@ def test_null_and_capacity_errors_launch_nothing(qsa):
 
 def test_fault_injection_arguments_are_validated(qsa):
     """Host-side checks of the failure-path switch (no device work)."""
-    for mode, wait, ok in [(3, 0.1, False), (-1, 0.1, False), (1, 0.0, False), (1, 11.0, False),
-                           (1, float("nan"), False), (2, 0.0, False), (1, 0.5, True), (2, 0.5, True),
-                           (0, 0.0, True)]:
+    for mode, wait, ok in [(4, 0.1, False), (-1, 0.1, False), (1, 0.0, False), (1, 11.0, False),
+                           (1, float("nan"), False), (2, 0.0, False), (3, 0.0, False), (1, 0.5, True),
+                           (2, 0.5, True), (3, 0.5, True), (0, 0.0, True)]:
         if ok:
             qsa.qsa_set_fault_injection(mode, wait)
         else:
