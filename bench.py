@@ -474,6 +474,7 @@ def run_cuda(args, w, rank, world):
     dev = torch.device("cuda", torch.cuda.current_device())
     b = Bench(w, dev, stage=args.stage, kv=args.kv, offload=args.offload)
     qsa = b.qsa
+    qsa.qsa_set_attention_kernel(qsa.ATTENTION_TCGEN05 if args.attention == "tcgen05" else qsa.ATTENTION_WARP)
     for k in range(args.warmup):
         b.step()
         if k == 0 and not args.no_graph:
@@ -597,7 +598,9 @@ def run_cuda(args, w, rank, world):
                    "kv_location": ("HBM" if not args.offload else
                                    f"pinned host memory, {args.offload} hot blocks per sequence in HBM"),
                    "kv_cache": ("bf16" if args.kv == "bf16" else
-                                "fp8 E4M3 codes + one fp32 scale per row: core K/V, and pooled keys for decode")},
+                                "fp8 E4M3 codes + one fp32 scale per row: core K/V, and pooled keys for decode"),
+                   "attention_kernel": ("tcgen05 tiles in TMEM, TMA block gathers" if args.attention == "tcgen05"
+                                        and args.kv == "bf16" else "warp-level mma.sync tiles, cp.async gathers")},
         "roofline": roofline, "stages": stages,
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -780,6 +783,9 @@ def main():
     ap.add_argument("--stage", choices=["all", "topk"], default="all",
                     help="topk: time only key pooling + the fused indexer (for profiling)")
     ap.add_argument("--n", type=int, default=None, help="override the workload's sequence length")
+    ap.add_argument("--attention", choices=["warp", "tcgen05"], default="warp",
+                    help="sparse-attention kernel on bf16 caches: warp-level tiles (default) or tcgen05 tiles in TMEM "
+                         "fed by TMA block gathers")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
     if args.n is not None:

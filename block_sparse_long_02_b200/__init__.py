@@ -28,7 +28,7 @@ EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_t
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
            "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection", "qsa_quantize_rows",
            "qsa_sparse_attention_q8", "qsa_decode_step_q8", "qsa_decode_step_offload",
-           "qsa_sparse_attention_backward", "qsa_distill_target", "qsa_distill_kl"]
+           "qsa_sparse_attention_backward", "qsa_distill_target", "qsa_distill_kl", "qsa_set_attention_kernel"]
 
 
 class QSAError(RuntimeError):
@@ -119,6 +119,8 @@ def lib() -> ctypes.CDLL:
         h.qsa_launch_count.argtypes = []
         h.qsa_set_fault_injection.restype = ctypes.c_int
         h.qsa_set_fault_injection.argtypes = [ctypes.c_int32, ctypes.c_double]
+        h.qsa_set_attention_kernel.restype = ctypes.c_int
+        h.qsa_set_attention_kernel.argtypes = [ctypes.c_int32]
         _lib_handle = h
     return _lib_handle
 
@@ -289,6 +291,15 @@ def qsa_last_error() -> str:
 def qsa_launch_count() -> int:
     """Kernel launches issued by libqsa.so so far in this process."""
     return int(lib().qsa_launch_count())
+
+
+ATTENTION_WARP, ATTENTION_TCGEN05 = 0, 1
+
+
+def qsa_set_attention_kernel(kernel: int) -> None:
+    """Kernel of qsa_sparse_attention on bf16 caches: ATTENTION_WARP (default)
+    or ATTENTION_TCGEN05 (see qsa.h)."""
+    _check(lib().qsa_set_attention_kernel(int(kernel)))
 
 
 def qsa_set_fault_injection(mode: int, wait_seconds: float = 0.0) -> None:

@@ -13,6 +13,7 @@
 
 namespace qsa {
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<int> g_attention_kernel{0};  // 0: warp-level tiles, 1: tensor-core tiles
 void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 }  // namespace qsa
 
@@ -185,6 +186,12 @@ qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds) {
     return QSA_OK;
 }
 
+qsa_status qsa_set_attention_kernel(int32_t kernel) {
+    if (kernel != 0 && kernel != 1) return fail(QSA_ERR_INVALID_ARG, "attention kernel %d (0 or 1)", kernel);
+    qsa::g_attention_kernel.store(kernel, std::memory_order_relaxed);
+    return QSA_OK;
+}
+
 qsa_status qsa_workspace_size(const qsa_config* cfg, int32_t op, int32_t batch, int64_t cap,
                               int64_t nq, size_t* bytes) {
     qsa::LayerDims L;
@@ -304,7 +311,7 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
     if (ws && (ws_bytes < (size_t)qsa::kWsHeader || !aligned16(ws)))
         return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes (%d needed) or misaligned", ws_bytes, qsa::kWsHeader);
     if (nq == 0) return QSA_OK;
-    if (qsa::attention_tc_supported(L, batch, cap, nq))
+    if (qsa::g_attention_kernel.load(std::memory_order_relaxed) == 1 && qsa::attention_tc_supported(L, batch, cap, nq))
         return cuda_check(qsa::launch_sparse_attention_tc(L, batch, q, q_begin, nq, k_cache, v_cache, cap, sel, nsel,
                                                           out, lse, reinterpret_cast<int32_t*>(ws),
                                                           (cudaStream_t)stream),

@@ -156,15 +156,27 @@ qsa_status qsa_topk_blocks(const qsa_config* cfg, int32_t batch, const qsa_bf16*
  *          header), or NULL. The tensor-core kernel's bounded waits record
  *          QSA_ERR_TIMEOUT there (qsa_workspace_status); without a workspace a
  *          timeout goes unreported.
- * Kernels: q_heads / kv_heads in {1, 2, 4, 8, 16} (and batch x cap, batch x
- * nq x q_heads below 2^31) run on the tensor cores, with whole blocks of every
- * kv head gathered by TMA; other groups run on the warp-level kernel. Both
- * compute the same values up to fp32 summation order. */
+ * Kernels (qsa_set_attention_kernel): the default runs warp-level tensor-core
+ * tiles (mma.sync) over 16-token chunks gathered by each warp; the other runs
+ * tcgen05 tiles in TMEM fed by TMA block gathers, for q_heads / kv_heads in
+ * {1, 2, 4, 8, 16} (and batch x cap, batch x nq x q_heads below 2^31; other
+ * shapes keep the default). Both compute the same values up to fp32 summation
+ * order. */
 qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_bf16* q,
                                 int64_t q_begin, int64_t nq, const qsa_bf16* k_cache,
                                 const qsa_bf16* v_cache, int64_t cap, const int32_t* sel,
                                 const int32_t* nsel, qsa_bf16* out, float* lse, void* ws,
                                 size_t ws_bytes, qsa_stream stream);
+
+/* Which kernel runs qsa_sparse_attention on bf16 caches (process-wide):
+ *   0 (default): warp-level tiles: every warp gathers its own 16-token chunks
+ *      with cp.async and runs mma.sync; the faster of the two on the
+ *      measured workloads (128K and 1M prefill);
+ *   1: tcgen05 tiles with TMEM accumulators, fed by TMA boxes of whole blocks
+ *      (a persistent, warp-specialised kernel; its bounded waits report
+ *      QSA_ERR_TIMEOUT in the attention workspace).
+ * Returns QSA_ERR_INVALID_ARG for another value. Launches nothing. */
+qsa_status qsa_set_attention_kernel(int32_t kernel);
 
 /* Gradient of qsa_sparse_attention (concept page, "Native trainability via
  * 2-stage continued pretraining": stage 2 trains the model and the indexer

@@ -155,3 +155,14 @@ def test_offload_decode_validates_before_launching(qsa):
     assert call(64) == 1                            # the host caches are not mapped host memory
     assert b"host" in lib.qsa_last_error()
     assert lib.qsa_launch_count() == n0
+
+
+def test_attention_kernel_switch_is_validated(qsa):
+    """Host-side check of the sparse-attention kernel switch (no device work)."""
+    for k in (0, 1):
+        qsa.qsa_set_attention_kernel(k)
+    for k in (-1, 2):
+        with pytest.raises(qsa.QSAError) as e:
+            qsa.qsa_set_attention_kernel(k)
+        assert e.value.status == 1
+    qsa.qsa_set_attention_kernel(0)

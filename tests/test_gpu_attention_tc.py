@@ -1,5 +1,6 @@
-"""The sparse core attention on the tensor cores (tcgen05 tiles fed by TMA block
-gathers) against the oracle, on the cases its design has to get right:
+"""The sparse core attention on the fifth-generation tensor cores (tcgen05 tiles
+fed by TMA block gathers; qsa_set_attention_kernel(1) for this module) against
+the oracle, on the cases its design has to get right:
 cache rows past the last query holding NaN (the tail's box reads them; they must
 be masked and their values cleared), block sizes whose pieces pad or split a
 tile, a logit maximum that only appears late in a query's tile stream (the
@@ -24,7 +25,9 @@ NAN_BF16 = 0x7FC0
 def qsa():
     import block_sparse_long_02_b200 as m
 
-    return m
+    m.qsa_set_attention_kernel(m.ATTENTION_TCGEN05)
+    yield m
+    m.qsa_set_attention_kernel(m.ATTENTION_WARP)
 
 
 def _oracle(cfg):

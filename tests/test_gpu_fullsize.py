@@ -117,7 +117,18 @@ def _check_prefill(w, cfg, L, q, iq, out, sel, nsel, rows, needles):
     return o
 
 
-def test_prefill_128k_full_size():
+@pytest.mark.parametrize("kernel", [0, 1], ids=["warp_tiles", "tcgen05_tiles"])
+def test_prefill_128k_full_size(kernel):
+    import block_sparse_long_02_b200 as qsa
+
+    qsa.qsa_set_attention_kernel(kernel)
+    try:
+        _prefill_128k()
+    finally:
+        qsa.qsa_set_attention_kernel(0)
+
+
+def _prefill_128k():
     w = synth.WORKLOADS["prefill_n128k"]
     cfg, L, q, iq, out, sel, nsel = _prefill(w)
     rows = _sample_rows(w, 24, 1) + sorted({p for _, p in w.needles(0)})[:16]

@@ -23,6 +23,14 @@ def qsa():
     return m
 
 
+@pytest.fixture(params=[0, 1], ids=["warp_tiles", "tcgen05_tiles"])
+def kernel(request, qsa):
+    """Runs a prefill test with each sparse-attention kernel."""
+    qsa.qsa_set_attention_kernel(request.param)
+    yield request.param
+    qsa.qsa_set_attention_kernel(0)
+
+
 def _layer(qsa, w, cap, **over):
     from block_sparse_long_02_b200.layer import QSALayer
 
@@ -184,14 +192,14 @@ def test_select_candidate_overflow_path(qsa):
 
 
 # ----------------------------------------------------------------------------- a1..a7 prefill
-def test_tiny_prefill_all_rows(qsa):
+def test_tiny_prefill_all_rows(qsa, kernel):
     w = synth.WORKLOADS["tiny_prefill_n256"]
     cfg, res = run_prefill(qsa, w)
     check_rows(w, cfg, res, range(w.n))
 
 
 @pytest.mark.parametrize("q_heads,kv_heads", [(32, 4), (8, 1), (16, 2), (64, 8), (16, 4)])
-def test_prefill_ragged_gqa(qsa, q_heads, kv_heads):
+def test_prefill_ragged_gqa(qsa, q_heads, kv_heads, kernel):
     w = synth.Workload(name="t", n=2003, K=128, q_heads=q_heads, kv_heads=kv_heads,
                        base_seed=0xE0 + q_heads, n_needles_prefill=6)
     cfg, res = run_prefill(qsa, w)
@@ -200,7 +208,7 @@ def test_prefill_ragged_gqa(qsa, q_heads, kv_heads):
     check_rows(w, cfg, res, rows)
 
 
-def test_prefill_chunk_with_offset_and_batch(qsa):
+def test_prefill_chunk_with_offset_and_batch(qsa, kernel):
     w = synth.Workload(name="t", n=1500, batch=2, K=96, q_heads=8, kv_heads=2, base_seed=0xE7)
     cfg, res = run_prefill(qsa, w, q_begin=701, nq=799)
     rows = list(range(701, 740)) + list(range(1460, 1500))
@@ -208,7 +216,7 @@ def test_prefill_chunk_with_offset_and_batch(qsa):
         check_rows(w, cfg, res, rows, s=s, q_begin=701)
 
 
-def test_budget_covering_all_blocks_is_dense(qsa):
+def test_budget_covering_all_blocks_is_dense(qsa, kernel):
     """k_B >= visible blocks: every visible block is selected, in order."""
     w = synth.Workload(name="t", n=600, K=4096, q_heads=8, kv_heads=2, base_seed=0xE8)
     cfg, res = run_prefill(qsa, w)
@@ -219,13 +227,13 @@ def test_budget_covering_all_blocks_is_dense(qsa):
 
 
 @pytest.mark.parametrize("r", [1, 8])
-def test_generic_block_size(qsa, r):
+def test_generic_block_size(qsa, r, kernel):
     w = synth.Workload(name="t", n=777, r=r, K=96, q_heads=8, kv_heads=2, base_seed=0xE9 + r)
     cfg, res = run_prefill(qsa, w)
     check_rows(w, cfg, res, list(range(0, 20)) + list(range(700, 777)))
 
 
-def test_invalid_selection_entries_are_skipped(qsa):
+def test_invalid_selection_entries_are_skipped(qsa, kernel):
     """Entries outside [0, floor(i/r)) never read memory; they drop out of the set."""
     w = synth.Workload(name="t", n=512, K=64, q_heads=8, kv_heads=2, base_seed=0xEA)
     cfg, L = _layer(qsa, w, 512)
