@@ -12,7 +12,10 @@ K/V 2.1 GB), and decode steps run back to back as in real decoding.
 
 Prints one JSON line (rank 0). With N > 1 (torchrun), every rank runs an
 independent replica (the layer has no cross-GPU exchange); time is the max
-over ranks and value counts the tokens of all ranks.
+over ranks and value counts the tokens of all ranks. On one GPU the default run
+also measures the metric's other workloads (32K and 8 x 256K decode, 128K
+prefill) and reports them under "configs", each with its stage rooflines and
+the oracle timed beside it (--no-configs skips them).
 """
 from __future__ import annotations
 
@@ -610,7 +613,7 @@ def run_cuda(args, w, rank, world):
         res["prefill_tokens_per_s"] = round(alg["prefill_tokens"] / (pre_ms * 1e-3), 1)
         res["decode_tokens_per_s"] = round(alg["decode_tokens"] / (stage_ms["decode"] * 1e-3), 1)
     if not args.no_e2e:
-        e_ms, h2d, d2h = b.e2e(max(1, min(args.steps, 2)), 1)
+        e_ms, h2d, d2h = b.e2e(max(5, args.steps), 1)
         e_ms = max_over_ranks(e_ms, world, dev)
         res["e2e"] = {"value": round(job_value(tokens, e_ms, world), 2), "unit": "tokens/s",
                       "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
@@ -740,6 +743,32 @@ def cpu_baseline(w, rows=64, dec=2, blocks=65536):
                                                         for k, v in parts.items()}}
 
 
+# The other workloads of the metric, measured in the same run as the headline
+# (one GPU): tokens/s, the stage rooflines and the oracle beside each.
+OTHER_CONFIGS = (("decode_b1_n32k", 50), ("prefill_n128k", 3), ("decode_b8_n256k", 50))
+
+
+def run_configs(args):
+    import copy
+
+    out = {}
+    for name, steps in OTHER_CONFIGS:
+        a = copy.copy(args)
+        a.workload, a.steps, a.warmup, a.no_e2e, a.n = name, steps, 3, True, None
+        w = synth.WORKLOADS[name]
+        r = run_cuda(a, w, 0, 1)
+        torch.cuda.empty_cache()
+        ent = {k: r[k] for k in ("value", "unit", "ms_per_step", "steps", "roofline", "stages", "gpu_launches",
+                                 "clocks", "config")}
+        for k in ("prefill_tokens_per_s", "decode_tokens_per_s"):
+            if k in r:
+                ent[k] = r[k]
+        if not args.no_cpu_baseline:
+            ent["cpu_baseline"] = cpu_baseline(w, rows=32)
+        out[name] = ent
+    return out
+
+
 def run_reference(args, w):
     times = []
     with one_core():
@@ -783,6 +812,9 @@ def main():
     ap.add_argument("--stage", choices=["all", "topk"], default="all",
                     help="topk: time only key pooling + the fused indexer (for profiling)")
     ap.add_argument("--n", type=int, default=None, help="override the workload's sequence length")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads that the default run also measures (32K and 8x256K decode, "
+                         "128K prefill)")
     ap.add_argument("--attention", choices=["warp", "tcgen05"], default="warp",
                     help="sparse-attention kernel on bf16 caches: warp-level tiles (default) or tcgen05 tiles in TMEM "
                          "fed by TMA block gathers")
@@ -813,6 +845,9 @@ def main():
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w)
+        if world == 1 and args.workload == DEFAULT_WORKLOAD and args.stage == "all" and args.n is None \
+                and not args.no_configs and not args.offload and args.kv == "bf16":
+            res["configs"] = run_configs(args)
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
