@@ -28,7 +28,8 @@ EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_t
            "qsa_sparse_attention", "qsa_decode_step", "qsa_workspace_status", "qsa_last_error",
            "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection", "qsa_quantize_rows",
            "qsa_sparse_attention_q8", "qsa_decode_step_q8", "qsa_decode_step_offload",
-           "qsa_sparse_attention_backward", "qsa_distill_target", "qsa_distill_kl", "qsa_set_attention_kernel"]
+           "qsa_sparse_attention_backward", "qsa_distill_target", "qsa_distill_kl", "qsa_set_attention_kernel",
+           "qsa_index_scores_varlen", "qsa_topk_blocks_varlen", "qsa_sparse_attention_varlen"]
 
 
 class QSAError(RuntimeError):
@@ -95,6 +96,9 @@ _SIGS = {
                                                            _vp],
     "qsa_sparse_attention_q8": [_CFG, _i32, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp,
                                 _sz, _vp],
+    "qsa_index_scores_varlen": [_CFG, _i32, _vp, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _sz, _vp],
+    "qsa_topk_blocks_varlen": [_CFG, _i32, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp],
+    "qsa_sparse_attention_varlen": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
     "qsa_decode_step_noalloc": [_CFG, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp,
                                 _vp, _vp, _vp],
 }
@@ -194,6 +198,35 @@ def qsa_sparse_attention(cfg: Config, batch: int, q: torch.Tensor, q_begin: int,
     _check(lib().qsa_sparse_attention(ctypes.byref(cfg.c()), batch, _ptr(q), q_begin, nq, _ptr(k_cache),
                                      _ptr(v_cache), cap, _ptr(sel), _ptr(nsel), _ptr(out), _ptr(lse),
                                      _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def _host_i64(values) -> ctypes.Array:
+    return (ctypes.c_int64 * len(values))(*[int(v) for v in values])
+
+
+def qsa_index_scores_varlen(cfg: Config, idx_q: torch.Tensor, q_begin, nq, pooled: torch.Tensor, cap: int,
+                            scores: torch.Tensor, ld: int, ws: torch.Tensor, stream=None) -> None:
+    """Per-sequence query ranges (q_begin[s], nq[s]: host lists), queries packed."""
+    _check(lib().qsa_index_scores_varlen(ctypes.byref(cfg.c()), len(nq), _ptr(idx_q), _host_i64(q_begin),
+                                         _host_i64(nq), _ptr(pooled), cap, _ptr(scores), ld, _ptr(ws), ws.numel(),
+                                         _stream(stream)))
+
+
+def qsa_topk_blocks_varlen(cfg: Config, idx_q: torch.Tensor, q_begin, nq, pooled: torch.Tensor, cap: int,
+                           sel: torch.Tensor, nsel: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    _check(lib().qsa_topk_blocks_varlen(ctypes.byref(cfg.c()), len(nq), _ptr(idx_q), _host_i64(q_begin),
+                                        _host_i64(nq), _ptr(pooled), cap, _ptr(sel), _ptr(nsel), _ptr(ws),
+                                        ws.numel(), _stream(stream)))
+
+
+def qsa_sparse_attention_varlen(cfg: Config, q: torch.Tensor, q_begin, nq, k_cache: torch.Tensor,
+                                v_cache: torch.Tensor, cap: int, sel: torch.Tensor, nsel: torch.Tensor,
+                                out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                                ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().qsa_sparse_attention_varlen(ctypes.byref(cfg.c()), len(nq), _ptr(q), _host_i64(q_begin),
+                                             _host_i64(nq), _ptr(k_cache), _ptr(v_cache), cap, _ptr(sel),
+                                             _ptr(nsel), _ptr(out), _ptr(lse), _ptr(ws),
+                                             0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def qsa_sparse_attention_backward(cfg: Config, batch: int, q: torch.Tensor, q_begin: int, nq: int,

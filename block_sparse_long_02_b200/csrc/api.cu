@@ -321,6 +321,117 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
                       "sparse attention");
 }
 
+// ---- Variable-length batches: one call over sequences with their own query
+// ranges. Every argument of every sequence is checked first; then each
+// sequence runs through the single-sequence path on `stream`, in order,
+// sharing the workspace (the launches on one stream never overlap).
+}  // extern "C"
+
+namespace {
+struct VarlenPlan {
+    int64_t total = 0, max_nq = 0, max_vis = 0;
+};
+
+qsa_status varlen_plan(const qsa::LayerDims& L, int32_t batch, const int64_t* q_begin, const int64_t* nq,
+                       int64_t cap, VarlenPlan* plan) {
+    if (batch < 1 || cap < 1) return fail(QSA_ERR_INVALID_ARG, "batch=%d cap=%lld", batch, (long long)cap);
+    if (!q_begin || !nq) return fail(QSA_ERR_INVALID_ARG, "q_begin and nq must be host arrays of batch entries");
+    VarlenPlan p;
+    for (int32_t s = 0; s < batch; ++s) {
+        if (q_begin[s] < 0 || nq[s] < 0)
+            return fail(QSA_ERR_INVALID_ARG, "sequence %d: q_begin=%lld nq=%lld", s, (long long)q_begin[s],
+                        (long long)nq[s]);
+        if (q_begin[s] + nq[s] > cap)
+            return fail(QSA_ERR_CAPACITY, "sequence %d: queries end at %lld > cap %lld", s,
+                        (long long)(q_begin[s] + nq[s]), (long long)cap);
+        p.total += nq[s];
+        p.max_nq = std::max(p.max_nq, nq[s]);
+        if (nq[s] > 0) p.max_vis = std::max(p.max_vis, visible_ld(L, q_begin[s], nq[s]));
+    }
+    *plan = p;
+    return QSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+qsa_status qsa_index_scores_varlen(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                                   const int64_t* q_begin, const int64_t* nq, const qsa_bf16* pooled, int64_t cap,
+                                   float* scores, int64_t ld, void* ws, size_t ws_bytes, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    VarlenPlan plan;
+    TRY(varlen_plan(L, batch, q_begin, nq, cap, &plan));
+    REQUIRE_PTR(idx_q);
+    REQUIRE_PTR(pooled);
+    if (!scores || ((uintptr_t)scores & 3u)) return fail(QSA_ERR_INVALID_ARG, "scores NULL or misaligned");
+    if (plan.total && ld < plan.max_vis)
+        return fail(QSA_ERR_INVALID_ARG, "ld=%lld below %lld visible blocks", (long long)ld, (long long)plan.max_vis);
+    TRY(check_ws(ws, ws_bytes, index_scores_ws(1, plan.max_nq)));
+    int64_t off = 0;
+    for (int32_t s = 0; s < batch; ++s) {
+        if (nq[s] > 0)
+            TRY(qsa_index_scores(cfg, 1, idx_q + off * qsa::kIdxHeads * qsa::kIdxDim, q_begin[s], nq[s],
+                                 pooled + (size_t)s * (cap / L.r) * qsa::kIdxDim, cap, scores + off * ld, ld, ws,
+                                 ws_bytes, stream));
+        off += nq[s];
+    }
+    return QSA_OK;
+}
+
+qsa_status qsa_topk_blocks_varlen(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                                  const int64_t* q_begin, const int64_t* nq, const qsa_bf16* pooled, int64_t cap,
+                                  int32_t* sel, int32_t* nsel, void* ws, size_t ws_bytes, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    VarlenPlan plan;
+    TRY(varlen_plan(L, batch, q_begin, nq, cap, &plan));
+    REQUIRE_PTR(idx_q);
+    REQUIRE_PTR(pooled);
+    REQUIRE_PTR(sel);
+    if (!nsel || ((uintptr_t)nsel & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel NULL or misaligned");
+    TRY(check_ws(ws, ws_bytes, topk_layout(L, 1, cap, plan.max_nq).total));
+    int64_t off = 0;
+    for (int32_t s = 0; s < batch; ++s) {
+        if (nq[s] > 0)
+            TRY(qsa_topk_blocks(cfg, 1, idx_q + off * qsa::kIdxHeads * qsa::kIdxDim, q_begin[s], nq[s],
+                                pooled + (size_t)s * (cap / L.r) * qsa::kIdxDim, cap, nullptr, 0, sel + off * L.kB,
+                                nsel + off, ws, ws_bytes, stream));
+        off += nq[s];
+    }
+    return QSA_OK;
+}
+
+qsa_status qsa_sparse_attention_varlen(const qsa_config* cfg, int32_t batch, const qsa_bf16* q,
+                                       const int64_t* q_begin, const int64_t* nq, const qsa_bf16* k_cache,
+                                       const qsa_bf16* v_cache, int64_t cap, const int32_t* sel, const int32_t* nsel,
+                                       qsa_bf16* out, float* lse, void* ws, size_t ws_bytes, qsa_stream stream) {
+    qsa::LayerDims L;
+    TRY(make_dims(cfg, &L));
+    VarlenPlan plan;
+    TRY(varlen_plan(L, batch, q_begin, nq, cap, &plan));
+    REQUIRE_PTR(q);
+    REQUIRE_PTR(k_cache);
+    REQUIRE_PTR(v_cache);
+    REQUIRE_PTR(sel);
+    REQUIRE_PTR(out);
+    if (!nsel || ((uintptr_t)nsel & 3u)) return fail(QSA_ERR_INVALID_ARG, "nsel NULL or misaligned");
+    if (lse && ((uintptr_t)lse & 3u)) return fail(QSA_ERR_INVALID_ARG, "lse misaligned");
+    if (ws && (ws_bytes < (size_t)qsa::kWsHeader || !aligned16(ws)))
+        return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes (%d needed) or misaligned", ws_bytes, qsa::kWsHeader);
+    const size_t row = (size_t)L.q_heads * L.head_dim;
+    const size_t seq = (size_t)cap * L.kv_heads * L.head_dim;
+    int64_t off = 0;
+    for (int32_t s = 0; s < batch; ++s) {
+        if (nq[s] > 0)
+            TRY(qsa_sparse_attention(cfg, 1, q + off * row, q_begin[s], nq[s], k_cache + s * seq, v_cache + s * seq,
+                                     cap, sel + off * L.kB, nsel + off, out + off * row,
+                                     lse ? lse + off * L.q_heads : nullptr, ws, ws_bytes, stream));
+        off += nq[s];
+    }
+    return QSA_OK;
+}
+
 qsa_status qsa_sparse_attention_backward(const qsa_config* cfg, int32_t batch, const qsa_bf16* q, int64_t q_begin,
                                          int64_t nq, const qsa_bf16* k_cache, const qsa_bf16* v_cache, int64_t cap,
                                          const int32_t* sel, const int32_t* nsel, const qsa_bf16* out,

@@ -68,6 +68,36 @@ class QSALayer:
         if mark:
             mark("attention")
 
+    def prefill_varlen(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin, nq, out: torch.Tensor,
+                       sel: torch.Tensor, nsel: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                       stream=None) -> None:
+        """Prefill of a different query range per sequence in one call each:
+        queries [q_begin[s], q_begin[s] + nq[s]) of sequence s (host lists),
+        packed one sequence after another in q ([total][q_heads][128]), idx_q,
+        out, sel, nsel and lse. Their keys and values are already in the caches."""
+        from . import qsa_sparse_attention_varlen, qsa_topk_blocks_varlen
+
+        r = self.cfg.r
+        for s, (b, m) in enumerate(zip(q_begin, nq)):
+            if m:
+                qsa_compress_keys(self.cfg, 1, self.idx_k_cache[s:s + 1], self.cap, self.rms_w, b // r,
+                                  (b + m) // r, self.pooled[s:s + 1], stream)
+        ws = self.workspace_for(OP_TOPK_BLOCKS, 1, max(nq))
+        qsa_topk_blocks_varlen(self.cfg, idx_q, q_begin, nq, self.pooled, self.cap, sel, nsel, ws, stream)
+        qsa_sparse_attention_varlen(self.cfg, q, q_begin, nq, self.k_cache, self.v_cache, self.cap, sel, nsel, out,
+                                    lse, self.workspace(OP_SPARSE_ATTENTION), stream)
+
+    def workspace_for(self, op: int, batch: int, nq: int) -> torch.Tensor:
+        """A workspace of `op` for `batch` sequences and nq queries (kept per op
+        and size class; grown as needed)."""
+        need = qsa_workspace_size(self.cfg, op, batch, self.cap, nq)
+        key = (op, batch)
+        ws = self._ws.get(key)
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=self.device)
+            self._ws[key] = ws
+        return ws
+
     # ------------------------------------------------ fp8 (E4M3) core K/V caches
     def quantize_kv(self, begin: int, end: int, stream=None) -> None:
         """FP8 copies of the core K/V cache rows [begin, end) of every sequence

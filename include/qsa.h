@@ -32,7 +32,8 @@
  *     message for the last non-OK status of the calling thread.
  *   - Positions are 0-based. Query i sees complete blocks b < floor(i/r) and
  *     the tail tokens r*floor(i/r) .. i. Prefill queries are the consecutive
- *     positions [q_begin, q_begin + nq); every sequence of a batch shares them.
+ *     positions [q_begin, q_begin + nq); every sequence of a batch shares them
+ *     (the *_varlen calls take a range per sequence).
  *   - Supported shapes: idx_heads = 4, idx_dim = 128, rope_dims even and
  *     <= 128, head_dim = 128, q_heads % kv_heads == 0 with q_heads/kv_heads <= 16,
  *     kv_heads <= 8, 1 <= r <= 64, k_B = ceil(K/r) <= 4096. Others return
@@ -177,6 +178,36 @@ qsa_status qsa_sparse_attention(const qsa_config* cfg, int32_t batch, const qsa_
  *      QSA_ERR_TIMEOUT in the attention workspace).
  * Returns QSA_ERR_INVALID_ARG for another value. Launches nothing. */
 qsa_status qsa_set_attention_kernel(int32_t kernel);
+
+/* ---- Variable-length batches ----
+ * One call over `batch` sequences whose queries are different ranges: query j
+ * (0 <= j < nq[s]) of sequence s sits at position q_begin[s] + j, and the
+ * queries of all sequences are packed one after another (sequence 0's first;
+ * total = sum of nq). This is the serving pattern of the "QSA" knowledge page's
+ * timeline (prefills of requests at different lengths, serial or interleaved
+ * with decoding), for the calls of a prefill. Caches, pooled keys and the
+ * workspace are as for the single-range calls (per sequence, capacity cap).
+ * q_begin, nq: HOST arrays of batch int64 each; q_begin[s] >= 0, nq[s] >= 0
+ * (0 skips the sequence), q_begin[s] + nq[s] <= cap (else QSA_ERR_CAPACITY).
+ * Packed layouts (total rows): idx_q [total][idx_heads][idx_dim], q and out
+ * [total][q_heads][head_dim], sel [total][k_B], nsel [total], lse
+ * [total][q_heads], scores [total][ld].
+ * Workspace: the single-range size for one sequence with the largest nq,
+ * qsa_workspace_size(op, 1, cap, max nq[s]).
+ * Every argument of every sequence is checked before anything is launched;
+ * then the sequences run in order on `stream` (a sequence's launches are the
+ * single-range call's), so the results equal those calls' bit for bit. */
+qsa_status qsa_index_scores_varlen(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                                   const int64_t* q_begin, const int64_t* nq, const qsa_bf16* pooled, int64_t cap,
+                                   float* scores, int64_t ld, void* ws, size_t ws_bytes, qsa_stream stream);
+/* The fused selection (qsa_topk_blocks with scores == NULL) of each range. */
+qsa_status qsa_topk_blocks_varlen(const qsa_config* cfg, int32_t batch, const qsa_bf16* idx_q,
+                                  const int64_t* q_begin, const int64_t* nq, const qsa_bf16* pooled, int64_t cap,
+                                  int32_t* sel, int32_t* nsel, void* ws, size_t ws_bytes, qsa_stream stream);
+qsa_status qsa_sparse_attention_varlen(const qsa_config* cfg, int32_t batch, const qsa_bf16* q,
+                                       const int64_t* q_begin, const int64_t* nq, const qsa_bf16* k_cache,
+                                       const qsa_bf16* v_cache, int64_t cap, const int32_t* sel, const int32_t* nsel,
+                                       qsa_bf16* out, float* lse, void* ws, size_t ws_bytes, qsa_stream stream);
 
 /* Gradient of qsa_sparse_attention (concept page, "Native trainability via
  * 2-stage continued pretraining": stage 2 trains the model and the indexer
