@@ -478,6 +478,7 @@ def run_cuda(args, w, rank, world):
     b = Bench(w, dev, stage=args.stage, kv=args.kv, offload=args.offload)
     qsa = b.qsa
     qsa.qsa_set_attention_kernel(qsa.ATTENTION_TCGEN05 if args.attention == "tcgen05" else qsa.ATTENTION_WARP)
+    qsa.qsa_set_decode_kernel(qsa.DECODE_THREE_KERNELS if args.decode == "three" else qsa.DECODE_STEP_KERNEL)
     for k in range(args.warmup):
         b.step()
         if k == 0 and not args.no_graph:
@@ -603,7 +604,9 @@ def run_cuda(args, w, rank, world):
                    "kv_cache": ("bf16" if args.kv == "bf16" else
                                 "fp8 E4M3 codes + one fp32 scale per row: core K/V, and pooled keys for decode"),
                    "attention_kernel": ("tcgen05 tiles in TMEM, TMA block gathers" if args.attention == "tcgen05"
-                                        and args.kv == "bf16" else "warp-level mma.sync tiles, cp.async gathers")},
+                                        and args.kv == "bf16" else "warp-level mma.sync tiles, cp.async gathers"),
+                   "decode_kernels": ("three per step: scores, selection, attention" if args.decode == "three"
+                                      else "one persistent kernel per step")},
         "roofline": roofline, "stages": stages,
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -815,6 +818,8 @@ def main():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads that the default run also measures (32K and 8x256K decode, "
                          "128K prefill)")
+    ap.add_argument("--decode", choices=["step", "three"], default="three",
+                    help="decode step as three kernels (default) or as one persistent kernel")
     ap.add_argument("--attention", choices=["warp", "tcgen05"], default="warp",
                     help="sparse-attention kernel on bf16 caches: warp-level tiles (default) or tcgen05 tiles in TMEM "
                          "fed by TMA block gathers")

@@ -29,7 +29,8 @@ EXPORTS = ["qsa_workspace_size", "qsa_compress_keys", "qsa_index_scores", "qsa_t
            "qsa_launch_count", "qsa_decode_step_noalloc", "qsa_set_fault_injection", "qsa_quantize_rows",
            "qsa_sparse_attention_q8", "qsa_decode_step_q8", "qsa_decode_step_offload",
            "qsa_sparse_attention_backward", "qsa_distill_target", "qsa_distill_kl", "qsa_set_attention_kernel",
-           "qsa_index_scores_varlen", "qsa_topk_blocks_varlen", "qsa_sparse_attention_varlen"]
+           "qsa_index_scores_varlen", "qsa_topk_blocks_varlen", "qsa_sparse_attention_varlen",
+           "qsa_set_decode_kernel"]
 
 
 class QSAError(RuntimeError):
@@ -125,6 +126,8 @@ def lib() -> ctypes.CDLL:
         h.qsa_set_fault_injection.argtypes = [ctypes.c_int32, ctypes.c_double]
         h.qsa_set_attention_kernel.restype = ctypes.c_int
         h.qsa_set_attention_kernel.argtypes = [ctypes.c_int32]
+        h.qsa_set_decode_kernel.restype = ctypes.c_int
+        h.qsa_set_decode_kernel.argtypes = [ctypes.c_int32]
         _lib_handle = h
     return _lib_handle
 
@@ -333,6 +336,15 @@ def qsa_set_attention_kernel(kernel: int) -> None:
     """Kernel of qsa_sparse_attention on bf16 caches: ATTENTION_WARP (default)
     or ATTENTION_TCGEN05 (see qsa.h)."""
     _check(lib().qsa_set_attention_kernel(int(kernel)))
+
+
+DECODE_STEP_KERNEL, DECODE_THREE_KERNELS = 0, 1
+
+
+def qsa_set_decode_kernel(kernel: int) -> None:
+    """Kernels of a decode step: DECODE_STEP_KERNEL (one persistent kernel) or
+    DECODE_THREE_KERNELS (the default; see qsa.h)."""
+    _check(lib().qsa_set_decode_kernel(int(kernel)))
 
 
 def qsa_set_fault_injection(mode: int, wait_seconds: float = 0.0) -> None:

@@ -14,6 +14,7 @@
 namespace qsa {
 static std::atomic<uint64_t> g_launches{0};
 static std::atomic<int> g_attention_kernel{0};  // 0: warp-level tiles, 1: tensor-core tiles
+static std::atomic<int> g_decode_kernel{1};     // 0: one persistent step kernel, 1: three kernels
 void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 }  // namespace qsa
 
@@ -124,7 +125,7 @@ TopkWs topk_layout(const qsa::LayerDims& L, int batch, int64_t cap, int64_t nq) 
 }
 
 struct DecodeWs {
-    size_t scores, sel, nsel, hist, counters, winners, cand, total;
+    size_t scores, sel, nsel, hist, counters, sync, est, winners, cand, part, pre, total;
 };
 
 DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
@@ -134,13 +135,18 @@ DecodeWs decode_layout(const qsa::LayerDims& L, int batch, int64_t cap) {
     DecodeWs w;
     w.hist = qsa::kWsHeader;
     w.counters = w.hist + align_up((size_t)batch * 2048 * 4);
-    w.scores = w.counters + align_up((size_t)batch * 4 * 4);
-    // (w.scores == qsa::decode_state_bytes(batch))
+    w.sync = w.counters + align_up((size_t)batch * 4 * 4);
+    w.est = w.sync + align_up((size_t)batch * qsa::step_sync_words(L.kv_heads) * 4);
+    w.scores = w.est + align_up((size_t)batch * 8);
+    // (w.scores == qsa::decode_state_bytes(batch, L.kv_heads))
     w.sel = w.scores + align_up((size_t)batch * std::max<int64_t>(1, cap / L.r) * 4);
     w.nsel = w.sel + align_up((size_t)batch * L.kB * 4);
     w.winners = w.nsel + align_up((size_t)batch * 4);
     w.cand = w.winners + align_up((size_t)batch * L.kB * 4);
-    w.total = w.cand + align_up((size_t)batch * qsa::kDecodeCand * 8);
+    w.part = w.cand + align_up((size_t)batch * qsa::kDecodeCand * 8);
+    const size_t G = (size_t)(L.q_heads / L.kv_heads);
+    w.pre = w.part + align_up((size_t)batch * L.kv_heads * qsa::kStepSplitCap * (G * L.head_dim + 2 * G) * 4);
+    w.total = w.pre + align_up((size_t)batch * qsa::kDecodePre * 8);
     return w;
 }
 
@@ -177,12 +183,19 @@ const char* qsa_last_error(void) { return g_err.c_str(); }
 uint64_t qsa_launch_count(void) { return qsa::g_launches.load(std::memory_order_relaxed); }
 
 qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds) {
-    if (mode < 0 || mode > 3) return fail(QSA_ERR_INVALID_ARG, "fault injection mode %d", mode);
+    if (mode < 0 || mode > 4) return fail(QSA_ERR_INVALID_ARG, "fault injection mode %d", mode);
     if (mode != 0 && !(wait_seconds > 0.0 && wait_seconds <= 10.0))
         return fail(QSA_ERR_INVALID_ARG, "fault injection wait of %g s (want (0, 10])", wait_seconds);
     const uint64_t ns = mode ? (uint64_t)(wait_seconds * 1e9) : 0;
-    qsa::set_fault_injection(mode == 3 ? 0 : mode, ns);
+    qsa::set_fault_injection(mode == 1 || mode == 2 ? mode : 0, ns);
     qsa::set_attention_fault_injection(mode == 3 ? 3 : 0, ns);
+    qsa::set_decode_fault_injection(mode == 4 ? 1 : 0, ns);
+    return QSA_OK;
+}
+
+qsa_status qsa_set_decode_kernel(int32_t kernel) {
+    if (kernel != 0 && kernel != 1) return fail(QSA_ERR_INVALID_ARG, "decode kernel %d (0 or 1)", kernel);
+    qsa::g_decode_kernel.store(kernel, std::memory_order_relaxed);
     return QSA_OK;
 }
 
@@ -583,12 +596,30 @@ qsa_status decode_step_impl(const qsa_config* cfg, int32_t batch, const int64_t*
     sw.counters = reinterpret_cast<int32_t*>(base + w.counters);
     sw.winners = reinterpret_cast<int32_t*>(base + w.winners);
     sw.cand = reinterpret_cast<uint2*>(base + w.cand);
+    sw.est = reinterpret_cast<float2*>(base + w.est);
+    sw.pre = reinterpret_cast<uint2*>(base + w.pre);
     cudaStream_t st = (cudaStream_t)stream;
     // Every argument is valid from here on. A caller whose scratch may hold
     // another call's state asks for the status header and the selection state
     // to be cleared first.
     if (clear_state)
-        TRY(cuda_check(cudaMemsetAsync(ws, 0, qsa::decode_state_bytes(batch), st), "decode state clear"));
+        TRY(cuda_check(cudaMemsetAsync(ws, 0, qsa::decode_state_bytes(batch, L.kv_heads), st), "decode state clear"));
+    if (qsa::g_decode_kernel.load(std::memory_order_relaxed) == 0 && qsa::decode_step_supported(L)) {
+        qsa::StepSync sy{};
+        sy.arrive = reinterpret_cast<int32_t*>(base + w.sync);
+        sy.ready = sy.arrive + batch;
+        sy.fin = sy.ready + batch;
+        sy.done = sy.fin + batch;
+        sy.part = reinterpret_cast<float*>(base + w.part);
+        TRY(cuda_check(qsa::launch_decode_step(L, batch, pos, q, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
+                                               pooled, cap, rms_w, scores, sw, sy, sel, nsel, out, status, q8, hot,
+                                               st),
+                       "decode step"));
+        if (!hot) return QSA_OK;
+        return cuda_check(qsa::launch_install_hot(L, batch, pos, cap, sel, nsel, k_cache, v_cache, hot->k, hot->v,
+                                                  hot->tags, hot->blocks, st),
+                          "hot-cache install");
+    }
     TRY(cuda_check(qsa::launch_decode_score(L, batch, pos, k, v, idx_q, idx_k, k_cache, v_cache, idx_k_cache,
                                             pooled, cap, rms_w, scores, sw, status, q8, hot, st),
                    "decode score"));
@@ -694,7 +725,8 @@ int decode_step_cleared(const qsa_config* cfg, int32_t batch, const int64_t* pos
                             rms_w, out, sel_out, nsel_out, ws, ws_bytes, stream, nullptr, nullptr, true);
 }
 
-size_t decode_state_bytes(int batch) {
-    return kWsHeader + align_up((size_t)batch * 2048 * 4) + align_up((size_t)batch * 4 * 4);
+size_t decode_state_bytes(int batch, int kv_heads) {
+    return kWsHeader + align_up((size_t)batch * 2048 * 4) + align_up((size_t)batch * 4 * 4) +
+           align_up((size_t)batch * step_sync_words(kv_heads) * 4) + align_up((size_t)batch * 8);
 }
 }  // namespace qsa

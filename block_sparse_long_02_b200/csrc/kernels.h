@@ -164,11 +164,14 @@ struct Q8Caches {
 
 // decode.cu. Per-sequence selection state in the decode workspace.
 constexpr int kDecodeCand = 4096;  // candidates of the threshold digit kept for the final pick
+constexpr int kDecodePre = 4096;  // blocks the step kernel's score pass can list per sequence
 struct DecodeSelWs {
     uint32_t* hist;     // [batch][2048] histogram of the scores' level-1 key digit
-    int32_t* counters;  // [batch][4]: sure winners, candidates, finished CTAs
+    int32_t* counters;  // [batch][4]: sure winners, candidates, finished CTAs, listed blocks
     int32_t* winners;   // [batch][k_B]
     uint2* cand;        // [batch][kDecodeCand] (key, block)
+    float2* est;        // [batch] (last k-th score / its query's summed head norms, this query's sum)
+    uint2* pre;         // [batch][kDecodePre] (key, block) of the blocks listed by the score pass
 };
 int decode_select_ctas(int batch);
 // Sparse attention (a6 + a7) on tcgen05 with TMA block gathers; `status` (a
@@ -181,9 +184,9 @@ cudaError_t launch_sparse_attention_tc(const LayerDims& L, int batch, const uint
                                        cudaStream_t st);
 void set_attention_fault_injection(int mode, uint64_t wait_ns);
 // Bytes at the start of a decode workspace (status header, histograms,
-// counters) that must be zero when a decode step starts; each step leaves
-// them zero.
-size_t decode_state_bytes(int batch);
+// counters, step synchronisation) that must be zero when a decode step
+// starts; each step leaves them zero.
+size_t decode_state_bytes(int batch, int kv_heads);
 // qsa_decode_step on a workspace whose state bytes may hold anything (another
 // call's leftovers): checks every argument first, then clears the state bytes
 // on `stream`, then launches the step. A bad argument returns its error status
@@ -201,5 +204,28 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
                                  const float* scores, DecodeSelWs sw, int32_t* sel, int32_t* nsel,
                                  int32_t* status, cudaStream_t st);
+
+// The decode step as one persistent kernel (decode.cu): inter-CTA state in the
+// decode workspace, zero between steps.
+constexpr int kStepSplitCap = 16;  // attention CTAs per (sequence, kv head)
+struct StepSync {
+    int32_t* arrive;  // [batch] CTAs whose histogram counts are in
+    int32_t* ready;   // [batch] 1 once the sequence's selection is written
+    int32_t* fin;     // [batch] CTAs done with the step
+    int32_t* done;    // [batch][kv_heads] attention CTAs whose partial state is written
+    float* part;      // [batch][kv_heads][kStepSplitCap][G * 128 + 2 G] partial states (o, m, l)
+    uint64_t wait_ns; // bound of every inter-CTA wait
+    int32_t inject;   // fault injection: CTA (0, 0) withholds its arrival
+};
+// int32 words of StepSync state per sequence (arrive, ready, fin, done[kv_heads]).
+inline size_t step_sync_words(int kv_heads) { return 3 + (size_t)kv_heads; }
+bool decode_step_supported(const LayerDims& L);
+cudaError_t launch_decode_step(const LayerDims& L, int batch, const int64_t* pos, const uint16_t* q,
+                               const uint16_t* k, const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
+                               uint16_t* kc, uint16_t* vc, uint16_t* idx_k_cache, uint16_t* pooled, int64_t cap,
+                               const float* rms_w, float* scores, DecodeSelWs sw, StepSync sy, int32_t* sel,
+                               int32_t* nsel, uint16_t* out, int32_t* status, const Q8Caches* q8,
+                               const HotCache* hot, cudaStream_t st);
+void set_decode_fault_injection(int mode, uint64_t wait_ns);
 
 }  // namespace qsa

@@ -381,6 +381,22 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
                            const float* rms_w, qsa_bf16* out, int32_t* sel_out, int32_t* nsel_out,
                            void* ws, size_t ws_bytes, qsa_stream stream);
 
+/* Which kernels run a decode step (qsa_decode_step, _q8, _offload, _noalloc;
+ * process-wide):
+ *   0: one persistent kernel per step, one CTA of 512 threads per
+ *      SM, X = max(1, SMs / batch) CTAs per sequence. Each sequence's CTAs
+ *      append the token and score their slices of the pooled keys, meet at a
+ *      counter in the workspace once the score histogram is complete, select
+ *      (the last CTA to finish its scan resolves the pick and publishes it with
+ *      a release flag), then attend their splits of the selection and combine
+ *      them. CTAs only wait for CTAs of the same sequence, all resident at
+ *      once; every wait is bounded (10 s) and reports QSA_ERR_TIMEOUT in the
+ *      workspace status. Runs q_heads / kv_heads <= 8; larger groups use 1.
+ *   1 (default): three kernels per step (scores, selection, attention).
+ * Both give the same selection; outputs agree up to fp32 summation order.
+ * Returns QSA_ERR_INVALID_ARG for another value. Launches nothing. */
+qsa_status qsa_set_decode_kernel(int32_t kernel);
+
 /* Bytes of the fixed device scratch array behind qsa_decode_step_noalloc. */
 #define QSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 
@@ -454,6 +470,13 @@ uint64_t qsa_launch_count(void);
  *           key tiles of each CTA's first group of queries are withheld; the
  *           timeout is recorded in the workspace passed to that call (none is
  *           recorded without one) and the outputs it leaves are incomplete.
+ *   mode 4: the same for the decode steps' one-kernel path (qsa_decode_step,
+ *           _q8, _offload with qsa_set_decode_kernel(0)): CTA 0 of sequence 0
+ *           withholds its arrival after the score stream, so the other CTAs of
+ *           that sequence (when the step scores, p / r > k_B) wait for it until
+ *           wait_seconds have passed, record QSA_ERR_TIMEOUT and skip the rest
+ *           of the step. The outputs of sequence 0 are then incomplete, and the
+ *           workspace must be zeroed before its next step.
  * Returns QSA_ERR_INVALID_ARG for another mode or wait. */
 qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds);
 

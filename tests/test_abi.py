@@ -65,9 +65,10 @@ def test_null_and_capacity_errors_launch_nothing(qsa):
 
 def test_fault_injection_arguments_are_validated(qsa):
     """Host-side checks of the failure-path switch (no device work)."""
-    for mode, wait, ok in [(4, 0.1, False), (-1, 0.1, False), (1, 0.0, False), (1, 11.0, False),
-                           (1, float("nan"), False), (2, 0.0, False), (3, 0.0, False), (1, 0.5, True),
-                           (2, 0.5, True), (3, 0.5, True), (0, 0.0, True)]:
+    for mode, wait, ok in [(5, 0.1, False), (-1, 0.1, False), (1, 0.0, False), (1, 11.0, False),
+                           (1, float("nan"), False), (2, 0.0, False), (3, 0.0, False), (4, 0.0, False),
+                           (4, 10.5, False), (1, 0.5, True), (2, 0.5, True), (3, 0.5, True), (4, 0.5, True),
+                           (0, 0.0, True)]:
         if ok:
             qsa.qsa_set_fault_injection(mode, wait)
         else:
@@ -166,3 +167,14 @@ def test_attention_kernel_switch_is_validated(qsa):
             qsa.qsa_set_attention_kernel(k)
         assert e.value.status == 1
     qsa.qsa_set_attention_kernel(0)
+
+
+def test_decode_kernel_switch_is_validated(qsa):
+    """Host-side check of the decode-step kernel switch (no device work)."""
+    for k in (qsa.DECODE_THREE_KERNELS, qsa.DECODE_STEP_KERNEL):
+        qsa.qsa_set_decode_kernel(k)
+    for k in (-1, 2):
+        with pytest.raises(qsa.QSAError) as e:
+            qsa.qsa_set_decode_kernel(k)
+        assert e.value.status == 1
+    qsa.qsa_set_decode_kernel(1)

@@ -31,6 +31,15 @@ def kernel(request, qsa):
     qsa.qsa_set_attention_kernel(0)
 
 
+@pytest.fixture(params=[0, 1], ids=["step_kernel", "three_kernels"])
+def decode_kernel(request, qsa):
+    """Runs a decode test with each decode path: one persistent step kernel,
+    and the three kernels (scores, selection, attention)."""
+    qsa.qsa_set_decode_kernel(request.param)
+    yield request.param
+    qsa.qsa_set_decode_kernel(1)
+
+
 def _layer(qsa, w, cap, **over):
     from block_sparse_long_02_b200.layer import QSALayer
 
@@ -343,13 +352,13 @@ def _decode_run(qsa, w, starts, steps, check=True):
     return L
 
 
-def test_decode_steps_match_oracle(qsa):
+def test_decode_steps_match_oracle(qsa, decode_kernel):
     w = synth.Workload(name="t", n=777, batch=2, decode_steps=12, prefill=False, K=128, q_heads=16,
                        kv_heads=2, base_seed=0xF0, n_needles_decode=3)
     _decode_run(qsa, w, [777, 782], 12)
 
 
-def test_decode_short_context_and_capacity_flag(qsa):
+def test_decode_short_context_and_capacity_flag(qsa, decode_kernel):
     w = synth.Workload(name="t", n=0, batch=1, decode_steps=9, prefill=False, K=16, q_heads=8,
                        kv_heads=2, base_seed=0xF1)
     L = _decode_run(qsa, w, [0], 9)
@@ -529,7 +538,7 @@ def test_forced_timeout_is_reported_and_the_context_survives(qsa):
         check_selection(g[i], gn[i], ref["scores"], tol, o.k_blocks, f"row {i}")
 
 
-def test_decode_graph_replay_matches_eager(qsa):
+def test_decode_graph_replay_matches_eager(qsa, decode_kernel):
     """Decode steps captured into one CUDA graph and replayed give the same
     outputs, bit for bit, and the same caches as the eager calls (the kernels'
     programmatic dependencies become graph edges)."""
@@ -634,7 +643,7 @@ def test_prefill_with_fp8_caches_matches_oracle(qsa, q_heads, kv_heads):
         assert np.abs(g_lse[i] - ref_lse).max() <= LSE_ATOL, i
 
 
-def test_decode_steps_with_fp8_caches_match_oracle(qsa):
+def test_decode_steps_with_fp8_caches_match_oracle(qsa, decode_kernel):
     """Decode on fp8 caches, step by step across block boundaries: the appended
     K/V rows and each newly pooled block are quantized exactly as the oracle
     does; the selection is the oracle's on the fp8 pooled keys (near-ties
@@ -693,7 +702,7 @@ def test_decode_steps_with_fp8_caches_match_oracle(qsa):
 
 # ----------------------------------------------------------------------------- host-offloaded K/V
 @pytest.mark.parametrize("n0,S,H,batch", [(9002, 8, 97, 2), (4097, 6, 61, 24)])
-def test_decode_offload_matches_hbm_decode_bit_for_bit(qsa, n0, S, H, batch):
+def test_decode_offload_matches_hbm_decode_bit_for_bit(qsa, n0, S, H, batch, decode_kernel):
     """K/V caches in pinned host memory with a small direct-mapped HBM hot
     cache (a prime number of slots, so selected blocks collide): every step's
     selection and output match the oracle on sampled sequences and equal the
