@@ -33,6 +33,17 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
     return v;
 }
 
+// cp.async of 16 bytes (zero-filled when !valid) with an L2 cache policy.
+__device__ __forceinline__ void cp_async16_zfill_hint(uint32_t dst, const void* src, bool valid, uint64_t pol) {
+    const int sz = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(dst), "l"(src), "r"(sz),
+                 "l"(pol));
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+    return pol;
+}
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -316,6 +327,9 @@ __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pr
         // Stage layout: piece i (0..7) of lane l at i * 512 + l * 16 (conflict-free
         // 16-byte accesses); each lane reads back only the pieces it copied.
         const uint32_t wring = smem_u32(ring) + (uint32_t)(warp * RING * 4096 + lane * 16);
+        // The pooled keys are read once per step: first out of L2, so that what
+        // the selection and the attention reuse (their code included) stays.
+        const uint64_t pol = l2_evict_first_policy();
         auto issue = [&](int64_t gb, int stage) {
             const int64_t b0 = gb + g, b1 = b0 + 8;
             const uint16_t* ra = keys + (size_t)(b0 < hi ? b0 : 0) * kIdxDim + 8 * t;
@@ -323,8 +337,8 @@ __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pr
             const uint32_t d = wring + (uint32_t)(stage * 4096);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                cp_async16_zfill(d + i * 512, ra + 32 * i, b0 < hi);
-                cp_async16_zfill(d + (4 + i) * 512, rb + 32 * i, b1 < hi);
+                cp_async16_zfill_hint(d + i * 512, ra + 32 * i, b0 < hi, pol);
+                cp_async16_zfill_hint(d + (4 + i) * 512, rb + 32 * i, b1 < hi, pol);
             }
             cp_async_commit();
         };
@@ -466,6 +480,7 @@ struct DecSelSmem {
     uint32_t wsum[NW];
     unsigned long long base;
     int32_t n_win, n_cand, n_l3, bin, above, last;
+    uint32_t kth_key;  // key of the k_B-th selected block (0: not known)
 };
 static_assert(sizeof(SelSmem) <= sizeof(DecSelSmem), "the row-selection fallback reuses this shared memory");
 
@@ -527,6 +542,7 @@ __device__ __noinline__ void select_tail(uint8_t* raw, const float* row, int64_t
                                          int32_t* status) {
     DecSelSmem& sm = *reinterpret_cast<DecSelSmem*>(raw);
     const int tid = threadIdx.x;
+    if (tid == 0) sm.kth_key = 0u;
     for (int c = tid; c < nc; c += T) atomicAdd(&sm.hist[dec_digit2(sm.cand_key[c])], 1u);
     find_bin(sm, BINS, need1);
     const uint32_t b2 = sm.bin;
@@ -563,6 +579,7 @@ __device__ __noinline__ void select_tail(uint8_t* raw, const float* row, int64_t
             const uint32_t ky = sm.cand_key[y];
             rk += (ky > kx || (ky == kx && sm.cand_idx[y] < ix)) ? 1u : 0u;
         }
+        if (rk + 1 == need2) sm.kth_key = kx;  // the last one taken: the k-th largest
         if (rk < need2) {
             if (use_bm) {
                 atomicOr(&sm.u.bitmap[ix >> 5], 1u << (ix & 31));
@@ -700,6 +717,7 @@ __device__ __forceinline__ bool select_body(uint8_t* raw, const int64_t* __restr
     if (!sm.last) return false;
 
     // ---- the last CTA of the sequence (it acquired every CTA's lists) ----
+    if (tid == 0) sm.kth_key = 0u;
     const int n_win = __ldcg(cnt + 0), nc = __ldcg(cnt + 1);
     if (b1 == 0u || nc > kDecodeCand || nc > CAND || n_win != kB - (int)need1) {
         __syncthreads();
@@ -799,28 +817,14 @@ __device__ int cta_wait_at_least(const int32_t* p, int target, uint64_t wait_ns,
 }
 
 // The pre-filter estimate for the sequence's next step: this step's k-th
-// largest score (its smallest selected one) per unit of this step's summed
-// indexer-query head norms; zero (no list next step) unless both are positive.
-__device__ __noinline__ void record_estimate(uint8_t* raw, const float* row, const int32_t* out, int kB,
-                                             float2* est) {
-    DecSelSmem& sm = *reinterpret_cast<DecSelSmem*>(raw);
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    float m = INFINITY;
-    for (int j = threadIdx.x; j < kB; j += T) {
-        const int32_t b = __ldcg(out + j);
-        if (b >= 0) m = fminf(m, __ldcg(row + b));
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fminf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) sm.wsum[w] = __float_as_uint(m);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float kth = INFINITY;
-        for (int k = 0; k < NW; ++k) kth = fminf(kth, __uint_as_float(sm.wsum[k]));
-        const float y = __ldcg(&est->y);
-        est->x = (kth > 0.f && kth < INFINITY && y > 0.f) ? kth / y : 0.f;
-    }
-    __syncthreads();
+// largest score (sm.kth_key, left by select_tail) per unit of this step's
+// summed indexer-query head norms; zero (no list next step) unless both are
+// positive. Thread 0 only.
+__device__ __forceinline__ void record_estimate(const DecSelSmem& sm, float2* est) {
+    const uint32_t key = sm.kth_key;
+    const float kth = __uint_as_float(key & 0x80000000u ? key & 0x7fffffffu : ~key);  // (float_key inverted)
+    const float y = __ldcg(&est->y);
+    est->x = (key != 0u && kth > 0.f && kth < INFINITY && y > 0.f) ? kth / y : 0.f;
 }
 
 constexpr int kListPerThread = kDecodePre / T;  // listed entries a thread of select_listed holds
@@ -956,7 +960,7 @@ __global__ void __launch_bounds__(T, 1) decode_step_kernel(
     int32_t* __restrict__ sel, int32_t* __restrict__ nsel, uint16_t* __restrict__ out, int32_t* __restrict__ status,
     Q8Caches q8, HotCache hot) {
     extern __shared__ __align__(128) uint8_t dsm[];
-    __shared__ int s_last, s_wait, s_done;  // (each written by thread 0, read by all after a barrier)
+    __shared__ int s_wait, s_done;  // (each written by thread 0, read by all after a barrier)
     const int s = blockIdx.y, x = blockIdx.x, X = (int)gridDim.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -973,22 +977,24 @@ __global__ void __launch_bounds__(T, 1) decode_step_kernel(
     // picked by the full selection.
     int ready;
     if (nvis > kB) {
-        // Arrive; the last CTA (every count and listed block is in) picks
-        // from the list when it holds the answer, else asks for the full path.
+        // The scoring CTAs arrive; CTA 0 (it scores only when alone) waits for
+        // them and picks from the list when it holds the answer, else asks
+        // every CTA for the full selection. (CTA 0 of every step is the same
+        // kind of CTA, so the pick's code tends to be warm in its caches.)
         __syncthreads();
-        if (tid == 0)
-            s_last = (sy.inject && s == 0 && x == 0) ? 0 : atom_add_acq_rel(sy.arrive + s, 1) == X - 1;
-        __syncthreads();
-        if (s_last) {
+        if (x > 0 && tid == 0 && !(sy.inject && s == 0 && x == X - 1)) red_add_release(sy.arrive + s, 1);
+        if (x == 0 && (X == 1 || cta_wait_at_least(sy.arrive + s, X - 1, sy.wait_ns, &s_wait, status))) {
             const int npre = __ldcg(cnt + 3);
             bool picked = false;
             if (npre >= kB && npre <= kDecodePre)
                 picked = select_listed(dsm, row, nvis, kB, npre, sw.pre + (size_t)s * kDecodePre, sel + (size_t)s * kB,
                                        nsel + s, status);
             if (picked) {
-                record_estimate(dsm, row, sel + (size_t)s * kB, kB, sw.est + s);
+                if (tid == 0) {
+                    record_estimate(*reinterpret_cast<const DecSelSmem*>(dsm), sw.est + s);
+                    cnt[3] = 0;  // (the other counters are untouched: zero)
+                }
                 for (int b = tid; b < BINS; b += T) sw.hist[(size_t)s * BINS + b] = 0u;
-                if (tid == 0) cnt[3] = 0;  // (the other counters are untouched: zero)
                 __syncthreads();
             }
             if (tid == 0) st_release(sy.ready + s, picked ? 1 : 2);
@@ -996,8 +1002,10 @@ __global__ void __launch_bounds__(T, 1) decode_step_kernel(
         ready = cta_wait_at_least(sy.ready + s, 1, sy.wait_ns, &s_wait, status);
         if (ready == 2) {  // every CTA scans its slice; the last to finish resolves
             if (select_body(dsm, pos, cap, r, kB, scores, sw, sel, nsel, status)) {
-                record_estimate(dsm, row, sel + (size_t)s * kB, kB, sw.est + s);
-                if (tid == 0) st_release(sy.ready + s, 3);
+                if (tid == 0) {
+                    record_estimate(*reinterpret_cast<const DecSelSmem*>(dsm), sw.est + s);
+                    st_release(sy.ready + s, 3);
+                }
             }
             __syncthreads();
             ready = cta_wait_at_least(sy.ready + s, 3, sy.wait_ns, &s_wait, status);

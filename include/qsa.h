@@ -471,12 +471,13 @@ uint64_t qsa_launch_count(void);
  *           timeout is recorded in the workspace passed to that call (none is
  *           recorded without one) and the outputs it leaves are incomplete.
  *   mode 4: the same for the decode steps' one-kernel path (qsa_decode_step,
- *           _q8, _offload with qsa_set_decode_kernel(0)): CTA 0 of sequence 0
- *           withholds its arrival after the score stream, so the other CTAs of
- *           that sequence (when the step scores, p / r > k_B) wait for it until
- *           wait_seconds have passed, record QSA_ERR_TIMEOUT and skip the rest
- *           of the step. The outputs of sequence 0 are then incomplete, and the
- *           workspace must be zeroed before its next step.
+ *           _q8, _offload with qsa_set_decode_kernel(0)): the last CTA of
+ *           sequence 0 withholds its arrival after the score stream, so that
+ *           sequence's CTAs (when it has more than one and the step scores,
+ *           p / r > k_B) wait until wait_seconds have passed, record
+ *           QSA_ERR_TIMEOUT and skip the rest of the step. The outputs of
+ *           sequence 0 are then incomplete, and the workspace must be zeroed
+ *           before its next step.
  * Returns QSA_ERR_INVALID_ARG for another mode or wait. */
 qsa_status qsa_set_fault_injection(int32_t mode, double wait_seconds);
 

@@ -114,8 +114,8 @@ def test_step_kernel_and_three_kernels_select_the_same_blocks(qsa, n, batch):
 
 def test_step_kernel_forced_timeout_is_reported_and_the_context_survives(qsa):
     """Failure path of the step kernel's inter-CTA waits, without a GPU fault:
-    fault injection mode 4 makes CTA 0 of sequence 0 withhold its arrival after
-    the score stream; that sequence's CTAs wait 0.25 s, record QSA_ERR_TIMEOUT
+    fault injection mode 4 makes the last CTA of sequence 0 withhold its arrival
+    after the score stream; that sequence's CTAs wait 0.25 s, record QSA_ERR_TIMEOUT
     and skip the rest of the step, while sequence 1 completes normally. After
     the workspace is zeroed the next step is normal and matches the oracle."""
     n, batch = 9001, 2
