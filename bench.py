@@ -199,7 +199,7 @@ def host_copy_gbs(dev, stream) -> float:
 
 # The sources that define each stage's kernels (their code and launch shape).
 STAGE_SOURCES = {
-    "attention": ("attention.cu", "common.cuh"),
+    "attention": ("attention.cu", "attend.cuh", "common.cuh"),
     "topk": ("indexer_tc.cu", "topk.cu", "select.cuh", "common.cuh"),
 }
 
