@@ -41,7 +41,7 @@ __device__ __forceinline__ void cp_async16_zfill_hint(uint32_t dst, const void* 
 }
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(pol));
     return pol;
 }
 __device__ __forceinline__ uint64_t global_ns() {
@@ -121,7 +121,7 @@ __device__ __forceinline__ uint32_t dec_digit2(uint32_t key) { return (key >> 9)
 // RING > 0, bf16 keys: each warp streams its groups of 16 keys through RING
 // 4 KB stages of shared memory at `ring` with cp.async (RING - 1 groups in
 // flight without holding registers) instead of a register double buffer.)
-template <bool Q8, int NWARPS, int RING = 0>
+template <bool Q8, int NWARPS, int RING = 0, bool STREAM = true>
 __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pre, int32_t* pre_count,
     const int64_t* __restrict__ pos, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
     const uint16_t* __restrict__ idx_q, const uint16_t* __restrict__ idx_k, uint16_t* __restrict__ kc,
@@ -254,25 +254,28 @@ __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pr
     float* dst = scores + (size_t)s * pcap;
     // bf16: four 16-byte pieces of each row; fp8: two (16 codes each), and the
     // rows' scales.
+    // STREAM: the batch's pooled keys outsize the L2, so they are read with
+    // streaming loads (ld.global.cs, evict-first) and what the selection and
+    // the attention reuse, their code included, stays in L2; otherwise plain
+    // loads, which let the keys stay in L2 for the next step.
+    auto ldk = [](const void* a) {
+        return STREAM ? __ldcs(reinterpret_cast<const uint4*>(a)) : __ldg(reinterpret_cast<const uint4*>(a));
+    };
     auto load = [&](int64_t base, uint4 (&ra)[4], uint4 (&rb)[4], float& sa_, float& sb_) {
         const int64_t b0 = base + g, b1 = b0 + 8;
         if constexpr (Q8) {
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                ra[i] = b0 < hi ? __ldg(reinterpret_cast<const uint4*>(keys8 + (size_t)b0 * kIdxDim + 64 * i + 16 * t))
-                                : make_uint4(0u, 0u, 0u, 0u);
-                rb[i] = b1 < hi ? __ldg(reinterpret_cast<const uint4*>(keys8 + (size_t)b1 * kIdxDim + 64 * i + 16 * t))
-                                : make_uint4(0u, 0u, 0u, 0u);
+                ra[i] = b0 < hi ? ldk(keys8 + (size_t)b0 * kIdxDim + 64 * i + 16 * t) : make_uint4(0u, 0u, 0u, 0u);
+                rb[i] = b1 < hi ? ldk(keys8 + (size_t)b1 * kIdxDim + 64 * i + 16 * t) : make_uint4(0u, 0u, 0u, 0u);
             }
             sa_ = (t == 0 && b0 < hi) ? __ldg(kscale + b0) : 0.f;
             sb_ = (t == 0 && b1 < hi) ? __ldg(kscale + b1) : 0.f;
         } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                ra[i] = b0 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b0 * kIdxDim + 32 * i + 8 * t))
-                                : make_uint4(0u, 0u, 0u, 0u);
-                rb[i] = b1 < hi ? __ldg(reinterpret_cast<const uint4*>(keys + (size_t)b1 * kIdxDim + 32 * i + 8 * t))
-                                : make_uint4(0u, 0u, 0u, 0u);
+                ra[i] = b0 < hi ? ldk(keys + (size_t)b0 * kIdxDim + 32 * i + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
+                rb[i] = b1 < hi ? ldk(keys + (size_t)b1 * kIdxDim + 32 * i + 8 * t) : make_uint4(0u, 0u, 0u, 0u);
             }
         }
     };
@@ -452,7 +455,7 @@ __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pr
         if (hist[b]) atomicAdd(&hist_g[(size_t)s * 2048 + b], hist[b]);
 }
 
-template <bool Q8>
+template <bool Q8, bool STREAM>
 __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     const int64_t* __restrict__ pos, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
     const uint16_t* __restrict__ idx_q, const uint16_t* __restrict__ idx_k, uint16_t* __restrict__ kc,
@@ -460,7 +463,7 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     int64_t cap, const float* __restrict__ rms_w, int kv_heads, int r, int kB, double eps, RopeTable rt,
     float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status, Q8Caches q8,
     HotCache hot) {
-    score_body<Q8, DS_WARPS>(nullptr, nullptr, nullptr, nullptr, pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache, pooled, cap, rms_w, kv_heads, r, kB, eps,
+    score_body<Q8, DS_WARPS, 0, STREAM>(nullptr, nullptr, nullptr, nullptr, pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache, pooled, cap, rms_w, kv_heads, r, kB, eps,
                              rt, scores, hist_g, status, q8, hot);
 }
 
@@ -1129,13 +1132,17 @@ int decode_score_ctas(int batch, bool q8) {
     int dev = 0, sms = 148, per_sm = 1;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const cudaError_t e = q8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<true>,
+    const cudaError_t e = q8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<true, true>,
                                                                              DS_THREADS, 0)
-                             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<false>,
+                             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_score_kernel<false, true>,
                                                                              DS_THREADS, 0);
     if (e != cudaSuccess || per_sm < 1) per_sm = 1;
     return std::max(1, per_sm * sms / std::max(batch, 1));
 }
+
+// Pooled-key bytes of a batch at its capacity above which the score stream
+// reads them as a stream (evict-first) rather than letting them stay in L2.
+constexpr double kStreamKeyBytes = 96e6;
 
 cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* pos, const uint16_t* k,
                                 const uint16_t* v, const uint16_t* idx_q, const uint16_t* idx_k,
@@ -1143,14 +1150,16 @@ cudaError_t launch_decode_score(const LayerDims& L, int batch, const int64_t* po
                                 int64_t cap, const float* rms_w, float* scores, DecodeSelWs sw,
                                 int32_t* status, const Q8Caches* q8, const HotCache* hot, cudaStream_t st) {
     const dim3 grid((unsigned)decode_score_ctas(batch, q8 != nullptr), (unsigned)batch);
+    const bool stream = (double)batch * (double)(cap / L.r) * kIdxDim * (q8 ? 1 : 2) > kStreamKeyBytes;
     note_launch();
-    if (q8)
-        return launch_pdl(decode_score_kernel<true>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,
-                          idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist,
-                          status, *q8, HotCache{});
-    return launch_pdl(decode_score_kernel<false>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,
-                      idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist,
-                      status, Q8Caches{}, hot ? *hot : HotCache{});
+#define QSA_SCORE(Q8_, S_, Q8C_, HOT_)                                                                                \
+    launch_pdl(decode_score_kernel<Q8_, S_>, grid, dim3(DS_THREADS), 0, st, pos, k, v, idx_q, idx_k, kc, vc,          \
+               idx_k_cache, pooled, cap, rms_w, L.kv_heads, L.r, L.kB, L.rms_eps, L.rope, scores, sw.hist, status,    \
+               Q8C_, HOT_)
+    const HotCache hc = hot ? *hot : HotCache{};
+    if (q8) return stream ? QSA_SCORE(true, true, *q8, HotCache{}) : QSA_SCORE(true, false, *q8, HotCache{});
+    return stream ? QSA_SCORE(false, true, Q8Caches{}, hc) : QSA_SCORE(false, false, Q8Caches{}, hc);
+#undef QSA_SCORE
 }
 
 cudaError_t launch_decode_select(const LayerDims& L, int batch, const int64_t* pos, int64_t cap,
