@@ -308,25 +308,58 @@ __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pr
             }
         }
     };
-    if constexpr (RING > 0 && !Q8) {
-        // The pre-filter threshold tau: the last step's k-th score per unit of
-        // its query's summed head norms, times this query's sum, times
-        // kPreFactor. Blocks scoring at least tau are also listed (key, block);
-        // when the list holds at least k_B of them it holds every top-k_B
-        // block, ties included, whatever tau was.
-        float tau = 0.f;
-        if (est) {
-            const float qsum = (qnorm[0] + qnorm[1]) + (qnorm[2] + qnorm[3]);
-            const float ratio = __ldcg(&est[s].x);
-            tau = ratio > 0.f ? ratio * qsum * kPreFactor : 0.f;
-            if (x == 0 && tid == 0) est[s].y = qsum;  // (the first scoring CTA)
+    // The pre-filter threshold tau: the last step's k-th score per unit of its
+    // query's summed head norms, times this query's sum, times kPreFactor.
+    // Blocks scoring at least tau are also listed (key, block); when the list
+    // holds at least k_B of them it holds every top-k_B block, ties included,
+    // whatever tau was. The CTA's listed blocks gather in shared memory (after
+    // the ring, if any) and go to the sequence's list with one reservation.
+    float tau = 0.f;
+    if (est) {
+        const float qsum = (qnorm[0] + qnorm[1]) + (qnorm[2] + qnorm[3]);
+        const float ratio = __ldcg(&est[s].x);
+        tau = ratio > 0.f ? ratio * qsum * kPreFactor : 0.f;
+        if (x == 0 && tid == 0) est[s].y = qsum;  // (the first scoring CTA)
+    }
+    const bool listing = est && tau > 0.f;  // (NaN: no list; est is null without a list in shared memory)
+    uint2* clist = est ? reinterpret_cast<uint2*>(ring + NWARPS * RING * 4096) : nullptr;
+    if (tid == 0) n_clist = 0;
+    __syncthreads();
+    auto list = [&](int64_t gb, float sa, float sb) {  // warp-aggregated appends (every lane calls)
+        const int64_t b0 = gb + g, b1 = b0 + 8;
+        const bool ha = t == 0 && b0 < hi && sa >= tau, hb = t == 0 && b1 < hi && sb >= tau;
+        const uint32_t ba = __ballot_sync(0xffffffffu, ha), bb = __ballot_sync(0xffffffffu, hb);
+        if (ba | bb) {
+            int at0 = 0;
+            if (lane == 0) at0 = atomicAdd(&n_clist, __popc(ba) + __popc(bb));
+            at0 = __shfl_sync(0xffffffffu, at0, 0);
+            const uint32_t below = (1u << lane) - 1u;
+            const int aa = at0 + __popc(ba & below), ab = at0 + __popc(ba) + __popc(bb & below);
+            if (ha && aa < kCtaList) clist[aa] = make_uint2(float_key(sa), (uint32_t)b0);
+            if (hb && ab < kCtaList) clist[ab] = make_uint2(float_key(sb), (uint32_t)b1);
         }
-        const bool listing = tau > 0.f;  // (NaN: no list)
-        // The CTA's listed blocks gather in shared memory after the ring and go
-        // to the sequence's list with one reservation at the end.
-        uint2* clist = reinterpret_cast<uint2*>(ring + NWARPS * RING * 4096);
-        if (tid == 0) n_clist = 0;
+    };
+    // After the stream: the CTA's histogram counts, and its list with one
+    // reservation (a CTA list that overflowed marks the sequence's list
+    // overflowed: the full selection runs).
+    auto finish = [&]() {
         __syncthreads();
+        for (int b = tid; b < 2048; b += DS_THREADS)
+            if (hist[b]) atomicAdd(&hist_g[(size_t)s * 2048 + b], hist[b]);
+        if (listing) {
+            const int n = n_clist;
+            if (tid == 0) clist_at = n > kCtaList ? -1 : (n ? atomicAdd(pre_count, n) : 0);
+            __syncthreads();
+            const int at = clist_at;
+            if (at < 0) {
+                if (tid == 0) atomicAdd(pre_count, kDecodePre + 1);
+            } else {
+                uint2* plist = pre + (size_t)s * kDecodePre;
+                for (int i = tid; i < n && at + i < kDecodePre; i += DS_THREADS) plist[at + i] = clist[i];
+            }
+        }
+    };
+    if constexpr (RING > 0 && !Q8) {
         // Stage layout: piece i (0..7) of lane l at i * 512 + l * 16 (conflict-free
         // 16-byte accesses); each lane reads back only the pieces it copied.
         const uint32_t wring = smem_u32(ring) + (uint32_t)(warp * RING * 4096 + lane * 16);
@@ -371,39 +404,10 @@ __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pr
             sa += __shfl_xor_sync(0xffffffffu, sa, 1);
             sb += __shfl_xor_sync(0xffffffffu, sb, 1);
             emit(base, sa, sb);
-            if (listing) {  // warp-aggregated appends of the blocks at or above tau
-                const int64_t b0 = base + g, b1 = b0 + 8;
-                const bool ha = t == 0 && b0 < hi && sa >= tau, hb = t == 0 && b1 < hi && sb >= tau;
-                const uint32_t ba = __ballot_sync(0xffffffffu, ha), bb = __ballot_sync(0xffffffffu, hb);
-                if (ba | bb) {
-                    int at0 = 0;
-                    if (lane == 0) at0 = atomicAdd(&n_clist, __popc(ba) + __popc(bb));
-                    at0 = __shfl_sync(0xffffffffu, at0, 0);
-                    const uint32_t below = (1u << lane) - 1u;
-                    const int aa = at0 + __popc(ba & below), ab = at0 + __popc(ba) + __popc(bb & below);
-                    if (ha && aa < kCtaList) clist[aa] = make_uint2(float_key(sa), (uint32_t)b0);
-                    if (hb && ab < kCtaList) clist[ab] = make_uint2(float_key(sb), (uint32_t)b1);
-                }
-            }
+            if (listing) list(base, sa, sb);
         }
         cp_async_wait<0>();
-        __syncthreads();
-        for (int b = tid; b < 2048; b += DS_THREADS)
-            if (hist[b]) atomicAdd(&hist_g[(size_t)s * 2048 + b], hist[b]);
-        if (listing) {
-            // One reservation for the CTA's list; a CTA list that overflowed
-            // marks the sequence's list overflowed (the full selection runs).
-            const int n = n_clist;
-            if (tid == 0) clist_at = n > kCtaList ? -1 : (n ? atomicAdd(pre_count, n) : 0);
-            __syncthreads();
-            const int at = clist_at;
-            if (at < 0) {
-                if (tid == 0) atomicAdd(pre_count, kDecodePre + 1);
-            } else {
-                uint2* plist = pre + (size_t)s * kDecodePre;
-                for (int i = tid; i < n && at + i < kDecodePre; i += DS_THREADS) plist[at + i] = clist[i];
-            }
-        }
+        finish();
         return;
     }
     uint4 ca[4], cb[4];
@@ -444,15 +448,14 @@ __device__ __forceinline__ void score_body(uint8_t* ring, float2* est, uint2* pr
             psb = nsb;
         }
         emit(base, sa, sb);
+        if (listing) list(base, sa, sb);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             ca[i] = na[i];
             cb[i] = nb[i];
         }
     }
-    __syncthreads();
-    for (int b = tid; b < 2048; b += DS_THREADS)
-        if (hist[b]) atomicAdd(&hist_g[(size_t)s * 2048 + b], hist[b]);
+    finish();
 }
 
 template <bool Q8, bool STREAM>
@@ -463,8 +466,9 @@ __global__ void __launch_bounds__(DS_THREADS) decode_score_kernel(
     int64_t cap, const float* __restrict__ rms_w, int kv_heads, int r, int kB, double eps, RopeTable rt,
     float* __restrict__ scores, uint32_t* __restrict__ hist_g, int32_t* __restrict__ status, Q8Caches q8,
     HotCache hot) {
-    score_body<Q8, DS_WARPS, 0, STREAM>(nullptr, nullptr, nullptr, nullptr, pos, k, v, idx_q, idx_k, kc, vc, idx_k_cache, pooled, cap, rms_w, kv_heads, r, kB, eps,
-                             rt, scores, hist_g, status, q8, hot);
+    score_body<Q8, DS_WARPS, 0, STREAM>(nullptr, nullptr, nullptr, nullptr, pos, k, v, idx_q, idx_k, kc, vc,
+                                        idx_k_cache, pooled, cap, rms_w, kv_heads, r, kB, eps, rt, scores, hist_g,
+                                        status, q8, hot);
 }
 
 constexpr int SEL_E = 8;                 // scores per thread per round of the scan
@@ -762,63 +766,6 @@ __device__ __forceinline__ bool select_body(uint8_t* raw, const int64_t* __restr
     return true;
 }
 
-__global__ void __launch_bounds__(T) decode_select_kernel(
-    const int64_t* __restrict__ pos, int64_t cap, int r, int kB, const float* __restrict__ scores,
-    DecodeSelWs sw, int32_t* __restrict__ sel, int32_t* __restrict__ nsel, int32_t* __restrict__ status) {
-    extern __shared__ __align__(16) uint8_t raw[];
-    pdl_wait();
-    pdl_trigger();
-    select_body(raw, pos, cap, r, kB, scores, sw, sel, nsel, status);
-}
-
-// ---------------------------------------------------------------------------
-// The decode step as one persistent kernel: grid (X, batch) of 512-thread
-// CTAs, one per SM, with the X CTAs of a sequence running its three phases
-// back to back and meeting only through counters in the workspace.
-//   1. a8, a3', a4: the score body above (CTA 0 appends and pools, the others
-//      score their slices and add their histogram counts).
-//   2. a5: each CTA arrives at the sequence's counter and waits for all X, so
-//      the histogram is complete; then the selection body above (every CTA
-//      scans its slice; the last to finish resolves the pick), whose resolver
-//      publishes the selection with a release store of the ready flag.
-//   3. a6, a7: after an acquire of the ready flag, CTA x takes kv head
-//      x % kv_heads and split x / kv_heads (at most kStepSplitCap splits per
-//      head); its first FA_WARPS warps attend their slices of the k_B + 1
-//      units (the selection entries, then the tail), their states are merged
-//      in shared memory into the CTA's partial (o, m, l) in the workspace, and
-//      the last split of a head to finish combines the partials into the
-//      output rows.
-// A sequence's CTAs only ever wait for each other, and all of them are
-// resident at once when batch x X CTAs fit on the GPU (X is chosen so); with
-// X = 1 nothing waits at all. Every wait is bounded by %globaltimer: one that
-// runs out flags QSA_ERR_TIMEOUT, and the CTA skips the rest of the step.
-constexpr int FS_WARPS = T / 32;  // warps of a step CTA: the score stream and the selection
-constexpr int FA_WARPS = 12;      // of which attend (each owns a WARP_SMEM ring)
-constexpr uint64_t kStepWaitNs = 10000000000ull;  // 10 s: the bound of every wait in normal use
-
-
-
-// Thread 0 waits (bounded) until *p >= target (acquire); every thread gets
-// the value it read, or 0 (and QSA_ERR_TIMEOUT flagged) when the wait ran out.
-__device__ int cta_wait_at_least(const int32_t* p, int target, uint64_t wait_ns, int* flag, int32_t* status) {
-    if (threadIdx.x == 0) {
-        int v = ld_acquire(p);
-        if (v < target) {
-            const uint64_t t0 = global_ns();
-            while ((v = ld_acquire(p)) < target && global_ns() - t0 < wait_ns) __nanosleep(100);
-        }
-        if (v < target) {
-            flag_status(status, 6 /* QSA_ERR_TIMEOUT */);
-            v = 0;
-        }
-        *flag = v;
-    }
-    __syncthreads();
-    const int v = *flag;
-    __syncthreads();
-    return v;
-}
-
 // The pre-filter estimate for the sequence's next step: this step's k-th
 // largest score (sm.kth_key, left by select_tail) per unit of this step's
 // summed indexer-query head norms; zero (no list next step) unless both are
@@ -891,6 +838,63 @@ __device__ __noinline__ bool select_listed(uint8_t* raw, const float* row, int64
     if (!fits) return false;
     select_tail(raw, row, nvis, kB, nc, need1, use_bm, per, out, nsel_s, status);
     return true;
+}
+
+__global__ void __launch_bounds__(T) decode_select_kernel(
+    const int64_t* __restrict__ pos, int64_t cap, int r, int kB, const float* __restrict__ scores,
+    DecodeSelWs sw, int32_t* __restrict__ sel, int32_t* __restrict__ nsel, int32_t* __restrict__ status) {
+    extern __shared__ __align__(16) uint8_t raw[];
+    pdl_wait();
+    pdl_trigger();
+    select_body(raw, pos, cap, r, kB, scores, sw, sel, nsel, status);
+}
+
+// ---------------------------------------------------------------------------
+// The decode step as one persistent kernel: grid (X, batch) of 512-thread
+// CTAs, one per SM, with the X CTAs of a sequence running its three phases
+// back to back and meeting only through counters in the workspace.
+//   1. a8, a3', a4: the score body above (CTA 0 appends and pools, the others
+//      score their slices and add their histogram counts).
+//   2. a5: each CTA arrives at the sequence's counter and waits for all X, so
+//      the histogram is complete; then the selection body above (every CTA
+//      scans its slice; the last to finish resolves the pick), whose resolver
+//      publishes the selection with a release store of the ready flag.
+//   3. a6, a7: after an acquire of the ready flag, CTA x takes kv head
+//      x % kv_heads and split x / kv_heads (at most kStepSplitCap splits per
+//      head); its first FA_WARPS warps attend their slices of the k_B + 1
+//      units (the selection entries, then the tail), their states are merged
+//      in shared memory into the CTA's partial (o, m, l) in the workspace, and
+//      the last split of a head to finish combines the partials into the
+//      output rows.
+// A sequence's CTAs only ever wait for each other, and all of them are
+// resident at once when batch x X CTAs fit on the GPU (X is chosen so); with
+// X = 1 nothing waits at all. Every wait is bounded by %globaltimer: one that
+// runs out flags QSA_ERR_TIMEOUT, and the CTA skips the rest of the step.
+constexpr int FS_WARPS = T / 32;  // warps of a step CTA: the score stream and the selection
+constexpr int FA_WARPS = 12;      // of which attend (each owns a WARP_SMEM ring)
+constexpr uint64_t kStepWaitNs = 10000000000ull;  // 10 s: the bound of every wait in normal use
+
+
+
+// Thread 0 waits (bounded) until *p >= target (acquire); every thread gets
+// the value it read, or 0 (and QSA_ERR_TIMEOUT flagged) when the wait ran out.
+__device__ int cta_wait_at_least(const int32_t* p, int target, uint64_t wait_ns, int* flag, int32_t* status) {
+    if (threadIdx.x == 0) {
+        int v = ld_acquire(p);
+        if (v < target) {
+            const uint64_t t0 = global_ns();
+            while ((v = ld_acquire(p)) < target && global_ns() - t0 < wait_ns) __nanosleep(100);
+        }
+        if (v < target) {
+            flag_status(status, 6 /* QSA_ERR_TIMEOUT */);
+            v = 0;
+        }
+        *flag = v;
+    }
+    __syncthreads();
+    const int v = *flag;
+    __syncthreads();
+    return v;
 }
 
 // One warp's slice [split of S] of the units of (sequence s, kv head g),
