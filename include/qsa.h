@@ -385,13 +385,17 @@ qsa_status qsa_decode_step(const qsa_config* cfg, int32_t batch, const int64_t* 
  * process-wide):
  *   0: one persistent kernel per step, one CTA of 512 threads per
  *      SM, X = max(1, SMs / batch) CTAs per sequence. Each sequence's CTAs
- *      append the token and score their slices of the pooled keys, meet at a
- *      counter in the workspace once the score histogram is complete, select
- *      (the last CTA to finish its scan resolves the pick and publishes it with
- *      a release flag), then attend their splits of the selection and combine
- *      them. CTAs only wait for CTAs of the same sequence, all resident at
- *      once; every wait is bounded (10 s) and reports QSA_ERR_TIMEOUT in the
- *      workspace status. Runs q_heads / kv_heads <= 8; larger groups use 1.
+ *      append the token and score their slices of the pooled keys, also
+ *      listing the blocks at or above a threshold estimated from the previous
+ *      step (kept per batch slot in the workspace). CTA 0 waits for the others
+ *      and, when the list holds between k_B and 4096 blocks (then it holds
+ *      every top-k_B block), picks from it alone; otherwise every CTA runs the
+ *      histogram selection. The pick is published with a release flag, then
+ *      the CTAs attend their splits of the selection and combine them. The
+ *      estimate affects speed only, never the result. CTAs only wait for CTAs
+ *      of the same sequence, all resident at once; every wait is bounded (10 s)
+ *      and reports QSA_ERR_TIMEOUT in the workspace status. Runs
+ *      q_heads / kv_heads <= 8; larger groups use 1.
  *   1 (default): three kernels per step (scores, selection, attention).
  * Both give the same selection; outputs agree up to fp32 summation order.
  * Returns QSA_ERR_INVALID_ARG for another value. Launches nothing. */
