@@ -68,6 +68,81 @@ class QSALayer:
         if mark:
             mark("attention")
 
+    def prefill_from_host(self, host_q: torch.Tensor, host_idx_q: torch.Tensor, host_k: torch.Tensor,
+                          host_v: torch.Tensor, host_idx_k: torch.Tensor, q_begin: int, nq: int,
+                          host_out: torch.Tensor, chunk: int = 131072) -> None:
+        """prefill of positions [q_begin, q_begin + nq) whose inputs and output
+        live in pinned host memory: host_q [batch][nq][q_heads][128], host_idx_q
+        [batch][nq][4][128], the new cache rows host_k, host_v
+        [batch][nq][kv_heads][128] and host_idx_k [batch][nq][128], and host_out
+        [batch][nq][q_heads][128] (rows before q_begin are already in the
+        caches). The positions go in chunks (multiples of r, the last one
+        ragged): chunk j's rows move to the device on one stream while chunk
+        j - 1 computes on the current stream, and its output returns on a third
+        stream while chunk j + 1 computes. Each chunk is the prefill call on a
+        double-buffered staging area, so the outputs equal prefill's bit for bit.
+        Returns when the work is queued; host_out is complete once the current
+        stream has synchronised."""
+        B, r = self.batch, self.cfg.r
+        chunk = max(r, min(chunk, nq) // r * r)
+        dev = self.device
+        bf = torch.bfloat16
+        cs = torch.cuda.current_stream(dev)
+        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        stage = [{"q": torch.empty(B, chunk, *host_q.shape[2:], dtype=bf, device=dev),
+                  "idx_q": torch.empty(B, chunk, *host_idx_q.shape[2:], dtype=bf, device=dev),
+                  "out": torch.empty(B, chunk, *host_out.shape[2:], dtype=bf, device=dev),
+                  "sel": torch.empty(B, chunk, self.cfg.k_blocks, dtype=torch.int32, device=dev),
+                  "nsel": torch.empty(B, chunk, dtype=torch.int32, device=dev)} for _ in range(2)]
+        for st in stage:  # the staging area is written on the side streams
+            for t in st.values():
+                t.record_stream(h2d)
+                t.record_stream(d2h)
+        computed, drained = [None, None], [None, None]  # per staging set: last compute / output copy
+        starts = list(range(0, nq, chunk))
+        cs_ready = torch.cuda.Event()
+        cs_ready.record(cs)
+        h2d.wait_event(cs_ready)  # the caches and staging exist before the first copy
+        for j, a in enumerate(starts):
+            m = min(chunk, nq - a)
+            st = stage[j % 2]
+            with torch.cuda.stream(h2d):
+                if computed[j % 2] is not None:  # chunk j - 2 has read this set
+                    h2d.wait_event(computed[j % 2])
+                p0 = q_begin + a
+                for s in range(B):
+                    self.k_cache[s, p0:p0 + m].copy_(host_k[s, a:a + m], non_blocking=True)
+                    self.v_cache[s, p0:p0 + m].copy_(host_v[s, a:a + m], non_blocking=True)
+                    self.idx_k_cache[s, p0:p0 + m].copy_(host_idx_k[s, a:a + m], non_blocking=True)
+                    st["q"][s, :m].copy_(host_q[s, a:a + m], non_blocking=True)
+                    st["idx_q"][s, :m].copy_(host_idx_q[s, a:a + m], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(h2d)
+            cs.wait_event(arrived)
+            if drained[j % 2] is not None:  # chunk j - 2's output has left this set
+                cs.wait_event(drained[j % 2])
+            q_in = st["q"] if m == chunk else st["q"][:, :m].contiguous()
+            iq_in = st["idx_q"] if m == chunk else st["idx_q"][:, :m].contiguous()
+            out = st["out"] if m == chunk else torch.empty(B, m, *host_out.shape[2:], dtype=bf, device=dev)
+            sel = st["sel"] if m == chunk else torch.empty(B, m, self.cfg.k_blocks, dtype=torch.int32, device=dev)
+            nsel = st["nsel"] if m == chunk else torch.empty(B, m, dtype=torch.int32, device=dev)
+            self.prefill(q_in, iq_in, p0, m, out, sel, nsel)
+            done = torch.cuda.Event()
+            done.record(cs)
+            computed[j % 2] = done
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done)
+                out.record_stream(d2h)
+                for s in range(B):
+                    host_out[s, a:a + m].copy_(out[s], non_blocking=True)
+                left = torch.cuda.Event()
+                left.record(d2h)
+            drained[j % 2] = left
+        # The current stream waits for the last output copies.
+        for ev in drained:
+            if ev is not None:
+                cs.wait_event(ev)
+
     def prefill_varlen(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin, nq, out: torch.Tensor,
                        sel: torch.Tensor, nsel: torch.Tensor, lse: Optional[torch.Tensor] = None,
                        stream=None) -> None:

@@ -1,7 +1,8 @@
 """Variable-length batched prefill (the *_varlen calls): three sequences with
 different query ranges (a whole prompt, a chunk against an existing cache, a
 short tail) in one call each, against the oracle row by row and against the
-single-range calls bit for bit."""
+single-range calls bit for bit. Also the prefill from pinned host memory with
+overlapped transfers (QSALayer.prefill_from_host) against the device prefill."""
 from __future__ import annotations
 
 import numpy as np
@@ -10,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from gpu_util import LSE_ATOL, bits, check_attention, check_selection, score_tol
+from gpu_util import LSE_ATOL, bits, check_attention, check_selection, dev_full, score_tol
 
 pytestmark = pytest.mark.gpu
 
@@ -115,3 +116,49 @@ def test_varlen_errors_launch_nothing(qsa):
         qsa.qsa_sparse_attention_varlen(cfg, t, [0, 0], [4, -1], t, t, 64, i32, i32, t)
     assert e.value.status == 1
     assert qsa.qsa_launch_count() == n0
+
+
+@pytest.mark.parametrize("q_begin", [0, 1000])
+def test_prefill_from_host_equals_prefill(q_begin):
+    """QSALayer.prefill_from_host (inputs and output in pinned host memory,
+    moved in chunks overlapped with the compute on side streams) gives the
+    device prefill's outputs and caches bit for bit: a ragged last chunk,
+    a batch of two, and a start after an existing cache."""
+    import block_sparse_long_02_b200 as m
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    n, B = 6007, 2
+    w = synth.Workload(name="pfh", n=n, batch=B, K=512, q_heads=32, kv_heads=4, base_seed=0x7A2F)
+    cfg = m.Config.of(w)
+    nq = n - q_begin
+    full = {nm: dev_full(w, nm, n, n) for nm in ("q", "k", "v", "idx_q", "idx_k")}
+
+    def layer():
+        L = QSALayer(cfg, B, n)
+        if q_begin:
+            for nm, c in (("k", L.k_cache), ("v", L.v_cache), ("idx_k", L.idx_k_cache)):
+                c.view(B, n, -1)[:, :q_begin] = full[nm][:, :q_begin]
+            L.compress(0, q_begin // cfg.r)
+        return L
+
+    La, Lb = layer(), layer()
+    for nm, c in (("k", La.k_cache), ("v", La.v_cache), ("idx_k", La.idx_k_cache)):
+        c.view(B, n, -1)[:, q_begin:] = full[nm][:, q_begin:]
+    q = full["q"][:, q_begin:].contiguous().view(B, nq, cfg.q_heads, 128)
+    iq = full["idx_q"][:, q_begin:].contiguous().view(B, nq, 4, 128)
+    out = torch.empty(B, nq, cfg.q_heads, 128, dtype=torch.bfloat16, device="cuda")
+    sel = torch.empty(B, nq, cfg.k_blocks, dtype=torch.int32, device="cuda")
+    nsel = torch.empty(B, nq, dtype=torch.int32, device="cuda")
+    La.prefill(q, iq, q_begin, nq, out, sel, nsel)
+
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    hq, hiq = pin(q), pin(iq)
+    hk = pin(full["k"][:, q_begin:].view(B, nq, cfg.kv_heads, 128))
+    hv = pin(full["v"][:, q_begin:].view(B, nq, cfg.kv_heads, 128))
+    hik = pin(full["idx_k"][:, q_begin:])
+    hout = torch.zeros(B, nq, cfg.q_heads, 128, dtype=torch.bfloat16).pin_memory()
+    Lb.prefill_from_host(hq, hiq, hk, hv, hik, q_begin, nq, hout, chunk=2048)
+    torch.cuda.synchronize()
+    assert torch.equal(hout, out.cpu())
+    for name in ("k_cache", "v_cache", "idx_k_cache", "pooled"):
+        assert torch.equal(getattr(La, name), getattr(Lb, name)), name
