@@ -6,6 +6,9 @@ calls in the order the layer runs them:
 
   prefill(q, idx_q, q_begin, nq):   qsa_compress_keys -> qsa_topk_blocks (fused)
                                     -> qsa_sparse_attention
+  prefill_from_host(...):           the same per chunk of positions, with the
+                                    host <-> device copies of the inputs and the
+                                    output overlapped on side streams
   decode_step(pos, q, k, v, idx_q, idx_k): qsa_decode_step
 
 Every step of the computation runs in libqsa.so; this class only owns memory
