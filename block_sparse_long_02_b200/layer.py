@@ -73,21 +73,24 @@ class QSALayer:
 
     def prefill_from_host(self, host_q: torch.Tensor, host_idx_q: torch.Tensor, host_k: torch.Tensor,
                           host_v: torch.Tensor, host_idx_k: torch.Tensor, q_begin: int, nq: int,
-                          host_out: torch.Tensor, chunk: int = 131072) -> None:
+                          host_out: torch.Tensor, chunk: int = 131072, first: int = 8192) -> None:
         """prefill of positions [q_begin, q_begin + nq) whose inputs and output
         live in pinned host memory: host_q [batch][nq][q_heads][128], host_idx_q
         [batch][nq][4][128], the new cache rows host_k, host_v
         [batch][nq][kv_heads][128] and host_idx_k [batch][nq][128], and host_out
         [batch][nq][q_heads][128] (rows before q_begin are already in the
-        caches). The positions go in chunks (multiples of r, the last one
-        ragged): chunk j's rows move to the device on one stream while chunk
-        j - 1 computes on the current stream, and its output returns on a third
-        stream while chunk j + 1 computes. Each chunk is the prefill call on a
+        caches). The positions go in chunks: chunk j's rows move to the device
+        on one stream while chunk j - 1 computes on the current stream, and its
+        output returns on a third stream while chunk j + 1 computes. The chunks
+        grow from `first` positions, doubling, to `chunk` and shrink the same way
+        at the end, so that only a small first transfer and a small last output
+        copy are not overlapped. Each chunk is the prefill call on a
         double-buffered staging area, so the outputs equal prefill's bit for bit.
         Returns when the work is queued; host_out is complete once the current
         stream has synchronised."""
         B, r = self.batch, self.cfg.r
         chunk = max(r, min(chunk, nq) // r * r)
+        plan = self.chunk_plan(nq, chunk, max(r, min(first, chunk) // r * r))
         dev = self.device
         bf = torch.bfloat16
         cs = torch.cuda.current_stream(dev)
@@ -102,12 +105,11 @@ class QSALayer:
                 t.record_stream(h2d)
                 t.record_stream(d2h)
         computed, drained = [None, None], [None, None]  # per staging set: last compute / output copy
-        starts = list(range(0, nq, chunk))
         cs_ready = torch.cuda.Event()
         cs_ready.record(cs)
         h2d.wait_event(cs_ready)  # the caches and staging exist before the first copy
-        for j, a in enumerate(starts):
-            m = min(chunk, nq - a)
+        a = 0
+        for j, m in enumerate(plan):
             st = stage[j % 2]
             with torch.cuda.stream(h2d):
                 if computed[j % 2] is not None:  # chunk j - 2 has read this set
@@ -141,10 +143,24 @@ class QSALayer:
                 left = torch.cuda.Event()
                 left.record(d2h)
             drained[j % 2] = left
+            a += m
         # The current stream waits for the last output copies.
         for ev in drained:
             if ev is not None:
                 cs.wait_event(ev)
+
+    @staticmethod
+    def chunk_plan(nq: int, chunk: int, first: int) -> list:
+        """Chunk sizes of prefill_from_host: first, 2 first, ... below chunk at
+        both ends (while they fit twice), chunk-sized ones between, and the
+        remainder as one more middle chunk; they sum to nq."""
+        ramp, c = [], first
+        while c < chunk and 2 * (sum(ramp) + c) <= nq:
+            ramp.append(c)
+            c *= 2
+        middle = nq - 2 * sum(ramp)
+        mids = [chunk] * (middle // chunk) + ([middle % chunk] if middle % chunk else [])
+        return ramp + mids + ramp[::-1]
 
     def prefill_varlen(self, q: torch.Tensor, idx_q: torch.Tensor, q_begin, nq, out: torch.Tensor,
                        sel: torch.Tensor, nsel: torch.Tensor, lse: Optional[torch.Tensor] = None,

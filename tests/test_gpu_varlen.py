@@ -118,12 +118,14 @@ def test_varlen_errors_launch_nothing(qsa):
     assert qsa.qsa_launch_count() == n0
 
 
-@pytest.mark.parametrize("q_begin", [0, 1000])
-def test_prefill_from_host_equals_prefill(q_begin):
+@pytest.mark.parametrize("q_begin,first", [(0, 2048), (1000, 2048), (0, 512), (1001, 512)])
+def test_prefill_from_host_equals_prefill(q_begin, first):
     """QSALayer.prefill_from_host (inputs and output in pinned host memory,
     moved in chunks overlapped with the compute on side streams) gives the
-    device prefill's outputs and caches bit for bit: a ragged last chunk,
-    a batch of two, and a start after an existing cache."""
+    device prefill's outputs and caches bit for bit: equal chunks with a
+    ragged last one, or chunks ramping 512 -> 2048 -> 512 with a ragged middle
+    one; a batch of two; a start after an existing cache (at a block boundary
+    or inside a block)."""
     import block_sparse_long_02_b200 as m
     from block_sparse_long_02_b200.layer import QSALayer
 
@@ -157,7 +159,7 @@ def test_prefill_from_host_equals_prefill(q_begin):
     hv = pin(full["v"][:, q_begin:].view(B, nq, cfg.kv_heads, 128))
     hik = pin(full["idx_k"][:, q_begin:])
     hout = torch.zeros(B, nq, cfg.q_heads, 128, dtype=torch.bfloat16).pin_memory()
-    Lb.prefill_from_host(hq, hiq, hk, hv, hik, q_begin, nq, hout, chunk=2048)
+    Lb.prefill_from_host(hq, hiq, hk, hv, hik, q_begin, nq, hout, chunk=2048, first=first)
     torch.cuda.synchronize()
     assert torch.equal(hout, out.cpu())
     for name in ("k_cache", "v_cache", "idx_k_cache", "pooled"):
