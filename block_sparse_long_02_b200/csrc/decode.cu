@@ -1,18 +1,23 @@
 // Decode step pieces ("QSA (Qwen Sparse Attention)" concept page, (A)-(B), for
 // one new token per sequence): a8 (cache append, block pooling) with a3' (query
 // rotation), the a4 score stream over every pooled key of a sequence, and the
-// a5 selection.
+// a5 selection; and the whole step as one persistent kernel.
 //
 // The score stream is the hot spot: 256 bytes of pooled key per block and
 // 4 x 128 multiply-adds, an L2/HBM stream spread over one wave of CTAs, each
 // scoring its slice on the tensor cores (mma.sync) from 16-byte loads issued a
-// group ahead. The same pass builds a per-sequence histogram of a level-1 key
-// digit of the scores, so the selection reads the score row once more and never
-// sorts it: one thread-block cluster per sequence finds the threshold digit,
-// collects the sure winners and the threshold-digit candidates of each CTA's
-// slice in shared memory, resolves the exact pick among all candidates over
-// distributed shared memory (ties to the lower block index), and writes the
-// k_B winners in ascending order.
+// group ahead (streaming, evict-first loads when the batch's keys outsize L2).
+// The same pass builds a per-sequence histogram of a level-1 key digit of the
+// scores, so the selection reads the score row once more and never sorts it:
+// every CTA of the selection grid finds the threshold digit, collects the sure
+// winners and the threshold-digit candidates of its slice, and reserves room
+// for them in the sequence's global lists; the last CTA to finish resolves the
+// exact pick among the candidates (ties to the lower block index) and writes
+// the k_B winners in ascending order.
+//
+// decode_step_kernel runs append, scores, selection and attention in one
+// launch (see its comment); the attention there is the warp-level code of
+// attend.cuh, and the three-kernel path's attention is in attention.cu.
 #include <algorithm>
 #include <atomic>
 
