@@ -84,3 +84,33 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["cpu_baseline"]["value"] == d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_host_prefill_chunk_plan():
+    """QSALayer.chunk_plan (prefill_from_host): chunks sum to nq, none above the
+    chunk size, ramping up and back down at the ends (host logic only)."""
+    from block_sparse_long_02_b200.layer import QSALayer
+
+    for nq, chunk, first in [(1 << 20, 131072, 8192), (6007, 2048, 512), (6007, 2048, 2048), (100, 100, 100),
+                             (7, 4, 4), (131072, 131072, 8192), (1 << 20, 131072, 131072)]:
+        plan = QSALayer.chunk_plan(nq, chunk, first)
+        assert sum(plan) == nq and all(0 < m <= chunk for m in plan), (nq, chunk, first, plan)
+        k = 0
+        while k + 1 < len(plan) and plan[k] < chunk and plan[k + 1] == 2 * plan[k]:
+            k += 1
+        assert plan[:k] == plan[::-1][:k]  # the ramp down mirrors the ramp up
+    assert QSALayer.chunk_plan(1 << 20, 131072, 8192)[:5] == [8192, 16384, 32768, 65536, 131072]
+    assert QSALayer.chunk_plan(1 << 20, 131072, 8192)[-4:] == [65536, 32768, 16384, 8192]
+
+
+def test_traffic_figures_follow_the_kernel_sources():
+    """roofline.traffic comes from profiles/dram_traffic.txt only while the
+    stage's kernel sources hash to what the figure was measured on."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        workload, stage, nbytes, sha = line.split()
+        want = float(nbytes) if sha == bench.stage_source_sha1(stage) else None
+        assert bench.traffic_for(workload, stage) == want, line
+    assert bench.traffic_for("decode_b8_n256k", "attention") is None  # never measured
