@@ -87,7 +87,8 @@ class QSALayer:
         copy are not overlapped. Each chunk is the prefill call on a
         double-buffered staging area, so the outputs equal prefill's bit for bit.
         Returns when the work is queued; host_out is complete once the current
-        stream has synchronised."""
+        stream has synchronised, and the host tensors must stay alive and
+        unchanged until then."""
         B, r = self.batch, self.cfg.r
         chunk = max(r, min(chunk, nq) // r * r)
         plan = self.chunk_plan(nq, chunk, max(r, min(first, chunk) // r * r))
