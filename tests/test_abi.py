@@ -38,6 +38,13 @@ def test_workspace_sizes_and_config_validation(qsa):
     cfg = qsa.Config()
     n = qsa.qsa_workspace_size(cfg, qsa.OP_DECODE_STEP, 8, 262144 + 64)
     assert n >= 8 * 65536 * 4  # at least the fp32 score row per sequence
+    # The step kernel's partial states (16 splits x (G x 128 + 2 G) floats per
+    # sequence and kv head) and listed blocks (4096 x 8 bytes per sequence) are in it.
+    assert n >= 8 * 65536 * 4 + 8 * 4 * 16 * (8 * 128 + 16) * 4 + 8 * 4096 * 8
+    # The documented no-allocation limits: 8 x 256K fits the 16 MiB scratch, 64 x 4M does not.
+    assert n <= 16 << 20
+    assert qsa.qsa_workspace_size(cfg, qsa.OP_DECODE_STEP, 64, 4 << 20) > 16 << 20
+    assert qsa.qsa_workspace_size(cfg, qsa.OP_DECODE_STEP, 16, 262144 + 64) > n  # grows with the batch
     assert qsa.qsa_workspace_size(cfg, qsa.OP_SPARSE_ATTENTION, 1, 1024, 1024) == 256
     for bad, status in ((dict(idx_heads=8), 2), (dict(head_dim=64), 2), (dict(q_heads=30, kv_heads=4), 2),
                         (dict(r=0), 2), (dict(K=0), 1), (dict(rope_dims=60), 2), (dict(kv_heads=3, q_heads=24), 2)):
