@@ -94,6 +94,17 @@ def test_step_kernel_launch_shapes_match_oracle(qsa, n, batch, K, q_heads, kv_he
         assert torch.equal(a, b)
 
 
+def test_step_kernel_falls_back_for_groups_above_8(qsa):
+    """q_heads / kv_heads = 16 is outside the step kernel (one n8 tile of heads):
+    with the step kernel selected the step runs the three kernels, and matches
+    the oracle."""
+    n, batch = 3001, 2
+    w, cfg, L, step = _setup(qsa, n, batch, 512, 64, 4, 0xDE)
+    res = _step(L, cfg, step, n)
+    assert qsa.qsa_workspace_status(L.workspace(qsa.OP_DECODE_STEP)) == 0
+    _check(w, cfg, L, n, res, [0, 1])
+
+
 @pytest.mark.parametrize("n,batch", [(20003, 8), (5000, 3), (700, 2)])
 def test_step_kernel_and_three_kernels_select_the_same_blocks(qsa, n, batch):
     """Same inputs through both decode paths: the selections are equal bit for
